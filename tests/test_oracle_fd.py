@@ -1,0 +1,122 @@
+"""Central finite differences of the whole oracle layer (float64).
+
+loss = <y, dy> + L_aux + L_z.  Routing and dispatch are piecewise constant,
+so every perturbation whose routing or dispatch changes is skipped; f in the
+aux loss is then constant, which is exactly the reading the analytic
+gradient uses.  Logits stay float64 here (Opts.logits_fp32=False) so the
+difference quotients are not polluted by the fp32 rounding of the router.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import workloads as W
+from oracle import moe_oracle as O
+from tests.helpers import oracle_layer
+
+H = 1e-5
+
+
+def _loss(L, o, dy):
+    fw = O.forward(L, o)
+    return float((fw["y"] * dy).sum() + fw["aux"] + fw["z"]), fw
+
+
+def _same_routing(fa, fb):
+    return (np.array_equal(fa["R"].idx, fb["R"].idx)
+            and np.array_equal(fa["Dp"].rank, fb["Dp"].rank))
+
+
+def _fd_check(cfg, n_per_tensor=12, seed=0):
+    L = oracle_layer(cfg)
+    w13 = L._w13_all.copy()
+    wd = L._wd_all.copy()
+    L.w13 = lambda e: w13[e]
+    L.wd = lambda e: wd[e]
+    o = O.opts_of(cfg)
+    o.logits_fp32 = False
+    dy = W.make_input(cfg, "dy").double().numpy()
+    base, fw = _loss(L, o, dy)
+    bw = O.backward(L, o, fw, dy)
+    rng = np.random.default_rng(seed)
+    targets = [("x", L.x, bw["dx"]), ("w_r", L.w_r, bw["dw_r"]),
+               ("w13", w13, np.stack([bw["dw13"][e] for e in range(cfg.E)])),
+               ("wd", wd, np.stack([bw["dwd"][e] for e in range(cfg.E)]))]
+    if cfg.n_shared:
+        targets += [("w13_s", L.w13_s, bw["dw13_s"]), ("wd_s", L.wd_s, bw["dwd_s"])]
+    checked = skipped = 0
+    for name, arr, grad in targets:
+        flat = arr.reshape(-1)
+        gflat = grad.reshape(-1)
+        for i in rng.choice(flat.size, size=min(n_per_tensor, flat.size),
+                            replace=False):
+            old = flat[i]
+            flat[i] = old + H
+            lp, fp = _loss(L, o, dy)
+            flat[i] = old - H
+            lm, fm = _loss(L, o, dy)
+            flat[i] = old
+            if not (_same_routing(fw, fp) and _same_routing(fw, fm)):
+                skipped += 1
+                continue
+            fd = (lp - lm) / (2 * H)
+            an = gflat[i]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)) + 1e-7, (name, i, fd, an)
+            checked += 1
+    assert checked >= 3 * skipped and checked > 0
+    return checked
+
+
+def test_fd_tiny_config():
+    assert _fd_check(W.CONFIGS["tiny"], n_per_tensor=20) > 50
+
+
+@pytest.mark.parametrize("variant", ["A_aux_z_sentinel_capacity",
+                                     "B_capacity_hotspot",
+                                     "sigmoid_groups_shared",
+                                     "sigmoid_A_top2sum"])
+def test_fd_feature_configs(variant):
+    base = W.CONFIGS["tiny"].replace(T=48, D=16, E=8, K=2, F=24, dtype="fp32")
+    cfg = {
+        "A_aux_z_sentinel_capacity": base.replace(
+            renorm=0, aux_alpha=0.05, z_lambda=0.01, sentinel_frac=0.15,
+            capacity_factor=0.75),
+        "B_capacity_hotspot": base.replace(
+            renorm=1, capacity_factor=1.0, hot_expert_offset=0.05,
+            route_scale=1.7),
+        "sigmoid_groups_shared": base.replace(
+            score_fn=W.SIGMOID, renorm=1, n_groups=4, topk_groups=2,
+            sel_bias_range=0.1, n_shared=1, K=3, z_lambda=0.01),
+        "sigmoid_A_top2sum": base.replace(
+            score_fn=W.SIGMOID, renorm=0, n_groups=4, topk_groups=3,
+            group_score=W.GROUP_TOP2SUM, sel_bias_range=0.1),
+    }[variant]
+    cfg = cfg.replace(w_std=0.3)   # larger logits: routing decisions matter
+    assert _fd_check(cfg) > 30
+
+
+def test_sentinel_zero_gate_grad_and_negative_control():
+    """Sentinel slots give dg = 0 and leave the router grad of the masked
+    layer intact; the batched_mm-style negative control (clamp the id to
+    expert 0, keep proj_out) has the same forward but a different router
+    gradient (transformers issue: loss identical, router grad wrong)."""
+    cfg = W.CONFIGS["tiny"].replace(T=64, D=16, E=4, K=2, F=24, renorm=0,
+                                    sentinel_frac=0.2, w_std=0.3)
+    L = oracle_layer(cfg)
+    o = O.opts_of(cfg)
+    dy = W.make_input(cfg, "dy").double().numpy()
+    fw = O.forward(L, o)
+    bw = O.backward(L, o, fw, dy)
+    sj = fw["Dp"].sentinel.reshape(cfg.T, cfg.K)
+    assert sj.sum() == cfg.n_sentinel > 0
+    assert np.all(bw["dg"][sj] == 0.0)
+    # bug mode: proj_out of expert 0 for the sentinel slots
+    x = L.x
+    _, _, _, o0 = O.swiglu_forward(np.repeat(x, cfg.K, axis=0), L.w13(0), L.wd(0))
+    bw_bug = O.backward(L, o, fw, dy, sentinel_unmasked=o0)
+    assert np.any(bw_bug["dg"][sj] != 0.0)
+    assert np.linalg.norm(bw_bug["dw_r"] - bw["dw_r"]) > 1e-3 * np.linalg.norm(bw["dw_r"])
+    # the expert weights' grads do not depend on the router-side leak
+    for e in range(cfg.E):
+        np.testing.assert_array_equal(bw_bug["dw13"][e], bw["dw13"][e])
