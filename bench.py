@@ -1,0 +1,494 @@
+"""Benchmark of the token-choice MoE layer step (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config mm_b]
+                    [--impl reference]
+
+One step = the whole hot path over one batch: router, dispatch, aux/z loss,
+grouped SwiGLU experts, combine, and the full backward (gate-weight
+gradient, expert dgrad/wgrad, router gradient, dx).  The default workload
+is the MiniMind-shaped layer (T=4096, D=768, E=4, K=1, F=2048, bf16,
+variant B, aux alpha 5e-4).  Multi-GPU (torchrun): data-parallel replicas,
+each rank runs its own batch (weak scaling, no data-path collective);
+timing is the max over ranks.
+
+Rank 0 prints one JSON line.  `value` is tokens/s from CUDA events around
+CUDA-graph replays of the step with inputs resident in HBM (L2 flushed
+between steps); `e2e` is the same metric through the Python API with the
+step's inputs copied from pinned host memory and y, dx read back; the
+roofline entry times the dominant kernel's launches with CUDA events on its
+launching stream inside the timed region.  `--impl reference` times the
+CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "MoE layer fwd+bwd tokens/s at 1 B200; grouped-GEMM % bf16 peak; HBM GB/s"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="mm_b", choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--cpu-sample-s", type=float, default=10.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_init(n_gpus, backend="nccl"):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t[0])
+
+
+def rank_config(cfg: W.LayerConfig, rank: int) -> W.LayerConfig:
+    """Each data-parallel rank draws its own tokens (weights are shared)."""
+    return cfg if rank == 0 else cfg.replace(seed=cfg.seed + 1000 * rank)
+
+
+# ---------------------------------------------------------------------------
+# work accounting (algorithmic, per step)
+# ---------------------------------------------------------------------------
+def expert_rows(cfg, kept_total):
+    return kept_total + (cfg.T if cfg.n_shared else 0)
+
+
+def gemm_flops(cfg, kept_total):
+    """Algorithmic FLOPs of each tensor-core GEMM family for one step."""
+    M = expert_rows(cfg, kept_total)
+    D, F = cfg.D, cfg.F
+    return {
+        "tc_gate_up_swiglu": 2 * M * D * 2 * F,
+        "tc_down": 2 * M * F * D,
+        "tc_dgrad_down_swiglu_bwd": 2 * M * D * F,
+        "tc_wgrad_down": 2 * M * D * F,
+        "tc_dgrad_gate_up": 2 * M * 2 * F * D,
+        "tc_wgrad_gate_up": 2 * M * 2 * F * D,
+    }
+
+
+def source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "mixture_experts_routing_fp32_b200", "csrc")
+    for n in sorted(os.listdir(d)):
+        with open(os.path.join(d, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return j.get("hbm_gbs", 6545.0), j.get("bf16_tflops", 1652.8), \
+            j.get("bf16_tflops_sustained", 1386.2), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if its kernel
+    source hash is the current one (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5], f[6], f[7], f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        load = [r for r in rows if r[0] > 0.5 * r[1]] or rows
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for n, v in zip(names, r[2:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in load),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    from mixture_experts_routing_fp32_b200 import (MoELayer, config_from, moe_check_status,
+                                                   moe_launch_count)
+    from mixture_experts_routing_fp32_b200.api import LaunchProfile
+    from mixture_experts_routing_fp32_b200.build import build
+
+    rank, world, local = dist_init(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        build()
+    barrier(world)
+    base = W.CONFIGS[args.config]
+    cfg = rank_config(base, rank)
+    names = ("x", "w_r", "w13", "w_down", "dy")
+    inp = {n: W.make_input(cfg if n in ("x", "dy") else base, n, dev) for n in names}
+    opt = {
+        "w13_s": W.make_input(base, "w13_s", dev) if base.n_shared else None,
+        "w_down_s": W.make_input(base, "w_down_s", dev) if base.n_shared else None,
+        "logit_offset": W.make_input(base, "logit_offset", dev) if base.hot_expert_offset else None,
+        "sel_bias": W.make_input(base, "sel_bias", dev) if base.sel_bias_range else None,
+        "sentinel_mask": W.make_input(cfg, "sentinel_mask", dev) if base.sentinel_frac else None,
+    }
+    layer = MoELayer(config_from(base), device=dev)
+    weights = dict(w_r=inp["w_r"], w13=inp["w13"], w_down=inp["w_down"], **opt)
+    x, dy = inp["x"], inp["dy"]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.forward(x, **weights)
+        layer.backward(dy)
+
+    # warm-up (eager), then capture one step in a CUDA graph with per-launch events
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    moe_check_status()
+    moe_launch_count(reset=True)
+    step()
+    torch.cuda.synchronize(dev)
+    launches_per_step = moe_launch_count(reset=True)
+    prof = LaunchProfile(128)
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            prof.reset()
+            with torch.cuda.graph(graph, stream=side):
+                step()
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+
+    def replay():
+        if graph is not None:
+            graph.replay()
+        else:
+            prof.reset()
+            step()
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        replay()
+    torch.cuda.synchronize(dev)
+    moe_check_status()
+
+    kept_total = int(layer.kept.sum())
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    per_launch = []
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_index) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)          # L2 flush between timed steps (untimed)
+            ev0[i].record(stream)
+            replay()
+            ev1[i].record(stream)
+            torch.cuda.synchronize(dev)
+            per_launch.append(prof.read())
+        barrier(world)
+        torch.cuda.synchronize(dev)
+    step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
+    ms = statistics.mean(step_ms)
+    ms_max = max_over_ranks(ms, world, dev)
+    moe_check_status()
+
+    # dominant kernel (largest share of the step), its average launch time
+    fam = {}
+    for launches in per_launch:
+        for name, t in launches:
+            fam.setdefault(name, []).append(t)
+    tot = {k: sum(v) / len(per_launch) for k, v in fam.items()}
+    dom = max(tot, key=tot.get)
+    n_dom = len(fam[dom]) / len(per_launch)
+    dom_ms = statistics.mean(fam[dom])
+    hbm, bf16, bf16_sus, peak_src = measured_peaks()
+    flops = gemm_flops(base, kept_total)
+    if dom in flops:
+        achieved = flops[dom] / n_dom / (dom_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2),
+                "peak": bf16_sus, "unit": "TFLOP/s",
+                "frac": round(achieved / bf16_sus, 4),
+                "peak_source": "%s bf16 dense, sustained (kernel timed inside a long step)" % peak_src}
+    else:
+        roof = {"bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s",
+                "frac": None, "peak_source": peak_src}
+    roof.update({"kernel": dom, "launch_ms": round(dom_ms, 5),
+                 "launches_per_step": n_dom,
+                 "traffic": recorded_traffic(dom, base.name)})
+    gemm_total_ms = sum(v for k, v in tot.items() if k.startswith("tc_"))
+    all_gemm_tflops = sum(flops.values()) / (gemm_total_ms * 1e-3) / 1e12 if gemm_total_ms else None
+
+    # e2e through the public API: pinned host inputs in, y and dx out, every step
+    hx = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    hdy = torch.empty(dy.shape, dtype=dy.dtype, pin_memory=True)
+    hx.copy_(x)
+    hdy.copy_(dy)
+    hy = torch.empty(layer.y.shape, dtype=layer.y.dtype, pin_memory=True)
+    hdx = torch.empty(layer.dx.shape, dtype=layer.dx.dtype, pin_memory=True)
+    dx_dev = torch.empty_like(x)
+    ddy = torch.empty_like(dy)
+    e2e_ms = []
+    h2d = hx.numel() * hx.element_size() + hdy.numel() * hdy.element_size()
+    d2h = hy.numel() * hy.element_size() + hdx.numel() * hdx.element_size()
+    for i in range(args.steps + 2):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dx_dev.copy_(hx, non_blocking=True)
+        ddy.copy_(hdy, non_blocking=True)
+        layer.forward(dx_dev, **weights)
+        layer.backward(ddy)
+        hy.copy_(layer.y, non_blocking=True)
+        hdx.copy_(layer.dx, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        if i >= 2:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e = max_over_ranks(statistics.mean(e2e_ms), world, dev)
+    moe_check_status()
+
+    clocks = clk.summary()
+    cpu = cpu_baseline(base, args.cpu_sample_s) if (rank == 0 and world == 1) else None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(base.T * world / (ms_max * 1e-3), 1),
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_max, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if base.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded counter-hash normals; shapes of the MiniMind-shaped layer)",
+            "config": {"workload": "%s: T=%d D=%d E=%d K=%d F=%d %s variant %s aux %.0e" % (
+                base.name, base.T, base.D, base.E, base.K, base.F, base.dtype,
+                "B" if base.renorm else "A", base.aux_alpha),
+                "global_batch_tokens": base.T * world, "parallelism": "dp%d (replicas)" % world,
+                "l2": "flushed between timed steps (256 MiB write)",
+                "cuda_graph": graph is not None},
+            "e2e": {"value": round(base.T * world / (e2e * 1e-3), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e, 4),
+                    "path": "Python API (MoELayer.forward/backward), eager launches"},
+            "gpu_launches": launches_per_step * args.steps,
+            "roofline": roof,
+            "gemm_all": {"tflops": round(all_gemm_tflops, 2) if all_gemm_tflops else None,
+                         "frac_of_sustained": round(all_gemm_tflops / bf16_sus, 4) if all_gemm_tflops else None,
+                         "ms_per_step": round(gemm_total_ms, 5)},
+            "kernels_ms_per_step": {k: round(v, 5) for k, v in sorted(tot.items(), key=lambda kv: -kv[1])},
+            "kept_rows": kept_total,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+            "source_hash": source_hash(),
+        }
+        print(json.dumps(line), flush=True)
+    prof.close()
+    if graph is not None:
+        del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+def cpu_sample_tokens(cfg):
+    return min(cfg.T, 512)
+
+
+def oracle_step(cfg, T_s):
+    """One forward + backward of the oracle on the first T_s tokens."""
+    import numpy as np
+    from oracle import moe_oracle as O
+    sub = cfg.replace(T=T_s)
+    f = lambda t: t.double().numpy()
+    w13 = {}
+    wd = {}
+
+    def g13(e):
+        if e not in w13:
+            w13[e] = f(W.make_input(cfg, "w13", expert=e))
+        return w13[e]
+
+    def gd(e):
+        if e not in wd:
+            wd[e] = f(W.make_input(cfg, "w_down", expert=e))
+        return wd[e]
+
+    L = O.Layer(x=f(W.make_input(cfg, "x", rows=np.arange(T_s))), w_r=f(W.make_input(cfg, "w_r")),
+                w13=g13, wd=gd)
+    if cfg.n_shared:
+        L.w13_s, L.wd_s = f(W.make_input(cfg, "w13_s")), f(W.make_input(cfg, "w_down_s"))
+    if cfg.hot_expert_offset:
+        L.logit_offset = f(W.make_input(cfg, "logit_offset"))
+    if cfg.sel_bias_range:
+        L.sel_bias = f(W.make_input(cfg, "sel_bias"))
+    dy = f(W.make_input(cfg, "dy", rows=np.arange(T_s)))
+    # weights are generated before the clock starts
+    for e in range(cfg.E):
+        g13(e), gd(e)
+    o = O.opts_of(sub)
+    t0 = time.perf_counter()
+    fw = O.forward(L, o)
+    O.backward(L, o, fw, dy)
+    return time.perf_counter() - t0
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, budget_s):
+    T_s = cpu_sample_tokens(cfg)
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while True:
+        times.append(oracle_step(cfg, T_s))
+        if time.perf_counter() > t_end or len(times) >= 20:
+            break
+    s = statistics.mean(times)
+    return {"value": round(T_s / s, 2), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": "first %d of %d tokens, full forward+backward in the float64 numpy "
+                      "oracle, mean of %d runs (%.2f s each)" % (T_s, cfg.T, len(times), s)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = W.CONFIGS[args.config]
+    T_s = cpu_sample_tokens(cfg)
+    for _ in range(args.warmup):
+        oracle_step(cfg, T_s)
+    times = [oracle_step(cfg, T_s) for _ in range(args.steps)]
+    s = statistics.mean(times)
+    v = round(T_s / s, 2)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "%s (oracle on the first %d tokens per step)" % (cfg.name, T_s)},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": "first %d of %d tokens per step" % (T_s, cfg.T)},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,274 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) token-choice MoE layer library
+ * (libmoe.so): router, dispatch, expert FFN, combine, aux/z losses and the
+ * full backward of one layer on one GPU.
+ *
+ * Pages this follows (cited by title and section):
+ *   [STA324]  "08 MoE：容量、路由、梯度、均衡和系统实现" (STA324 notes), §8.1-§8.9
+ *   [TRAIN]   "MoE 训练：稀疏计算背后的路由与通信" (MoE training course page)
+ *   [8MOE]    "8-MoE" lecture notes (Router / Gating Network, KeepTopK,
+ *             Expert Capacity, GShard, Switch Transformers, ST-MoE,
+ *             MoE 高效推理 — token grouping and permutation)
+ *   [HF48687] "Wrong router gradient with experts_implementation=batched_mm
+ *             under expert parallelism" (transformers issue summary)
+ *   [MM858]   "[Bug] num_experts_per_tok=1 时 MoE 路由器收不到梯度" (MiniMind issue)
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise;
+ *     `cfg` is a HOST pointer.  All buffers are owned and allocated by the
+ *     caller; the library never allocates or frees memory.
+ *   - All layouts are row-major and contiguous.  T tokens, D model dim,
+ *     E routed experts, K experts per token, F expert FFN dim.
+ *     "act" = activation / expert-weight element type, cfg->dtype:
+ *     MOE_BF16 (__nv_bfloat16) or MOE_FP32 (float).  The router is fp32.
+ *   - Calls are asynchronous on `stream` and never synchronise, except
+ *     moe_check_status().  They may issue cudaMemsetAsync on `stream`.
+ *   - Return value: MOE_OK (0) or a negative moe_status; on MOE_ERR_ARG
+ *     nothing was launched.  Errors detected on the device (an expert id
+ *     outside [-1, E), a pipeline wait that timed out) set a device error
+ *     word that moe_check_status() reads and clears.
+ *   - Permuted row space: routed expert e owns rows
+ *     [offsets[e], offsets[e+1]); its kept slots occupy the first kept[e]
+ *     rows in flat-slot order, the rest up to the next multiple of 128 are
+ *     zero padding.  The shared expert (n_shared = 1) owns rows
+ *     [offsets[E], offsets[E+1]) = its T tokens in order, then padding.
+ *     Buffers indexed by row are sized rows_max (moe_get_sizes).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_ARG = -1,          /* invalid argument / unsupported configuration */
+  MOE_ERR_CUDA = -2,         /* a CUDA call or launch failed (moe_last_cuda_error) */
+  MOE_ERR_DEVICE = -3,       /* device error word set (see moe_check_status) */
+  MOE_ERR_TIMEOUT = -4       /* reserved: a bounded device wait gave up */
+} moe_status;
+
+enum { MOE_FP32 = 0, MOE_BF16 = 1 };             /* cfg.dtype */
+enum { MOE_SOFTMAX = 0, MOE_SIGMOID = 1 };       /* cfg.score_fn */
+enum { MOE_GMAX = 0, MOE_GTOP2SUM = 1 };         /* cfg.group_score */
+enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SIMT = 1 };   /* cfg.gemm_impl */
+
+/* Device error word bits (moe_check_status). */
+#define MOE_DEVERR_EXPERT_ID  1u   /* an expert id outside [-1, E): slot treated as sentinel */
+#define MOE_DEVERR_TIMEOUT    2u   /* a tensor-core pipeline wait gave up */
+#define MOE_DEVERR_ROWS       4u   /* permuted rows exceeded rows_max */
+
+/*
+ * Layer configuration.
+ *   score_fn   MOE_SOFTMAX: p = softmax(s), top-K on s          [STA324 §8.2]
+ *              MOE_SIGMOID: p = sigmoid(s), top-K on p + b      [STA324 §8.6]
+ *   renorm     0 = variant A (g = p_sel, no renormalisation),
+ *              1 = variant B (g = softmax over the selected logits; for
+ *                  sigmoid g = p_sel / (sum p_sel + 1e-20))     [STA324 §8.2]
+ *   n_groups, topk_groups, group_score
+ *              group-limited routing: E splits into n_groups contiguous
+ *              groups scored by their max (MOE_GMAX) or the sum of their
+ *              two largest (MOE_GTOP2SUM) selection scores; only experts of
+ *              the topk_groups best groups are eligible.  1,1 = off.
+ *              [STA324 §8.2], [TRAIN] (capacity, dropless and group routing)
+ *   capacity_factor, min_capacity
+ *              C = max(ceil(c*T*K/E), min_capacity); c <= 0: no limit.
+ *              [STA324 §8.5], [8MOE] Expert Capacity
+ *   route_scale multiplies g after renormalisation               [TRAIN]
+ *   aux_alpha  Switch load-balance loss alpha*E*sum_e f_e P_e; softmax only
+ *              [STA324 §8.5], [TRAIN]
+ *   z_lambda   router z-loss lambda*mean_t lse_t^2           [8MOE] ST-MoE
+ *   n_shared   0 or 1: a shared SwiGLU expert on every token, weight 1,
+ *              no top-K slot                                 [STA324 §8.7]
+ *   gemm_impl  MOE_GEMM_AUTO: tcgen05 tensor cores for bf16 when D and F
+ *              are multiples of 128, CUDA-core SIMT otherwise (fp32 always);
+ *              MOE_GEMM_SIMT: force the SIMT kernels (cross-checks).
+ * Limits: 1 <= K <= min(E, 16); E <= 512; n_groups <= 32, E % n_groups == 0,
+ * topk_groups * (E / n_groups) >= K; D % 8 == 0; F % 8 == 0.
+ */
+typedef struct {
+  int32_t T, D, E, K, F, n_shared;
+  int32_t dtype;
+  int32_t score_fn, renorm;
+  int32_t n_groups, topk_groups, group_score;
+  float capacity_factor;
+  int32_t min_capacity;
+  float route_scale, aux_alpha, z_lambda;
+  int32_t gemm_impl;
+} moe_config_t;
+
+typedef struct {
+  int64_t rows_max;     /* rows of every permuted-row buffer (multiple of 128) */
+  int64_t tiles_max;    /* rows_max / 128 */
+  int64_t capacity;     /* C, or -1 when unlimited */
+  size_t ws_bytes;      /* workspace needed by any call (256-byte aligned base) */
+} moe_sizes_t;
+
+/* Buffer sizes for cfg.  Host-only, no CUDA calls. */
+int moe_get_sizes(const moe_config_t* cfg, moe_sizes_t* out);
+
+/*
+ * moe_router — fp32 router logits, scores, group limit, top-K and gate
+ * weights.  [STA324 §8.2, §8.6], [8MOE] Router / Gating Network, KeepTopK,
+ * [TRAIN] (TopKRouter flow), [MM858] §2.
+ *   x            [T,D] act
+ *   w_r          [E,D] f32 router weight (logits s = x w_r^T)
+ *   logit_offset [E] f32 or NULL: constant added to the logits
+ *   sel_bias     [E] f32 or NULL: selection-only bias (sigmoid scoring)
+ *   logits       [T,E] f32 out
+ *   probs        [T,E] f32 out: softmax probabilities or sigmoid affinities
+ *   lse          [T]   f32 out: logsumexp of the logits
+ *   topk_idx     [T,K] i32 out: selected experts, best first; equal
+ *                selection scores go to the lower expert index
+ *   topk_w       [T,K] f32 out: gate weights g
+ *   near_ties    [1] i32 out: tokens whose K-th/(K+1)-th selection margin
+ *                (or group-boundary margin) is below 1e-5
+ *   ws           workspace (moe_get_sizes)
+ */
+int moe_router(const moe_config_t* cfg, const void* x, const float* w_r,
+               const float* logit_offset, const float* sel_bias,
+               float* logits, float* probs, float* lse,
+               int32_t* topk_idx, float* topk_w, int32_t* near_ties,
+               void* ws, cudaStream_t stream);
+
+/*
+ * moe_dispatch — counting-sort permutation with capacity drop and sentinel
+ * slots, and the gather of token rows into expert order.
+ * [8MOE] MoE 高效推理 (sort tokens by expert, gather), Expert Capacity,
+ * GShard drop tokens; [STA324 §8.5, §8.8]; [HF48687] cause analysis.
+ *   topk_idx      [T,K] i32: expert per slot; -1 = sentinel (no local expert)
+ *   sentinel_mask [T*K] u8 or NULL: nonzero marks a slot as sentinel
+ *   x             [T,D] act
+ *   counts        [E] i32 out: valid slots per expert before drops
+ *   kept          [E] i32 out: min(counts, C)
+ *   offsets       [E+2] i32 out: permuted-row offsets (see header)
+ *   slot_row      [T*K] i32 out: row of each slot, -1 if sentinel/dropped
+ *   row_slot      [rows_max] i32 out: slot of each routed row, -1 otherwise
+ *   tile_expert   [tiles_max] i32 out: expert of each 128-row tile (E = shared)
+ *   stats         [4] i32 out: n_dropped, n_sentinel, n_rows, n_tiles
+ *   x_perm        [rows_max,D] act out: gathered rows, zero padding
+ * Slots of one expert are ranked in flat slot order j = t*K + k; ranks >= C
+ * are dropped.
+ */
+int moe_dispatch(const moe_config_t* cfg, const int32_t* topk_idx,
+                 const uint8_t* sentinel_mask, const void* x,
+                 int32_t* counts, int32_t* kept, int32_t* offsets,
+                 int32_t* slot_row, int32_t* row_slot, int32_t* tile_expert,
+                 int32_t* stats, void* x_perm, void* ws, cudaStream_t stream);
+
+/*
+ * moe_aux_loss — losses[0] = alpha*E*sum_e f_e P_e with f_e = counts_e /
+ * sum(counts), P_e = mean_t probs[t,e]; losses[1] = lambda*mean_t lse_t^2.
+ * [STA324 §8.5, §8.6], [TRAIN], [8MOE] ST-MoE.  losses: [2] f32 out.
+ * Deterministic (fixed-order reductions).
+ */
+int moe_aux_loss(const moe_config_t* cfg, const float* probs, const float* lse,
+                 const int32_t* counts, float* losses, void* ws,
+                 cudaStream_t stream);
+
+/*
+ * moe_expert_ffn — grouped SwiGLU experts over the permuted rows.
+ * [STA324 §8.1, §8.8] (SwiGLU ~3DF parameters; grouped GEMM over experts).
+ *   x_perm   [rows_max,D] act (moe_dispatch)
+ *   w13      [E,2F,D] act: rows 0..F-1 gate projection, F..2F-1 up
+ *   w_down   [E,D,F]  act
+ *   w13_s, w_down_s  [2F,D], [D,F] act: shared expert (NULL if n_shared=0)
+ *   a13      [rows_max,2F] act out: pre-activations (saved for backward)
+ *   h        [rows_max,F]  act out: silu(a) * b
+ *   o        [rows_max,D]  act out: expert outputs h w_down^T
+ * Tiles of experts without rows are skipped on the device (no host sync).
+ */
+int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
+                   const int32_t* offsets,
+                   const int32_t* tile_expert, const int32_t* stats,
+                   const void* w13, const void* w_down,
+                   const void* w13_s, const void* w_down_s,
+                   void* a13, void* h, void* o, void* ws, cudaStream_t stream);
+
+/*
+ * moe_combine — y_t = sum_{k kept} g_{t,k} o[slot_row[t*K+k]] (k ascending,
+ * fp32 accumulation) + o[offsets[E] + t] when n_shared.  Deterministic
+ * gather, no atomics.  [8MOE] Router / Gating Network (y = sum G(x)_i
+ * E_i(x)); [STA324 §8.7, §8.8].
+ *   y [T,D] act out
+ */
+int moe_combine(const moe_config_t* cfg, const void* o,
+                const int32_t* slot_row, const float* topk_w,
+                const int32_t* offsets, void* y, cudaStream_t stream);
+
+/*
+ * moe_backward — all gradients of <y, dy> + L_aux + L_z.
+ * [STA324 §8.3, §8.5], [MM858] §2-§3, [HF48687] cause analysis.
+ * Inputs are the forward's inputs and outputs above, plus
+ *   dy        [T,D] act: upstream gradient of y
+ * Outputs:
+ *   dx        [T,D] act: expert path + shared expert + router path
+ *   dw_r      [E,D] f32
+ *   dw13      [E,2F,D] act, dw_down [E,D,F] act (expert with no rows: 0)
+ *   dw13_s, dw_down_s  shared expert grads (NULL if n_shared = 0)
+ *   dg_out    [T,K] f32 or NULL: dL/dg = <o, dy>, 0 on sentinel/dropped
+ *   dlogits_out [T,E] f32 or NULL: dL/ds
+ * The gate gradient of a sentinel or dropped slot is zero (its expert
+ * output is treated as zero), so such slots send no gradient to the router
+ * through the gate path.  Deterministic: no floating-point atomics.
+ */
+int moe_backward(const moe_config_t* cfg,
+                 const void* x, const float* w_r, const float* logits,
+                 const float* probs, const float* lse,
+                 const int32_t* topk_idx, const float* topk_w,
+                 const int32_t* counts, const int32_t* kept,
+                 const int32_t* offsets, const int32_t* slot_row,
+                 const int32_t* row_slot, const int32_t* tile_expert,
+                 const int32_t* stats,
+                 const void* x_perm, const void* a13, const void* h,
+                 const void* o,
+                 const void* w13, const void* w_down,
+                 const void* w13_s, const void* w_down_s,
+                 const void* dy,
+                 void* dx, float* dw_r, void* dw13, void* dw_down,
+                 void* dw13_s, void* dw_down_s,
+                 float* dg_out, float* dlogits_out,
+                 void* ws, cudaStream_t stream);
+
+/* Synchronises `stream`, reads and clears the device error word (bits in
+ * *bits if non-NULL).  MOE_OK, MOE_ERR_DEVICE or MOE_ERR_CUDA. */
+int moe_check_status(cudaStream_t stream, uint32_t* bits);
+
+/* Text for a moe_status value (static storage). */
+const char* moe_status_string(int status);
+
+/* The cudaError_t behind the last MOE_ERR_CUDA on this thread. */
+int moe_last_cuda_error(void);
+
+/* Number of kernel launches issued by this thread since the last reset. */
+int64_t moe_launch_count(int reset);
+
+/*
+ * Per-launch timing (measurement support; not part of the layer's math).
+ * While enabled, every kernel launch of this thread is bracketed by a begin
+ * and an end cudaEvent recorded on the launching stream (inside a CUDA
+ * graph capture they become event-record nodes, re-recorded on every
+ * replay).  Up to max_launches launches (<= 256) are recorded after each
+ * moe_profile_reset().
+ *   moe_profile_enable  creates the events (the library's only resource
+ *                       other than device code; no device memory)
+ *   moe_profile_read    after the caller synchronised: writes the elapsed
+ *                       milliseconds of each recorded launch to ms (host
+ *                       array) and returns how many were written
+ *   moe_profile_name    kernel family name of recorded launch i
+ */
+int moe_profile_enable(int max_launches);
+int moe_profile_reset(void);
+int moe_profile_read(float* ms, int max);
+const char* moe_profile_name(int i);
+int moe_profile_disable(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,389 @@
+// Combine and the memory-bound parts of the backward.
+//
+// Combine: y_t = sum_{k kept} g_{t,k} o[row(t,k)] (+ shared expert row),
+// the weighted sum of the "8-MoE" lecture notes (Router / Gating Network:
+// y = sum_i G(x)_i E_i(x)) and STA324 notes "08 MoE" §8.7-§8.8 (a token
+// appears K times so its outputs accumulate; the shared expert is added
+// unweighted).  A gather in fixed k order: deterministic, no atomics.
+//
+// Gate gradient: dL/dg_{t,k} = <o_{t,k}, dy_t> for kept slots only.  The
+// transformers batched_mm issue (cause analysis) shows why: the gradient of
+// a sample weight is the expert output, so a slot with no local expert
+// (sentinel) must contribute a zero expert output; dropped slots likewise.
+//
+// Router backward: STA324 §8.3 (fixed selected set, g differentiable in the
+// logits; for K=1 variant B the weight is the constant 1), §8.5 (aux
+// gradient alpha*E*f_e/T with f constant), "8-MoE" ST-MoE (z-loss), and the
+// MiniMind issue §2 (the gate weight is the router's only differentiable
+// path).
+#pragma once
+#include "common.cuh"
+#include "router.cuh"
+
+namespace moe {
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ slot_row,
+               const float* __restrict__ topk_w, const int32_t* __restrict__ offsets,
+               int n_shared, int Tn, int D, int K, int E, T* __restrict__ y) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < Tn; t += (int64_t)gridDim.x * 8) {
+    int64_t rows[kMaxK];
+    float g[kMaxK];
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) {
+      rows[k] = -1;
+      g[k] = 0.f;
+      if (k < K) {
+        rows[k] = slot_row[t * K + k];
+        g[k] = topk_w[t * K + k];
+      }
+    }
+    const int64_t srow = n_shared ? (int64_t)offsets[E] + t : -1;
+    for (int d = lane * 8; d < D; d += 256) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < kMaxK; ++k) {
+        if (k < K && rows[k] >= 0) {
+          float v[8];
+          load8(o + rows[k] * D + d, v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(g[k], v[i], acc[i]);
+        }
+      }
+      if (srow >= 0) {
+        float v[8];
+        load8(o + srow * D + d, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += v[i];
+      }
+      store8(y + t * D + d, acc);
+    }
+  }
+}
+
+// Per permuted row: routed rows -> dg[slot] = <o[r], dy[t]> and
+// dO[r] = g * dy[t]; shared rows -> dO[r] = dy[t]; padding -> 0.
+template <typename T>
+__global__ void __launch_bounds__(256)
+bwd_rows_kernel(const T* __restrict__ o, const T* __restrict__ dy,
+                const float* __restrict__ topk_w, const int32_t* __restrict__ row_slot,
+                const int32_t* __restrict__ offsets, const int32_t* __restrict__ kept,
+                const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ stats,
+                int K, int E, int Tn, int D, float* __restrict__ dg_slot,
+                T* __restrict__ dO) {
+  const int n_rows = stats[2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t r = (int64_t)blockIdx.x * 8 + warp; r < n_rows; r += (int64_t)gridDim.x * 8) {
+    const int e = tile_expert[r / kRowTile];
+    int64_t t = -1, slot = -1;
+    if (e < E) {
+      if (r - offsets[e] < kept[e]) {
+        slot = row_slot[r];
+        t = slot / K;
+      }
+    } else if (r - offsets[E] < Tn) {
+      t = r - offsets[E];
+    }
+    T* dst = dO + r * D;
+    if (t < 0) {
+      for (int d = lane * 8; d < D; d += 256) zero8(dst + d);
+      continue;
+    }
+    const float g = slot >= 0 ? topk_w[slot] : 1.0f;
+    float dot = 0.f;
+    for (int d = lane * 8; d < D; d += 256) {
+      float dv[8], ov[8];
+      load8(dy + t * D + d, dv);
+      if (slot >= 0) {
+        load8(o + r * D + d, ov);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dot = fmaf(ov[i], dv[i], dot);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dv[i] *= g;
+      store8(dst + d, dv);
+    }
+    if (slot >= 0) {
+      dot = warp_sum(dot);
+      if (lane == 0) dg_slot[slot] = dot;
+    }
+  }
+}
+
+struct RouterBwdArgs {
+  int T, E, K;
+  int score_fn, renorm;
+  float route_scale, aux_alpha, z_lambda;
+  const float* logits;     // [T,E]
+  const float* probs;      // [T,E]
+  const float* lse;        // [T]
+  const int32_t* topk_idx; // [T,K]
+  const float* topk_w;     // [T,K]
+  const int32_t* slot_row; // [T*K]
+  const float* dg_slot;    // [T*K] (valid where slot_row >= 0)
+  const int32_t* counts;   // [E]
+  float* ds;               // [T,E]
+  float* dlogits_out;      // [T,E] or null
+  float* dg_out;           // [T,K] or null
+};
+
+template <int NV>
+__global__ void __launch_bounds__(256)
+router_bwd_kernel(RouterBwdArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = a.E, K = a.K;
+  float cnt_tot = 0.f;
+  if (a.aux_alpha != 0.f) {
+    for (int e = lane; e < E; e += 32) cnt_tot += (float)a.counts[e];
+    cnt_tot = warp_sum(cnt_tot);
+  }
+  const float rs = a.route_scale;
+  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < a.T; t += (int64_t)gridDim.x * 8) {
+    float dgk[kMaxK], gk[kMaxK];
+    int ik[kMaxK];
+#pragma unroll
+    for (int k = 0; k < kMaxK; ++k) {
+      dgk[k] = 0.f; gk[k] = 0.f; ik[k] = -1;
+      if (k < K) {
+        const int64_t j = t * K + k;
+        ik[k] = a.topk_idx[j];
+        gk[k] = a.topk_w[j];
+        dgk[k] = a.slot_row[j] >= 0 ? a.dg_slot[j] : 0.f;
+      }
+    }
+    float p[NV], ds[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      p[i] = e < E ? a.probs[t * E + e] : 0.f;
+      ds[i] = 0.f;
+    }
+    if (a.score_fn == MOE_SOFTMAX) {
+      float dp[NV];
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int e = lane + 32 * i;
+        dp[i] = (a.aux_alpha != 0.f && e < E && cnt_tot > 0.f)
+                    ? a.aux_alpha * (float)E * ((float)a.counts[e] / cnt_tot) / (float)a.T
+                    : 0.f;
+      }
+      if (!a.renorm) {
+#pragma unroll
+        for (int k = 0; k < kMaxK; ++k) {
+          if (k < K && ik[k] >= 0 && (ik[k] & 31) == lane) {
+#pragma unroll
+            for (int i = 0; i < NV; ++i) if (i == (ik[k] >> 5)) dp[i] += rs * dgk[k];
+          }
+        }
+      }
+      float inner = 0.f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) inner += p[i] * dp[i];
+      inner = warp_sum(inner);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) ds[i] = p[i] * (dp[i] - inner);
+      if (a.renorm) {
+        float innerB = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxK; ++k)
+          if (k < K && ik[k] >= 0) innerB += (gk[k] / rs) * (rs * dgk[k]);
+#pragma unroll
+        for (int k = 0; k < kMaxK; ++k) {
+          if (k < K && ik[k] >= 0 && (ik[k] & 31) == lane) {
+            const float add = (gk[k] / rs) * (rs * dgk[k] - innerB);
+#pragma unroll
+            for (int i = 0; i < NV; ++i) if (i == (ik[k] >> 5)) ds[i] += add;
+          }
+        }
+      }
+    } else {
+      float S = 0.f, innerS = 0.f;
+      float sp[kMaxK];
+#pragma unroll
+      for (int k = 0; k < kMaxK; ++k) {
+        sp[k] = 0.f;
+        if (k < K && ik[k] >= 0) {
+          sp[k] = a.probs[t * E + ik[k]];
+          S += sp[k];
+          innerS += dgk[k] * gk[k];
+        }
+      }
+      S += 1e-20f;
+      innerS /= rs;
+#pragma unroll
+      for (int k = 0; k < kMaxK; ++k) {
+        if (k < K && ik[k] >= 0 && (ik[k] & 31) == lane) {
+          const float dsig = a.renorm ? rs / S * (dgk[k] - innerS) : rs * dgk[k];
+          const float add = dsig * sp[k] * (1.f - sp[k]);
+#pragma unroll
+          for (int i = 0; i < NV; ++i) if (i == (ik[k] >> 5)) ds[i] += add;
+        }
+      }
+    }
+    if (a.z_lambda != 0.f) {
+      const float l = a.lse[t];
+      const float c = 2.f * a.z_lambda * l / (float)a.T;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) ds[i] += c * expf(a.logits[t * E + e] - l);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) {
+        a.ds[t * E + e] = ds[i];
+        if (a.dlogits_out) a.dlogits_out[t * E + e] = ds[i];
+      }
+    }
+    if (a.dg_out != nullptr && lane < K) {
+      float v = 0.f;
+#pragma unroll
+      for (int k = 0; k < kMaxK; ++k) if (k == lane) v = dgk[k];
+      a.dg_out[t * K + lane] = v;
+    }
+  }
+}
+
+// dW_r partials: part[c][e][d] = sum_{t in chunk c} ds[t,e] x[t,d].
+// Block tile BE x BD, thread tile TE x TD, token steps of 32.
+template <typename TX, int BE, int BD, int TE, int TD>
+__global__ void __launch_bounds__(256)
+dwr_partial_kernel(const float* __restrict__ ds, const TX* __restrict__ x,
+                   int Tn, int E, int D, int chunk, float* __restrict__ part) {
+  static_assert((BE / TE) * (BD / TD) == 256, "thread tile");
+  __shared__ __align__(16) float sds[32][BE + 4];
+  __shared__ __align__(16) float sx[32][BD + 4];
+  const int tid = threadIdx.x;
+  const int nd = BD / TD;
+  const int td = tid % nd, te = tid / nd;
+  const int d0 = blockIdx.x * BD, e0 = blockIdx.y * BE;
+  const int64_t t_beg = (int64_t)blockIdx.z * chunk;
+  const int64_t t_end = min(t_beg + chunk, (int64_t)Tn);
+  float acc[TE][TD] = {};
+  for (int64_t tb = t_beg; tb < t_end; tb += 32) {
+    for (int i = tid; i < 32 * BE; i += 256) {
+      const int r = i / BE, c = i % BE;
+      const int64_t t = tb + r;
+      sds[r][c] = (t < t_end && e0 + c < E) ? ds[t * E + e0 + c] : 0.f;
+    }
+    for (int i = tid * 8; i < 32 * BD; i += 256 * 8) {
+      const int r = i / BD, c = i % BD;
+      const int64_t t = tb + r;
+      float v[8];
+      if (t < t_end && d0 + c < D) load8(x + t * D + d0 + c, v);
+      else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sx[r][c + j] = v[j];
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int r = 0; r < 32; ++r) {
+      float av[TE], bv[TD];
+#pragma unroll
+      for (int i = 0; i < TE; ++i) av[i] = sds[r][te * TE + i];
+#pragma unroll
+      for (int j = 0; j < TD; ++j) bv[j] = sx[r][td * TD + j];
+#pragma unroll
+      for (int i = 0; i < TE; ++i)
+#pragma unroll
+        for (int j = 0; j < TD; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < TE; ++i) {
+    const int e = e0 + te * TE + i;
+    if (e >= E) continue;
+#pragma unroll
+    for (int j = 0; j < TD; ++j) {
+      const int d = d0 + td * TD + j;
+      if (d < D) part[((size_t)blockIdx.z * E + e) * D + d] = acc[i][j];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256)
+dwr_reduce_kernel(const float* __restrict__ part, int n_chunks, int64_t n,
+                  float* __restrict__ dw_r) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int c = 0; c < n_chunks; ++c) s += part[(size_t)c * n + i];
+    dw_r[i] = s;
+  }
+}
+
+// dx[t,:] = sum_e ds[t,e] W_r[e,:] + sum_{k kept} dXp[row(t,k),:] (+ shared
+// row).  64 tokens x 128 columns per block, 4 x 8 per thread.
+template <typename T>
+__global__ void __launch_bounds__(256)
+dx_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
+          const T* __restrict__ dXp, const int32_t* __restrict__ slot_row,
+          const int32_t* __restrict__ offsets, int n_shared, int Tn, int D, int E,
+          int K, T* __restrict__ dx) {
+  constexpr int BT = 64, BD = 128, BK = 16;
+  __shared__ __align__(16) float sds[BK][BT + 4];
+  __shared__ __align__(16) float sw[BK][BD + 4];
+  const int tid = threadIdx.x;
+  const int td = tid & 15, tt = tid >> 4;   // 16 x 16 threads: 8 cols, 4 tokens
+  const int64_t t0 = (int64_t)blockIdx.x * BT;
+  const int d0 = blockIdx.y * BD;
+  float acc[4][8] = {};
+  for (int k0 = 0; k0 < E; k0 += BK) {
+    for (int i = tid; i < BT * BK; i += 256) {
+      const int r = i / BK, c = i % BK;
+      const int64_t t = t0 + r;
+      sds[c][r] = (t < Tn && k0 + c < E) ? ds[t * E + k0 + c] : 0.f;
+    }
+    for (int i = tid; i < BK * BD; i += 256) {
+      const int r = i / BD, c = i % BD;
+      sw[r][c] = (k0 + r < E && d0 + c < D) ? w_r[(size_t)(k0 + r) * D + d0 + c] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < BK; ++k) {
+      float av[4], bv[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = sds[k][tt * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) bv[j] = sw[k][td * 8 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  const int d = d0 + td * 8;
+  if (d >= D) return;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t t = t0 + tt * 4 + i;
+    if (t >= Tn) continue;
+    for (int k = 0; k < K; ++k) {
+      const int64_t row = slot_row[t * K + k];
+      if (row >= 0) {
+        float v[8];
+        load8(dXp + row * D + d, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
+      }
+    }
+    if (n_shared) {
+      float v[8];
+      load8(dXp + ((int64_t)offsets[E] + t) * D + d, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
+    }
+    store8(dx + t * D + d, acc[i]);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,766 @@
+// libmoe.so: the extern "C" entry points declared in include/moe.h.
+// One translation unit (the device error word is a single __device__
+// variable); the kernels live in the .cuh files beside this one.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "router.cuh"
+#include "dispatch.cuh"
+#include "combine.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+
+using namespace moe;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+thread_local int64_t g_launches = 0;
+
+// Optional per-launch timing: a begin and an end event recorded on the
+// launching stream around every kernel (moe_profile_* entry points).
+constexpr int kProfMax = 256;
+struct Prof {
+  cudaEvent_t ev[2 * kProfMax];
+  const char* name[kProfMax];
+  int n = 0, cap = 0;
+};
+thread_local Prof g_prof;
+
+inline void prof_begin(cudaStream_t s) {
+  if (g_prof.n < g_prof.cap) cudaEventRecord(g_prof.ev[2 * g_prof.n], s);
+}
+inline void prof_end(cudaStream_t s, const char* name) {
+  if (g_prof.n < g_prof.cap) {
+    cudaEventRecord(g_prof.ev[2 * g_prof.n + 1], s);
+    g_prof.name[g_prof.n++] = name;
+  }
+}
+
+#define MOE_CK(expr)                                   \
+  do {                                                 \
+    cudaError_t e__ = (expr);                          \
+    if (e__ != cudaSuccess) {                          \
+      g_last_cuda_error = (int)e__;                    \
+      return MOE_ERR_CUDA;                             \
+    }                                                  \
+  } while (0)
+#define MOE_LAUNCHED(s, name)                          \
+  do {                                                 \
+    ++g_launches;                                      \
+    cudaError_t e__ = cudaGetLastError();              \
+    if (e__ != cudaSuccess) {                          \
+      g_last_cuda_error = (int)e__;                    \
+      return MOE_ERR_CUDA;                             \
+    }                                                  \
+    prof_end((s), (name));                             \
+  } while (0)
+#define MOE_TRY(expr)                                  \
+  do {                                                 \
+    int r__ = (expr);                                  \
+    if (r__ != MOE_OK) return r__;                     \
+  } while (0)
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+size_t act_bytes(const moe_config_t* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
+
+int validate(const moe_config_t* c) {
+  if (c == nullptr) return MOE_ERR_ARG;
+  if (c->T < 1 || c->D < 8 || (c->D % 8) || c->F < 8 || (c->F % 8)) return MOE_ERR_ARG;
+  if (c->E < 1 || c->E > 512) return MOE_ERR_ARG;
+  if (c->K < 1 || c->K > c->E || c->K > kMaxK) return MOE_ERR_ARG;
+  if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_ARG;
+  if (c->dtype != MOE_FP32 && c->dtype != MOE_BF16) return MOE_ERR_ARG;
+  if (c->score_fn != MOE_SOFTMAX && c->score_fn != MOE_SIGMOID) return MOE_ERR_ARG;
+  if (c->renorm != 0 && c->renorm != 1) return MOE_ERR_ARG;
+  if (c->n_groups < 1 || c->n_groups > 32 || (c->E % c->n_groups)) return MOE_ERR_ARG;
+  if (c->topk_groups < 1 || c->topk_groups > c->n_groups) return MOE_ERR_ARG;
+  if ((int64_t)c->topk_groups * (c->E / c->n_groups) < c->K) return MOE_ERR_ARG;
+  if (c->group_score != MOE_GMAX && c->group_score != MOE_GTOP2SUM) return MOE_ERR_ARG;
+  if (c->n_groups > 1 && c->group_score == MOE_GTOP2SUM && c->E / c->n_groups < 2)
+    return MOE_ERR_ARG;
+  if (c->aux_alpha != 0.f && c->score_fn != MOE_SOFTMAX) return MOE_ERR_ARG;
+  if (!(c->route_scale == c->route_scale) || c->min_capacity < 0) return MOE_ERR_ARG;
+  if ((int64_t)c->T * c->K > (int64_t)INT32_MAX / 2) return MOE_ERR_ARG;
+  if (c->gemm_impl != MOE_GEMM_AUTO && c->gemm_impl != MOE_GEMM_SIMT) return MOE_ERR_ARG;
+  return MOE_OK;
+}
+
+int64_t capacity_of(const moe_config_t* c) {
+  if (!(c->capacity_factor > 0.f)) return -1;
+  const double v = std::ceil((double)c->capacity_factor * (double)((int64_t)c->T * c->K) /
+                             (double)c->E);
+  return std::max<int64_t>((int64_t)v, c->min_capacity);
+}
+
+bool use_tc(const moe_config_t* c) {
+  return c->dtype == MOE_BF16 && c->gemm_impl == MOE_GEMM_AUTO && (c->D % 128) == 0 &&
+         (c->F % 128) == 0;
+}
+
+struct Layout {
+  int64_t rows_max, tiles_max, C, n_slots;
+  int n_disp_blocks, n_aux_chunks, n_dwr_chunks;
+  size_t off_bhist, off_bsent, off_aux, off_dg, off_ds, off_dwr, off_dO, off_dA13, off_dX,
+      off_dH, total;
+};
+constexpr int kAuxChunk = 512;
+constexpr int kDwrChunk = 1024;
+
+Layout layout_of(const moe_config_t* c) {
+  Layout L{};
+  L.C = capacity_of(c);
+  L.n_slots = (int64_t)c->T * c->K;
+  const int64_t kept_total = L.C < 0 ? L.n_slots : std::min<int64_t>(L.n_slots, (int64_t)c->E * L.C);
+  const int64_t pad = (int64_t)(kRowTile - 1) * std::min<int64_t>(c->E, kept_total);
+  L.rows_max = round_up(kept_total + pad, kRowTile) +
+               (c->n_shared ? round_up(c->T, kRowTile) : 0);
+  if (L.rows_max == 0) L.rows_max = kRowTile;
+  L.tiles_max = L.rows_max / kRowTile;
+  L.n_disp_blocks = (int)ceil_div(L.n_slots, kDispChunk);
+  L.n_aux_chunks = (int)ceil_div(c->T, kAuxChunk);
+  L.n_dwr_chunks = (int)ceil_div(c->T, kDwrChunk);
+  const size_t a = act_bytes(c);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += round_up((int64_t)bytes, 256); return o; };
+  L.off_bhist = take((size_t)L.n_disp_blocks * c->E * 4);
+  L.off_bsent = take((size_t)L.n_disp_blocks * 4);
+  L.off_aux = take((size_t)L.n_aux_chunks * (c->E + 1) * 4);
+  L.off_dg = take((size_t)L.n_slots * 4);
+  L.off_ds = take((size_t)c->T * c->E * 4);
+  L.off_dwr = take((size_t)L.n_dwr_chunks * c->E * c->D * 4);
+  L.off_dO = take((size_t)L.rows_max * c->D * a);
+  L.off_dA13 = take((size_t)L.rows_max * 2 * c->F * a);
+  L.off_dX = take((size_t)L.rows_max * c->D * a);
+  L.off_dH = use_tc(c) ? off : take((size_t)L.rows_max * c->F * a);
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* wsp(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// ---------------------------------------------------------------------------
+// TMA tensor maps (driver entry point fetched through the runtime)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor [n3][rows][cols] (n3 = 1 for 2D), box {64, box_rows}, 128B swizzle.
+int make_map(CUtensorMap* m, const void* ptr, int64_t n3, int64_t rows, int64_t cols,
+             uint32_t box_rows, bool three_d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) { g_last_cuda_error = (int)cudaErrorNotSupported; return MOE_ERR_CUDA; }
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)n3};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)(rows * cols * 2)};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, three_d ? 3 : 2, const_cast<void*>(ptr),
+                  dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { g_last_cuda_error = (int)cudaErrorInvalidValue; return MOE_ERR_CUDA; }
+  return MOE_OK;
+}
+
+template <int BN, int ST, int MODE, bool AMN, bool BMN, int EPI>
+int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
+              const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
+              cudaStream_t s) {
+  using S = tc::Smem<BN, ST>;
+  auto k = tc::gemm_kernel<BN, ST, MODE, AMN, BMN, EPI>;
+  MOE_CK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes));
+  const int grid = (int)std::min<int64_t>(num_sms(), total_max);
+  if (grid <= 0) return MOE_OK;
+  prof_begin(s);
+  k<<<grid, tc::kThreads, S::kBytes, s>>>(a, b, bs, p, total_hint);
+  MOE_LAUNCHED(s, name);
+  return MOE_OK;
+}
+
+int grid_for(int64_t items_per_8, int cap_mult = 8) {
+  return (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(items_per_8, 8), (int64_t)num_sms() * cap_mult));
+}
+
+// ---------------------------------------------------------------------------
+// router
+// ---------------------------------------------------------------------------
+template <typename TX>
+int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const float* off,
+                const float* bias, float* logits, float* probs, float* lse, int32_t* idx,
+                float* w, int32_t* ties, cudaStream_t s) {
+  RouteArgs a{c->T, c->E, c->K, c->score_fn, c->renorm, c->n_groups, c->topk_groups,
+              c->group_score, c->route_scale, bias, logits, probs, lse, idx, w, ties};
+  MOE_CK(cudaMemsetAsync(ties, 0, sizeof(int32_t), s));
+  const size_t fused_smem = (size_t)c->E * c->D * 4 + 8 * (size_t)c->E * 4;
+  if (c->E <= 32 && fused_smem <= 200 * 1024) {
+    const int grid = grid_for(c->T, 2);
+    auto go = [&](auto kern) -> int {
+      MOE_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fused_smem));
+      prof_begin(s);
+      kern<<<grid, 256, fused_smem, s>>>(x, w_r, off, c->D, a);
+      MOE_LAUNCHED(s, "router_fused");
+      return MOE_OK;
+    };
+    if (c->E <= 4) return go(router_fused_kernel<TX, 4>);
+    if (c->E <= 8) return go(router_fused_kernel<TX, 8>);
+    if (c->E <= 16) return go(router_fused_kernel<TX, 16>);
+    return go(router_fused_kernel<TX, 32>);
+  }
+  dim3 g1((unsigned)ceil_div(c->T, 64), (unsigned)ceil_div(c->E, 64));
+  prof_begin(s);
+  router_logits_kernel<TX><<<g1, 256, 0, s>>>(x, w_r, off, logits, c->T, c->D, c->E);
+  MOE_LAUNCHED(s, "router_logits");
+  const size_t sm = 8 * (size_t)c->E * 4;
+  const int grid = grid_for(c->T);
+  prof_begin(s);
+  if (c->E <= 32) router_route_kernel<1><<<grid, 256, sm, s>>>(logits, a);
+  else if (c->E <= 64) router_route_kernel<2><<<grid, 256, sm, s>>>(logits, a);
+  else if (c->E <= 128) router_route_kernel<4><<<grid, 256, sm, s>>>(logits, a);
+  else if (c->E <= 256) router_route_kernel<8><<<grid, 256, sm, s>>>(logits, a);
+  else router_route_kernel<16><<<grid, 256, sm, s>>>(logits, a);
+  MOE_LAUNCHED(s, "router_route");
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// aux / z loss
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+aux_partial_kernel(const float* __restrict__ probs, const float* __restrict__ lse, int T, int E,
+                   float* __restrict__ part) {
+  const int c = blockIdx.x;
+  const int t0 = c * kAuxChunk, t1 = min(T, t0 + kAuxChunk);
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    float s = 0.f;
+    if (e < E) for (int t = t0; t < t1; ++t) s += probs[(size_t)t * E + e];
+    else for (int t = t0; t < t1; ++t) s += lse[t] * lse[t];
+    part[(size_t)c * (E + 1) + e] = s;
+  }
+}
+
+__global__ void __launch_bounds__(512)
+aux_final_kernel(const float* __restrict__ part, const int32_t* __restrict__ counts, int n_chunks,
+                 int T, int E, float alpha, float lambda, float* __restrict__ losses) {
+  __shared__ float red[512];
+  __shared__ float cnt_tot_s;
+  float cnt = 0.f;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt += (float)counts[e];
+  red[threadIdx.x] = cnt;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) cnt_tot_s = red[0];
+  __syncthreads();
+  const float ctot = cnt_tot_s;
+  float acc = 0.f;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float P = 0.f;
+    for (int c = 0; c < n_chunks; ++c) P += part[(size_t)c * (E + 1) + e];
+    P /= (float)T;
+    const float f = ctot > 0.f ? (float)counts[e] / ctot : 0.f;
+    acc += f * P;
+  }
+  __syncthreads();
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    float z = 0.f;
+    for (int c = 0; c < n_chunks; ++c) z += part[(size_t)c * (E + 1) + E];
+    losses[0] = alpha * (float)E * red[0];
+    losses[1] = lambda * z / (float)T;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// expert FFN / backward GEMM sequences
+// ---------------------------------------------------------------------------
+template <typename TE>
+int simt_rows(const moe_config_t* c, const Layout& L, const void* A, int64_t lda, const void* B,
+              int64_t sbn, int64_t sbk, int64_t strideBE, const void* Bs, void* C, int64_t ldc,
+              int N, int Kd, const int32_t* tile_expert, const int32_t* stats, cudaStream_t s) {
+  SimtGemm g{};
+  g.A = A; g.lda = lda; g.B = B; g.sbn = sbn; g.sbk = sbk; g.strideBE = strideBE;
+  g.Bs = Bs ? Bs : B; g.C = C; g.ldc = ldc; g.N = N; g.Kd = Kd;
+  g.tile_expert = tile_expert; g.stats = stats; g.E = c->E;
+  dim3 grid((unsigned)(L.tiles_max * 2), (unsigned)ceil_div(N, 64));
+  prof_begin(s);
+  simt_rows_kernel<TE><<<grid, 256, 0, s>>>(g);
+  MOE_LAUNCHED(s, "simt_rows_gemm");
+  return MOE_OK;
+}
+
+template <typename TE>
+int simt_wgrad(const moe_config_t* c, const void* A, int64_t lda, const void* B, int64_t ldb,
+               int Mo, int No, void* C, void* Cs, const int32_t* offsets, const int32_t* kept,
+               cudaStream_t s) {
+  SimtGemm g{};
+  g.A = A; g.lda = lda; g.B = B; g.ldb = ldb; g.Mo = Mo; g.No = No;
+  g.C = C; g.Cs = Cs; g.offsets = offsets; g.kept = kept; g.T = c->T; g.E = c->E;
+  g.strideCE = (int64_t)Mo * No;
+  dim3 grid((unsigned)ceil_div(No, 64), (unsigned)ceil_div(Mo, 64), (unsigned)(c->E + c->n_shared));
+  prof_begin(s);
+  simt_wgrad_kernel<TE><<<grid, 256, 0, s>>>(g);
+  MOE_LAUNCHED(s, "simt_wgrad_gemm");
+  return MOE_OK;
+}
+
+tc::Params rows_params(const moe_config_t* c, int Kd, int nN, const int32_t* tile_expert,
+                       const int32_t* stats) {
+  tc::Params p{};
+  p.E = c->E; p.F = c->F; p.Kd = Kd; p.nN = nN;
+  p.tile_expert = tile_expert; p.stats = stats; p.T = c->T;
+  return p;
+}
+
+}  // namespace
+
+// ===========================================================================
+// extern "C" entry points
+// ===========================================================================
+extern "C" {
+
+int moe_get_sizes(const moe_config_t* cfg, moe_sizes_t* out) {
+  MOE_TRY(validate(cfg));
+  if (out == nullptr) return MOE_ERR_ARG;
+  const Layout L = layout_of(cfg);
+  out->rows_max = L.rows_max;
+  out->tiles_max = L.tiles_max;
+  out->capacity = L.C;
+  out->ws_bytes = L.total;
+  return MOE_OK;
+}
+
+int moe_router(const moe_config_t* c, const void* x, const float* w_r, const float* logit_offset,
+               const float* sel_bias, float* logits, float* probs, float* lse, int32_t* topk_idx,
+               float* topk_w, int32_t* near_ties, void* ws, cudaStream_t s) {
+  (void)ws;
+  MOE_TRY(validate(c));
+  if (!x || !w_r || !logits || !probs || !lse || !topk_idx || !topk_w || !near_ties)
+    return MOE_ERR_ARG;
+  if (c->dtype == MOE_BF16)
+    return router_impl(c, static_cast<const __nv_bfloat16*>(x), w_r, logit_offset, sel_bias,
+                       logits, probs, lse, topk_idx, topk_w, near_ties, s);
+  return router_impl(c, static_cast<const float*>(x), w_r, logit_offset, sel_bias, logits, probs,
+                     lse, topk_idx, topk_w, near_ties, s);
+}
+
+int moe_dispatch(const moe_config_t* c, const int32_t* topk_idx, const uint8_t* sentinel_mask,
+                 const void* x, int32_t* counts, int32_t* kept, int32_t* offsets,
+                 int32_t* slot_row, int32_t* row_slot, int32_t* tile_expert, int32_t* stats,
+                 void* x_perm, void* ws, cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!topk_idx || !x || !counts || !kept || !offsets || !slot_row || !row_slot ||
+      !tile_expert || !stats || !x_perm || !ws)
+    return MOE_ERR_ARG;
+  const Layout L = layout_of(c);
+  int32_t* bhist = wsp<int32_t>(ws, L.off_bhist);
+  int32_t* bsent = wsp<int32_t>(ws, L.off_bsent);
+  prof_begin(s);
+  disp_hist_kernel<<<L.n_disp_blocks, 256, c->E * 4, s>>>(topk_idx, sentinel_mask, L.n_slots,
+                                                          c->E, bhist, bsent);
+  MOE_LAUNCHED(s, "dispatch_hist");
+  prof_begin(s);
+  disp_scan_kernel<<<1, 1024, c->E * 8, s>>>(bhist, bsent, L.n_disp_blocks, c->E, c->T,
+                                             c->n_shared, L.C, L.rows_max, counts, kept,
+                                             offsets, tile_expert, stats);
+  MOE_LAUNCHED(s, "dispatch_scan");
+  prof_begin(s);
+  disp_rank_kernel<<<L.n_disp_blocks, 256, kDispWarps * c->E * 4, s>>>(
+      topk_idx, sentinel_mask, L.n_slots, c->E, L.C, L.rows_max, bhist, offsets, slot_row,
+      row_slot);
+  MOE_LAUNCHED(s, "dispatch_rank");
+  const int grid = grid_for(L.rows_max);
+  prof_begin(s);
+  if (c->dtype == MOE_BF16)
+    disp_gather_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), c->D, c->K, c->E, c->T, offsets, kept, tile_expert,
+        stats, row_slot, static_cast<__nv_bfloat16*>(x_perm));
+  else
+    disp_gather_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), c->D, c->K,
+                                                    c->E, c->T, offsets, kept, tile_expert,
+                                                    stats, row_slot, static_cast<float*>(x_perm));
+  MOE_LAUNCHED(s, "dispatch_gather");
+  return MOE_OK;
+}
+
+int moe_aux_loss(const moe_config_t* c, const float* probs, const float* lse,
+                 const int32_t* counts, float* losses, void* ws, cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!probs || !lse || !counts || !losses || !ws) return MOE_ERR_ARG;
+  const Layout L = layout_of(c);
+  float* part = wsp<float>(ws, L.off_aux);
+  prof_begin(s);
+  aux_partial_kernel<<<L.n_aux_chunks, 256, 0, s>>>(probs, lse, c->T, c->E, part);
+  MOE_LAUNCHED(s, "aux_partial");
+  prof_begin(s);
+  aux_final_kernel<<<1, 512, 0, s>>>(part, counts, L.n_aux_chunks, c->T, c->E, c->aux_alpha,
+                                     c->z_lambda, losses);
+  MOE_LAUNCHED(s, "aux_final");
+  return MOE_OK;
+}
+
+int moe_expert_ffn(const moe_config_t* c, const void* x_perm, const int32_t* offsets,
+                   const int32_t* tile_expert, const int32_t* stats, const void* w13,
+                   const void* w_down, const void* w13_s, const void* w_down_s, void* a13,
+                   void* h, void* o, void* ws, cudaStream_t s) {
+  (void)offsets;
+  (void)ws;
+  MOE_TRY(validate(c));
+  if (!x_perm || !tile_expert || !stats || !w13 || !w_down || !a13 || !h || !o)
+    return MOE_ERR_ARG;
+  if (c->n_shared && (!w13_s || !w_down_s)) return MOE_ERR_ARG;
+  const Layout L = layout_of(c);
+  const int D = c->D, F = c->F, E = c->E;
+  if (use_tc(c)) {
+    CUtensorMap mA, mB, mBs;
+    // gate/up + SwiGLU: A = x_perm [rows, D]; B = w13 [E, 2F, D] K-major
+    constexpr int BN1 = 256;
+    MOE_TRY(make_map(&mA, x_perm, 1, L.rows_max, D, 128, false));
+    MOE_TRY(make_map(&mB, w13, E, 2 * F, D, BN1 / 2, true));
+    MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, BN1 / 2, true));
+    tc::Params p = rows_params(c, D, F / (BN1 / 2), tile_expert, stats);
+    p.out = static_cast<__nv_bfloat16*>(a13); p.ld_out = 2 * F;
+    p.out2 = static_cast<__nv_bfloat16*>(h); p.ld_out2 = F;
+    MOE_TRY((launch_tc<BN1, 4, tc::MODE_ROWS, false, false, tc::EPI_SWIGLU>(
+        "tc_gate_up_swiglu", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
+    // down: A = h [rows, F]; B = w_down [E, D, F] K-major
+    MOE_TRY(make_map(&mA, h, 1, L.rows_max, F, 128, false));
+    if (D % 256 == 0) {
+      MOE_TRY(make_map(&mB, w_down, E, D, F, 256, true));
+      MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, 256, true));
+      tc::Params q = rows_params(c, F, D / 256, tile_expert, stats);
+      q.out = static_cast<__nv_bfloat16*>(o); q.ld_out = D;
+      return launch_tc<256, 4, tc::MODE_ROWS, false, false, tc::EPI_STORE>(
+          "tc_down", mA, mB, mBs, q, L.tiles_max * q.nN, 0, s);
+    }
+    MOE_TRY(make_map(&mB, w_down, E, D, F, 128, true));
+    MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, 128, true));
+    tc::Params q = rows_params(c, F, D / 128, tile_expert, stats);
+    q.out = static_cast<__nv_bfloat16*>(o); q.ld_out = D;
+    return launch_tc<128, 6, tc::MODE_ROWS, false, false, tc::EPI_STORE>(
+        "tc_down", mA, mB, mBs, q, L.tiles_max * q.nN, 0, s);
+  }
+  auto go = [&](auto tag) -> int {
+    using TE = decltype(tag);
+    MOE_TRY(simt_rows<TE>(c, L, x_perm, D, w13, D, 1, (int64_t)2 * F * D, w13_s, a13, 2 * F,
+                          2 * F, D, tile_expert, stats, s));
+    prof_begin(s);
+    swiglu_fwd_kernel<TE><<<num_sms() * 8, 256, 0, s>>>(static_cast<const TE*>(a13),
+                                                         static_cast<TE*>(h), stats, F);
+    MOE_LAUNCHED(s, "swiglu_fwd");
+    return simt_rows<TE>(c, L, h, F, w_down, F, 1, (int64_t)D * F, w_down_s, o, D, D, F,
+                         tile_expert, stats, s);
+  };
+  if (c->dtype == MOE_BF16) return go(__nv_bfloat16{});
+  return go(float{});
+}
+
+int moe_combine(const moe_config_t* c, const void* o, const int32_t* slot_row,
+                const float* topk_w, const int32_t* offsets, void* y, cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!o || !slot_row || !topk_w || !offsets || !y) return MOE_ERR_ARG;
+  const int grid = grid_for(c->T);
+  prof_begin(s);
+  if (c->dtype == MOE_BF16)
+    combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(o), slot_row, topk_w, offsets, c->n_shared, c->T,
+        c->D, c->K, c->E, static_cast<__nv_bfloat16*>(y));
+  else
+    combine_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(o), slot_row, topk_w,
+                                               offsets, c->n_shared, c->T, c->D, c->K, c->E,
+                                               static_cast<float*>(y));
+  MOE_LAUNCHED(s, "combine");
+  return MOE_OK;
+}
+
+int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const float* logits,
+                 const float* probs, const float* lse, const int32_t* topk_idx,
+                 const float* topk_w, const int32_t* counts, const int32_t* kept,
+                 const int32_t* offsets, const int32_t* slot_row, const int32_t* row_slot,
+                 const int32_t* tile_expert, const int32_t* stats, const void* x_perm,
+                 const void* a13, const void* h, const void* o, const void* w13,
+                 const void* w_down, const void* w13_s, const void* w_down_s, const void* dy,
+                 void* dx, float* dw_r, void* dw13, void* dw_down, void* dw13_s,
+                 void* dw_down_s, float* dg_out, float* dlogits_out, void* ws, cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!x || !w_r || !logits || !probs || !lse || !topk_idx || !topk_w || !counts || !kept ||
+      !offsets || !slot_row || !row_slot || !tile_expert || !stats || !x_perm || !a13 || !h ||
+      !o || !w13 || !w_down || !dy || !dx || !dw_r || !dw13 || !dw_down || !ws)
+    return MOE_ERR_ARG;
+  if (c->n_shared && (!w13_s || !w_down_s || !dw13_s || !dw_down_s)) return MOE_ERR_ARG;
+  const Layout L = layout_of(c);
+  const int D = c->D, F = c->F, E = c->E, T = c->T, K = c->K;
+  float* dg = wsp<float>(ws, L.off_dg);
+  float* ds = wsp<float>(ws, L.off_ds);
+  float* dwr_part = wsp<float>(ws, L.off_dwr);
+  void* dO = wsp<void>(ws, L.off_dO);
+  void* dA13 = wsp<void>(ws, L.off_dA13);
+  void* dXp = wsp<void>(ws, L.off_dX);
+  void* dH = wsp<void>(ws, L.off_dH);
+  const bool bf = c->dtype == MOE_BF16;
+
+  // 1. per row: gate gradient dg = <o, dy>, and dO = g * dy
+  {
+    const int grid = grid_for(L.rows_max);
+    prof_begin(s);
+    if (bf)
+      bwd_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dy), topk_w,
+          row_slot, offsets, kept, tile_expert, stats, K, E, T, D, dg,
+          static_cast<__nv_bfloat16*>(dO));
+    else
+      bwd_rows_kernel<float><<<grid, 256, 0, s>>>(
+          static_cast<const float*>(o), static_cast<const float*>(dy), topk_w, row_slot, offsets,
+          kept, tile_expert, stats, K, E, T, D, dg, static_cast<float*>(dO));
+    MOE_LAUNCHED(s, "bwd_gate_grad_rows");
+  }
+  // 2. router backward: dlogits
+  {
+    RouterBwdArgs a{T, E, K, c->score_fn, c->renorm, c->route_scale, c->aux_alpha, c->z_lambda,
+                    logits, probs, lse, topk_idx, topk_w, slot_row, dg, counts, ds, dlogits_out,
+                    dg_out};
+    const int grid = grid_for(T);
+    prof_begin(s);
+    if (E <= 32) router_bwd_kernel<1><<<grid, 256, 0, s>>>(a);
+    else if (E <= 64) router_bwd_kernel<2><<<grid, 256, 0, s>>>(a);
+    else if (E <= 128) router_bwd_kernel<4><<<grid, 256, 0, s>>>(a);
+    else if (E <= 256) router_bwd_kernel<8><<<grid, 256, 0, s>>>(a);
+    else router_bwd_kernel<16><<<grid, 256, 0, s>>>(a);
+    MOE_LAUNCHED(s, "router_bwd");
+  }
+  // 3-6. expert GEMMs
+  if (use_tc(c)) {
+    CUtensorMap mA, mB, mBs;
+    const int BNf = (F % 256 == 0) ? 256 : 128;
+    const int BNd = (D % 256 == 0) ? 256 : 128;
+    // 3. dgrad down + SwiGLU backward: dA13 = swiglu'(dO . w_down[e])
+    MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 128, false));
+    MOE_TRY(make_map(&mB, w_down, E, D, F, 64, true));                 // dims {F, D, E}
+    MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, 64, true));
+    {
+      tc::Params p = rows_params(c, D, F / BNf, tile_expert, stats);
+      p.out = static_cast<__nv_bfloat16*>(dA13); p.ld_out = 2 * F;
+      p.aux = static_cast<const __nv_bfloat16*>(a13); p.ld_aux = 2 * F;
+      if (BNf == 256)
+        MOE_TRY((launch_tc<256, 4, tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD>(
+            "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
+      else
+        MOE_TRY((launch_tc<128, 6, tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD>(
+            "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
+    }
+    // 4. wgrad down: dW_down[e] = dO^T h over the expert's rows
+    MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 64, false));
+    MOE_TRY(make_map(&mB, h, 1, L.rows_max, F, 64, false));
+    {
+      tc::Params p{};
+      p.E = E; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
+      p.n_groups = E + c->n_shared; p.nMo = D / 128; p.nNo = F / BNf; p.No = F;
+      p.strideCE = (int64_t)D * F;
+      p.out = static_cast<__nv_bfloat16*>(dw_down);
+      p.out_shared = static_cast<__nv_bfloat16*>(dw_down_s);
+      const int total = p.n_groups * p.nMo * p.nNo;
+      if (BNf == 256)
+        MOE_TRY((launch_tc<256, 4, tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
+            "tc_wgrad_down", mA, mB, mB, p, total, total, s)));
+      else
+        MOE_TRY((launch_tc<128, 6, tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
+            "tc_wgrad_down", mA, mB, mB, p, total, total, s)));
+    }
+    // 5. dgrad gate/up: dX_perm = dA13 . w13[e]
+    MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 128, false));
+    MOE_TRY(make_map(&mB, w13, E, 2 * F, D, 64, true));                  // dims {D, 2F, E}
+    MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, 64, true));
+    {
+      tc::Params p = rows_params(c, 2 * F, D / BNd, tile_expert, stats);
+      p.out = static_cast<__nv_bfloat16*>(dXp); p.ld_out = D;
+      if (BNd == 256)
+        MOE_TRY((launch_tc<256, 4, tc::MODE_ROWS, false, true, tc::EPI_STORE>(
+            "tc_dgrad_gate_up", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
+      else
+        MOE_TRY((launch_tc<128, 6, tc::MODE_ROWS, false, true, tc::EPI_STORE>(
+            "tc_dgrad_gate_up", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
+    }
+    // 6. wgrad gate/up: dW13[e] = dA13^T x_perm
+    MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 64, false));
+    MOE_TRY(make_map(&mB, x_perm, 1, L.rows_max, D, 64, false));
+    {
+      tc::Params p{};
+      p.E = E; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
+      p.n_groups = E + c->n_shared; p.nMo = 2 * F / 128; p.nNo = D / BNd; p.No = D;
+      p.strideCE = (int64_t)2 * F * D;
+      p.out = static_cast<__nv_bfloat16*>(dw13);
+      p.out_shared = static_cast<__nv_bfloat16*>(dw13_s);
+      const int total = p.n_groups * p.nMo * p.nNo;
+      if (BNd == 256)
+        MOE_TRY((launch_tc<256, 4, tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
+            "tc_wgrad_gate_up", mA, mB, mB, p, total, total, s)));
+      else
+        MOE_TRY((launch_tc<128, 6, tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
+            "tc_wgrad_gate_up", mA, mB, mB, p, total, total, s)));
+    }
+  } else {
+    auto go = [&](auto tag) -> int {
+      using TE = decltype(tag);
+      // 3. dH = dO . w_down[e]  (B(n=j, k=d) = w_down[e][d][j])
+      MOE_TRY(simt_rows<TE>(c, L, dO, D, w_down, 1, F, (int64_t)D * F, w_down_s, dH, F, F, D,
+                            tile_expert, stats, s));
+      prof_begin(s);
+      swiglu_bwd_kernel<TE><<<num_sms() * 8, 256, 0, s>>>(
+          static_cast<const TE*>(dH), static_cast<const TE*>(a13), static_cast<TE*>(dA13),
+          stats, F);
+      MOE_LAUNCHED(s, "swiglu_bwd");
+      // 4. dW_down[e] = dO^T h
+      MOE_TRY(simt_wgrad<TE>(c, dO, D, h, F, D, F, dw_down, dw_down_s, offsets, kept, s));
+      // 5. dX_perm = dA13 . w13[e]  (B(n=d, k=j) = w13[e][j][d])
+      MOE_TRY(simt_rows<TE>(c, L, dA13, 2 * F, w13, 1, D, (int64_t)2 * F * D, w13_s, dXp, D, D,
+                            2 * F, tile_expert, stats, s));
+      // 6. dW13[e] = dA13^T x_perm
+      return simt_wgrad<TE>(c, dA13, 2 * F, x_perm, D, 2 * F, D, dw13, dw13_s, offsets, kept, s);
+    };
+    if (bf) MOE_TRY(go(__nv_bfloat16{}));
+    else MOE_TRY(go(float{}));
+  }
+  // 7. dW_r = ds^T x (two deterministic stages)
+  {
+    const int nc = L.n_dwr_chunks;
+    prof_begin(s);
+    if (E <= 8) {
+      dim3 g((unsigned)ceil_div(D, 256), 1, (unsigned)nc);
+      if (bf) dwr_partial_kernel<__nv_bfloat16, 8, 256, 2, 4><<<g, 256, 0, s>>>(
+          ds, static_cast<const __nv_bfloat16*>(x), T, E, D, kDwrChunk, dwr_part);
+      else dwr_partial_kernel<float, 8, 256, 2, 4><<<g, 256, 0, s>>>(
+          ds, static_cast<const float*>(x), T, E, D, kDwrChunk, dwr_part);
+    } else {
+      dim3 g((unsigned)ceil_div(D, 64), (unsigned)ceil_div(E, 64), (unsigned)nc);
+      if (bf) dwr_partial_kernel<__nv_bfloat16, 64, 64, 4, 4><<<g, 256, 0, s>>>(
+          ds, static_cast<const __nv_bfloat16*>(x), T, E, D, kDwrChunk, dwr_part);
+      else dwr_partial_kernel<float, 64, 64, 4, 4><<<g, 256, 0, s>>>(
+          ds, static_cast<const float*>(x), T, E, D, kDwrChunk, dwr_part);
+    }
+    MOE_LAUNCHED(s, "router_dw_partial");
+    const int64_t n = (int64_t)E * D;
+    prof_begin(s);
+    dwr_reduce_kernel<<<(int)std::min<int64_t>(ceil_div(n, 256), num_sms() * 8), 256, 0, s>>>(
+        dwr_part, nc, n, dw_r);
+    MOE_LAUNCHED(s, "router_dw_reduce");
+  }
+  // 8. dx = unpermute-sum(dX_perm) + shared + ds . w_r
+  {
+    dim3 g((unsigned)ceil_div(T, 64), (unsigned)ceil_div(D, 128));
+    prof_begin(s);
+    if (bf)
+      dx_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(ds, w_r, static_cast<const __nv_bfloat16*>(dXp),
+                                                 slot_row, offsets, c->n_shared, T, D, E, K,
+                                                 static_cast<__nv_bfloat16*>(dx));
+    else
+      dx_kernel<float><<<g, 256, 0, s>>>(ds, w_r, static_cast<const float*>(dXp), slot_row,
+                                         offsets, c->n_shared, T, D, E, K,
+                                         static_cast<float*>(dx));
+    MOE_LAUNCHED(s, "dx_unpermute_router");
+  }
+  return MOE_OK;
+}
+
+int moe_check_status(cudaStream_t s, uint32_t* bits) {
+  MOE_CK(cudaStreamSynchronize(s));
+  unsigned v = 0, zero = 0;
+  MOE_CK(cudaMemcpyFromSymbol(&v, moe::g_dev_error, sizeof(v)));
+  MOE_CK(cudaMemcpyToSymbol(moe::g_dev_error, &zero, sizeof(zero)));
+  if (bits) *bits = v;
+  return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+const char* moe_status_string(int st) {
+  switch (st) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_ARG: return "invalid argument or unsupported configuration";
+    case MOE_ERR_CUDA: return "CUDA error (see moe_last_cuda_error)";
+    case MOE_ERR_DEVICE: return "device error word set (bad expert id, timeout or row overflow)";
+    case MOE_ERR_TIMEOUT: return "bounded device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+int moe_profile_enable(int max_launches) {
+  if (max_launches < 1 || max_launches > kProfMax) return MOE_ERR_ARG;
+  for (int i = 0; i < 2 * g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
+  g_prof.cap = 0;
+  g_prof.n = 0;
+  for (int i = 0; i < 2 * max_launches; ++i) MOE_CK(cudaEventCreate(&g_prof.ev[i]));
+  g_prof.cap = max_launches;
+  return MOE_OK;
+}
+
+int moe_profile_reset(void) {
+  g_prof.n = 0;
+  return MOE_OK;
+}
+
+int moe_profile_read(float* ms, int max) {
+  if (ms == nullptr) return MOE_ERR_ARG;
+  const int n = std::min(g_prof.n, max);
+  for (int i = 0; i < n; ++i)
+    MOE_CK(cudaEventElapsedTime(&ms[i], g_prof.ev[2 * i], g_prof.ev[2 * i + 1]));
+  return n;
+}
+
+const char* moe_profile_name(int i) {
+  return (i >= 0 && i < g_prof.n) ? g_prof.name[i] : "";
+}
+
+int moe_profile_disable(void) {
+  for (int i = 0; i < 2 * g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
+  g_prof.cap = 0;
+  g_prof.n = 0;
+  return MOE_OK;
+}
+
+int64_t moe_launch_count(int reset) {
+  const int64_t v = g_launches;
+  if (reset) g_launches = 0;
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,319 @@
+// Router: fp32 logits, softmax / sigmoid scores, group-limited top-K and
+// gate weights (variants A and B).
+//
+// Follows "08 MoE" (STA324 notes) §8.2 (s = x W_r, TopK on the logits,
+// variant A = truncate, variant B = softmax over the selected logits) and
+// §8.6 (sigmoid affinities, selection-only bias b_e, weights from the raw
+// affinity), the "8-MoE" lecture notes (router in full precision) and the
+// MoE training course page (group-limited routing, optional scaling).
+//
+// One warp routes one token.  Lane l holds experts e = l + 32*i, i < NV.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+struct RouteArgs {
+  int T, E, K;
+  int score_fn, renorm;
+  int n_groups, topk_groups, group_score;
+  float route_scale;
+  const float* sel_bias;   // [E] or null
+  float* logits;           // [T,E] (written by the fused path only)
+  float* probs;            // [T,E]
+  float* lse;              // [T]
+  int32_t* topk_idx;       // [T,K]
+  float* topk_w;           // [T,K]
+  int32_t* near_ties;      // [1]
+};
+
+constexpr int kMaxK = 16;
+
+// (value, index) argmax across the warp: larger value wins, then lower index.
+__device__ __forceinline__ void warp_argmax(float& v, int& e) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    float ov = __shfl_xor_sync(0xffffffffu, v, o);
+    int oe = __shfl_xor_sync(0xffffffffu, e, o);
+    if (ov > v || (ov == v && oe < e)) { v = ov; e = oe; }
+  }
+}
+
+template <int NV>
+__device__ __forceinline__ float pick(const float (&a)[NV], int i) {
+  float r = 0.f;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) if (j == i) r = a[j];
+  return r;
+}
+
+// Routes token t given its logits s[i] (expert lane + 32 i).  `gsm` is
+// per-warp shared scratch of at least E floats (group-limited routing).
+template <int NV>
+__device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
+                            float* gsm, int lane) {
+  const int E = a.E;
+  const float NEG = -INFINITY;
+  // logsumexp (z-loss, and softmax normaliser)
+  float m = NEG;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) if (lane + 32 * i < E) m = fmaxf(m, s[i]);
+  m = warp_max(m);
+  float ex[NV];
+  float z = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    ex[i] = (lane + 32 * i < E) ? expf(s[i] - m) : 0.f;
+    z += ex[i];
+  }
+  z = warp_sum(z);
+  const float lse = m + logf(z);
+  float p[NV], u[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int e = lane + 32 * i;
+    if (a.score_fn == MOE_SOFTMAX) {
+      p[i] = ex[i] / z;
+      u[i] = s[i];
+    } else {
+      p[i] = 1.0f / (1.0f + expf(-s[i]));
+      u[i] = p[i] + (a.sel_bias != nullptr && e < E ? a.sel_bias[e] : 0.f);
+    }
+    if (e >= E) u[i] = NEG;
+    else a.probs[(size_t)t * E + e] = p[i];
+  }
+  if (lane == 0) a.lse[t] = lse;
+
+  // group limit
+  float gmargin = INFINITY;
+  if (a.n_groups > 1) {
+    const int gsz = E / a.n_groups;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) gsm[e] = u[i];
+    }
+    __syncwarp();
+    float gs = NEG;
+    if (lane < a.n_groups) {
+      float b1 = NEG, b2 = NEG;
+      for (int j = 0; j < gsz; ++j) {
+        const float v = gsm[lane * gsz + j];
+        if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
+      }
+      gs = (a.group_score == MOE_GMAX) ? b1 : b1 + b2;
+    }
+    __syncwarp();
+    unsigned keep = 0u;
+    bool taken = false;
+    float last = NEG;
+    for (int r = 0; r <= a.topk_groups && r < a.n_groups; ++r) {
+      float v = taken ? NEG : gs;
+      int g = (lane < a.n_groups && !taken) ? lane : 0x7fffffff;
+      warp_argmax(v, g);
+      if (r < a.topk_groups) {
+        keep |= 1u << g;
+        if (lane == g) taken = true;
+        last = v;
+      } else {
+        gmargin = last - v;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((keep >> (e / gsz)) & 1u)) u[i] = NEG;
+    }
+  }
+
+  // top-K (+1 round for the boundary margin)
+  int sel_e[kMaxK];
+  float sel_s[kMaxK], sel_p[kMaxK];
+  unsigned taken = 0u;
+  float uk = NEG, margin = INFINITY;
+#pragma unroll
+  for (int k = 0; k <= kMaxK; ++k) {
+    if (k > a.K) break;
+    float v = NEG;
+    int e = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int ei = lane + 32 * i;
+      const bool ok = ei < E && !((taken >> i) & 1u);
+      if (ok && (u[i] > v || (u[i] == v && ei < e))) { v = u[i]; e = ei; }
+    }
+    warp_argmax(v, e);
+    if (k < a.K) {
+      const int owner = e & 31, slot = e >> 5;
+      const float sv = __shfl_sync(0xffffffffu, pick<NV>(s, slot), owner);
+      const float pv = __shfl_sync(0xffffffffu, pick<NV>(p, slot), owner);
+      if (lane == owner) taken |= 1u << slot;
+      if (k < kMaxK) { sel_e[k] = e; sel_s[k] = sv; sel_p[k] = pv; }
+      uk = v;
+    } else if (v != NEG) {
+      margin = uk - v;
+    }
+  }
+  if (lane == 0 && (margin < kNearTie || gmargin < kNearTie))
+    atomicAdd(a.near_ties, 1);
+
+  // gate weights
+  float g[kMaxK];
+  float denom = 0.f;
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) {
+    if (k >= a.K) break;
+    if (a.score_fn == MOE_SOFTMAX) {
+      g[k] = a.renorm ? expf(sel_s[k] - sel_s[0]) : sel_p[k];
+    } else {
+      g[k] = sel_p[k];
+    }
+    denom += g[k];
+  }
+  if (a.renorm) denom = (a.score_fn == MOE_SOFTMAX) ? denom : denom + 1e-20f;
+#pragma unroll
+  for (int k = 0; k < kMaxK; ++k) {
+    if (k >= a.K) break;
+    float w = a.renorm ? g[k] / denom : g[k];
+    w *= a.route_scale;
+    if (lane == k) {
+      a.topk_idx[(size_t)t * a.K + k] = sel_e[k];
+      a.topk_w[(size_t)t * a.K + k] = w;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// E <= 32: logits and routing fused; W_r staged once per block in shared
+// memory, one warp per token, grid-stride over tokens.
+// ---------------------------------------------------------------------------
+template <typename TX, int EB>
+__global__ void __launch_bounds__(256)
+router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
+                    const float* __restrict__ offset, int D, RouteArgs a) {
+  extern __shared__ __align__(16) float smem[];
+  float* ws = smem;                         // [E, D]
+  float* gsm_all = smem + (size_t)a.E * D;  // [8 warps, E]
+  const int E = a.E;
+  for (int i = threadIdx.x * 4; i < E * D; i += blockDim.x * 4)
+    *reinterpret_cast<float4*>(ws + i) = *reinterpret_cast<const float4*>(w_r + i);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* gsm = gsm_all + warp * E;
+  for (int t = blockIdx.x * 8 + warp; t < a.T; t += gridDim.x * 8) {
+    const TX* xr = x + (size_t)t * D;
+    float acc[EB];
+#pragma unroll
+    for (int e = 0; e < EB; ++e) acc[e] = 0.f;
+    for (int d = lane * 8; d < D; d += 256) {
+      float xv[8];
+      load8(xr + d, xv);
+#pragma unroll
+      for (int e = 0; e < EB; ++e) {
+        if (e < E) {
+          const float* wrow = ws + (size_t)e * D + d;
+          float4 w0 = *reinterpret_cast<const float4*>(wrow);
+          float4 w1 = *reinterpret_cast<const float4*>(wrow + 4);
+          acc[e] = fmaf(xv[0], w0.x, acc[e]); acc[e] = fmaf(xv[1], w0.y, acc[e]);
+          acc[e] = fmaf(xv[2], w0.z, acc[e]); acc[e] = fmaf(xv[3], w0.w, acc[e]);
+          acc[e] = fmaf(xv[4], w1.x, acc[e]); acc[e] = fmaf(xv[5], w1.y, acc[e]);
+          acc[e] = fmaf(xv[6], w1.z, acc[e]); acc[e] = fmaf(xv[7], w1.w, acc[e]);
+        }
+      }
+    }
+    float s[1];
+    s[0] = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < EB; ++e) {
+      const float v = warp_sum(acc[e]);
+      if (lane == e) s[0] = v;
+    }
+    if (lane < E) {
+      if (offset != nullptr) s[0] += offset[lane];
+      a.logits[(size_t)t * E + lane] = s[0];
+    }
+    route_token<1>(t, s, a, gsm, lane);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// E > 32: tiled fp32 logits GEMM (64 tokens x 64 experts per block, 4x4 per
+// thread), then a routing kernel reading the logits back.
+// ---------------------------------------------------------------------------
+template <typename TX>
+__global__ void __launch_bounds__(256)
+router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
+                     const float* __restrict__ offset, float* __restrict__ logits,
+                     int T, int D, int E) {
+  constexpr int BT = 64, BE = 64, BK = 32;
+  __shared__ __align__(16) float xs[BK][BT + 4];
+  __shared__ __align__(16) float wsm[BK][BE + 4];
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int t0 = blockIdx.x * BT, e0 = blockIdx.y * BE;
+  float acc[4][4] = {};
+  const int lr = tid >> 2, lc = (tid & 3) * 8;   // loader: row, 8-wide column
+  for (int k0 = 0; k0 < D; k0 += BK) {
+    {
+      float v[8];
+      const int t = t0 + lr;
+      if (t < T && k0 + lc < D) load8(x + (size_t)t * D + k0 + lc, v);
+      else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xs[lc + j][lr] = v[j];
+      const int e = e0 + lr;
+      if (e < E && k0 + lc < D) load8(w_r + (size_t)e * D + k0 + lc, v);
+      else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) wsm[lc + j][lr] = v[j];
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < BK; ++k) {
+      const float4 av = *reinterpret_cast<const float4*>(&xs[k][ty * 4]);
+      const float4 bv = *reinterpret_cast<const float4*>(&wsm[k][tx * 4]);
+      const float ar[4] = {av.x, av.y, av.z, av.w};
+      const float br[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(ar[i], br[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) logits[(size_t)t * E + e] = acc[i][j] + (offset ? offset[e] : 0.f);
+    }
+  }
+}
+
+template <int NV>
+__global__ void __launch_bounds__(256)
+router_route_kernel(const float* __restrict__ logits, RouteArgs a) {
+  extern __shared__ __align__(16) float gsm_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* gsm = gsm_all + warp * a.E;
+  for (int t = blockIdx.x * 8 + warp; t < a.T; t += gridDim.x * 8) {
+    float s[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      s[i] = e < a.E ? logits[(size_t)t * a.E + e] : -INFINITY;
+    }
+    route_token<NV>(t, s, a, gsm, lane);
+  }
+}
+
+}  // namespace moe

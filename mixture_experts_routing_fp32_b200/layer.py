@@ -1,0 +1,90 @@
+"""One MoE layer on one GPU: buffers + the forward/backward call sequence.
+
+The layer owns every device buffer the C ABI needs (allocated once with
+torch, stable pointers, so a whole step can be captured in a CUDA graph)
+and issues the entry points in order on the current stream:
+
+  forward : moe_router -> moe_dispatch -> moe_aux_loss -> moe_expert_ffn
+            -> moe_combine
+  backward: moe_backward
+
+No host synchronisation happens inside forward or backward.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import api
+from ._lib import MOE_BF16
+
+
+class MoELayer:
+    def __init__(self, cfg, device="cuda"):
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.sizes = api.moe_get_sizes(cfg)
+        c, z = cfg, self.sizes
+        dev = self.device
+        act = torch.bfloat16 if c.dtype == MOE_BF16 else torch.float32
+        self.act_dtype = act
+        T, D, E, K, F = c.T, c.D, c.E, c.K, c.F
+        R = int(z.rows_max)
+        f32, i32 = torch.float32, torch.int32
+        e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
+        self.logits, self.probs, self.lse = e((T, E), f32), e((T, E), f32), e((T,), f32)
+        self.topk_idx, self.topk_w = e((T, K), i32), e((T, K), f32)
+        self.near_ties = e((1,), i32)
+        self.counts, self.kept = e((E,), i32), e((E,), i32)
+        self.offsets = e((E + 2,), i32)
+        self.slot_row, self.row_slot = e((T * K,), i32), e((R,), i32)
+        self.tile_expert, self.stats = e((int(z.tiles_max),), i32), e((4,), i32)
+        self.x_perm, self.a13 = e((R, D), act), e((R, 2 * F), act)
+        self.h, self.o = e((R, F), act), e((R, D), act)
+        self.y = e((T, D), act)
+        self.losses = torch.zeros(2, dtype=f32, device=dev)
+        self.ws = e((max(int(z.ws_bytes), 256),), torch.uint8)
+        # gradients
+        self.dx = e((T, D), act)
+        self.dw_r = e((E, D), f32)
+        self.dw13, self.dw_down = e((E, 2 * F, D), act), e((E, D, F), act)
+        self.dw13_s = e((2 * F, D), act) if c.n_shared else None
+        self.dw_down_s = e((D, F), act) if c.n_shared else None
+        self.dg = e((T, K), f32)
+        self.dlogits = e((T, E), f32)
+        self._inputs = None
+
+    # -- forward -----------------------------------------------------------
+    def forward(self, x, w_r, w13, w_down, w13_s=None, w_down_s=None,
+                logit_offset=None, sel_bias=None, sentinel_mask=None):
+        c = self.cfg
+        api.moe_router(c, x, w_r, logit_offset, sel_bias, self.logits, self.probs,
+                       self.lse, self.topk_idx, self.topk_w, self.near_ties, self.ws)
+        api.moe_dispatch(c, self.topk_idx, sentinel_mask, x, self.counts, self.kept,
+                         self.offsets, self.slot_row, self.row_slot, self.tile_expert,
+                         self.stats, self.x_perm, self.ws)
+        if c.aux_alpha != 0.0 or c.z_lambda != 0.0:
+            api.moe_aux_loss(c, self.probs, self.lse, self.counts, self.losses, self.ws)
+        api.moe_expert_ffn(c, self.x_perm, self.offsets, self.tile_expert, self.stats,
+                           w13, w_down, w13_s, w_down_s, self.a13, self.h, self.o,
+                           self.ws)
+        api.moe_combine(c, self.o, self.slot_row, self.topk_w, self.offsets, self.y)
+        self._inputs = (x, w_r, w13, w_down, w13_s, w_down_s)
+        return self.y
+
+    # -- backward ----------------------------------------------------------
+    def backward(self, dy, want_dg=True, want_dlogits=True):
+        x, w_r, w13, w_down, w13_s, w_down_s = self._inputs
+        api.moe_backward(
+            self.cfg, x, w_r, self.logits, self.probs, self.lse, self.topk_idx,
+            self.topk_w, self.counts, self.kept, self.offsets, self.slot_row,
+            self.row_slot, self.tile_expert, self.stats, self.x_perm, self.a13,
+            self.h, self.o, w13, w_down, w13_s, w_down_s, dy, self.dx, self.dw_r,
+            self.dw13, self.dw_down, self.dw13_s, self.dw_down_s,
+            self.dg if want_dg else None, self.dlogits if want_dlogits else None,
+            self.ws)
+        return self.dx
+
+    def step(self, x, dy, **weights):
+        """One forward + backward pass (the unit the benchmark times)."""
+        self.forward(x, **weights)
+        return self.backward(dy)

@@ -1,0 +1,111 @@
+"""The C-ABI library: builds, loads, exports every declared symbol, and
+validates configurations on the host (no CUDA calls, no GPU needed)."""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from mixture_experts_routing_fp32_b200 import _lib as C
+from mixture_experts_routing_fp32_b200 import api
+from mixture_experts_routing_fp32_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return C.lib()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|int64_t|const char\*)\s+(moe_\w+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(C.EXPORTS) == names
+
+
+def test_config_struct_layout_matches_header():
+    # 12 int32 fields, then float, int32, 3 floats, int32 = 18 x 4 bytes
+    assert ctypes.sizeof(C.MoeConfig) == 18 * 4
+    assert ctypes.sizeof(C.MoeSizes) == 32
+
+
+def _rows_max(T, K, E, C_, n_shared):
+    kept_total = T * K if C_ is None else min(T * K, E * C_)
+    pad = 127 * min(E, kept_total)
+    r = -(-(kept_total + pad) // 128) * 128
+    return r + (-(-T // 128) * 128 if n_shared else 0)
+
+
+@pytest.mark.parametrize("T,D,E,K,F,c,ns", [
+    (4096, 768, 4, 1, 2048, 0.0, 0),
+    (32768, 4096, 8, 2, 14336, 1.25, 0),
+    (8192, 7168, 256, 8, 2048, 0.0, 1),
+    (256, 64, 4, 2, 64, 1.1, 0),
+])
+def test_sizes(lib, T, D, E, K, F, c, ns):
+    cfg = api.make_config(T, D, E, K, F, capacity_factor=c, n_shared=ns,
+                          score_fn=1 if ns else 0)
+    s = api.moe_get_sizes(cfg)
+    Cap = None if c <= 0 else max(math.ceil(c * T * K / E), 0)
+    assert s.capacity == (-1 if Cap is None else Cap)
+    assert s.rows_max == _rows_max(T, K, E, Cap, ns)
+    assert s.tiles_max * 128 == s.rows_max
+    assert s.ws_bytes > 0
+    if T == 256:
+        assert s.capacity == 141        # the course page's lab: ceil(1.1*256*2/4)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(K=5),                        # K > E
+    dict(K=17, E=32),                 # K > 16
+    dict(D=30),                       # D % 8
+    dict(E=513, K=2),                 # E > 512
+    dict(n_groups=3),                 # E % n_groups
+    dict(n_groups=2, topk_groups=1, K=3),   # topk_groups * E/n_groups < K
+    dict(aux_alpha=0.01, score_fn=1),       # aux needs softmax scores
+    dict(dtype="fp16"),               # maps to fp32 -> still valid; replaced below
+])
+def test_invalid_configs_rejected(lib, bad):
+    kw = dict(T=64, D=32, E=4, K=2, F=64)
+    kw.update(bad)
+    if kw.get("dtype") == "fp16":
+        cfg = api.make_config(**{k: v for k, v in kw.items() if k != "dtype"})
+        cfg.dtype = 7
+    else:
+        cfg = api.make_config(**kw)
+    out = C.MoeSizes()
+    assert lib.moe_get_sizes(ctypes.byref(cfg), ctypes.byref(out)) == C.MOE_ERR_ARG
+
+
+def test_null_pointers_rejected_before_any_launch(lib):
+    cfg = api.make_config(64, 32, 4, 2, 64, dtype="fp32")
+    args = [None] * 12
+    assert lib.moe_router(ctypes.byref(cfg), *args) == C.MOE_ERR_ARG
+    assert lib.moe_dispatch(ctypes.byref(cfg), *([None] * 13)) == C.MOE_ERR_ARG
+    assert lib.moe_backward(ctypes.byref(cfg), *([None] * 33)) == C.MOE_ERR_ARG
+    assert lib.moe_status_string(C.MOE_ERR_ARG).startswith(b"invalid")
+    with pytest.raises(C.MoEError):
+        C.check(C.MOE_ERR_ARG, "x")
+
+
+def test_package_has_no_cpu_fallback():
+    # the product path never imports the oracle
+    pkg = os.path.join(ROOT, "mixture_experts_routing_fp32_b200")
+    for name in os.listdir(pkg):
+        if name.endswith(".py"):
+            src = open(os.path.join(pkg, name)).read()
+            assert "oracle" not in src.replace("never imports the oracle", ""), name

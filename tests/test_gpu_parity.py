@@ -1,0 +1,202 @@
+"""GPU path vs the CPU oracle, element by element, on the reduced configs.
+
+Every config keeps its full-size options (variants, sentinels, capacity,
+groups, sigmoid + bias, shared expert) at sizes the oracle finishes in
+seconds while spanning several 128-row tiles with ragged tails.
+
+Bar (the layer's stated tolerances): routing indices, counts, kept,
+drops, sentinels and the permutation bit-exact except top-k near-ties
+(fp32 margin < 1e-5, counted); every float output and gradient within
+relative L2 2e-2 for bf16 compute and 1e-4 for the fp32 config.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import moe_oracle as O
+from tests.helpers import oracle_layer, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def tol(cfg):
+    return 1e-4 if cfg.dtype == "fp32" else 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from mixture_experts_routing_fp32_b200.build import build
+    build()
+
+
+def gpu_inputs(cfg, dev="cuda"):
+    d = {n: W.make_input(cfg, n, dev) for n in ("x", "w_r", "w13", "w_down", "dy")}
+    d["w13_s"] = W.make_input(cfg, "w13_s", dev) if cfg.n_shared else None
+    d["w_down_s"] = W.make_input(cfg, "w_down_s", dev) if cfg.n_shared else None
+    d["logit_offset"] = W.make_input(cfg, "logit_offset", dev) if cfg.hot_expert_offset else None
+    d["sel_bias"] = W.make_input(cfg, "sel_bias", dev) if cfg.sel_bias_range else None
+    d["sentinel_mask"] = W.make_input(cfg, "sentinel_mask", dev) if cfg.sentinel_frac else None
+    return d
+
+
+def run_gpu(cfg, gemm_impl=0, inp=None):
+    from mixture_experts_routing_fp32_b200 import MoELayer, config_from, moe_check_status
+    layer = MoELayer(config_from(cfg, gemm_impl=gemm_impl))
+    inp = inp or gpu_inputs(cfg)
+    layer.forward(inp["x"], inp["w_r"], inp["w13"], inp["w_down"], inp["w13_s"],
+                  inp["w_down_s"], inp["logit_offset"], inp["sel_bias"],
+                  inp["sentinel_mask"])
+    layer.backward(inp["dy"])
+    assert moe_check_status() == 0
+    return layer, inp
+
+
+def host(t):
+    return t.detach().float().cpu().numpy() if t.dtype != torch.int32 else t.cpu().numpy()
+
+
+def check_dispatch(cfg, layer, R, Dp):
+    """Bit-exact routing / permutation (or validity when a near-tie flipped)."""
+    idx = layer.topk_idx.cpu().numpy()
+    diff = np.nonzero((idx != R.idx).any(axis=1))[0]
+    assert np.all(R.margin[diff] < O.NEAR_TIE), ("non-near-tie routing mismatch", diff[:10])
+    E, K, T = cfg.E, cfg.K, cfg.T
+    counts, kept = host(layer.counts), host(layer.kept)
+    offsets, stats = host(layer.offsets), host(layer.stats)
+    slot_row, row_slot = host(layer.slot_row), host(layer.row_slot)
+    tile_e = host(layer.tile_expert)
+    n_rows = int(stats[2])
+    assert n_rows % 128 == 0 and stats[3] * 128 == n_rows
+    # permutation in the GPU's padded row space -> (expert, rank) per slot
+    ex = np.full(T * K, -1)
+    rk = np.full(T * K, -1)
+    kept_slots = np.nonzero(slot_row >= 0)[0]
+    rows = slot_row[kept_slots]
+    assert np.all(rows < n_rows)
+    ex[kept_slots] = tile_e[rows // 128]
+    rk[kept_slots] = rows - offsets[ex[kept_slots]]
+    assert np.all(row_slot[rows] == kept_slots)                    # inverse map
+    assert np.all(ex[kept_slots] < E)
+    for e in range(E):                                             # padded layout
+        assert offsets[e] % 128 == 0
+        assert offsets[e + 1] - offsets[e] == -(-kept[e] // 128) * 128
+    pad_rows = np.ones(n_rows, dtype=bool)
+    pad_rows[rows] = False
+    if cfg.n_shared:
+        pad_rows[offsets[E]:offsets[E] + T] = False
+    assert np.all(row_slot[:n_rows][pad_rows] == -1)
+    assert np.all(host(layer.x_perm)[:n_rows][pad_rows] == 0)
+    if diff.size == 0:
+        assert np.array_equal(counts, Dp.counts)
+        assert np.array_equal(kept, Dp.kept)
+        assert int(stats[0]) == Dp.n_drop
+        assert int(stats[1]) == Dp.n_sentinel
+        assert np.array_equal(ex, np.where(Dp.rank >= 0, Dp.expert, -1))
+        assert np.array_equal(rk, Dp.rank)
+    else:   # a near-tie flipped: the permutation must still be the stable sort of GPU idx
+        e_slot = idx.reshape(-1).copy()
+        if cfg.sentinel_frac:
+            e_slot[W.make_input(cfg, "sentinel_mask").numpy().astype(bool)] = -1
+        Dg = O.dispatch(e_slot.reshape(T, K), E, cfg.capacity_factor, cfg.min_capacity)
+        assert np.array_equal(counts, Dg.counts)
+        assert np.array_equal(rk, Dg.rank)
+    return diff.size
+
+
+@pytest.mark.parametrize("name", list(W.REDUCED))
+def test_parity_reduced(name):
+    cfg = W.REDUCED[name]
+    layer, inp = run_gpu(cfg)
+    L = oracle_layer(cfg)
+    o = O.opts_of(cfg)
+    fw = O.forward(L, o)
+    dy = W.make_input(cfg, "dy").double().numpy()
+    bw = O.backward(L, o, fw, dy)
+    R, Dp = fw["R"], fw["Dp"]
+    tl = tol(cfg)
+    # router (fp32 on both sides)
+    assert rel_l2(host(layer.logits), R.logits) < 1e-5
+    assert rel_l2(host(layer.probs), R.p) < 1e-5
+    assert rel_l2(host(layer.lse), R.lse) < 1e-5
+    flips = check_dispatch(cfg, layer, R, Dp)
+    same = (layer.topk_idx.cpu().numpy() == R.idx).all(axis=1)
+    assert rel_l2(host(layer.topk_w)[same], R.g[same]) < 1e-5
+    # forward output and losses
+    assert rel_l2(host(layer.y), fw["y"]) < tl
+    if cfg.aux_alpha:
+        assert abs(float(layer.losses[0]) - fw["aux"]) <= 1e-5 * abs(fw["aux"])
+    if cfg.z_lambda:
+        assert abs(float(layer.losses[1]) - fw["z"]) <= 1e-5 * abs(fw["z"])
+    # gradients
+    assert rel_l2(host(layer.dg), bw["dg"]) < tl
+    assert rel_l2(host(layer.dlogits), bw["ds"]) < tl
+    assert rel_l2(host(layer.dw_r), bw["dw_r"]) < tl
+    assert rel_l2(host(layer.dx), bw["dx"]) < tl
+    dw13 = np.stack([bw["dw13"][e] for e in range(cfg.E)])
+    dwd = np.stack([bw["dwd"][e] for e in range(cfg.E)])
+    assert rel_l2(host(layer.dw13), dw13) < tl
+    assert rel_l2(host(layer.dw_down), dwd) < tl
+    if cfg.n_shared:
+        assert rel_l2(host(layer.dw13_s), bw["dw13_s"]) < tl
+        assert rel_l2(host(layer.dw_down_s), bw["dwd_s"]) < tl
+    # sentinel and dropped slots: zero gate gradient, exactly
+    masked = (host(layer.slot_row) < 0).reshape(cfg.T, cfg.K)
+    assert np.all(host(layer.dg)[masked] == 0.0)
+    print("%s: near-tie flips %d, GPU near-tie count %d, drops %d, sentinels %d" % (
+        name, flips, int(layer.near_ties[0]), int(layer.stats[0]), int(layer.stats[1])))
+
+
+@pytest.mark.parametrize("name", ["mm_a", "olmoe", "mix", "ds3"])
+def test_tensor_core_path_matches_simt_path(name):
+    """The tcgen05 GEMMs against the CUDA-core GEMMs on the same inputs."""
+    cfg = W.REDUCED[name]
+    tc, inp = run_gpu(cfg, gemm_impl=0)
+    simt, _ = run_gpu(cfg, gemm_impl=1, inp=inp)
+    for attr in ("y", "dx", "dw13", "dw_down", "dw_r", "dg"):
+        a, b = getattr(tc, attr).float(), getattr(simt, attr).float()
+        assert (a - b).norm() / b.norm() < 1e-2, attr
+    assert torch.equal(tc.topk_idx, simt.topk_idx)
+    assert torch.equal(tc.slot_row, simt.slot_row)
+
+
+def test_k1_variant_b_router_grad_is_exactly_aux_only():
+    """MiniMind-shaped K=1: variant B's router gradient does not depend on
+    the upstream gradient at all (only the aux loss reaches the router);
+    variant A's does (STA324 §8.3; MiniMind issue §2)."""
+    for name, zero in (("mm_b", True), ("mm_a", False)):
+        cfg = W.REDUCED[name]
+        layer, inp = run_gpu(cfg)
+        d1, w1 = layer.dlogits.clone(), layer.dw_r.clone()
+        layer.backward(inp["dy"] * -3.0)
+        torch.cuda.synchronize()
+        same = torch.equal(d1, layer.dlogits) and torch.equal(w1, layer.dw_r)
+        assert same == zero, name
+        if zero:
+            assert float(layer.dw_r.abs().sum()) > 0     # the aux gradient is there
+
+
+def test_generator_identical_on_gpu_and_cpu():
+    cfg = W.REDUCED["ds3"]
+    for n in ("x", "w13", "w_r", "sel_bias"):
+        assert torch.equal(W.make_input(cfg, n, "cuda").cpu(), W.make_input(cfg, n))
+
+
+def test_device_error_word_on_bad_expert_id():
+    """An expert id outside [-1, E) is reported through the error word and
+    the slot is treated as a sentinel (host-planted; no GPU fault)."""
+    from mixture_experts_routing_fp32_b200 import MoELayer, config_from, api, MoEError
+    cfg = W.REDUCED["mm_a"]
+    layer = MoELayer(config_from(cfg))
+    x = W.make_input(cfg, "x", "cuda")
+    idx = torch.zeros(cfg.T, cfg.K, dtype=torch.int32, device="cuda")
+    idx[5, 0] = cfg.E + 3
+    api.moe_dispatch(layer.cfg, idx, None, x, layer.counts, layer.kept, layer.offsets,
+                     layer.slot_row, layer.row_slot, layer.tile_expert, layer.stats,
+                     layer.x_perm, layer.ws)
+    with pytest.raises(MoEError):
+        api.moe_check_status()
+    assert int(layer.stats[1]) == 1 and int(layer.slot_row[5 * cfg.K]) == -1
+    assert api.moe_check_status() == 0          # the word was cleared
