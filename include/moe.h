@@ -126,8 +126,10 @@ int moe_get_sizes(const moe_config_t* cfg, moe_sizes_t* out);
  *   topk_idx     [T,K] i32 out: selected experts, best first; equal
  *                selection scores go to the lower expert index
  *   topk_w       [T,K] f32 out: gate weights g
- *   near_ties    [1] i32 out: tokens whose K-th/(K+1)-th selection margin
- *                (or group-boundary margin) is below 1e-5
+ *   near_ties    [1] i32 out: tokens where two consecutive selection scores
+ *                among the top K+1 (or the kept/next group scores) are
+ *                closer than 1e-5: the choice or the slot order of such a
+ *                token may differ from an exact computation
  *   ws           workspace (moe_get_sizes)
  */
 int moe_router(const moe_config_t* cfg, const void* x, const float* w_r,

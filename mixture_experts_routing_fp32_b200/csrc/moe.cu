@@ -33,12 +33,23 @@ struct Prof {
 };
 thread_local Prof g_prof;
 
+// Under stream capture the records must be real event-record nodes
+// (cudaEventRecordExternal; re-recorded on every replay), not the
+// capture-internal dependency markers a plain record becomes; outside
+// capture that flag is invalid, so a plain record is used.
+inline void prof_record(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &st) == cudaSuccess && st == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, s);
+}
 inline void prof_begin(cudaStream_t s) {
-  if (g_prof.n < g_prof.cap) cudaEventRecord(g_prof.ev[2 * g_prof.n], s);
+  if (g_prof.n < g_prof.cap) prof_record(g_prof.ev[2 * g_prof.n], s);
 }
 inline void prof_end(cudaStream_t s, const char* name) {
   if (g_prof.n < g_prof.cap) {
-    cudaEventRecord(g_prof.ev[2 * g_prof.n + 1], s);
+    prof_record(g_prof.ev[2 * g_prof.n + 1], s);
     g_prof.name[g_prof.n++] = name;
   }
 }
@@ -115,12 +126,20 @@ bool use_tc(const moe_config_t* c) {
 
 struct Layout {
   int64_t rows_max, tiles_max, C, n_slots;
-  int n_disp_blocks, n_aux_chunks, n_dwr_chunks;
+  int n_disp_blocks, n_aux_chunks, n_dwr_chunks, dwr_chunk;
   size_t off_bhist, off_bsent, off_aux, off_dg, off_ds, off_dwr, off_dO, off_dA13, off_dX,
       off_dH, total;
 };
-constexpr int kAuxChunk = 512;
-constexpr int kDwrChunk = 1024;
+constexpr int kAuxChunk = 128;
+
+// Tokens per dW_r partial: enough chunks that the (E x D) tiles of all
+// chunks fill about two waves of 148 SMs; one chunk when the tiles alone do.
+int64_t dwr_chunk_tokens(const moe_config_t* c) {
+  const int64_t tiles = (c->E <= 8) ? ceil_div(c->D, 256)
+                                    : ceil_div(c->D, 64) * ceil_div(c->E, 64);
+  const int64_t want = std::max<int64_t>(1, ceil_div(2 * 148, tiles));
+  return std::max<int64_t>(32, round_up(ceil_div(c->T, want), 32));
+}
 
 Layout layout_of(const moe_config_t* c) {
   Layout L{};
@@ -134,7 +153,8 @@ Layout layout_of(const moe_config_t* c) {
   L.tiles_max = L.rows_max / kRowTile;
   L.n_disp_blocks = (int)ceil_div(L.n_slots, kDispChunk);
   L.n_aux_chunks = (int)ceil_div(c->T, kAuxChunk);
-  L.n_dwr_chunks = (int)ceil_div(c->T, kDwrChunk);
+  L.dwr_chunk = (int)dwr_chunk_tokens(c);
+  L.n_dwr_chunks = (int)ceil_div(c->T, L.dwr_chunk);
   const size_t a = act_bytes(c);
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += round_up((int64_t)bytes, 256); return o; };
@@ -262,14 +282,37 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
 __global__ void __launch_bounds__(256)
 aux_partial_kernel(const float* __restrict__ probs, const float* __restrict__ lse, int T, int E,
                    float* __restrict__ part) {
-  const int c = blockIdx.x;
+  // chunk c of kAuxChunk tokens: column sums of probs and the sum of lse^2,
+  // each reduced in a fixed order (deterministic)
+  __shared__ float red[256];
+  const int c = blockIdx.x, tid = threadIdx.x;
   const int t0 = c * kAuxChunk, t1 = min(T, t0 + kAuxChunk);
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+  for (int e0 = 0; e0 < E; e0 += 256) {
+    const int EB = min(256, E - e0);
+    const int S = 256 / EB;             // token sub-streams per expert
     float s = 0.f;
-    if (e < E) for (int t = t0; t < t1; ++t) s += probs[(size_t)t * E + e];
-    else for (int t = t0; t < t1; ++t) s += lse[t] * lse[t];
-    part[(size_t)c * (E + 1) + e] = s;
+    if (tid < S * EB) {
+      const int e = e0 + tid % EB, sub = tid / EB;
+      for (int t = t0 + sub; t < t1; t += S) s += probs[(size_t)t * E + e];
+    }
+    red[tid] = s;
+    __syncthreads();
+    if (tid < EB) {
+      float acc = 0.f;
+      for (int k = 0; k < S; ++k) acc += red[k * EB + tid];
+      part[(size_t)c * (E + 1) + e0 + tid] = acc;
+    }
+    __syncthreads();
   }
+  float z = 0.f;
+  for (int t = t0 + tid; t < t1; t += 256) z += lse[t] * lse[t];
+  red[tid] = z;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (tid < o) red[tid] += red[tid + o];
+    __syncthreads();
+  }
+  if (tid == 0) part[(size_t)c * (E + 1) + E] = red[0];
 }
 
 __global__ void __launch_bounds__(512)
@@ -667,15 +710,15 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     if (E <= 8) {
       dim3 g((unsigned)ceil_div(D, 256), 1, (unsigned)nc);
       if (bf) dwr_partial_kernel<__nv_bfloat16, 8, 256, 2, 4><<<g, 256, 0, s>>>(
-          ds, static_cast<const __nv_bfloat16*>(x), T, E, D, kDwrChunk, dwr_part);
+          ds, static_cast<const __nv_bfloat16*>(x), T, E, D, L.dwr_chunk, dwr_part);
       else dwr_partial_kernel<float, 8, 256, 2, 4><<<g, 256, 0, s>>>(
-          ds, static_cast<const float*>(x), T, E, D, kDwrChunk, dwr_part);
+          ds, static_cast<const float*>(x), T, E, D, L.dwr_chunk, dwr_part);
     } else {
       dim3 g((unsigned)ceil_div(D, 64), (unsigned)ceil_div(E, 64), (unsigned)nc);
       if (bf) dwr_partial_kernel<__nv_bfloat16, 64, 64, 4, 4><<<g, 256, 0, s>>>(
-          ds, static_cast<const __nv_bfloat16*>(x), T, E, D, kDwrChunk, dwr_part);
+          ds, static_cast<const __nv_bfloat16*>(x), T, E, D, L.dwr_chunk, dwr_part);
       else dwr_partial_kernel<float, 64, 64, 4, 4><<<g, 256, 0, s>>>(
-          ds, static_cast<const float*>(x), T, E, D, kDwrChunk, dwr_part);
+          ds, static_cast<const float*>(x), T, E, D, L.dwr_chunk, dwr_part);
     }
     MOE_LAUNCHED(s, "router_dw_partial");
     const int64_t n = (int64_t)E * D;

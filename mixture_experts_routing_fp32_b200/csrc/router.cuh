@@ -126,7 +126,8 @@ __device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
     }
   }
 
-  // top-K (+1 round for the boundary margin)
+  // top-K (+1 round): the near-tie margin is the smallest gap between
+  // consecutive selection scores among the top K+1
   int sel_e[kMaxK];
   float sel_s[kMaxK], sel_p[kMaxK];
   unsigned taken = 0u;
@@ -143,6 +144,7 @@ __device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
       if (ok && (u[i] > v || (u[i] == v && ei < e))) { v = u[i]; e = ei; }
     }
     warp_argmax(v, e);
+    if (k > 0 && v != NEG) margin = fminf(margin, uk - v);
     if (k < a.K) {
       const int owner = e & 31, slot = e >> 5;
       const float sv = __shfl_sync(0xffffffffu, pick<NV>(s, slot), owner);
@@ -150,8 +152,6 @@ __device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
       if (lane == owner) taken |= 1u << slot;
       if (k < kMaxK) { sel_e[k] = e; sel_s[k] = sv; sel_p[k] = pv; }
       uk = v;
-    } else if (v != NEG) {
-      margin = uk - v;
     }
   }
   if (lane == 0 && (margin < kNearTie || gmargin < kNearTie))
@@ -226,7 +226,7 @@ router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
 #pragma unroll
     for (int e = 0; e < EB; ++e) {
       const float v = warp_sum(acc[e]);
-      if (lane == e) s[0] = v;
+      if (lane == e && e < E) s[0] = v;
     }
     if (lane < E) {
       if (offset != nullptr) s[0] += offset[lane];

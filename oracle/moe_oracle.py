@@ -86,7 +86,7 @@ class Routing:
     lse: np.ndarray         # [T]   logsumexp of the logits (z-loss)
     idx: np.ndarray         # [T,K] int, selected experts, best first
     g: np.ndarray           # [T,K] gate weights (after route_scale)
-    margin: np.ndarray      # [T]   min(top-k boundary margin, group boundary margin)
+    margin: np.ndarray      # [T]   min gap among the top K+1 scores and at the group boundary
 
 
 def route(logits, K, *, score_fn=SOFTMAX, renorm=1, n_groups=1,
@@ -147,11 +147,13 @@ def route(logits, K, *, score_fn=SOFTMAX, renorm=1, n_groups=1,
     order = np.argsort(-u, axis=1, kind="stable")
     idx = order[:, :K].copy()
     usorted = np.take_along_axis(u, order, axis=1)
-    if K < E:
-        nxt = usorted[:, K]
-        mk = usorted[:, K - 1] - nxt
-        mk = np.where(np.isfinite(nxt), mk, np.inf)
-        margin = np.minimum(margin, mk)
+    # smallest gap between consecutive selection scores among the top K+1:
+    # both which experts are chosen and their slot order hang on these
+    top = usorted[:, :min(K + 1, E)]
+    if top.shape[1] > 1:
+        gaps = top[:, :-1] - top[:, 1:]
+        gaps = np.where(np.isfinite(top[:, 1:]), gaps, np.inf)
+        margin = np.minimum(margin, gaps.min(axis=1))
 
     if score_fn == SOFTMAX:
         if renorm:

@@ -96,13 +96,26 @@ def check_dispatch(cfg, layer, R, Dp):
         assert int(stats[1]) == Dp.n_sentinel
         assert np.array_equal(ex, np.where(Dp.rank >= 0, Dp.expert, -1))
         assert np.array_equal(rk, Dp.rank)
-    else:   # a near-tie flipped: the permutation must still be the stable sort of GPU idx
-        e_slot = idx.reshape(-1).copy()
+    else:
+        # A near-tie flipped a choice or a slot order, so the permutation is
+        # checked for validity against the GPU's own indices: each expert's
+        # kept slots are its first min(n_e, C) valid slots in flat-slot
+        # order, ranked 0, 1, ... (the definition of the stable counting
+        # sort with capacity), and everything else is dropped or sentinel.
+        e_slot = idx.reshape(-1).astype(np.int64)
         if cfg.sentinel_frac:
-            e_slot[W.make_input(cfg, "sentinel_mask").numpy().astype(bool)] = -1
-        Dg = O.dispatch(e_slot.reshape(T, K), E, cfg.capacity_factor, cfg.min_capacity)
-        assert np.array_equal(counts, Dg.counts)
-        assert np.array_equal(rk, Dg.rank)
+            e_slot = np.where(W.make_input(cfg, "sentinel_mask").numpy().astype(bool), -1, e_slot)
+        C = None if cfg.capacity_factor <= 0 else max(
+            int(np.ceil(cfg.capacity_factor * T * K / E)), cfg.min_capacity)
+        for e in range(E):
+            js = np.nonzero(e_slot == e)[0]                # increasing flat order
+            assert counts[e] == js.size
+            keep = js if C is None else js[:C]
+            assert kept[e] == keep.size
+            assert np.array_equal(rk[keep], np.arange(keep.size))
+            assert np.all(ex[keep] == e)
+            assert np.all(rk[js[keep.size:]] == -1)
+        assert np.all(rk[e_slot < 0] == -1)
     return diff.size
 
 

@@ -120,3 +120,29 @@ def test_sentinel_zero_gate_grad_and_negative_control():
     # the expert weights' grads do not depend on the router-side leak
     for e in range(cfg.E):
         np.testing.assert_array_equal(bw_bug["dw13"][e], bw["dw13"][e])
+
+
+@pytest.mark.parametrize("name", ["olmoe", "mix", "ds3"])
+def test_sampled_helpers_match_full_oracle(name):
+    """The per-token and per-column pieces used for full-size checks give the
+    same values as the finite-difference-pinned full forward/backward."""
+    from tests.helpers import LazyLayer
+    cfg = W.REDUCED[name].replace(T=160, D=64, F=48)
+    L = oracle_layer(cfg)
+    o = O.opts_of(cfg)
+    dy = W.make_input(cfg, "dy").double().numpy()
+    fw = O.forward(L, o)
+    bw = O.backward(L, o, fw, dy)
+    R, Dp = fw["R"], fw["Dp"]
+    for t in (0, 7, cfg.T - 1):
+        r = O.token_forward_backward(L, o, R, Dp, t, dy[t])
+        np.testing.assert_allclose(r["y"], fw["y"][t], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(r["dg"], bw["dg"][t], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(r["ds"], bw["ds"][t], rtol=1e-9, atol=1e-13)
+        np.testing.assert_allclose(r["dx"], bw["dx"][t], rtol=1e-9, atol=1e-12)
+    LL = LazyLayer(cfg, L.x)              # row/column slices regenerated on demand
+    for e, j in ((0, 3), (cfg.E - 1, cfg.F - 1)):
+        a, b, c = O.expert_column_grads(LL, o, R, Dp, e, j, lambda rows: dy[rows])
+        np.testing.assert_allclose(a, bw["dw13"][e][j], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(b, bw["dw13"][e][cfg.F + j], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(c, bw["dwd"][e][:, j], rtol=1e-9, atol=1e-12)
