@@ -164,6 +164,36 @@ int moe_dispatch(const moe_config_t* cfg, const int32_t* topk_idx,
                  int32_t* stats, void* x_perm, void* ws, cudaStream_t stream);
 
 /*
+ * moe_dispatch_static — moe_dispatch without a workspace (allocates nothing).
+ * The pages have no counterpart: this entry point serves callers that are
+ * given only their input and output buffers and cannot allocate device
+ * memory, such as a plugin or custom-op host with no workspace hook that
+ * forbids cudaMalloc inside the op, or a serving runtime whose device memory
+ * plan is fixed in advance.  Arguments, outputs and results are those of
+ * moe_dispatch, minus `ws`.
+ *   - Scratch (per-block expert histograms and sentinel counts) lives in a
+ *     file-scope device array of MOE_STATIC_SCRATCH_BYTES that every GPU
+ *     loading the library holds until the process exits.  It needs
+ *     (ceil(T*K / 4096) * (E + 1)) * 4 bytes; larger problems are rejected
+ *     with MOE_ERR_ARG before anything is launched (1 MiB covers, e.g.,
+ *     T*K up to about 4.1 M slots at E = 256).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture on that device.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (every call rewrites what it reads, nothing must start at zero).
+ *     Calls that overlap on the GPU — on different streams, or from
+ *     different threads, at the same time — race on it: serialise them.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define MOE_STATIC_SCRATCH_BYTES (1u << 20)
+int moe_dispatch_static(const moe_config_t* cfg, const int32_t* topk_idx,
+                        const uint8_t* sentinel_mask, const void* x,
+                        int32_t* counts, int32_t* kept, int32_t* offsets,
+                        int32_t* slot_row, int32_t* row_slot, int32_t* tile_expert,
+                        int32_t* stats, void* x_perm, cudaStream_t stream);
+
+/*
  * moe_aux_loss — losses[0] = alpha*E*sum_e f_e P_e with f_e = counts_e /
  * sum(counts), P_e = mean_t probs[t,e]; losses[1] = lambda*mean_t lse_t^2.
  * [STA324 §8.5, §8.6], [TRAIN], [8MOE] ST-MoE.  losses: [2] f32 out.

@@ -70,6 +70,18 @@ def moe_dispatch(cfg, topk_idx, sentinel_mask, x, counts, kept, offsets,
           "moe_dispatch")
 
 
+def moe_dispatch_static(cfg, topk_idx, sentinel_mask, x, counts, kept, offsets,
+                        slot_row, row_slot, tile_expert, stats, x_perm, stream=None):
+    """moe_dispatch without a workspace, for callers that cannot allocate
+    device memory (see include/moe.h): scratch is the library's static
+    device array, so overlapping calls race."""
+    check(lib().moe_dispatch_static(ctypes.byref(cfg), _p(topk_idx), _p(sentinel_mask),
+                                    _p(x), _p(counts), _p(kept), _p(offsets),
+                                    _p(slot_row), _p(row_slot), _p(tile_expert),
+                                    _p(stats), _p(x_perm), _s(stream)),
+          "moe_dispatch_static")
+
+
 def moe_aux_loss(cfg, probs, lse, counts, losses, ws, stream=None):
     check(lib().moe_aux_loss(ctypes.byref(cfg), _p(probs), _p(lse), _p(counts),
                              _p(losses), _p(ws), _s(stream)), "moe_aux_loss")
@@ -139,6 +151,7 @@ class LaunchProfile:
 
 
 __all__ = ["LaunchProfile", "MoEError", "MoeConfig", "MoeSizes", "make_config", "config_from",
-           "moe_get_sizes", "moe_router", "moe_dispatch", "moe_aux_loss",
+           "moe_get_sizes", "moe_router", "moe_dispatch", "moe_dispatch_static",
+           "moe_aux_loss",
            "moe_expert_ffn", "moe_combine", "moe_backward", "moe_check_status",
            "moe_launch_count"]

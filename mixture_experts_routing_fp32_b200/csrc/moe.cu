@@ -466,6 +466,93 @@ int moe_dispatch(const moe_config_t* c, const int32_t* topk_idx, const uint8_t* 
   return MOE_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free dispatch.
+//
+// Some callers are handed only their input and output buffers and may not
+// allocate device memory themselves: a plugin or custom-op host that offers
+// no workspace hook and forbids cudaMalloc inside the op, or a serving
+// runtime whose device memory plan is fixed before the first request.  They
+// cannot provide the workspace moe_dispatch takes, so this variant keeps its
+// only scratch (per-block expert histograms and sentinel counts) in the
+// file-scope device array below.  Every GPU that loads the library holds the
+// array until the process exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) int32_t moe_static_scratch[MOE_STATIC_SCRATCH_BYTES / sizeof(int32_t)];
+
+namespace {
+constexpr int kMaxStaticDevices = 64;
+std::mutex g_static_mu;
+int32_t* g_static_scratch_ptr[kMaxStaticDevices] = {};
+
+// Device address of the array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+int static_scratch_ptr(int32_t** out) {
+  int dev = 0;
+  MOE_CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxStaticDevices) return MOE_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    MOE_CK(cudaGetSymbolAddress(&p, moe_static_scratch));
+    g_static_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_static_scratch_ptr[dev];
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int moe_dispatch_static(const moe_config_t* c, const int32_t* topk_idx,
+                        const uint8_t* sentinel_mask, const void* x, int32_t* counts,
+                        int32_t* kept, int32_t* offsets, int32_t* slot_row, int32_t* row_slot,
+                        int32_t* tile_expert, int32_t* stats, void* x_perm, cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!topk_idx || !x || !counts || !kept || !offsets || !slot_row || !row_slot ||
+      !tile_expert || !stats || !x_perm)
+    return MOE_ERR_ARG;
+  const Layout L = layout_of(c);
+  // scratch: n_blocks x E histogram entries + n_blocks sentinel counts.  Both
+  // are written in full by the histogram kernel before anything reads them,
+  // so nothing has to start at zero.
+  const size_t need = ((size_t)L.n_disp_blocks * c->E + (size_t)L.n_disp_blocks) * sizeof(int32_t);
+  if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_ARG;
+  int32_t* base = nullptr;
+  MOE_TRY(static_scratch_ptr(&base));
+  int32_t* bhist = base;
+  int32_t* bsent = base + (size_t)L.n_disp_blocks * c->E;
+  prof_begin(s);
+  disp_hist_kernel<<<L.n_disp_blocks, 256, c->E * 4, s>>>(topk_idx, sentinel_mask, L.n_slots,
+                                                          c->E, bhist, bsent);
+  MOE_LAUNCHED(s, "dispatch_hist");
+  prof_begin(s);
+  disp_scan_kernel<<<1, 1024, c->E * 8, s>>>(bhist, bsent, L.n_disp_blocks, c->E, c->T,
+                                             c->n_shared, L.C, L.rows_max, counts, kept,
+                                             offsets, tile_expert, stats);
+  MOE_LAUNCHED(s, "dispatch_scan");
+  prof_begin(s);
+  disp_rank_kernel<<<L.n_disp_blocks, 256, kDispWarps * c->E * 4, s>>>(
+      topk_idx, sentinel_mask, L.n_slots, c->E, L.C, L.rows_max, bhist, offsets, slot_row,
+      row_slot);
+  MOE_LAUNCHED(s, "dispatch_rank");
+  const int grid = grid_for(L.rows_max);
+  prof_begin(s);
+  if (c->dtype == MOE_BF16)
+    disp_gather_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), c->D, c->K, c->E, c->T, offsets, kept, tile_expert,
+        stats, row_slot, static_cast<__nv_bfloat16*>(x_perm));
+  else
+    disp_gather_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), c->D, c->K,
+                                                    c->E, c->T, offsets, kept, tile_expert,
+                                                    stats, row_slot, static_cast<float*>(x_perm));
+  MOE_LAUNCHED(s, "dispatch_gather");
+  return MOE_OK;
+}
+
 int moe_aux_loss(const moe_config_t* c, const float* probs, const float* lse,
                  const int32_t* counts, float* losses, void* ws, cudaStream_t s) {
   MOE_TRY(validate(c));
