@@ -12,9 +12,10 @@
 //     experts without rows cost nothing;
 //   * warp 0: TMA producer (128B-swizzled boxes into a STAGES-deep ring);
 //     warp 1: one thread issues tcgen05.mma (M=128, N=BN, K=16) into a
-//     double-buffered fp32 accumulator in tensor memory; warps 2-5: epilogue
-//     (tcgen05.ld, fused SwiGLU / SwiGLU-backward, bf16 stores), overlapped
-//     with the next tile's main loop;
+//     double-buffered fp32 accumulator in tensor memory; warps 2-9: epilogue
+//     (two warps per tensor-memory lane quarter; tcgen05.ld, fused SwiGLU /
+//     SwiGLU-backward, bf16 stores), overlapped with the next tile's main
+//     loop;
 //   * ROWS mode: C[r, n] = sum_k A[r, k] B_e[n, k] (forward, data gradients);
 //     WGRAD mode: C_g[m, n] = sum_{r in rows(g)} A[r, m] B[r, n] (weight
 //     gradients; the reduction runs over the group's own rows and the zero
@@ -31,7 +32,8 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                    // one 128-byte swizzle row of bf16
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                  // two per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
 enum { MODE_ROWS = 0, MODE_WGRAD = 1 };
@@ -148,9 +150,9 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 // 32 TMEM lanes x 32 consecutive fp32 columns: thread i of the warp gets lane
-// (base lane + i), columns [col, col+32).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
+// (base lane + i), columns [col, col+32).  tmem_wait() must follow before
+// the registers are read.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -162,9 +164,28 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
         "=r"(r[31])
       : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void u2f32(const uint32_t (&r)[32], float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// Epilogue math on bf16-rounded outputs: the hardware approximate divide
+// (__fdividef) and exponential (__expf) instead of IEEE division, which
+// would compile to a branchy subroutine.
+__device__ __forceinline__ float fast_sigmoid(float a) {
+  return __fdividef(1.0f, 1.0f + __expf(-a));
+}
+__device__ __forceinline__ void bf16x8_to_f(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 v = __bfloat1622float2(h[i]);
+    f[2 * i] = v.x;
+    f[2 * i + 1] = v.y;
+  }
 }
 
 // 32 floats -> 32 bf16 at p (64 bytes, 16-byte aligned).
@@ -240,12 +261,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * S::kStage + S::kBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr uint32_t kCols = 2 * BN;
+  // tensor memory: two BN-column fp32 accumulators; tcgen05.alloc takes a
+  // power of two between 32 and 512 columns
+  constexpr uint32_t kCols = (2 * BN <= 128) ? 128u : (2 * BN <= 256) ? 256u : 512u;
+  static_assert(2 * BN <= 512 && (kCols & (kCols - 1)) == 0, "tensor-memory columns");
 
   if (threadIdx.x == 0) {
     abort_flag_s = 0;
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(accf_bar(b), 1); mbar_init(acce_bar(b), 4); }
+    for (int b = 0; b < 2; ++b) { mbar_init(accf_bar(b), 1); mbar_init(acce_bar(b), kEpiWarps); }
     mbar_init(done_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -354,75 +378,99 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       mbar_wait(done_bar, 0, abort_flag);
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..9) ----------------
+    // Two warps per TMEM lane quarter q = warp % 4 (the lanes a warp may
+    // read); warp half hh takes the first or second half of the columns.
     const int q = warp & 3;
+    const int hh = (warp - 2) >> 2;
     const int rloc = q * 32 + lane;
+    constexpr int HC = BN / 2;           // columns per warp (plain epilogues)
+    constexpr int HJ = BN / 4;           // gate (= up) columns per warp (SwiGLU)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile d = decode<MODE, EPI, BN>(t, p);
       if (MODE == MODE_WGRAD && d.nk == 0) {
         __nv_bfloat16* og = d.e < p.E ? p.out + (int64_t)d.e * p.strideCE : p.out_shared;
-        __nv_bfloat16* dst = og + (int64_t)(d.m0 + rloc) * p.No + d.n0;
-        for (int c = 0; c < BN; c += 8) zero8(dst + c);
+        __nv_bfloat16* dst = og + (int64_t)(d.m0 + rloc) * p.No + d.n0 + hh * HC;
+        for (int c = 0; c < HC; c += 8) zero8(dst + c);
         continue;
+      }
+      const int64_t row = d.m0 + rloc;
+      // SwiGLU backward: this warp's a and b values are fetched before the
+      // accumulator wait so their latency overlaps the tile's main loop.
+      uint4 pa[EPI == EPI_SWIGLU_BWD ? HC / 8 : 1], pb[EPI == EPI_SWIGLU_BWD ? HC / 8 : 1];
+      if constexpr (EPI == EPI_SWIGLU_BWD) {
+        const __nv_bfloat16* a13 = p.aux + row * p.ld_aux + d.n0 + hh * HC;
+#pragma unroll
+        for (int i = 0; i < HC / 8; ++i) {
+          pa[i] = *reinterpret_cast<const uint4*>(a13 + 8 * i);
+          pb[i] = *reinterpret_cast<const uint4*>(a13 + p.F + 8 * i);
+        }
       }
       bool ok = (lane == 0) ? mbar_wait(accf_bar(acc), acc_phase, abort_flag) : true;
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * BN;
-      if (EPI == EPI_STORE) {
-        __nv_bfloat16* dst = p.out + (int64_t)(d.m0 + rloc) * p.ld_out + d.n0;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+      if constexpr (EPI == EPI_STORE || EPI == EPI_WGRAD) {
+        __nv_bfloat16* dst;
+        if (EPI == EPI_STORE) {
+          dst = p.out + row * p.ld_out + d.n0 + hh * HC;
+        } else {
+          __nv_bfloat16* og = d.e < p.E ? p.out + (int64_t)d.e * p.strideCE : p.out_shared;
+          dst = og + row * p.No + d.n0 + hh * HC;
+        }
+#pragma unroll
+        for (int c = 0; c < HC; c += 32) {
+          uint32_t r[32];
           float v[32];
-          tmem_ld32(tbase + c, v);
+          tmem_ld32(tbase + hh * HC + c, r);
+          tmem_wait();
+          u2f32(r, v);
           store32_bf16(dst + c, v);
         }
-      } else if (EPI == EPI_SWIGLU) {
-        const int64_t row = d.m0 + rloc;
-        __nv_bfloat16* a13 = p.out + row * p.ld_out;
-        __nv_bfloat16* hr = p.out2 + row * p.ld_out2;
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          float ga[32], ub[32];
-          tmem_ld32(tbase + c, ga);
-          tmem_ld32(tbase + BN / 2 + c, ub);
-          store32_bf16(a13 + d.n0 + c, ga);
-          store32_bf16(a13 + p.F + d.n0 + c, ub);
+      } else if constexpr (EPI == EPI_SWIGLU) {
+        __nv_bfloat16* a13 = p.out + row * p.ld_out + d.n0 + hh * HJ;
+        __nv_bfloat16* hr = p.out2 + row * p.ld_out2 + d.n0 + hh * HJ;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ga[i] = silu_f(ga[i]) * ub[i];
-          store32_bf16(hr + d.n0 + c, ga);
+        for (int c = 0; c < HJ; c += 32) {
+          uint32_t rg[32], ru[32];
+          float ga[32], ub[32];
+          tmem_ld32(tbase + hh * HJ + c, rg);
+          tmem_ld32(tbase + BN / 2 + hh * HJ + c, ru);
+          tmem_wait();
+          u2f32(rg, ga);
+          u2f32(ru, ub);
+          store32_bf16(a13 + c, ga);
+          store32_bf16(a13 + p.F + c, ub);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ga[i] = ga[i] * fast_sigmoid(ga[i]) * ub[i];
+          store32_bf16(hr + c, ga);
         }
-      } else if (EPI == EPI_SWIGLU_BWD) {
-        const int64_t row = d.m0 + rloc;
-        const __nv_bfloat16* a13 = p.aux + row * p.ld_aux;
-        __nv_bfloat16* da13 = p.out + row * p.ld_out;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+      } else {  // EPI_SWIGLU_BWD
+        __nv_bfloat16* da13 = p.out + row * p.ld_out + d.n0 + hh * HC;
+#pragma unroll
+        for (int c = 0; c < HC; c += 32) {
+          uint32_t r[32];
           float dh[32], av[32], bv[32];
-          tmem_ld32(tbase + c, dh);
-          load32_bf16(a13 + d.n0 + c, av);
-          load32_bf16(a13 + p.F + d.n0 + c, bv);
+          tmem_ld32(tbase + hh * HC + c, r);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            bf16x8_to_f(pa[c / 8 + i], av + 8 * i);
+            bf16x8_to_f(pb[c / 8 + i], bv + 8 * i);
+          }
+          tmem_wait();
+          u2f32(r, dh);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float s = sigmoid_f(av[i]);
-            const float da = dh[i] * bv[i] * s * (1.f + av[i] * (1.f - s));
-            bv[i] = dh[i] * av[i] * s;
+            const float sg = fast_sigmoid(av[i]);
+            const float da = dh[i] * bv[i] * sg * (1.f + av[i] * (1.f - sg));
+            bv[i] = dh[i] * av[i] * sg;
             av[i] = da;
           }
-          store32_bf16(da13 + d.n0 + c, av);
-          store32_bf16(da13 + p.F + d.n0 + c, bv);
-        }
-      } else {  // EPI_WGRAD
-        __nv_bfloat16* og = d.e < p.E ? p.out + (int64_t)d.e * p.strideCE : p.out_shared;
-        __nv_bfloat16* dst = og + (int64_t)(d.m0 + rloc) * p.No + d.n0;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          float v[32];
-          tmem_ld32(tbase + c, v);
-          store32_bf16(dst + c, v);
+          store32_bf16(da13 + c, av);
+          store32_bf16(da13 + p.F + c, bv);
         }
       }
       tc_fence_before();

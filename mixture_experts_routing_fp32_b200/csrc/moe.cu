@@ -231,6 +231,52 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
   return MOE_OK;
 }
 
+template <int MODE, bool AMN, bool BMN, int EPI>
+int run_tc(int bn, const char* name, const CUtensorMap& a, const CUtensorMap& b,
+           const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
+           cudaStream_t s) {
+  if (bn == 256)
+    return launch_tc<256, 4, MODE, AMN, BMN, EPI>(name, a, b, bs, p, total_max, total_hint, s);
+  if constexpr (EPI != tc::EPI_SWIGLU) {
+    if (bn == 192)
+      return launch_tc<192, 5, MODE, AMN, BMN, EPI>(name, a, b, bs, p, total_max, total_hint, s);
+  }
+  if (bn == 128)
+    return launch_tc<128, 6, MODE, AMN, BMN, EPI>(name, a, b, bs, p, total_max, total_hint, s);
+  return MOE_ERR_ARG;
+}
+
+// Expected 128-row tiles of the permuted rows (half a tile of padding per
+// expert on average), used only to choose tile widths.
+int64_t row_tiles_estimate(const moe_config_t* c, const Layout& L) {
+  const int64_t kept_total =
+      L.C < 0 ? L.n_slots : std::min<int64_t>(L.n_slots, (int64_t)c->E * L.C);
+  const int64_t rows = kept_total + 64 * std::min<int64_t>(c->E, kept_total);
+  return ceil_div(rows, kRowTile) + (c->n_shared ? ceil_div(c->T, kRowTile) : 0);
+}
+
+// Output tile width BN in {256, 192, 128} minimising waves x BN (the time of
+// the busiest SM); ties keep the wider tile.  SwiGLU tiles hold BN/2 gate
+// and BN/2 up columns of F.
+int pick_bn(int64_t N, int64_t mtiles, bool swiglu, int64_t F) {
+  const int64_t sms = num_sms();
+  int best = 0;
+  int64_t best_cost = INT64_MAX;
+  for (int bn : {256, 192, 128}) {
+    int64_t nt;
+    if (swiglu) {
+      if (bn == 192 || F % (bn / 2)) continue;
+      nt = F / (bn / 2);
+    } else {
+      if (N % bn) continue;
+      nt = N / bn;
+    }
+    const int64_t cost = ceil_div(mtiles * nt, sms) * bn;
+    if (cost < best_cost) { best_cost = cost; best = bn; }
+  }
+  return best;
+}
+
 int grid_for(int64_t items_per_8, int cap_mult = 8) {
   return (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(items_per_8, 8), (int64_t)num_sms() * cap_mult));
 }
@@ -583,32 +629,26 @@ int moe_expert_ffn(const moe_config_t* c, const void* x_perm, const int32_t* off
   const int D = c->D, F = c->F, E = c->E;
   if (use_tc(c)) {
     CUtensorMap mA, mB, mBs;
+    const int64_t mt = row_tiles_estimate(c, L);
     // gate/up + SwiGLU: A = x_perm [rows, D]; B = w13 [E, 2F, D] K-major
-    constexpr int BN1 = 256;
+    const int bn1 = pick_bn(2 * F, mt, true, F);
     MOE_TRY(make_map(&mA, x_perm, 1, L.rows_max, D, 128, false));
-    MOE_TRY(make_map(&mB, w13, E, 2 * F, D, BN1 / 2, true));
-    MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, BN1 / 2, true));
-    tc::Params p = rows_params(c, D, F / (BN1 / 2), tile_expert, stats);
+    MOE_TRY(make_map(&mB, w13, E, 2 * F, D, bn1 / 2, true));
+    MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, bn1 / 2, true));
+    tc::Params p = rows_params(c, D, F / (bn1 / 2), tile_expert, stats);
     p.out = static_cast<__nv_bfloat16*>(a13); p.ld_out = 2 * F;
     p.out2 = static_cast<__nv_bfloat16*>(h); p.ld_out2 = F;
-    MOE_TRY((launch_tc<BN1, 4, tc::MODE_ROWS, false, false, tc::EPI_SWIGLU>(
-        "tc_gate_up_swiglu", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU>(
+        bn1, "tc_gate_up_swiglu", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
     // down: A = h [rows, F]; B = w_down [E, D, F] K-major
+    const int bn2 = pick_bn(D, mt, false, F);
     MOE_TRY(make_map(&mA, h, 1, L.rows_max, F, 128, false));
-    if (D % 256 == 0) {
-      MOE_TRY(make_map(&mB, w_down, E, D, F, 256, true));
-      MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, 256, true));
-      tc::Params q = rows_params(c, F, D / 256, tile_expert, stats);
-      q.out = static_cast<__nv_bfloat16*>(o); q.ld_out = D;
-      return launch_tc<256, 4, tc::MODE_ROWS, false, false, tc::EPI_STORE>(
-          "tc_down", mA, mB, mBs, q, L.tiles_max * q.nN, 0, s);
-    }
-    MOE_TRY(make_map(&mB, w_down, E, D, F, 128, true));
-    MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, 128, true));
-    tc::Params q = rows_params(c, F, D / 128, tile_expert, stats);
+    MOE_TRY(make_map(&mB, w_down, E, D, F, bn2, true));
+    MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, bn2, true));
+    tc::Params q = rows_params(c, F, D / bn2, tile_expert, stats);
     q.out = static_cast<__nv_bfloat16*>(o); q.ld_out = D;
-    return launch_tc<128, 6, tc::MODE_ROWS, false, false, tc::EPI_STORE>(
-        "tc_down", mA, mB, mBs, q, L.tiles_max * q.nN, 0, s);
+    return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE>(
+        bn2, "tc_down", mA, mB, mBs, q, L.tiles_max * q.nN, 0, s);
   }
   auto go = [&](auto tag) -> int {
     using TE = decltype(tag);
@@ -701,72 +741,60 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   // 3-6. expert GEMMs
   if (use_tc(c)) {
     CUtensorMap mA, mB, mBs;
-    const int BNf = (F % 256 == 0) ? 256 : 128;
-    const int BNd = (D % 256 == 0) ? 256 : 128;
+    const int64_t mt = row_tiles_estimate(c, L);
+    const int groups = E + c->n_shared;
     // 3. dgrad down + SwiGLU backward: dA13 = swiglu'(dO . w_down[e])
+    const int bn3 = pick_bn(F, mt, false, F);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 128, false));
     MOE_TRY(make_map(&mB, w_down, E, D, F, 64, true));                 // dims {F, D, E}
     MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, 64, true));
     {
-      tc::Params p = rows_params(c, D, F / BNf, tile_expert, stats);
+      tc::Params p = rows_params(c, D, F / bn3, tile_expert, stats);
       p.out = static_cast<__nv_bfloat16*>(dA13); p.ld_out = 2 * F;
       p.aux = static_cast<const __nv_bfloat16*>(a13); p.ld_aux = 2 * F;
-      if (BNf == 256)
-        MOE_TRY((launch_tc<256, 4, tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD>(
-            "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
-      else
-        MOE_TRY((launch_tc<128, 6, tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD>(
-            "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
+      MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD>(
+          bn3, "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
     }
     // 4. wgrad down: dW_down[e] = dO^T h over the expert's rows
+    const int bn4 = pick_bn(F, (int64_t)groups * (D / 128), false, F);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 64, false));
     MOE_TRY(make_map(&mB, h, 1, L.rows_max, F, 64, false));
     {
       tc::Params p{};
       p.E = E; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
-      p.n_groups = E + c->n_shared; p.nMo = D / 128; p.nNo = F / BNf; p.No = F;
+      p.n_groups = groups; p.nMo = D / 128; p.nNo = F / bn4; p.No = F;
       p.strideCE = (int64_t)D * F;
       p.out = static_cast<__nv_bfloat16*>(dw_down);
       p.out_shared = static_cast<__nv_bfloat16*>(dw_down_s);
       const int total = p.n_groups * p.nMo * p.nNo;
-      if (BNf == 256)
-        MOE_TRY((launch_tc<256, 4, tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-            "tc_wgrad_down", mA, mB, mB, p, total, total, s)));
-      else
-        MOE_TRY((launch_tc<128, 6, tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-            "tc_wgrad_down", mA, mB, mB, p, total, total, s)));
+      MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
+          bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, s)));
     }
     // 5. dgrad gate/up: dX_perm = dA13 . w13[e]
+    const int bn5 = pick_bn(D, mt, false, F);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 128, false));
     MOE_TRY(make_map(&mB, w13, E, 2 * F, D, 64, true));                  // dims {D, 2F, E}
     MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, 64, true));
     {
-      tc::Params p = rows_params(c, 2 * F, D / BNd, tile_expert, stats);
+      tc::Params p = rows_params(c, 2 * F, D / bn5, tile_expert, stats);
       p.out = static_cast<__nv_bfloat16*>(dXp); p.ld_out = D;
-      if (BNd == 256)
-        MOE_TRY((launch_tc<256, 4, tc::MODE_ROWS, false, true, tc::EPI_STORE>(
-            "tc_dgrad_gate_up", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
-      else
-        MOE_TRY((launch_tc<128, 6, tc::MODE_ROWS, false, true, tc::EPI_STORE>(
-            "tc_dgrad_gate_up", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
+      MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE>(
+          bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
     }
     // 6. wgrad gate/up: dW13[e] = dA13^T x_perm
+    const int bn6 = pick_bn(D, (int64_t)groups * (2 * F / 128), false, F);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 64, false));
     MOE_TRY(make_map(&mB, x_perm, 1, L.rows_max, D, 64, false));
     {
       tc::Params p{};
       p.E = E; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
-      p.n_groups = E + c->n_shared; p.nMo = 2 * F / 128; p.nNo = D / BNd; p.No = D;
+      p.n_groups = groups; p.nMo = 2 * F / 128; p.nNo = D / bn6; p.No = D;
       p.strideCE = (int64_t)2 * F * D;
       p.out = static_cast<__nv_bfloat16*>(dw13);
       p.out_shared = static_cast<__nv_bfloat16*>(dw13_s);
       const int total = p.n_groups * p.nMo * p.nNo;
-      if (BNd == 256)
-        MOE_TRY((launch_tc<256, 4, tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-            "tc_wgrad_gate_up", mA, mB, mB, p, total, total, s)));
-      else
-        MOE_TRY((launch_tc<128, 6, tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-            "tc_wgrad_gate_up", mA, mB, mB, p, total, total, s)));
+      MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
+          bn6, "tc_wgrad_gate_up", mA, mB, mB, p, total, total, s)));
     }
   } else {
     auto go = [&](auto tag) -> int {
