@@ -248,6 +248,11 @@ int moe_combine(const moe_config_t* cfg, const void* o,
  * The gate gradient of a sentinel or dropped slot is zero (its expert
  * output is treated as zero), so such slots send no gradient to the router
  * through the gate path.  Deterministic: no floating-point atomics.
+ * Inside the call, independent chains (the router gradient, the two
+ * weight-gradient GEMMs) are forked onto side streams that the library
+ * creates once per host thread and device (on first use: make that first
+ * call outside stream capture) and joined back into `stream` before the
+ * call returns, so the results are ordered on `stream` like any other call.
  */
 int moe_backward(const moe_config_t* cfg,
                  const void* x, const float* w_r, const float* logits,
@@ -293,11 +298,16 @@ int64_t moe_launch_count(int reset);
  *                       milliseconds of each recorded launch to ms (host
  *                       array) and returns how many were written
  *   moe_profile_name    kernel family name of recorded launch i
+ *   moe_profile_side    1 if launch i ran on one of the library's side
+ *                       streams (concurrently with other work, so its
+ *                       duration includes sharing the GPU), 0 if on the
+ *                       caller's stream, -1 if i is out of range
  */
 int moe_profile_enable(int max_launches);
 int moe_profile_reset(void);
 int moe_profile_read(float* ms, int max);
 const char* moe_profile_name(int i);
+int moe_profile_side(int i);
 int moe_profile_disable(void);
 
 #ifdef __cplusplus

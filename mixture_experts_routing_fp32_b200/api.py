@@ -139,12 +139,14 @@ class LaunchProfile:
         lib().moe_profile_reset()
 
     def read(self):
-        """[(kernel name, ms)] of the launches since reset (caller synced)."""
+        """[(kernel name, ms, on_side_stream)] of the launches since reset
+        (the caller has synchronised)."""
         buf = (ctypes.c_float * self.max)()
         n = lib().moe_profile_read(buf, self.max)
         if n < 0:
             check(n, "moe_profile_read")
-        return [(lib().moe_profile_name(i).decode(), float(buf[i])) for i in range(n)]
+        return [(lib().moe_profile_name(i).decode(), float(buf[i]),
+                 lib().moe_profile_side(i) == 1) for i in range(n)]
 
     def close(self):
         lib().moe_profile_disable()

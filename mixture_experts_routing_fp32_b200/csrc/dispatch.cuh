@@ -42,11 +42,19 @@ disp_hist_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ ma
   __syncthreads();
   const int64_t j0 = (int64_t)blockIdx.x * kDispChunk;
   const int64_t j1 = min(j0 + kDispChunk, n_slots);
+  // every load of this thread first (one memory latency, not one per slot)
+  constexpr int kPer = kDispChunk / 256;
+  int ev[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int64_t j = j0 + threadIdx.x + (int64_t)k * 256;
+    ev[k] = (j < j1) ? slot_expert(idx, mask, j, E) : -2;
+  }
   int my_sent = 0;
-  for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-    const int e = slot_expert(idx, mask, j, E);
-    if (e >= 0) atomicAdd(&hist[e], 1);
-    else ++my_sent;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    if (ev[k] >= 0) atomicAdd(&hist[ev[k]], 1);
+    else if (ev[k] == -1) ++my_sent;
   }
   if (my_sent) atomicAdd(&sent, my_sent);
   __syncthreads();
@@ -70,6 +78,7 @@ disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ b
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int32_t run = 0;
+#pragma unroll 8
     for (int b = 0; b < n_blocks; ++b) {
       const int32_t c = block_hist[(size_t)b * E + e];
       block_hist[(size_t)b * E + e] = run;   // becomes the block's base rank
@@ -124,10 +133,17 @@ disp_rank_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ ma
   __syncthreads();
   const int64_t base = (int64_t)blockIdx.x * kDispChunk + (int64_t)warp * kDispIters * 32;
   const unsigned lt = (1u << lane) - 1u;
-  // per-warp histogram
+  // the warp's slots, loaded once up front
+  int ev[kDispIters];
+#pragma unroll
   for (int it = 0; it < kDispIters; ++it) {
     const int64_t j = base + it * 32 + lane;
-    const int e = (j < n_slots) ? slot_expert(idx, mask, j, E) : -1;
+    ev[it] = (j < n_slots) ? slot_expert(idx, mask, j, E) : -1;
+  }
+  // per-warp histogram
+#pragma unroll
+  for (int it = 0; it < kDispIters; ++it) {
+    const int e = ev[it];
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && (peers & lt) == 0) wh[warp * E + e] += __popc(peers);
   }
@@ -142,9 +158,10 @@ disp_rank_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ ma
     }
   }
   __syncthreads();
+#pragma unroll
   for (int it = 0; it < kDispIters; ++it) {
     const int64_t j = base + it * 32 + lane;
-    const int e = (j < n_slots) ? slot_expert(idx, mask, j, E) : -1;
+    const int e = ev[it];
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     int32_t rank = 0;
     if (e >= 0) rank = wh[warp * E + e] + __popc(peers & lt);

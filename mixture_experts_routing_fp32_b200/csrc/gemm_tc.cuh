@@ -42,6 +42,7 @@ enum { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2, EPI_WGRAD = 3 };
 struct Params {
   int E, F, Kd;
   int nN;                      // ROWS: output column tiles
+  int group_m;                 // ROWS: row tiles per rasterisation group
   const int32_t* tile_expert;  // ROWS
   const int32_t* stats;        // ROWS: stats[3] = 128-row tiles in use
   const int32_t* offsets;      // WGRAD: first row of each group
@@ -188,10 +189,42 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4& u, float* f) {
   }
 }
 
-// 32 floats -> 32 bf16 at p (64 bytes, 16-byte aligned).
-__device__ __forceinline__ void store32_bf16(__nv_bfloat16* p, const float (&v)[32]) {
+// L2 cache policies: epilogue outputs are written once and read by a later
+// kernel (evict first, so they do not push out operand tiles that are still
+// being reused); row tiles of the ROWS GEMMs are reused across the whole
+// column sweep of their rasterisation group (evict last).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar), "l"(pol)
+      : "memory");
+}
+
+// 32 floats -> 32 bf16 at p (64 bytes, 16-byte aligned), with an L2 policy.
+__device__ __forceinline__ void store32_bf16(__nv_bfloat16* p, const float (&v)[32],
+                                             uint64_t pol) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) store8(p + 8 * q, v + 8 * q);
+  for (int q = 0; q < 4; ++q) {
+    uint4 u;
+    __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h2[i] = __floats2bfloat162_rn(v[8 * q + 2 * i], v[8 * q + 2 * i + 1]);
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p + 8 * q),
+                 "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w), "l"(pol)
+                 : "memory");
+  }
 }
 __device__ __forceinline__ void load32_bf16(const __nv_bfloat16* p, float (&v)[32]) {
 #pragma unroll
@@ -213,7 +246,16 @@ template <int MODE, int EPI, int BN>
 __device__ __forceinline__ Tile decode(int t, const Params& p) {
   Tile d;
   if (MODE == MODE_ROWS) {
-    const int mt = t / p.nN, nt = t % p.nN;
+    // Grouped rasterisation: tiles run in groups of p.group_m row tiles, the
+    // column tile outermost inside a group, so the CTAs that run at the same
+    // time share their row tiles (kept in L2) and a few weight column
+    // slices, instead of streaming an expert's weights once per row tile.
+    const int n_mt = p.stats[3];
+    const int group = t / (p.group_m * p.nN);
+    const int first = group * p.group_m;
+    const int gm = min(p.group_m, n_mt - first);
+    const int local = t - group * p.group_m * p.nN;
+    const int mt = first + local % gm, nt = local / gm;
     d.e = p.tile_expert[mt];
     d.m0 = mt * BM;
     d.n0 = nt * (EPI == EPI_SWIGLU ? BN / 2 : BN);
@@ -294,6 +336,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
+      const uint64_t pol_a = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       int issued_parity[STAGES];
@@ -312,7 +355,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           mbar_expect_tx(fb, S::kStage);
           issued_parity[stage] = (int)phase;
           if (MODE == MODE_ROWS) {
-            tma_2d(sa, &mapA, fb, kb * BK, d.m0);
+            tma_2d_hint(sa, &mapA, fb, kb * BK, d.m0, pol_a);
             if (EPI == EPI_SWIGLU) {
               tma_3d(sb, mb, fb, kb * BK, d.n0, eb);
               tma_3d(sb + (BN / 2) * 128, mb, fb, kb * BK, p.F + d.n0, eb);
@@ -386,6 +429,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     const int rloc = q * 32 + lane;
     constexpr int HC = BN / 2;           // columns per warp (plain epilogues)
     constexpr int HJ = BN / 4;           // gate (= up) columns per warp (SwiGLU)
+    const uint64_t pol_out = policy_evict_first();
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -428,7 +472,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_ld32(tbase + hh * HC + c, r);
           tmem_wait();
           u2f32(r, v);
-          store32_bf16(dst + c, v);
+          store32_bf16(dst + c, v, pol_out);
         }
       } else if constexpr (EPI == EPI_SWIGLU) {
         __nv_bfloat16* a13 = p.out + row * p.ld_out + d.n0 + hh * HJ;
@@ -442,11 +486,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_wait();
           u2f32(rg, ga);
           u2f32(ru, ub);
-          store32_bf16(a13 + c, ga);
-          store32_bf16(a13 + p.F + c, ub);
+          store32_bf16(a13 + c, ga, pol_out);
+          store32_bf16(a13 + p.F + c, ub, pol_out);
 #pragma unroll
           for (int i = 0; i < 32; ++i) ga[i] = ga[i] * fast_sigmoid(ga[i]) * ub[i];
-          store32_bf16(hr + c, ga);
+          store32_bf16(hr + c, ga, pol_out);
         }
       } else {  // EPI_SWIGLU_BWD
         __nv_bfloat16* da13 = p.out + row * p.ld_out + d.n0 + hh * HC;
@@ -469,8 +513,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
             bv[i] = dh[i] * av[i] * sg;
             av[i] = da;
           }
-          store32_bf16(da13 + c, av);
-          store32_bf16(da13 + p.F + c, bv);
+          store32_bf16(da13 + c, av, pol_out);
+          store32_bf16(da13 + p.F + c, bv, pol_out);
         }
       }
       tc_fence_before();

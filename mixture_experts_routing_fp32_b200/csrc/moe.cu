@@ -29,6 +29,7 @@ constexpr int kProfMax = 256;
 struct Prof {
   cudaEvent_t ev[2 * kProfMax];
   const char* name[kProfMax];
+  int side[kProfMax];
   int n = 0, cap = 0;
 };
 thread_local Prof g_prof;
@@ -47,8 +48,10 @@ inline void prof_record(cudaEvent_t ev, cudaStream_t s) {
 inline void prof_begin(cudaStream_t s) {
   if (g_prof.n < g_prof.cap) prof_record(g_prof.ev[2 * g_prof.n], s);
 }
+bool is_side_stream(cudaStream_t s);
 inline void prof_end(cudaStream_t s, const char* name) {
   if (g_prof.n < g_prof.cap) {
+    g_prof.side[g_prof.n] = is_side_stream(s) ? 1 : 0;
     prof_record(g_prof.ev[2 * g_prof.n + 1], s);
     g_prof.name[g_prof.n++] = name;
   }
@@ -255,14 +258,18 @@ int64_t row_tiles_estimate(const moe_config_t* c, const Layout& L) {
   return ceil_div(rows, kRowTile) + (c->n_shared ? ceil_div(c->T, kRowTile) : 0);
 }
 
-// Output tile width BN in {256, 192, 128} minimising waves x BN (the time of
-// the busiest SM); ties keep the wider tile.  SwiGLU tiles hold BN/2 gate
-// and BN/2 up columns of F.
+// Output tile width BN in {256, 192, 128} minimising the busiest SM's time,
+// waves x BN / efficiency(BN): a narrower tile loads the same 128-row A
+// tile for fewer columns, so it moves more bytes per FLOP and keeps the
+// tensor pipe less busy (measured: BN=128 about 0.8 of BN=256 per column).
+// Ties keep the wider tile.  SwiGLU tiles hold BN/2 gate and BN/2 up
+// columns of F.
 int pick_bn(int64_t N, int64_t mtiles, bool swiglu, int64_t F) {
   const int64_t sms = num_sms();
   int best = 0;
   int64_t best_cost = INT64_MAX;
   for (int bn : {256, 192, 128}) {
+    const int64_t eff_pct = bn == 256 ? 100 : bn == 192 ? 95 : 80;
     int64_t nt;
     if (swiglu) {
       if (bn == 192 || F % (bn / 2)) continue;
@@ -271,7 +278,7 @@ int pick_bn(int64_t N, int64_t mtiles, bool swiglu, int64_t F) {
       if (N % bn) continue;
       nt = N / bn;
     }
-    const int64_t cost = ceil_div(mtiles * nt, sms) * bn;
+    const int64_t cost = ceil_div(mtiles * nt, sms) * bn * 100 / eff_pct;
     if (cost < best_cost) { best_cost = cost; best = bn; }
   }
   return best;
@@ -433,10 +440,57 @@ int simt_wgrad(const moe_config_t* c, const void* A, int64_t lda, const void* B,
   return MOE_OK;
 }
 
+// Side streams for the independent chains inside moe_backward (forked from
+// and joined back into the caller's stream within the call; under stream
+// capture the fork and join become graph edges).  Created once per host
+// thread and device, on first use.
+constexpr int kMaxSideDevices = 64;
+struct Side {
+  cudaStream_t st[3];
+  cudaEvent_t ev[6];
+  bool ok = false;
+};
+thread_local Side g_side[kMaxSideDevices];
+
+int side_streams(Side** out) {
+  int dev = 0;
+  MOE_CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxSideDevices) return MOE_ERR_ARG;
+  Side& sd = g_side[dev];
+  if (!sd.ok) {
+    for (auto& st : sd.st) MOE_CK(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
+    for (auto& ev : sd.ev) MOE_CK(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    sd.ok = true;
+  }
+  *out = &sd;
+  return MOE_OK;
+}
+
+bool is_side_stream(cudaStream_t s) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return false;
+  const Side& sd = g_side[dev];
+  return sd.ok && (s == sd.st[0] || s == sd.st[1] || s == sd.st[2]);
+}
+
+// `to` waits for everything issued so far on `from`.
+int fork_join(cudaEvent_t ev, cudaStream_t from, cudaStream_t to) {
+  MOE_CK(cudaEventRecord(ev, from));
+  MOE_CK(cudaStreamWaitEvent(to, ev, 0));
+  return MOE_OK;
+}
+
+// Row tiles per rasterisation group: as many 128-row A tiles of depth Kd as
+// fit in about 48 MiB of L2, so they stay resident while the group sweeps
+// the weight column slices.
+int group_rows(int64_t Kd) {
+  return (int)std::max<int64_t>(1, std::min<int64_t>(64, (48ll << 20) / (128ll * Kd * 2)));
+}
+
 tc::Params rows_params(const moe_config_t* c, int Kd, int nN, const int32_t* tile_expert,
                        const int32_t* stats) {
   tc::Params p{};
-  p.E = c->E; p.F = c->F; p.Kd = Kd; p.nN = nN;
+  p.E = c->E; p.F = c->F; p.Kd = Kd; p.nN = nN; p.group_m = group_rows(Kd);
   p.tile_expert = tile_expert; p.stats = stats; p.T = c->T;
   return p;
 }
@@ -724,12 +778,22 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
           kept, tile_expert, stats, K, E, T, D, dg, static_cast<float*>(dO));
     MOE_LAUNCHED(s, "bwd_gate_grad_rows");
   }
+  // The router gradient chain (2, 7) runs on side stream r, concurrently
+  // with the expert GEMMs (3-6); the two weight-gradient GEMMs run on side
+  // streams w1, w2 once the SwiGLU-backward GEMM is done.  Everything joins
+  // back into s before the dx kernel (8) and before returning.
+  Side* sd = nullptr;
+  MOE_TRY(side_streams(&sd));
+  cudaStream_t r = sd->st[0], w1 = sd->st[1], w2 = sd->st[2];
+  MOE_TRY(fork_join(sd->ev[0], s, r));
   // 2. router backward: dlogits
   {
     RouterBwdArgs a{T, E, K, c->score_fn, c->renorm, c->route_scale, c->aux_alpha, c->z_lambda,
                     logits, probs, lse, topk_idx, topk_w, slot_row, dg, counts, ds, dlogits_out,
                     dg_out};
     const int grid = grid_for(T);
+    {
+    cudaStream_t s = r;
     prof_begin(s);
     if (E <= 32) router_bwd_kernel<1><<<grid, 256, 0, s>>>(a);
     else if (E <= 64) router_bwd_kernel<2><<<grid, 256, 0, s>>>(a);
@@ -737,6 +801,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     else if (E <= 256) router_bwd_kernel<8><<<grid, 256, 0, s>>>(a);
     else router_bwd_kernel<16><<<grid, 256, 0, s>>>(a);
     MOE_LAUNCHED(s, "router_bwd");
+    }
   }
   // 3-6. expert GEMMs
   if (use_tc(c)) {
@@ -755,6 +820,8 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD>(
           bn3, "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
     }
+    MOE_TRY(fork_join(sd->ev[1], s, w1));
+    MOE_TRY(fork_join(sd->ev[2], s, w2));
     // 4. wgrad down: dW_down[e] = dO^T h over the expert's rows
     const int bn4 = pick_bn(F, (int64_t)groups * (D / 128), false, F);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 64, false));
@@ -768,7 +835,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       p.out_shared = static_cast<__nv_bfloat16*>(dw_down_s);
       const int total = p.n_groups * p.nMo * p.nNo;
       MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-          bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, s)));
+          bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1)));
     }
     // 5. dgrad gate/up: dX_perm = dA13 . w13[e]
     const int bn5 = pick_bn(D, mt, false, F);
@@ -794,7 +861,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       p.out_shared = static_cast<__nv_bfloat16*>(dw13_s);
       const int total = p.n_groups * p.nMo * p.nNo;
       MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-          bn6, "tc_wgrad_gate_up", mA, mB, mB, p, total, total, s)));
+          bn6, "tc_wgrad_gate_up", mA, mB, mB, p, total, total, w2)));
     }
   } else {
     auto go = [&](auto tag) -> int {
@@ -818,8 +885,9 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     if (bf) MOE_TRY(go(__nv_bfloat16{}));
     else MOE_TRY(go(float{}));
   }
-  // 7. dW_r = ds^T x (two deterministic stages)
+  // 7. dW_r = ds^T x (two deterministic stages), on the router stream
   {
+    cudaStream_t s = r;
     const int nc = L.n_dwr_chunks;
     prof_begin(s);
     if (E <= 8) {
@@ -842,7 +910,8 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
         dwr_part, nc, n, dw_r);
     MOE_LAUNCHED(s, "router_dw_reduce");
   }
-  // 8. dx = unpermute-sum(dX_perm) + shared + ds . w_r
+  // join the router chain, then 8. dx = unpermute-sum(dX_perm) + shared + ds . w_r
+  MOE_TRY(fork_join(sd->ev[3], r, s));
   {
     dim3 g((unsigned)ceil_div(T, 64), (unsigned)ceil_div(D, 128));
     prof_begin(s);
@@ -856,6 +925,9 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
                                          static_cast<float*>(dx));
     MOE_LAUNCHED(s, "dx_unpermute_router");
   }
+  // join the weight-gradient streams (no-ops on the SIMT path)
+  MOE_TRY(fork_join(sd->ev[4], w1, s));
+  MOE_TRY(fork_join(sd->ev[5], w2, s));
   return MOE_OK;
 }
 
@@ -906,6 +978,10 @@ int moe_profile_read(float* ms, int max) {
 
 const char* moe_profile_name(int i) {
   return (i >= 0 && i < g_prof.n) ? g_prof.name[i] : "";
+}
+
+int moe_profile_side(int i) {
+  return (i >= 0 && i < g_prof.n) ? g_prof.side[i] : -1;
 }
 
 int moe_profile_disable(void) {

@@ -43,7 +43,17 @@ class MoELayer:
         self.y = e((T, D), act)
         self.losses = torch.zeros(2, dtype=f32, device=dev)
         self.ws = e((max(int(z.ws_bytes), 256),), torch.uint8)
-        # gradients
+        self._grads_ready = False
+        self._inputs = None
+
+    def _alloc_grads(self):
+        """Gradient buffers, allocated on the first backward (a forward-only
+        user never holds them)."""
+        if self._grads_ready:
+            return
+        c, dev, act, f32 = self.cfg, self.device, self.act_dtype, torch.float32
+        T, D, E, K, F = c.T, c.D, c.E, c.K, c.F
+        e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
         self.dx = e((T, D), act)
         self.dw_r = e((E, D), f32)
         self.dw13, self.dw_down = e((E, 2 * F, D), act), e((E, D, F), act)
@@ -51,7 +61,7 @@ class MoELayer:
         self.dw_down_s = e((D, F), act) if c.n_shared else None
         self.dg = e((T, K), f32)
         self.dlogits = e((T, E), f32)
-        self._inputs = None
+        self._grads_ready = True
 
     # -- forward -----------------------------------------------------------
     def forward(self, x, w_r, w13, w_down, w13_s=None, w_down_s=None,
@@ -73,6 +83,7 @@ class MoELayer:
 
     # -- backward ----------------------------------------------------------
     def backward(self, dy, want_dg=True, want_dlogits=True):
+        self._alloc_grads()
         x, w_r, w13, w_down, w13_s, w_down_s = self._inputs
         api.moe_backward(
             self.cfg, x, w_r, self.logits, self.probs, self.lse, self.topk_idx,
