@@ -29,8 +29,9 @@
  *     word that moe_check_status() reads and clears.
  *   - Permuted row space: routed expert e owns rows
  *     [offsets[e], offsets[e+1]); its kept slots occupy the first kept[e]
- *     rows in flat-slot order, the rest up to the next multiple of 128 are
- *     zero padding.  The shared expert (n_shared = 1) owns rows
+ *     rows in flat-slot order, the rest up to the next multiple of
+ *     row_align (128, or 256 when the expert GEMMs run on CTA pairs; see
+ *     moe_get_sizes) are zero padding.  The shared expert (n_shared = 1) owns rows
  *     [offsets[E], offsets[E+1]) = its T tokens in order, then padding.
  *     Buffers indexed by row are sized rows_max (moe_get_sizes).
  */
@@ -107,6 +108,7 @@ typedef struct {
   int64_t tiles_max;    /* rows_max / 128 */
   int64_t capacity;     /* C, or -1 when unlimited */
   size_t ws_bytes;      /* workspace needed by any call (256-byte aligned base) */
+  int64_t row_align;    /* expert segments start at multiples of this (128 or 256) */
 } moe_sizes_t;
 
 /* Buffer sizes for cfg.  Host-only, no CUDA calls. */

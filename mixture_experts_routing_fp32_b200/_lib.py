@@ -42,7 +42,8 @@ class MoeConfig(ctypes.Structure):
 
 class MoeSizes(ctypes.Structure):
     _fields_ = [("rows_max", c_int64), ("tiles_max", c_int64),
-                ("capacity", c_int64), ("ws_bytes", ctypes.c_size_t)]
+                ("capacity", c_int64), ("ws_bytes", ctypes.c_size_t),
+                ("row_align", c_int64)]
 
 
 class MoEError(RuntimeError):

@@ -64,11 +64,12 @@ disp_hist_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ ma
 }
 
 // Pass 2 (one block): per-expert totals, exclusive scan over blocks (block
-// bases), capacity, padded offsets, tile -> expert map, stats.
+// bases), capacity, padded offsets (segments aligned to `align` rows, a
+// multiple of the 128-row tile), tile -> expert map, stats.
 __global__ void __launch_bounds__(1024)
 disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ block_sent,
                  int n_blocks, int E, int T, int n_shared, int64_t C,
-                 int64_t rows_max, int32_t* __restrict__ counts,
+                 int64_t rows_max, int align, int32_t* __restrict__ counts,
                  int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
                  int32_t* __restrict__ tile_expert, int32_t* __restrict__ stats) {
   extern __shared__ int64_t sh[];     // [E] padded sizes -> offsets
@@ -89,7 +90,7 @@ disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ b
     kept[e] = k;
     if (run > k) atomicAdd((unsigned long long*)&drop_total,
                            (unsigned long long)(run - k));
-    sh[e] = ((int64_t)k + kRowTile - 1) / kRowTile * kRowTile;
+    sh[e] = ((int64_t)k + align - 1) / align * align;
   }
   for (int b = threadIdx.x; b < n_blocks; b += blockDim.x)
     atomicAdd(&sent_total, block_sent[b]);
@@ -97,7 +98,7 @@ disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ b
   if (threadIdx.x == 0) {   // E <= 512: a serial scan is negligible
     int64_t run = 0;
     for (int e = 0; e < E; ++e) { const int64_t v = sh[e]; sh[e] = run; run += v; }
-    const int64_t shared_rows = n_shared ? ((int64_t)T + kRowTile - 1) / kRowTile * kRowTile : 0;
+    const int64_t shared_rows = n_shared ? ((int64_t)T + align - 1) / align * align : 0;
     int64_t total = run + shared_rows;
     if (total > rows_max) { set_dev_error(MOE_DEVERR_ROWS); total = rows_max; }
     offsets[E] = (int32_t)run;

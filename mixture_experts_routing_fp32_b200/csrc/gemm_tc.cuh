@@ -121,6 +121,78 @@ __device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, uin
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
       : "memory");
 }
+// ---- CTA-pair (cta_group::2) forms: two SMs of one cluster share each MMA
+// (each holds half of A's rows and half of B's columns; each gets its own
+// 128-row slice of the accumulator) -------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory completing on the pair leader's
+// barrier (`bar` is a shared::cluster address).  No multicast.
+__device__ __forceinline__ void tma_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_2d_pair_nohint(uint32_t dst, const CUtensorMap* map,
+                                                   uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                          uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+// Arrive on the barrier at this offset in both CTAs of the pair once the
+// MMAs issued so far are complete.
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar), "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair_local(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// Arrive on a barrier in another CTA of the cluster (cluster address).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
@@ -242,22 +314,26 @@ struct Tile {
   int nk;       // K blocks (0: empty group)
 };
 
-template <int MODE, int EPI, int BN>
-__device__ __forceinline__ Tile decode(int t, const Params& p) {
+// M rows per tile: 128, or 256 for a CTA pair (this CTA holds 128 of them).
+template <int MODE, int EPI, int BN, bool PAIR>
+__device__ __forceinline__ Tile decode(int t, const Params& p, int rank) {
+  constexpr int MU = PAIR ? 2 * BM : BM;
   Tile d;
   if (MODE == MODE_ROWS) {
     // Grouped rasterisation: tiles run in groups of p.group_m row tiles, the
     // column tile outermost inside a group, so the CTAs that run at the same
     // time share their row tiles (kept in L2) and a few weight column
     // slices, instead of streaming an expert's weights once per row tile.
-    const int n_mt = p.stats[3];
+    // With a CTA pair a row tile is 256 rows: two 128-row tiles of one
+    // expert (expert segments are then 256-row aligned).
+    const int n_mt = p.stats[3] / (PAIR ? 2 : 1);
     const int group = t / (p.group_m * p.nN);
     const int first = group * p.group_m;
     const int gm = min(p.group_m, n_mt - first);
     const int local = t - group * p.group_m * p.nN;
     const int mt = first + local % gm, nt = local / gm;
-    d.e = p.tile_expert[mt];
-    d.m0 = mt * BM;
+    d.e = p.tile_expert[mt * (MU / BM)];
+    d.m0 = mt * MU + rank * BM;
     d.n0 = nt * (EPI == EPI_SWIGLU ? BN / 2 : BN);
     d.row0 = 0;
     d.nk = p.Kd / BK;
@@ -265,7 +341,7 @@ __device__ __forceinline__ Tile decode(int t, const Params& p) {
     const int per = p.nMo * p.nNo;
     const int g = t / per, rem = t % per;
     d.e = g;
-    d.m0 = (rem / p.nNo) * BM;
+    d.m0 = (rem / p.nNo) * MU + rank * BM;
     d.n0 = (rem % p.nNo) * BN;
     d.row0 = p.offsets[g];
     const int rows = g < p.E ? p.kept[g] : p.T;
@@ -274,20 +350,24 @@ __device__ __forceinline__ Tile decode(int t, const Params& p) {
   return d;
 }
 
-template <int BN, int STAGES>
+// Shared memory per CTA: BNC = columns of B this CTA holds (BN, or BN/2
+// for a CTA pair).
+template <int BN, int STAGES, bool PAIR>
 struct Smem {
+  static constexpr int BNC = PAIR ? BN / 2 : BN;
   static constexpr int kA = BM * BK * 2;        // 16 KB
-  static constexpr int kB = BN * BK * 2;
+  static constexpr int kB = BNC * BK * 2;
   static constexpr int kStage = kA + kB;
   static constexpr int kBars = (2 * STAGES + 5) * 8;
   static constexpr int kBytes = 1024 + STAGES * kStage + kBars + 16;
 };
 
-template <int BN, int STAGES, int MODE, bool A_MN, bool B_MN, int EPI>
+template <int BN, int STAGES, int MODE, bool A_MN, bool B_MN, int EPI, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
             const __grid_constant__ CUtensorMap mapBs, const Params p, int total_hint) {
-  using S = Smem<BN, STAGES>;
+  using S = Smem<BN, STAGES, PAIR>;
+  constexpr int BNC = S::BNC;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int abort_flag_s;
   volatile int* abort_flag = &abort_flag_s;
@@ -303,38 +383,55 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * S::kStage + S::kBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = PAIR ? (int)cluster_rank() : 0;        // 0 = pair leader
+  const bool leader = rank == 0;
+  const int unit = PAIR ? blockIdx.x >> 1 : blockIdx.x;   // this CTA's tile stream
+  const int n_units = PAIR ? gridDim.x >> 1 : gridDim.x;
   // tensor memory: two BN-column fp32 accumulators; tcgen05.alloc takes a
   // power of two between 32 and 512 columns
   constexpr uint32_t kCols = (2 * BN <= 128) ? 128u : (2 * BN <= 256) ? 256u : 512u;
   static_assert(2 * BN <= 512 && (kCols & (kCols - 1)) == 0, "tensor-memory columns");
+  static_assert(!PAIR || (BNC % 64 == 0), "pair tiles hold whole 64-column B boxes");
 
   if (threadIdx.x == 0) {
     abort_flag_s = 0;
     for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(accf_bar(b), 1); mbar_init(acce_bar(b), kEpiWarps); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), kEpiWarps * (PAIR ? 2 : 1));   // both CTAs' epilogues
+    }
     mbar_init(done_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0) {
     __syncwarp();
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(kCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(kCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(kCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   int total;
-  if (MODE == MODE_ROWS) total = p.stats[3] * p.nN;
+  if (MODE == MODE_ROWS) total = (p.stats[3] / (PAIR ? 2 : 1)) * p.nN;
   else total = total_hint;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (both CTAs of a pair) ----------------
     if (lane == 0) {
       const uint64_t pol_a = policy_evict_last();
       int stage = 0;
@@ -343,8 +440,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile d = decode<MODE, EPI, BN>(t, p);
+      for (int t = unit; t < total && ok; t += n_units) {
+        const Tile d = decode<MODE, EPI, BN, PAIR>(t, p, rank);
         const CUtensorMap* mb = (MODE == MODE_ROWS && d.e >= p.E) ? &mapBs : &mapB;
         const int eb = (MODE == MODE_ROWS && d.e >= p.E) ? 0 : d.e;
         for (int kb = 0; kb < d.nk; ++kb) {
@@ -352,45 +449,71 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           const uint32_t sa = base + stage * S::kStage;
           const uint32_t sb = sa + S::kA;
           const uint32_t fb = full_bar(stage);
-          mbar_expect_tx(fb, S::kStage);
+          if (!PAIR || leader) mbar_expect_tx(fb, S::kStage * (PAIR ? 2 : 1));
           issued_parity[stage] = (int)phase;
-          if (MODE == MODE_ROWS) {
-            tma_2d_hint(sa, &mapA, fb, kb * BK, d.m0, pol_a);
-            if (EPI == EPI_SWIGLU) {
-              tma_3d(sb, mb, fb, kb * BK, d.n0, eb);
-              tma_3d(sb + (BN / 2) * 128, mb, fb, kb * BK, p.F + d.n0, eb);
-            } else if (!B_MN) {
-              tma_3d(sb, mb, fb, kb * BK, d.n0, eb);
-            } else {
+          if constexpr (PAIR) {
+            const uint32_t lfb = mapa(fb, 0);           // the leader's full barrier
+            if (MODE == MODE_ROWS) {
+              tma_2d_pair(sa, &mapA, lfb, kb * BK, d.m0, pol_a);
+              if (EPI == EPI_SWIGLU) {
+                // this CTA holds the gate (rank 0) or the up (rank 1) half
+                tma_3d_pair(sb, mb, lfb, kb * BK, (rank ? p.F : 0) + d.n0, eb);
+              } else if (!B_MN) {
+                tma_3d_pair(sb, mb, lfb, kb * BK, d.n0 + rank * BNC, eb);
+              } else {
 #pragma unroll
-              for (int c = 0; c < BN / 64; ++c)
-                tma_3d(sb + c * 8192, mb, fb, d.n0 + c * 64, kb * BK, eb);
+                for (int c = 0; c < BNC / 64; ++c)
+                  tma_3d_pair(sb + c * 8192, mb, lfb, d.n0 + rank * BNC + c * 64, kb * BK, eb);
+              }
+            } else {
+              const int r = d.row0 + kb * BK;
+              tma_2d_pair_nohint(sa, &mapA, lfb, d.m0, r);
+              tma_2d_pair_nohint(sa + 8192, &mapA, lfb, d.m0 + 64, r);
+#pragma unroll
+              for (int c = 0; c < BNC / 64; ++c)
+                tma_2d_pair_nohint(sb + c * 8192, &mapB, lfb, d.n0 + rank * BNC + c * 64, r);
             }
           } else {
-            const int r = d.row0 + kb * BK;
-            tma_2d(sa, &mapA, fb, d.m0, r);
-            tma_2d(sa + 8192, &mapA, fb, d.m0 + 64, r);
+            if (MODE == MODE_ROWS) {
+              tma_2d_hint(sa, &mapA, fb, kb * BK, d.m0, pol_a);
+              if (EPI == EPI_SWIGLU) {
+                tma_3d(sb, mb, fb, kb * BK, d.n0, eb);
+                tma_3d(sb + (BN / 2) * 128, mb, fb, kb * BK, p.F + d.n0, eb);
+              } else if (!B_MN) {
+                tma_3d(sb, mb, fb, kb * BK, d.n0, eb);
+              } else {
 #pragma unroll
-            for (int c = 0; c < BN / 64; ++c) tma_2d(sb + c * 8192, &mapB, fb, d.n0 + c * 64, r);
+                for (int c = 0; c < BN / 64; ++c)
+                  tma_3d(sb + c * 8192, mb, fb, d.n0 + c * 64, kb * BK, eb);
+              }
+            } else {
+              const int r = d.row0 + kb * BK;
+              tma_2d(sa, &mapA, fb, d.m0, r);
+              tma_2d(sa + 8192, &mapA, fb, d.m0 + 64, r);
+#pragma unroll
+              for (int c = 0; c < BN / 64; ++c) tma_2d(sb + c * 8192, &mapB, fb, d.n0 + c * 64, r);
+            }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      // drain: every copy this thread issued has landed before teardown
-      for (int s = 0; s < STAGES; ++s)
-        if (issued_parity[s] >= 0) mbar_wait(full_bar(s), (uint32_t)issued_parity[s], abort_flag);
+      // drain: the copies this CTA's barriers track have landed before
+      // teardown (a pair's copies all complete on the leader's barriers)
+      if (!PAIR || leader)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_parity[s] >= 0) mbar_wait(full_bar(s), (uint32_t)issued_parity[s], abort_flag);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc(BM, BN, A_MN, B_MN);
+    // ---------------- MMA issuer (the pair leader only) ----------------
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = make_idesc(PAIR ? 2 * BM : BM, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile d = decode<MODE, EPI, BN>(t, p);
+      for (int t = unit; t < total && ok; t += n_units) {
+        const Tile d = decode<MODE, EPI, BN, PAIR>(t, p, rank);
         if (d.nk == 0) continue;
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
@@ -406,18 +529,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
                                      : sw128_desc(sa + ks * 32, 16, 1024);
             const uint64_t bd = B_MN ? sw128_desc(sb + ks * 2048, 8192, 1024)
                                      : sw128_desc(sb + ks * 32, 16, 1024);
-            umma(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+            if constexpr (PAIR) umma_pair(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+            else umma(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
           }
-          umma_commit(empty_bar(stage));
+          if constexpr (PAIR) umma_commit_pair_both(empty_bar(stage));
+          else umma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(accf_bar(acc));
+        if constexpr (PAIR) umma_commit_pair_both(accf_bar(acc));
+        else umma_commit(accf_bar(acc));
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       // all MMAs issued by this thread complete before teardown
-      umma_commit(done_bar);
+      if constexpr (PAIR) umma_commit_pair_local(done_bar);
+      else umma_commit(done_bar);
       mbar_wait(done_bar, 0, abort_flag);
     }
   } else {
@@ -432,8 +559,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     const uint64_t pol_out = policy_evict_first();
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile d = decode<MODE, EPI, BN>(t, p);
+    for (int t = unit; t < total; t += n_units) {
+      const Tile d = decode<MODE, EPI, BN, PAIR>(t, p, rank);
       if (MODE == MODE_WGRAD && d.nk == 0) {
         __nv_bfloat16* og = d.e < p.E ? p.out + (int64_t)d.e * p.strideCE : p.out_shared;
         __nv_bfloat16* dst = og + (int64_t)(d.m0 + rloc) * p.No + d.n0 + hh * HC;
@@ -519,18 +646,26 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce_bar(acc));
+      if (lane == 0) {
+        if (!PAIR || leader) mbar_arrive(acce_bar(acc));
+        else mbar_arrive_remote(mapa(acce_bar(acc), 0));   // the leader's barrier
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // the leader's MMAs into both CTAs are done
   tc_fence_after();
   if (warp == 0) {
     __syncwarp();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols)
-                 : "memory");
+    if constexpr (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols)
+                   : "memory");
   }
 }
 

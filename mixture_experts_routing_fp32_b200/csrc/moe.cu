@@ -127,9 +127,27 @@ bool use_tc(const moe_config_t* c) {
          (c->F % 128) == 0;
 }
 
+int64_t capacity_of(const moe_config_t* c);
+
+// Row GEMMs run on CTA pairs (two SMs share each 256-row MMA) when experts
+// hold enough rows that aligning their segments to 256 rows wastes little
+// and the extra operand reuse pays (at least 1536 rows on average: measured
+// faster for the OLMoE- and Mixtral-shaped layers, slower for 1024-row
+// experts); the permuted row space is then 256-row aligned.  Otherwise
+// segments are 128-row aligned and single-CTA tiles run.
+bool pair_rows(const moe_config_t* c) {
+  if (!use_tc(c)) return false;
+  const int64_t C = capacity_of(c);
+  const int64_t slots = (int64_t)c->T * c->K;
+  const int64_t kept = C < 0 ? slots : std::min<int64_t>(slots, (int64_t)c->E * C);
+  return kept / c->E >= 1536;
+}
+
+int row_align(const moe_config_t* c) { return pair_rows(c) ? 256 : kRowTile; }
+
 struct Layout {
   int64_t rows_max, tiles_max, C, n_slots;
-  int n_disp_blocks, n_aux_chunks, n_dwr_chunks, dwr_chunk;
+  int n_disp_blocks, n_aux_chunks, n_dwr_chunks, dwr_chunk, align;
   size_t off_bhist, off_bsent, off_aux, off_dg, off_ds, off_dwr, off_dO, off_dA13, off_dX,
       off_dH, total;
 };
@@ -149,10 +167,11 @@ Layout layout_of(const moe_config_t* c) {
   L.C = capacity_of(c);
   L.n_slots = (int64_t)c->T * c->K;
   const int64_t kept_total = L.C < 0 ? L.n_slots : std::min<int64_t>(L.n_slots, (int64_t)c->E * L.C);
-  const int64_t pad = (int64_t)(kRowTile - 1) * std::min<int64_t>(c->E, kept_total);
-  L.rows_max = round_up(kept_total + pad, kRowTile) +
-               (c->n_shared ? round_up(c->T, kRowTile) : 0);
-  if (L.rows_max == 0) L.rows_max = kRowTile;
+  const int64_t align = row_align(c);
+  const int64_t pad = (align - 1) * std::min<int64_t>(c->E, kept_total);
+  L.rows_max = round_up(kept_total + pad, align) + (c->n_shared ? round_up(c->T, align) : 0);
+  if (L.rows_max == 0) L.rows_max = align;
+  L.align = (int)align;
   L.tiles_max = L.rows_max / kRowTile;
   L.n_disp_blocks = (int)ceil_div(L.n_slots, kDispChunk);
   L.n_aux_chunks = (int)ceil_div(c->T, kAuxChunk);
@@ -219,34 +238,76 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t n3, int64_t rows, int64_t 
   return MOE_OK;
 }
 
-template <int BN, int ST, int MODE, bool AMN, bool BMN, int EPI>
+template <int BN, int ST, int MODE, bool AMN, bool BMN, int EPI, bool PAIR>
 int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
               const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
               cudaStream_t s) {
-  using S = tc::Smem<BN, ST>;
-  auto k = tc::gemm_kernel<BN, ST, MODE, AMN, BMN, EPI>;
+  using S = tc::Smem<BN, ST, PAIR>;
+  auto k = tc::gemm_kernel<BN, ST, MODE, AMN, BMN, EPI, PAIR>;
   MOE_CK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes));
-  const int grid = (int)std::min<int64_t>(num_sms(), total_max);
-  if (grid <= 0) return MOE_OK;
-  prof_begin(s);
-  k<<<grid, tc::kThreads, S::kBytes, s>>>(a, b, bs, p, total_hint);
-  MOE_LAUNCHED(s, name);
+  if constexpr (PAIR) {
+    // as many CTA pairs as can be resident at once (one per two SMs of a GPC)
+    static int max_pairs = 0;
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.blockDim = dim3(tc::kThreads);
+    lc.dynamicSmemBytes = S::kBytes;
+    lc.stream = s;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    if (max_pairs == 0) {
+      lc.gridDim = dim3(2 * (num_sms() / 2));
+      int n = 0;
+      MOE_CK(cudaOccupancyMaxActiveClusters(&n, k, &lc));
+      max_pairs = n > 0 ? n : num_sms() / 2;
+    }
+    const int pairs = (int)std::min<int64_t>(max_pairs, total_max);
+    if (pairs <= 0) return MOE_OK;
+    lc.gridDim = dim3(2 * pairs);
+    prof_begin(s);
+    MOE_CK(cudaLaunchKernelEx(&lc, k, a, b, bs, p, total_hint));
+    MOE_LAUNCHED(s, name);
+  } else {
+    const int grid = (int)std::min<int64_t>(num_sms(), total_max);
+    if (grid <= 0) return MOE_OK;
+    prof_begin(s);
+    k<<<grid, tc::kThreads, S::kBytes, s>>>(a, b, bs, p, total_hint);
+    MOE_LAUNCHED(s, name);
+  }
   return MOE_OK;
 }
 
-template <int MODE, bool AMN, bool BMN, int EPI>
+template <int MODE, bool AMN, bool BMN, int EPI, bool PAIR = false>
 int run_tc(int bn, const char* name, const CUtensorMap& a, const CUtensorMap& b,
            const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
            cudaStream_t s) {
-  if (bn == 256)
-    return launch_tc<256, 4, MODE, AMN, BMN, EPI>(name, a, b, bs, p, total_max, total_hint, s);
-  if constexpr (EPI != tc::EPI_SWIGLU) {
-    if (bn == 192)
-      return launch_tc<192, 5, MODE, AMN, BMN, EPI>(name, a, b, bs, p, total_max, total_hint, s);
+  if constexpr (PAIR) {
+    // per CTA: A 16 KB + half of B per stage
+    if (bn == 256)
+      return launch_tc<256, 6, MODE, AMN, BMN, EPI, true>(name, a, b, bs, p, total_max,
+                                                         total_hint, s);
+    if (bn == 128)
+      return launch_tc<128, 8, MODE, AMN, BMN, EPI, true>(name, a, b, bs, p, total_max,
+                                                         total_hint, s);
+    return MOE_ERR_ARG;
+  } else {
+    if (bn == 256)
+      return launch_tc<256, 4, MODE, AMN, BMN, EPI, false>(name, a, b, bs, p, total_max,
+                                                          total_hint, s);
+    if constexpr (EPI != tc::EPI_SWIGLU) {
+      if (bn == 192)
+        return launch_tc<192, 5, MODE, AMN, BMN, EPI, false>(name, a, b, bs, p, total_max,
+                                                            total_hint, s);
+    }
+    if (bn == 128)
+      return launch_tc<128, 6, MODE, AMN, BMN, EPI, false>(name, a, b, bs, p, total_max,
+                                                          total_hint, s);
+    return MOE_ERR_ARG;
   }
-  if (bn == 128)
-    return launch_tc<128, 6, MODE, AMN, BMN, EPI>(name, a, b, bs, p, total_max, total_hint, s);
-  return MOE_ERR_ARG;
 }
 
 // Expected 128-row tiles of the permuted rows (half a tile of padding per
@@ -264,11 +325,13 @@ int64_t row_tiles_estimate(const moe_config_t* c, const Layout& L) {
 // tensor pipe less busy (measured: BN=128 about 0.8 of BN=256 per column).
 // Ties keep the wider tile.  SwiGLU tiles hold BN/2 gate and BN/2 up
 // columns of F.
-int pick_bn(int64_t N, int64_t mtiles, bool swiglu, int64_t F) {
-  const int64_t sms = num_sms();
+int pick_bn(int64_t N, int64_t mtiles, bool swiglu, int64_t F, bool pair = false) {
+  const int64_t sms = pair ? num_sms() / 2 : num_sms();
+  if (pair) mtiles = ceil_div(mtiles, 2);
   int best = 0;
   int64_t best_cost = INT64_MAX;
   for (int bn : {256, 192, 128}) {
+    if (pair && bn == 192) continue;
     const int64_t eff_pct = bn == 256 ? 100 : bn == 192 ? 95 : 80;
     int64_t nt;
     if (swiglu) {
@@ -483,14 +546,15 @@ int fork_join(cudaEvent_t ev, cudaStream_t from, cudaStream_t to) {
 // Row tiles per rasterisation group: as many 128-row A tiles of depth Kd as
 // fit in about 48 MiB of L2, so they stay resident while the group sweeps
 // the weight column slices.
-int group_rows(int64_t Kd) {
-  return (int)std::max<int64_t>(1, std::min<int64_t>(64, (48ll << 20) / (128ll * Kd * 2)));
+int group_rows(int64_t Kd, bool pair = false) {
+  const int64_t rows = pair ? 256 : 128;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(64, (48ll << 20) / (rows * Kd * 2)));
 }
 
 tc::Params rows_params(const moe_config_t* c, int Kd, int nN, const int32_t* tile_expert,
-                       const int32_t* stats) {
+                       const int32_t* stats, bool pair = false) {
   tc::Params p{};
-  p.E = c->E; p.F = c->F; p.Kd = Kd; p.nN = nN; p.group_m = group_rows(Kd);
+  p.E = c->E; p.F = c->F; p.Kd = Kd; p.nN = nN; p.group_m = group_rows(Kd, pair);
   p.tile_expert = tile_expert; p.stats = stats; p.T = c->T;
   return p;
 }
@@ -510,6 +574,7 @@ int moe_get_sizes(const moe_config_t* cfg, moe_sizes_t* out) {
   out->tiles_max = L.tiles_max;
   out->capacity = L.C;
   out->ws_bytes = L.total;
+  out->row_align = L.align;
   return MOE_OK;
 }
 
@@ -544,8 +609,8 @@ int moe_dispatch(const moe_config_t* c, const int32_t* topk_idx, const uint8_t* 
   MOE_LAUNCHED(s, "dispatch_hist");
   prof_begin(s);
   disp_scan_kernel<<<1, 1024, c->E * 8, s>>>(bhist, bsent, L.n_disp_blocks, c->E, c->T,
-                                             c->n_shared, L.C, L.rows_max, counts, kept,
-                                             offsets, tile_expert, stats);
+                                             c->n_shared, L.C, L.rows_max, L.align, counts,
+                                             kept, offsets, tile_expert, stats);
   MOE_LAUNCHED(s, "dispatch_scan");
   prof_begin(s);
   disp_rank_kernel<<<L.n_disp_blocks, 256, kDispWarps * c->E * 4, s>>>(
@@ -631,8 +696,8 @@ int moe_dispatch_static(const moe_config_t* c, const int32_t* topk_idx,
   MOE_LAUNCHED(s, "dispatch_hist");
   prof_begin(s);
   disp_scan_kernel<<<1, 1024, c->E * 8, s>>>(bhist, bsent, L.n_disp_blocks, c->E, c->T,
-                                             c->n_shared, L.C, L.rows_max, counts, kept,
-                                             offsets, tile_expert, stats);
+                                             c->n_shared, L.C, L.rows_max, L.align, counts,
+                                             kept, offsets, tile_expert, stats);
   MOE_LAUNCHED(s, "dispatch_scan");
   prof_begin(s);
   disp_rank_kernel<<<L.n_disp_blocks, 256, kDispWarps * c->E * 4, s>>>(
@@ -684,25 +749,36 @@ int moe_expert_ffn(const moe_config_t* c, const void* x_perm, const int32_t* off
   if (use_tc(c)) {
     CUtensorMap mA, mB, mBs;
     const int64_t mt = row_tiles_estimate(c, L);
+    const bool pr = pair_rows(c);                 // CTA-pair row tiles
+    const int64_t units = pr ? L.tiles_max / 2 : L.tiles_max;
     // gate/up + SwiGLU: A = x_perm [rows, D]; B = w13 [E, 2F, D] K-major
-    const int bn1 = pick_bn(2 * F, mt, true, F);
+    const int bn1 = pick_bn(2 * F, mt, true, F, pr);
     MOE_TRY(make_map(&mA, x_perm, 1, L.rows_max, D, 128, false));
     MOE_TRY(make_map(&mB, w13, E, 2 * F, D, bn1 / 2, true));
     MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, bn1 / 2, true));
-    tc::Params p = rows_params(c, D, F / (bn1 / 2), tile_expert, stats);
+    tc::Params p = rows_params(c, D, F / (bn1 / 2), tile_expert, stats, pr);
     p.out = static_cast<__nv_bfloat16*>(a13); p.ld_out = 2 * F;
     p.out2 = static_cast<__nv_bfloat16*>(h); p.ld_out2 = F;
-    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU>(
-        bn1, "tc_gate_up_swiglu", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
-    // down: A = h [rows, F]; B = w_down [E, D, F] K-major
-    const int bn2 = pick_bn(D, mt, false, F);
+    if (pr)
+      MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, true>(
+          bn1, "tc_gate_up_swiglu", mA, mB, mBs, p, units * p.nN, 0, s)));
+    else
+      MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU>(
+          bn1, "tc_gate_up_swiglu", mA, mB, mBs, p, units * p.nN, 0, s)));
+    // down: A = h [rows, F]; B = w_down [E, D, F] K-major (a pair CTA loads
+    // half of the BN rows)
+    const int bn2 = pick_bn(D, mt, false, F, pr);
+    const uint32_t box2 = pr ? bn2 / 2 : bn2;
     MOE_TRY(make_map(&mA, h, 1, L.rows_max, F, 128, false));
-    MOE_TRY(make_map(&mB, w_down, E, D, F, bn2, true));
-    MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, bn2, true));
-    tc::Params q = rows_params(c, F, D / bn2, tile_expert, stats);
+    MOE_TRY(make_map(&mB, w_down, E, D, F, box2, true));
+    MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, box2, true));
+    tc::Params q = rows_params(c, F, D / bn2, tile_expert, stats, pr);
     q.out = static_cast<__nv_bfloat16*>(o); q.ld_out = D;
+    if (pr)
+      return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE, true>(
+          bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
     return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE>(
-        bn2, "tc_down", mA, mB, mBs, q, L.tiles_max * q.nN, 0, s);
+        bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
   }
   auto go = [&](auto tag) -> int {
     using TE = decltype(tag);
@@ -808,60 +884,81 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     CUtensorMap mA, mB, mBs;
     const int64_t mt = row_tiles_estimate(c, L);
     const int groups = E + c->n_shared;
+    const bool pr = pair_rows(c);                 // CTA-pair row tiles
+    const int64_t units = pr ? L.tiles_max / 2 : L.tiles_max;
     // 3. dgrad down + SwiGLU backward: dA13 = swiglu'(dO . w_down[e])
-    const int bn3 = pick_bn(F, mt, false, F);
+    const int bn3 = pick_bn(F, mt, false, F, pr);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 128, false));
     MOE_TRY(make_map(&mB, w_down, E, D, F, 64, true));                 // dims {F, D, E}
     MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, 64, true));
     {
-      tc::Params p = rows_params(c, D, F / bn3, tile_expert, stats);
+      tc::Params p = rows_params(c, D, F / bn3, tile_expert, stats, pr);
       p.out = static_cast<__nv_bfloat16*>(dA13); p.ld_out = 2 * F;
       p.aux = static_cast<const __nv_bfloat16*>(a13); p.ld_aux = 2 * F;
-      MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD>(
-          bn3, "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
+      if (pr)
+        MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD, true>(
+            bn3, "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, units * p.nN, 0, s)));
+      else
+        MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD>(
+            bn3, "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, units * p.nN, 0, s)));
     }
     MOE_TRY(fork_join(sd->ev[1], s, w1));
     MOE_TRY(fork_join(sd->ev[2], s, w2));
-    // 4. wgrad down: dW_down[e] = dO^T h over the expert's rows
-    const int bn4 = pick_bn(F, (int64_t)groups * (D / 128), false, F);
+    // 4. wgrad down: dW_down[e] = dO^T h over the expert's rows (CTA pairs
+    // split the 256-row output tiles)
+    const bool pw4 = (D % 256) == 0;
+    const int bn4 = pick_bn(F, (int64_t)groups * (D / 128), false, F, pw4);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 64, false));
     MOE_TRY(make_map(&mB, h, 1, L.rows_max, F, 64, false));
     {
       tc::Params p{};
       p.E = E; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
-      p.n_groups = groups; p.nMo = D / 128; p.nNo = F / bn4; p.No = F;
+      p.n_groups = groups; p.nMo = D / (pw4 ? 256 : 128); p.nNo = F / bn4; p.No = F;
       p.strideCE = (int64_t)D * F;
       p.out = static_cast<__nv_bfloat16*>(dw_down);
       p.out_shared = static_cast<__nv_bfloat16*>(dw_down_s);
       const int total = p.n_groups * p.nMo * p.nNo;
-      MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-          bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1)));
+      if (pw4)
+        MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, true>(
+            bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1)));
+      else
+        MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
+            bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1)));
     }
     // 5. dgrad gate/up: dX_perm = dA13 . w13[e]
-    const int bn5 = pick_bn(D, mt, false, F);
+    const int bn5 = pick_bn(D, mt, false, F, pr);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 128, false));
     MOE_TRY(make_map(&mB, w13, E, 2 * F, D, 64, true));                  // dims {D, 2F, E}
     MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, 64, true));
     {
-      tc::Params p = rows_params(c, 2 * F, D / bn5, tile_expert, stats);
+      tc::Params p = rows_params(c, 2 * F, D / bn5, tile_expert, stats, pr);
       p.out = static_cast<__nv_bfloat16*>(dXp); p.ld_out = D;
-      MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE>(
-          bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, L.tiles_max * p.nN, 0, s)));
+      if (pr)
+        MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE, true>(
+            bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s)));
+      else
+        MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE>(
+            bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s)));
     }
     // 6. wgrad gate/up: dW13[e] = dA13^T x_perm
-    const int bn6 = pick_bn(D, (int64_t)groups * (2 * F / 128), false, F);
+    const bool pw6 = ((2 * F) % 256) == 0;
+    const int bn6 = pick_bn(D, (int64_t)groups * (2 * F / 128), false, F, pw6);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 64, false));
     MOE_TRY(make_map(&mB, x_perm, 1, L.rows_max, D, 64, false));
     {
       tc::Params p{};
       p.E = E; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
-      p.n_groups = groups; p.nMo = 2 * F / 128; p.nNo = D / bn6; p.No = D;
+      p.n_groups = groups; p.nMo = 2 * F / (pw6 ? 256 : 128); p.nNo = D / bn6; p.No = D;
       p.strideCE = (int64_t)2 * F * D;
       p.out = static_cast<__nv_bfloat16*>(dw13);
       p.out_shared = static_cast<__nv_bfloat16*>(dw13_s);
       const int total = p.n_groups * p.nMo * p.nNo;
-      MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-          bn6, "tc_wgrad_gate_up", mA, mB, mB, p, total, total, w2)));
+      if (pw6)
+        MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, true>(
+            bn6, "tc_wgrad_gate_up", mA, mB, mB, p, total, total, w2)));
+      else
+        MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
+            bn6, "tc_wgrad_gate_up", mA, mB, mB, p, total, total, w2)));
     }
   } else {
     auto go = [&](auto tag) -> int {

@@ -40,14 +40,14 @@ def test_exports_every_declared_symbol(lib):
 def test_config_struct_layout_matches_header():
     # 12 int32 fields, then float, int32, 3 floats, int32 = 18 x 4 bytes
     assert ctypes.sizeof(C.MoeConfig) == 18 * 4
-    assert ctypes.sizeof(C.MoeSizes) == 32
+    assert ctypes.sizeof(C.MoeSizes) == 40
 
 
-def _rows_max(T, K, E, C_, n_shared):
+def _rows_max(T, K, E, C_, n_shared, align):
     kept_total = T * K if C_ is None else min(T * K, E * C_)
-    pad = 127 * min(E, kept_total)
-    r = -(-(kept_total + pad) // 128) * 128
-    return r + (-(-T // 128) * 128 if n_shared else 0)
+    pad = (align - 1) * min(E, kept_total)
+    r = -(-(kept_total + pad) // align) * align
+    return r + (-(-T // align) * align if n_shared else 0)
 
 
 @pytest.mark.parametrize("T,D,E,K,F,c,ns", [
@@ -62,7 +62,9 @@ def test_sizes(lib, T, D, E, K, F, c, ns):
     s = api.moe_get_sizes(cfg)
     Cap = None if c <= 0 else max(math.ceil(c * T * K / E), 0)
     assert s.capacity == (-1 if Cap is None else Cap)
-    assert s.rows_max == _rows_max(T, K, E, Cap, ns)
+    align = 256 if (K * T if Cap is None else min(K * T, E * Cap)) // E >= 1536 else 128
+    assert s.row_align == align
+    assert s.rows_max == _rows_max(T, K, E, Cap, ns, align)
     assert s.tiles_max * 128 == s.rows_max
     assert s.ws_bytes > 0
     if T == 256:

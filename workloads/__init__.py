@@ -102,6 +102,9 @@ REDUCED = {
     "olmoe": CONFIGS["olmoe"].replace(name="olmoe_small", T=700, D=256, F=256),
     "mix": CONFIGS["mix"].replace(name="mix_small", T=2000, D=512, F=640),
     "ds3": CONFIGS["ds3"].replace(name="ds3_small", T=300, D=256, F=128),
+    # enough rows per expert (>= 1536) that the expert GEMMs run on CTA pairs
+    "mm_pair": CONFIGS["mm_b"].replace(name="mm_pair_small", T=6500, D=256, F=512),
+    "mix_pair": CONFIGS["mix"].replace(name="mix_pair_small", T=7000, D=512, F=640),
 }
 
 
