@@ -286,29 +286,37 @@ def run_ours(args):
     moe_check_status()
 
 
-    prof = LaunchProfile(128)
-    graph = None
-    if not args.no_graph:
-        graph = torch.cuda.CUDAGraph()
+    def capture():
+        g = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(dev)
         side.wait_stream(stream)
         with torch.cuda.stream(side):
-            prof.reset()
-            with torch.cuda.graph(graph, stream=side):
+            with torch.cuda.graph(g, stream=side):
                 step()
         stream.wait_stream(side)
         torch.cuda.synchronize(dev)
+        return g
 
-    def replay():
-        if graph is not None:
-            graph.replay()
+    # `value` comes from a graph with no measurement nodes in it; the
+    # per-launch timing comes from a second graph captured with the
+    # library's begin/end events around every launch, replayed in its own
+    # timed loop below.
+    graph = None if args.no_graph else capture()
+    prof = LaunchProfile(128)
+    prof.reset()
+    graph_prof = None if args.no_graph else capture()
+
+    def replay(g):
+        if g is not None:
+            g.replay()
         else:
             prof.reset()
             step()
 
-    for _ in range(max(args.warmup, 3)):
-        flush.fill_(1)
-        replay()
+    for g in (graph, graph_prof):
+        for _ in range(max(args.warmup, 3)):
+            flush.fill_(1)
+            replay(g)
     torch.cuda.synchronize(dev)
     moe_check_status()
 
@@ -325,19 +333,23 @@ def run_ours(args):
         for i in range(args.steps):
             flush.fill_(i & 0xFF)          # L2 flush between timed steps (untimed)
             ev0[i].record(stream)
-            replay()
+            replay(graph)
             ev1[i].record(stream)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        # per-launch durations: the profiled graph, same flushes
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            replay(graph_prof)
             torch.cuda.synchronize(dev)
             if prof_ok:
                 try:
                     per_launch.append(prof.read())
                 except Exception:
                     prof_ok = False
-        barrier(world)
-        torch.cuda.synchronize(dev)
     step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
     ms = statistics.mean(step_ms)
-    timing_src = "events inside the timed graph replays"
+    timing_src = "begin/end events around each launch inside timed replays of the step graph"
     if not prof_ok or not per_launch or not per_launch[0]:
         # events recorded by graph nodes unreadable: time the same launches
         # eagerly (L2 flushed between steps) in a separate pass
@@ -420,8 +432,7 @@ def run_ours(args):
         }
         print(json.dumps(line), flush=True)
     prof.close()
-    if graph is not None:
-        del graph
+    graph = graph_prof = None
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
