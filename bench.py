@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--config", default="mm_b", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--timeline", action="store_true",
+                    help="print one profiled step's launch timeline to stderr")
     ap.add_argument("--cpu-sample-s", type=float, default=10.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--tokens", type=int, default=0,
@@ -116,10 +118,11 @@ def gemm_flops(cfg, kept_total):
     }
 
 
-def source_hash():
+def source_hash(files=None):
+    """Hash of the kernel sources (all of csrc/, or the named files)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "mixture_experts_routing_fp32_b200", "csrc")
-    for n in sorted(os.listdir(d)):
+    for n in sorted(files or os.listdir(d)):
         with open(os.path.join(d, n), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -136,15 +139,16 @@ def measured_peaks():
 
 
 def recorded_traffic(kernel, workload):
-    """DRAM bytes per launch from a committed ncu summary, if its kernel
-    source hash is the current one (else None)."""
+    """DRAM bytes per launch from a committed ncu summary, if the files that
+    define that kernel still hash to what they were when it was captured
+    (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         j = json.load(f)
     e = j.get(workload, {}).get(kernel)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash(e.get("files")):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -347,6 +351,14 @@ def run_ours(args):
                     per_launch.append(prof.read())
                 except Exception:
                     prof_ok = False
+    if args.timeline and rank == 0:
+        flush.fill_(7)
+        replay(graph_prof)
+        torch.cuda.synchronize(dev)
+        for (name, t, on_side), t0 in zip(prof.read(), prof.starts()):
+            print("%9.2f us  %8.2f us  %s%s" % (t0 * 1e3, t * 1e3, name,
+                                                 " [side]" if on_side else ""),
+                  file=sys.stderr)
     step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
     ms = statistics.mean(step_ms)
     timing_src = "begin/end events around each launch inside timed replays of the step graph"
@@ -411,7 +423,8 @@ def run_ours(args):
                 "B" if base.renorm else "A", base.aux_alpha),
                 "global_batch_tokens": base.T * world, "parallelism": "dp%d (replicas)" % world,
                 "l2": "flushed between timed steps (256 MiB write)",
-                "cuda_graph": graph is not None},
+                "cuda_graph": graph is not None,
+                "programmatic_dependent_launch": os.environ.get("MOE_PDL", "1") != "0"},
             "e2e": {"value": round(base.T * world / (e2e * 1e-3), 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e, 4),

@@ -299,6 +299,9 @@ int64_t moe_launch_count(int reset);
  *   moe_profile_read    after the caller synchronised: writes the elapsed
  *                       milliseconds of each recorded launch to ms (host
  *                       array) and returns how many were written
+ *   moe_profile_starts  like moe_profile_read, but writes the start of each
+ *                       recorded launch relative to the start of launch 0
+ *                       (a timeline of one step; gaps show launch overhead)
  *   moe_profile_name    kernel family name of recorded launch i
  *   moe_profile_side    1 if launch i ran on one of the library's side
  *                       streams (concurrently with other work, so its
@@ -308,6 +311,7 @@ int64_t moe_launch_count(int reset);
 int moe_profile_enable(int max_launches);
 int moe_profile_reset(void);
 int moe_profile_read(float* ms, int max);
+int moe_profile_starts(float* ms, int max);
 const char* moe_profile_name(int i);
 int moe_profile_side(int i);
 int moe_profile_disable(void);

@@ -25,7 +25,7 @@ c_int32, c_int64, c_float, c_void_p = ctypes.c_int32, ctypes.c_int64, ctypes.c_f
 EXPORTS = ("moe_get_sizes", "moe_router", "moe_dispatch", "moe_aux_loss",
            "moe_expert_ffn", "moe_combine", "moe_backward", "moe_check_status",
            "moe_status_string", "moe_last_cuda_error", "moe_launch_count",
-           "moe_profile_enable", "moe_profile_reset", "moe_profile_read",
+           "moe_profile_enable", "moe_profile_reset", "moe_profile_read", "moe_profile_starts",
            "moe_profile_name", "moe_profile_side", "moe_profile_disable",
            "moe_dispatch_static")
 
@@ -80,6 +80,7 @@ def lib():
         "moe_profile_enable": [ctypes.c_int],
         "moe_profile_reset": [],
         "moe_profile_read": [ctypes.POINTER(ctypes.c_float), ctypes.c_int],
+        "moe_profile_starts": [ctypes.POINTER(ctypes.c_float), ctypes.c_int],
         "moe_profile_name": [ctypes.c_int],
         "moe_profile_side": [ctypes.c_int],
         "moe_profile_disable": [],

@@ -148,6 +148,14 @@ class LaunchProfile:
         return [(lib().moe_profile_name(i).decode(), float(buf[i]),
                  lib().moe_profile_side(i) == 1) for i in range(n)]
 
+    def starts(self):
+        """Start of each launch since reset, in ms after the first one."""
+        buf = (ctypes.c_float * self.max)()
+        n = lib().moe_profile_starts(buf, self.max)
+        if n < 0:
+            check(n, "moe_profile_starts")
+        return [float(buf[i]) for i in range(n)]
+
     def close(self):
         lib().moe_profile_disable()
 

@@ -27,6 +27,7 @@ __global__ void __launch_bounds__(256)
 combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ slot_row,
                const float* __restrict__ topk_w, const int32_t* __restrict__ offsets,
                int n_shared, int Tn, int D, int K, int E, T* __restrict__ y) {
+  pdl_begin();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < Tn; t += (int64_t)gridDim.x * 8) {
     int64_t rows[kMaxK];
@@ -73,6 +74,7 @@ bwd_rows_kernel(const T* __restrict__ o, const T* __restrict__ dy,
                 const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ stats,
                 int K, int E, int Tn, int D, float* __restrict__ dg_slot,
                 T* __restrict__ dO) {
+  pdl_begin();
   const int n_rows = stats[2];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t r = (int64_t)blockIdx.x * 8 + warp; r < n_rows; r += (int64_t)gridDim.x * 8) {
@@ -132,6 +134,7 @@ struct RouterBwdArgs {
 template <int NV>
 __global__ void __launch_bounds__(256)
 router_bwd_kernel(RouterBwdArgs a) {
+  pdl_begin();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = a.E, K = a.K;
   float cnt_tot = 0.f;
@@ -254,6 +257,7 @@ template <typename TX, int BE, int BD, int TE, int TD>
 __global__ void __launch_bounds__(256)
 dwr_partial_kernel(const float* __restrict__ ds, const TX* __restrict__ x,
                    int Tn, int E, int D, int chunk, float* __restrict__ part) {
+  pdl_begin();
   static_assert((BE / TE) * (BD / TD) == 256, "thread tile");
   __shared__ __align__(16) float sds[32][BE + 4];
   __shared__ __align__(16) float sx[32][BD + 4];
@@ -312,6 +316,7 @@ dwr_partial_kernel(const float* __restrict__ ds, const TX* __restrict__ x,
 __global__ void __launch_bounds__(256)
 dwr_reduce_kernel(const float* __restrict__ part, int n_chunks, int64_t n,
                   float* __restrict__ dw_r) {
+  pdl_begin();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
     float s = 0.f;
@@ -328,6 +333,7 @@ dx_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
           const T* __restrict__ dXp, const int32_t* __restrict__ slot_row,
           const int32_t* __restrict__ offsets, int n_shared, int Tn, int D, int E,
           int K, T* __restrict__ dx) {
+  pdl_begin();
   constexpr int BT = 64, BD = 128, BK = 16;
   __shared__ __align__(16) float sds[BK][BT + 4];
   __shared__ __align__(16) float sw[BK][BD + 4];

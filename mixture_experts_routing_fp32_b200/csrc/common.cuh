@@ -16,7 +16,27 @@ __device__ __forceinline__ void set_dev_error(unsigned bits) {
 }
 
 constexpr int kRowTile = 128;       // rows per permuted tile (tensor-core M)
+constexpr int kMaxExperts = 512;    // routed experts per layer
 constexpr float kNearTie = 1e-5f;   // top-k margin reported as a near-tie
+
+// --- programmatic dependent launch ---------------------------------------------
+// Every kernel of the library may be launched with programmatic stream
+// serialisation: it can then be scheduled while the previous kernel of its
+// stream is still running.  pdl_wait() blocks until that kernel has finished
+// and its writes are visible, so it comes before the first global-memory
+// access; pdl_launch_dependents() lets the next kernel of the stream be
+// scheduled once every block of this one has started.  Without the launch
+// attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_begin() {
+  pdl_wait();
+  pdl_launch_dependents();
+}
 
 // --- element type helpers --------------------------------------------------
 template <typename T> struct Elem;

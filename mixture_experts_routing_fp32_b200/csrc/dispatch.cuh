@@ -18,6 +18,10 @@ namespace moe {
 constexpr int kDispWarps = 8;
 constexpr int kDispIters = 16;                                // 32-slot groups per warp
 constexpr int kDispChunk = kDispWarps * kDispIters * 32;      // slots per block
+// single-block dispatch (histogram, scan and rank in one kernel) up to
+// kSmallWarps * kDispIters * 32 slots
+constexpr int kSmallWarps = 32;
+constexpr int kSmallSlots = kSmallWarps * kDispIters * 32;
 
 __device__ __forceinline__ int slot_expert(const int32_t* idx, const uint8_t* mask,
                                            int64_t j, int E) {
@@ -30,33 +34,152 @@ __device__ __forceinline__ int slot_expert(const int32_t* idx, const uint8_t* ma
   return e;
 }
 
+// Expert ids of one warp's n_it groups of 32 consecutive slots starting at
+// slot j0 (-1 sentinel, -2 past the end), every load issued up front.
+__device__ __forceinline__ void warp_load_slots(const int32_t* idx, const uint8_t* mask,
+                                                int64_t n_slots, int E, int64_t j0, int n_it,
+                                                int (&ev)[kDispIters]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int it = 0; it < kDispIters; ++it) {
+    const int64_t j = j0 + it * 32 + lane;
+    ev[it] = (it < n_it && j < n_slots) ? slot_expert(idx, mask, j, E) : -2;
+  }
+}
+
+// Adds this warp's slots to row[e] (shared memory, one row per warp or per
+// block) with one update per distinct expert of each group; returns the
+// number of sentinel slots (same value in every lane).
+__device__ __forceinline__ int warp_count(const int (&ev)[kDispIters], int32_t* row,
+                                          bool shared_row) {
+  const unsigned lt = (1u << (threadIdx.x & 31)) - 1u;
+  int sent = 0;
+#pragma unroll
+  for (int it = 0; it < kDispIters; ++it) {
+    const int e = ev[it];
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (peers & lt) == 0) {
+      if (shared_row) atomicAdd(&row[e], __popc(peers));
+      else row[e] += __popc(peers);
+    }
+    sent += __popc(__ballot_sync(0xffffffffu, e == -1));
+    __syncwarp();
+  }
+  return sent;
+}
+
+// Stable rank of this warp's slots (row[e] holds the rank of the warp's
+// first slot of expert e, and is advanced), capacity drop, slot <-> row maps.
+__device__ __forceinline__ void warp_rank(const int (&ev)[kDispIters], int64_t j0,
+                                          int64_t n_slots, int64_t C, int64_t rows_max,
+                                          int32_t* row, const int32_t* seg_off,
+                                          int32_t* __restrict__ slot_row,
+                                          int32_t* __restrict__ row_slot) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int it = 0; it < kDispIters; ++it) {
+    const int64_t j = j0 + it * 32 + lane;
+    const int e = ev[it];
+    if (__all_sync(0xffffffffu, e == -2)) break;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    int32_t rank = 0;
+    if (e >= 0) rank = row[e] + __popc(peers & lt);
+    __syncwarp();
+    if (e >= 0 && (peers & lt) == 0) row[e] += __popc(peers);
+    __syncwarp();
+    if (e != -2) {
+      int32_t r = -1;
+      if (e >= 0 && (C < 0 || rank < C)) {
+        r = seg_off[e] + rank;
+        if (r < rows_max) row_slot[r] = (int32_t)j;
+        else { set_dev_error(MOE_DEVERR_ROWS); r = -1; }
+      }
+      slot_row[j] = r;
+    }
+  }
+}
+
+// Block-wide: from per-expert totals (tot[e], shared) derive counts, kept
+// (capacity), segment offsets aligned to `align` rows (seg[e], shared, and
+// offsets[] in global memory), the tile -> expert map and the stats words.
+// Called by every thread of the block; ends with a __syncthreads.
+__device__ void finish_layout(const int32_t* tot, int32_t* seg, int E, int T, int n_shared,
+                              int64_t C, int64_t rows_max, int align, int32_t sentinels,
+                              int32_t* __restrict__ counts, int32_t* __restrict__ kept,
+                              int32_t* __restrict__ offsets, int32_t* __restrict__ tile_expert,
+                              int32_t* __restrict__ stats) {
+  __shared__ unsigned long long drop_s;
+  __shared__ int32_t total_s;
+  if (threadIdx.x == 0) drop_s = 0;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int32_t run = tot[e];
+    counts[e] = run;
+    const int32_t k = (C >= 0 && run > C) ? (int32_t)C : run;
+    kept[e] = k;
+    if (run > k) atomicAdd(&drop_s, (unsigned long long)(run - k));
+    seg[e] = (k + align - 1) / align * align;
+  }
+  __syncthreads();
+  // exclusive scan of the padded sizes by warp 0 (E <= 512: 16 per lane)
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = (E + 31) / 32;
+    const int e0 = lane * per, e1 = min(E, e0 + per);
+    int64_t local = 0;
+    for (int e = e0; e < e1; ++e) local += seg[e];
+    int64_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int64_t run = incl - local;
+    for (int e = e0; e < e1; ++e) { const int64_t v = seg[e]; seg[e] = (int32_t)run; run += v; }
+    if (lane == 31) {
+      const int64_t routed = incl;
+      const int64_t shared_rows = n_shared ? ((int64_t)T + align - 1) / align * align : 0;
+      int64_t total = routed + shared_rows;
+      if (total > rows_max) { set_dev_error(MOE_DEVERR_ROWS); total = rows_max; }
+      offsets[E] = (int32_t)routed;
+      offsets[E + 1] = (int32_t)total;
+      stats[0] = (int32_t)drop_s;
+      stats[1] = sentinels;
+      stats[2] = (int32_t)total;
+      stats[3] = (int32_t)(total / kRowTile);
+      seg[E] = (int32_t)routed;
+      total_s = (int32_t)total;
+    }
+  }
+  __syncthreads();
+  const int64_t total = total_s;
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    const int64_t beg = seg[e];
+    const int64_t end = (e < E) ? seg[e + 1] : total;
+    if (e < E) offsets[e] = (int32_t)beg;
+    for (int64_t r = beg; r < end && r < total; r += kRowTile) tile_expert[r / kRowTile] = e;
+  }
+  __syncthreads();
+}
+
 // Pass 1: per-block histograms of valid slots and sentinel counts.
 __global__ void __launch_bounds__(256)
 disp_hist_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ mask,
                  int64_t n_slots, int E, int32_t* __restrict__ block_hist,
                  int32_t* __restrict__ block_sent) {
+  pdl_begin();
   extern __shared__ int32_t hist[];   // [E]
   __shared__ int32_t sent;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   if (threadIdx.x == 0) sent = 0;
   __syncthreads();
-  const int64_t j0 = (int64_t)blockIdx.x * kDispChunk;
-  const int64_t j1 = min(j0 + kDispChunk, n_slots);
-  // every load of this thread first (one memory latency, not one per slot)
-  constexpr int kPer = kDispChunk / 256;
-  int ev[kPer];
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int64_t j = j0 + threadIdx.x + (int64_t)k * 256;
-    ev[k] = (j < j1) ? slot_expert(idx, mask, j, E) : -2;
-  }
-  int my_sent = 0;
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    if (ev[k] >= 0) atomicAdd(&hist[ev[k]], 1);
-    else if (ev[k] == -1) ++my_sent;
-  }
-  if (my_sent) atomicAdd(&sent, my_sent);
+  const int warp = threadIdx.x >> 5;
+  const int64_t j0 = (int64_t)blockIdx.x * kDispChunk + (int64_t)warp * kDispIters * 32;
+  int ev[kDispIters];
+  warp_load_slots(idx, mask, n_slots, E, j0, kDispIters, ev);
+  const int my_sent = warp_count(ev, hist, true);
+  if ((threadIdx.x & 31) == 0 && my_sent) atomicAdd(&sent, my_sent);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     block_hist[(size_t)blockIdx.x * E + e] = hist[e];
@@ -64,18 +187,19 @@ disp_hist_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ ma
 }
 
 // Pass 2 (one block): per-expert totals, exclusive scan over blocks (block
-// bases), capacity, padded offsets (segments aligned to `align` rows, a
-// multiple of the 128-row tile), tile -> expert map, stats.
+// bases), then the layout (counts, kept, offsets, tile map, stats).
 __global__ void __launch_bounds__(1024)
 disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ block_sent,
                  int n_blocks, int E, int T, int n_shared, int64_t C,
                  int64_t rows_max, int align, int32_t* __restrict__ counts,
                  int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
                  int32_t* __restrict__ tile_expert, int32_t* __restrict__ stats) {
-  extern __shared__ int64_t sh[];     // [E] padded sizes -> offsets
-  __shared__ int64_t drop_total;
+  pdl_begin();
+  extern __shared__ int32_t sh[];     // tot[E], seg[E + 1]
+  int32_t* tot = sh;
+  int32_t* seg = sh + E;
   __shared__ int32_t sent_total;
-  if (threadIdx.x == 0) { drop_total = 0; sent_total = 0; }
+  if (threadIdx.x == 0) sent_total = 0;
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int32_t run = 0;
@@ -85,38 +209,14 @@ disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ b
       block_hist[(size_t)b * E + e] = run;   // becomes the block's base rank
       run += c;
     }
-    counts[e] = run;
-    const int32_t k = (C >= 0 && run > C) ? (int32_t)C : run;
-    kept[e] = k;
-    if (run > k) atomicAdd((unsigned long long*)&drop_total,
-                           (unsigned long long)(run - k));
-    sh[e] = ((int64_t)k + align - 1) / align * align;
+    tot[e] = run;
   }
-  for (int b = threadIdx.x; b < n_blocks; b += blockDim.x)
-    atomicAdd(&sent_total, block_sent[b]);
+  int32_t ls = 0;
+  for (int b = threadIdx.x; b < n_blocks; b += blockDim.x) ls += block_sent[b];
+  if (ls) atomicAdd(&sent_total, ls);
   __syncthreads();
-  if (threadIdx.x == 0) {   // E <= 512: a serial scan is negligible
-    int64_t run = 0;
-    for (int e = 0; e < E; ++e) { const int64_t v = sh[e]; sh[e] = run; run += v; }
-    const int64_t shared_rows = n_shared ? ((int64_t)T + align - 1) / align * align : 0;
-    int64_t total = run + shared_rows;
-    if (total > rows_max) { set_dev_error(MOE_DEVERR_ROWS); total = rows_max; }
-    offsets[E] = (int32_t)run;
-    offsets[E + 1] = (int32_t)total;
-    stats[0] = (int32_t)drop_total;
-    stats[1] = sent_total;
-    stats[2] = (int32_t)total;
-    stats[3] = (int32_t)(total / kRowTile);
-  }
-  __syncthreads();
-  const int64_t total = offsets[E + 1];
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
-    const int64_t beg = (e < E) ? sh[e] : offsets[E];
-    const int64_t end = (e + 1 < E) ? sh[e + 1] : (e < E ? offsets[E] : total);
-    if (e < E) offsets[e] = (int32_t)beg;
-    for (int64_t r = beg; r < end && r < total; r += kRowTile)
-      tile_expert[r / kRowTile] = e;
-  }
+  finish_layout(tot, seg, E, T, n_shared, C, rows_max, align, sent_total, counts, kept, offsets,
+                tile_expert, stats);
 }
 
 // Pass 3: stable rank of every slot inside its expert, capacity drop,
@@ -128,26 +228,17 @@ disp_rank_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ ma
                  const int32_t* __restrict__ block_base,
                  const int32_t* __restrict__ offsets,
                  int32_t* __restrict__ slot_row, int32_t* __restrict__ row_slot) {
-  extern __shared__ int32_t wh[];   // [kDispWarps][E] per-warp counters
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_begin();
+  extern __shared__ int32_t wh[];   // [kDispWarps][E] per-warp counters, then seg_off[E]
+  int32_t* seg_off = wh + kDispWarps * E;
+  const int warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kDispWarps * E; i += blockDim.x) wh[i] = 0;
-  __syncthreads();
-  const int64_t base = (int64_t)blockIdx.x * kDispChunk + (int64_t)warp * kDispIters * 32;
-  const unsigned lt = (1u << lane) - 1u;
-  // the warp's slots, loaded once up front
+  for (int e = threadIdx.x; e < E; e += blockDim.x) seg_off[e] = offsets[e];
+  const int64_t j0 = (int64_t)blockIdx.x * kDispChunk + (int64_t)warp * kDispIters * 32;
   int ev[kDispIters];
-#pragma unroll
-  for (int it = 0; it < kDispIters; ++it) {
-    const int64_t j = base + it * 32 + lane;
-    ev[it] = (j < n_slots) ? slot_expert(idx, mask, j, E) : -1;
-  }
-  // per-warp histogram
-#pragma unroll
-  for (int it = 0; it < kDispIters; ++it) {
-    const int e = ev[it];
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && (peers & lt) == 0) wh[warp * E + e] += __popc(peers);
-  }
+  warp_load_slots(idx, mask, n_slots, E, j0, kDispIters, ev);
+  __syncthreads();
+  warp_count(ev, wh + warp * E, false);
   __syncthreads();
   // exclusive scan over warps, seeded with the block's base rank
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -159,26 +250,48 @@ disp_rank_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ ma
     }
   }
   __syncthreads();
-#pragma unroll
-  for (int it = 0; it < kDispIters; ++it) {
-    const int64_t j = base + it * 32 + lane;
-    const int e = ev[it];
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    int32_t rank = 0;
-    if (e >= 0) rank = wh[warp * E + e] + __popc(peers & lt);
-    __syncwarp();
-    if (e >= 0 && (peers & lt) == 0) wh[warp * E + e] += __popc(peers);
-    __syncwarp();
-    if (j < n_slots) {
-      int32_t row = -1;
-      if (e >= 0 && (C < 0 || rank < C)) {
-        row = offsets[e] + rank;
-        if (row < rows_max) row_slot[row] = (int32_t)j;
-        else { set_dev_error(MOE_DEVERR_ROWS); row = -1; }
-      }
-      slot_row[j] = row;
+  warp_rank(ev, j0, n_slots, C, rows_max, wh + warp * E, seg_off, slot_row, row_slot);
+}
+
+// Passes 1-3 in one block for up to kSmallSlots slots: 32 warps each own
+// a run of consecutive slots, so scanning the per-warp counts in warp
+// order gives the same stable ranks as the multi-block passes.
+__global__ void __launch_bounds__(1024)
+disp_small_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ mask,
+                  int64_t n_slots, int E, int T, int n_shared, int64_t C, int64_t rows_max,
+                  int align, int32_t* __restrict__ counts, int32_t* __restrict__ kept,
+                  int32_t* __restrict__ offsets, int32_t* __restrict__ tile_expert,
+                  int32_t* __restrict__ stats, int32_t* __restrict__ slot_row,
+                  int32_t* __restrict__ row_slot) {
+  pdl_begin();
+  extern __shared__ int32_t wh[];   // [kSmallWarps][E] counters, tot[E], seg[E + 1]
+  int32_t* tot = wh + kSmallWarps * E;
+  int32_t* seg = tot + E;
+  __shared__ int32_t sent_total;
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) wh[i] = 0;
+  if (threadIdx.x == 0) sent_total = 0;
+  const int n_it = (int)((n_slots + kSmallWarps * 32 - 1) / (kSmallWarps * 32));
+  const int64_t j0 = (int64_t)warp * n_it * 32;
+  int ev[kDispIters];
+  warp_load_slots(idx, mask, n_slots, E, j0, n_it, ev);
+  __syncthreads();
+  const int sent = warp_count(ev, wh + warp * E, false);
+  if ((threadIdx.x & 31) == 0 && sent) atomicAdd(&sent_total, sent);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t run = 0;
+    for (int w = 0; w < kSmallWarps; ++w) {
+      const int32_t c = wh[w * E + e];
+      wh[w * E + e] = run;
+      run += c;
     }
+    tot[e] = run;
   }
+  __syncthreads();
+  finish_layout(tot, seg, E, T, n_shared, C, rows_max, align, sent_total, counts, kept, offsets,
+                tile_expert, stats);
+  warp_rank(ev, j0, n_slots, C, rows_max, wh + warp * E, seg, slot_row, row_slot);
 }
 
 // Pass 4: gather x rows into expert order; zero padding rows; shared rows.
@@ -188,6 +301,7 @@ disp_gather_kernel(const TX* __restrict__ x, int D, int K, int E, int T,
                    const int32_t* __restrict__ offsets, const int32_t* __restrict__ kept,
                    const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ stats,
                    int32_t* __restrict__ row_slot, TX* __restrict__ x_perm) {
+  pdl_begin();
   const int n_rows = stats[2];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t r = (int64_t)blockIdx.x * 8 + warp; r < n_rows; r += (int64_t)gridDim.x * 8) {

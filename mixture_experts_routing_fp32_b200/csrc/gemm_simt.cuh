@@ -37,6 +37,7 @@ struct SimtGemm {
 template <typename TE>
 __global__ void __launch_bounds__(256)
 simt_rows_kernel(SimtGemm g) {
+  pdl_begin();
   __shared__ __align__(16) float As[16][64 + 4];
   __shared__ __align__(16) float Bs[16][64 + 4];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -83,6 +84,7 @@ simt_rows_kernel(SimtGemm g) {
 template <typename TE>
 __global__ void __launch_bounds__(256)
 simt_wgrad_kernel(SimtGemm g) {
+  pdl_begin();
   __shared__ __align__(16) float As[16][64 + 4];
   __shared__ __align__(16) float Bs[16][64 + 4];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -133,6 +135,7 @@ template <typename TE>
 __global__ void __launch_bounds__(256)
 swiglu_fwd_kernel(const TE* __restrict__ a13, TE* __restrict__ h,
                   const int32_t* __restrict__ stats, int F) {
+  pdl_begin();
   const int64_t n = (int64_t)stats[2] * F;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -147,6 +150,7 @@ template <typename TE>
 __global__ void __launch_bounds__(256)
 swiglu_bwd_kernel(const TE* __restrict__ dh, const TE* __restrict__ a13,
                   TE* __restrict__ da13, const int32_t* __restrict__ stats, int F) {
+  pdl_begin();
   const int64_t n = (int64_t)stats[2] * F;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {

@@ -298,6 +298,76 @@ __device__ __forceinline__ void store32_bf16(__nv_bfloat16* p, const float (&v)[
                  : "memory");
   }
 }
+// ---- warp-staged epilogue I/O ------------------------------------------------
+// An epilogue lane owns one accumulator row, so writing its 32 columns
+// directly would make every warp-wide 16-byte access touch 32 different
+// rows.  Instead each warp passes a 32-row x 32-column bf16 block through a
+// private shared-memory tile (row stride 80 bytes: the 16-byte accesses of
+// both the row-wise and the segment-wise pass fall in distinct banks), and
+// global memory sees 64-byte row segments, 8 rows per instruction.
+constexpr int kStgRow = 80;
+constexpr int kStgBytes = 32 * kStgRow;
+
+__device__ __forceinline__ void sts128(uint32_t a, const uint4& u) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(u.x), "r"(u.y), "r"(u.z),
+               "r"(u.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 u;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
+               : "r"(a)
+               : "memory");
+  return u;
+}
+__device__ __forceinline__ uint4 pack8_bf16(const float* v) {
+  uint4 u;
+  __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h2[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  return u;
+}
+
+// Stores this lane's 32 values (its row of the block) as bf16; w0 addresses
+// the block's first row and column, ld is the row stride in elements.
+__device__ __forceinline__ void staged_store32(uint32_t stg, const float (&v)[32],
+                                               __nv_bfloat16* w0, int64_t ld, uint64_t pol) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) sts128(stg + lane * kStgRow + j * 16, pack8_bf16(v + 8 * j));
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i * 8 + (lane >> 2), pc = lane & 3;
+    const uint4 u = lds128(stg + r * kStgRow + pc * 16);
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(
+                     w0 + r * ld + pc * 8),
+                 "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w), "l"(pol)
+                 : "memory");
+  }
+  __syncwarp();
+}
+
+// Coalesced load of a 32 x 32 bf16 block (w0: first row and column): piece
+// i of this lane is row 8 i + lane / 4, columns 8 (lane % 4) .. + 7.
+__device__ __forceinline__ void block_load32(const __nv_bfloat16* w0, int64_t ld, uint4 (&u)[4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    u[i] = *reinterpret_cast<const uint4*>(w0 + (i * 8 + (lane >> 2)) * ld + (lane & 3) * 8);
+}
+// The pieces of block_load32 -> this lane's row (32 floats).
+__device__ __forceinline__ void staged_rows32(uint32_t stg, const uint4 (&u)[4], float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sts128(stg + (i * 8 + (lane >> 2)) * kStgRow + (lane & 3) * 16, u[i]);
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 4; ++j) bf16x8_to_f(lds128(stg + lane * kStgRow + j * 16), v + 8 * j);
+  __syncwarp();
+}
+
 __device__ __forceinline__ void load32_bf16(const __nv_bfloat16* p, float (&v)[32]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) load8(p + 8 * q, v + 8 * q);
@@ -315,8 +385,9 @@ struct Tile {
 };
 
 // M rows per tile: 128, or 256 for a CTA pair (this CTA holds 128 of them).
+// n_mt: row tiles in use (ROWS; read once per kernel from stats).
 template <int MODE, int EPI, int BN, bool PAIR>
-__device__ __forceinline__ Tile decode(int t, const Params& p, int rank) {
+__device__ __forceinline__ Tile decode(int t, const Params& p, int rank, int n_mt) {
   constexpr int MU = PAIR ? 2 * BM : BM;
   Tile d;
   if (MODE == MODE_ROWS) {
@@ -326,7 +397,6 @@ __device__ __forceinline__ Tile decode(int t, const Params& p, int rank) {
     // slices, instead of streaming an expert's weights once per row tile.
     // With a CTA pair a row tile is 256 rows: two 128-row tiles of one
     // expert (expert segments are then 256-row aligned).
-    const int n_mt = p.stats[3] / (PAIR ? 2 : 1);
     const int group = t / (p.group_m * p.nN);
     const int first = group * p.group_m;
     const int gm = min(p.group_m, n_mt - first);
@@ -359,7 +429,10 @@ struct Smem {
   static constexpr int kB = BNC * BK * 2;
   static constexpr int kStage = kA + kB;
   static constexpr int kBars = (2 * STAGES + 5) * 8;
-  static constexpr int kBytes = 1024 + STAGES * kStage + kBars + 16;
+  // epilogue staging tiles (one per epilogue warp), 128-byte aligned
+  static constexpr int kEpiOff = (STAGES * kStage + kBars + 16 + 127) / 128 * 128;
+  static constexpr int kBytes = 1024 + kEpiOff + kEpiWarps * kStgBytes;
+  static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
 template <int BN, int STAGES, int MODE, bool A_MN, bool B_MN, int EPI, bool PAIR>
@@ -425,10 +498,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   if constexpr (PAIR) cluster_sync();   // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the set-up above touched only this CTA's shared and tensor memory
+  pdl_begin();
 
-  int total;
-  if (MODE == MODE_ROWS) total = (p.stats[3] / (PAIR ? 2 : 1)) * p.nN;
-  else total = total_hint;
+  // Each role decodes tile t + n_units while it works on tile t, so the
+  // global loads a decode needs (tile -> expert map, group offsets) never
+  // stall a tile boundary.
+  const int n_mt = (MODE == MODE_ROWS) ? p.stats[3] / (PAIR ? 2 : 1) : 0;
+  const int total = (MODE == MODE_ROWS) ? n_mt * p.nN : total_hint;
+  auto decode_at = [&](int t) {
+    return t < total ? decode<MODE, EPI, BN, PAIR>(t, p, rank, n_mt) : Tile{0, 0, 0, 0, 0};
+  };
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs of a pair) ----------------
@@ -440,8 +520,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
       bool ok = true;
+      Tile nxt = decode_at(unit);
       for (int t = unit; t < total && ok; t += n_units) {
-        const Tile d = decode<MODE, EPI, BN, PAIR>(t, p, rank);
+        const Tile d = nxt;
+        nxt = decode_at(t + n_units);
         const CUtensorMap* mb = (MODE == MODE_ROWS && d.e >= p.E) ? &mapBs : &mapB;
         const int eb = (MODE == MODE_ROWS && d.e >= p.E) ? 0 : d.e;
         for (int kb = 0; kb < d.nk; ++kb) {
@@ -512,8 +594,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      Tile nxt = decode_at(unit);
       for (int t = unit; t < total && ok; t += n_units) {
-        const Tile d = decode<MODE, EPI, BN, PAIR>(t, p, rank);
+        const Tile d = nxt;
+        nxt = decode_at(t + n_units);
         if (d.nk == 0) continue;
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
@@ -557,26 +641,29 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     constexpr int HC = BN / 2;           // columns per warp (plain epilogues)
     constexpr int HJ = BN / 4;           // gate (= up) columns per warp (SwiGLU)
     const uint64_t pol_out = policy_evict_first();
+    const uint32_t stg = base + S::kEpiOff + (warp - 2) * kStgBytes;   // staging tile
     int acc = 0;
     uint32_t acc_phase = 0;
+    Tile nxt = decode_at(unit);
     for (int t = unit; t < total; t += n_units) {
-      const Tile d = decode<MODE, EPI, BN, PAIR>(t, p, rank);
+      const Tile d = nxt;
+      nxt = decode_at(t + n_units);
       if (MODE == MODE_WGRAD && d.nk == 0) {
         __nv_bfloat16* og = d.e < p.E ? p.out + (int64_t)d.e * p.strideCE : p.out_shared;
         __nv_bfloat16* dst = og + (int64_t)(d.m0 + rloc) * p.No + d.n0 + hh * HC;
         for (int c = 0; c < HC; c += 8) zero8(dst + c);
         continue;
       }
-      const int64_t row = d.m0 + rloc;
-      // SwiGLU backward: this warp's a and b values are fetched before the
-      // accumulator wait so their latency overlaps the tile's main loop.
-      uint4 pa[EPI == EPI_SWIGLU_BWD ? HC / 8 : 1], pb[EPI == EPI_SWIGLU_BWD ? HC / 8 : 1];
+      const int64_t row0 = d.m0 + q * 32;   // this warp's first row
+      // SwiGLU backward: this warp's a and b blocks are fetched (coalesced)
+      // before the accumulator wait so their latency overlaps the main loop.
+      uint4 pa[EPI == EPI_SWIGLU_BWD ? HC / 32 : 1][4], pb[EPI == EPI_SWIGLU_BWD ? HC / 32 : 1][4];
       if constexpr (EPI == EPI_SWIGLU_BWD) {
-        const __nv_bfloat16* a13 = p.aux + row * p.ld_aux + d.n0 + hh * HC;
+        const __nv_bfloat16* a13 = p.aux + row0 * p.ld_aux + d.n0 + hh * HC;
 #pragma unroll
-        for (int i = 0; i < HC / 8; ++i) {
-          pa[i] = *reinterpret_cast<const uint4*>(a13 + 8 * i);
-          pb[i] = *reinterpret_cast<const uint4*>(a13 + p.F + 8 * i);
+        for (int c = 0; c < HC / 32; ++c) {
+          block_load32(a13 + 32 * c, p.ld_aux, pa[c]);
+          block_load32(a13 + p.F + 32 * c, p.ld_aux, pb[c]);
         }
       }
       bool ok = (lane == 0) ? mbar_wait(accf_bar(acc), acc_phase, abort_flag) : true;
@@ -585,12 +672,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * BN;
       if constexpr (EPI == EPI_STORE || EPI == EPI_WGRAD) {
-        __nv_bfloat16* dst;
+        __nv_bfloat16* w0;
+        int64_t ld;
         if (EPI == EPI_STORE) {
-          dst = p.out + row * p.ld_out + d.n0 + hh * HC;
+          w0 = p.out + row0 * p.ld_out + d.n0 + hh * HC;
+          ld = p.ld_out;
         } else {
           __nv_bfloat16* og = d.e < p.E ? p.out + (int64_t)d.e * p.strideCE : p.out_shared;
-          dst = og + row * p.No + d.n0 + hh * HC;
+          w0 = og + row0 * p.No + d.n0 + hh * HC;
+          ld = p.No;
         }
 #pragma unroll
         for (int c = 0; c < HC; c += 32) {
@@ -599,11 +689,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_ld32(tbase + hh * HC + c, r);
           tmem_wait();
           u2f32(r, v);
-          store32_bf16(dst + c, v, pol_out);
+          staged_store32(stg, v, w0 + c, ld, pol_out);
         }
       } else if constexpr (EPI == EPI_SWIGLU) {
-        __nv_bfloat16* a13 = p.out + row * p.ld_out + d.n0 + hh * HJ;
-        __nv_bfloat16* hr = p.out2 + row * p.ld_out2 + d.n0 + hh * HJ;
+        __nv_bfloat16* a13 = p.out + row0 * p.ld_out + d.n0 + hh * HJ;
+        __nv_bfloat16* hr = p.out2 + row0 * p.ld_out2 + d.n0 + hh * HJ;
 #pragma unroll
         for (int c = 0; c < HJ; c += 32) {
           uint32_t rg[32], ru[32];
@@ -613,24 +703,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_wait();
           u2f32(rg, ga);
           u2f32(ru, ub);
-          store32_bf16(a13 + c, ga, pol_out);
-          store32_bf16(a13 + p.F + c, ub, pol_out);
+          staged_store32(stg, ga, a13 + c, p.ld_out, pol_out);
+          staged_store32(stg, ub, a13 + p.F + c, p.ld_out, pol_out);
 #pragma unroll
           for (int i = 0; i < 32; ++i) ga[i] = ga[i] * fast_sigmoid(ga[i]) * ub[i];
-          store32_bf16(hr + c, ga, pol_out);
+          staged_store32(stg, ga, hr + c, p.ld_out2, pol_out);
         }
       } else {  // EPI_SWIGLU_BWD
-        __nv_bfloat16* da13 = p.out + row * p.ld_out + d.n0 + hh * HC;
+        __nv_bfloat16* da13 = p.out + row0 * p.ld_out + d.n0 + hh * HC;
 #pragma unroll
         for (int c = 0; c < HC; c += 32) {
           uint32_t r[32];
           float dh[32], av[32], bv[32];
           tmem_ld32(tbase + hh * HC + c, r);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            bf16x8_to_f(pa[c / 8 + i], av + 8 * i);
-            bf16x8_to_f(pb[c / 8 + i], bv + 8 * i);
-          }
+          staged_rows32(stg, pa[c / 32], av);
+          staged_rows32(stg, pb[c / 32], bv);
           tmem_wait();
           u2f32(r, dh);
 #pragma unroll
@@ -640,8 +727,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
             bv[i] = dh[i] * av[i] * sg;
             av[i] = da;
           }
-          store32_bf16(da13 + c, av, pol_out);
-          store32_bf16(da13 + p.F + c, bv, pol_out);
+          staged_store32(stg, av, da13 + c, p.ld_out, pol_out);
+          staged_store32(stg, bv, da13 + p.F + c, p.ld_out, pol_out);
         }
       }
       tc_fence_before();

@@ -6,8 +6,10 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "router.cuh"
@@ -96,7 +98,7 @@ size_t act_bytes(const moe_config_t* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
 int validate(const moe_config_t* c) {
   if (c == nullptr) return MOE_ERR_ARG;
   if (c->T < 1 || c->D < 8 || (c->D % 8) || c->F < 8 || (c->F % 8)) return MOE_ERR_ARG;
-  if (c->E < 1 || c->E > 512) return MOE_ERR_ARG;
+  if (c->E < 1 || c->E > kMaxExperts) return MOE_ERR_ARG;
   if (c->K < 1 || c->K > c->E || c->K > kMaxK) return MOE_ERR_ARG;
   if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_ARG;
   if (c->dtype != MOE_FP32 && c->dtype != MOE_BF16) return MOE_ERR_ARG;
@@ -238,6 +240,34 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t n3, int64_t rows, int64_t 
   return MOE_OK;
 }
 
+// Programmatic dependent launch on by default (MOE_PDL=0 turns it off):
+// every kernel waits for its stream predecessor with griddepcontrol.wait
+// before its first global access, so the launch attribute only lets the
+// next kernel be scheduled, and its set-up run, while this one drains.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("MOE_PDL");
+    return !(v != nullptr && v[0] == '0');
+  }();
+  return on;
+}
+
+template <typename... KP, typename... A>
+cudaError_t launch_k(void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     A&&... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&lc, kern, std::forward<A>(args)...);
+}
+
 template <int BN, int ST, int MODE, bool AMN, bool BMN, int EPI, bool PAIR>
 int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
               const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
@@ -249,11 +279,13 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
     // as many CTA pairs as can be resident at once (one per two SMs of a GPC)
     static int max_pairs = 0;
     cudaLaunchConfig_t lc = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     lc.blockDim = dim3(tc::kThreads);
     lc.dynamicSmemBytes = S::kBytes;
     lc.stream = s;
@@ -268,6 +300,7 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
     const int pairs = (int)std::min<int64_t>(max_pairs, total_max);
     if (pairs <= 0) return MOE_OK;
     lc.gridDim = dim3(2 * pairs);
+    lc.numAttrs = pdl_enabled() ? 2 : 1;
     prof_begin(s);
     MOE_CK(cudaLaunchKernelEx(&lc, k, a, b, bs, p, total_hint));
     MOE_LAUNCHED(s, name);
@@ -275,7 +308,7 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
     const int grid = (int)std::min<int64_t>(num_sms(), total_max);
     if (grid <= 0) return MOE_OK;
     prof_begin(s);
-    k<<<grid, tc::kThreads, S::kBytes, s>>>(a, b, bs, p, total_hint);
+    MOE_CK((launch_k(k, grid, tc::kThreads, S::kBytes, s, a, b, bs, p, total_hint)));
     MOE_LAUNCHED(s, name);
   }
   return MOE_OK;
@@ -367,7 +400,7 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
     auto go = [&](auto kern) -> int {
       MOE_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fused_smem));
       prof_begin(s);
-      kern<<<grid, 256, fused_smem, s>>>(x, w_r, off, c->D, a);
+      MOE_CK((launch_k(kern, grid, 256, fused_smem, s, x, w_r, off, c->D, a)));
       MOE_LAUNCHED(s, "router_fused");
       return MOE_OK;
     };
@@ -378,16 +411,16 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
   }
   dim3 g1((unsigned)ceil_div(c->T, 64), (unsigned)ceil_div(c->E, 64));
   prof_begin(s);
-  router_logits_kernel<TX><<<g1, 256, 0, s>>>(x, w_r, off, logits, c->T, c->D, c->E);
+  MOE_CK((launch_k(router_logits_kernel<TX>, g1, 256, 0, s, x, w_r, off, logits, c->T, c->D, c->E)));
   MOE_LAUNCHED(s, "router_logits");
   const size_t sm = 8 * (size_t)c->E * 4;
   const int grid = grid_for(c->T);
   prof_begin(s);
-  if (c->E <= 32) router_route_kernel<1><<<grid, 256, sm, s>>>(logits, a);
-  else if (c->E <= 64) router_route_kernel<2><<<grid, 256, sm, s>>>(logits, a);
-  else if (c->E <= 128) router_route_kernel<4><<<grid, 256, sm, s>>>(logits, a);
-  else if (c->E <= 256) router_route_kernel<8><<<grid, 256, sm, s>>>(logits, a);
-  else router_route_kernel<16><<<grid, 256, sm, s>>>(logits, a);
+  if (c->E <= 32) MOE_CK((launch_k(router_route_kernel<1>, grid, 256, sm, s, logits, a)));
+  else if (c->E <= 64) MOE_CK((launch_k(router_route_kernel<2>, grid, 256, sm, s, logits, a)));
+  else if (c->E <= 128) MOE_CK((launch_k(router_route_kernel<4>, grid, 256, sm, s, logits, a)));
+  else if (c->E <= 256) MOE_CK((launch_k(router_route_kernel<8>, grid, 256, sm, s, logits, a)));
+  else MOE_CK((launch_k(router_route_kernel<16>, grid, 256, sm, s, logits, a)));
   MOE_LAUNCHED(s, "router_route");
   return MOE_OK;
 }
@@ -398,6 +431,7 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
 __global__ void __launch_bounds__(256)
 aux_partial_kernel(const float* __restrict__ probs, const float* __restrict__ lse, int T, int E,
                    float* __restrict__ part) {
+  pdl_begin();
   // chunk c of kAuxChunk tokens: column sums of probs and the sum of lse^2,
   // each reduced in a fixed order (deterministic)
   __shared__ float red[256];
@@ -434,6 +468,7 @@ aux_partial_kernel(const float* __restrict__ probs, const float* __restrict__ ls
 __global__ void __launch_bounds__(512)
 aux_final_kernel(const float* __restrict__ part, const int32_t* __restrict__ counts, int n_chunks,
                  int T, int E, float alpha, float lambda, float* __restrict__ losses) {
+  pdl_begin();
   __shared__ float red[512];
   __shared__ float cnt_tot_s;
   float cnt = 0.f;
@@ -483,7 +518,7 @@ int simt_rows(const moe_config_t* c, const Layout& L, const void* A, int64_t lda
   g.tile_expert = tile_expert; g.stats = stats; g.E = c->E;
   dim3 grid((unsigned)(L.tiles_max * 2), (unsigned)ceil_div(N, 64));
   prof_begin(s);
-  simt_rows_kernel<TE><<<grid, 256, 0, s>>>(g);
+  MOE_CK((launch_k(simt_rows_kernel<TE>, grid, 256, 0, s, g)));
   MOE_LAUNCHED(s, "simt_rows_gemm");
   return MOE_OK;
 }
@@ -498,7 +533,7 @@ int simt_wgrad(const moe_config_t* c, const void* A, int64_t lda, const void* B,
   g.strideCE = (int64_t)Mo * No;
   dim3 grid((unsigned)ceil_div(No, 64), (unsigned)ceil_div(Mo, 64), (unsigned)(c->E + c->n_shared));
   prof_begin(s);
-  simt_wgrad_kernel<TE><<<grid, 256, 0, s>>>(g);
+  MOE_CK((launch_k(simt_wgrad_kernel<TE>, grid, 256, 0, s, g)));
   MOE_LAUNCHED(s, "simt_wgrad_gemm");
   return MOE_OK;
 }
@@ -510,7 +545,7 @@ int simt_wgrad(const moe_config_t* c, const void* A, int64_t lda, const void* B,
 constexpr int kMaxSideDevices = 64;
 struct Side {
   cudaStream_t st[3];
-  cudaEvent_t ev[6];
+  cudaEvent_t ev[8];
   bool ok = false;
 };
 thread_local Side g_side[kMaxSideDevices];
@@ -561,6 +596,53 @@ tc::Params rows_params(const moe_config_t* c, int Kd, int nN, const int32_t* til
 
 }  // namespace
 
+// Dispatch passes: one block (histogram, scan and rank together) when the
+// slots fit it, else the three multi-block passes through the per-block
+// histograms in bhist/bsent; then the gather of x rows.
+int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_idx,
+                  const uint8_t* sentinel_mask, const void* x, int32_t* counts, int32_t* kept,
+                  int32_t* offsets, int32_t* slot_row, int32_t* row_slot, int32_t* tile_expert,
+                  int32_t* stats, void* x_perm, int32_t* bhist, int32_t* bsent, cudaStream_t s) {
+  const int E = c->E;
+  if (L.n_slots <= kSmallSlots) {
+    const size_t smem = ((size_t)kSmallWarps * E + 2 * E + 1) * sizeof(int32_t);
+    MOE_CK(cudaFuncSetAttribute(disp_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem));
+    prof_begin(s);
+    MOE_CK((launch_k(disp_small_kernel, 1, kSmallWarps * 32, smem, s, topk_idx, sentinel_mask,
+                     L.n_slots, E, c->T, c->n_shared, L.C, L.rows_max, L.align, counts, kept,
+                     offsets, tile_expert, stats, slot_row, row_slot)));
+    MOE_LAUNCHED(s, "dispatch_small");
+  } else {
+    prof_begin(s);
+    MOE_CK((launch_k(disp_hist_kernel, L.n_disp_blocks, 256, E * sizeof(int32_t), s, topk_idx,
+                     sentinel_mask, L.n_slots, E, bhist, bsent)));
+    MOE_LAUNCHED(s, "dispatch_hist");
+    prof_begin(s);
+    MOE_CK((launch_k(disp_scan_kernel, 1, 1024, (2 * E + 1) * sizeof(int32_t), s, bhist, bsent,
+                     L.n_disp_blocks, E, c->T, c->n_shared, L.C, L.rows_max, L.align, counts,
+                     kept, offsets, tile_expert, stats)));
+    MOE_LAUNCHED(s, "dispatch_scan");
+    prof_begin(s);
+    MOE_CK((launch_k(disp_rank_kernel, L.n_disp_blocks, 256,
+                     (size_t)(kDispWarps + 1) * E * sizeof(int32_t), s, topk_idx, sentinel_mask,
+                     L.n_slots, E, L.C, L.rows_max, bhist, offsets, slot_row, row_slot)));
+    MOE_LAUNCHED(s, "dispatch_rank");
+  }
+  const int grid = grid_for(L.rows_max);
+  prof_begin(s);
+  if (c->dtype == MOE_BF16)
+    MOE_CK((launch_k(disp_gather_kernel<__nv_bfloat16>, grid, 256, 0, s,
+                     static_cast<const __nv_bfloat16*>(x), c->D, c->K, E, c->T, offsets, kept,
+                     tile_expert, stats, row_slot, static_cast<__nv_bfloat16*>(x_perm))));
+  else
+    MOE_CK((launch_k(disp_gather_kernel<float>, grid, 256, 0, s, static_cast<const float*>(x),
+                     c->D, c->K, E, c->T, offsets, kept, tile_expert, stats, row_slot,
+                     static_cast<float*>(x_perm))));
+  MOE_LAUNCHED(s, "dispatch_gather");
+  return MOE_OK;
+}
+
 // ===========================================================================
 // extern "C" entry points
 // ===========================================================================
@@ -601,34 +683,9 @@ int moe_dispatch(const moe_config_t* c, const int32_t* topk_idx, const uint8_t* 
       !tile_expert || !stats || !x_perm || !ws)
     return MOE_ERR_ARG;
   const Layout L = layout_of(c);
-  int32_t* bhist = wsp<int32_t>(ws, L.off_bhist);
-  int32_t* bsent = wsp<int32_t>(ws, L.off_bsent);
-  prof_begin(s);
-  disp_hist_kernel<<<L.n_disp_blocks, 256, c->E * 4, s>>>(topk_idx, sentinel_mask, L.n_slots,
-                                                          c->E, bhist, bsent);
-  MOE_LAUNCHED(s, "dispatch_hist");
-  prof_begin(s);
-  disp_scan_kernel<<<1, 1024, c->E * 8, s>>>(bhist, bsent, L.n_disp_blocks, c->E, c->T,
-                                             c->n_shared, L.C, L.rows_max, L.align, counts,
-                                             kept, offsets, tile_expert, stats);
-  MOE_LAUNCHED(s, "dispatch_scan");
-  prof_begin(s);
-  disp_rank_kernel<<<L.n_disp_blocks, 256, kDispWarps * c->E * 4, s>>>(
-      topk_idx, sentinel_mask, L.n_slots, c->E, L.C, L.rows_max, bhist, offsets, slot_row,
-      row_slot);
-  MOE_LAUNCHED(s, "dispatch_rank");
-  const int grid = grid_for(L.rows_max);
-  prof_begin(s);
-  if (c->dtype == MOE_BF16)
-    disp_gather_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), c->D, c->K, c->E, c->T, offsets, kept, tile_expert,
-        stats, row_slot, static_cast<__nv_bfloat16*>(x_perm));
-  else
-    disp_gather_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), c->D, c->K,
-                                                    c->E, c->T, offsets, kept, tile_expert,
-                                                    stats, row_slot, static_cast<float*>(x_perm));
-  MOE_LAUNCHED(s, "dispatch_gather");
-  return MOE_OK;
+  return dispatch_impl(c, L, topk_idx, sentinel_mask, x, counts, kept, offsets, slot_row,
+                       row_slot, tile_expert, stats, x_perm, wsp<int32_t>(ws, L.off_bhist),
+                       wsp<int32_t>(ws, L.off_bsent), s);
 }
 
 }  // extern "C"
@@ -688,34 +745,9 @@ int moe_dispatch_static(const moe_config_t* c, const int32_t* topk_idx,
   if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_ARG;
   int32_t* base = nullptr;
   MOE_TRY(static_scratch_ptr(&base));
-  int32_t* bhist = base;
-  int32_t* bsent = base + (size_t)L.n_disp_blocks * c->E;
-  prof_begin(s);
-  disp_hist_kernel<<<L.n_disp_blocks, 256, c->E * 4, s>>>(topk_idx, sentinel_mask, L.n_slots,
-                                                          c->E, bhist, bsent);
-  MOE_LAUNCHED(s, "dispatch_hist");
-  prof_begin(s);
-  disp_scan_kernel<<<1, 1024, c->E * 8, s>>>(bhist, bsent, L.n_disp_blocks, c->E, c->T,
-                                             c->n_shared, L.C, L.rows_max, L.align, counts,
-                                             kept, offsets, tile_expert, stats);
-  MOE_LAUNCHED(s, "dispatch_scan");
-  prof_begin(s);
-  disp_rank_kernel<<<L.n_disp_blocks, 256, kDispWarps * c->E * 4, s>>>(
-      topk_idx, sentinel_mask, L.n_slots, c->E, L.C, L.rows_max, bhist, offsets, slot_row,
-      row_slot);
-  MOE_LAUNCHED(s, "dispatch_rank");
-  const int grid = grid_for(L.rows_max);
-  prof_begin(s);
-  if (c->dtype == MOE_BF16)
-    disp_gather_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), c->D, c->K, c->E, c->T, offsets, kept, tile_expert,
-        stats, row_slot, static_cast<__nv_bfloat16*>(x_perm));
-  else
-    disp_gather_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), c->D, c->K,
-                                                    c->E, c->T, offsets, kept, tile_expert,
-                                                    stats, row_slot, static_cast<float*>(x_perm));
-  MOE_LAUNCHED(s, "dispatch_gather");
-  return MOE_OK;
+  return dispatch_impl(c, L, topk_idx, sentinel_mask, x, counts, kept, offsets, slot_row,
+                       row_slot, tile_expert, stats, x_perm, base,
+                       base + (size_t)L.n_disp_blocks * c->E, s);
 }
 
 int moe_aux_loss(const moe_config_t* c, const float* probs, const float* lse,
@@ -725,11 +757,11 @@ int moe_aux_loss(const moe_config_t* c, const float* probs, const float* lse,
   const Layout L = layout_of(c);
   float* part = wsp<float>(ws, L.off_aux);
   prof_begin(s);
-  aux_partial_kernel<<<L.n_aux_chunks, 256, 0, s>>>(probs, lse, c->T, c->E, part);
+  MOE_CK((launch_k(aux_partial_kernel, L.n_aux_chunks, 256, 0, s, probs, lse, c->T, c->E, part)));
   MOE_LAUNCHED(s, "aux_partial");
   prof_begin(s);
-  aux_final_kernel<<<1, 512, 0, s>>>(part, counts, L.n_aux_chunks, c->T, c->E, c->aux_alpha,
-                                     c->z_lambda, losses);
+  MOE_CK((launch_k(aux_final_kernel, 1, 512, 0, s, part, counts, L.n_aux_chunks, c->T, c->E, c->aux_alpha,
+                                     c->z_lambda, losses)));
   MOE_LAUNCHED(s, "aux_final");
   return MOE_OK;
 }
@@ -785,8 +817,8 @@ int moe_expert_ffn(const moe_config_t* c, const void* x_perm, const int32_t* off
     MOE_TRY(simt_rows<TE>(c, L, x_perm, D, w13, D, 1, (int64_t)2 * F * D, w13_s, a13, 2 * F,
                           2 * F, D, tile_expert, stats, s));
     prof_begin(s);
-    swiglu_fwd_kernel<TE><<<num_sms() * 8, 256, 0, s>>>(static_cast<const TE*>(a13),
-                                                         static_cast<TE*>(h), stats, F);
+    MOE_CK((launch_k(swiglu_fwd_kernel<TE>, num_sms() * 8, 256, 0, s, static_cast<const TE*>(a13),
+                                                         static_cast<TE*>(h), stats, F)));
     MOE_LAUNCHED(s, "swiglu_fwd");
     return simt_rows<TE>(c, L, h, F, w_down, F, 1, (int64_t)D * F, w_down_s, o, D, D, F,
                          tile_expert, stats, s);
@@ -802,13 +834,13 @@ int moe_combine(const moe_config_t* c, const void* o, const int32_t* slot_row,
   const int grid = grid_for(c->T);
   prof_begin(s);
   if (c->dtype == MOE_BF16)
-    combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+    MOE_CK((launch_k(combine_kernel<__nv_bfloat16>, grid, 256, 0, s,
         static_cast<const __nv_bfloat16*>(o), slot_row, topk_w, offsets, c->n_shared, c->T,
-        c->D, c->K, c->E, static_cast<__nv_bfloat16*>(y));
+        c->D, c->K, c->E, static_cast<__nv_bfloat16*>(y))));
   else
-    combine_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(o), slot_row, topk_w,
+    MOE_CK((launch_k(combine_kernel<float>, grid, 256, 0, s, static_cast<const float*>(o), slot_row, topk_w,
                                                offsets, c->n_shared, c->T, c->D, c->K, c->E,
-                                               static_cast<float*>(y));
+                                               static_cast<float*>(y))));
   MOE_LAUNCHED(s, "combine");
   return MOE_OK;
 }
@@ -844,24 +876,26 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     const int grid = grid_for(L.rows_max);
     prof_begin(s);
     if (bf)
-      bwd_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+      MOE_CK((launch_k(bwd_rows_kernel<__nv_bfloat16>, grid, 256, 0, s,
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dy), topk_w,
           row_slot, offsets, kept, tile_expert, stats, K, E, T, D, dg,
-          static_cast<__nv_bfloat16*>(dO));
+          static_cast<__nv_bfloat16*>(dO))));
     else
-      bwd_rows_kernel<float><<<grid, 256, 0, s>>>(
+      MOE_CK((launch_k(bwd_rows_kernel<float>, grid, 256, 0, s,
           static_cast<const float*>(o), static_cast<const float*>(dy), topk_w, row_slot, offsets,
-          kept, tile_expert, stats, K, E, T, D, dg, static_cast<float*>(dO));
+          kept, tile_expert, stats, K, E, T, D, dg, static_cast<float*>(dO))));
     MOE_LAUNCHED(s, "bwd_gate_grad_rows");
   }
   // The router gradient chain (2, 7) runs on side stream r, concurrently
-  // with the expert GEMMs (3-6); the two weight-gradient GEMMs run on side
-  // streams w1, w2 once the SwiGLU-backward GEMM is done.  Everything joins
-  // back into s before the dx kernel (8) and before returning.
+  // with the expert GEMMs (3-6).  The weight-gradient GEMMs run on side
+  // streams: w1 (dW_down, which needs only dO and h) from here on, w2
+  // (dW13) once the SwiGLU-backward GEMM is done.  The dx kernel (8) waits
+  // only for ds; every side stream joins back into s before returning.
   Side* sd = nullptr;
   MOE_TRY(side_streams(&sd));
   cudaStream_t r = sd->st[0], w1 = sd->st[1], w2 = sd->st[2];
   MOE_TRY(fork_join(sd->ev[0], s, r));
+  if (use_tc(c)) MOE_TRY(fork_join(sd->ev[1], s, w1));
   // 2. router backward: dlogits
   {
     RouterBwdArgs a{T, E, K, c->score_fn, c->renorm, c->route_scale, c->aux_alpha, c->z_lambda,
@@ -871,12 +905,13 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     {
     cudaStream_t s = r;
     prof_begin(s);
-    if (E <= 32) router_bwd_kernel<1><<<grid, 256, 0, s>>>(a);
-    else if (E <= 64) router_bwd_kernel<2><<<grid, 256, 0, s>>>(a);
-    else if (E <= 128) router_bwd_kernel<4><<<grid, 256, 0, s>>>(a);
-    else if (E <= 256) router_bwd_kernel<8><<<grid, 256, 0, s>>>(a);
-    else router_bwd_kernel<16><<<grid, 256, 0, s>>>(a);
+    if (E <= 32) MOE_CK((launch_k(router_bwd_kernel<1>, grid, 256, 0, s, a)));
+    else if (E <= 64) MOE_CK((launch_k(router_bwd_kernel<2>, grid, 256, 0, s, a)));
+    else if (E <= 128) MOE_CK((launch_k(router_bwd_kernel<4>, grid, 256, 0, s, a)));
+    else if (E <= 256) MOE_CK((launch_k(router_bwd_kernel<8>, grid, 256, 0, s, a)));
+    else MOE_CK((launch_k(router_bwd_kernel<16>, grid, 256, 0, s, a)));
     MOE_LAUNCHED(s, "router_bwd");
+    MOE_CK(cudaEventRecord(sd->ev[6], r));   // ds is ready
     }
   }
   // 3-6. expert GEMMs
@@ -902,7 +937,6 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
         MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD>(
             bn3, "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, units * p.nN, 0, s)));
     }
-    MOE_TRY(fork_join(sd->ev[1], s, w1));
     MOE_TRY(fork_join(sd->ev[2], s, w2));
     // 4. wgrad down: dW_down[e] = dO^T h over the expert's rows (CTA pairs
     // split the 256-row output tiles)
@@ -967,9 +1001,9 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       MOE_TRY(simt_rows<TE>(c, L, dO, D, w_down, 1, F, (int64_t)D * F, w_down_s, dH, F, F, D,
                             tile_expert, stats, s));
       prof_begin(s);
-      swiglu_bwd_kernel<TE><<<num_sms() * 8, 256, 0, s>>>(
+      MOE_CK((launch_k(swiglu_bwd_kernel<TE>, num_sms() * 8, 256, 0, s,
           static_cast<const TE*>(dH), static_cast<const TE*>(a13), static_cast<TE*>(dA13),
-          stats, F);
+          stats, F)));
       MOE_LAUNCHED(s, "swiglu_bwd");
       // 4. dW_down[e] = dO^T h
       MOE_TRY(simt_wgrad<TE>(c, dO, D, h, F, D, F, dw_down, dw_down_s, offsets, kept, s));
@@ -989,40 +1023,42 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     prof_begin(s);
     if (E <= 8) {
       dim3 g((unsigned)ceil_div(D, 256), 1, (unsigned)nc);
-      if (bf) dwr_partial_kernel<__nv_bfloat16, 8, 256, 2, 4><<<g, 256, 0, s>>>(
-          ds, static_cast<const __nv_bfloat16*>(x), T, E, D, L.dwr_chunk, dwr_part);
-      else dwr_partial_kernel<float, 8, 256, 2, 4><<<g, 256, 0, s>>>(
-          ds, static_cast<const float*>(x), T, E, D, L.dwr_chunk, dwr_part);
+      if (bf) MOE_CK((launch_k(dwr_partial_kernel<__nv_bfloat16, 8, 256, 2, 4>, g, 256, 0, s,
+          ds, static_cast<const __nv_bfloat16*>(x), T, E, D, L.dwr_chunk, dwr_part)));
+      else MOE_CK((launch_k(dwr_partial_kernel<float, 8, 256, 2, 4>, g, 256, 0, s,
+          ds, static_cast<const float*>(x), T, E, D, L.dwr_chunk, dwr_part)));
     } else {
       dim3 g((unsigned)ceil_div(D, 64), (unsigned)ceil_div(E, 64), (unsigned)nc);
-      if (bf) dwr_partial_kernel<__nv_bfloat16, 64, 64, 4, 4><<<g, 256, 0, s>>>(
-          ds, static_cast<const __nv_bfloat16*>(x), T, E, D, L.dwr_chunk, dwr_part);
-      else dwr_partial_kernel<float, 64, 64, 4, 4><<<g, 256, 0, s>>>(
-          ds, static_cast<const float*>(x), T, E, D, L.dwr_chunk, dwr_part);
+      if (bf) MOE_CK((launch_k(dwr_partial_kernel<__nv_bfloat16, 64, 64, 4, 4>, g, 256, 0, s,
+          ds, static_cast<const __nv_bfloat16*>(x), T, E, D, L.dwr_chunk, dwr_part)));
+      else MOE_CK((launch_k(dwr_partial_kernel<float, 64, 64, 4, 4>, g, 256, 0, s,
+          ds, static_cast<const float*>(x), T, E, D, L.dwr_chunk, dwr_part)));
     }
     MOE_LAUNCHED(s, "router_dw_partial");
     const int64_t n = (int64_t)E * D;
     prof_begin(s);
-    dwr_reduce_kernel<<<(int)std::min<int64_t>(ceil_div(n, 256), num_sms() * 8), 256, 0, s>>>(
-        dwr_part, nc, n, dw_r);
+    MOE_CK((launch_k(dwr_reduce_kernel, (int)std::min<int64_t>(ceil_div(n, 256), num_sms() * 8), 256, 0, s,
+        dwr_part, nc, n, dw_r)));
     MOE_LAUNCHED(s, "router_dw_reduce");
   }
-  // join the router chain, then 8. dx = unpermute-sum(dX_perm) + shared + ds . w_r
-  MOE_TRY(fork_join(sd->ev[3], r, s));
+  // 8. dx = unpermute-sum(dX_perm) + shared + ds . w_r, once ds is ready
+  MOE_CK(cudaStreamWaitEvent(s, sd->ev[6], 0));
   {
     dim3 g((unsigned)ceil_div(T, 64), (unsigned)ceil_div(D, 128));
     prof_begin(s);
     if (bf)
-      dx_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(ds, w_r, static_cast<const __nv_bfloat16*>(dXp),
+      MOE_CK((launch_k(dx_kernel<__nv_bfloat16>, g, 256, 0, s, ds, w_r, static_cast<const __nv_bfloat16*>(dXp),
                                                  slot_row, offsets, c->n_shared, T, D, E, K,
-                                                 static_cast<__nv_bfloat16*>(dx));
+                                                 static_cast<__nv_bfloat16*>(dx))));
     else
-      dx_kernel<float><<<g, 256, 0, s>>>(ds, w_r, static_cast<const float*>(dXp), slot_row,
+      MOE_CK((launch_k(dx_kernel<float>, g, 256, 0, s, ds, w_r, static_cast<const float*>(dXp), slot_row,
                                          offsets, c->n_shared, T, D, E, K,
-                                         static_cast<float*>(dx));
+                                         static_cast<float*>(dx))));
     MOE_LAUNCHED(s, "dx_unpermute_router");
   }
-  // join the weight-gradient streams (no-ops on the SIMT path)
+  // join the router chain and the weight-gradient streams (the latter are
+  // no-ops on the SIMT path)
+  MOE_TRY(fork_join(sd->ev[3], r, s));
   MOE_TRY(fork_join(sd->ev[4], w1, s));
   MOE_TRY(fork_join(sd->ev[5], w2, s));
   return MOE_OK;
@@ -1070,6 +1106,14 @@ int moe_profile_read(float* ms, int max) {
   const int n = std::min(g_prof.n, max);
   for (int i = 0; i < n; ++i)
     MOE_CK(cudaEventElapsedTime(&ms[i], g_prof.ev[2 * i], g_prof.ev[2 * i + 1]));
+  return n;
+}
+
+int moe_profile_starts(float* ms, int max) {
+  if (ms == nullptr) return MOE_ERR_ARG;
+  const int n = std::min(g_prof.n, max);
+  for (int i = 0; i < n; ++i)
+    MOE_CK(cudaEventElapsedTime(&ms[i], g_prof.ev[0], g_prof.ev[2 * i]));
   return n;
 }
 

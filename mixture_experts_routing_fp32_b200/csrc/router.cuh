@@ -191,6 +191,7 @@ template <typename TX, int EB>
 __global__ void __launch_bounds__(256)
 router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
                     const float* __restrict__ offset, int D, RouteArgs a) {
+  pdl_begin();
   extern __shared__ __align__(16) float smem[];
   float* ws = smem;                         // [E, D]
   float* gsm_all = smem + (size_t)a.E * D;  // [8 warps, E]
@@ -245,6 +246,7 @@ __global__ void __launch_bounds__(256)
 router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
                      const float* __restrict__ offset, float* __restrict__ logits,
                      int T, int D, int E) {
+  pdl_begin();
   constexpr int BT = 64, BE = 64, BK = 32;
   __shared__ __align__(16) float xs[BK][BT + 4];
   __shared__ __align__(16) float wsm[BK][BE + 4];
@@ -302,6 +304,7 @@ router_logits_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
 template <int NV>
 __global__ void __launch_bounds__(256)
 router_route_kernel(const float* __restrict__ logits, RouteArgs a) {
+  pdl_begin();
   extern __shared__ __align__(16) float gsm_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* gsm = gsm_all + warp * a.E;

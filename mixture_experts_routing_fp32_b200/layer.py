@@ -4,8 +4,8 @@ The layer owns every device buffer the C ABI needs (allocated once with
 torch, stable pointers, so a whole step can be captured in a CUDA graph)
 and issues the entry points in order on the current stream:
 
-  forward : moe_router -> moe_dispatch -> moe_aux_loss -> moe_expert_ffn
-            -> moe_combine
+  forward : moe_router -> moe_dispatch -> moe_expert_ffn -> moe_combine,
+            with moe_aux_loss on a side stream (joined before returning)
   backward: moe_backward
 
 No host synchronisation happens inside forward or backward.
@@ -45,6 +45,7 @@ class MoELayer:
         self.ws = e((max(int(z.ws_bytes), 256),), torch.uint8)
         self._grads_ready = False
         self._inputs = None
+        self._aux_stream = None
 
     def _alloc_grads(self):
         """Gradient buffers, allocated on the first backward (a forward-only
@@ -72,12 +73,22 @@ class MoELayer:
         api.moe_dispatch(c, self.topk_idx, sentinel_mask, x, self.counts, self.kept,
                          self.offsets, self.slot_row, self.row_slot, self.tile_expert,
                          self.stats, self.x_perm, self.ws)
-        if c.aux_alpha != 0.0 or c.z_lambda != 0.0:
-            api.moe_aux_loss(c, self.probs, self.lse, self.counts, self.losses, self.ws)
+        main = torch.cuda.current_stream(self.device)
+        aux = c.aux_alpha != 0.0 or c.z_lambda != 0.0
+        if aux:
+            # the losses depend only on the router and the counts: computed
+            # on a side stream while the expert GEMMs run
+            if self._aux_stream is None:
+                self._aux_stream = torch.cuda.Stream(self.device)
+            self._aux_stream.wait_stream(main)
+            api.moe_aux_loss(c, self.probs, self.lse, self.counts, self.losses, self.ws,
+                             stream=self._aux_stream)
         api.moe_expert_ffn(c, self.x_perm, self.offsets, self.tile_expert, self.stats,
                            w13, w_down, w13_s, w_down_s, self.a13, self.h, self.o,
                            self.ws)
         api.moe_combine(c, self.o, self.slot_row, self.topk_w, self.offsets, self.y)
+        if aux:
+            main.wait_stream(self._aux_stream)
         self._inputs = (x, w_r, w13, w_down, w13_s, w_down_s)
         return self.y
 

@@ -105,6 +105,8 @@ REDUCED = {
     # enough rows per expert (>= 1536) that the expert GEMMs run on CTA pairs
     "mm_pair": CONFIGS["mm_b"].replace(name="mm_pair_small", T=6500, D=256, F=512),
     "mix_pair": CONFIGS["mix"].replace(name="mix_pair_small", T=7000, D=512, F=640),
+    # more than 16384 slots: the multi-block dispatch passes (ragged last block)
+    "olmoe_multi": CONFIGS["olmoe"].replace(name="olmoe_multi_small", T=2600, D=128, F=128),
 }
 
 
