@@ -118,6 +118,24 @@ def gemm_flops(cfg, kept_total):
     }
 
 
+def hbm_bytes(cfg, kept_total, rows_used):
+    """Algorithmic DRAM bytes of each memory-bound kernel for one step: every
+    operand read once and every result written once (activations in the
+    layer dtype, router tensors fp32)."""
+    a = 2 if cfg.dtype == "bf16" else 4
+    T, D, E, K = cfg.T, cfg.D, cfg.E, cfg.K
+    M = expert_rows(cfg, kept_total)
+    router = T * D * a + E * D * 4 + 2 * T * E * 4 + T * 4 + T * K * 8
+    return {
+        "router_fused": router, "router_logits": T * D * a + E * D * 4 + T * E * 4,
+        "router_route": 3 * T * E * 4 + T * 4 + T * K * 8,
+        "dispatch_gather": M * D * a + rows_used * D * a,
+        "combine": M * D * a + T * D * a + T * K * 8,
+        "bwd_gate_grad_rows": 2 * M * D * a + rows_used * D * a + T * K * 8,
+        "dx_unpermute_router": M * D * a + T * D * a + T * E * 4 + E * D * 4,
+    }
+
+
 def source_hash(files=None):
     """Hash of the kernel sources (all of csrc/, or the named files)."""
     h = hashlib.sha256()
@@ -409,6 +427,15 @@ def run_ours(args):
     main_flops = sum(v for k, v in flops.items() if k in tot and k not in side)
     main_gemm_tflops = main_flops / (gemm_total_ms * 1e-3) / 1e12 if gemm_total_ms else None
 
+    # memory-bound kernels: algorithmic bytes / live launch time vs HBM peak
+    rows_used = int(layer.stats[2])
+    hbm_table = {}
+    for k, b in hbm_bytes(base, kept_total, rows_used).items():
+        if k in tot and tot[k] > 0:
+            gbs = b / (tot[k] * 1e-3) / 1e9
+            hbm_table[k] = {"bytes": b, "ms": round(tot[k], 5), "GB/s": round(gbs, 1),
+                            "frac_of_hbm": round(gbs / hbm, 4),
+                            "side_stream": k in side}
     clocks = clk.summary()
     cpu = cpu_baseline(base, args.cpu_sample_s) if (rank == 0 and world == 1 and not args.no_cpu) else None
     if rank == 0:
@@ -438,6 +465,7 @@ def run_ours(args):
                 "kernels": sorted(k for k in tot if k.startswith("tc_") and k not in side)},
             "kernels_ms_per_step": {k + (" [side stream]" if k in side else ""): round(v, 5)
                                     for k, v in sorted(tot.items(), key=lambda kv: -kv[1])},
+            "hbm_kernels": hbm_table,
             "kept_rows": kept_total,
             "clocks": clocks,
             "cpu_baseline": cpu,

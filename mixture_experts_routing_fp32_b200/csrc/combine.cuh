@@ -129,6 +129,11 @@ struct RouterBwdArgs {
   float* ds;               // [T,E]
   float* dlogits_out;      // [T,E] or null
   float* dg_out;           // [T,K] or null
+  // bf16 splits of ds for the tensor-core router products (or null):
+  // dsf [T, 3 Ep] = (hi | mid | lo), dsb [T, 3 Ep] = (hi | hi | mid)
+  __nv_bfloat16* dsf;
+  __nv_bfloat16* dsb;
+  int Ep;
 };
 
 template <int NV>
@@ -240,6 +245,24 @@ router_bwd_kernel(RouterBwdArgs a) {
       if (e < E) {
         a.ds[t * E + e] = ds[i];
         if (a.dlogits_out) a.dlogits_out[t * E + e] = ds[i];
+      }
+    }
+    if (a.dsf != nullptr) {
+      const int64_t b = t * 3 * (int64_t)a.Ep;
+      const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+          __nv_bfloat16 hi, mid, lo;
+          split3_bf16(ds[i], hi, mid, lo);
+          a.dsf[b + e] = hi; a.dsf[b + a.Ep + e] = mid; a.dsf[b + 2 * a.Ep + e] = lo;
+          a.dsb[b + e] = hi; a.dsb[b + a.Ep + e] = hi; a.dsb[b + 2 * a.Ep + e] = mid;
+        }
+      }
+      for (int e = E + lane; e < a.Ep; e += 32) {
+        a.dsf[b + e] = z; a.dsf[b + a.Ep + e] = z; a.dsf[b + 2 * a.Ep + e] = z;
+        a.dsb[b + e] = z; a.dsb[b + a.Ep + e] = z; a.dsb[b + 2 * a.Ep + e] = z;
       }
     }
     if (a.dg_out != nullptr && lane < K) {
@@ -390,6 +413,18 @@ dx_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
     }
     store8(dx + t * D + d, acc[i]);
   }
+}
+
+// dW_r from the three partial products of the tensor-core path
+// (part [3 Ep, D]: ds_hi^T x | ds_mid^T x | ds_lo^T x), summed in that order.
+__global__ void __launch_bounds__(256)
+dwr_reduce3_kernel(const float* __restrict__ part, int E, int Ep, int D,
+                   float* __restrict__ dw_r) {
+  pdl_begin();
+  const int64_t n = (int64_t)E * D, stride = (int64_t)Ep * D;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    dw_r[i] = (part[i] + part[stride + i]) + part[2 * stride + i];
 }
 
 }  // namespace moe

@@ -20,6 +20,10 @@
 //     WGRAD mode: C_g[m, n] = sum_{r in rows(g)} A[r, m] B[r, n] (weight
 //     gradients; the reduction runs over the group's own rows and the zero
 //     padding rows beyond them contribute nothing);
+//   * dense variants (no tile map, one group) serve the router's fp32
+//     products, which run as bf16 MMAs on three-way bf16 splits of the fp32
+//     operand (x . W_r^T, ds^T . x, ds . W_r): fp32 epilogues, and a dx
+//     epilogue that adds the unpermute-sum of the expert data gradients;
 //   * every mbarrier wait is bounded in time; on timeout the kernel records
 //     MOE_DEVERR_TIMEOUT, drains its own copies and MMAs, frees tensor
 //     memory and returns.
@@ -37,7 +41,15 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
 enum { MODE_ROWS = 0, MODE_WGRAD = 1 };
-enum { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2, EPI_WGRAD = 3 };
+enum {
+  EPI_STORE = 0,       // bf16 C
+  EPI_SWIGLU = 1,      // a13 = C (gate | up) and h = silu(gate) * up
+  EPI_SWIGLU_BWD = 2,  // da13 from dh = C and the saved a13
+  EPI_WGRAD = 3,       // bf16 weight gradient per group
+  EPI_F32 = 4,         // fp32 C, rows < dense_m (dense ROWS)
+  EPI_WGRAD_F32 = 5,   // fp32 C, rows < m_limit (dense WGRAD)
+  EPI_DX = 6           // dx = C + unpermute-sum of dXp rows (+ shared row), bf16
+};
 
 struct Params {
   int E, F, Kd;
@@ -55,6 +67,16 @@ struct Params {
   __nv_bfloat16* out2; int64_t ld_out2;    // SwiGLU: h
   const __nv_bfloat16* aux; int64_t ld_aux;  // SwiGLU bwd: a13
   __nv_bfloat16* out_shared;               // WGRAD: shared group output
+  // dense variants
+  int dense_m;                 // ROWS: > 0 = one group of dense_m rows, no tile map
+  int dense_rows;              // WGRAD: > 0 = one group of dense_rows rows
+  int m_limit;                 // WGRAD_F32: output rows
+  float* out_f32; int64_t ld_f32;          // F32 epilogues
+  // EPI_DX: rows of dXp summed into each token's output row
+  const __nv_bfloat16* dxp;    // [rows, No]
+  const int32_t* slot_row;     // [dense_m, K]
+  const int32_t* dx_offsets;   // offsets[E_routed] = first shared row
+  int K, n_shared, E_routed;
 };
 
 // ----------------------------------------------------------------------------
@@ -332,7 +354,8 @@ __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
 // Stores this lane's 32 values (its row of the block) as bf16; w0 addresses
 // the block's first row and column, ld is the row stride in elements.
 __device__ __forceinline__ void staged_store32(uint32_t stg, const float (&v)[32],
-                                               __nv_bfloat16* w0, int64_t ld, uint64_t pol) {
+                                               __nv_bfloat16* w0, int64_t ld, uint64_t pol,
+                                               int nrows = 32) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int j = 0; j < 4; ++j) sts128(stg + lane * kStgRow + j * 16, pack8_bf16(v + 8 * j));
@@ -341,12 +364,21 @@ __device__ __forceinline__ void staged_store32(uint32_t stg, const float (&v)[32
   for (int i = 0; i < 4; ++i) {
     const int r = i * 8 + (lane >> 2), pc = lane & 3;
     const uint4 u = lds128(stg + r * kStgRow + pc * 16);
-    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(
-                     w0 + r * ld + pc * 8),
-                 "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w), "l"(pol)
-                 : "memory");
+    if (r < nrows)
+      asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(
+                       w0 + r * ld + pc * 8),
+                   "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w), "l"(pol)
+                   : "memory");
   }
   __syncwarp();
+}
+
+// 32 fp32 values of one row (16-byte stores).
+__device__ __forceinline__ void store32_f32(float* p, const float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    *reinterpret_cast<float4*>(p + 4 * i) = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2],
+                                                        v[4 * i + 3]);
 }
 
 // Coalesced load of a 32 x 32 bf16 block (w0: first row and column): piece
@@ -402,7 +434,7 @@ __device__ __forceinline__ Tile decode(int t, const Params& p, int rank, int n_m
     const int gm = min(p.group_m, n_mt - first);
     const int local = t - group * p.group_m * p.nN;
     const int mt = first + local % gm, nt = local / gm;
-    d.e = p.tile_expert[mt * (MU / BM)];
+    d.e = p.dense_m > 0 ? 0 : p.tile_expert[mt * (MU / BM)];
     d.m0 = mt * MU + rank * BM;
     d.n0 = nt * (EPI == EPI_SWIGLU ? BN / 2 : BN);
     d.row0 = 0;
@@ -413,8 +445,8 @@ __device__ __forceinline__ Tile decode(int t, const Params& p, int rank, int n_m
     d.e = g;
     d.m0 = (rem / p.nNo) * MU + rank * BM;
     d.n0 = (rem % p.nNo) * BN;
-    d.row0 = p.offsets[g];
-    const int rows = g < p.E ? p.kept[g] : p.T;
+    d.row0 = p.dense_rows > 0 ? 0 : p.offsets[g];
+    const int rows = p.dense_rows > 0 ? p.dense_rows : g < p.E ? p.kept[g] : p.T;
     d.nk = (rows + BK - 1) / BK;
   }
   return d;
@@ -504,7 +536,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   // Each role decodes tile t + n_units while it works on tile t, so the
   // global loads a decode needs (tile -> expert map, group offsets) never
   // stall a tile boundary.
-  const int n_mt = (MODE == MODE_ROWS) ? p.stats[3] / (PAIR ? 2 : 1) : 0;
+  constexpr int kMU = PAIR ? 2 * BM : BM;
+  const int n_mt = (MODE != MODE_ROWS) ? 0
+                   : p.dense_m > 0    ? (p.dense_m + kMU - 1) / kMU
+                                      : p.stats[3] / (PAIR ? 2 : 1);
   const int total = (MODE == MODE_ROWS) ? n_mt * p.nN : total_hint;
   auto decode_at = [&](int t) {
     return t < total ? decode<MODE, EPI, BN, PAIR>(t, p, rank, n_mt) : Tile{0, 0, 0, 0, 0};
@@ -648,7 +683,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     for (int t = unit; t < total; t += n_units) {
       const Tile d = nxt;
       nxt = decode_at(t + n_units);
-      if (MODE == MODE_WGRAD && d.nk == 0) {
+      if (EPI == EPI_WGRAD && d.nk == 0) {
         __nv_bfloat16* og = d.e < p.E ? p.out + (int64_t)d.e * p.strideCE : p.out_shared;
         __nv_bfloat16* dst = og + (int64_t)(d.m0 + rloc) * p.No + d.n0 + hh * HC;
         for (int c = 0; c < HC; c += 8) zero8(dst + c);
@@ -708,6 +743,58 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
 #pragma unroll
           for (int i = 0; i < 32; ++i) ga[i] = ga[i] * fast_sigmoid(ga[i]) * ub[i];
           staged_store32(stg, ga, hr + c, p.ld_out2, pol_out);
+        }
+      } else if constexpr (EPI == EPI_F32 || EPI == EPI_WGRAD_F32) {
+        const int64_t row = row0 + lane;
+        const bool rv = row < (EPI == EPI_F32 ? (int64_t)p.dense_m : (int64_t)p.m_limit);
+        float* dst = p.out_f32 + row * p.ld_f32 + d.n0 + hh * HC;
+#pragma unroll
+        for (int c = 0; c < HC; c += 32) {
+          uint32_t r[32];
+          float v[32];
+          tmem_ld32(tbase + hh * HC + c, r);
+          tmem_wait();
+          u2f32(r, v);
+          if (rv) store32_f32(dst + c, v);
+        }
+      } else if constexpr (EPI == EPI_DX) {
+        // this lane's token t = row0 + lane: its kept slots' rows and its
+        // shared-expert row of dXp are added to C (the router term)
+        constexpr int kDxMaxK = 16;
+        const int64_t t = row0 + lane;
+        const int64_t left = (int64_t)p.dense_m - row0;
+        const int nrows = left <= 0 ? 0 : left >= 32 ? 32 : (int)left;
+        const bool tv = t < p.dense_m;
+        int32_t rk[kDxMaxK];
+#pragma unroll
+        for (int k = 0; k < kDxMaxK; ++k)
+          rk[k] = (tv && k < p.K) ? p.slot_row[t * p.K + k] : -1;
+        const int64_t srow = (tv && p.n_shared) ? (int64_t)p.dx_offsets[p.E_routed] + t : -1;
+        __nv_bfloat16* w0 = p.out + row0 * p.ld_out + d.n0 + hh * HC;
+        const __nv_bfloat16* src = p.dxp + d.n0 + hh * HC;
+#pragma unroll
+        for (int c = 0; c < HC; c += 32) {
+          uint32_t r[32];
+          float v[32];
+          tmem_ld32(tbase + hh * HC + c, r);
+          tmem_wait();
+          u2f32(r, v);
+#pragma unroll
+          for (int k = 0; k < kDxMaxK; ++k) {
+            if (rk[k] >= 0) {
+              float g[32];
+              load32_bf16(src + (int64_t)rk[k] * p.No + c, g);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] += g[i];
+            }
+          }
+          if (srow >= 0) {
+            float g[32];
+            load32_bf16(src + srow * p.No + c, g);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] += g[i];
+          }
+          staged_store32(stg, v, w0 + c, p.ld_out, pol_out, nrows);
         }
       } else {  // EPI_SWIGLU_BWD
         __nv_bfloat16* da13 = p.out + row0 * p.ld_out + d.n0 + hh * HC;

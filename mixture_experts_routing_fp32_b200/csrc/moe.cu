@@ -9,6 +9,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include "common.cuh"
@@ -131,6 +132,13 @@ bool use_tc(const moe_config_t* c) {
 
 int64_t capacity_of(const moe_config_t* c);
 
+// The router's fp32 products (logits, dW_r, the router part of dx) run on
+// tensor cores as bf16 MMAs over three-way bf16 splits of the fp32 operand
+// when the expert GEMMs do and E >= 8; below that the SIMT kernels are as
+// fast.  Ep = E rounded up to 64 (split width).
+bool router_tc(const moe_config_t* c) { return use_tc(c) && c->E >= 8; }
+int64_t router_ep(const moe_config_t* c) { return (c->E + 63) / 64 * 64; }
+
 // Row GEMMs run on CTA pairs (two SMs share each 256-row MMA) when experts
 // hold enough rows that aligning their segments to 256 rows wastes little
 // and the extra operand reuse pays (at least 1536 rows on average: measured
@@ -152,6 +160,9 @@ struct Layout {
   int n_disp_blocks, n_aux_chunks, n_dwr_chunks, dwr_chunk, align;
   size_t off_bhist, off_bsent, off_aux, off_dg, off_ds, off_dwr, off_dO, off_dA13, off_dX,
       off_dH, total;
+  // tensor-core router products (router_tc)
+  int64_t Ep;
+  size_t off_wf, off_wb, off_rparts, off_dsf, off_dsb, off_dwr3;
 };
 constexpr int kAuxChunk = 128;
 
@@ -192,6 +203,15 @@ Layout layout_of(const moe_config_t* c) {
   L.off_dA13 = take((size_t)L.rows_max * 2 * c->F * a);
   L.off_dX = take((size_t)L.rows_max * c->D * a);
   L.off_dH = use_tc(c) ? off : take((size_t)L.rows_max * c->F * a);
+  if (router_tc(c)) {
+    L.Ep = router_ep(c);
+    L.off_wf = take((size_t)3 * L.Ep * c->D * 2);
+    L.off_wb = take((size_t)3 * L.Ep * c->D * 2);
+    L.off_rparts = take((size_t)c->T * 3 * L.Ep * 4);
+    L.off_dsf = take((size_t)c->T * 3 * L.Ep * 2);
+    L.off_dsb = take((size_t)c->T * 3 * L.Ep * 2);
+    L.off_dwr3 = take((size_t)3 * L.Ep * c->D * 4);
+  }
   L.total = off;
   return L;
 }
@@ -387,13 +407,62 @@ int grid_for(int64_t items_per_8, int cap_mult = 8) {
 // ---------------------------------------------------------------------------
 // router
 // ---------------------------------------------------------------------------
+int group_rows(int64_t Kd, bool pair = false);
+
+// Routing of each token from logits (or from the tensor-core partial
+// logits), one warp per token.
+int route_launch(const moe_config_t* c, const RouteArgs& a, const float* logits,
+                 const float* parts, int64_t Ep, const float* off, cudaStream_t s) {
+  const size_t sm = 8 * (size_t)c->E * 4;
+  const int grid = grid_for(c->T);
+  auto go = [&](auto nv) -> int {
+    constexpr int NV = decltype(nv)::value;
+    prof_begin(s);
+    if (parts != nullptr)
+      MOE_CK((launch_k(router_route_parts_kernel<NV>, grid, 256, sm, s, parts, (int)Ep, off, a)));
+    else
+      MOE_CK((launch_k(router_route_kernel<NV>, grid, 256, sm, s, logits, a)));
+    MOE_LAUNCHED(s, "router_route");
+    return MOE_OK;
+  };
+  if (c->E <= 32) return go(std::integral_constant<int, 1>{});
+  if (c->E <= 64) return go(std::integral_constant<int, 2>{});
+  if (c->E <= 128) return go(std::integral_constant<int, 4>{});
+  if (c->E <= 256) return go(std::integral_constant<int, 8>{});
+  return go(std::integral_constant<int, 16>{});
+}
+
 template <typename TX>
 int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const float* off,
                 const float* bias, float* logits, float* probs, float* lse, int32_t* idx,
-                float* w, int32_t* ties, cudaStream_t s) {
+                float* w, int32_t* ties, void* ws, cudaStream_t s) {
   RouteArgs a{c->T, c->E, c->K, c->score_fn, c->renorm, c->n_groups, c->topk_groups,
               c->group_score, c->route_scale, bias, logits, probs, lse, idx, w, ties};
   MOE_CK(cudaMemsetAsync(ties, 0, sizeof(int32_t), s));
+  if (router_tc(c)) {
+    // logits parts = x . (W_hi | W_mid | W_lo)^T on tensor cores (dense GEMM,
+    // fp32 out), then routing sums the parts
+    const Layout L = layout_of(c);
+    const int64_t Ep = L.Ep, n3 = 3 * Ep;
+    auto* wf = wsp<__nv_bfloat16>(ws, L.off_wf);
+    float* parts = wsp<float>(ws, L.off_rparts);
+    prof_begin(s);
+    MOE_CK((launch_k(split_w_kernel, grid_for(Ep * c->D / 32), 256, 0, s, w_r, c->E, (int)Ep,
+                     c->D, wf, (__nv_bfloat16*)nullptr)));
+    MOE_LAUNCHED(s, "router_split_w");
+    const int64_t mtiles = ceil_div(c->T, kRowTile);
+    const int bn = pick_bn(n3, mtiles, false, 0, false);
+    CUtensorMap mA, mB;
+    MOE_TRY(make_map(&mA, x, 1, c->T, c->D, 128, false));
+    MOE_TRY(make_map(&mB, wf, 1, n3, c->D, bn, true));       // dims {D, 3Ep, 1}
+    tc::Params p{};
+    p.E = 1; p.Kd = c->D; p.nN = (int)(n3 / bn); p.group_m = group_rows(c->D);
+    p.dense_m = c->T;
+    p.out_f32 = parts; p.ld_f32 = n3;
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_F32>(
+        bn, "router_logits_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+    return route_launch(c, a, nullptr, parts, Ep, off, s);
+  }
   const size_t fused_smem = (size_t)c->E * c->D * 4 + 8 * (size_t)c->E * 4;
   if (c->E <= 32 && fused_smem <= 200 * 1024) {
     const int grid = grid_for(c->T, 2);
@@ -411,18 +480,10 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
   }
   dim3 g1((unsigned)ceil_div(c->T, 64), (unsigned)ceil_div(c->E, 64));
   prof_begin(s);
-  MOE_CK((launch_k(router_logits_kernel<TX>, g1, 256, 0, s, x, w_r, off, logits, c->T, c->D, c->E)));
+  MOE_CK((launch_k(router_logits_kernel<TX>, g1, 256, 0, s, x, w_r, off, logits, c->T, c->D,
+                   c->E)));
   MOE_LAUNCHED(s, "router_logits");
-  const size_t sm = 8 * (size_t)c->E * 4;
-  const int grid = grid_for(c->T);
-  prof_begin(s);
-  if (c->E <= 32) MOE_CK((launch_k(router_route_kernel<1>, grid, 256, sm, s, logits, a)));
-  else if (c->E <= 64) MOE_CK((launch_k(router_route_kernel<2>, grid, 256, sm, s, logits, a)));
-  else if (c->E <= 128) MOE_CK((launch_k(router_route_kernel<4>, grid, 256, sm, s, logits, a)));
-  else if (c->E <= 256) MOE_CK((launch_k(router_route_kernel<8>, grid, 256, sm, s, logits, a)));
-  else MOE_CK((launch_k(router_route_kernel<16>, grid, 256, sm, s, logits, a)));
-  MOE_LAUNCHED(s, "router_route");
-  return MOE_OK;
+  return route_launch(c, a, logits, nullptr, 0, nullptr, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -581,7 +642,7 @@ int fork_join(cudaEvent_t ev, cudaStream_t from, cudaStream_t to) {
 // Row tiles per rasterisation group: as many 128-row A tiles of depth Kd as
 // fit in about 48 MiB of L2, so they stay resident while the group sweeps
 // the weight column slices.
-int group_rows(int64_t Kd, bool pair = false) {
+int group_rows(int64_t Kd, bool pair) {
   const int64_t rows = pair ? 256 : 128;
   return (int)std::max<int64_t>(1, std::min<int64_t>(64, (48ll << 20) / (rows * Kd * 2)));
 }
@@ -663,15 +724,15 @@ int moe_get_sizes(const moe_config_t* cfg, moe_sizes_t* out) {
 int moe_router(const moe_config_t* c, const void* x, const float* w_r, const float* logit_offset,
                const float* sel_bias, float* logits, float* probs, float* lse, int32_t* topk_idx,
                float* topk_w, int32_t* near_ties, void* ws, cudaStream_t s) {
-  (void)ws;
   MOE_TRY(validate(c));
   if (!x || !w_r || !logits || !probs || !lse || !topk_idx || !topk_w || !near_ties)
     return MOE_ERR_ARG;
+  if (router_tc(c) && ws == nullptr) return MOE_ERR_ARG;
   if (c->dtype == MOE_BF16)
     return router_impl(c, static_cast<const __nv_bfloat16*>(x), w_r, logit_offset, sel_bias,
-                       logits, probs, lse, topk_idx, topk_w, near_ties, s);
+                       logits, probs, lse, topk_idx, topk_w, near_ties, ws, s);
   return router_impl(c, static_cast<const float*>(x), w_r, logit_offset, sel_bias, logits, probs,
-                     lse, topk_idx, topk_w, near_ties, s);
+                     lse, topk_idx, topk_w, near_ties, ws, s);
 }
 
 int moe_dispatch(const moe_config_t* c, const int32_t* topk_idx, const uint8_t* sentinel_mask,
@@ -870,6 +931,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   void* dXp = wsp<void>(ws, L.off_dX);
   void* dH = wsp<void>(ws, L.off_dH);
   const bool bf = c->dtype == MOE_BF16;
+  const bool rtc = router_tc(c);
 
   // 1. per row: gate gradient dg = <o, dy>, and dO = g * dy
   {
@@ -900,7 +962,12 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   {
     RouterBwdArgs a{T, E, K, c->score_fn, c->renorm, c->route_scale, c->aux_alpha, c->z_lambda,
                     logits, probs, lse, topk_idx, topk_w, slot_row, dg, counts, ds, dlogits_out,
-                    dg_out};
+                    dg_out, nullptr, nullptr, 0};
+    if (rtc) {
+      a.dsf = wsp<__nv_bfloat16>(ws, L.off_dsf);
+      a.dsb = wsp<__nv_bfloat16>(ws, L.off_dsb);
+      a.Ep = (int)L.Ep;
+    }
     const int grid = grid_for(T);
     {
     cudaStream_t s = r;
@@ -911,7 +978,14 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     else if (E <= 256) MOE_CK((launch_k(router_bwd_kernel<8>, grid, 256, 0, s, a)));
     else MOE_CK((launch_k(router_bwd_kernel<16>, grid, 256, 0, s, a)));
     MOE_LAUNCHED(s, "router_bwd");
-    MOE_CK(cudaEventRecord(sd->ev[6], r));   // ds is ready
+    if (rtc) {
+      // (hi; mid; hi) split of W_r for the router part of dx
+      prof_begin(s);
+      MOE_CK((launch_k(split_w_kernel, grid_for(L.Ep * D / 32), 256, 0, s, w_r, E, (int)L.Ep, D,
+                       (__nv_bfloat16*)nullptr, wsp<__nv_bfloat16>(ws, L.off_wb))));
+      MOE_LAUNCHED(s, "router_split_w");
+    }
+    MOE_CK(cudaEventRecord(sd->ev[6], r));   // ds (and its splits) ready
     }
   }
   // 3-6. expert GEMMs
@@ -1016,8 +1090,30 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     if (bf) MOE_TRY(go(__nv_bfloat16{}));
     else MOE_TRY(go(float{}));
   }
-  // 7. dW_r = ds^T x (two deterministic stages), on the router stream
-  {
+  // 7. dW_r = ds^T x on the router stream: on tensor cores as
+  // (ds_hi | ds_mid | ds_lo)^T x then the sum of the three parts; else two
+  // deterministic SIMT stages
+  if (rtc) {
+    cudaStream_t s = r;
+    const int64_t n3 = 3 * L.Ep;
+    CUtensorMap mA, mB;
+    MOE_TRY(make_map(&mA, wsp<__nv_bfloat16>(ws, L.off_dsf), 1, T, n3, 64, false));
+    MOE_TRY(make_map(&mB, x, 1, T, D, 64, false));
+    const int64_t nmo = ceil_div(n3, kRowTile);
+    const int bn = pick_bn(D, nmo, false, 0, false);
+    tc::Params p{};
+    p.E = 1; p.n_groups = 1; p.dense_rows = T; p.T = T;
+    p.nMo = (int)nmo; p.nNo = D / bn; p.No = D;
+    p.m_limit = (int)n3;
+    p.out_f32 = wsp<float>(ws, L.off_dwr3); p.ld_f32 = D;
+    const int total = p.nMo * p.nNo;
+    MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD_F32>(
+        bn, "router_dw_tc", mA, mB, mB, p, total, total, s)));
+    prof_begin(s);
+    MOE_CK((launch_k(dwr_reduce3_kernel, grid_for((int64_t)E * D / 32), 256, 0, s,
+                     wsp<const float>(ws, L.off_dwr3), E, (int)L.Ep, D, dw_r)));
+    MOE_LAUNCHED(s, "router_dw_reduce3");
+  } else {
     cudaStream_t s = r;
     const int nc = L.n_dwr_chunks;
     prof_begin(s);
@@ -1041,9 +1137,27 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
         dwr_part, nc, n, dw_r)));
     MOE_LAUNCHED(s, "router_dw_reduce");
   }
-  // 8. dx = unpermute-sum(dX_perm) + shared + ds . w_r, once ds is ready
+  // 8. dx = unpermute-sum(dX_perm) + shared + ds . w_r, once ds is ready;
+  // on tensor cores the router part is (ds_hi | ds_hi | ds_mid) .
+  // (W_hi; W_mid; W_hi) and the epilogue adds the dX_perm rows
   MOE_CK(cudaStreamWaitEvent(s, sd->ev[6], 0));
-  {
+  if (rtc) {
+    const int64_t n3 = 3 * L.Ep;
+    CUtensorMap mA, mB;
+    MOE_TRY(make_map(&mA, wsp<__nv_bfloat16>(ws, L.off_dsb), 1, T, n3, 128, false));
+    MOE_TRY(make_map(&mB, wsp<__nv_bfloat16>(ws, L.off_wb), 1, n3, D, 64, true));  // {D, 3Ep, 1}
+    const int64_t mtiles = ceil_div(T, kRowTile);
+    const int bn = pick_bn(D, mtiles, false, 0, false);
+    tc::Params p{};
+    p.E = 1; p.Kd = (int)n3; p.nN = D / bn; p.group_m = group_rows(n3);
+    p.dense_m = T;
+    p.out = static_cast<__nv_bfloat16*>(dx); p.ld_out = D;
+    p.dxp = static_cast<const __nv_bfloat16*>(dXp); p.No = D;
+    p.slot_row = slot_row; p.K = K; p.n_shared = c->n_shared; p.dx_offsets = offsets;
+    p.E_routed = E;
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_DX>(
+        bn, "dx_unpermute_router_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+  } else {
     dim3 g((unsigned)ceil_div(T, 64), (unsigned)ceil_div(D, 128));
     prof_begin(s);
     if (bf)

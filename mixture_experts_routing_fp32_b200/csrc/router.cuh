@@ -319,4 +319,66 @@ router_route_kernel(const float* __restrict__ logits, RouteArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Router products on tensor cores.  An fp32 value v is the sum of three bf16
+// terms up to 2^-24 |v|: hi = bf16(v), mid = bf16(v - hi), lo = bf16(v - hi
+// - mid) (each difference is exact in fp32).  With x already bf16, the
+// logits x . W_r^T are x . W_hi^T + x . W_mid^T + x . W_lo^T: bf16 MMAs
+// with fp32 accumulation give fp32-accurate logits.  Ep is E rounded up to
+// 64; split rows e >= E are zero.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void split3_bf16(float v, __nv_bfloat16& hi, __nv_bfloat16& mid,
+                                            __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(hi);
+  mid = __float2bfloat16_rn(r1);
+  lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+}
+
+// w [E,D] f32 -> wf [3 Ep, D] = (hi; mid; lo) and, if wb, wb = (hi; mid; hi)
+// (the latter pairs with (hi | hi | mid) splits of a second fp32 operand).
+__global__ void __launch_bounds__(256)
+split_w_kernel(const float* __restrict__ w, int E, int Ep, int D,
+               __nv_bfloat16* __restrict__ wf, __nv_bfloat16* __restrict__ wb) {
+  pdl_begin();
+  const int64_t n = (int64_t)Ep * D;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = i / D;
+    const float v = e < E ? w[i] : 0.f;
+    __nv_bfloat16 hi, mid, lo;
+    split3_bf16(v, hi, mid, lo);
+    if (wf != nullptr) { wf[i] = hi; wf[n + i] = mid; wf[2 * n + i] = lo; }
+    if (wb != nullptr) { wb[i] = hi; wb[n + i] = mid; wb[2 * n + i] = hi; }
+  }
+}
+
+// Routing from the three partial logit blocks of the tensor-core product
+// (parts [T, 3 Ep]: x W_hi^T | x W_mid^T | x W_lo^T): logits are summed in
+// that order, the offset added, written out, and the token routed.
+template <int NV>
+__global__ void __launch_bounds__(256)
+router_route_parts_kernel(const float* __restrict__ parts, int Ep,
+                          const float* __restrict__ offset, RouteArgs a) {
+  pdl_begin();
+  extern __shared__ __align__(16) float gsm_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* gsm = gsm_all + warp * a.E;
+  for (int t = blockIdx.x * 8 + warp; t < a.T; t += gridDim.x * 8) {
+    const float* pr = parts + (size_t)t * 3 * Ep;
+    float s[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      s[i] = -INFINITY;
+      if (e < a.E) {
+        s[i] = (pr[e] + pr[Ep + e]) + pr[2 * Ep + e];
+        if (offset != nullptr) s[i] += offset[e];
+        a.logits[(size_t)t * a.E + e] = s[i];
+      }
+    }
+    route_token<NV>(t, s, a, gsm, lane);
+  }
+}
+
 }  // namespace moe

@@ -170,10 +170,23 @@ def test_tensor_core_path_matches_simt_path(name):
     cfg = W.REDUCED[name]
     tc, inp = run_gpu(cfg, gemm_impl=0)
     simt, _ = run_gpu(cfg, gemm_impl=1, inp=inp)
-    for attr in ("y", "dx", "dw13", "dw_down", "dw_r", "dg"):
-        a, b = getattr(tc, attr).float(), getattr(simt, attr).float()
+    # both paths compute fp32-accurate logits (tensor cores on three-way
+    # bf16 splits for E >= 8, CUDA cores otherwise), in different orders
+    assert rel_l2(host(tc.logits), host(simt.logits).astype(np.float64)) < 2e-6
+    # a token may pick differently only where the exact logits nearly tie
+    flip = (tc.topk_idx != simt.topk_idx).any(dim=1).cpu().numpy()
+    if flip.any():
+        R = O.forward(oracle_layer(cfg), O.opts_of(cfg))["R"]
+        assert np.all(R.margin[flip] < O.NEAR_TIE), np.nonzero(flip)[0][:10]
+    keep = torch.from_numpy(~flip).to(tc.y.device)
+    for attr in ("y", "dx", "dg"):
+        a, b = getattr(tc, attr).float()[keep], getattr(simt, attr).float()[keep]
         assert (a - b).norm() / b.norm() < 1e-2, attr
-    assert torch.equal(tc.topk_idx, simt.topk_idx)
+    for attr in ("dw13", "dw_down", "dw_r"):
+        a, b = getattr(tc, attr).float(), getattr(simt, attr).float()
+        assert (a - b).norm() / b.norm() < (1e-2 if not flip.any() else 5e-2), attr
+    if flip.any():
+        return
     # the two paths may align expert segments differently (CTA-pair tiles
     # use 256-row segments): compare every slot's expert and rank instead
     def expert_rank(L):
