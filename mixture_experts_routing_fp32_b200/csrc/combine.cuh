@@ -64,6 +64,96 @@ combine_kernel(const T* __restrict__ o, const int32_t* __restrict__ slot_row,
   }
 }
 
+// bf16 combine for a compile-time K: one warp per token, each lane 8
+// columns of two 256-column chunks per step, with the K row loads of both
+// chunks in flight together (the row indices are read once per token and
+// broadcast).  Same fixed k order and fp32 accumulation as combine_kernel.
+template <int KT>
+__global__ void __launch_bounds__(256)
+combine_bf16_kernel(const __nv_bfloat16* __restrict__ o, const int32_t* __restrict__ slot_row,
+                    const float* __restrict__ topk_w, const int32_t* __restrict__ offsets,
+                    int n_shared, int Tn, int D, int E, __nv_bfloat16* __restrict__ y) {
+  pdl_begin();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t shared0 = n_shared ? (int64_t)offsets[E] : -1;
+  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < Tn; t += (int64_t)gridDim.x * 8) {
+    int32_t my_row = -1;
+    float my_g = 0.f;
+    if (lane < KT) {
+      my_row = slot_row[t * KT + lane];
+      my_g = topk_w[t * KT + lane];
+    }
+    int32_t rows[KT];
+    float g[KT];
+#pragma unroll
+    for (int k = 0; k < KT; ++k) {
+      rows[k] = __shfl_sync(0xffffffffu, my_row, k);
+      g[k] = __shfl_sync(0xffffffffu, my_g, k);
+    }
+    const int64_t srow = n_shared ? shared0 + t : -1;
+    for (int d0 = lane * 8; d0 < D; d0 += 512) {
+      const int d1 = d0 + 256;
+      const bool has1 = d1 < D;
+      uint4 r0[KT + 1], r1[KT + 1];
+#pragma unroll
+      for (int k = 0; k <= KT; ++k) {
+        const int64_t row = k < KT ? (int64_t)rows[k] : srow;
+        r0[k] = make_uint4(0, 0, 0, 0);
+        r1[k] = make_uint4(0, 0, 0, 0);
+        if (row >= 0) {
+          r0[k] = *reinterpret_cast<const uint4*>(o + row * D + d0);
+          if (has1) r1[k] = *reinterpret_cast<const uint4*>(o + row * D + d1);
+        }
+      }
+      float a0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float a1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < KT; ++k) {
+        if (rows[k] >= 0) {
+          float v[8];
+          const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&r0[k]);
+          const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&r1[k]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h0[i]);
+            v[2 * i] = f.x; v[2 * i + 1] = f.y;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a0[i] = fmaf(g[k], v[i], a0[i]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h1[i]);
+            v[2 * i] = f.x; v[2 * i + 1] = f.y;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a1[i] = fmaf(g[k], v[i], a1[i]);
+        }
+      }
+      if (srow >= 0) {
+        float v[8];
+        const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&r0[KT]);
+        const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&r1[KT]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(h0[i]);
+          v[2 * i] = f.x; v[2 * i + 1] = f.y;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a0[i] += v[i];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(h1[i]);
+          v[2 * i] = f.x; v[2 * i + 1] = f.y;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a1[i] += v[i];
+      }
+      store8(y + t * D + d0, a0);
+      if (has1) store8(y + t * D + d1, a1);
+    }
+  }
+}
+
 // Per permuted row: routed rows -> dg[slot] = <o[r], dy[t]> and
 // dO[r] = g * dy[t]; shared rows -> dO[r] = dy[t]; padding -> 0.
 template <typename T>
@@ -412,6 +502,64 @@ dx_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
       for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
     }
     store8(dx + t * D + d, acc[i]);
+  }
+}
+
+// bf16 dx for few experts (E <= 8) and a compile-time K: one warp per
+// token, dx_t = sum_e ds[t,e] w_r[e,:] + sum_k dX_perm[row(t,k)] (k
+// ascending) + the shared row; each lane 8 columns of a 256-column chunk,
+// every row load of a chunk in flight together.
+template <int KT>
+__global__ void __launch_bounds__(256)
+dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
+                const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__ slot_row,
+                const int32_t* __restrict__ offsets, int n_shared, int Tn, int D, int E,
+                __nv_bfloat16* __restrict__ dx) {
+  pdl_begin();
+  constexpr int kE = 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t shared0 = n_shared ? (int64_t)offsets[E] : -1;
+  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < Tn; t += (int64_t)gridDim.x * 8) {
+    int32_t my_row = -1;
+    float my_ds = 0.f;
+    if (lane < KT) my_row = slot_row[t * KT + lane];
+    if (lane < E) my_ds = ds[t * E + lane];
+    int32_t rows[KT];
+    float dse[kE];
+#pragma unroll
+    for (int k = 0; k < KT; ++k) rows[k] = __shfl_sync(0xffffffffu, my_row, k);
+#pragma unroll
+    for (int e = 0; e < kE; ++e) dse[e] = __shfl_sync(0xffffffffu, my_ds, e);
+    const int64_t srow = n_shared ? shared0 + t : -1;
+    for (int d = lane * 8; d < D; d += 256) {
+      uint4 r[KT + 1];
+#pragma unroll
+      for (int k = 0; k <= KT; ++k) {
+        const int64_t row = k < KT ? (int64_t)rows[k] : srow;
+        r[k] = row >= 0 ? *reinterpret_cast<const uint4*>(dXp + row * D + d)
+                        : make_uint4(0, 0, 0, 0);
+      }
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < kE; ++e) {
+        if (e < E) {
+          float w[8];
+          load8(w_r + (int64_t)e * D + d, w);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(dse[e], w[i], acc[i]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k <= KT; ++k) {
+        if ((k < KT && rows[k] >= 0) || (k == KT && srow >= 0)) {
+          float v[8];
+          bf16x8_to_f32(r[k], v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] += v[i];
+        }
+      }
+      store8(dx + t * D + d, acc);
+    }
   }
 }
 

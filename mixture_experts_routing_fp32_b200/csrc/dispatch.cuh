@@ -57,6 +57,7 @@ __device__ __forceinline__ int warp_count(const int (&ev)[kDispIters], int32_t* 
 #pragma unroll
   for (int it = 0; it < kDispIters; ++it) {
     const int e = ev[it];
+    if (__all_sync(0xffffffffu, e == -2)) break;   // past this warp's slots
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && (peers & lt) == 0) {
       if (shared_row) atomicAdd(&row[e], __popc(peers));

@@ -463,11 +463,10 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
         bn, "router_logits_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
     return route_launch(c, a, nullptr, parts, Ep, off, s);
   }
-  const size_t fused_smem = (size_t)c->E * c->D * 4 + 8 * (size_t)c->E * 4;
-  if (c->E <= 32 && fused_smem <= 200 * 1024) {
-    const int grid = grid_for(c->T, 2);
+  const size_t fused_smem = 8 * (size_t)c->E * 4;
+  if (c->E <= 32) {
+    const int grid = grid_for(c->T);
     auto go = [&](auto kern) -> int {
-      MOE_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fused_smem));
       prof_begin(s);
       MOE_CK((launch_k(kern, grid, 256, fused_smem, s, x, w_r, off, c->D, a)));
       MOE_LAUNCHED(s, "router_fused");
@@ -530,8 +529,13 @@ __global__ void __launch_bounds__(512)
 aux_final_kernel(const float* __restrict__ part, const int32_t* __restrict__ counts, int n_chunks,
                  int T, int E, float alpha, float lambda, float* __restrict__ losses) {
   pdl_begin();
+  // Every sum below runs in a fixed order that does not depend on timing:
+  // a warp sums one expert's chunk partials (lane-strided, then a fixed
+  // butterfly), the z partials likewise, then fixed-order block sums.
   __shared__ float red[512];
-  __shared__ float cnt_tot_s;
+  __shared__ float fp_s[kMaxExperts];
+  __shared__ float z_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   float cnt = 0.f;
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt += (float)counts[e];
   red[threadIdx.x] = cnt;
@@ -540,18 +544,20 @@ aux_final_kernel(const float* __restrict__ part, const int32_t* __restrict__ cou
     if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
     __syncthreads();
   }
-  if (threadIdx.x == 0) cnt_tot_s = red[0];
+  const float ctot = red[0];
   __syncthreads();
-  const float ctot = cnt_tot_s;
-  float acc = 0.f;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    float P = 0.f;
-    for (int c = 0; c < n_chunks; ++c) P += part[(size_t)c * (E + 1) + e];
-    P /= (float)T;
-    const float f = ctot > 0.f ? (float)counts[e] / ctot : 0.f;
-    acc += f * P;
+  for (int e = warp; e <= E; e += nw) {        // e == E: the z partials
+    float v = 0.f;
+    for (int c = lane; c < n_chunks; c += 32) v += part[(size_t)c * (E + 1) + e];
+    v = warp_sum(v);
+    if (lane == 0) {
+      if (e < E) fp_s[e] = (ctot > 0.f ? (float)counts[e] / ctot : 0.f) * (v / (float)T);
+      else z_s = v;
+    }
   }
   __syncthreads();
+  float acc = 0.f;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) acc += fp_s[e];
   red[threadIdx.x] = acc;
   __syncthreads();
   for (int o = blockDim.x / 2; o > 0; o >>= 1) {
@@ -559,10 +565,8 @@ aux_final_kernel(const float* __restrict__ part, const int32_t* __restrict__ cou
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    float z = 0.f;
-    for (int c = 0; c < n_chunks; ++c) z += part[(size_t)c * (E + 1) + E];
     losses[0] = alpha * (float)E * red[0];
-    losses[1] = lambda * z / (float)T;
+    losses[1] = lambda * z_s / (float)T;
   }
 }
 
@@ -893,6 +897,20 @@ int moe_combine(const moe_config_t* c, const void* o, const int32_t* slot_row,
   MOE_TRY(validate(c));
   if (!o || !slot_row || !topk_w || !offsets || !y) return MOE_ERR_ARG;
   const int grid = grid_for(c->T);
+  if (c->dtype == MOE_BF16 && (c->K == 1 || c->K == 2 || c->K == 4 || c->K == 8)) {
+    auto go = [&](auto kt) -> int {
+      prof_begin(s);
+      MOE_CK((launch_k(combine_bf16_kernel<decltype(kt)::value>, grid, 256, 0, s,
+                       static_cast<const __nv_bfloat16*>(o), slot_row, topk_w, offsets,
+                       c->n_shared, c->T, c->D, c->E, static_cast<__nv_bfloat16*>(y))));
+      MOE_LAUNCHED(s, "combine");
+      return MOE_OK;
+    };
+    if (c->K == 1) return go(std::integral_constant<int, 1>{});
+    if (c->K == 2) return go(std::integral_constant<int, 2>{});
+    if (c->K == 4) return go(std::integral_constant<int, 4>{});
+    return go(std::integral_constant<int, 8>{});
+  }
   prof_begin(s);
   if (c->dtype == MOE_BF16)
     MOE_CK((launch_k(combine_kernel<__nv_bfloat16>, grid, 256, 0, s,
@@ -1157,6 +1175,19 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     p.E_routed = E;
     MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_DX>(
         bn, "dx_unpermute_router_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+  } else if (bf && E <= 8 && (K == 1 || K == 2 || K == 4 || K == 8)) {
+    auto go = [&](auto kt) -> int {
+      prof_begin(s);
+      MOE_CK((launch_k(dx_small_kernel<decltype(kt)::value>, grid_for(T), 256, 0, s, ds, w_r,
+                       static_cast<const __nv_bfloat16*>(dXp), slot_row, offsets, c->n_shared,
+                       T, D, E, static_cast<__nv_bfloat16*>(dx))));
+      MOE_LAUNCHED(s, "dx_unpermute_router");
+      return MOE_OK;
+    };
+    if (K == 1) MOE_TRY(go(std::integral_constant<int, 1>{}));
+    else if (K == 2) MOE_TRY(go(std::integral_constant<int, 2>{}));
+    else if (K == 4) MOE_TRY(go(std::integral_constant<int, 4>{}));
+    else MOE_TRY(go(std::integral_constant<int, 8>{}));
   } else {
     dim3 g((unsigned)ceil_div(T, 64), (unsigned)ceil_div(D, 128));
     prof_begin(s);

@@ -184,21 +184,17 @@ __device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
 }
 
 // ---------------------------------------------------------------------------
-// E <= 32: logits and routing fused; W_r staged once per block in shared
-// memory, one warp per token, grid-stride over tokens.
+// Few experts: logits and routing fused, one warp per token, grid-stride
+// over tokens.  W_r rows are read through the read-only cache (after the
+// first touch they are L1 hits), so the x row loads start at once.
 // ---------------------------------------------------------------------------
 template <typename TX, int EB>
 __global__ void __launch_bounds__(256)
 router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
                     const float* __restrict__ offset, int D, RouteArgs a) {
   pdl_begin();
-  extern __shared__ __align__(16) float smem[];
-  float* ws = smem;                         // [E, D]
-  float* gsm_all = smem + (size_t)a.E * D;  // [8 warps, E]
+  extern __shared__ __align__(16) float gsm_all[];   // [8 warps, E]
   const int E = a.E;
-  for (int i = threadIdx.x * 4; i < E * D; i += blockDim.x * 4)
-    *reinterpret_cast<float4*>(ws + i) = *reinterpret_cast<const float4*>(w_r + i);
-  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* gsm = gsm_all + warp * E;
   for (int t = blockIdx.x * 8 + warp; t < a.T; t += gridDim.x * 8) {
@@ -212,9 +208,8 @@ router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
 #pragma unroll
       for (int e = 0; e < EB; ++e) {
         if (e < E) {
-          const float* wrow = ws + (size_t)e * D + d;
-          float4 w0 = *reinterpret_cast<const float4*>(wrow);
-          float4 w1 = *reinterpret_cast<const float4*>(wrow + 4);
+          const float4* wrow = reinterpret_cast<const float4*>(w_r + (size_t)e * D + d);
+          const float4 w0 = __ldg(wrow), w1 = __ldg(wrow + 1);
           acc[e] = fmaf(xv[0], w0.x, acc[e]); acc[e] = fmaf(xv[1], w0.y, acc[e]);
           acc[e] = fmaf(xv[2], w0.z, acc[e]); acc[e] = fmaf(xv[3], w0.w, acc[e]);
           acc[e] = fmaf(xv[4], w1.x, acc[e]); acc[e] = fmaf(xv[5], w1.y, acc[e]);
