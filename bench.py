@@ -120,8 +120,9 @@ def gemm_flops(cfg, kept_total):
 
 def hbm_bytes(cfg, kept_total, rows_used):
     """Algorithmic DRAM bytes of each memory-bound kernel for one step: every
-    operand read once and every result written once (activations in the
-    layer dtype, router tensors fp32)."""
+    distinct operand element read once (a token row gathered K times counts
+    once) and every result written once (activations in the layer dtype,
+    router tensors fp32)."""
     a = 2 if cfg.dtype == "bf16" else 4
     T, D, E, K = cfg.T, cfg.D, cfg.E, cfg.K
     M = expert_rows(cfg, kept_total)
@@ -129,9 +130,9 @@ def hbm_bytes(cfg, kept_total, rows_used):
     return {
         "router_fused": router, "router_logits": T * D * a + E * D * 4 + T * E * 4,
         "router_route": 3 * T * E * 4 + T * 4 + T * K * 8,
-        "dispatch_gather": M * D * a + rows_used * D * a,
+        "dispatch_gather": T * D * a + rows_used * D * a,
         "combine": M * D * a + T * D * a + T * K * 8,
-        "bwd_gate_grad_rows": 2 * M * D * a + rows_used * D * a + T * K * 8,
+        "bwd_gate_grad_rows": M * D * a + T * D * a + rows_used * D * a + T * K * 8,
         "dx_unpermute_router": M * D * a + T * D * a + T * E * 4 + E * D * 4,
     }
 
