@@ -134,6 +134,7 @@ def hbm_bytes(cfg, kept_total, rows_used):
         "combine": M * D * a + T * D * a + T * K * 8,
         "bwd_gate_grad_rows": M * D * a + T * D * a + rows_used * D * a + T * K * 8,
         "dx_unpermute_router": M * D * a + T * D * a + T * E * 4 + E * D * 4,
+        "dx_unpermute_sum": M * D * a + T * D * 4 + T * D * a,
     }
 
 
@@ -234,7 +235,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 def run_ours(args):
     from mixture_experts_routing_fp32_b200 import (MoELayer, config_from, moe_check_status,
-                                                   moe_launch_count)
+                                                   moe_launch_count, moe_set_side_streams)
     from mixture_experts_routing_fp32_b200.api import LaunchProfile
     from mixture_experts_routing_fp32_b200.build import build
 
@@ -322,12 +323,18 @@ def run_ours(args):
 
     # `value` comes from a graph with no measurement nodes in it; the
     # per-launch timing comes from a second graph captured with the
-    # library's begin/end events around every launch, replayed in its own
-    # timed loop below.
+    # library's begin/end events around every launch and with the side
+    # streams folded into the caller's stream, so that every launch has the
+    # GPU to itself while it is timed; it is replayed in its own loop below.
     graph = None if args.no_graph else capture()
     prof = LaunchProfile(128)
     prof.reset()
+    moe_set_side_streams(False)
+    layer.side_streams = False
     graph_prof = None if args.no_graph else capture()
+    if graph is not None:
+        moe_set_side_streams(True)
+        layer.side_streams = True
 
     def replay(g):
         if g is not None:
@@ -380,7 +387,9 @@ def run_ours(args):
                   file=sys.stderr)
     step_ms = [a.elapsed_time(b) for a, b in zip(ev0, ev1)]
     ms = statistics.mean(step_ms)
-    timing_src = "begin/end events around each launch inside timed replays of the step graph"
+    timing_src = ("begin/end events around each launch inside replays of the step graph "
+                  "captured with the backward's side streams folded into the caller's stream "
+                  "(each launch has the GPU to itself)")
     if not prof_ok or not per_launch or not per_launch[0]:
         # events recorded by graph nodes unreadable: time the same launches
         # eagerly (L2 flushed between steps) in a separate pass
@@ -395,7 +404,8 @@ def run_ours(args):
     ms_max = max_over_ranks(ms, world, dev)
     moe_check_status()
 
-    # dominant kernel (largest share of the step), its average launch time
+    # per-kernel totals per step (side-stream launches, if any were timed
+    # concurrently, are marked: their event times include GPU sharing)
     fam, side = {}, set()
     for launches in per_launch:
         for name, t, on_side in launches:
@@ -403,15 +413,15 @@ def run_ours(args):
             if on_side:
                 side.add(name)
     tot = {k: sum(v) / len(per_launch) for k, v in fam.items()}
-    # dominant kernel: largest share among launches on the caller's stream
-    # (side-stream launches share the GPU with them, so their event times
-    # include that sharing)
+    hbm, bf16, bf16_sus, peak_src = measured_peaks()
+    flops = gemm_flops(base, kept_total)
+    rows_used = int(layer.stats[2])
+    hbm_b = hbm_bytes(base, kept_total, rows_used)
+    # dominant kernel: the largest share of the step among launches timed alone
     main = {k: v for k, v in tot.items() if k not in side} or tot
     dom = max(main, key=main.get)
     n_dom = len(fam[dom]) / len(per_launch)
     dom_ms = statistics.mean(fam[dom])
-    hbm, bf16, bf16_sus, peak_src = measured_peaks()
-    flops = gemm_flops(base, kept_total)
     if dom in flops:
         achieved = flops[dom] / n_dom / (dom_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 2),
@@ -419,19 +429,21 @@ def run_ours(args):
                 "frac": round(achieved / bf16_sus, 4),
                 "peak_source": "%s bf16 dense, sustained (kernel timed inside a long step)" % peak_src}
     else:
-        roof = {"bound": "hbm", "achieved": None, "peak": hbm, "unit": "GB/s",
-                "frac": None, "peak_source": peak_src}
+        gbs = hbm_b[dom] / n_dom / (dom_ms * 1e-3) / 1e9 if dom in hbm_b else None
+        roof = {"bound": "hbm", "achieved": round(gbs, 1) if gbs else None, "peak": hbm,
+                "unit": "GB/s", "frac": round(gbs / hbm, 4) if gbs else None,
+                "peak_source": "%s copy bandwidth" % peak_src}
     roof.update({"kernel": dom, "launch_ms": round(dom_ms, 5), "timing": timing_src,
                  "launches_per_step": n_dom,
                  "traffic": recorded_traffic(dom, base.name)})
-    gemm_total_ms = sum(v for k, v in tot.items() if k.startswith("tc_") and k not in side)
-    main_flops = sum(v for k, v in flops.items() if k in tot and k not in side)
-    main_gemm_tflops = main_flops / (gemm_total_ms * 1e-3) / 1e12 if gemm_total_ms else None
+    gemm_names = sorted(k for k in flops if k in tot)
+    gemm_total_ms = sum(tot[k] for k in gemm_names)
+    gemm_tflops = (sum(flops[k] for k in gemm_names) / (gemm_total_ms * 1e-3) / 1e12
+                   if gemm_total_ms else None)
 
-    # memory-bound kernels: algorithmic bytes / live launch time vs HBM peak
-    rows_used = int(layer.stats[2])
+    # memory-bound kernels: algorithmic bytes / launch time vs HBM peak
     hbm_table = {}
-    for k, b in hbm_bytes(base, kept_total, rows_used).items():
+    for k, b in hbm_b.items():
         if k in tot and tot[k] > 0:
             gbs = b / (tot[k] * 1e-3) / 1e9
             hbm_table[k] = {"bytes": b, "ms": round(tot[k], 5), "GB/s": round(gbs, 1),
@@ -459,11 +471,11 @@ def run_ours(args):
                     "path": "Python API (MoELayer.forward/backward), eager launches"},
             "gpu_launches": launches_per_step * args.steps,
             "roofline": roof,
-            "gemm_main_stream": {
-                "tflops": round(main_gemm_tflops, 2) if main_gemm_tflops else None,
-                "frac_of_sustained": round(main_gemm_tflops / bf16_sus, 4) if main_gemm_tflops else None,
-                "ms_per_step": round(gemm_total_ms, 5),
-                "kernels": sorted(k for k in tot if k.startswith("tc_") and k not in side)},
+            "expert_gemms": {
+                "tflops": round(gemm_tflops, 2) if gemm_tflops else None,
+                "frac_of_sustained": round(gemm_tflops / bf16_sus, 4) if gemm_tflops else None,
+                "ms_per_step": round(gemm_total_ms, 5), "kernels": gemm_names,
+                "timing": "sum of the expert GEMM launches timed one by one"},
             "kernels_ms_per_step": {k + (" [side stream]" if k in side else ""): round(v, 5)
                                     for k, v in sorted(tot.items(), key=lambda kv: -kv[1])},
             "hbm_kernels": hbm_table,

@@ -288,6 +288,14 @@ int moe_last_cuda_error(void);
 int64_t moe_launch_count(int reset);
 
 /*
+ * Side streams inside moe_backward (default on).  With 0, every kernel of
+ * moe_backward runs on the caller's stream in issue order: slower, but
+ * each launch then has the GPU to itself (used to time kernels one by one).
+ * Applies to later calls from this host thread; returns the previous value.
+ */
+int moe_set_side_streams(int enable);
+
+/*
  * Per-launch timing (measurement support; not part of the layer's math).
  * While enabled, every kernel launch of this thread is bracketed by a begin
  * and an end cudaEvent recorded on the launching stream (inside a CUDA

@@ -27,7 +27,7 @@ EXPORTS = ("moe_get_sizes", "moe_router", "moe_dispatch", "moe_aux_loss",
            "moe_status_string", "moe_last_cuda_error", "moe_launch_count",
            "moe_profile_enable", "moe_profile_reset", "moe_profile_read", "moe_profile_starts",
            "moe_profile_name", "moe_profile_side", "moe_profile_disable",
-           "moe_dispatch_static")
+           "moe_dispatch_static", "moe_set_side_streams")
 
 
 class MoeConfig(ctypes.Structure):
@@ -78,6 +78,7 @@ def lib():
         "moe_last_cuda_error": [],
         "moe_launch_count": [ctypes.c_int],
         "moe_profile_enable": [ctypes.c_int],
+        "moe_set_side_streams": [ctypes.c_int],
         "moe_profile_reset": [],
         "moe_profile_read": [ctypes.POINTER(ctypes.c_float), ctypes.c_int],
         "moe_profile_starts": [ctypes.POINTER(ctypes.c_float), ctypes.c_int],

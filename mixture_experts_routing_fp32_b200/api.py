@@ -128,6 +128,11 @@ def moe_launch_count(reset: bool = False) -> int:
     return int(lib().moe_launch_count(1 if reset else 0))
 
 
+def moe_set_side_streams(enable: bool) -> bool:
+    """Side streams inside moe_backward for this thread; returns the previous setting."""
+    return bool(lib().moe_set_side_streams(1 if enable else 0))
+
+
 class LaunchProfile:
     """Per-launch CUDA-event timing of this thread's library launches."""
 
@@ -164,4 +169,4 @@ __all__ = ["LaunchProfile", "MoEError", "MoeConfig", "MoeSizes", "make_config", 
            "moe_get_sizes", "moe_router", "moe_dispatch", "moe_dispatch_static",
            "moe_aux_loss",
            "moe_expert_ffn", "moe_combine", "moe_backward", "moe_check_status",
-           "moe_launch_count"]
+           "moe_launch_count", "moe_set_side_streams"]

@@ -563,6 +563,61 @@ dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
   }
 }
 
+// bf16 dx when the router part R = ds . W_r [T, D] fp32 comes from the
+// tensor-core product: dx_t = R_t + sum_k dX_perm[row(t,k)] (k ascending) +
+// the shared row.  One warp per token, each lane 8 columns of two
+// 256-column chunks per step, every load of both chunks in flight together.
+// KT = compile-time K (0: runtime K, up to 16, one chunk per step).
+template <int KT>
+__global__ void __launch_bounds__(256)
+dx_sum_kernel(const float* __restrict__ R, const __nv_bfloat16* __restrict__ dXp,
+              const int32_t* __restrict__ slot_row, const int32_t* __restrict__ offsets,
+              int n_shared, int Tn, int D, int E, int K, __nv_bfloat16* __restrict__ dx) {
+  pdl_begin();
+  constexpr int NK = KT > 0 ? KT : 16;
+  constexpr int NC = KT > 0 ? 2 : 1;        // 256-column chunks per step
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kk = KT > 0 ? KT : K;
+  const int64_t shared0 = n_shared ? (int64_t)offsets[E] : -1;
+  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < Tn; t += (int64_t)gridDim.x * 8) {
+    const int32_t my_row = lane < kk ? slot_row[t * kk + lane] : -1;
+    int32_t rows[NK + 1];
+#pragma unroll
+    for (int k = 0; k < NK; ++k) rows[k] = __shfl_sync(0xffffffffu, my_row, k);
+    rows[NK] = n_shared ? (int32_t)(shared0 + t) : -1;
+    for (int d0 = lane * 8; d0 < D; d0 += 256 * NC) {
+      uint4 raw[NC][NK + 1];
+      float acc[NC][8];
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int d = d0 + 256 * c;
+        if (d < D) load8(R + t * D + d, acc[c]);
+#pragma unroll
+        for (int k = 0; k <= NK; ++k) {
+          raw[c][k] = make_uint4(0, 0, 0, 0);
+          if ((k < kk || k == NK) && rows[k] >= 0 && d < D)
+            raw[c][k] = *reinterpret_cast<const uint4*>(dXp + (int64_t)rows[k] * D + d);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int d = d0 + 256 * c;
+        if (d >= D) break;
+#pragma unroll
+        for (int k = 0; k <= NK; ++k) {
+          if ((k < kk || k == NK) && rows[k] >= 0) {
+            float v[8];
+            bf16x8_to_f32(raw[c][k], v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[c][i] += v[i];
+          }
+        }
+        store8(dx + t * D + d, acc[c]);
+      }
+    }
+  }
+}
+
 // dW_r from the three partial products of the tensor-core path
 // (part [3 Ep, D]: ds_hi^T x | ds_mid^T x | ds_lo^T x), summed in that order.
 __global__ void __launch_bounds__(256)

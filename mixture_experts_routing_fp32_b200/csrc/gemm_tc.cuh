@@ -20,10 +20,9 @@
 //     WGRAD mode: C_g[m, n] = sum_{r in rows(g)} A[r, m] B[r, n] (weight
 //     gradients; the reduction runs over the group's own rows and the zero
 //     padding rows beyond them contribute nothing);
-//   * dense variants (no tile map, one group) serve the router's fp32
-//     products, which run as bf16 MMAs on three-way bf16 splits of the fp32
-//     operand (x . W_r^T, ds^T . x, ds . W_r): fp32 epilogues, and a dx
-//     epilogue that adds the unpermute-sum of the expert data gradients;
+//   * dense variants (no tile map, one group, fp32 epilogues) serve the
+//     router's fp32 products, which run as bf16 MMAs on three-way bf16
+//     splits of the fp32 operand (x . W_r^T, ds^T . x, ds . W_r);
 //   * every mbarrier wait is bounded in time; on timeout the kernel records
 //     MOE_DEVERR_TIMEOUT, drains its own copies and MMAs, frees tensor
 //     memory and returns.
@@ -47,8 +46,7 @@ enum {
   EPI_SWIGLU_BWD = 2,  // da13 from dh = C and the saved a13
   EPI_WGRAD = 3,       // bf16 weight gradient per group
   EPI_F32 = 4,         // fp32 C, rows < dense_m (dense ROWS)
-  EPI_WGRAD_F32 = 5,   // fp32 C, rows < m_limit (dense WGRAD)
-  EPI_DX = 6           // dx = C + unpermute-sum of dXp rows (+ shared row), bf16
+  EPI_WGRAD_F32 = 5    // fp32 C, rows < m_limit (dense WGRAD)
 };
 
 struct Params {
@@ -72,11 +70,6 @@ struct Params {
   int dense_rows;              // WGRAD: > 0 = one group of dense_rows rows
   int m_limit;                 // WGRAD_F32: output rows
   float* out_f32; int64_t ld_f32;          // F32 epilogues
-  // EPI_DX: rows of dXp summed into each token's output row
-  const __nv_bfloat16* dxp;    // [rows, No]
-  const int32_t* slot_row;     // [dense_m, K]
-  const int32_t* dx_offsets;   // offsets[E_routed] = first shared row
-  int K, n_shared, E_routed;
 };
 
 // ----------------------------------------------------------------------------
@@ -756,45 +749,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_wait();
           u2f32(r, v);
           if (rv) store32_f32(dst + c, v);
-        }
-      } else if constexpr (EPI == EPI_DX) {
-        // this lane's token t = row0 + lane: its kept slots' rows and its
-        // shared-expert row of dXp are added to C (the router term)
-        constexpr int kDxMaxK = 16;
-        const int64_t t = row0 + lane;
-        const int64_t left = (int64_t)p.dense_m - row0;
-        const int nrows = left <= 0 ? 0 : left >= 32 ? 32 : (int)left;
-        const bool tv = t < p.dense_m;
-        int32_t rk[kDxMaxK];
-#pragma unroll
-        for (int k = 0; k < kDxMaxK; ++k)
-          rk[k] = (tv && k < p.K) ? p.slot_row[t * p.K + k] : -1;
-        const int64_t srow = (tv && p.n_shared) ? (int64_t)p.dx_offsets[p.E_routed] + t : -1;
-        __nv_bfloat16* w0 = p.out + row0 * p.ld_out + d.n0 + hh * HC;
-        const __nv_bfloat16* src = p.dxp + d.n0 + hh * HC;
-#pragma unroll
-        for (int c = 0; c < HC; c += 32) {
-          uint32_t r[32];
-          float v[32];
-          tmem_ld32(tbase + hh * HC + c, r);
-          tmem_wait();
-          u2f32(r, v);
-#pragma unroll
-          for (int k = 0; k < kDxMaxK; ++k) {
-            if (rk[k] >= 0) {
-              float g[32];
-              load32_bf16(src + (int64_t)rk[k] * p.No + c, g);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] += g[i];
-            }
-          }
-          if (srow >= 0) {
-            float g[32];
-            load32_bf16(src + srow * p.No + c, g);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] += g[i];
-          }
-          staged_store32(stg, v, w0 + c, p.ld_out, pol_out, nrows);
         }
       } else {  // EPI_SWIGLU_BWD
         __nv_bfloat16* da13 = p.out + row0 * p.ld_out + d.n0 + hh * HC;

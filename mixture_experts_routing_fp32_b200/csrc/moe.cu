@@ -162,7 +162,7 @@ struct Layout {
       off_dH, total;
   // tensor-core router products (router_tc)
   int64_t Ep;
-  size_t off_wf, off_wb, off_rparts, off_dsf, off_dsb, off_dwr3;
+  size_t off_wf, off_wb, off_rparts, off_dsf, off_dsb, off_dwr3, off_rdx;
 };
 constexpr int kAuxChunk = 128;
 
@@ -211,6 +211,7 @@ Layout layout_of(const moe_config_t* c) {
     L.off_dsf = take((size_t)c->T * 3 * L.Ep * 2);
     L.off_dsb = take((size_t)c->T * 3 * L.Ep * 2);
     L.off_dwr3 = take((size_t)3 * L.Ep * c->D * 4);
+    L.off_rdx = take((size_t)c->T * c->D * 4);
   }
   L.total = off;
   return L;
@@ -614,6 +615,7 @@ struct Side {
   bool ok = false;
 };
 thread_local Side g_side[kMaxSideDevices];
+thread_local bool g_side_enabled = true;   // moe_set_side_streams
 
 int side_streams(Side** out) {
   int dev = 0;
@@ -974,6 +976,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   Side* sd = nullptr;
   MOE_TRY(side_streams(&sd));
   cudaStream_t r = sd->st[0], w1 = sd->st[1], w2 = sd->st[2];
+  if (!g_side_enabled) r = w1 = w2 = s;
   MOE_TRY(fork_join(sd->ev[0], s, r));
   if (use_tc(c)) MOE_TRY(fork_join(sd->ev[1], s, w1));
   // 2. router backward: dlogits
@@ -1156,11 +1159,13 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     MOE_LAUNCHED(s, "router_dw_reduce");
   }
   // 8. dx = unpermute-sum(dX_perm) + shared + ds . w_r, once ds is ready;
-  // on tensor cores the router part is (ds_hi | ds_hi | ds_mid) .
-  // (W_hi; W_mid; W_hi) and the epilogue adds the dX_perm rows
+  // on tensor cores the router part R = (ds_hi | ds_hi | ds_mid) .
+  // (W_hi; W_mid; W_hi) is written in fp32 and a gather kernel adds the
+  // dX_perm rows
   MOE_CK(cudaStreamWaitEvent(s, sd->ev[6], 0));
   if (rtc) {
     const int64_t n3 = 3 * L.Ep;
+    float* R = wsp<float>(ws, L.off_rdx);
     CUtensorMap mA, mB;
     MOE_TRY(make_map(&mA, wsp<__nv_bfloat16>(ws, L.off_dsb), 1, T, n3, 128, false));
     MOE_TRY(make_map(&mB, wsp<__nv_bfloat16>(ws, L.off_wb), 1, n3, D, 64, true));  // {D, 3Ep, 1}
@@ -1169,12 +1174,22 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     tc::Params p{};
     p.E = 1; p.Kd = (int)n3; p.nN = D / bn; p.group_m = group_rows(n3);
     p.dense_m = T;
-    p.out = static_cast<__nv_bfloat16*>(dx); p.ld_out = D;
-    p.dxp = static_cast<const __nv_bfloat16*>(dXp); p.No = D;
-    p.slot_row = slot_row; p.K = K; p.n_shared = c->n_shared; p.dx_offsets = offsets;
-    p.E_routed = E;
-    MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_DX>(
-        bn, "dx_unpermute_router_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+    p.out_f32 = R; p.ld_f32 = D;
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_F32>(
+        bn, "router_dx_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+    auto go = [&](auto kt) -> int {
+      prof_begin(s);
+      MOE_CK((launch_k(dx_sum_kernel<decltype(kt)::value>, grid_for(T), 256, 0, s, R,
+                       static_cast<const __nv_bfloat16*>(dXp), slot_row, offsets, c->n_shared,
+                       T, D, E, K, static_cast<__nv_bfloat16*>(dx))));
+      MOE_LAUNCHED(s, "dx_unpermute_sum");
+      return MOE_OK;
+    };
+    if (K == 1) MOE_TRY(go(std::integral_constant<int, 1>{}));
+    else if (K == 2) MOE_TRY(go(std::integral_constant<int, 2>{}));
+    else if (K == 4) MOE_TRY(go(std::integral_constant<int, 4>{}));
+    else if (K == 8) MOE_TRY(go(std::integral_constant<int, 8>{}));
+    else MOE_TRY(go(std::integral_constant<int, 0>{}));
   } else if (bf && E <= 8 && (K == 1 || K == 2 || K == 4 || K == 8)) {
     auto go = [&](auto kt) -> int {
       prof_begin(s);
@@ -1230,6 +1245,12 @@ const char* moe_status_string(int st) {
 }
 
 int moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+int moe_set_side_streams(int enable) {
+  const int prev = g_side_enabled ? 1 : 0;
+  g_side_enabled = enable != 0;
+  return prev;
+}
 
 int moe_profile_enable(int max_launches) {
   if (max_launches < 1 || max_launches > kProfMax) return MOE_ERR_ARG;

@@ -46,6 +46,9 @@ class MoELayer:
         self._grads_ready = False
         self._inputs = None
         self._aux_stream = None
+        # aux/z losses on a side stream during the expert GEMMs (False: in
+        # order on the caller's stream)
+        self.side_streams = True
 
     def _alloc_grads(self):
         """Gradient buffers, allocated on the first backward (a forward-only
@@ -75,6 +78,9 @@ class MoELayer:
                          self.stats, self.x_perm, self.ws)
         main = torch.cuda.current_stream(self.device)
         aux = c.aux_alpha != 0.0 or c.z_lambda != 0.0
+        if aux and not self.side_streams:
+            api.moe_aux_loss(c, self.probs, self.lse, self.counts, self.losses, self.ws)
+            aux = False
         if aux:
             # the losses depend only on the router and the counts: computed
             # on a side stream while the expert GEMMs run
