@@ -155,29 +155,25 @@ combine_bf16_kernel(const __nv_bfloat16* __restrict__ o, const int32_t* __restri
 }
 
 // Per permuted row: routed rows -> dg[slot] = <o[r], dy[t]> and
-// dO[r] = g * dy[t]; shared rows -> dO[r] = dy[t]; padding -> 0.
+// dO[r] = g * dy[t]; shared rows -> dO[r] = dy[t]; padding -> 0.  A row's
+// kind is decided by row_slot alone (the dispatch sets -1 on padding and
+// shared rows), so each warp's chain is one index load then the row work.
 template <typename T>
 __global__ void __launch_bounds__(256)
 bwd_rows_kernel(const T* __restrict__ o, const T* __restrict__ dy,
                 const float* __restrict__ topk_w, const int32_t* __restrict__ row_slot,
-                const int32_t* __restrict__ offsets, const int32_t* __restrict__ kept,
-                const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ stats,
+                const int32_t* __restrict__ offsets, const int32_t* __restrict__ stats,
                 int K, int E, int Tn, int D, float* __restrict__ dg_slot,
                 T* __restrict__ dO) {
   pdl_begin();
   const int n_rows = stats[2];
+  const int64_t shared0 = offsets[E];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t r = (int64_t)blockIdx.x * 8 + warp; r < n_rows; r += (int64_t)gridDim.x * 8) {
-    const int e = tile_expert[r / kRowTile];
-    int64_t t = -1, slot = -1;
-    if (e < E) {
-      if (r - offsets[e] < kept[e]) {
-        slot = row_slot[r];
-        t = slot / K;
-      }
-    } else if (r - offsets[E] < Tn) {
-      t = r - offsets[E];
-    }
+    const int64_t slot = row_slot[r];
+    int64_t t = -1;
+    if (slot >= 0) t = slot / K;
+    else if (r >= shared0 && r - shared0 < Tn) t = r - shared0;
     T* dst = dO + r * D;
     if (t < 0) {
       for (int d = lane * 8; d < D; d += 256) zero8(dst + d);

@@ -109,7 +109,7 @@ __device__ void finish_layout(const int32_t* tot, int32_t* seg, int E, int T, in
                               int64_t C, int64_t rows_max, int align, int32_t sentinels,
                               int32_t* __restrict__ counts, int32_t* __restrict__ kept,
                               int32_t* __restrict__ offsets, int32_t* __restrict__ tile_expert,
-                              int32_t* __restrict__ stats) {
+                              int32_t* __restrict__ stats, int32_t* __restrict__ row_slot) {
   __shared__ unsigned long long drop_s;
   __shared__ int32_t total_s;
   if (threadIdx.x == 0) drop_s = 0;
@@ -161,6 +161,15 @@ __device__ void finish_layout(const int32_t* tot, int32_t* seg, int E, int T, in
     if (e < E) offsets[e] = (int32_t)beg;
     for (int64_t r = beg; r < end && r < total; r += kRowTile) tile_expert[r / kRowTile] = e;
   }
+  // rows that hold no routed slot (each expert's padding, the shared
+  // expert's rows) get row_slot = -1; the rank pass fills the others
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int e = warp; e < E; e += nw) {
+    const int32_t k = (C >= 0 && tot[e] > C) ? (int32_t)C : tot[e];
+    const int64_t end = seg[e + 1] < total ? (int64_t)seg[e + 1] : total;
+    for (int64_t r = seg[e] + k + lane; r < end; r += 32) row_slot[r] = -1;
+  }
+  for (int64_t r = (int64_t)seg[E] + threadIdx.x; r < total; r += blockDim.x) row_slot[r] = -1;
   __syncthreads();
 }
 
@@ -194,7 +203,8 @@ disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ b
                  int n_blocks, int E, int T, int n_shared, int64_t C,
                  int64_t rows_max, int align, int32_t* __restrict__ counts,
                  int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
-                 int32_t* __restrict__ tile_expert, int32_t* __restrict__ stats) {
+                 int32_t* __restrict__ tile_expert, int32_t* __restrict__ stats,
+                 int32_t* __restrict__ row_slot) {
   pdl_begin();
   extern __shared__ int32_t sh[];     // tot[E], seg[E + 1]
   int32_t* tot = sh;
@@ -217,7 +227,7 @@ disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ b
   if (ls) atomicAdd(&sent_total, ls);
   __syncthreads();
   finish_layout(tot, seg, E, T, n_shared, C, rows_max, align, sent_total, counts, kept, offsets,
-                tile_expert, stats);
+                tile_expert, stats, row_slot);
 }
 
 // Pass 3: stable rank of every slot inside its expert, capacity drop,
@@ -291,32 +301,28 @@ disp_small_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ m
   }
   __syncthreads();
   finish_layout(tot, seg, E, T, n_shared, C, rows_max, align, sent_total, counts, kept, offsets,
-                tile_expert, stats);
+                tile_expert, stats, row_slot);
   warp_rank(ev, j0, n_slots, C, rows_max, wh + warp * E, seg, slot_row, row_slot);
 }
 
 // Pass 4: gather x rows into expert order; zero padding rows; shared rows.
+// A row's source is decided by row_slot alone (-1: padding below the shared
+// segment, or a shared row), so each warp's chain is one index load then
+// the row copy.
 template <typename TX>
 __global__ void __launch_bounds__(256)
 disp_gather_kernel(const TX* __restrict__ x, int D, int K, int E, int T,
-                   const int32_t* __restrict__ offsets, const int32_t* __restrict__ kept,
-                   const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ stats,
-                   int32_t* __restrict__ row_slot, TX* __restrict__ x_perm) {
+                   const int32_t* __restrict__ offsets, const int32_t* __restrict__ stats,
+                   const int32_t* __restrict__ row_slot, TX* __restrict__ x_perm) {
   pdl_begin();
   const int n_rows = stats[2];
+  const int64_t shared0 = offsets[E];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t r = (int64_t)blockIdx.x * 8 + warp; r < n_rows; r += (int64_t)gridDim.x * 8) {
-    const int e = tile_expert[r / kRowTile];
+    const int32_t slot = row_slot[r];
     int64_t src = -1;
-    if (e < E) {
-      const int64_t local = r - offsets[e];
-      if (local < kept[e]) src = row_slot[r] / K;
-      else if (lane == 0) row_slot[r] = -1;
-    } else {
-      const int64_t t = r - offsets[E];
-      if (t < T) src = t;
-      if (lane == 0) row_slot[r] = -1;
-    }
+    if (slot >= 0) src = slot / K;
+    else if (r >= shared0 && r - shared0 < T) src = r - shared0;
     TX* dst = x_perm + r * D;
     if (src >= 0) {
       const TX* s = x + src * D;

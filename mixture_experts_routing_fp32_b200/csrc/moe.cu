@@ -688,7 +688,7 @@ int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_id
     prof_begin(s);
     MOE_CK((launch_k(disp_scan_kernel, 1, 1024, (2 * E + 1) * sizeof(int32_t), s, bhist, bsent,
                      L.n_disp_blocks, E, c->T, c->n_shared, L.C, L.rows_max, L.align, counts,
-                     kept, offsets, tile_expert, stats)));
+                     kept, offsets, tile_expert, stats, row_slot)));
     MOE_LAUNCHED(s, "dispatch_scan");
     prof_begin(s);
     MOE_CK((launch_k(disp_rank_kernel, L.n_disp_blocks, 256,
@@ -700,11 +700,11 @@ int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_id
   prof_begin(s);
   if (c->dtype == MOE_BF16)
     MOE_CK((launch_k(disp_gather_kernel<__nv_bfloat16>, grid, 256, 0, s,
-                     static_cast<const __nv_bfloat16*>(x), c->D, c->K, E, c->T, offsets, kept,
-                     tile_expert, stats, row_slot, static_cast<__nv_bfloat16*>(x_perm))));
+                     static_cast<const __nv_bfloat16*>(x), c->D, c->K, E, c->T, offsets, stats,
+                     row_slot, static_cast<__nv_bfloat16*>(x_perm))));
   else
     MOE_CK((launch_k(disp_gather_kernel<float>, grid, 256, 0, s, static_cast<const float*>(x),
-                     c->D, c->K, E, c->T, offsets, kept, tile_expert, stats, row_slot,
+                     c->D, c->K, E, c->T, offsets, stats, row_slot,
                      static_cast<float*>(x_perm))));
   MOE_LAUNCHED(s, "dispatch_gather");
   return MOE_OK;
@@ -960,12 +960,11 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     if (bf)
       MOE_CK((launch_k(bwd_rows_kernel<__nv_bfloat16>, grid, 256, 0, s,
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dy), topk_w,
-          row_slot, offsets, kept, tile_expert, stats, K, E, T, D, dg,
-          static_cast<__nv_bfloat16*>(dO))));
+          row_slot, offsets, stats, K, E, T, D, dg, static_cast<__nv_bfloat16*>(dO))));
     else
       MOE_CK((launch_k(bwd_rows_kernel<float>, grid, 256, 0, s,
           static_cast<const float*>(o), static_cast<const float*>(dy), topk_w, row_slot, offsets,
-          kept, tile_expert, stats, K, E, T, D, dg, static_cast<float*>(dO))));
+          stats, K, E, T, D, dg, static_cast<float*>(dO))));
     MOE_LAUNCHED(s, "bwd_gate_grad_rows");
   }
   // The router gradient chain (2, 7) runs on side stream r, concurrently
