@@ -34,6 +34,8 @@ from typing import Callable, Optional
 
 import numpy as np
 
+from . import balance
+
 SOFTMAX, SIGMOID = 0, 1
 GROUP_MAX, GROUP_TOP2SUM = 0, 1
 NEAR_TIE = 1e-5          # fp32-margin below which a top-k decision is a near-tie
@@ -358,6 +360,7 @@ class Opts:
     route_scale: float = 1.0
     aux_alpha: float = 0.0
     z_lambda: float = 0.0
+    seq_len: int = 0             # > 0: the aux loss is sequence-wise (oracle/balance.py)
     logits_fp32: bool = True     # False only for finite-difference checks
 
 
@@ -368,7 +371,8 @@ def opts_of(cfg) -> Opts:
                 group_score=cfg.group_score,
                 capacity_factor=cfg.capacity_factor,
                 min_capacity=cfg.min_capacity, route_scale=cfg.route_scale,
-                aux_alpha=cfg.aux_alpha, z_lambda=cfg.z_lambda)
+                aux_alpha=cfg.aux_alpha, z_lambda=cfg.z_lambda,
+                seq_len=getattr(cfg, "seq_len", 0))
 
 
 def route_layer(L: Layer, o: Opts) -> Routing:
@@ -418,7 +422,12 @@ def forward(L: Layer, o: Opts):
     if L.w13_s is not None:
         shared = swiglu_forward(x, L.w13_s, L.wd_s)
         y += shared[3]
-    laux, f, P = aux_loss(Dp.counts, R.p, o.aux_alpha, E) if o.aux_alpha else (0.0, None, None)
+    if o.aux_alpha and o.seq_len:
+        laux, f, P = balance.seq_aux_loss(R.p, Dp.expert, K, o.aux_alpha, o.seq_len, o.score_fn)
+    elif o.aux_alpha:
+        laux, f, P = aux_loss(Dp.counts, R.p, o.aux_alpha, E)
+    else:
+        laux, f, P = 0.0, None, None
     lz = z_loss(R.lse, o.z_lambda) if o.z_lambda else 0.0
     return dict(R=R, Dp=Dp, slot_act=slot_act, o_slot=o_slot, y=y,
                 shared=shared, aux=laux, z=lz, f=f, P=P)
@@ -444,7 +453,7 @@ def gate_grad(o_slot, dy, Dp: Dispatch, K, sentinel_unmasked=None):
     return dg.reshape(T, K)
 
 
-def router_backward(R: Routing, dg, o: Opts, counts=None, T_total=None):
+def router_backward(R: Routing, dg, o: Opts, counts=None, T_total=None, seq_f=None):
     """dL/dlogits from the gate path, the aux loss and the z-loss.
 
     Gate path ([STA324] §8.3: with the selected set fixed, g is differentiable
@@ -456,7 +465,9 @@ def router_backward(R: Routing, dg, o: Opts, counts=None, T_total=None):
       B sigmoid: g_k = rs*p_k/S, S = sum_sel p + eps:
                  dp_k = rs/S * (dg_k - sum_j dg_j g_j / rs), ds = dp p (1-p)
       A sigmoid: dp_k = rs * dg_k, ds = dp p (1-p)
-    Aux ([STA324] §8.5): dL/dp_{t,e} = alpha E f_e / T, f held constant.
+    Aux ([STA324] §8.5): dL/dp_{t,e} = alpha E f_e / T, f held constant;
+    sequence-wise aux (o.seq_len > 0, per-sequence f in seq_f): see
+    oracle/balance.py.
     z ([8MOE] ST-MoE): dL/ds_{t,e} = 2 lambda lse_t softmax(s_t)_e / T.
     The hot-spot offset and the selection bias receive no gradient.
     """
@@ -476,7 +487,9 @@ def router_backward(R: Routing, dg, o: Opts, counts=None, T_total=None):
         dp = np.zeros((T, E))
         if not o.renorm:
             np.add.at(dp, (np.repeat(rows, K, axis=1), idx), rs * dgv)
-        if o.aux_alpha:
+        if o.aux_alpha and o.seq_len:
+            dp += balance.seq_aux_grad_scores(p, seq_f, o.aux_alpha, o.seq_len, SOFTMAX)
+        elif o.aux_alpha:
             cnt = f64(counts)
             f = cnt / cnt.sum() if cnt.sum() > 0 else np.zeros(E)
             dp += o.aux_alpha * E * f[None, :] / Tn
@@ -497,8 +510,10 @@ def router_backward(R: Routing, dg, o: Opts, counts=None, T_total=None):
             dpk = rs * dgv
         dsk = np.where(valid, dpk * sel * (1.0 - sel), 0.0)
         np.add.at(ds, (np.repeat(rows, K, axis=1), idx), dsk)
-        if o.aux_alpha:
-            raise ValueError("aux loss is defined for softmax scores only")
+        if o.aux_alpha and o.seq_len:
+            ds += balance.seq_aux_grad_scores(R.p, seq_f, o.aux_alpha, o.seq_len, SIGMOID)
+        elif o.aux_alpha:
+            raise ValueError("the batch aux loss is defined for softmax scores only")
     if o.z_lambda:
         ds += 2.0 * o.z_lambda * R.lse[:, None] * softmax_rows(s) / Tn
     return ds
@@ -536,7 +551,7 @@ def backward(L: Layer, o: Opts, fw, dy, sentinel_unmasked=None):
         a, b, h, _ = fw["shared"]
         dxs, dw13_s, dwd_s = swiglu_backward(x, a, b, h, dy, L.w13_s, L.wd_s)
         dx += dxs
-    ds = router_backward(R, dg, o, Dp.counts)
+    ds = router_backward(R, dg, o, Dp.counts, seq_f=fw["f"] if o.seq_len else None)
     dw_r = ds.T @ x
     dx += ds @ f64(L.w_r)
     return dict(dx=dx, dw_r=dw_r, dw13=dw13, dwd=dwd, dw13_s=dw13_s,

@@ -75,7 +75,9 @@ def test_fd_tiny_config():
 @pytest.mark.parametrize("variant", ["A_aux_z_sentinel_capacity",
                                      "B_capacity_hotspot",
                                      "sigmoid_groups_shared",
-                                     "sigmoid_A_top2sum"])
+                                     "sigmoid_A_top2sum",
+                                     "A_seq_aux",
+                                     "sigmoid_B_seq_aux_groups"])
 def test_fd_feature_configs(variant):
     base = W.CONFIGS["tiny"].replace(T=48, D=16, E=8, K=2, F=24, dtype="fp32")
     cfg = {
@@ -91,6 +93,13 @@ def test_fd_feature_configs(variant):
         "sigmoid_A_top2sum": base.replace(
             score_fn=W.SIGMOID, renorm=0, n_groups=4, topk_groups=3,
             group_score=W.GROUP_TOP2SUM, sel_bias_range=0.1),
+        # sequence-wise aux loss (3 sequences of 16 tokens), softmax and
+        # sigmoid scores, with sentinels / groups
+        "A_seq_aux": base.replace(
+            renorm=0, aux_alpha=0.2, seq_len=16, sentinel_frac=0.1),
+        "sigmoid_B_seq_aux_groups": base.replace(
+            score_fn=W.SIGMOID, renorm=1, n_groups=4, topk_groups=2,
+            sel_bias_range=0.1, aux_alpha=0.2, seq_len=16),
     }[variant]
     cfg = cfg.replace(w_std=0.3)   # larger logits: routing decisions matter
     assert _fd_check(cfg) > 30

@@ -48,6 +48,7 @@ class LayerConfig:
     route_scale: float = 1.0
     aux_alpha: float = 0.0
     z_lambda: float = 0.0
+    seq_len: int = 0            # > 0: sequence-wise aux loss over seq_len tokens
     # input recipe
     seed: int = 0
     x_std: float = 1.0
