@@ -50,6 +50,11 @@ def parse():
     ap.add_argument("--config", default="mm_b", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="sequence-wise aux loss over groups of this many tokens")
+    ap.add_argument("--aux-alpha", type=float, default=None)
+    ap.add_argument("--bias-gamma", type=float, default=0.0,
+                    help="selection-bias update step after each forward (sigmoid routing)")
     ap.add_argument("--timeline", action="store_true",
                     help="print one profiled step's launch timeline to stderr")
     ap.add_argument("--cpu-sample-s", type=float, default=10.0)
@@ -250,6 +255,10 @@ def run_ours(args):
         base = base.replace(T=args.tokens)
     if args.experts:
         base = base.replace(E=args.experts)
+    if args.seq_len:
+        base = base.replace(seq_len=args.seq_len)
+    if args.aux_alpha is not None:
+        base = base.replace(aux_alpha=args.aux_alpha)
     cfg = rank_config(base, rank)
     names = ("x", "w_r", "w13", "w_down", "dy")
     inp = {n: W.make_input(cfg if n in ("x", "dy") else base, n, dev) for n in names}
@@ -268,6 +277,8 @@ def run_ours(args):
 
     def step():
         layer.forward(x, **weights)
+        if args.bias_gamma and weights.get("sel_bias") is not None:
+            layer.update_bias(weights["sel_bias"], args.bias_gamma)
         layer.backward(dy)
 
     # warm-up (eager), then capture one step in a CUDA graph with per-launch events
@@ -299,6 +310,8 @@ def run_ours(args):
         dx_dev.copy_(hx, non_blocking=True)
         ddy.copy_(hdy, non_blocking=True)
         layer.forward(dx_dev, **weights)
+        if args.bias_gamma and weights.get("sel_bias") is not None:
+            layer.update_bias(weights["sel_bias"], args.bias_gamma)
         layer.backward(ddy)
         hy.copy_(layer.y, non_blocking=True)
         hdx.copy_(layer.dx, non_blocking=True)
@@ -458,9 +471,11 @@ def run_ours(args):
             "ms_per_step": round(ms_max, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if base.dtype == "bf16" else "f32",
             "data": "synthetic (seeded counter-hash normals; shapes of the MiniMind-shaped layer)",
-            "config": {"workload": "%s: T=%d D=%d E=%d K=%d F=%d %s variant %s aux %.0e" % (
+            "config": {"workload": "%s: T=%d D=%d E=%d K=%d F=%d %s variant %s aux %.0e%s%s" % (
                 base.name, base.T, base.D, base.E, base.K, base.F, base.dtype,
-                "B" if base.renorm else "A", base.aux_alpha),
+                "B" if base.renorm else "A", base.aux_alpha,
+                " sequence-wise over %d tokens" % base.seq_len if base.seq_len else "",
+                " bias update gamma %g" % args.bias_gamma if args.bias_gamma else ""),
                 "global_batch_tokens": base.T * world, "parallelism": "dp%d (replicas)" % world,
                 "l2": "flushed between timed steps (256 MiB write)",
                 "cuda_graph": graph is not None,

@@ -81,8 +81,14 @@ enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SIMT = 1 };   /* cfg.gemm_impl */
  *              C = max(ceil(c*T*K/E), min_capacity); c <= 0: no limit.
  *              [STA324 §8.5], [8MOE] Expert Capacity
  *   route_scale multiplies g after renormalisation               [TRAIN]
- *   aux_alpha  Switch load-balance loss alpha*E*sum_e f_e P_e; softmax only
- *              [STA324 §8.5], [TRAIN]
+ *   aux_alpha  Switch load-balance loss alpha*E*sum_e f_e P_e
+ *              [STA324 §8.5], [TRAIN]; over the whole batch (softmax
+ *              scores only) or, with seq_len > 0, per sequence
+ *   seq_len    > 0: sequence-wise aux loss, the same loss on each group of
+ *              seq_len consecutive tokens, averaged over the groups; with
+ *              sigmoid scores P uses the affinities divided by their sum
+ *              over experts [STA324 §8.6], [TRAIN] (DeepSeek-V3's
+ *              complementary sequence-wise term); seq_len divides T
  *   z_lambda   router z-loss lambda*mean_t lse_t^2           [8MOE] ST-MoE
  *   n_shared   0 or 1: a shared SwiGLU expert on every token, weight 1,
  *              no top-K slot                                 [STA324 §8.7]
@@ -101,6 +107,8 @@ typedef struct {
   int32_t min_capacity;
   float route_scale, aux_alpha, z_lambda;
   int32_t gemm_impl;
+  int32_t seq_len;      /* 0: batch aux loss; > 0: sequence-wise aux loss over
+                           consecutive groups of seq_len tokens (divides T) */
 } moe_config_t;
 
 typedef struct {
@@ -151,7 +159,8 @@ int moe_router(const moe_config_t* cfg, const void* x, const float* w_r,
  *   counts        [E] i32 out: valid slots per expert before drops
  *   kept          [E] i32 out: min(counts, C)
  *   offsets       [E+2] i32 out: permuted-row offsets (see header)
- *   slot_row      [T*K] i32 out: row of each slot, -1 if sentinel/dropped
+ *   slot_row      [T*K] i32 out: row of each slot, -1 if dropped, -2 if
+ *                 sentinel
  *   row_slot      [rows_max] i32 out: slot of each routed row, -1 otherwise
  *   tile_expert   [tiles_max] i32 out: expert of each 128-row tile (E = shared)
  *   stats         [4] i32 out: n_dropped, n_sentinel, n_rows, n_tiles
@@ -204,6 +213,30 @@ int moe_dispatch_static(const moe_config_t* cfg, const int32_t* topk_idx,
 int moe_aux_loss(const moe_config_t* cfg, const float* probs, const float* lse,
                  const int32_t* counts, float* losses, void* ws,
                  cudaStream_t stream);
+
+/*
+ * moe_aux_loss_seq — the sequence-wise aux loss (cfg.seq_len > 0):
+ * losses[0] = alpha*E*mean_s sum_e f_{s,e} P_{s,e}, f_{s,e} = share of
+ * sequence s's valid (non-sentinel, pre-drop) slots that chose e, P_{s,e} =
+ * mean over its tokens of probs (softmax) or of probs / sum_e probs
+ * (sigmoid affinities); losses[1] as in moe_aux_loss.  [STA324 §8.5, §8.6],
+ * [TRAIN].  topk_idx and slot_row from moe_router / moe_dispatch (slot_row
+ * -2 marks sentinels).  Deterministic; MOE_ERR_ARG if seq_len == 0.
+ */
+int moe_aux_loss_seq(const moe_config_t* cfg, const float* probs, const float* lse,
+                     const int32_t* topk_idx, const int32_t* slot_row, float* losses,
+                     void* ws, cudaStream_t stream);
+
+/*
+ * moe_bias_update — the selection-bias load-control step of sigmoid
+ * routing: sel_bias[e] -= gamma * sign(counts[e] - mean(counts)) in place
+ * (overloaded experts' bias goes down, underloaded ones' up; the sign is
+ * taken exactly, on counts[e]*E - sum(counts)).  [STA324 §8.6], [TRAIN]
+ * (DeepSeek-V3's dynamic expert bias).  counts from moe_dispatch (valid
+ * slots, pre-drop); sel_bias [E] f32 in/out.
+ */
+int moe_bias_update(const moe_config_t* cfg, const int32_t* counts, float* sel_bias,
+                    float gamma, cudaStream_t stream);
 
 /*
  * moe_expert_ffn — grouped SwiGLU experts over the permuted rows.

@@ -27,7 +27,8 @@ EXPORTS = ("moe_get_sizes", "moe_router", "moe_dispatch", "moe_aux_loss",
            "moe_status_string", "moe_last_cuda_error", "moe_launch_count",
            "moe_profile_enable", "moe_profile_reset", "moe_profile_read", "moe_profile_starts",
            "moe_profile_name", "moe_profile_side", "moe_profile_disable",
-           "moe_dispatch_static", "moe_set_side_streams")
+           "moe_dispatch_static", "moe_set_side_streams", "moe_aux_loss_seq",
+           "moe_bias_update")
 
 
 class MoeConfig(ctypes.Structure):
@@ -37,7 +38,7 @@ class MoeConfig(ctypes.Structure):
                 ("topk_groups", c_int32), ("group_score", c_int32),
                 ("capacity_factor", c_float), ("min_capacity", c_int32),
                 ("route_scale", c_float), ("aux_alpha", c_float),
-                ("z_lambda", c_float), ("gemm_impl", c_int32)]
+                ("z_lambda", c_float), ("gemm_impl", c_int32), ("seq_len", c_int32)]
 
 
 class MoeSizes(ctypes.Structure):
@@ -86,6 +87,8 @@ def lib():
         "moe_profile_side": [ctypes.c_int],
         "moe_profile_disable": [],
         "moe_dispatch_static": [cfg, P, P, P, P, P, P, P, P, P, P, P, P],
+        "moe_aux_loss_seq": [cfg, P, P, P, P, P, P, P],
+        "moe_bias_update": [cfg, P, P, ctypes.c_float, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)

@@ -26,7 +26,7 @@ def _s(stream=None):
 def make_config(T, D, E, K, F, *, n_shared=0, dtype="bf16", score_fn=0,
                 renorm=1, n_groups=1, topk_groups=1, group_score=0,
                 capacity_factor=0.0, min_capacity=0, route_scale=1.0,
-                aux_alpha=0.0, z_lambda=0.0, gemm_impl=0) -> MoeConfig:
+                aux_alpha=0.0, z_lambda=0.0, gemm_impl=0, seq_len=0) -> MoeConfig:
     return MoeConfig(
         T=T, D=D, E=E, K=K, F=F, n_shared=n_shared,
         dtype=C.MOE_BF16 if dtype in ("bf16", torch.bfloat16) else C.MOE_FP32,
@@ -34,14 +34,14 @@ def make_config(T, D, E, K, F, *, n_shared=0, dtype="bf16", score_fn=0,
         topk_groups=topk_groups, group_score=group_score,
         capacity_factor=capacity_factor, min_capacity=min_capacity,
         route_scale=route_scale, aux_alpha=aux_alpha, z_lambda=z_lambda,
-        gemm_impl=gemm_impl)
+        gemm_impl=gemm_impl, seq_len=seq_len)
 
 
 def config_from(obj, **over) -> MoeConfig:
     """MoeConfig from any object carrying the layer fields by name."""
     names = ("n_shared", "dtype", "score_fn", "renorm", "n_groups",
              "topk_groups", "group_score", "capacity_factor", "min_capacity",
-             "route_scale", "aux_alpha", "z_lambda")
+             "route_scale", "aux_alpha", "z_lambda", "seq_len")
     kw = {n: getattr(obj, n) for n in names if hasattr(obj, n)}
     kw.update(over)
     return make_config(obj.T, obj.D, obj.E, obj.K, obj.F, **kw)
@@ -80,6 +80,17 @@ def moe_dispatch_static(cfg, topk_idx, sentinel_mask, x, counts, kept, offsets,
                                     _p(slot_row), _p(row_slot), _p(tile_expert),
                                     _p(stats), _p(x_perm), _s(stream)),
           "moe_dispatch_static")
+
+
+def moe_aux_loss_seq(cfg, probs, lse, topk_idx, slot_row, losses, ws, stream=None):
+    check(lib().moe_aux_loss_seq(ctypes.byref(cfg), _p(probs), _p(lse), _p(topk_idx),
+                                 _p(slot_row), _p(losses), _p(ws), _s(stream)),
+          "moe_aux_loss_seq")
+
+
+def moe_bias_update(cfg, counts, sel_bias, gamma, stream=None):
+    check(lib().moe_bias_update(ctypes.byref(cfg), _p(counts), _p(sel_bias),
+                                ctypes.c_float(gamma), _s(stream)), "moe_bias_update")
 
 
 def moe_aux_loss(cfg, probs, lse, counts, losses, ws, stream=None):
@@ -169,4 +180,5 @@ __all__ = ["LaunchProfile", "MoEError", "MoeConfig", "MoeSizes", "make_config", 
            "moe_get_sizes", "moe_router", "moe_dispatch", "moe_dispatch_static",
            "moe_aux_loss",
            "moe_expert_ffn", "moe_combine", "moe_backward", "moe_check_status",
-           "moe_launch_count", "moe_set_side_streams"]
+           "moe_launch_count", "moe_set_side_streams", "moe_aux_loss_seq",
+           "moe_bias_update"]

@@ -215,6 +215,9 @@ struct RouterBwdArgs {
   float* ds;               // [T,E]
   float* dlogits_out;      // [T,E] or null
   float* dg_out;           // [T,K] or null
+  // sequence-wise aux (seq_len > 0): f[s][e] per sequence
+  int seq_len;
+  const float* seq_f;
   // bf16 splits of ds for the tensor-core router products (or null):
   // dsf [T, 3 Ep] = (hi | mid | lo), dsb [T, 3 Ep] = (hi | hi | mid)
   __nv_bfloat16* dsf;
@@ -259,9 +262,14 @@ router_bwd_kernel(RouterBwdArgs a) {
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int e = lane + 32 * i;
-        dp[i] = (a.aux_alpha != 0.f && e < E && cnt_tot > 0.f)
-                    ? a.aux_alpha * (float)E * ((float)a.counts[e] / cnt_tot) / (float)a.T
-                    : 0.f;
+        if (a.aux_alpha != 0.f && a.seq_len > 0)
+          dp[i] = e < E ? a.aux_alpha * (float)E * a.seq_f[(t / a.seq_len) * E + e] /
+                              (float)a.T
+                        : 0.f;
+        else
+          dp[i] = (a.aux_alpha != 0.f && e < E && cnt_tot > 0.f)
+                      ? a.aux_alpha * (float)E * ((float)a.counts[e] / cnt_tot) / (float)a.T
+                      : 0.f;
       }
       if (!a.renorm) {
 #pragma unroll
@@ -315,6 +323,25 @@ router_bwd_kernel(RouterBwdArgs a) {
           for (int i = 0; i < NV; ++i) if (i == (ik[k] >> 5)) ds[i] += add;
         }
       }
+    }
+    if (a.score_fn != MOE_SOFTMAX && a.aux_alpha != 0.f && a.seq_len > 0) {
+      // sequence-wise aux on q = sigma / sum sigma: dq = alpha E f / T,
+      // dsigma = (dq - <dq, q>) / sum sigma, ds += dsigma sigma (1 - sigma)
+      float S = 0.f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) S += p[i];
+      S = warp_sum(S);
+      float dq[NV], inner = 0.f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int e = lane + 32 * i;
+        dq[i] = e < E ? a.aux_alpha * (float)E * a.seq_f[(t / a.seq_len) * E + e] / (float)a.T
+                      : 0.f;
+        inner += dq[i] * (p[i] / S);
+      }
+      inner = warp_sum(inner);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) ds[i] += (dq[i] - inner) / S * p[i] * (1.f - p[i]);
     }
     if (a.z_lambda != 0.f) {
       const float l = a.lse[t];
@@ -498,6 +525,153 @@ dx_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
       for (int j = 0; j < 8; ++j) acc[i][j] += v[j];
     }
     store8(dx + t * D + d, acc[i]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Sequence-wise aux loss and the selection-bias update ([STA324] §8.5-§8.6,
+// [TRAIN]).  One block per sequence of S tokens; every sum runs in a fixed
+// order (per-warp token strides, then warps in order), so results do not
+// depend on timing.
+// ---------------------------------------------------------------------------
+// counts of sequence s per expert (valid slots: slot_row != -2, pre-drop)
+__device__ void seq_counts_block(const int32_t* __restrict__ topk_idx,
+                                 const int32_t* __restrict__ slot_row, int64_t s, int S, int K,
+                                 int E, int32_t* cnt_s) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = 0;
+  __syncthreads();
+  const int64_t j0 = s * S * (int64_t)K, j1 = j0 + (int64_t)S * K;
+  for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+    const int e = topk_idx[j];
+    if (slot_row[j] != -2 && e >= 0 && e < E) atomicAdd(&cnt_s[e], 1);
+  }
+  __syncthreads();
+}
+
+// f[s][e] = n_{s,e} / sum_e n_{s,e}
+__global__ void __launch_bounds__(256)
+seq_f_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ slot_row,
+             int S, int K, int E, float* __restrict__ f) {
+  pdl_begin();
+  __shared__ int32_t cnt_s[kMaxExperts];
+  __shared__ int32_t tot_s;
+  seq_counts_block(topk_idx, slot_row, blockIdx.x, S, K, E, cnt_s);
+  if (threadIdx.x == 0) {
+    int32_t t = 0;
+    for (int e = 0; e < E; ++e) t += cnt_s[e];
+    tot_s = t;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    f[(size_t)blockIdx.x * E + e] = tot_s > 0 ? (float)cnt_s[e] / (float)tot_s : 0.f;
+}
+
+// Per sequence: part[s] = sum_e f_{s,e} P_{s,e} and zpart[s] = sum_t lse_t^2.
+// q = probs (softmax) or probs / sum_e probs (sigmoid); lane l of a warp
+// holds experts l + 32 i.
+template <int NV>
+__global__ void __launch_bounds__(256)
+seq_aux_kernel(const float* __restrict__ probs, const float* __restrict__ lse,
+               const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ slot_row,
+               int S, int K, int E, int normalise, float* __restrict__ part,
+               float* __restrict__ zpart) {
+  pdl_begin();
+  __shared__ int32_t cnt_s[kMaxExperts];
+  __shared__ float pw[8][kMaxExperts];
+  __shared__ float zw[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t s = blockIdx.x;
+  seq_counts_block(topk_idx, slot_row, s, S, K, E, cnt_s);
+  float acc[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) acc[i] = 0.f;
+  float z = 0.f;
+  for (int64_t t = s * S + warp; t < (s + 1) * S; t += 8) {
+    float q[NV], rs = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int e = lane + 32 * i;
+      q[i] = e < E ? probs[t * E + e] : 0.f;
+      rs += q[i];
+    }
+    if (normalise) {
+      rs = warp_sum(rs);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) q[i] /= rs;
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) acc[i] += q[i];
+    if (lane == 0) z += lse[t] * lse[t];
+  }
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) pw[warp][e] = acc[i];
+  }
+  if (lane == 0) zw[warp] = z;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t tot = 0;
+    for (int e = lane; e < E; e += 32) tot += cnt_s[e];
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    float v = 0.f;
+    for (int e = lane; e < E; e += 32) {
+      float P = 0.f;
+      for (int w = 0; w < 8; ++w) P += pw[w][e];
+      P /= (float)S;
+      const float f = tot > 0 ? (float)cnt_s[e] / (float)tot : 0.f;
+      v += f * P;
+    }
+    v = warp_sum(v);
+    if (lane == 0) {
+      part[s] = v;
+      float zz = 0.f;
+      for (int w = 0; w < 8; ++w) zz += zw[w];
+      zpart[s] = zz;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256)
+seq_aux_final_kernel(const float* __restrict__ part, const float* __restrict__ zpart,
+                     int n_seq, int T, int E, float alpha, float lambda,
+                     float* __restrict__ losses) {
+  pdl_begin();
+  __shared__ float red[2][256];
+  float a = 0.f, z = 0.f;
+  for (int i = threadIdx.x; i < n_seq; i += blockDim.x) { a += part[i]; z += zpart[i]; }
+  red[0][threadIdx.x] = a;
+  red[1][threadIdx.x] = z;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) {
+      red[0][threadIdx.x] += red[0][threadIdx.x + o];
+      red[1][threadIdx.x] += red[1][threadIdx.x + o];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    losses[0] = alpha * (float)E * red[0][0] / (float)n_seq;
+    losses[1] = lambda * red[1][0] / (float)T;
+  }
+}
+
+// b_e -= gamma * sign(n_e - mean n), the sign taken exactly on n_e*E - sum n
+__global__ void __launch_bounds__(256)
+bias_update_kernel(const int32_t* __restrict__ counts, int E, float gamma,
+                   float* __restrict__ bias) {
+  pdl_begin();
+  __shared__ long long tot_s;
+  if (threadIdx.x == 0) {
+    long long t = 0;
+    for (int e = 0; e < E; ++e) t += counts[e];
+    tot_s = t;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const long long d = (long long)counts[e] * E - tot_s;
+    if (d > 0) bias[e] -= gamma;
+    else if (d < 0) bias[e] += gamma;
   }
 }
 

@@ -90,7 +90,7 @@ __device__ __forceinline__ void warp_rank(const int (&ev)[kDispIters], int64_t j
     if (e >= 0 && (peers & lt) == 0) row[e] += __popc(peers);
     __syncwarp();
     if (e != -2) {
-      int32_t r = -1;
+      int32_t r = e == -1 ? -2 : -1;     // -2: sentinel, -1: dropped
       if (e >= 0 && (C < 0 || rank < C)) {
         r = seg_off[e] + rank;
         if (r < rows_max) row_slot[r] = (int32_t)j;

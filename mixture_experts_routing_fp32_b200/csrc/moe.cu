@@ -111,7 +111,10 @@ int validate(const moe_config_t* c) {
   if (c->group_score != MOE_GMAX && c->group_score != MOE_GTOP2SUM) return MOE_ERR_ARG;
   if (c->n_groups > 1 && c->group_score == MOE_GTOP2SUM && c->E / c->n_groups < 2)
     return MOE_ERR_ARG;
-  if (c->aux_alpha != 0.f && c->score_fn != MOE_SOFTMAX) return MOE_ERR_ARG;
+  if (c->seq_len < 0 || (c->seq_len > 0 && (c->T % c->seq_len))) return MOE_ERR_ARG;
+  // the batch aux loss is defined for softmax scores; the sequence-wise
+  // one also for sigmoid affinities (normalised over experts)
+  if (c->aux_alpha != 0.f && c->score_fn != MOE_SOFTMAX && c->seq_len == 0) return MOE_ERR_ARG;
   if (!(c->route_scale == c->route_scale) || c->min_capacity < 0) return MOE_ERR_ARG;
   if ((int64_t)c->T * c->K > (int64_t)INT32_MAX / 2) return MOE_ERR_ARG;
   if (c->gemm_impl != MOE_GEMM_AUTO && c->gemm_impl != MOE_GEMM_SIMT) return MOE_ERR_ARG;
@@ -163,6 +166,9 @@ struct Layout {
   // tensor-core router products (router_tc)
   int64_t Ep;
   size_t off_wf, off_wb, off_rparts, off_dsf, off_dsb, off_dwr3, off_rdx;
+  // sequence-wise aux (seq_len > 0): per-sequence f [n_seq, E], partials
+  int64_t n_seq;
+  size_t off_seqf, off_seqp;
 };
 constexpr int kAuxChunk = 128;
 
@@ -212,6 +218,11 @@ Layout layout_of(const moe_config_t* c) {
     L.off_dsb = take((size_t)c->T * 3 * L.Ep * 2);
     L.off_dwr3 = take((size_t)3 * L.Ep * c->D * 4);
     L.off_rdx = take((size_t)c->T * c->D * 4);
+  }
+  if (c->seq_len > 0) {
+    L.n_seq = c->T / c->seq_len;
+    L.off_seqf = take((size_t)L.n_seq * c->E * 4);
+    L.off_seqp = take((size_t)2 * L.n_seq * 4);
   }
   L.total = off;
   return L;
@@ -821,6 +832,7 @@ int moe_aux_loss(const moe_config_t* c, const float* probs, const float* lse,
                  const int32_t* counts, float* losses, void* ws, cudaStream_t s) {
   MOE_TRY(validate(c));
   if (!probs || !lse || !counts || !losses || !ws) return MOE_ERR_ARG;
+  if (c->seq_len > 0) return MOE_ERR_ARG;   // moe_aux_loss_seq
   const Layout L = layout_of(c);
   float* part = wsp<float>(ws, L.off_aux);
   prof_begin(s);
@@ -830,6 +842,45 @@ int moe_aux_loss(const moe_config_t* c, const float* probs, const float* lse,
   MOE_CK((launch_k(aux_final_kernel, 1, 512, 0, s, part, counts, L.n_aux_chunks, c->T, c->E, c->aux_alpha,
                                      c->z_lambda, losses)));
   MOE_LAUNCHED(s, "aux_final");
+  return MOE_OK;
+}
+
+int moe_aux_loss_seq(const moe_config_t* c, const float* probs, const float* lse,
+                     const int32_t* topk_idx, const int32_t* slot_row, float* losses, void* ws,
+                     cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!probs || !lse || !topk_idx || !slot_row || !losses || !ws || c->seq_len <= 0)
+    return MOE_ERR_ARG;
+  const Layout L = layout_of(c);
+  float* part = wsp<float>(ws, L.off_seqp);
+  float* zpart = part + L.n_seq;
+  const int norm = c->score_fn == MOE_SOFTMAX ? 0 : 1;
+  auto go = [&](auto nv) -> int {
+    prof_begin(s);
+    MOE_CK((launch_k(seq_aux_kernel<decltype(nv)::value>, (int)L.n_seq, 256, 0, s, probs, lse,
+                     topk_idx, slot_row, c->seq_len, c->K, c->E, norm, part, zpart)));
+    MOE_LAUNCHED(s, "seq_aux");
+    return MOE_OK;
+  };
+  if (c->E <= 32) MOE_TRY(go(std::integral_constant<int, 1>{}));
+  else if (c->E <= 64) MOE_TRY(go(std::integral_constant<int, 2>{}));
+  else if (c->E <= 128) MOE_TRY(go(std::integral_constant<int, 4>{}));
+  else if (c->E <= 256) MOE_TRY(go(std::integral_constant<int, 8>{}));
+  else MOE_TRY(go(std::integral_constant<int, 16>{}));
+  prof_begin(s);
+  MOE_CK((launch_k(seq_aux_final_kernel, 1, 256, 0, s, part, zpart, (int)L.n_seq, c->T, c->E,
+                   c->aux_alpha, c->z_lambda, losses)));
+  MOE_LAUNCHED(s, "seq_aux_final");
+  return MOE_OK;
+}
+
+int moe_bias_update(const moe_config_t* c, const int32_t* counts, float* sel_bias, float gamma,
+                    cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!counts || !sel_bias || !(gamma == gamma)) return MOE_ERR_ARG;
+  prof_begin(s);
+  MOE_CK((launch_k(bias_update_kernel, 1, 256, 0, s, counts, c->E, gamma, sel_bias)));
+  MOE_LAUNCHED(s, "bias_update");
   return MOE_OK;
 }
 
@@ -982,7 +1033,16 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   {
     RouterBwdArgs a{T, E, K, c->score_fn, c->renorm, c->route_scale, c->aux_alpha, c->z_lambda,
                     logits, probs, lse, topk_idx, topk_w, slot_row, dg, counts, ds, dlogits_out,
-                    dg_out, nullptr, nullptr, 0};
+                    dg_out, 0, nullptr, nullptr, nullptr, 0};
+    if (c->seq_len > 0 && c->aux_alpha != 0.f) {
+      // per-sequence f for the sequence-wise aux gradient
+      a.seq_len = c->seq_len;
+      a.seq_f = wsp<float>(ws, L.off_seqf);
+      prof_begin(r);
+      MOE_CK((launch_k(seq_f_kernel, (int)L.n_seq, 256, 0, r, topk_idx, slot_row, c->seq_len, K,
+                       E, wsp<float>(ws, L.off_seqf))));
+      MOE_LAUNCHED(r, "seq_f");
+    }
     if (rtc) {
       a.dsf = wsp<__nv_bfloat16>(ws, L.off_dsf);
       a.dsb = wsp<__nv_bfloat16>(ws, L.off_dsb);

@@ -79,16 +79,15 @@ class MoELayer:
         main = torch.cuda.current_stream(self.device)
         aux = c.aux_alpha != 0.0 or c.z_lambda != 0.0
         if aux and not self.side_streams:
-            api.moe_aux_loss(c, self.probs, self.lse, self.counts, self.losses, self.ws)
+            self._aux(None)
             aux = False
         if aux:
-            # the losses depend only on the router and the counts: computed
+            # the losses depend only on the router and the dispatch: computed
             # on a side stream while the expert GEMMs run
             if self._aux_stream is None:
                 self._aux_stream = torch.cuda.Stream(self.device)
             self._aux_stream.wait_stream(main)
-            api.moe_aux_loss(c, self.probs, self.lse, self.counts, self.losses, self.ws,
-                             stream=self._aux_stream)
+            self._aux(self._aux_stream)
         api.moe_expert_ffn(c, self.x_perm, self.offsets, self.tile_expert, self.stats,
                            w13, w_down, w13_s, w_down_s, self.a13, self.h, self.o,
                            self.ws)
@@ -97,6 +96,21 @@ class MoELayer:
             main.wait_stream(self._aux_stream)
         self._inputs = (x, w_r, w13, w_down, w13_s, w_down_s)
         return self.y
+
+    def _aux(self, stream):
+        c = self.cfg
+        if c.seq_len > 0:
+            api.moe_aux_loss_seq(c, self.probs, self.lse, self.topk_idx, self.slot_row,
+                                 self.losses, self.ws, stream=stream)
+        else:
+            api.moe_aux_loss(c, self.probs, self.lse, self.counts, self.losses, self.ws,
+                             stream=stream)
+
+    def update_bias(self, sel_bias, gamma):
+        """Selection-bias load-control step on this batch's counts (in place,
+        on the current stream; after forward)."""
+        api.moe_bias_update(self.cfg, self.counts, sel_bias, gamma)
+        return sel_bias
 
     # -- backward ----------------------------------------------------------
     def backward(self, dy, want_dg=True, want_dlogits=True):

@@ -38,8 +38,8 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_config_struct_layout_matches_header():
-    # 12 int32 fields, then float, int32, 3 floats, int32 = 18 x 4 bytes
-    assert ctypes.sizeof(C.MoeConfig) == 18 * 4
+    # 12 int32 fields, then float, int32, 3 floats, 2 int32 = 19 x 4 bytes
+    assert ctypes.sizeof(C.MoeConfig) == 19 * 4
     assert ctypes.sizeof(C.MoeSizes) == 40
 
 
@@ -78,7 +78,9 @@ def test_sizes(lib, T, D, E, K, F, c, ns):
     dict(E=513, K=2),                 # E > 512
     dict(n_groups=3),                 # E % n_groups
     dict(n_groups=2, topk_groups=1, K=3),   # topk_groups * E/n_groups < K
-    dict(aux_alpha=0.01, score_fn=1),       # aux needs softmax scores
+    dict(aux_alpha=0.01, score_fn=1),       # batch aux needs softmax scores
+    dict(seq_len=48),                 # seq_len must divide T
+    dict(seq_len=-1),
     dict(dtype="fp16"),               # maps to fp32 -> still valid; replaced below
 ])
 def test_invalid_configs_rejected(lib, bad):

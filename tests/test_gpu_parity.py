@@ -237,5 +237,32 @@ def test_device_error_word_on_bad_expert_id():
                      layer.x_perm, layer.ws)
     with pytest.raises(MoEError):
         api.moe_check_status()
-    assert int(layer.stats[1]) == 1 and int(layer.slot_row[5 * cfg.K]) == -1
+    assert int(layer.stats[1]) == 1 and int(layer.slot_row[5 * cfg.K]) == -2
     assert api.moe_check_status() == 0          # the word was cleared
+
+
+def test_bias_update_matches_oracle():
+    """The selection-bias step on the GPU's own counts, bit for bit: each
+    side subtracts or adds the same fp32 gamma once."""
+    from oracle import balance as B
+    cfg = W.REDUCED["ds3"]
+    layer, inp = run_gpu(cfg)
+    bias = inp["sel_bias"].clone()
+    gamma = 1e-3
+    layer.update_bias(bias, gamma)
+    torch.cuda.synchronize()
+    exp = B.bias_update(layer.counts.cpu().numpy(), inp["sel_bias"].cpu().double().numpy(),
+                        float(np.float32(gamma))).astype(np.float32)
+    np.testing.assert_array_equal(bias.cpu().numpy(), exp)
+    n = layer.counts.cpu().numpy()
+    moved = bias.cpu().numpy() - inp["sel_bias"].cpu().numpy()
+    assert np.all(moved[n * cfg.E > n.sum()] < 0) and np.all(moved[n * cfg.E < n.sum()] > 0)
+
+
+def test_sentinel_slots_are_marked_minus_two():
+    cfg = W.REDUCED["olmoe"]
+    layer, _ = run_gpu(cfg)
+    mask = W.make_input(cfg, "sentinel_mask").numpy().astype(bool)
+    sr = layer.slot_row.cpu().numpy()
+    assert np.all(sr[mask] == -2)
+    assert np.all(sr[~mask] >= -1)

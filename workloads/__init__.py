@@ -108,6 +108,12 @@ REDUCED = {
     "mix_pair": CONFIGS["mix"].replace(name="mix_pair_small", T=7000, D=512, F=640),
     # more than 16384 slots: the multi-block dispatch passes (ragged last block)
     "olmoe_multi": CONFIGS["olmoe"].replace(name="olmoe_multi_small", T=2600, D=128, F=128),
+    # sequence-wise aux loss: softmax (OLMoE-shaped, 7 sequences) and sigmoid
+    # affinities with groups and the shared expert (DeepSeek-shaped, 3 sequences)
+    "olmoe_seq": CONFIGS["olmoe"].replace(name="olmoe_seq_small", T=700, D=256, F=256,
+                                          seq_len=100),
+    "ds3_seq": CONFIGS["ds3"].replace(name="ds3_seq_small", T=300, D=256, F=128,
+                                      aux_alpha=1e-3, seq_len=100),
 }
 
 
