@@ -391,10 +391,15 @@ def forward(L: Layer, o: Opts):
     runs on every token, unweighted, and takes no top-K slot.
     Returns a dict with routing, dispatch, per-slot SwiGLU values and y.
     """
+    return forward_routed(L, o, route_layer(L, o))
+
+
+def forward_routed(L: Layer, o: Opts, R: Routing):
+    """forward() from a given routing (token choice, or the slot form of
+    expert choice in oracle/expert_choice.py)."""
     x = f64(L.x)
     T, D = x.shape
     E = L.w_r.shape[0]
-    R = route_layer(L, o)
     Dp = dispatch(R.idx, E, o.capacity_factor, o.min_capacity,
                   L.sentinel_mask)
     K = o.K
