@@ -92,10 +92,20 @@ enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SIMT = 1 };   /* cfg.gemm_impl */
  *   z_lambda   router z-loss lambda*mean_t lse_t^2           [8MOE] ST-MoE
  *   n_shared   0 or 1: a shared SwiGLU expert on every token, weight 1,
  *              no top-K slot                                 [STA324 §8.7]
+ *   expert_choice
+ *              1: every expert picks C = min(T, max(ceil(c*T/E),
+ *              min_capacity)) tokens, the ones with the largest softmax
+ *              probability p[t,e] (equal scores: lower token first); the
+ *              gate weight is p[t,e]; a token may be picked by several
+ *              experts or none.  [STA324 §8.4]  The layer then runs in the
+ *              token-choice layout with one slot per (t, e) pair: K must
+ *              equal E, topk_idx[t,e] = e, and the pairs an expert did not
+ *              pick are sentinel slots.  Requires softmax, renorm = 0,
+ *              capacity_factor > 0, no groups, no aux loss, route_scale 1.
  *   gemm_impl  MOE_GEMM_AUTO: tcgen05 tensor cores for bf16 when D and F
  *              are multiples of 128, CUDA-core SIMT otherwise (fp32 always);
  *              MOE_GEMM_SIMT: force the SIMT kernels (cross-checks).
- * Limits: 1 <= K <= min(E, 16); E <= 512; n_groups <= 32, E % n_groups == 0,
+ * Limits: 1 <= K <= min(E, 16) (expert choice: K = E); E <= 512; n_groups <= 32, E % n_groups == 0,
  * topk_groups * (E / n_groups) >= K; D % 8 == 0; F % 8 == 0.
  */
 typedef struct {
@@ -109,6 +119,8 @@ typedef struct {
   int32_t gemm_impl;
   int32_t seq_len;      /* 0: batch aux loss; > 0: sequence-wise aux loss over
                            consecutive groups of seq_len tokens (divides T) */
+  int32_t expert_choice; /* 0: token choice (top-K per token); 1: expert choice
+                            (moe_route_expert_choice) */
 } moe_config_t;
 
 typedef struct {
@@ -213,6 +225,24 @@ int moe_dispatch_static(const moe_config_t* cfg, const int32_t* topk_idx,
 int moe_aux_loss(const moe_config_t* cfg, const float* probs, const float* lse,
                  const int32_t* counts, float* losses, void* ws,
                  cudaStream_t stream);
+
+/*
+ * moe_route_expert_choice — router of expert choice (cfg.expert_choice = 1,
+ * K = E).  fp32 logits (tensor cores on bf16 splits of w_r, as moe_router),
+ * probs = softmax, lse, then each expert's C picks.  [STA324 §8.4]
+ *   logits, probs [T,E] f32 out; lse [T] f32 out
+ *   topk_idx  [T,E] i32 out: e (slot (t,e) belongs to expert e)
+ *   topk_w    [T,E] f32 out: p[t,e]
+ *   sentinel_mask [T*E] u8 out: 1 where expert e did not pick token t
+ *             (pass it to moe_dispatch)
+ *   near_ties [1] i32 out: experts whose C-th and (C+1)-th scores differ by
+ *             less than 1e-5
+ */
+int moe_route_expert_choice(const moe_config_t* cfg, const void* x, const float* w_r,
+                            const float* logit_offset, float* logits, float* probs,
+                            float* lse, int32_t* topk_idx, float* topk_w,
+                            uint8_t* sentinel_mask, int32_t* near_ties, void* ws,
+                            cudaStream_t stream);
 
 /*
  * moe_aux_loss_seq — the sequence-wise aux loss (cfg.seq_len > 0):

@@ -28,7 +28,7 @@ EXPORTS = ("moe_get_sizes", "moe_router", "moe_dispatch", "moe_aux_loss",
            "moe_profile_enable", "moe_profile_reset", "moe_profile_read", "moe_profile_starts",
            "moe_profile_name", "moe_profile_side", "moe_profile_disable",
            "moe_dispatch_static", "moe_set_side_streams", "moe_aux_loss_seq",
-           "moe_bias_update")
+           "moe_bias_update", "moe_route_expert_choice")
 
 
 class MoeConfig(ctypes.Structure):
@@ -38,7 +38,8 @@ class MoeConfig(ctypes.Structure):
                 ("topk_groups", c_int32), ("group_score", c_int32),
                 ("capacity_factor", c_float), ("min_capacity", c_int32),
                 ("route_scale", c_float), ("aux_alpha", c_float),
-                ("z_lambda", c_float), ("gemm_impl", c_int32), ("seq_len", c_int32)]
+                ("z_lambda", c_float), ("gemm_impl", c_int32), ("seq_len", c_int32),
+                ("expert_choice", c_int32)]
 
 
 class MoeSizes(ctypes.Structure):
@@ -89,6 +90,7 @@ def lib():
         "moe_dispatch_static": [cfg, P, P, P, P, P, P, P, P, P, P, P, P],
         "moe_aux_loss_seq": [cfg, P, P, P, P, P, P, P],
         "moe_bias_update": [cfg, P, P, ctypes.c_float, P],
+        "moe_route_expert_choice": [cfg] + [P] * 12,
     }
     for name, args in sig.items():
         fn = getattr(L, name)

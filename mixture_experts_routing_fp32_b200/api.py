@@ -26,7 +26,8 @@ def _s(stream=None):
 def make_config(T, D, E, K, F, *, n_shared=0, dtype="bf16", score_fn=0,
                 renorm=1, n_groups=1, topk_groups=1, group_score=0,
                 capacity_factor=0.0, min_capacity=0, route_scale=1.0,
-                aux_alpha=0.0, z_lambda=0.0, gemm_impl=0, seq_len=0) -> MoeConfig:
+                aux_alpha=0.0, z_lambda=0.0, gemm_impl=0, seq_len=0,
+                expert_choice=0) -> MoeConfig:
     return MoeConfig(
         T=T, D=D, E=E, K=K, F=F, n_shared=n_shared,
         dtype=C.MOE_BF16 if dtype in ("bf16", torch.bfloat16) else C.MOE_FP32,
@@ -34,14 +35,14 @@ def make_config(T, D, E, K, F, *, n_shared=0, dtype="bf16", score_fn=0,
         topk_groups=topk_groups, group_score=group_score,
         capacity_factor=capacity_factor, min_capacity=min_capacity,
         route_scale=route_scale, aux_alpha=aux_alpha, z_lambda=z_lambda,
-        gemm_impl=gemm_impl, seq_len=seq_len)
+        gemm_impl=gemm_impl, seq_len=seq_len, expert_choice=expert_choice)
 
 
 def config_from(obj, **over) -> MoeConfig:
     """MoeConfig from any object carrying the layer fields by name."""
     names = ("n_shared", "dtype", "score_fn", "renorm", "n_groups",
              "topk_groups", "group_score", "capacity_factor", "min_capacity",
-             "route_scale", "aux_alpha", "z_lambda", "seq_len")
+             "route_scale", "aux_alpha", "z_lambda", "seq_len", "expert_choice")
     kw = {n: getattr(obj, n) for n in names if hasattr(obj, n)}
     kw.update(over)
     return make_config(obj.T, obj.D, obj.E, obj.K, obj.F, **kw)
@@ -80,6 +81,14 @@ def moe_dispatch_static(cfg, topk_idx, sentinel_mask, x, counts, kept, offsets,
                                     _p(slot_row), _p(row_slot), _p(tile_expert),
                                     _p(stats), _p(x_perm), _s(stream)),
           "moe_dispatch_static")
+
+
+def moe_route_expert_choice(cfg, x, w_r, logit_offset, logits, probs, lse, topk_idx, topk_w,
+                            sentinel_mask, near_ties, ws, stream=None):
+    check(lib().moe_route_expert_choice(
+        ctypes.byref(cfg), _p(x), _p(w_r), _p(logit_offset), _p(logits), _p(probs), _p(lse),
+        _p(topk_idx), _p(topk_w), _p(sentinel_mask), _p(near_ties), _p(ws), _s(stream)),
+        "moe_route_expert_choice")
 
 
 def moe_aux_loss_seq(cfg, probs, lse, topk_idx, slot_row, losses, ws, stream=None):
@@ -181,4 +190,4 @@ __all__ = ["LaunchProfile", "MoEError", "MoeConfig", "MoeSizes", "make_config", 
            "moe_aux_loss",
            "moe_expert_ffn", "moe_combine", "moe_backward", "moe_check_status",
            "moe_launch_count", "moe_set_side_streams", "moe_aux_loss_seq",
-           "moe_bias_update"]
+           "moe_bias_update", "moe_route_expert_choice"]

@@ -16,6 +16,7 @@
 #include "router.cuh"
 #include "dispatch.cuh"
 #include "combine.cuh"
+#include "expert_choice.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 
@@ -100,7 +101,16 @@ int validate(const moe_config_t* c) {
   if (c == nullptr) return MOE_ERR_ARG;
   if (c->T < 1 || c->D < 8 || (c->D % 8) || c->F < 8 || (c->F % 8)) return MOE_ERR_ARG;
   if (c->E < 1 || c->E > kMaxExperts) return MOE_ERR_ARG;
-  if (c->K < 1 || c->K > c->E || c->K > kMaxK) return MOE_ERR_ARG;
+  if (c->expert_choice != 0 && c->expert_choice != 1) return MOE_ERR_ARG;
+  if (c->expert_choice) {
+    // expert choice in the slot layout: one slot per (token, expert) pair
+    if (c->K != c->E || c->score_fn != MOE_SOFTMAX || c->renorm != 0 || c->n_groups != 1 ||
+        !(c->capacity_factor > 0.f) || c->aux_alpha != 0.f || c->seq_len != 0 ||
+        c->route_scale != 1.f)
+      return MOE_ERR_ARG;
+  } else if (c->K < 1 || c->K > c->E || c->K > kMaxK) {
+    return MOE_ERR_ARG;
+  }
   if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_ARG;
   if (c->dtype != MOE_FP32 && c->dtype != MOE_BF16) return MOE_ERR_ARG;
   if (c->score_fn != MOE_SOFTMAX && c->score_fn != MOE_SIGMOID) return MOE_ERR_ARG;
@@ -121,7 +131,16 @@ int validate(const moe_config_t* c) {
   return MOE_OK;
 }
 
+// Expert choice: tokens each expert picks, C = min(T, max(ceil(c*T/E), min_capacity)).
+int64_t ec_capacity(const moe_config_t* c) {
+  const double v = std::ceil((double)c->capacity_factor * (double)c->T / (double)c->E);
+  return std::min<int64_t>(c->T, std::max<int64_t>((int64_t)v, c->min_capacity));
+}
+
+// Token-choice drop capacity (-1: none; expert choice never drops in the
+// dispatch, its picks already hold C slots per expert).
 int64_t capacity_of(const moe_config_t* c) {
+  if (c->expert_choice) return -1;
   if (!(c->capacity_factor > 0.f)) return -1;
   const double v = std::ceil((double)c->capacity_factor * (double)((int64_t)c->T * c->K) /
                              (double)c->E);
@@ -152,7 +171,9 @@ bool pair_rows(const moe_config_t* c) {
   if (!use_tc(c)) return false;
   const int64_t C = capacity_of(c);
   const int64_t slots = (int64_t)c->T * c->K;
-  const int64_t kept = C < 0 ? slots : std::min<int64_t>(slots, (int64_t)c->E * C);
+  const int64_t kept = c->expert_choice ? (int64_t)c->E * ec_capacity(c)
+                       : C < 0          ? slots
+                                        : std::min<int64_t>(slots, (int64_t)c->E * C);
   return kept / c->E >= 1536;
 }
 
@@ -185,7 +206,9 @@ Layout layout_of(const moe_config_t* c) {
   Layout L{};
   L.C = capacity_of(c);
   L.n_slots = (int64_t)c->T * c->K;
-  const int64_t kept_total = L.C < 0 ? L.n_slots : std::min<int64_t>(L.n_slots, (int64_t)c->E * L.C);
+  const int64_t kept_total = c->expert_choice ? (int64_t)c->E * ec_capacity(c)
+                             : L.C < 0        ? L.n_slots
+                                              : std::min<int64_t>(L.n_slots, (int64_t)c->E * L.C);
   const int64_t align = row_align(c);
   const int64_t pad = (align - 1) * std::min<int64_t>(c->E, kept_total);
   L.rows_max = round_up(kept_total + pad, align) + (c->n_shared ? round_up(c->T, align) : 0);
@@ -378,8 +401,9 @@ int run_tc(int bn, const char* name, const CUtensorMap& a, const CUtensorMap& b,
 // Expected 128-row tiles of the permuted rows (half a tile of padding per
 // expert on average), used only to choose tile widths.
 int64_t row_tiles_estimate(const moe_config_t* c, const Layout& L) {
-  const int64_t kept_total =
-      L.C < 0 ? L.n_slots : std::min<int64_t>(L.n_slots, (int64_t)c->E * L.C);
+  const int64_t kept_total = c->expert_choice ? (int64_t)c->E * ec_capacity(c)
+                             : L.C < 0        ? L.n_slots
+                                              : std::min<int64_t>(L.n_slots, (int64_t)c->E * L.C);
   const int64_t rows = kept_total + 64 * std::min<int64_t>(c->E, kept_total);
   return ceil_div(rows, kRowTile) + (c->n_shared ? ceil_div(c->T, kRowTile) : 0);
 }
@@ -744,12 +768,91 @@ int moe_router(const moe_config_t* c, const void* x, const float* w_r, const flo
   MOE_TRY(validate(c));
   if (!x || !w_r || !logits || !probs || !lse || !topk_idx || !topk_w || !near_ties)
     return MOE_ERR_ARG;
+  if (c->expert_choice) return MOE_ERR_ARG;   // moe_route_expert_choice
   if (router_tc(c) && ws == nullptr) return MOE_ERR_ARG;
   if (c->dtype == MOE_BF16)
     return router_impl(c, static_cast<const __nv_bfloat16*>(x), w_r, logit_offset, sel_bias,
                        logits, probs, lse, topk_idx, topk_w, near_ties, ws, s);
   return router_impl(c, static_cast<const float*>(x), w_r, logit_offset, sel_bias, logits, probs,
                      lse, topk_idx, topk_w, near_ties, ws, s);
+}
+
+}  // extern "C"
+
+template <typename TX>
+int route_ec_impl(const moe_config_t* c, const TX* x, const float* w_r, const float* off,
+                  float* logits, float* probs, float* lse, int32_t* idx, float* w,
+                  uint8_t* mask, int32_t* ties, void* ws, cudaStream_t s) {
+  MOE_CK(cudaMemsetAsync(ties, 0, sizeof(int32_t), s));
+  const int E = c->E;
+  const float* parts = nullptr;
+  int64_t Ep = 0;
+  if (router_tc(c)) {
+    const Layout L = layout_of(c);
+    Ep = L.Ep;
+    const int64_t n3 = 3 * Ep;
+    auto* wf = wsp<__nv_bfloat16>(ws, L.off_wf);
+    float* pt = wsp<float>(ws, L.off_rparts);
+    prof_begin(s);
+    MOE_CK((launch_k(split_w_kernel, grid_for(Ep * c->D / 32), 256, 0, s, w_r, E, (int)Ep,
+                     c->D, wf, (__nv_bfloat16*)nullptr)));
+    MOE_LAUNCHED(s, "router_split_w");
+    const int64_t mtiles = ceil_div(c->T, kRowTile);
+    const int bn = pick_bn(n3, mtiles, false, 0, false);
+    CUtensorMap mA, mB;
+    MOE_TRY(make_map(&mA, x, 1, c->T, c->D, 128, false));
+    MOE_TRY(make_map(&mB, wf, 1, n3, c->D, bn, true));
+    tc::Params p{};
+    p.E = 1; p.Kd = c->D; p.nN = (int)(n3 / bn); p.group_m = group_rows(c->D);
+    p.dense_m = c->T;
+    p.out_f32 = pt; p.ld_f32 = n3;
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_F32>(
+        bn, "router_logits_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+    parts = pt;
+  } else {
+    dim3 g1((unsigned)ceil_div(c->T, 64), (unsigned)ceil_div(E, 64));
+    prof_begin(s);
+    MOE_CK((launch_k(router_logits_kernel<TX>, g1, 256, 0, s, x, w_r, off, logits, c->T, c->D,
+                     E)));
+    MOE_LAUNCHED(s, "router_logits");
+  }
+  auto go = [&](auto nv) -> int {
+    prof_begin(s);
+    MOE_CK((launch_k(ec_scores_kernel<decltype(nv)::value>, grid_for(c->T), 256, 0, s, parts,
+                     (int)Ep, parts != nullptr ? off : nullptr, c->T, E, logits, probs, lse,
+                     idx, w)));
+    MOE_LAUNCHED(s, "ec_scores");
+    return MOE_OK;
+  };
+  if (E <= 32) MOE_TRY(go(std::integral_constant<int, 1>{}));
+  else if (E <= 64) MOE_TRY(go(std::integral_constant<int, 2>{}));
+  else if (E <= 128) MOE_TRY(go(std::integral_constant<int, 4>{}));
+  else if (E <= 256) MOE_TRY(go(std::integral_constant<int, 8>{}));
+  else MOE_TRY(go(std::integral_constant<int, 16>{}));
+  prof_begin(s);
+  MOE_CK((launch_k(ec_select_kernel, E, kEcThreads, 0, s, probs, c->T, E, (int)ec_capacity(c),
+                   mask, ties)));
+  MOE_LAUNCHED(s, "ec_select");
+  return MOE_OK;
+}
+
+extern "C" {
+
+int moe_route_expert_choice(const moe_config_t* c, const void* x, const float* w_r,
+                                       const float* logit_offset, float* logits, float* probs,
+                                       float* lse, int32_t* topk_idx, float* topk_w,
+                                       uint8_t* sentinel_mask, int32_t* near_ties, void* ws,
+                                       cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!c->expert_choice || !x || !w_r || !logits || !probs || !lse || !topk_idx || !topk_w ||
+      !sentinel_mask || !near_ties)
+    return MOE_ERR_ARG;
+  if (router_tc(c) && ws == nullptr) return MOE_ERR_ARG;
+  if (c->dtype == MOE_BF16)
+    return route_ec_impl(c, static_cast<const __nv_bfloat16*>(x), w_r, logit_offset, logits,
+                         probs, lse, topk_idx, topk_w, sentinel_mask, near_ties, ws, s);
+  return route_ec_impl(c, static_cast<const float*>(x), w_r, logit_offset, logits, probs, lse,
+                       topk_idx, topk_w, sentinel_mask, near_ties, ws, s);
 }
 
 int moe_dispatch(const moe_config_t* c, const int32_t* topk_idx, const uint8_t* sentinel_mask,
@@ -950,6 +1053,19 @@ int moe_combine(const moe_config_t* c, const void* o, const int32_t* slot_row,
   MOE_TRY(validate(c));
   if (!o || !slot_row || !topk_w || !offsets || !y) return MOE_ERR_ARG;
   const int grid = grid_for(c->T);
+  if (c->expert_choice) {
+    prof_begin(s);
+    if (c->dtype == MOE_BF16)
+      MOE_CK((launch_k(ec_combine_kernel<__nv_bfloat16>, grid, 256, 0, s,
+                       static_cast<const __nv_bfloat16*>(o), slot_row, topk_w, offsets,
+                       c->n_shared, c->T, c->D, c->E, static_cast<__nv_bfloat16*>(y))));
+    else
+      MOE_CK((launch_k(ec_combine_kernel<float>, grid, 256, 0, s, static_cast<const float*>(o),
+                       slot_row, topk_w, offsets, c->n_shared, c->T, c->D, c->E,
+                       static_cast<float*>(y))));
+    MOE_LAUNCHED(s, "combine");
+    return MOE_OK;
+  }
   if (c->dtype == MOE_BF16 && (c->K == 1 || c->K == 2 || c->K == 4 || c->K == 8)) {
     auto go = [&](auto kt) -> int {
       prof_begin(s);
@@ -1051,6 +1167,22 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     const int grid = grid_for(T);
     {
     cudaStream_t s = r;
+    if (c->expert_choice) {
+      // dp = dg on the picked pairs, then the softmax backward
+      auto go = [&](auto nv) -> int {
+        prof_begin(s);
+        MOE_CK((launch_k(ec_router_bwd_kernel<decltype(nv)::value>, grid, 256, 0, s, probs,
+                         logits, lse, slot_row, dg, T, E, c->z_lambda, ds, dlogits_out, dg_out,
+                         a.dsf, a.dsb, a.Ep)));
+        MOE_LAUNCHED(s, "router_bwd");
+        return MOE_OK;
+      };
+      if (E <= 32) MOE_TRY(go(std::integral_constant<int, 1>{}));
+      else if (E <= 64) MOE_TRY(go(std::integral_constant<int, 2>{}));
+      else if (E <= 128) MOE_TRY(go(std::integral_constant<int, 4>{}));
+      else if (E <= 256) MOE_TRY(go(std::integral_constant<int, 8>{}));
+      else MOE_TRY(go(std::integral_constant<int, 16>{}));
+    } else {
     prof_begin(s);
     if (E <= 32) MOE_CK((launch_k(router_bwd_kernel<1>, grid, 256, 0, s, a)));
     else if (E <= 64) MOE_CK((launch_k(router_bwd_kernel<2>, grid, 256, 0, s, a)));
@@ -1058,6 +1190,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     else if (E <= 256) MOE_CK((launch_k(router_bwd_kernel<8>, grid, 256, 0, s, a)));
     else MOE_CK((launch_k(router_bwd_kernel<16>, grid, 256, 0, s, a)));
     MOE_LAUNCHED(s, "router_bwd");
+    }
     if (rtc) {
       // (hi; mid; hi) split of W_r for the router part of dx
       prof_begin(s);
@@ -1222,7 +1355,36 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   // (W_hi; W_mid; W_hi) is written in fp32 and a gather kernel adds the
   // dX_perm rows
   MOE_CK(cudaStreamWaitEvent(s, sd->ev[6], 0));
-  if (rtc) {
+  float* Rdx = nullptr;
+  if (rtc && c->expert_choice) {
+    // expert choice: the router term R on tensor cores, then a ballot-based
+    // gather over each token's picked rows
+    const int64_t n3 = 3 * L.Ep;
+    Rdx = wsp<float>(ws, L.off_rdx);
+    CUtensorMap mA, mB;
+    MOE_TRY(make_map(&mA, wsp<__nv_bfloat16>(ws, L.off_dsb), 1, T, n3, 128, false));
+    MOE_TRY(make_map(&mB, wsp<__nv_bfloat16>(ws, L.off_wb), 1, n3, D, 64, true));
+    const int64_t mtiles = ceil_div(T, kRowTile);
+    const int bn = pick_bn(D, mtiles, false, 0, false);
+    tc::Params p{};
+    p.E = 1; p.Kd = (int)n3; p.nN = D / bn; p.group_m = group_rows(n3);
+    p.dense_m = T;
+    p.out_f32 = Rdx; p.ld_f32 = D;
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_F32>(
+        bn, "router_dx_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+  }
+  if (c->expert_choice) {
+    prof_begin(s);
+    if (bf)
+      MOE_CK((launch_k(ec_dx_kernel<__nv_bfloat16>, grid_for(T), 256, 0, s, Rdx, ds, w_r,
+                       static_cast<const __nv_bfloat16*>(dXp), slot_row, offsets, c->n_shared,
+                       T, D, E, static_cast<__nv_bfloat16*>(dx))));
+    else
+      MOE_CK((launch_k(ec_dx_kernel<float>, grid_for(T), 256, 0, s, Rdx, ds, w_r,
+                       static_cast<const float*>(dXp), slot_row, offsets, c->n_shared, T, D, E,
+                       static_cast<float*>(dx))));
+    MOE_LAUNCHED(s, "dx_unpermute_sum");
+  } else if (rtc) {
     const int64_t n3 = 3 * L.Ep;
     float* R = wsp<float>(ws, L.off_rdx);
     CUtensorMap mA, mB;

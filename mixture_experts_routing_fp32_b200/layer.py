@@ -43,6 +43,8 @@ class MoELayer:
         self.y = e((T, D), act)
         self.losses = torch.zeros(2, dtype=f32, device=dev)
         self.ws = e((max(int(z.ws_bytes), 256),), torch.uint8)
+        # expert choice: 1 where expert e did not pick token t (slot t*E + e)
+        self.ec_mask = e((T * K,), torch.uint8) if c.expert_choice else None
         self._grads_ready = False
         self._inputs = None
         self._aux_stream = None
@@ -71,8 +73,14 @@ class MoELayer:
     def forward(self, x, w_r, w13, w_down, w13_s=None, w_down_s=None,
                 logit_offset=None, sel_bias=None, sentinel_mask=None):
         c = self.cfg
-        api.moe_router(c, x, w_r, logit_offset, sel_bias, self.logits, self.probs,
-                       self.lse, self.topk_idx, self.topk_w, self.near_ties, self.ws)
+        if c.expert_choice:
+            api.moe_route_expert_choice(c, x, w_r, logit_offset, self.logits, self.probs,
+                                        self.lse, self.topk_idx, self.topk_w, self.ec_mask,
+                                        self.near_ties, self.ws)
+            sentinel_mask = self.ec_mask
+        else:
+            api.moe_router(c, x, w_r, logit_offset, sel_bias, self.logits, self.probs,
+                           self.lse, self.topk_idx, self.topk_w, self.near_ties, self.ws)
         api.moe_dispatch(c, self.topk_idx, sentinel_mask, x, self.counts, self.kept,
                          self.offsets, self.slot_row, self.row_slot, self.tile_expert,
                          self.stats, self.x_perm, self.ws)

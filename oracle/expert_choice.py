@@ -72,15 +72,17 @@ def layer_for(L: O.Layer, chosen) -> O.Layer:
     return replace(L, sentinel_mask=~chosen.reshape(-1))
 
 
-def opts_for(E) -> O.Opts:
-    return O.Opts(K=E, score_fn=O.SOFTMAX, renorm=0)
+def opts_for(E, z_lambda=0.0) -> O.Opts:
+    return O.Opts(K=E, score_fn=O.SOFTMAX, renorm=0, z_lambda=z_lambda)
 
 
-def forward(L: O.Layer, capacity_factor, min_capacity=0, logits_fp32=True):
+def forward(L: O.Layer, capacity_factor, min_capacity=0, logits_fp32=True, z_lambda=0.0):
+    """(layer with the unchosen pairs as sentinels, Opts, forward dict);
+    O.backward(layer, opts, fw, dy) then gives every gradient."""
     R, chosen, C = route(L, capacity_factor, min_capacity, logits_fp32)
     E = chosen.shape[1]
     Lc = layer_for(L, chosen)
-    o = opts_for(E)
+    o = opts_for(E, z_lambda)
     o.logits_fp32 = logits_fp32
     fw = O.forward_routed(Lc, o, R)
     fw["chosen"], fw["C"] = chosen, C

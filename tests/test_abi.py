@@ -38,8 +38,8 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_config_struct_layout_matches_header():
-    # 12 int32 fields, then float, int32, 3 floats, 2 int32 = 19 x 4 bytes
-    assert ctypes.sizeof(C.MoeConfig) == 19 * 4
+    # 12 int32 fields, then float, int32, 3 floats, 3 int32 = 20 x 4 bytes
+    assert ctypes.sizeof(C.MoeConfig) == 20 * 4
     assert ctypes.sizeof(C.MoeSizes) == 40
 
 
@@ -81,6 +81,9 @@ def test_sizes(lib, T, D, E, K, F, c, ns):
     dict(aux_alpha=0.01, score_fn=1),       # batch aux needs softmax scores
     dict(seq_len=48),                 # seq_len must divide T
     dict(seq_len=-1),
+    dict(expert_choice=1),            # expert choice needs K = E and a capacity
+    dict(expert_choice=1, K=4, capacity_factor=1.0, renorm=1),   # ... and variant A
+    dict(expert_choice=1, K=4, capacity_factor=1.0, renorm=0, aux_alpha=0.01),
     dict(dtype="fp16"),               # maps to fp32 -> still valid; replaced below
 ])
 def test_invalid_configs_rejected(lib, bad):

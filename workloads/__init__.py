@@ -49,6 +49,7 @@ class LayerConfig:
     aux_alpha: float = 0.0
     z_lambda: float = 0.0
     seq_len: int = 0            # > 0: sequence-wise aux loss over seq_len tokens
+    expert_choice: int = 0      # 1: each expert picks its C tokens (K = E slots per token)
     # input recipe
     seed: int = 0
     x_std: float = 1.0
@@ -93,6 +94,10 @@ CONFIGS = {
     "ds3": LayerConfig("ds3", T=8192, D=7168, E=256, K=8, F=2048, n_shared=1,
                        score_fn=SIGMOID, renorm=1, n_groups=8, topk_groups=4,
                        sel_bias_range=0.1),
+    # expert choice on the OLMoE shape: each of the 64 experts picks
+    # C = 8*T/64 = 2048 tokens (the same expert FLOPs as top-8 token choice)
+    "olmoe_ec": LayerConfig("olmoe_ec", T=16384, D=2048, E=64, K=64, F=1024, renorm=0,
+                            capacity_factor=8.0, z_lambda=1e-3, expert_choice=1),
 }
 
 # Reduced variants: same options, sizes the oracle handles element by element.
@@ -114,6 +119,12 @@ REDUCED = {
                                           seq_len=100),
     "ds3_seq": CONFIGS["ds3"].replace(name="ds3_seq_small", T=300, D=256, F=128,
                                       aux_alpha=1e-3, seq_len=100),
+    # expert choice: 8 experts (with z-loss, C = 128 of 512 tokens) and the
+    # OLMoE-shaped 64 experts at reduced size
+    "ec8": LayerConfig("ec8_small", T=512, D=256, E=8, K=8, F=256, renorm=0,
+                       capacity_factor=2.0, z_lambda=1e-3, expert_choice=1),
+    "olmoe_ec": CONFIGS["olmoe_ec"].replace(name="olmoe_ec_small", T=1024, D=128, F=128,
+                                            capacity_factor=2.0),
 }
 
 
