@@ -545,10 +545,17 @@ def oracle_step(cfg, T_s):
     # weights are generated before the clock starts
     for e in range(cfg.E):
         g13(e), gd(e)
-    o = O.opts_of(sub)
     t0 = time.perf_counter()
-    fw = O.forward(L, o)
-    O.backward(L, o, fw, dy)
+    if cfg.expert_choice:
+        # expert choice picks across the batch: the sample is its own batch
+        # (each expert picks ceil(c * T_s / E) of its tokens)
+        from oracle import expert_choice as X
+        Lc, o, fw = X.forward(L, cfg.capacity_factor, cfg.min_capacity, z_lambda=cfg.z_lambda)
+        O.backward(Lc, o, fw, dy)
+    else:
+        o = O.opts_of(sub)
+        fw = O.forward(L, o)
+        O.backward(L, o, fw, dy)
     return time.perf_counter() - t0
 
 

@@ -534,59 +534,38 @@ dx_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
 // order (per-warp token strides, then warps in order), so results do not
 // depend on timing.
 // ---------------------------------------------------------------------------
-// counts of sequence s per expert (valid slots: slot_row != -2, pre-drop)
-__device__ void seq_counts_block(const int32_t* __restrict__ topk_idx,
-                                 const int32_t* __restrict__ slot_row, int64_t s, int S, int K,
-                                 int E, int32_t* cnt_s) {
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = 0;
-  __syncthreads();
-  const int64_t j0 = s * S * (int64_t)K, j1 = j0 + (int64_t)S * K;
-  for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-    const int e = topk_idx[j];
-    if (slot_row[j] != -2 && e >= 0 && e < E) atomicAdd(&cnt_s[e], 1);
-  }
-  __syncthreads();
-}
-
-// f[s][e] = n_{s,e} / sum_e n_{s,e}
-__global__ void __launch_bounds__(256)
-seq_f_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ slot_row,
-             int S, int K, int E, float* __restrict__ f) {
-  pdl_begin();
-  __shared__ int32_t cnt_s[kMaxExperts];
-  __shared__ int32_t tot_s;
-  seq_counts_block(topk_idx, slot_row, blockIdx.x, S, K, E, cnt_s);
-  if (threadIdx.x == 0) {
-    int32_t t = 0;
-    for (int e = 0; e < E; ++e) t += cnt_s[e];
-    tot_s = t;
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    f[(size_t)blockIdx.x * E + e] = tot_s > 0 ? (float)cnt_s[e] / (float)tot_s : 0.f;
-}
-
-// Per sequence: part[s] = sum_e f_{s,e} P_{s,e} and zpart[s] = sum_t lse_t^2.
-// q = probs (softmax) or probs / sum_e probs (sigmoid); lane l of a warp
-// holds experts l + 32 i.
+// Partial sums of one piece of a sequence (block (b, s): tokens
+// [s S + b L, s S + (b+1) L) with L = ceil(S / gridDim.x)): slot counts per
+// expert, sums of q per expert, sum of lse^2.  q = probs (softmax) or
+// probs / sum_e probs (sigmoid); lane l of a warp holds experts l + 32 i.
 template <int NV>
 __global__ void __launch_bounds__(256)
-seq_aux_kernel(const float* __restrict__ probs, const float* __restrict__ lse,
-               const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ slot_row,
-               int S, int K, int E, int normalise, float* __restrict__ part,
-               float* __restrict__ zpart) {
+seq_aux_partial_kernel(const float* __restrict__ probs, const float* __restrict__ lse,
+                       const int32_t* __restrict__ topk_idx,
+                       const int32_t* __restrict__ slot_row, int S, int K, int E,
+                       int normalise, int32_t* __restrict__ cnt_part,
+                       float* __restrict__ q_part, float* __restrict__ z_part) {
   pdl_begin();
   __shared__ int32_t cnt_s[kMaxExperts];
   __shared__ float pw[8][kMaxExperts];
   __shared__ float zw[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t s = blockIdx.x;
-  seq_counts_block(topk_idx, slot_row, s, S, K, E, cnt_s);
+  const int nb = gridDim.x, b = blockIdx.x;
+  const int64_t s = blockIdx.y;
+  const int L = (S + nb - 1) / nb;
+  const int64_t t0 = s * S + (int64_t)b * L;
+  const int64_t t1 = t0 + L < (s + 1) * S ? t0 + L : (s + 1) * S;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = 0;
+  __syncthreads();
+  for (int64_t j = t0 * K + threadIdx.x; j < t1 * K; j += blockDim.x) {
+    const int e = topk_idx[j];
+    if (slot_row[j] != -2 && e >= 0 && e < E) atomicAdd(&cnt_s[e], 1);
+  }
   float acc[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i) acc[i] = 0.f;
   float z = 0.f;
-  for (int64_t t = s * S + warp; t < (s + 1) * S; t += 8) {
+  for (int64_t t = t0 + warp; t < t1; t += 8) {
     float q[NV], rs = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
@@ -610,36 +589,80 @@ seq_aux_kernel(const float* __restrict__ probs, const float* __restrict__ lse,
   }
   if (lane == 0) zw[warp] = z;
   __syncthreads();
-  if (warp == 0) {
-    int32_t tot = 0;
-    for (int e = lane; e < E; e += 32) tot += cnt_s[e];
-    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    float v = 0.f;
-    for (int e = lane; e < E; e += 32) {
-      float P = 0.f;
-      for (int w = 0; w < 8; ++w) P += pw[w][e];
-      P /= (float)S;
-      const float f = tot > 0 ? (float)cnt_s[e] / (float)tot : 0.f;
-      v += f * P;
-    }
-    v = warp_sum(v);
-    if (lane == 0) {
-      part[s] = v;
-      float zz = 0.f;
-      for (int w = 0; w < 8; ++w) zz += zw[w];
-      zpart[s] = zz;
-    }
+  const int64_t o = (s * nb + b) * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float P = 0.f;
+    for (int w = 0; w < 8; ++w) P += pw[w][e];
+    q_part[o + e] = P;
+    cnt_part[o + e] = cnt_s[e];
+  }
+  if (threadIdx.x == 0) {
+    float zz = 0.f;
+    for (int w = 0; w < 8; ++w) zz += zw[w];
+    z_part[s * nb + b] = zz;
   }
 }
 
+// One block per sequence s: n and P from its pieces (summed in piece
+// order), f = n / sum n, part[s] = sum_e f P (fixed-order block sums);
+// f [n_seq, E] is written for the backward when f_out is given.
 __global__ void __launch_bounds__(256)
-seq_aux_final_kernel(const float* __restrict__ part, const float* __restrict__ zpart,
-                     int n_seq, int T, int E, float alpha, float lambda,
+seq_aux_seq_kernel(const int32_t* __restrict__ cnt_part, const float* __restrict__ q_part,
+                   int nb, int S, int E, float* __restrict__ part,
+                   float* __restrict__ f_out) {
+  pdl_begin();
+  __shared__ int32_t n_s[kMaxExperts];
+  __shared__ float p_s[kMaxExperts];
+  __shared__ float red[256];
+  const int64_t s = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t n = 0;
+    float P = 0.f;
+#pragma unroll 8
+    for (int b = 0; b < nb; ++b) {
+      n += cnt_part[(s * nb + b) * E + e];
+      P += q_part[(s * nb + b) * E + e];
+    }
+    n_s[e] = n;
+    p_s[e] = P / (float)S;
+  }
+  __syncthreads();
+  float tot = 0.f;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) tot += (float)n_s[e];
+  red[threadIdx.x] = tot;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  const float ntot = red[0];
+  __syncthreads();
+  float v = 0.f;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const float f = ntot > 0.f ? (float)n_s[e] / ntot : 0.f;
+    if (f_out != nullptr) f_out[s * E + e] = f;
+    v += f * p_s[e];
+  }
+  red[threadIdx.x] = v;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) part[s] = red[0];
+}
+
+// losses[0] = alpha E mean_s part[s], losses[1] = lambda mean_t lse^2
+// (fixed-order block sums).
+__global__ void __launch_bounds__(256)
+seq_aux_final_kernel(const float* __restrict__ part, const float* __restrict__ z_part,
+                     int n_seq, int n_z, int T, int E, float alpha, float lambda,
                      float* __restrict__ losses) {
   pdl_begin();
   __shared__ float red[2][256];
   float a = 0.f, z = 0.f;
-  for (int i = threadIdx.x; i < n_seq; i += blockDim.x) { a += part[i]; z += zpart[i]; }
+  for (int i = threadIdx.x; i < n_seq; i += blockDim.x) a += part[i];
+  for (int i = threadIdx.x; i < n_z; i += blockDim.x) z += z_part[i];
   red[0][threadIdx.x] = a;
   red[1][threadIdx.x] = z;
   __syncthreads();

@@ -187,9 +187,10 @@ struct Layout {
   // tensor-core router products (router_tc)
   int64_t Ep;
   size_t off_wf, off_wb, off_rparts, off_dsf, off_dsb, off_dwr3, off_rdx;
-  // sequence-wise aux (seq_len > 0): per-sequence f [n_seq, E], partials
-  int64_t n_seq;
-  size_t off_seqf, off_seqp;
+  // sequence-wise aux (seq_len > 0): per-sequence f [n_seq, E]; partial
+  // counts / sums of n_split pieces of each sequence
+  int64_t n_seq, n_split;
+  size_t off_seqf, off_seqc, off_seqq, off_seqz, off_seqs;
 };
 constexpr int kAuxChunk = 128;
 
@@ -244,8 +245,14 @@ Layout layout_of(const moe_config_t* c) {
   }
   if (c->seq_len > 0) {
     L.n_seq = c->T / c->seq_len;
+    // pieces of up to 32 tokens, about two waves of blocks over all sequences
+    L.n_split = std::max<int64_t>(1, std::min<int64_t>(ceil_div(c->seq_len, 32),
+                                                       ceil_div(2 * 148, L.n_seq)));
     L.off_seqf = take((size_t)L.n_seq * c->E * 4);
-    L.off_seqp = take((size_t)2 * L.n_seq * 4);
+    L.off_seqc = take((size_t)L.n_seq * L.n_split * c->E * 4);
+    L.off_seqq = take((size_t)L.n_seq * L.n_split * c->E * 4);
+    L.off_seqz = take((size_t)L.n_seq * L.n_split * 4);
+    L.off_seqs = take((size_t)L.n_seq * 4);
   }
   L.total = off;
   return L;
@@ -779,6 +786,42 @@ int moe_router(const moe_config_t* c, const void* x, const float* w_r, const flo
 
 }  // extern "C"
 
+// Sequence-wise aux partials over (piece, sequence) blocks, then the final
+// reduction: losses (if given) and the per-sequence f (if given).
+int seq_aux_launch(const moe_config_t* c, const Layout& L, const float* probs, const float* lse,
+                   const int32_t* topk_idx, const int32_t* slot_row, int norm, float* losses,
+                   float* f_out, void* ws, cudaStream_t s) {
+  int32_t* cnt = wsp<int32_t>(ws, L.off_seqc);
+  float* qp = wsp<float>(ws, L.off_seqq);
+  float* zp = wsp<float>(ws, L.off_seqz);
+  const dim3 grid((unsigned)L.n_split, (unsigned)L.n_seq);
+  auto go = [&](auto nv) -> int {
+    prof_begin(s);
+    MOE_CK((launch_k(seq_aux_partial_kernel<decltype(nv)::value>, grid, 256, 0, s, probs, lse,
+                     topk_idx, slot_row, c->seq_len, c->K, c->E, norm, cnt, qp, zp)));
+    MOE_LAUNCHED(s, "seq_aux_partial");
+    return MOE_OK;
+  };
+  if (c->E <= 32) MOE_TRY(go(std::integral_constant<int, 1>{}));
+  else if (c->E <= 64) MOE_TRY(go(std::integral_constant<int, 2>{}));
+  else if (c->E <= 128) MOE_TRY(go(std::integral_constant<int, 4>{}));
+  else if (c->E <= 256) MOE_TRY(go(std::integral_constant<int, 8>{}));
+  else MOE_TRY(go(std::integral_constant<int, 16>{}));
+  float* part = wsp<float>(ws, L.off_seqs);
+  prof_begin(s);
+  MOE_CK((launch_k(seq_aux_seq_kernel, (int)L.n_seq, 256, 0, s, cnt, qp, (int)L.n_split,
+                   c->seq_len, c->E, part, f_out)));
+  MOE_LAUNCHED(s, "seq_aux_seq");
+  if (losses != nullptr) {
+    prof_begin(s);
+    MOE_CK((launch_k(seq_aux_final_kernel, 1, 256, 0, s, part, zp, (int)L.n_seq,
+                     (int)(L.n_seq * L.n_split), c->T, c->E, c->aux_alpha, c->z_lambda,
+                     losses)));
+    MOE_LAUNCHED(s, "seq_aux_final");
+  }
+  return MOE_OK;
+}
+
 template <typename TX>
 int route_ec_impl(const moe_config_t* c, const TX* x, const float* w_r, const float* off,
                   float* logits, float* probs, float* lse, int32_t* idx, float* w,
@@ -955,25 +998,8 @@ int moe_aux_loss_seq(const moe_config_t* c, const float* probs, const float* lse
   if (!probs || !lse || !topk_idx || !slot_row || !losses || !ws || c->seq_len <= 0)
     return MOE_ERR_ARG;
   const Layout L = layout_of(c);
-  float* part = wsp<float>(ws, L.off_seqp);
-  float* zpart = part + L.n_seq;
   const int norm = c->score_fn == MOE_SOFTMAX ? 0 : 1;
-  auto go = [&](auto nv) -> int {
-    prof_begin(s);
-    MOE_CK((launch_k(seq_aux_kernel<decltype(nv)::value>, (int)L.n_seq, 256, 0, s, probs, lse,
-                     topk_idx, slot_row, c->seq_len, c->K, c->E, norm, part, zpart)));
-    MOE_LAUNCHED(s, "seq_aux");
-    return MOE_OK;
-  };
-  if (c->E <= 32) MOE_TRY(go(std::integral_constant<int, 1>{}));
-  else if (c->E <= 64) MOE_TRY(go(std::integral_constant<int, 2>{}));
-  else if (c->E <= 128) MOE_TRY(go(std::integral_constant<int, 4>{}));
-  else if (c->E <= 256) MOE_TRY(go(std::integral_constant<int, 8>{}));
-  else MOE_TRY(go(std::integral_constant<int, 16>{}));
-  prof_begin(s);
-  MOE_CK((launch_k(seq_aux_final_kernel, 1, 256, 0, s, part, zpart, (int)L.n_seq, c->T, c->E,
-                   c->aux_alpha, c->z_lambda, losses)));
-  MOE_LAUNCHED(s, "seq_aux_final");
+  MOE_TRY(seq_aux_launch(c, L, probs, lse, topk_idx, slot_row, norm, losses, nullptr, ws, s));
   return MOE_OK;
 }
 
@@ -1154,10 +1180,9 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       // per-sequence f for the sequence-wise aux gradient
       a.seq_len = c->seq_len;
       a.seq_f = wsp<float>(ws, L.off_seqf);
-      prof_begin(r);
-      MOE_CK((launch_k(seq_f_kernel, (int)L.n_seq, 256, 0, r, topk_idx, slot_row, c->seq_len, K,
-                       E, wsp<float>(ws, L.off_seqf))));
-      MOE_LAUNCHED(r, "seq_f");
+      MOE_TRY(seq_aux_launch(c, L, probs, lse, topk_idx, slot_row,
+                             c->score_fn == MOE_SOFTMAX ? 0 : 1, nullptr,
+                             wsp<float>(ws, L.off_seqf), ws, r));
     }
     if (rtc) {
       a.dsf = wsp<__nv_bfloat16>(ws, L.off_dsf);
