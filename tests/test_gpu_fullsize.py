@@ -98,3 +98,77 @@ def test_parity_full_size(name):
     print("%s full: near-tie flips %d, GPU near-ties %d, drops %d, sentinels %d, "
           "sampled tokens %s" % (name, flips, int(layer.near_ties[0]), int(layer.stats[0]),
                                   int(layer.stats[1]), toks))
+
+
+def test_expert_choice_full_size():
+    """Expert choice on the OLMoE shape at full size (64 experts, each
+    picking 2048 of 16384 tokens): every expert's picks against the oracle
+    (near-ties excepted), then sampled tokens and weight-gradient columns."""
+    from oracle import expert_choice as X
+    cfg = W.CONFIGS["olmoe_ec"]
+    tl = 2e-2
+    layer, inp = run_gpu(cfg)
+    torch.cuda.synchronize()
+    x = np64(W.make_input(cfg, "x"))
+    L = LazyLayer(cfg, x)
+    R, chosen, C = X.route(L, cfg.capacity_factor, cfg.min_capacity)
+    assert rel_l2(host(layer.logits), R.logits) < 1e-5
+    assert rel_l2(host(layer.probs), R.p) < 1e-5
+    got = layer.ec_mask.cpu().numpy().reshape(cfg.T, cfg.E) == 0
+    assert np.all(got.sum(axis=0) == C)
+    flip = (got != chosen).any(axis=0)
+    assert np.all(X.ec_margin(R.p, C)[flip] < O.NEAR_TIE), np.nonzero(flip)[0]
+    if flip.any():
+        return
+    L.sentinel_mask = ~chosen.reshape(-1)
+    o = X.opts_for(cfg.E, cfg.z_lambda)
+    Dp = O.dispatch(R.idx, cfg.E, 0.0, 0, L.sentinel_mask)
+    assert np.array_equal(host(layer.counts), np.full(cfg.E, C))
+    z = O.z_loss(R.lse, cfg.z_lambda)
+    assert abs(float(layer.losses[1]) - z) <= 1e-4 * z
+    rng = np.random.default_rng(1)
+    picked = chosen.sum(axis=1)
+    toks = sorted({0, cfg.T - 1, int(np.argmax(picked)), int(np.argmin(picked)),
+                   *[int(t) for t in rng.integers(0, cfg.T, size=4)]})
+    dyt = np64(W.make_input(cfg, "dy", rows=np.array(toks)))
+    ref = {k: [] for k in ("y", "dg", "ds", "dx")}
+    for i, t in enumerate(toks):
+        r = O.token_forward_backward(L, o, R, Dp, t, dyt[i])
+        for k in ref:
+            ref[k].append(r[k])
+    got = {"y": host(layer.y[toks]), "dg": host(layer.dg[toks]),
+           "ds": host(layer.dlogits[toks]), "dx": host(layer.dx[toks])}
+    for k in ref:
+        assert rel_l2(got[k], np.stack(ref[k])) < tl, (k, rel_l2(got[k], np.stack(ref[k])))
+    dy_rows = lambda rows: np64(W.make_input(cfg, "dy", rows=np.asarray(rows)))
+    for e in (0, int(rng.integers(1, cfg.E))):
+        j = int(rng.integers(0, cfg.F))
+        g_gate, g_up, g_down = O.expert_column_grads(L, o, R, Dp, e, j, dy_rows)
+        assert rel_l2(host(layer.dw13[e, j]), g_gate) < tl
+        assert rel_l2(host(layer.dw13[e, cfg.F + j]), g_up) < tl
+        assert rel_l2(host(layer.dw_down[e, :, j]), g_down) < tl
+    dwr = host(layer.dlogits).astype(np.float64).T @ x
+    assert rel_l2(host(layer.dw_r), dwr) < 1e-4
+    print("olmoe_ec full: picks per token %d..%d, sampled tokens %s, GPU near-ties %d" % (
+        picked.min(), picked.max(), toks, int(layer.near_ties[0])))
+
+
+@pytest.mark.parametrize("n_seq", [1, 4])
+def test_sequence_wise_aux_full_size(n_seq):
+    """The sequence-wise aux loss on the full OLMoE-shaped layer against the
+    oracle's own routing: one sequence equals the batch loss; four sequences
+    follow oracle/balance.py."""
+    from oracle import balance as B
+    cfg = W.CONFIGS["olmoe"].replace(seq_len=W.CONFIGS["olmoe"].T // n_seq)
+    layer, inp = run_gpu(cfg)
+    torch.cuda.synchronize()
+    x = np64(W.make_input(cfg, "x"))
+    L = LazyLayer(cfg, x)
+    o = O.opts_of(cfg)
+    R = O.route_layer(L, o)
+    Dp = O.dispatch(R.idx, cfg.E, cfg.capacity_factor, cfg.min_capacity, L.sentinel_mask)
+    ref, _, _ = B.seq_aux_loss(R.p, Dp.expert, cfg.K, cfg.aux_alpha, cfg.seq_len, B.SOFTMAX)
+    if n_seq == 1:
+        batch, _, _ = O.aux_loss(Dp.counts, R.p, cfg.aux_alpha, cfg.E)
+        assert abs(ref - batch) <= 1e-12 * batch
+    assert abs(float(layer.losses[0]) - ref) <= 1e-4 * ref
