@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--config", default="mm_b", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--gather", type=int, default=0, choices=[0, 1],
+                    help="1: the gate/up GEMMs read token rows of x by tile::gather4 "
+                         "(no permuted copy of x); 0: the dispatch writes x_perm")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="sequence-wise aux loss over groups of this many tokens")
     ap.add_argument("--aux-alpha", type=float, default=None)
@@ -287,7 +290,7 @@ def run_ours(args):
         "sel_bias": W.make_input(base, "sel_bias", dev) if base.sel_bias_range else None,
         "sentinel_mask": W.make_input(cfg, "sentinel_mask", dev) if base.sentinel_frac else None,
     }
-    layer = MoELayer(config_from(base), device=dev)
+    layer = MoELayer(config_from(base), device=dev, gather=bool(args.gather))
     weights = dict(w_r=inp["w_r"], w13=inp["w13"], w_down=inp["w_down"], **opt)
     x, dy = inp["x"], inp["dy"]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -560,6 +563,8 @@ def run_ours(args):
                 "global_batch_tokens": base.T * world, "parallelism": "dp%d (replicas)" % world,
                 "l2": "flushed between timed steps (256 MiB write)",
                 "cuda_graph": graph is not None,
+                "row_gather": ("inside the gate/up GEMMs (tile::gather4 rows of x)"
+                               if args.gather else "dispatch kernel writes x_perm"),
                 "programmatic_dependent_launch": os.environ.get("MOE_PDL", "1") != "0"},
             "e2e": {"value": round(base.T * world / (e2e * 1e-3), 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -176,7 +176,9 @@ int moe_router(const moe_config_t* cfg, const void* x, const float* w_r,
  *   row_slot      [rows_max] i32 out: slot of each routed row, -1 otherwise
  *   tile_expert   [tiles_max] i32 out: expert of each 128-row tile (E = shared)
  *   stats         [4] i32 out: n_dropped, n_sentinel, n_rows, n_tiles
- *   x_perm        [rows_max,D] act out: gathered rows, zero padding
+ *   x_perm        [rows_max,D] act out: gathered rows, zero padding; NULL:
+ *                 layout only (no gather launched), for the fused-gather
+ *                 path (moe_expert_ffn_gather, moe_backward with NULL x_perm)
  * Slots of one expert are ranked in flat slot order j = t*K + k; ranks >= C
  * are dropped.
  */
@@ -288,6 +290,31 @@ int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
                    void* a13, void* h, void* o, void* ws, cudaStream_t stream);
 
 /*
+ * moe_expert_ffn_gather — moe_expert_ffn without the permuted copy of x:
+ * the gate/up GEMM loads its A rows straight from the token rows of x with
+ * TMA tile::gather4 copies (four rows of 64 columns per copy), so x_perm is
+ * never written or read.  Same method, one HBM round trip less: the pages
+ * group tokens into contiguous per-expert blocks before the grouped GEMM
+ * ([8MOE] MoE 高效推理; [STA324 §8.8]); here the grouping happens inside the
+ * GEMM's operand load.
+ *   x         [T,D] act: layer input (the tensor moe_dispatch was given)
+ *   row_slot  [rows_max] i32 (moe_dispatch): permuted row r holds token
+ *             row_slot[r] / K; rows of the shared group hold token
+ *             r - offsets[E]; padding rows load as zeros
+ *   offsets   [E+2] i32 (moe_dispatch)
+ *   the rest as moe_expert_ffn; the outputs are identical to moe_expert_ffn
+ *   on the x_perm that moe_dispatch would have written.
+ * bf16 layers on the tensor-core path only (MOE_ERR_ARG for fp32 layers or
+ * gemm_mode MOE_GEMM_SIMT).
+ */
+int moe_expert_ffn_gather(const moe_config_t* cfg, const void* x,
+                          const int32_t* row_slot, const int32_t* offsets,
+                          const int32_t* tile_expert, const int32_t* stats,
+                          const void* w13, const void* w_down,
+                          const void* w13_s, const void* w_down_s,
+                          void* a13, void* h, void* o, void* ws, cudaStream_t stream);
+
+/*
  * moe_combine — y_t = sum_{k kept} g_{t,k} o[slot_row[t*K+k]] (k ascending,
  * fp32 accumulation) + o[offsets[E] + t] when n_shared.  Deterministic
  * gather, no atomics.  [8MOE] Router / Gating Network (y = sum G(x)_i
@@ -313,6 +340,10 @@ int moe_combine(const moe_config_t* cfg, const void* o,
  * The gate gradient of a sentinel or dropped slot is zero (its expert
  * output is treated as zero), so such slots send no gradient to the router
  * through the gate path.  Deterministic: no floating-point atomics.
+ * x_perm may be NULL on the tensor-core path (bf16 layers): the gate/up
+ * weight-gradient GEMM then gathers its x rows by row_slot with tile::gather4
+ * copies, as moe_expert_ffn_gather does (MOE_ERR_ARG for NULL x_perm on the
+ * SIMT path).
  * Inside the call, independent chains (the router gradient, the two
  * weight-gradient GEMMs) are forked onto side streams that the library
  * creates once per host thread and device (on first use: make that first

@@ -20,6 +20,9 @@
 //     WGRAD mode: C_g[m, n] = sum_{r in rows(g)} A[r, m] B[r, n] (weight
 //     gradients; the reduction runs over the group's own rows and the zero
 //     padding rows beyond them contribute nothing);
+//   * GATHER variants copy the row operand (gate/up A rows, gate/up wgrad B
+//     rows) straight from the token rows of x with cp.async in the
+//     producer warp, instead of TMA boxes of a permuted copy;
 //   * dense variants (no tile map, one group, fp32 epilogues) serve the
 //     router's fp32 products, which run as bf16 MMAs on three-way bf16
 //     splits of the fp32 operand (x . W_r^T, ds^T . x, ds . W_r);
@@ -70,6 +73,13 @@ struct Params {
   int dense_rows;              // WGRAD: > 0 = one group of dense_rows rows
   int m_limit;                 // WGRAD_F32: output rows
   float* out_f32; int64_t ld_f32;          // F32 epilogues
+  // gathered rows (the GATHER kernels copy token rows of x instead of
+  // reading a permuted copy): row r holds token row_slot[r] / gK, or token
+  // r - offsets[E] inside the shared group, or zeros (padding)
+  const __nv_bfloat16* gx;     // x [T, Kd] (ROWS) or [T, No] (WGRAD)
+  const int32_t* row_slot;
+  int gK;                      // slots per token
+  int shared_T;                // rows of the shared group (0: none)
 };
 
 // ----------------------------------------------------------------------------
@@ -99,17 +109,35 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same with cluster-scope acquire: the phase was completed by arrivals
+// (release.cluster) from the other CTA of a pair after it wrote shared
+// memory that this CTA's tensor-core instructions read.
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
 // Bounded wait for phase `parity` of `bar`.  False once the kernel aborted.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       bool cluster_acquire = false) {
+  auto probe = [&] {
+    return cluster_acquire ? mbar_try_cluster(bar, parity) : mbar_try(bar, parity);
+  };
+  if (probe()) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try(bar, parity)) return true;
+    if (probe()) return true;
     if ((i & 63u) == 0u) {
       if (*abort_flag) return false;
       if (global_ns() - t0 > kWaitLimitNs) {
@@ -299,6 +327,32 @@ __device__ __forceinline__ void tma_2d_hint(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// ---- row gather: 16-byte cp.async copies ------------------------------------
+// A gathered operand row (128 bytes of one k block) is copied by 8 lanes,
+// 16 bytes each, into the 128B-swizzled layout a TMA box load would have
+// produced: chunk c of tile row r lands at r * 128 + ((c ^ (r & 7)) << 4)
+// from a 1024-byte aligned tile.  src_bytes = 0 writes zeros (padding rows)
+// without reading.  Each copying lane arrives on the stage's full barrier
+// when its copies complete (no wait in the producer); the copies are
+// generic-proxy writes, so the MMA thread fences them into the async proxy
+// after its barrier wait and before the tensor cores read the stage.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` (counted in its expected arrivals) once every cp.async
+// this thread issued so far has completed; the thread does not wait.
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // 32 floats -> 32 bf16 at p (64 bytes, 16-byte aligned), with an L2 policy.
 __device__ __forceinline__ void store32_bf16(__nv_bfloat16* p, const float (&v)[32],
                                              uint64_t pol) {
@@ -453,14 +507,22 @@ struct Smem {
   static constexpr int kA = BM * BK * 2;        // 16 KB
   static constexpr int kB = BNC * BK * 2;
   static constexpr int kStage = kA + kB;
-  static constexpr int kBars = (2 * STAGES + 5) * 8;
+  static constexpr int kBars = (3 * STAGES + 5) * 8;   // full, empty, copies-done, acc, done
+  // token table of the gathering producer (128 rows)
+  static constexpr int kTokOff = STAGES * kStage + kBars + 16;
   // epilogue staging tiles (one per epilogue warp), 128-byte aligned
-  static constexpr int kEpiOff = (STAGES * kStage + kBars + 16 + 127) / 128 * 128;
+  static constexpr int kEpiOff = (kTokOff + 512 + 127) / 128 * 128;
   static constexpr int kBytes = 1024 + kEpiOff + kEpiWarps * kStgBytes;
   static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
-template <int BN, int STAGES, int MODE, bool A_MN, bool B_MN, int EPI, bool PAIR>
+// GATHER: the row operand comes from the token rows of x (Params.row_slot)
+// by tile::gather4 copies issued by the whole producer warp: the A rows of a
+// ROWS tile (gate/up + SwiGLU), or the B rows of a WGRAD k block (gate/up
+// weight gradient).  mapA (ROWS) or mapB (WGRAD) is then x [T, D] with a
+// {64, 1} box.
+template <int BN, int STAGES, int MODE, bool A_MN, bool B_MN, int EPI, bool PAIR,
+          bool GATHER = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
             const __grid_constant__ CUtensorMap mapBs, const Params p, int total_hint) {
@@ -478,6 +540,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   auto accf_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
   auto acce_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
   const uint32_t done_bar = bars + 8u * (2 * STAGES + 4);
+  // gathered rows in a pair's second CTA: its lanes' cp.async copies arrive
+  // here; warp 1 forwards each completed stage to the leader's full barrier
+  auto cpd_bar = [&](int s) { return bars + 8u * (2 * STAGES + 5 + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * S::kStage + S::kBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -493,7 +558,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
 
   if (threadIdx.x == 0) {
     abort_flag_s = 0;
-    for (int s = 0; s < STAGES; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+    // full barrier: the arming arrive (TMA bytes); with gathered rows also
+    // one arrive per producer lane when its copies of the stage complete,
+    // and in a pair the other CTA's forwarded arrive
+    const uint32_t n_full = GATHER ? (PAIR ? 34u : 33u) : 1u;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), n_full);
+      mbar_init(empty_bar(s), 1);
+      mbar_init(cpd_bar(s), 32);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(accf_bar(b), 1);
       mbar_init(acce_bar(b), kEpiWarps * (PAIR ? 2 : 1));   // both CTAs' epilogues
@@ -539,8 +612,146 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   };
 
   if (warp == 0) {
-    // ---------------- TMA producer (both CTAs of a pair) ----------------
-    if (lane == 0) {
+    if constexpr (GATHER) {
+      // ---------- producer with gathered rows (whole warp) ----------
+      // The row operand (A of a ROWS tile, B of a WGRAD k block) is copied
+      // from the token rows of x with 16-byte cp.async: one warp
+      // instruction moves 4 rows x 128 bytes (lane = 8 * row + chunk).  The
+      // tile's (ROWS) or k block's (WGRAD) tokens go through a small
+      // shared table; row slots are loaded one tile / k block ahead.  Lane 0
+      // waits for free stages, arms the barrier for the TMA box loads of
+      // the other operand and issues them.
+      static_assert((MODE == MODE_ROWS && EPI == EPI_SWIGLU && !A_MN) ||
+                        (MODE == MODE_WGRAD && B_MN),
+                    "gathered operands: gate/up A rows or gate/up wgrad B rows");
+      constexpr int kRowsG = MODE == MODE_ROWS ? BM : BK;   // gathered rows per stage
+      int32_t* tok_s = reinterpret_cast<int32_t*>(gbase + S::kTokOff);
+      const uint32_t tok_a = smem_u32(tok_s);
+      const int shared0 = p.offsets[p.E];
+      const int cch = lane & 7, rsub = lane >> 3;
+      // first row of the gathered rows this lane's slot loads cover
+      auto lane_row = [&](const Tile& d, int kb) {
+        return MODE == MODE_ROWS ? d.m0 + 4 * lane : d.row0 + kb * BK + 2 * lane;
+      };
+      constexpr int kSl = kRowsG / 32;   // slots per lane: 4 (ROWS) or 2 (WGRAD)
+      auto load_slots = [&](const Tile& d, int kb, bool valid, int (&v)[kSl]) {
+        const int32_t* q = p.row_slot + lane_row(d, kb);
+#pragma unroll
+        for (int i = 0; i < kSl; ++i) v[i] = valid ? q[i] : -1;
+      };
+      auto token = [&](int r, int sl) {
+        if (sl >= 0) return sl / p.gK;
+        const int u = r - shared0;
+        return (u >= 0 && u < p.shared_T) ? u : -1;   // -1: zeros
+      };
+      int sl[kSl];
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued_parity[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+      // the gathered rows of one stage -> this lane's tokens (row rsub + 4 i)
+      int tk[kRowsG / 4];
+      auto publish = [&](const Tile& d, int kb) {
+        const int r = lane_row(d, kb);
+        __syncwarp();   // every lane has read the previous table
+#pragma unroll
+        for (int i = 0; i < kSl; ++i)
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(tok_a + 4u * (kSl * lane + i)),
+                       "r"(token(r + i, sl[i]))
+                       : "memory");
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kRowsG / 4; ++i) {
+          int v;
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(tok_a + 4u * (rsub + 4 * i)) : "memory");
+          tk[i] = v;
+        }
+      };
+      bool ok = true;
+      Tile nxt = decode_at(unit);
+      load_slots(nxt, 0, unit < total && nxt.nk > 0, sl);
+      for (int t = unit; t < total && ok; t += n_units) {
+        const Tile d = nxt;
+        nxt = decode_at(t + n_units);
+        const bool nxt_ok = t + n_units < total && nxt.nk > 0;
+        if (d.nk == 0) { load_slots(nxt, 0, nxt_ok, sl); continue; }
+        const CUtensorMap* mb = (MODE == MODE_ROWS && d.e >= p.E) ? &mapBs : &mapB;
+        const int eb = (MODE == MODE_ROWS && d.e >= p.E) ? 0 : d.e;
+        if (MODE == MODE_ROWS) {
+          publish(d, 0);
+          load_slots(nxt, 0, nxt_ok, sl);
+        }
+        for (int kb = 0; kb < d.nk; ++kb) {
+          if (MODE == MODE_WGRAD) {
+            publish(d, kb);
+            if (kb + 1 < d.nk) load_slots(d, kb + 1, true, sl);
+            else load_slots(nxt, 0, nxt_ok, sl);
+          }
+          int w = 1;
+          if (lane == 0) w = mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) ? 1 : 0;
+          if (__shfl_sync(0xffffffffu, w, 0) == 0) { ok = false; break; }
+          const uint32_t sa = base + stage * S::kStage;
+          const uint32_t sb = sa + S::kA;
+          const uint32_t fb = full_bar(stage);
+          if (lane == 0) {
+            const uint32_t tb = PAIR ? mapa(fb, 0) : fb;   // barrier the TMA copies complete on
+            const uint32_t box_bytes = MODE == MODE_ROWS ? S::kB : S::kA;
+            if (!PAIR || leader) mbar_expect_tx(fb, box_bytes * (PAIR ? 2 : 1));
+            issued_parity[stage] = (int)phase;
+            if constexpr (MODE == MODE_ROWS) {
+              if constexpr (PAIR) {
+                tma_3d_pair(sb, mb, tb, kb * BK, (rank ? p.F : 0) + d.n0, eb);
+              } else {
+                tma_3d(sb, mb, tb, kb * BK, d.n0, eb);
+                tma_3d(sb + (BN / 2) * 128, mb, tb, kb * BK, p.F + d.n0, eb);
+              }
+            } else {
+              const int r = d.row0 + kb * BK;
+              if constexpr (PAIR) {
+                tma_2d_pair_nohint(sa, &mapA, tb, d.m0, r);
+                tma_2d_pair_nohint(sa + 8192, &mapA, tb, d.m0 + 64, r);
+              } else {
+                tma_2d(sa, &mapA, tb, d.m0, r);
+                tma_2d(sa + 8192, &mapA, tb, d.m0 + 64, r);
+              }
+            }
+          }
+          if constexpr (MODE == MODE_ROWS) {
+            // A: 128 rows x 64 columns of x; row rsub + 4 i, chunk cch
+            const __nv_bfloat16* src0 = p.gx + kb * BK + cch * 8;
+#pragma unroll
+            for (int i = 0; i < BM / 4; ++i) {
+              const int r = rsub + 4 * i;
+              const int tkn = tk[i];
+              cp_async16(sa + r * 128 + ((cch ^ (r & 7)) << 4),
+                         src0 + (int64_t)(tkn < 0 ? 0 : tkn) * p.Kd, tkn < 0 ? 0u : 16u);
+            }
+          } else {
+            // B: 64 rows (k) x BNC columns of x, in 64-column boxes
+            const int col0 = d.n0 + (PAIR ? rank * BNC : 0) + cch * 8;
+#pragma unroll
+            for (int c = 0; c < BNC / 64; ++c) {
+              const __nv_bfloat16* src0 = p.gx + col0 + c * 64;
+#pragma unroll
+              for (int i = 0; i < BK / 4; ++i) {
+                const int r = rsub + 4 * i;
+                const int tkn = tk[i];
+                cp_async16(sb + c * 8192 + r * 128 + ((cch ^ (r & 7)) << 4),
+                           src0 + (int64_t)(tkn < 0 ? 0 : tkn) * p.No, tkn < 0 ? 0u : 16u);
+              }
+            }
+          }
+          cp_async_arrive(PAIR && !leader ? cpd_bar(stage) : fb);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      cp_async_wait_all();   // no copy of this CTA in flight at teardown
+      if (lane == 0 && (!PAIR || leader))
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_parity[s] >= 0) mbar_wait(full_bar(s), (uint32_t)issued_parity[s], abort_flag);
+    } else if (lane == 0) {
+      // ---------------- TMA producer (both CTAs of a pair) ----------------
       const uint64_t pol_a = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
@@ -614,6 +825,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           if (issued_parity[s] >= 0) mbar_wait(full_bar(s), (uint32_t)issued_parity[s], abort_flag);
     }
   } else if (warp == 1) {
+    if constexpr (PAIR && GATHER) {
+      // ---- second CTA of a pair: forward completed gathered stages ----
+      if (lane == 0 && !leader) {
+        int stage = 0;
+        uint32_t phase = 0;
+        Tile nxt = decode_at(unit);
+        bool ok = true;
+        for (int t = unit; t < total && ok; t += n_units) {
+          const Tile d = nxt;
+          nxt = decode_at(t + n_units);
+          for (int kb = 0; kb < d.nk; ++kb) {
+            if (!mbar_wait(cpd_bar(stage), phase, abort_flag)) { ok = false; break; }
+            fence_proxy_async();
+            mbar_arrive_remote(mapa(full_bar(stage), 0));
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
+        }
+      }
+    }
     // ---------------- MMA issuer (the pair leader only) ----------------
     if (lane == 0 && leader) {
       constexpr uint32_t idesc = make_idesc(PAIR ? 2 * BM : BM, BN, A_MN, B_MN);
@@ -631,7 +861,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
         tc_fence_after();
         const uint32_t dt = tmem + acc * BN;
         for (int kb = 0; kb < d.nk; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, PAIR && GATHER)) { ok = false; break; }
+          if constexpr (GATHER) fence_proxy_async();   // cp.async rows -> async proxy
           tc_fence_after();
           const uint32_t sa = base + stage * S::kStage;
           const uint32_t sb = sa + S::kA;

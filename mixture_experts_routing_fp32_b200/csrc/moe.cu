@@ -330,12 +330,12 @@ cudaError_t launch_k(void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&lc, kern, std::forward<A>(args)...);
 }
 
-template <int BN, int ST, int MODE, bool AMN, bool BMN, int EPI, bool PAIR>
+template <int BN, int ST, int MODE, bool AMN, bool BMN, int EPI, bool PAIR, bool GATHER>
 int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
               const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
               cudaStream_t s) {
   using S = tc::Smem<BN, ST, PAIR>;
-  auto k = tc::gemm_kernel<BN, ST, MODE, AMN, BMN, EPI, PAIR>;
+  auto k = tc::gemm_kernel<BN, ST, MODE, AMN, BMN, EPI, PAIR, GATHER>;
   MOE_CK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes));
   if constexpr (PAIR) {
     // as many CTA pairs as can be resident at once (one per two SMs of a GPC)
@@ -376,31 +376,31 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
   return MOE_OK;
 }
 
-template <int MODE, bool AMN, bool BMN, int EPI, bool PAIR = false>
+template <int MODE, bool AMN, bool BMN, int EPI, bool PAIR = false, bool GATHER = false>
 int run_tc(int bn, const char* name, const CUtensorMap& a, const CUtensorMap& b,
            const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
            cudaStream_t s) {
   if constexpr (PAIR) {
     // per CTA: A 16 KB + half of B per stage
     if (bn == 256)
-      return launch_tc<256, 6, MODE, AMN, BMN, EPI, true>(name, a, b, bs, p, total_max,
-                                                         total_hint, s);
+      return launch_tc<256, 6, MODE, AMN, BMN, EPI, true, GATHER>(name, a, b, bs, p, total_max,
+                                                                 total_hint, s);
     if (bn == 128)
-      return launch_tc<128, 8, MODE, AMN, BMN, EPI, true>(name, a, b, bs, p, total_max,
-                                                         total_hint, s);
+      return launch_tc<128, 8, MODE, AMN, BMN, EPI, true, GATHER>(name, a, b, bs, p, total_max,
+                                                                 total_hint, s);
     return MOE_ERR_ARG;
   } else {
     if (bn == 256)
-      return launch_tc<256, 4, MODE, AMN, BMN, EPI, false>(name, a, b, bs, p, total_max,
-                                                          total_hint, s);
+      return launch_tc<256, 4, MODE, AMN, BMN, EPI, false, GATHER>(name, a, b, bs, p, total_max,
+                                                                  total_hint, s);
     if constexpr (EPI != tc::EPI_SWIGLU) {
       if (bn == 192)
-        return launch_tc<192, 5, MODE, AMN, BMN, EPI, false>(name, a, b, bs, p, total_max,
-                                                            total_hint, s);
+        return launch_tc<192, 5, MODE, AMN, BMN, EPI, false, GATHER>(name, a, b, bs, p,
+                                                                    total_max, total_hint, s);
     }
     if (bn == 128)
-      return launch_tc<128, 6, MODE, AMN, BMN, EPI, false>(name, a, b, bs, p, total_max,
-                                                          total_hint, s);
+      return launch_tc<128, 6, MODE, AMN, BMN, EPI, false, GATHER>(name, a, b, bs, p, total_max,
+                                                                  total_hint, s);
     return MOE_ERR_ARG;
   }
 }
@@ -738,6 +738,7 @@ int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_id
                      L.n_slots, E, L.C, L.rows_max, bhist, offsets, slot_row, row_slot)));
     MOE_LAUNCHED(s, "dispatch_rank");
   }
+  if (x_perm == nullptr) return MOE_OK;   // layout only: the GEMMs gather x rows
   const int grid = grid_for(L.rows_max);
   prof_begin(s);
   if (c->dtype == MOE_BF16)
@@ -904,7 +905,7 @@ int moe_dispatch(const moe_config_t* c, const int32_t* topk_idx, const uint8_t* 
                  void* x_perm, void* ws, cudaStream_t s) {
   MOE_TRY(validate(c));
   if (!topk_idx || !x || !counts || !kept || !offsets || !slot_row || !row_slot ||
-      !tile_expert || !stats || !x_perm || !ws)
+      !tile_expert || !stats || !ws)
     return MOE_ERR_ARG;
   const Layout L = layout_of(c);
   return dispatch_impl(c, L, topk_idx, sentinel_mask, x, counts, kept, offsets, slot_row,
@@ -959,7 +960,7 @@ int moe_dispatch_static(const moe_config_t* c, const int32_t* topk_idx,
                         int32_t* tile_expert, int32_t* stats, void* x_perm, cudaStream_t s) {
   MOE_TRY(validate(c));
   if (!topk_idx || !x || !counts || !kept || !offsets || !slot_row || !row_slot ||
-      !tile_expert || !stats || !x_perm)
+      !tile_expert || !stats)
     return MOE_ERR_ARG;
   const Layout L = layout_of(c);
   // scratch: n_blocks x E histogram entries + n_blocks sentinel counts.  Both
@@ -1013,52 +1014,77 @@ int moe_bias_update(const moe_config_t* c, const int32_t* counts, float* sel_bia
   return MOE_OK;
 }
 
+}  // extern "C"
+
+namespace {
+// gate/up + SwiGLU and down on the tensor cores.  The gate/up A rows are
+// read from x_perm, or, with x_perm == nullptr, gathered from the token rows
+// of x by the GEMM itself (row_slot, offsets[E] for the shared group).
+int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, const void* x,
+                  const int32_t* row_slot, const int32_t* offsets, const int32_t* tile_expert,
+                  const int32_t* stats, const void* w13, const void* w_down, const void* w13_s,
+                  const void* w_down_s, void* a13, void* h, void* o, cudaStream_t s) {
+  const int D = c->D, F = c->F, E = c->E;
+  const bool gather = x_perm == nullptr;
+  CUtensorMap mA, mB, mBs;
+  const int64_t mt = row_tiles_estimate(c, L);
+  const bool pr = pair_rows(c);                 // CTA-pair row tiles
+  const int64_t units = pr ? L.tiles_max / 2 : L.tiles_max;
+  // gate/up + SwiGLU: A = x_perm [rows, D] (or rows of x [T, D] copied by
+  // the GEMM's producer warp: mapA unused); B = w13 [E, 2F, D] K-major
+  const int bn1 = pick_bn(2 * F, mt, true, F, pr);
+  MOE_TRY(make_map(&mA, gather ? x : x_perm, 1, gather ? c->T : L.rows_max, D, 128, false));
+  MOE_TRY(make_map(&mB, w13, E, 2 * F, D, bn1 / 2, true));
+  MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, bn1 / 2, true));
+  tc::Params p = rows_params(c, D, F / (bn1 / 2), tile_expert, stats, pr);
+  p.out = static_cast<__nv_bfloat16*>(a13); p.ld_out = 2 * F;
+  p.out2 = static_cast<__nv_bfloat16*>(h); p.ld_out2 = F;
+  p.offsets = offsets; p.row_slot = row_slot; p.gK = c->K;
+  p.shared_T = c->n_shared ? c->T : 0;
+  p.gx = static_cast<const __nv_bfloat16*>(x);
+  const char* n1 = "tc_gate_up_swiglu";
+  const int64_t tot1 = units * p.nN;
+  if (pr && gather)
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, true, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
+  else if (pr)
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
+  else if (gather)
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, false, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
+  else
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
+  // down: A = h [rows, F]; B = w_down [E, D, F] K-major (a pair CTA loads
+  // half of the BN rows)
+  const int bn2 = pick_bn(D, mt, false, F, pr);
+  const uint32_t box2 = pr ? bn2 / 2 : bn2;
+  MOE_TRY(make_map(&mA, h, 1, L.rows_max, F, 128, false));
+  MOE_TRY(make_map(&mB, w_down, E, D, F, box2, true));
+  MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, box2, true));
+  tc::Params q = rows_params(c, F, D / bn2, tile_expert, stats, pr);
+  q.out = static_cast<__nv_bfloat16*>(o); q.ld_out = D;
+  if (pr)
+    return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE, true>(
+        bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
+  return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE>(
+      bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
+}
+}  // namespace
+
+extern "C" {
+
 int moe_expert_ffn(const moe_config_t* c, const void* x_perm, const int32_t* offsets,
                    const int32_t* tile_expert, const int32_t* stats, const void* w13,
                    const void* w_down, const void* w13_s, const void* w_down_s, void* a13,
                    void* h, void* o, void* ws, cudaStream_t s) {
-  (void)offsets;
   (void)ws;
   MOE_TRY(validate(c));
   if (!x_perm || !tile_expert || !stats || !w13 || !w_down || !a13 || !h || !o)
     return MOE_ERR_ARG;
   if (c->n_shared && (!w13_s || !w_down_s)) return MOE_ERR_ARG;
   const Layout L = layout_of(c);
-  const int D = c->D, F = c->F, E = c->E;
-  if (use_tc(c)) {
-    CUtensorMap mA, mB, mBs;
-    const int64_t mt = row_tiles_estimate(c, L);
-    const bool pr = pair_rows(c);                 // CTA-pair row tiles
-    const int64_t units = pr ? L.tiles_max / 2 : L.tiles_max;
-    // gate/up + SwiGLU: A = x_perm [rows, D]; B = w13 [E, 2F, D] K-major
-    const int bn1 = pick_bn(2 * F, mt, true, F, pr);
-    MOE_TRY(make_map(&mA, x_perm, 1, L.rows_max, D, 128, false));
-    MOE_TRY(make_map(&mB, w13, E, 2 * F, D, bn1 / 2, true));
-    MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, bn1 / 2, true));
-    tc::Params p = rows_params(c, D, F / (bn1 / 2), tile_expert, stats, pr);
-    p.out = static_cast<__nv_bfloat16*>(a13); p.ld_out = 2 * F;
-    p.out2 = static_cast<__nv_bfloat16*>(h); p.ld_out2 = F;
-    if (pr)
-      MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, true>(
-          bn1, "tc_gate_up_swiglu", mA, mB, mBs, p, units * p.nN, 0, s)));
-    else
-      MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU>(
-          bn1, "tc_gate_up_swiglu", mA, mB, mBs, p, units * p.nN, 0, s)));
-    // down: A = h [rows, F]; B = w_down [E, D, F] K-major (a pair CTA loads
-    // half of the BN rows)
-    const int bn2 = pick_bn(D, mt, false, F, pr);
-    const uint32_t box2 = pr ? bn2 / 2 : bn2;
-    MOE_TRY(make_map(&mA, h, 1, L.rows_max, F, 128, false));
-    MOE_TRY(make_map(&mB, w_down, E, D, F, box2, true));
-    MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, box2, true));
-    tc::Params q = rows_params(c, F, D / bn2, tile_expert, stats, pr);
-    q.out = static_cast<__nv_bfloat16*>(o); q.ld_out = D;
-    if (pr)
-      return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE, true>(
-          bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
-    return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE>(
-        bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
-  }
+  const int D = c->D, F = c->F;
+  if (use_tc(c))
+    return expert_ffn_tc(c, L, x_perm, nullptr, nullptr, offsets, tile_expert, stats, w13,
+                         w_down, w13_s, w_down_s, a13, h, o, s);
   auto go = [&](auto tag) -> int {
     using TE = decltype(tag);
     MOE_TRY(simt_rows<TE>(c, L, x_perm, D, w13, D, 1, (int64_t)2 * F * D, w13_s, a13, 2 * F,
@@ -1072,6 +1098,23 @@ int moe_expert_ffn(const moe_config_t* c, const void* x_perm, const int32_t* off
   };
   if (c->dtype == MOE_BF16) return go(__nv_bfloat16{});
   return go(float{});
+}
+
+int moe_expert_ffn_gather(const moe_config_t* c, const void* x, const int32_t* row_slot,
+                          const int32_t* offsets, const int32_t* tile_expert,
+                          const int32_t* stats, const void* w13, const void* w_down,
+                          const void* w13_s, const void* w_down_s, void* a13, void* h, void* o,
+                          void* ws, cudaStream_t s) {
+  (void)ws;
+  MOE_TRY(validate(c));
+  if (!use_tc(c)) return MOE_ERR_ARG;   // the gather rides on the tensor-core GEMM
+  if (!x || !row_slot || !offsets || !tile_expert || !stats || !w13 || !w_down || !a13 || !h ||
+      !o)
+    return MOE_ERR_ARG;
+  if (c->n_shared && (!w13_s || !w_down_s)) return MOE_ERR_ARG;
+  const Layout L = layout_of(c);
+  return expert_ffn_tc(c, L, nullptr, x, row_slot, offsets, tile_expert, stats, w13, w_down,
+                       w13_s, w_down_s, a13, h, o, s);
 }
 
 int moe_combine(const moe_config_t* c, const void* o, const int32_t* slot_row,
@@ -1130,9 +1173,10 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
                  void* dw_down_s, float* dg_out, float* dlogits_out, void* ws, cudaStream_t s) {
   MOE_TRY(validate(c));
   if (!x || !w_r || !logits || !probs || !lse || !topk_idx || !topk_w || !counts || !kept ||
-      !offsets || !slot_row || !row_slot || !tile_expert || !stats || !x_perm || !a13 || !h ||
+      !offsets || !slot_row || !row_slot || !tile_expert || !stats || !a13 || !h ||
       !o || !w13 || !w_down || !dy || !dx || !dw_r || !dw13 || !dw_down || !ws)
     return MOE_ERR_ARG;
+  if (!x_perm && !use_tc(c)) return MOE_ERR_ARG;   // only the tensor-core wgrad gathers
   if (c->n_shared && (!w13_s || !w_down_s || !dw13_s || !dw_down_s)) return MOE_ERR_ARG;
   const Layout L = layout_of(c);
   const int D = c->D, F = c->F, E = c->E, T = c->T, K = c->K;
@@ -1286,11 +1330,13 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
         MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE>(
             bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s)));
     }
-    // 6. wgrad gate/up: dW13[e] = dA13^T x_perm
+    // 6. wgrad gate/up: dW13[e] = dA13^T x_perm (x_perm == nullptr: the
+    // producer warp copies the B rows from x by row_slot; mapB unused)
     const bool pw6 = ((2 * F) % 256) == 0;
+    const bool g6 = x_perm == nullptr;
     const int bn6 = pick_bn(D, (int64_t)groups * (2 * F / 128), false, F, pw6);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 64, false));
-    MOE_TRY(make_map(&mB, x_perm, 1, L.rows_max, D, 64, false));
+    MOE_TRY(make_map(&mB, g6 ? x : x_perm, 1, g6 ? T : L.rows_max, D, 64, false));
     {
       tc::Params p{};
       p.E = E; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
@@ -1298,13 +1344,22 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       p.strideCE = (int64_t)2 * F * D;
       p.out = static_cast<__nv_bfloat16*>(dw13);
       p.out_shared = static_cast<__nv_bfloat16*>(dw13_s);
+      p.row_slot = row_slot; p.gK = K; p.shared_T = c->n_shared ? T : 0;
+      p.gx = static_cast<const __nv_bfloat16*>(x);
       const int total = p.n_groups * p.nMo * p.nNo;
-      if (pw6)
+      const char* n6 = "tc_wgrad_gate_up";
+      if (pw6 && g6)
+        MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, true, true>(
+            bn6, n6, mA, mB, mB, p, total, total, w2)));
+      else if (pw6)
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, true>(
-            bn6, "tc_wgrad_gate_up", mA, mB, mB, p, total, total, w2)));
+            bn6, n6, mA, mB, mB, p, total, total, w2)));
+      else if (g6)
+        MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, false, true>(
+            bn6, n6, mA, mB, mB, p, total, total, w2)));
       else
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-            bn6, "tc_wgrad_gate_up", mA, mB, mB, p, total, total, w2)));
+            bn6, n6, mA, mB, mB, p, total, total, w2)));
     }
   } else {
     auto go = [&](auto tag) -> int {

@@ -5,7 +5,10 @@ torch, stable pointers, so a whole step can be captured in a CUDA graph)
 and issues the entry points in order on the current stream:
 
   forward : moe_router -> moe_dispatch -> moe_expert_ffn -> moe_combine,
-            with moe_aux_loss on a side stream (joined before returning)
+            with moe_aux_loss on a side stream (joined before returning);
+            gather=True: moe_dispatch computes the layout only and
+            moe_expert_ffn_gather reads the token rows of x inside the
+            gate/up GEMM (no permuted copy of x; bf16 layers)
   backward: moe_backward
 
 No host synchronisation happens inside forward or backward.
@@ -19,8 +22,9 @@ from ._lib import MOE_BF16
 
 
 class MoELayer:
-    def __init__(self, cfg, device="cuda"):
+    def __init__(self, cfg, device="cuda", gather=False):
         self.cfg = cfg
+        self.gather = bool(gather)
         self.device = torch.device(device)
         self.sizes = api.moe_get_sizes(cfg)
         c, z = cfg, self.sizes
@@ -38,7 +42,8 @@ class MoELayer:
         self.offsets = e((E + 2,), i32)
         self.slot_row, self.row_slot = e((T * K,), i32), e((R,), i32)
         self.tile_expert, self.stats = e((int(z.tiles_max),), i32), e((4,), i32)
-        self.x_perm, self.a13 = e((R, D), act), e((R, 2 * F), act)
+        self.x_perm = None if self.gather else e((R, D), act)
+        self.a13 = e((R, 2 * F), act)
         self.h, self.o = e((R, F), act), e((R, D), act)
         self.y = e((T, D), act)
         self.losses = torch.zeros(2, dtype=f32, device=dev)
@@ -96,9 +101,14 @@ class MoELayer:
                 self._aux_stream = torch.cuda.Stream(self.device)
             self._aux_stream.wait_stream(main)
             self._aux(self._aux_stream)
-        api.moe_expert_ffn(c, self.x_perm, self.offsets, self.tile_expert, self.stats,
-                           w13, w_down, w13_s, w_down_s, self.a13, self.h, self.o,
-                           self.ws)
+        if self.gather:
+            api.moe_expert_ffn_gather(c, x, self.row_slot, self.offsets, self.tile_expert,
+                                      self.stats, w13, w_down, w13_s, w_down_s, self.a13,
+                                      self.h, self.o, self.ws)
+        else:
+            api.moe_expert_ffn(c, self.x_perm, self.offsets, self.tile_expert, self.stats,
+                               w13, w_down, w13_s, w_down_s, self.a13, self.h, self.o,
+                               self.ws)
         api.moe_combine(c, self.o, self.slot_row, self.topk_w, self.offsets, self.y)
         if aux:
             main.wait_stream(self._aux_stream)

@@ -21,7 +21,8 @@ import torch
 import workloads as W
 from oracle import moe_oracle as O
 from tests.helpers import LazyLayer, np64, rel_l2
-from tests.test_gpu_parity import check_dispatch, gpu_inputs, host, run_gpu
+from tests.test_gpu_parity import (assert_gather_identical, check_dispatch, gpu_inputs, host,
+                                   run_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -172,3 +173,16 @@ def test_sequence_wise_aux_full_size(n_seq):
         batch, _, _ = O.aux_loss(Dp.counts, R.p, cfg.aux_alpha, cfg.E)
         assert abs(ref - batch) <= 1e-12 * batch
     assert abs(float(layer.losses[0]) - ref) <= 1e-4 * ref
+
+
+@pytest.mark.parametrize("name", ["mm_b", "olmoe", "olmoe_ec"])
+def test_fused_gather_full_size(name):
+    """The fused-gather layer (tile::gather4 rows of x inside the gate/up GEMM
+    and its weight gradient) at full size is bit-identical to the permuted-
+    copy layer that test_parity_full_size and test_expert_choice_full_size
+    check against the oracle; padding rows load as zeros."""
+    cfg = W.CONFIGS[name]
+    ref, inp = run_gpu(cfg)
+    fused, _ = run_gpu(cfg, inp=inp, gather=True)
+    torch.cuda.synchronize()
+    assert_gather_identical(cfg, ref, fused)
