@@ -123,6 +123,9 @@ def gemm_flops(cfg, kept_total):
         "tc_wgrad_down": 2 * M * D * F,
         "tc_dgrad_gate_up": 2 * M * 2 * F * D,
         "tc_wgrad_gate_up": 2 * M * 2 * F * D,
+        # one slot per token: combine / unpermute-sum in the epilogue
+        "tc_down_combine": 2 * M * F * D,
+        "tc_dgrad_gate_up_dx": 2 * M * 2 * F * D,
     }
 
 
@@ -141,6 +144,11 @@ def gemm_bytes(cfg, kept_total):
         "tc_dgrad_gate_up": M * 2 * F * a + w13 + M * D * a,
         "tc_wgrad_down": M * D * a + M * F * a + wd,
         "tc_wgrad_gate_up": M * 2 * F * a + M * D * a + w13,
+        # + y rows and gate weights / dx rows written in token order from the
+        # fp32 accumulator, ds and W_r read (no dX_perm round trip)
+        "tc_down_combine": M * F * a + wd + M * D * a + cfg.T * D * a + cfg.T * 4,
+        "tc_dgrad_gate_up_dx": (M * 2 * F * a + w13 + cfg.T * D * a + cfg.T * cfg.E * 4
+                                + cfg.E * D * 4),
     }
 
 

@@ -315,6 +315,31 @@ int moe_expert_ffn_gather(const moe_config_t* cfg, const void* x,
                           void* a13, void* h, void* o, void* ws, cudaStream_t stream);
 
 /*
+ * moe_expert_ffn_combine — moe_expert_ffn (x_perm != NULL) or
+ * moe_expert_ffn_gather (x_perm == NULL) followed by moe_combine, in one
+ * call.  With one slot per token (K = 1) and no shared expert on the
+ * tensor-core path, the combine y_t = g_t o[slot_row[t]] is a row scatter:
+ * the down-projection GEMM's epilogue writes y from its fp32 accumulator
+ * (scaled by g, rounded once) next to o, and tokens whose slot holds no
+ * row (sentinel, dropped) get y_t = 0 — no combine kernel runs.  Otherwise
+ * the separate combine runs.  [8MOE] Router / Gating Network; [STA324
+ * §8.7, §8.8].
+ *   x, x_perm   as moe_expert_ffn_gather / moe_expert_ffn (x may be NULL
+ *               when x_perm is given)
+ *   slot_row, row_slot, topk_w, offsets, tile_expert, stats: moe_router /
+ *               moe_dispatch outputs
+ *   a13, h, o   as moe_expert_ffn;  y [T,D] act out, as moe_combine
+ */
+int moe_expert_ffn_combine(const moe_config_t* cfg, const void* x, const void* x_perm,
+                           const int32_t* offsets, const int32_t* slot_row,
+                           const int32_t* row_slot, const float* topk_w,
+                           const int32_t* tile_expert, const int32_t* stats,
+                           const void* w13, const void* w_down,
+                           const void* w13_s, const void* w_down_s,
+                           void* a13, void* h, void* o, void* y, void* ws,
+                           cudaStream_t stream);
+
+/*
  * moe_combine — y_t = sum_{k kept} g_{t,k} o[slot_row[t*K+k]] (k ascending,
  * fp32 accumulation) + o[offsets[E] + t] when n_shared.  Deterministic
  * gather, no atomics.  [8MOE] Router / Gating Network (y = sum G(x)_i
@@ -340,6 +365,10 @@ int moe_combine(const moe_config_t* cfg, const void* o,
  * The gate gradient of a sentinel or dropped slot is zero (its expert
  * output is treated as zero), so such slots send no gradient to the router
  * through the gate path.  Deterministic: no floating-point atomics.
+ * With one slot per token (K = 1), no shared expert and E < 8 on the
+ * tensor-core path, dx is written by the dgrad gate/up GEMM's epilogue
+ * (dX_perm row + ds_t . W_r, rounded once; tokens without a row get the
+ * router part alone) instead of a separate unpermute-sum.
  * x_perm may be NULL on the tensor-core path (bf16 layers): the gate/up
  * weight-gradient GEMM then gathers its x rows by row_slot with tile::gather4
  * copies, as moe_expert_ffn_gather does (MOE_ERR_ARG for NULL x_perm on the

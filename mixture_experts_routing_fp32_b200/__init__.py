@@ -9,11 +9,13 @@ from .api import (MoEError, MoeConfig, MoeSizes, config_from, make_config,
                   moe_aux_loss, moe_backward, moe_check_status, moe_combine,
                   moe_dispatch, moe_expert_ffn, moe_get_sizes, moe_launch_count,
                   moe_router, moe_set_side_streams, moe_aux_loss_seq, moe_bias_update,
-                  moe_route_expert_choice, moe_expert_ffn_gather)
+                  moe_route_expert_choice, moe_expert_ffn_gather,
+                  moe_expert_ffn_combine)
 from .layer import MoELayer
 
 __all__ = ["MoEError", "MoeConfig", "MoeSizes", "config_from", "make_config",
            "moe_aux_loss", "moe_backward", "moe_check_status", "moe_combine",
            "moe_dispatch", "moe_expert_ffn", "moe_get_sizes", "moe_launch_count",
            "moe_router", "moe_set_side_streams", "moe_aux_loss_seq", "moe_bias_update",
-           "moe_route_expert_choice", "moe_expert_ffn_gather", "MoELayer"]
+           "moe_route_expert_choice", "moe_expert_ffn_gather",
+           "moe_expert_ffn_combine", "MoELayer"]

@@ -28,7 +28,8 @@ EXPORTS = ("moe_get_sizes", "moe_router", "moe_dispatch", "moe_aux_loss",
            "moe_profile_enable", "moe_profile_reset", "moe_profile_read", "moe_profile_starts",
            "moe_profile_name", "moe_profile_side", "moe_profile_disable",
            "moe_dispatch_static", "moe_set_side_streams", "moe_aux_loss_seq",
-           "moe_bias_update", "moe_route_expert_choice", "moe_expert_ffn_gather")
+           "moe_bias_update", "moe_route_expert_choice", "moe_expert_ffn_gather",
+           "moe_expert_ffn_combine")
 
 
 class MoeConfig(ctypes.Structure):
@@ -74,6 +75,7 @@ def lib():
         "moe_aux_loss": [cfg, P, P, P, P, P, P],
         "moe_expert_ffn": [cfg, P, P, P, P, P, P, P, P, P, P, P, P, P],
         "moe_expert_ffn_gather": [cfg] + [P] * 14,
+        "moe_expert_ffn_combine": [cfg] + [P] * 18,
         "moe_combine": [cfg, P, P, P, P, P, P],
         "moe_backward": [cfg] + [P] * 33,
         "moe_check_status": [P, ctypes.POINTER(ctypes.c_uint32)],

@@ -123,6 +123,14 @@ def moe_expert_ffn_gather(cfg, x, row_slot, offsets, tile_expert, stats, w13, w_
                                       _p(ws), _s(stream)), "moe_expert_ffn_gather")
 
 
+def moe_expert_ffn_combine(cfg, x, x_perm, offsets, slot_row, row_slot, topk_w, tile_expert,
+                           stats, w13, w_down, w13_s, w_down_s, a13, h, o, y, ws, stream=None):
+    check(lib().moe_expert_ffn_combine(
+        ctypes.byref(cfg), _p(x), _p(x_perm), _p(offsets), _p(slot_row), _p(row_slot),
+        _p(topk_w), _p(tile_expert), _p(stats), _p(w13), _p(w_down), _p(w13_s), _p(w_down_s),
+        _p(a13), _p(h), _p(o), _p(y), _p(ws), _s(stream)), "moe_expert_ffn_combine")
+
+
 def moe_combine(cfg, o, slot_row, topk_w, offsets, y, stream=None):
     check(lib().moe_combine(ctypes.byref(cfg), _p(o), _p(slot_row), _p(topk_w),
                             _p(offsets), _p(y), _s(stream)), "moe_combine")
@@ -198,4 +206,5 @@ __all__ = ["LaunchProfile", "MoEError", "MoeConfig", "MoeSizes", "make_config", 
            "moe_aux_loss",
            "moe_expert_ffn", "moe_combine", "moe_backward", "moe_check_status",
            "moe_launch_count", "moe_set_side_streams", "moe_aux_loss_seq",
-           "moe_bias_update", "moe_route_expert_choice", "moe_expert_ffn_gather"]
+           "moe_bias_update", "moe_route_expert_choice", "moe_expert_ffn_gather",
+           "moe_expert_ffn_combine"]

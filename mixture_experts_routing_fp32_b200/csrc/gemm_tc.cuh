@@ -49,7 +49,11 @@ enum {
   EPI_SWIGLU_BWD = 2,  // da13 from dh = C and the saved a13
   EPI_WGRAD = 3,       // bf16 weight gradient per group
   EPI_F32 = 4,         // fp32 C, rows < dense_m (dense ROWS)
-  EPI_WGRAD_F32 = 5    // fp32 C, rows < m_limit (dense WGRAD)
+  EPI_WGRAD_F32 = 5,   // fp32 C, rows < m_limit (dense WGRAD)
+  // one slot per token (K = 1, no shared expert): the row of token t is
+  // row_slot^-1(t), so combine and unpermute-sum are row scatters
+  EPI_COMBINE1 = 6,    // bf16 C (o) and y[token(r)] = g_token * C
+  EPI_DX1 = 7          // dx[token(r)] = C + ds_token . W_r (no row output)
 };
 
 struct Params {
@@ -80,6 +84,14 @@ struct Params {
   const int32_t* row_slot;
   int gK;                      // slots per token
   int shared_T;                // rows of the shared group (0: none)
+  // token-order epilogues (COMBINE1, DX1): token of row r = row_slot[r];
+  // tokens whose slot has no row (slot_row < 0) are written at kernel start
+  const int32_t* slot_row;
+  const float* tw;             // COMBINE1: gate weight per token
+  __nv_bfloat16* tout;         // y or dx [T, ld_out]
+  const float* ds;             // DX1: router logit gradient [T, Er]
+  const float* w_r;            // DX1: router weight [Er, ld_out]
+  int Er;                      // DX1: router experts (<= 8)
 };
 
 // ----------------------------------------------------------------------------
@@ -414,6 +426,29 @@ __device__ __forceinline__ void staged_store32(uint32_t stg, const float (&v)[32
     if (r < nrows)
       asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(
                        w0 + r * ld + pc * 8),
+                   "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w), "l"(pol)
+                   : "memory");
+  }
+  __syncwarp();
+}
+
+// staged_store32 to scattered rows: block row i goes to w0 + tok_i * ld,
+// where tok_i is lane i's `tok` (rows with tok < 0 are skipped).
+__device__ __forceinline__ void staged_store32_tok(uint32_t stg, const float (&v)[32],
+                                                   __nv_bfloat16* w0, int64_t ld, int tok,
+                                                   uint64_t pol) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) sts128(stg + lane * kStgRow + j * 16, pack8_bf16(v + 8 * j));
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i * 8 + (lane >> 2), pc = lane & 3;
+    const int tr = __shfl_sync(0xffffffffu, tok, r);
+    const uint4 u = lds128(stg + r * kStgRow + pc * 16);
+    if (tr >= 0)
+      asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(
+                       w0 + (int64_t)tr * ld + pc * 8),
                    "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w), "l"(pol)
                    : "memory");
   }
@@ -901,6 +936,40 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     constexpr int HJ = BN / 4;           // gate (= up) columns per warp (SwiGLU)
     const uint64_t pol_out = policy_evict_first();
     const uint32_t stg = base + S::kEpiOff + (warp - 2) * kStgBytes;   // staging tile
+    if constexpr (EPI == EPI_COMBINE1 || EPI == EPI_DX1) {
+      // tokens whose slot holds no row (sentinel, dropped): y_t = 0, or
+      // dx_t = ds_t . W_r (the router part alone), while the first tile's
+      // main loop runs.  Each lane checks one token (one load per lane for
+      // a whole grid's worth of tokens); the warp writes the masked ones.
+      const int stride = gridDim.x * kEpiWarps * 32;
+      for (int t0 = (blockIdx.x * kEpiWarps + (warp - 2)) * 32; t0 < p.T; t0 += stride) {
+        const bool masked = t0 + lane < p.T && p.slot_row[t0 + lane] < 0;
+        unsigned todo = __ballot_sync(0xffffffffu, masked);
+        while (todo != 0u) {
+          const int t = t0 + __ffs(todo) - 1;
+          todo &= todo - 1u;
+          __nv_bfloat16* dst = p.tout + (int64_t)t * p.ld_out;
+          float dse[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dse[e] = (EPI == EPI_DX1 && e < p.Er) ? p.ds[(int64_t)t * p.Er + e] : 0.f;
+          for (int c = lane * 8; c < p.ld_out; c += 256) {
+            float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if constexpr (EPI == EPI_DX1) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                if (e < p.Er) {
+                  float w[8];
+                  load8(p.w_r + (int64_t)e * p.ld_out + c, w);
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) a[i] = fmaf(dse[e], w[i], a[i]);
+                }
+              }
+            }
+            store8(dst + c, a);
+          }
+        }
+      }
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
     Tile nxt = decode_at(unit);
@@ -923,6 +992,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
         for (int c = 0; c < HC / 32; ++c) {
           block_load32(a13 + 32 * c, p.ld_aux, pa[c]);
           block_load32(a13 + p.F + 32 * c, p.ld_aux, pb[c]);
+        }
+      }
+      // token-order epilogues: this lane's row -> token, gate weight or ds
+      int my_tok = -1;
+      float my_g = 0.f, dse[EPI == EPI_DX1 ? 8 : 1];
+      if constexpr (EPI == EPI_COMBINE1 || EPI == EPI_DX1) {
+        my_tok = p.row_slot[row0 + lane];
+        if constexpr (EPI == EPI_COMBINE1) {
+          if (my_tok >= 0) my_g = p.tw[my_tok];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dse[e] = (my_tok >= 0 && e < p.Er) ? p.ds[(int64_t)my_tok * p.Er + e] : 0.f;
         }
       }
       bool ok = (lane == 0) ? mbar_wait(accf_bar(acc), acc_phase, abort_flag) : true;
@@ -949,6 +1031,38 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_wait();
           u2f32(r, v);
           staged_store32(stg, v, w0 + c, ld, pol_out);
+        }
+      } else if constexpr (EPI == EPI_COMBINE1 || EPI == EPI_DX1) {
+        const int col0 = d.n0 + hh * HC;
+        __nv_bfloat16* w0 = p.out + row0 * p.ld_out + col0;
+#pragma unroll
+        for (int c = 0; c < HC; c += 32) {
+          uint32_t r[32];
+          float v[32];
+          tmem_ld32(tbase + hh * HC + c, r);
+          tmem_wait();
+          u2f32(r, v);
+          if constexpr (EPI == EPI_COMBINE1) {
+            staged_store32(stg, v, w0 + c, p.ld_out, pol_out);   // o, row order
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= my_g;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              if (e < p.Er) {
+                const float* wr = p.w_r + (int64_t)e * p.ld_out + col0 + c;
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                  const float4 w = *reinterpret_cast<const float4*>(wr + 4 * q4);
+                  v[4 * q4] = fmaf(dse[e], w.x, v[4 * q4]);
+                  v[4 * q4 + 1] = fmaf(dse[e], w.y, v[4 * q4 + 1]);
+                  v[4 * q4 + 2] = fmaf(dse[e], w.z, v[4 * q4 + 2]);
+                  v[4 * q4 + 3] = fmaf(dse[e], w.w, v[4 * q4 + 3]);
+                }
+              }
+            }
+          }
+          staged_store32_tok(stg, v, p.tout + col0 + c, p.ld_out, my_tok, pol_out);
         }
       } else if constexpr (EPI == EPI_SWIGLU) {
         __nv_bfloat16* a13 = p.out + row0 * p.ld_out + d.n0 + hh * HJ;

@@ -515,6 +515,8 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
       MOE_LAUNCHED(s, "router_fused");
       return MOE_OK;
     };
+    if (c->K == 1 && c->E <= 4) return go(router_fused_kernel<TX, 4, 1>);
+    if (c->K == 1 && c->E <= 8) return go(router_fused_kernel<TX, 8, 1>);
     if (c->E <= 4) return go(router_fused_kernel<TX, 4>);
     if (c->E <= 8) return go(router_fused_kernel<TX, 8>);
     if (c->E <= 16) return go(router_fused_kernel<TX, 16>);
@@ -1020,10 +1022,14 @@ namespace {
 // gate/up + SwiGLU and down on the tensor cores.  The gate/up A rows are
 // read from x_perm, or, with x_perm == nullptr, gathered from the token rows
 // of x by the GEMM itself (row_slot, offsets[E] for the shared group).
+// With y != nullptr (one slot per token, no shared expert) the down GEMM
+// also writes the combined output y[t] = g_t o[row(t)] from its epilogue.
 int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, const void* x,
                   const int32_t* row_slot, const int32_t* offsets, const int32_t* tile_expert,
                   const int32_t* stats, const void* w13, const void* w_down, const void* w13_s,
-                  const void* w_down_s, void* a13, void* h, void* o, cudaStream_t s) {
+                  const void* w_down_s, void* a13, void* h, void* o, cudaStream_t s,
+                  const int32_t* slot_row = nullptr, const float* topk_w = nullptr,
+                  void* y = nullptr) {
   const int D = c->D, F = c->F, E = c->E;
   const bool gather = x_perm == nullptr;
   CUtensorMap mA, mB, mBs;
@@ -1061,11 +1067,29 @@ int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, co
   MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, box2, true));
   tc::Params q = rows_params(c, F, D / bn2, tile_expert, stats, pr);
   q.out = static_cast<__nv_bfloat16*>(o); q.ld_out = D;
+  if (y != nullptr) {
+    q.row_slot = row_slot; q.slot_row = slot_row; q.tw = topk_w;
+    q.tout = static_cast<__nv_bfloat16*>(y);
+    const char* n2 = "tc_down_combine";
+    if (pr)
+      return run_tc<tc::MODE_ROWS, false, false, tc::EPI_COMBINE1, true>(
+          bn2, n2, mA, mB, mBs, q, units * q.nN, 0, s);
+    return run_tc<tc::MODE_ROWS, false, false, tc::EPI_COMBINE1>(
+        bn2, n2, mA, mB, mBs, q, units * q.nN, 0, s);
+  }
   if (pr)
     return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE, true>(
         bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
   return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE>(
       bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
+}
+
+// One slot per token and no shared expert: the combine and the
+// unpermute-sum are row scatters, done in the down / dgrad gate-up GEMM
+// epilogues (bf16 tensor-core layers; dx only with the CUDA-core router
+// term, E < 8).
+bool token_epilogues(const moe_config_t* c) {
+  return use_tc(c) && c->K == 1 && c->n_shared == 0 && !c->expert_choice;
 }
 }  // namespace
 
@@ -1115,6 +1139,31 @@ int moe_expert_ffn_gather(const moe_config_t* c, const void* x, const int32_t* r
   const Layout L = layout_of(c);
   return expert_ffn_tc(c, L, nullptr, x, row_slot, offsets, tile_expert, stats, w13, w_down,
                        w13_s, w_down_s, a13, h, o, s);
+}
+
+int moe_expert_ffn_combine(const moe_config_t* c, const void* x, const void* x_perm,
+                           const int32_t* offsets, const int32_t* slot_row,
+                           const int32_t* row_slot, const float* topk_w,
+                           const int32_t* tile_expert, const int32_t* stats, const void* w13,
+                           const void* w_down, const void* w13_s, const void* w_down_s,
+                           void* a13, void* h, void* o, void* y, void* ws, cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!offsets || !slot_row || !row_slot || !topk_w || !tile_expert || !stats || !w13 ||
+      !w_down || !a13 || !h || !o || !y)
+    return MOE_ERR_ARG;
+  if (!x_perm && (!x || !use_tc(c))) return MOE_ERR_ARG;
+  if (c->n_shared && (!w13_s || !w_down_s)) return MOE_ERR_ARG;
+  const Layout L = layout_of(c);
+  if (token_epilogues(c))
+    return expert_ffn_tc(c, L, x_perm, x, row_slot, offsets, tile_expert, stats, w13, w_down,
+                         w13_s, w_down_s, a13, h, o, s, slot_row, topk_w, y);
+  if (x_perm)
+    MOE_TRY(moe_expert_ffn(c, x_perm, offsets, tile_expert, stats, w13, w_down, w13_s, w_down_s,
+                           a13, h, o, ws, s));
+  else
+    MOE_TRY(moe_expert_ffn_gather(c, x, row_slot, offsets, tile_expert, stats, w13, w_down,
+                                  w13_s, w_down_s, a13, h, o, ws, s));
+  return moe_combine(c, o, slot_row, topk_w, offsets, y, s);
 }
 
 int moe_combine(const moe_config_t* c, const void* o, const int32_t* slot_row,
@@ -1189,6 +1238,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   void* dH = wsp<void>(ws, L.off_dH);
   const bool bf = c->dtype == MOE_BF16;
   const bool rtc = router_tc(c);
+  const bool dx1 = token_epilogues(c) && !rtc;   // dx from the dgrad gate/up epilogue
 
   // 1. per row: gate gradient dg = <o, dy>, and dO = g * dy
   {
@@ -1315,7 +1365,9 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
             bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1)));
     }
-    // 5. dgrad gate/up: dX_perm = dA13 . w13[e]
+    // 5. dgrad gate/up: dX_perm = dA13 . w13[e]; with one slot per token
+    // (no shared expert, CUDA-core router term) the epilogue writes dx
+    // itself: dx[t] = dX_perm[row(t)] + ds_t . W_r, once ds is ready
     const int bn5 = pick_bn(D, mt, false, F, pr);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 128, false));
     MOE_TRY(make_map(&mB, w13, E, 2 * F, D, 64, true));                  // dims {D, 2F, E}
@@ -1323,7 +1375,17 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     {
       tc::Params p = rows_params(c, 2 * F, D / bn5, tile_expert, stats, pr);
       p.out = static_cast<__nv_bfloat16*>(dXp); p.ld_out = D;
-      if (pr)
+      if (dx1) {
+        MOE_CK(cudaStreamWaitEvent(s, sd->ev[6], 0));
+        p.row_slot = row_slot; p.slot_row = slot_row; p.tout = static_cast<__nv_bfloat16*>(dx);
+        p.ds = ds; p.w_r = w_r; p.Er = E;
+        if (pr)
+          MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_DX1, true>(
+              bn5, "tc_dgrad_gate_up_dx", mA, mB, mBs, p, units * p.nN, 0, s)));
+        else
+          MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_DX1>(
+              bn5, "tc_dgrad_gate_up_dx", mA, mB, mBs, p, units * p.nN, 0, s)));
+      } else if (pr)
         MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE, true>(
             bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s)));
       else
@@ -1430,7 +1492,8 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
         dwr_part, nc, n, dw_r)));
     MOE_LAUNCHED(s, "router_dw_reduce");
   }
-  // 8. dx = unpermute-sum(dX_perm) + shared + ds . w_r, once ds is ready;
+  // 8. dx = unpermute-sum(dX_perm) + shared + ds . w_r, once ds is ready
+  // (already written by the dgrad gate/up epilogue when dx1);
   // on tensor cores the router part R = (ds_hi | ds_hi | ds_mid) .
   // (W_hi; W_mid; W_hi) is written in fp32 and a gather kernel adds the
   // dX_perm rows
@@ -1453,7 +1516,9 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_F32>(
         bn, "router_dx_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
   }
-  if (c->expert_choice) {
+  if (dx1) {
+    // done
+  } else if (c->expert_choice) {
     prof_begin(s);
     if (bf)
       MOE_CK((launch_k(ec_dx_kernel<__nv_bfloat16>, grid_for(T), 256, 0, s, Rdx, ds, w_r,

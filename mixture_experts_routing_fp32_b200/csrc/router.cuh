@@ -49,7 +49,8 @@ __device__ __forceinline__ float pick(const float (&a)[NV], int i) {
 
 // Routes token t given its logits s[i] (expert lane + 32 i).  `gsm` is
 // per-warp shared scratch of at least E floats (group-limited routing).
-template <int NV>
+// KM: compile-time bound on K (the selection arrays are sized by it).
+template <int NV, int KM = kMaxK>
 __device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
                             float* gsm, int lane) {
   const int E = a.E;
@@ -128,12 +129,12 @@ __device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
 
   // top-K (+1 round): the near-tie margin is the smallest gap between
   // consecutive selection scores among the top K+1
-  int sel_e[kMaxK];
-  float sel_s[kMaxK], sel_p[kMaxK];
+  int sel_e[KM];
+  float sel_s[KM], sel_p[KM];
   unsigned taken = 0u;
   float uk = NEG, margin = INFINITY;
 #pragma unroll
-  for (int k = 0; k <= kMaxK; ++k) {
+  for (int k = 0; k <= KM; ++k) {
     if (k > a.K) break;
     float v = NEG;
     int e = 0x7fffffff;
@@ -150,7 +151,7 @@ __device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
       const float sv = __shfl_sync(0xffffffffu, pick<NV>(s, slot), owner);
       const float pv = __shfl_sync(0xffffffffu, pick<NV>(p, slot), owner);
       if (lane == owner) taken |= 1u << slot;
-      if (k < kMaxK) { sel_e[k] = e; sel_s[k] = sv; sel_p[k] = pv; }
+      if (k < KM) { sel_e[k] = e; sel_s[k] = sv; sel_p[k] = pv; }
       uk = v;
     }
   }
@@ -158,10 +159,10 @@ __device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
     atomicAdd(a.near_ties, 1);
 
   // gate weights
-  float g[kMaxK];
+  float g[KM];
   float denom = 0.f;
 #pragma unroll
-  for (int k = 0; k < kMaxK; ++k) {
+  for (int k = 0; k < KM; ++k) {
     if (k >= a.K) break;
     if (a.score_fn == MOE_SOFTMAX) {
       g[k] = a.renorm ? expf(sel_s[k] - sel_s[0]) : sel_p[k];
@@ -172,7 +173,7 @@ __device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
   }
   if (a.renorm) denom = (a.score_fn == MOE_SOFTMAX) ? denom : denom + 1e-20f;
 #pragma unroll
-  for (int k = 0; k < kMaxK; ++k) {
+  for (int k = 0; k < KM; ++k) {
     if (k >= a.K) break;
     float w = a.renorm ? g[k] / denom : g[k];
     w *= a.route_scale;
@@ -188,7 +189,7 @@ __device__ void route_token(int t, float (&s)[NV], const RouteArgs& a,
 // over tokens.  W_r rows are read through the read-only cache (after the
 // first touch they are L1 hits), so the x row loads start at once.
 // ---------------------------------------------------------------------------
-template <typename TX, int EB>
+template <typename TX, int EB, int KM = kMaxK>
 __global__ void __launch_bounds__(256)
 router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
                     const float* __restrict__ offset, int D, RouteArgs a) {
@@ -202,6 +203,9 @@ router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
     float acc[EB];
 #pragma unroll
     for (int e = 0; e < EB; ++e) acc[e] = 0.f;
+    // one-slot routing keeps few registers: unroll so that the x and W_r
+    // loads of several 256-column steps are in flight together
+#pragma unroll (KM == 1 ? 4 : 1)
     for (int d = lane * 8; d < D; d += 256) {
       float xv[8];
       load8(xr + d, xv);
@@ -228,7 +232,7 @@ router_fused_kernel(const TX* __restrict__ x, const float* __restrict__ w_r,
       if (offset != nullptr) s[0] += offset[lane];
       a.logits[(size_t)t * E + lane] = s[0];
     }
-    route_token<1>(t, s, a, gsm, lane);
+    route_token<1, KM>(t, s, a, gsm, lane);
   }
 }
 

@@ -4,11 +4,11 @@ The layer owns every device buffer the C ABI needs (allocated once with
 torch, stable pointers, so a whole step can be captured in a CUDA graph)
 and issues the entry points in order on the current stream:
 
-  forward : moe_router -> moe_dispatch -> moe_expert_ffn -> moe_combine,
-            with moe_aux_loss on a side stream (joined before returning);
-            gather=True: moe_dispatch computes the layout only and
-            moe_expert_ffn_gather reads the token rows of x inside the
-            gate/up GEMM (no permuted copy of x; bf16 layers)
+  forward : moe_router -> moe_dispatch -> moe_expert_ffn_combine (expert
+            FFN + combine), with moe_aux_loss on a side stream (joined
+            before returning); gather=True: moe_dispatch computes the
+            layout only and the gate/up GEMM reads the token rows of x
+            itself (no permuted copy of x; bf16 layers)
   backward: moe_backward
 
 No host synchronisation happens inside forward or backward.
@@ -101,15 +101,12 @@ class MoELayer:
                 self._aux_stream = torch.cuda.Stream(self.device)
             self._aux_stream.wait_stream(main)
             self._aux(self._aux_stream)
-        if self.gather:
-            api.moe_expert_ffn_gather(c, x, self.row_slot, self.offsets, self.tile_expert,
-                                      self.stats, w13, w_down, w13_s, w_down_s, self.a13,
-                                      self.h, self.o, self.ws)
-        else:
-            api.moe_expert_ffn(c, self.x_perm, self.offsets, self.tile_expert, self.stats,
-                               w13, w_down, w13_s, w_down_s, self.a13, self.h, self.o,
-                               self.ws)
-        api.moe_combine(c, self.o, self.slot_row, self.topk_w, self.offsets, self.y)
+        # expert FFN + combine (one slot per token: the combine is done by
+        # the down projection's epilogue)
+        api.moe_expert_ffn_combine(c, x, self.x_perm, self.offsets, self.slot_row,
+                                   self.row_slot, self.topk_w, self.tile_expert, self.stats,
+                                   w13, w_down, w13_s, w_down_s, self.a13, self.h, self.o,
+                                   self.y, self.ws)
         if aux:
             main.wait_stream(self._aux_stream)
         self._inputs = (x, w_r, w13, w_down, w13_s, w_down_s)

@@ -111,6 +111,10 @@ REDUCED = {
     # enough rows per expert (>= 1536) that the expert GEMMs run on CTA pairs
     "mm_pair": CONFIGS["mm_b"].replace(name="mm_pair_small", T=6500, D=256, F=512),
     "mix_pair": CONFIGS["mix"].replace(name="mix_pair_small", T=7000, D=512, F=640),
+    # one slot per token with capacity drops and sentinel slots: the tokens
+    # without a row in the token-order (combine / dx) epilogues
+    "mm_mask": CONFIGS["mm_a"].replace(name="mm_mask_small", T=1000, D=256, F=512,
+                                       capacity_factor=0.9, sentinel_frac=0.05),
     # more than 16384 slots: the multi-block dispatch passes (ragged last block)
     "olmoe_multi": CONFIGS["olmoe"].replace(name="olmoe_multi_small", T=2600, D=128, F=128),
     # sequence-wise aux loss: softmax (OLMoE-shaped, 7 sequences) and sigmoid
