@@ -159,42 +159,108 @@ ec_select_kernel(const float* __restrict__ probs, int T, int E, int C,
   }
 }
 
+// A token's picked slots in increasing e, compacted into the warp's shared
+// list (rows, and gate weights when g != nullptr); returns their number.
+constexpr int kEcBatch = 8;   // picked rows whose loads are in flight together
+__device__ __forceinline__ int ec_picks(const int32_t* __restrict__ slot_row,
+                                       const float* __restrict__ g, int64_t t, int E,
+                                       int32_t* rows, float* gs) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  int n = 0;
+  __syncwarp();   // the previous token's list has been read
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    const int32_t r = e < E ? slot_row[t * E + e] : -1;
+    const unsigned bal = __ballot_sync(0xffffffffu, r >= 0);
+    if (r >= 0) {
+      const int pos = n + __popc(bal & lt);
+      rows[pos] = r;
+      if (g != nullptr) gs[pos] = g[t * E + e];
+    }
+    n += __popc(bal);
+  }
+  __syncwarp();
+  return n;
+}
+
+// 8 consecutive elements loaded raw (one or two 16-byte loads, no
+// conversion, so a batch of them is in flight at once) and widened later.
+template <typename TX> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+    u = *reinterpret_cast<const uint4*>(p);
+  }
+  __device__ __forceinline__ void widen(float* f) const { bf16x8_to_f32(u, f); }
+};
+template <> struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = *reinterpret_cast<const float4*>(p);
+    b = *reinterpret_cast<const float4*>(p + 4);
+  }
+  __device__ __forceinline__ void widen(float* f) const {
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+};
+
+// acc += sum over the n listed rows (in list order) of w_i * src[row_i, d..d+7]
+// (w_i = 1 when gs == nullptr).  The loads of kEcBatch rows are issued
+// unconditionally (a slot past the list reads the first listed row, or row
+// 0) before any is used, so they are in flight together.
+template <typename TX>
+__device__ __forceinline__ void ec_accumulate(const TX* __restrict__ src, int64_t D, int d,
+                                              bool act, int n, const int32_t* rows,
+                                              const float* gs, float (&acc)[8]) {
+  const int dd = act ? d : 0;
+  for (int i0 = 0; i0 < n; i0 += kEcBatch) {
+    Raw8<TX> raw[kEcBatch];
+#pragma unroll
+    for (int j = 0; j < kEcBatch; ++j) {
+      const int64_t r = i0 + j < n ? rows[i0 + j] : rows[0];
+      raw[j].load(src + r * D + dd);
+    }
+#pragma unroll
+    for (int j = 0; j < kEcBatch; ++j) {
+      if (i0 + j < n) {
+        float v[8];
+        raw[j].widen(v);
+        if (gs != nullptr) {
+          const float w = gs[i0 + j];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] = fmaf(w, v[k], acc[k]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] += v[k];
+        }
+      }
+    }
+  }
+}
+
 // y_t = sum over the experts that picked t (increasing e) of p[t,e] o[row]
-// (+ the shared row).  One warp per token: a ballot over 32 slots at a time
-// finds the picked ones; every lane then adds 8 columns of each row.
+// (+ the shared row).  One warp per token: its picked slots are compacted
+// into a shared list once, then every lane adds 8 columns of each listed
+// row, kEcBatch rows' loads at a time.
 template <typename TX>
 __global__ void __launch_bounds__(256)
 ec_combine_kernel(const TX* __restrict__ o, const int32_t* __restrict__ slot_row,
                   const float* __restrict__ topk_w, const int32_t* __restrict__ offsets,
                   int n_shared, int T, int D, int E, TX* __restrict__ y) {
   pdl_begin();
+  __shared__ int32_t rows_s[8][kMaxExperts];
+  __shared__ float g_s[8][kMaxExperts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t shared0 = n_shared ? (int64_t)offsets[E] : -1;
   for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < T; t += (int64_t)gridDim.x * 8) {
-    // the column loop is warp-uniform (the ballots and shuffles need every
-    // lane); lanes past D only skip the loads and the store
+    const int n = ec_picks(slot_row, topk_w, t, E, rows_s[warp], g_s[warp]);
     for (int d0 = 0; d0 < D; d0 += 256) {
       const int d = d0 + lane * 8;
       const bool act = d < D;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int e0 = 0; e0 < E; e0 += 32) {
-        const int e = e0 + lane;
-        const int32_t r = e < E ? slot_row[t * E + e] : -1;
-        const float g = e < E ? topk_w[t * E + e] : 0.f;
-        unsigned bal = __ballot_sync(0xffffffffu, r >= 0);
-        while (bal) {
-          const int src = __ffs(bal) - 1;
-          bal &= bal - 1;
-          const int64_t row = __shfl_sync(0xffffffffu, r, src);
-          const float gg = __shfl_sync(0xffffffffu, g, src);
-          if (act) {
-            float v[8];
-            load8(o + row * D + d, v);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = fmaf(gg, v[i], acc[i]);
-          }
-        }
-      }
+      ec_accumulate(o, D, d, act, n, rows_s[warp], g_s[warp], acc);
       if (act) {
         if (shared0 >= 0) {
           float v[8];
@@ -218,10 +284,12 @@ ec_dx_kernel(const float* __restrict__ R, const float* __restrict__ ds,
              const int32_t* __restrict__ slot_row, const int32_t* __restrict__ offsets,
              int n_shared, int T, int D, int E, TX* __restrict__ dx) {
   pdl_begin();
+  __shared__ int32_t rows_s[8][kMaxExperts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t shared0 = n_shared ? (int64_t)offsets[E] : -1;
   for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < T; t += (int64_t)gridDim.x * 8) {
-    for (int d0 = 0; d0 < D; d0 += 256) {     // warp-uniform, as in ec_combine_kernel
+    const int n = ec_picks(slot_row, nullptr, t, E, rows_s[warp], nullptr);
+    for (int d0 = 0; d0 < D; d0 += 256) {
       const int d = d0 + lane * 8;
       const bool act = d < D;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -238,22 +306,7 @@ ec_dx_kernel(const float* __restrict__ R, const float* __restrict__ ds,
           }
         }
       }
-      for (int e0 = 0; e0 < E; e0 += 32) {
-        const int e = e0 + lane;
-        const int32_t r = e < E ? slot_row[t * E + e] : -1;
-        unsigned bal = __ballot_sync(0xffffffffu, r >= 0);
-        while (bal) {
-          const int src = __ffs(bal) - 1;
-          bal &= bal - 1;
-          const int64_t row = __shfl_sync(0xffffffffu, r, src);
-          if (act) {
-            float v[8];
-            load8(dXp + row * D + d, v);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] += v[i];
-          }
-        }
-      }
+      ec_accumulate(dXp, D, d, act, n, rows_s[warp], nullptr, acc);
       if (act) {
         if (shared0 >= 0) {
           float v[8];
