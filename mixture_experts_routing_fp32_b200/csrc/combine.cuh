@@ -158,6 +158,10 @@ combine_bf16_kernel(const __nv_bfloat16* __restrict__ o, const int32_t* __restri
 // dO[r] = g * dy[t]; shared rows -> dO[r] = dy[t]; padding -> 0.  A row's
 // kind is decided by row_slot alone (the dispatch sets -1 on padding and
 // shared rows), so each warp's chain is one index load then the row work.
+// 256-column steps of a row whose loads are batched (rows of up to
+// 256 * kRowBatch elements need one round trip to memory).
+constexpr int kRowBatch = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(256)
 bwd_rows_kernel(const T* __restrict__ o, const T* __restrict__ dy,
@@ -181,17 +185,33 @@ bwd_rows_kernel(const T* __restrict__ o, const T* __restrict__ dy,
     }
     const float g = slot >= 0 ? topk_w[slot] : 1.0f;
     float dot = 0.f;
-    for (int d = lane * 8; d < D; d += 256) {
-      float dv[8], ov[8];
-      load8(dy + t * D + d, dv);
-      if (slot >= 0) {
-        load8(o + r * D + d, ov);
+    // kRowBatch 256-column steps per batch: every load of the batch is
+    // issued (unconditionally, clamped to the row) before any is used
+    for (int d0 = 0; d0 < D; d0 += 256 * kRowBatch) {
+      Raw8<T> rd[kRowBatch], ro[kRowBatch];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dot = fmaf(ov[i], dv[i], dot);
+      for (int j = 0; j < kRowBatch; ++j) {
+        const int d = d0 + 256 * j + lane * 8;
+        const int dc = d < D ? d : lane * 8;
+        rd[j].load(dy + t * D + dc);
+        ro[j].load(o + r * D + dc);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dv[i] *= g;
-      store8(dst + d, dv);
+      for (int j = 0; j < kRowBatch; ++j) {
+        const int d = d0 + 256 * j + lane * 8;
+        if (d < D) {
+          float dv[8], ov[8];
+          rd[j].widen(dv);
+          if (slot >= 0) {
+            ro[j].widen(ov);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dot = fmaf(ov[i], dv[i], dot);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dv[i] *= g;
+          store8(dst + d, dv);
+        }
+      }
     }
     if (slot >= 0) {
       dot = warp_sum(dot);

@@ -325,11 +325,20 @@ disp_gather_kernel(const TX* __restrict__ x, int D, int K, int E, int T,
     else if (r >= shared0 && r - shared0 < T) src = r - shared0;
     TX* dst = x_perm + r * D;
     if (src >= 0) {
+      // four 256-column steps' loads in flight before their stores
       const TX* s = x + src * D;
-      for (int d = lane * 8; d < D; d += 256) {
-        float v[8];
-        load8(s + d, v);
-        store8(dst + d, v);
+      for (int d0 = 0; d0 < D; d0 += 1024) {
+        Raw8<TX> v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int d = d0 + 256 * j + lane * 8;
+          v[j].load(s + (d < D ? d : lane * 8));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int d = d0 + 256 * j + lane * 8;
+          if (d < D) v[j].store(dst + d);
+        }
       }
     } else {
       for (int d = lane * 8; d < D; d += 256) zero8(dst + d);

@@ -184,28 +184,6 @@ __device__ __forceinline__ int ec_picks(const int32_t* __restrict__ slot_row,
   return n;
 }
 
-// 8 consecutive elements loaded raw (one or two 16-byte loads, no
-// conversion, so a batch of them is in flight at once) and widened later.
-template <typename TX> struct Raw8;
-template <> struct Raw8<__nv_bfloat16> {
-  uint4 u;
-  __device__ __forceinline__ void load(const __nv_bfloat16* p) {
-    u = *reinterpret_cast<const uint4*>(p);
-  }
-  __device__ __forceinline__ void widen(float* f) const { bf16x8_to_f32(u, f); }
-};
-template <> struct Raw8<float> {
-  float4 a, b;
-  __device__ __forceinline__ void load(const float* p) {
-    a = *reinterpret_cast<const float4*>(p);
-    b = *reinterpret_cast<const float4*>(p + 4);
-  }
-  __device__ __forceinline__ void widen(float* f) const {
-    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-  }
-};
-
 // acc += sum over the n listed rows (in list order) of w_i * src[row_i, d..d+7]
 // (w_i = 1 when gs == nullptr).  The loads of kEcBatch rows are issued
 // unconditionally (a slot past the list reads the first listed row, or row
