@@ -983,15 +983,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
         continue;
       }
       const int64_t row0 = d.m0 + q * 32;   // this warp's first row
-      // SwiGLU backward: this warp's a and b blocks are fetched (coalesced)
-      // before the accumulator wait so their latency overlaps the main loop.
-      uint4 pa[EPI == EPI_SWIGLU_BWD ? HC / 32 : 1][4], pb[EPI == EPI_SWIGLU_BWD ? HC / 32 : 1][4];
+      // SwiGLU backward: this warp's first a and b blocks are fetched
+      // (coalesced) before the accumulator wait so their latency overlaps
+      // the main loop; each later block is fetched kPf blocks ahead.
+      constexpr int kNch = HC / 32;
+      constexpr int kPf = kNch < 2 ? kNch : 2;
+      uint4 pa[EPI == EPI_SWIGLU_BWD ? kPf : 1][4], pb[EPI == EPI_SWIGLU_BWD ? kPf : 1][4];
+      const __nv_bfloat16* a13s = p.aux + row0 * p.ld_aux + d.n0 + hh * HC;
       if constexpr (EPI == EPI_SWIGLU_BWD) {
-        const __nv_bfloat16* a13 = p.aux + row0 * p.ld_aux + d.n0 + hh * HC;
 #pragma unroll
-        for (int c = 0; c < HC / 32; ++c) {
-          block_load32(a13 + 32 * c, p.ld_aux, pa[c]);
-          block_load32(a13 + p.F + 32 * c, p.ld_aux, pb[c]);
+        for (int c = 0; c < kPf; ++c) {
+          block_load32(a13s + 32 * c, p.ld_aux, pa[c]);
+          block_load32(a13s + p.F + 32 * c, p.ld_aux, pb[c]);
         }
       }
       // token-order epilogues: this lane's row -> token, gate weight or ds
@@ -1101,9 +1104,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
         for (int c = 0; c < HC; c += 32) {
           uint32_t r[32];
           float dh[32], av[32], bv[32];
+          const int ci = c / 32, slot = ci % kPf;
           tmem_ld32(tbase + hh * HC + c, r);
-          staged_rows32(stg, pa[c / 32], av);
-          staged_rows32(stg, pb[c / 32], bv);
+          staged_rows32(stg, pa[slot], av);
+          staged_rows32(stg, pb[slot], bv);
+          if (ci + kPf < kNch) {
+            block_load32(a13s + 32 * (ci + kPf), p.ld_aux, pa[slot]);
+            block_load32(a13s + p.F + 32 * (ci + kPf), p.ld_aux, pb[slot]);
+          }
           tmem_wait();
           u2f32(r, dh);
 #pragma unroll
