@@ -109,6 +109,30 @@ def test_null_pointers_rejected_before_any_launch(lib):
         C.check(C.MOE_ERR_ARG, "x")
 
 
+def test_fused_paths_rejected_where_unsupported(lib):
+    """The gathered expert FFN and a NULL x_perm in the backward exist only on
+    the tensor-core path: fp32 layers are refused on the host, before any
+    pointer is used (the dummy addresses below are never dereferenced)."""
+    cfg = api.make_config(64, 32, 4, 2, 64, dtype="fp32")
+    dummy = ctypes.c_void_p(256)
+    assert lib.moe_expert_ffn_gather(ctypes.byref(cfg), *([dummy] * 13), None) == C.MOE_ERR_ARG
+    args = [dummy] * 33
+    args[14] = None                      # x_perm
+    args[-1] = None                      # stream
+    assert lib.moe_backward(ctypes.byref(cfg), *args) == C.MOE_ERR_ARG
+    # fused FFN + combine: y is required; with x_perm NULL also x and the
+    # tensor-core path
+    bf = api.make_config(4096, 768, 4, 1, 2048)
+    a = [dummy] * 18
+    a[15] = None                         # y
+    a[17] = None                         # stream
+    assert lib.moe_expert_ffn_combine(ctypes.byref(bf), *a) == C.MOE_ERR_ARG
+    a = [dummy] * 18
+    a[1] = None                          # x_perm
+    a[17] = None
+    assert lib.moe_expert_ffn_combine(ctypes.byref(cfg), *a) == C.MOE_ERR_ARG
+
+
 def test_package_has_no_cpu_fallback():
     # the product path never imports the oracle
     pkg = os.path.join(ROOT, "mixture_experts_routing_fp32_b200")
