@@ -1,13 +1,15 @@
 """Benchmark of the token-choice MoE layer step (forward + backward) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config mm_b]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config mix]
                     [--impl reference]
 
 One step = the whole hot path over one batch: router, dispatch, aux/z loss,
 grouped SwiGLU experts, combine, and the full backward (gate-weight
 gradient, expert dgrad/wgrad, router gradient, dx).  The default workload
-is the MiniMind-shaped layer (T=4096, D=768, E=4, K=1, F=2048, bf16,
-variant B, aux alpha 5e-4).  Multi-GPU (torchrun): data-parallel replicas,
+is the largest of the five layer shapes, the Mixtral-shaped layer (T=32768,
+D=4096, E=8, K=2, F=14336, bf16, variant B, capacity factor 1.25 with +2.0
+on expert 0's logit, so the hot expert overflows and drops).  Multi-GPU
+(torchrun): data-parallel replicas,
 each rank runs its own batch (weak scaling, no data-path collective);
 timing is the max over ranks.
 
@@ -40,6 +42,8 @@ import workloads as W  # noqa: E402
 METRIC = "MoE layer fwd+bwd tokens/s at 1 B200; grouped-GEMM % bf16 peak; HBM GB/s"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
+SHAPE_NAMES = {"tiny": "tiny fp32", "mm": "MiniMind-shaped", "olmoe": "OLMoE-shaped",
+               "mix": "Mixtral-shaped", "ds3": "DeepSeek-V3-shaped"}
 
 
 def parse():
@@ -47,12 +51,12 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="mm_b", choices=sorted(W.CONFIGS))
+    ap.add_argument("--config", default="mix", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--gather", type=int, default=0, choices=[0, 1],
-                    help="1: the gate/up GEMMs read token rows of x by tile::gather4 "
-                         "(no permuted copy of x); 0: the dispatch writes x_perm")
+                    help="1: the gate/up GEMMs' producer warp copies token rows of x "
+                         "(cp.async; no permuted copy of x); 0: the dispatch writes x_perm")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="sequence-wise aux loss over groups of this many tokens")
     ap.add_argument("--aux-alpha", type=float, default=None)
@@ -503,6 +507,14 @@ def run_ours(args):
                 side.add(name)
     tot = {k: sum(v) / len(per_launch) for k, v in fam.items()}
     hbm, bf16, bf16_sus, peak_src = measured_peaks()
+    clocks = clk.summary()
+    # tensor peak: the sustained figure when the power cap engaged during the
+    # timed region (the GPU ran long enough to settle at its capped clock),
+    # else the burst figure (each launch is timed on its own at full clock)
+    capped = "sw_power_cap" in (clocks.get("reasons") or [])
+    tc_peak = bf16_sus if capped else bf16
+    tc_kind = ("sustained: sw_power_cap was active during the timed region" if capped else
+               "burst: no power cap during the timed region, each launch timed alone")
     flops = gemm_flops(base, kept_total)
     rows_used = int(layer.stats[2])
     hbm_b = hbm_bytes(base, kept_total, rows_used)
@@ -515,15 +527,14 @@ def run_ours(args):
     if dom in flops:
         # a fused GEMM is bound by the slower of its tensor work and its
         # DRAM traffic at the measured peaks; report against that bound
-        t_tensor = flops[dom] / (bf16_sus * 1e12)
+        t_tensor = flops[dom] / (tc_peak * 1e12)
         t_hbm = gbytes[dom] / (hbm * 1e9)
         if t_tensor >= t_hbm:
             achieved = flops[dom] / n_dom / (dom_ms * 1e-3) / 1e12
             roof = {"bound": "tensor", "achieved": round(achieved, 2),
-                    "peak": bf16_sus, "unit": "TFLOP/s",
-                    "frac": round(achieved / bf16_sus, 4),
-                    "peak_source": "%s bf16 dense, sustained (kernel timed inside a long step)"
-                                   % peak_src}
+                    "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": round(achieved / tc_peak, 4),
+                    "peak_source": "%s bf16 dense, %s" % (peak_src, tc_kind)}
         else:
             achieved = gbytes[dom] / n_dom / (dom_ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
@@ -554,7 +565,6 @@ def run_ours(args):
             hbm_table[k] = {"bytes": b, "ms": round(tot[k], 5), "GB/s": round(gbs, 1),
                             "frac_of_hbm": round(gbs / hbm, 4),
                             "side_stream": k in side}
-    clocks = clk.summary()
     cpu = cpu_baseline(base, args.cpu_sample_s) if (rank == 0 and world == 1 and not args.no_cpu) else None
     if rank == 0:
         line = {
@@ -562,7 +572,8 @@ def run_ours(args):
             "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_max, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if base.dtype == "bf16" else "f32",
-            "data": "synthetic (seeded counter-hash normals; shapes of the MiniMind-shaped layer)",
+            "data": "synthetic (seeded counter-hash normals, bf16-rounded; shapes of the %s "
+                    "layer)" % SHAPE_NAMES.get(base.name.split("_")[0], base.name),
             "config": {"workload": "%s: T=%d D=%d E=%d K=%d F=%d %s variant %s aux %.0e%s%s" % (
                 base.name, base.T, base.D, base.E, base.K, base.F, base.dtype,
                 "B" if base.renorm else "A", base.aux_alpha,
@@ -571,8 +582,8 @@ def run_ours(args):
                 "global_batch_tokens": base.T * world, "parallelism": "dp%d (replicas)" % world,
                 "l2": "flushed between timed steps (256 MiB write)",
                 "cuda_graph": graph is not None,
-                "row_gather": ("inside the gate/up GEMMs (tile::gather4 rows of x)"
-                               if args.gather else "dispatch kernel writes x_perm"),
+                "row_gather": ("inside the gate/up GEMMs (producer-warp cp.async copies of "
+                               "x rows)" if args.gather else "dispatch kernel writes x_perm"),
                 "programmatic_dependent_launch": os.environ.get("MOE_PDL", "1") != "0"},
             "e2e": {"value": round(base.T * world / (e2e * 1e-3), 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -587,19 +598,29 @@ def run_ours(args):
                 "per_kernel": {k: {"ms": round(tot[k], 5),
                                    "TFLOP/s": round(flops[k] / (tot[k] * 1e-3) / 1e12, 1),
                                    "frac_of_tensor": round(flops[k] / (tot[k] * 1e-3) / 1e12
-                                                           / bf16_sus, 3),
+                                                           / tc_peak, 3),
                                    "GB/s": round(gbytes[k] / (tot[k] * 1e-3) / 1e9, 1),
                                    "frac_of_hbm": round(gbytes[k] / (tot[k] * 1e-3) / 1e9 / hbm,
                                                         3)}
                                for k in gemm_names},
                 "tflops": round(gemm_tflops, 2) if gemm_tflops else None,
                 "frac_of_sustained": round(gemm_tflops / bf16_sus, 4) if gemm_tflops else None,
+                "frac_of_burst": round(gemm_tflops / bf16, 4) if gemm_tflops else None,
+                "frac_of_peak": round(gemm_tflops / tc_peak, 4) if gemm_tflops else None,
+                "peak": tc_peak, "peak_kind": tc_kind,
                 "ms_per_step": round(gemm_total_ms, 5), "kernels": gemm_names,
                 "timing": "sum of the expert GEMM launches timed one by one"},
             "kernels_ms_per_step": {k + (" [side stream]" if k in side else ""): round(v, 5)
                                     for k, v in sorted(tot.items(), key=lambda kv: -kv[1])},
             "hbm_kernels": hbm_table,
             "kept_rows": kept_total,
+            "routing": {"near_ties": int(layer.near_ties[0]), "n_drop": int(layer.stats[0]),
+                        "n_sentinel": int(layer.stats[1]),
+                        "capacity": int(layer.sizes.capacity),
+                        "expert_counts": [int(v) for v in layer.counts.cpu()],
+                        "note": "near_ties: tokens whose selection margin among the top K+1 "
+                                "fp32 scores is below 1e-5 (the GPU's count); n_drop: "
+                                "assignments beyond capacity"},
             "clocks": clocks,
             "cpu_baseline": cpu,
             "source_hash": source_hash(),
@@ -615,53 +636,87 @@ def run_ours(args):
 # ---------------------------------------------------------------------------
 # the CPU oracle (baseline / reference arm)
 # ---------------------------------------------------------------------------
+CPU_SAMPLE_FLOP = 0.3e12          # expert FLOPs of one oracle sample step (seconds)
+CPU_WEIGHT_BYTES = 16 << 30       # host bytes of the sample's expert weights
+
+
 def cpu_sample_tokens(cfg):
-    return min(cfg.T, 512)
+    """Tokens of one CPU-oracle sample: a power of two up to 512 whose expert
+    work (18*D*F FLOPs per kept slot, shared expert included) stays under
+    CPU_SAMPLE_FLOP, so one sample takes seconds on the host cores."""
+    per_tok = 18.0 * cfg.D * cfg.F * (cfg.K + cfg.n_shared)
+    T_s = 512
+    while T_s > 16 and T_s * per_tok > CPU_SAMPLE_FLOP:
+        T_s //= 2
+    return min(cfg.T, T_s)
 
 
-def oracle_step(cfg, T_s):
-    """One forward + backward of the oracle on the first T_s tokens."""
-    import numpy as np
-    from oracle import moe_oracle as O
-    sub = cfg.replace(T=T_s)
-    f = lambda t: t.double().numpy()
-    w13 = {}
-    wd = {}
+class OracleSample:
+    """The oracle's inputs for the first T_s tokens of cfg, built before any
+    clock starts.  Only the experts those tokens route to are materialised,
+    held as float32 (the bf16 weights exactly; the oracle widens what it is
+    given to float64 as its first step); if they would exceed
+    CPU_WEIGHT_BYTES the sample shrinks until they fit."""
 
-    def g13(e):
-        if e not in w13:
-            w13[e] = f(W.make_input(cfg, "w13", expert=e))
-        return w13[e]
+    def __init__(self, cfg, T_s):
+        import numpy as np
+        from oracle import moe_oracle as O
+        f32 = lambda t: t.float().numpy()
+        while True:
+            x = f32(W.make_input(cfg, "x", rows=np.arange(T_s)))
+            w_r = f32(W.make_input(cfg, "w_r"))
+            self.L = O.Layer(x=x, w_r=w_r, w13=self._w13, wd=self._wd)
+            if cfg.n_shared:
+                self.L.w13_s, self.L.wd_s = f32(W.make_input(cfg, "w13_s")), \
+                    f32(W.make_input(cfg, "w_down_s"))
+            if cfg.hot_expert_offset:
+                self.L.logit_offset = f32(W.make_input(cfg, "logit_offset"))
+            if cfg.sel_bias_range:
+                self.L.sel_bias = f32(W.make_input(cfg, "sel_bias"))
+            if cfg.expert_choice:
+                hit = range(cfg.E)
+            else:
+                sub = cfg.replace(T=T_s)
+                R = O.route_layer(self.L, O.opts_of(sub))
+                hit = sorted(set(int(e) for e in R.idx.reshape(-1)))
+            per_e = 3 * cfg.D * cfg.F * 4
+            if len(hit) * per_e <= CPU_WEIGHT_BYTES or T_s <= 8:
+                break
+            T_s //= 2
+        self.T_s, self.hit = T_s, list(hit)
+        self.w13 = {e: f32(W.make_input(cfg, "w13", expert=e)) for e in hit}
+        self.wd = {e: f32(W.make_input(cfg, "w_down", expert=e)) for e in hit}
+        self.dy = f32(W.make_input(cfg, "dy", rows=np.arange(T_s)))
+        self.cfg = cfg
 
-    def gd(e):
-        if e not in wd:
-            wd[e] = f(W.make_input(cfg, "w_down", expert=e))
-        return wd[e]
+    def _w13(self, e):
+        return self.w13[e]
 
-    L = O.Layer(x=f(W.make_input(cfg, "x", rows=np.arange(T_s))), w_r=f(W.make_input(cfg, "w_r")),
-                w13=g13, wd=gd)
-    if cfg.n_shared:
-        L.w13_s, L.wd_s = f(W.make_input(cfg, "w13_s")), f(W.make_input(cfg, "w_down_s"))
-    if cfg.hot_expert_offset:
-        L.logit_offset = f(W.make_input(cfg, "logit_offset"))
-    if cfg.sel_bias_range:
-        L.sel_bias = f(W.make_input(cfg, "sel_bias"))
-    dy = f(W.make_input(cfg, "dy", rows=np.arange(T_s)))
-    # weights are generated before the clock starts
-    for e in range(cfg.E):
-        g13(e), gd(e)
-    t0 = time.perf_counter()
-    if cfg.expert_choice:
-        # expert choice picks across the batch: the sample is its own batch
-        # (each expert picks ceil(c * T_s / E) of its tokens)
-        from oracle import expert_choice as X
-        Lc, o, fw = X.forward(L, cfg.capacity_factor, cfg.min_capacity, z_lambda=cfg.z_lambda)
-        O.backward(Lc, o, fw, dy)
-    else:
-        o = O.opts_of(sub)
-        fw = O.forward(L, o)
-        O.backward(L, o, fw, dy)
-    return time.perf_counter() - t0
+    def _wd(self, e):
+        return self.wd[e]
+
+    def describe(self):
+        return ("first %d of %d tokens, full forward+backward in the float64 numpy oracle "
+                "(%d of %d experts routed to, their weights materialised before timing)"
+                % (self.T_s, self.cfg.T, len(self.hit), self.cfg.E))
+
+    def step(self):
+        """One forward + backward of the oracle on the sample; seconds."""
+        from oracle import moe_oracle as O
+        cfg = self.cfg
+        t0 = time.perf_counter()
+        if cfg.expert_choice:
+            # expert choice picks across the batch: the sample is its own batch
+            # (each expert picks ceil(c * T_s / E) of its tokens)
+            from oracle import expert_choice as X
+            Lc, o, fw = X.forward(self.L, cfg.capacity_factor, cfg.min_capacity,
+                                  z_lambda=cfg.z_lambda)
+            O.backward(Lc, o, fw, self.dy)
+        else:
+            o = O.opts_of(cfg.replace(T=self.T_s))
+            fw = O.forward(self.L, o)
+            O.backward(self.L, o, fw, self.dy)
+        return time.perf_counter() - t0
 
 
 def cpu_threads():
@@ -676,17 +731,17 @@ def cpu_threads():
 
 
 def cpu_baseline(cfg, budget_s):
-    T_s = cpu_sample_tokens(cfg)
+    smp = OracleSample(cfg, cpu_sample_tokens(cfg))
     times = []
     t_end = time.perf_counter() + budget_s
     while True:
-        times.append(oracle_step(cfg, T_s))
+        times.append(smp.step())
         if time.perf_counter() > t_end or len(times) >= 20:
             break
     s = statistics.mean(times)
-    return {"value": round(T_s / s, 2), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": "first %d of %d tokens, full forward+backward in the float64 numpy "
-                      "oracle, mean of %d runs (%.2f s each)" % (T_s, cfg.T, len(times), s)}
+    return {"value": round(smp.T_s / s, 2), "unit": UNIT, "cores": cpu_threads(),
+            "kind": "oracle",
+            "sample": "%s, mean of %d runs (%.2f s each)" % (smp.describe(), len(times), s)}
 
 
 def run_reference(args):
@@ -694,20 +749,21 @@ def run_reference(args):
     if rank != 0:
         return
     cfg = W.CONFIGS[args.config]
-    T_s = cpu_sample_tokens(cfg)
+    smp = OracleSample(cfg, cpu_sample_tokens(cfg))
     for _ in range(args.warmup):
-        oracle_step(cfg, T_s)
-    times = [oracle_step(cfg, T_s) for _ in range(args.steps)]
+        smp.step()
+    times = [smp.step() for _ in range(args.steps)]
     s = statistics.mean(times)
-    v = round(T_s / s, 2)
+    v = round(smp.T_s / s, 2)
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "%s (oracle on the first %d tokens per step)" % (cfg.name, T_s)},
+        "config": {"workload": "%s (oracle on the first %d tokens per step)" % (cfg.name,
+                                                                                 smp.T_s)},
         "cpu_baseline": {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                         "sample": "first %d of %d tokens per step" % (T_s, cfg.T)},
+                         "sample": smp.describe() + " per step"},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 

@@ -105,6 +105,12 @@ enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SIMT = 1 };   /* cfg.gemm_impl */
  *   gemm_impl  MOE_GEMM_AUTO: tcgen05 tensor cores for bf16 when D and F
  *              are multiples of 128, CUDA-core SIMT otherwise (fp32 always);
  *              MOE_GEMM_SIMT: force the SIMT kernels (cross-checks).
+ *   loss_tokens  0, or the global token count N >= T when the batch aux
+ *              loss and the z-loss are scoped over all data-parallel ranks
+ *              ([STA324 §8.5]: the balance statistic may be taken over the
+ *              whole batch or all devices): the aux gradient then uses the
+ *              counts passed to moe_backward (the all-reduced ones) and both
+ *              gradients divide by N.  Requires seq_len = 0, expert_choice = 0.
  * Limits: 1 <= K <= min(E, 16) (expert choice: K = E); E <= 512; n_groups <= 32, E % n_groups == 0,
  * topk_groups * (E / n_groups) >= K; D % 8 == 0; F % 8 == 0.
  */
@@ -121,6 +127,11 @@ typedef struct {
                            consecutive groups of seq_len tokens (divides T) */
   int32_t expert_choice; /* 0: token choice (top-K per token); 1: expert choice
                             (moe_route_expert_choice) */
+  int32_t loss_tokens;   /* tokens the batch aux and z losses average over:
+                            0 = T (this call's batch); data-parallel ranks that
+                            scope the losses over the global batch set the
+                            global token count (>= T) and pass the all-reduced
+                            counts (moe_aux_stats, moe_aux_loss_global) */
 } moe_config_t;
 
 typedef struct {
@@ -202,9 +213,11 @@ int moe_dispatch(const moe_config_t* cfg, const int32_t* topk_idx,
  *     (ceil(T*K / 4096) * (E + 1)) * 4 bytes; larger problems are rejected
  *     with MOE_ERR_ARG before anything is launched (1 MiB covers, e.g.,
  *     T*K up to about 4.1 M slots at E = 256).
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture on that device.
+ *   - Each call outside stream capture looks up the array's device address
+ *     (cudaGetSymbolAddress, with the calling thread's current device) and
+ *     remembers it per device; a call made while `stream` is being captured
+ *     uses the remembered address, so make the first call on each device
+ *     before any stream capture on it (else MOE_ERR_ARG).
  *   - All calls share the one array and it keeps the last call's contents
  *     (every call rewrites what it reads, nothing must start at zero).
  *     Calls that overlap on the GPU — on different streams, or from
@@ -227,6 +240,31 @@ int moe_dispatch_static(const moe_config_t* cfg, const int32_t* topk_idx,
 int moe_aux_loss(const moe_config_t* cfg, const float* probs, const float* lse,
                  const int32_t* counts, float* losses, void* ws,
                  cudaStream_t stream);
+
+/*
+ * moe_aux_stats — this batch's share of the load-balance statistics, for
+ * aux and z losses scoped over several data-parallel ranks ([STA324 §8.5]:
+ * the balance statistic over the whole batch or all devices).
+ *   sums [E+1] f32 out: sums[e] = sum_t probs[t,e], sums[E] = sum_t lse_t^2,
+ *        each reduced in a fixed order (deterministic)
+ * The caller all-reduces (sums) `sums` and the dispatch's `counts` over the
+ * ranks (NCCL), then calls moe_aux_loss_global; moe_backward with
+ * cfg.loss_tokens = N and the all-reduced counts gives each rank's share of
+ * the gradient of the global losses.
+ */
+int moe_aux_stats(const moe_config_t* cfg, const float* probs, const float* lse,
+                  float* sums, void* ws, cudaStream_t stream);
+
+/*
+ * moe_aux_loss_global — losses from all-reduced statistics:
+ * losses[0] = alpha*E*sum_e (counts_e / sum counts) (sums_e / N),
+ * losses[1] = lambda * sums[E] / N, N = cfg.loss_tokens (T if 0).
+ * [STA324 §8.5, §8.6], [TRAIN], [8MOE] ST-MoE.  counts [E] i32 and sums
+ * [E+1] f32 summed over ranks; with one rank the result equals moe_aux_loss
+ * bit for bit.  losses [2] f32 out.
+ */
+int moe_aux_loss_global(const moe_config_t* cfg, const int32_t* counts, const float* sums,
+                        float* losses, cudaStream_t stream);
 
 /*
  * moe_route_expert_choice — router of expert choice (cfg.expert_choice = 1,
@@ -374,10 +412,18 @@ int moe_combine(const moe_config_t* cfg, const void* o,
  * copies, as moe_expert_ffn_gather does (MOE_ERR_ARG for NULL x_perm on the
  * SIMT path).
  * Inside the call, independent chains (the router gradient, the two
- * weight-gradient GEMMs) are forked onto side streams that the library
- * creates once per host thread and device (on first use: make that first
- * call outside stream capture) and joined back into `stream` before the
- * call returns, so the results are ordered on `stream` like any other call.
+ * weight-gradient GEMMs) are forked onto three side streams and joined back
+ * into `stream` before the call returns, so the results are ordered on
+ * `stream` like any other call.  The side streams are the caller's when set
+ * with moe_set_backward_streams (recommended: one set per layer, so that
+ * independent layers' backward passes do not queue behind one another);
+ * otherwise the library creates three streams and eight events per host
+ * thread and device on first use (make that first call outside stream
+ * capture), shared by every call on that thread and device and kept until
+ * the process exits — the one resource besides moe_profile_enable's events
+ * that the library creates itself (no device memory).  The fork/join
+ * events are always the library's (eight per host thread and device).
+ * The counts argument feeds only the aux-loss gradient (f = counts/sum).
  */
 int moe_backward(const moe_config_t* cfg,
                  const void* x, const float* w_r, const float* logits,
@@ -417,6 +463,15 @@ int64_t moe_launch_count(int reset);
  * Applies to later calls from this host thread; returns the previous value.
  */
 int moe_set_side_streams(int enable);
+
+/*
+ * Caller-owned side streams for moe_backward on this host thread:
+ * streams[3] (created by the caller on the device the calls run on, kept
+ * alive while set), or NULL to return to the library's own.  Applies to
+ * later moe_backward calls from this thread; a layer sets its own streams
+ * before each of its backward calls.
+ */
+int moe_set_backward_streams(const cudaStream_t* streams);
 
 /*
  * Per-launch timing (measurement support; not part of the layer's math).

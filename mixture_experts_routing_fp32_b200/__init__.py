@@ -10,7 +10,8 @@ from .api import (MoEError, MoeConfig, MoeSizes, config_from, make_config,
                   moe_dispatch, moe_expert_ffn, moe_get_sizes, moe_launch_count,
                   moe_router, moe_set_side_streams, moe_aux_loss_seq, moe_bias_update,
                   moe_route_expert_choice, moe_expert_ffn_gather,
-                  moe_expert_ffn_combine)
+                  moe_expert_ffn_combine, moe_aux_stats, moe_aux_loss_global,
+                  moe_set_backward_streams)
 from .layer import MoELayer
 
 __all__ = ["MoEError", "MoeConfig", "MoeSizes", "config_from", "make_config",
@@ -18,4 +19,5 @@ __all__ = ["MoEError", "MoeConfig", "MoeSizes", "config_from", "make_config",
            "moe_dispatch", "moe_expert_ffn", "moe_get_sizes", "moe_launch_count",
            "moe_router", "moe_set_side_streams", "moe_aux_loss_seq", "moe_bias_update",
            "moe_route_expert_choice", "moe_expert_ffn_gather",
-           "moe_expert_ffn_combine", "MoELayer"]
+           "moe_expert_ffn_combine", "moe_aux_stats", "moe_aux_loss_global",
+           "moe_set_backward_streams", "MoELayer"]

@@ -29,7 +29,8 @@ EXPORTS = ("moe_get_sizes", "moe_router", "moe_dispatch", "moe_aux_loss",
            "moe_profile_name", "moe_profile_side", "moe_profile_disable",
            "moe_dispatch_static", "moe_set_side_streams", "moe_aux_loss_seq",
            "moe_bias_update", "moe_route_expert_choice", "moe_expert_ffn_gather",
-           "moe_expert_ffn_combine")
+           "moe_expert_ffn_combine", "moe_aux_stats", "moe_aux_loss_global",
+           "moe_set_backward_streams")
 
 
 class MoeConfig(ctypes.Structure):
@@ -40,7 +41,7 @@ class MoeConfig(ctypes.Structure):
                 ("capacity_factor", c_float), ("min_capacity", c_int32),
                 ("route_scale", c_float), ("aux_alpha", c_float),
                 ("z_lambda", c_float), ("gemm_impl", c_int32), ("seq_len", c_int32),
-                ("expert_choice", c_int32)]
+                ("expert_choice", c_int32), ("loss_tokens", c_int32)]
 
 
 class MoeSizes(ctypes.Structure):
@@ -94,6 +95,9 @@ def lib():
         "moe_aux_loss_seq": [cfg, P, P, P, P, P, P, P],
         "moe_bias_update": [cfg, P, P, ctypes.c_float, P],
         "moe_route_expert_choice": [cfg] + [P] * 12,
+        "moe_aux_stats": [cfg, P, P, P, P, P],
+        "moe_aux_loss_global": [cfg, P, P, P, P],
+        "moe_set_backward_streams": [P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)

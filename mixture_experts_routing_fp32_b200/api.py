@@ -27,7 +27,7 @@ def make_config(T, D, E, K, F, *, n_shared=0, dtype="bf16", score_fn=0,
                 renorm=1, n_groups=1, topk_groups=1, group_score=0,
                 capacity_factor=0.0, min_capacity=0, route_scale=1.0,
                 aux_alpha=0.0, z_lambda=0.0, gemm_impl=0, seq_len=0,
-                expert_choice=0) -> MoeConfig:
+                expert_choice=0, loss_tokens=0) -> MoeConfig:
     return MoeConfig(
         T=T, D=D, E=E, K=K, F=F, n_shared=n_shared,
         dtype=C.MOE_BF16 if dtype in ("bf16", torch.bfloat16) else C.MOE_FP32,
@@ -35,14 +35,16 @@ def make_config(T, D, E, K, F, *, n_shared=0, dtype="bf16", score_fn=0,
         topk_groups=topk_groups, group_score=group_score,
         capacity_factor=capacity_factor, min_capacity=min_capacity,
         route_scale=route_scale, aux_alpha=aux_alpha, z_lambda=z_lambda,
-        gemm_impl=gemm_impl, seq_len=seq_len, expert_choice=expert_choice)
+        gemm_impl=gemm_impl, seq_len=seq_len, expert_choice=expert_choice,
+        loss_tokens=loss_tokens)
 
 
 def config_from(obj, **over) -> MoeConfig:
     """MoeConfig from any object carrying the layer fields by name."""
     names = ("n_shared", "dtype", "score_fn", "renorm", "n_groups",
              "topk_groups", "group_score", "capacity_factor", "min_capacity",
-             "route_scale", "aux_alpha", "z_lambda", "seq_len", "expert_choice")
+             "route_scale", "aux_alpha", "z_lambda", "seq_len", "expert_choice",
+             "loss_tokens")
     kw = {n: getattr(obj, n) for n in names if hasattr(obj, n)}
     kw.update(over)
     return make_config(obj.T, obj.D, obj.E, obj.K, obj.F, **kw)
@@ -105,6 +107,28 @@ def moe_bias_update(cfg, counts, sel_bias, gamma, stream=None):
 def moe_aux_loss(cfg, probs, lse, counts, losses, ws, stream=None):
     check(lib().moe_aux_loss(ctypes.byref(cfg), _p(probs), _p(lse), _p(counts),
                              _p(losses), _p(ws), _s(stream)), "moe_aux_loss")
+
+
+def moe_aux_stats(cfg, probs, lse, sums, ws, stream=None):
+    """This batch's load statistics (sums [E+1]) for globally scoped losses."""
+    check(lib().moe_aux_stats(ctypes.byref(cfg), _p(probs), _p(lse), _p(sums), _p(ws),
+                              _s(stream)), "moe_aux_stats")
+
+
+def moe_aux_loss_global(cfg, counts, sums, losses, stream=None):
+    """Aux and z losses from all-reduced counts and sums (cfg.loss_tokens tokens)."""
+    check(lib().moe_aux_loss_global(ctypes.byref(cfg), _p(counts), _p(sums), _p(losses),
+                                    _s(stream)), "moe_aux_loss_global")
+
+
+def moe_set_backward_streams(streams=None):
+    """Caller-owned side streams (three torch.cuda.Stream) for moe_backward on
+    this thread, or None for the library's own."""
+    if streams is None:
+        check(lib().moe_set_backward_streams(None), "moe_set_backward_streams")
+        return
+    arr = (ctypes.c_void_p * 3)(*[s.cuda_stream for s in streams])
+    check(lib().moe_set_backward_streams(arr), "moe_set_backward_streams")
 
 
 def moe_expert_ffn(cfg, x_perm, offsets, tile_expert, stats, w13, w_down,
@@ -207,4 +231,5 @@ __all__ = ["LaunchProfile", "MoEError", "MoeConfig", "MoeSizes", "make_config", 
            "moe_expert_ffn", "moe_combine", "moe_backward", "moe_check_status",
            "moe_launch_count", "moe_set_side_streams", "moe_aux_loss_seq",
            "moe_bias_update", "moe_route_expert_choice", "moe_expert_ffn_gather",
-           "moe_expert_ffn_combine"]
+           "moe_expert_ffn_combine", "moe_aux_stats", "moe_aux_loss_global",
+           "moe_set_backward_streams"]

@@ -243,6 +243,8 @@ struct RouterBwdArgs {
   __nv_bfloat16* dsf;
   __nv_bfloat16* dsb;
   int Ep;
+  float Tn;                // tokens the batch aux and z losses average over (T, or the
+                           // data-parallel global count)
 };
 
 template <int NV>
@@ -288,7 +290,7 @@ router_bwd_kernel(RouterBwdArgs a) {
                         : 0.f;
         else
           dp[i] = (a.aux_alpha != 0.f && e < E && cnt_tot > 0.f)
-                      ? a.aux_alpha * (float)E * ((float)a.counts[e] / cnt_tot) / (float)a.T
+                      ? a.aux_alpha * (float)E * ((float)a.counts[e] / cnt_tot) / a.Tn
                       : 0.f;
       }
       if (!a.renorm) {
@@ -365,7 +367,7 @@ router_bwd_kernel(RouterBwdArgs a) {
     }
     if (a.z_lambda != 0.f) {
       const float l = a.lse[t];
-      const float c = 2.f * a.z_lambda * l / (float)a.T;
+      const float c = 2.f * a.z_lambda * l / a.Tn;
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int e = lane + 32 * i;

@@ -128,8 +128,15 @@ int validate(const moe_config_t* c) {
   if (!(c->route_scale == c->route_scale) || c->min_capacity < 0) return MOE_ERR_ARG;
   if ((int64_t)c->T * c->K > (int64_t)INT32_MAX / 2) return MOE_ERR_ARG;
   if (c->gemm_impl != MOE_GEMM_AUTO && c->gemm_impl != MOE_GEMM_SIMT) return MOE_ERR_ARG;
+  // globally scoped batch losses: N >= T tokens; not for the sequence-wise
+  // loss (its sequences live on one rank) or expert choice
+  if (c->loss_tokens < 0 || (c->loss_tokens > 0 && c->loss_tokens < c->T)) return MOE_ERR_ARG;
+  if (c->loss_tokens > 0 && (c->seq_len != 0 || c->expert_choice)) return MOE_ERR_ARG;
   return MOE_OK;
 }
+
+// Token count the batch aux and z losses average over.
+int64_t loss_tokens_of(const moe_config_t* c) { return c->loss_tokens > 0 ? c->loss_tokens : c->T; }
 
 // Expert choice: tokens each expert picks, C = min(T, max(ceil(c*T/E), min_capacity)).
 int64_t ec_capacity(const moe_config_t* c) {
@@ -615,6 +622,22 @@ aux_final_kernel(const float* __restrict__ part, const int32_t* __restrict__ cou
   }
 }
 
+// Column sums of the aux partials: sums[e] = sum_t probs[t,e] (e < E),
+// sums[E] = sum_t lse_t^2, each in aux_final_kernel's fixed order (a warp per
+// column, lane-strided over the chunks, then the butterfly), so that
+// aux_final_kernel on these sums (one "chunk") reproduces the local loss.
+__global__ void __launch_bounds__(512)
+aux_sums_kernel(const float* __restrict__ part, int n_chunks, int E, float* __restrict__ sums) {
+  pdl_begin();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int e = warp; e <= E; e += nw) {
+    float v = 0.f;
+    for (int c = lane; c < n_chunks; c += 32) v += part[(size_t)c * (E + 1) + e];
+    v = warp_sum(v);
+    if (lane == 0) sums[e] = v;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // expert FFN / backward GEMM sequences
 // ---------------------------------------------------------------------------
@@ -661,6 +684,9 @@ struct Side {
 thread_local Side g_side[kMaxSideDevices];
 thread_local bool g_side_enabled = true;   // moe_set_side_streams
 
+thread_local const cudaStream_t* g_caller_side = nullptr;   // moe_set_backward_streams
+thread_local cudaStream_t g_caller_side_st[3];
+
 int side_streams(Side** out) {
   int dev = 0;
   MOE_CK(cudaGetDevice(&dev));
@@ -676,6 +702,9 @@ int side_streams(Side** out) {
 }
 
 bool is_side_stream(cudaStream_t s) {
+  if (g_caller_side != nullptr &&
+      (s == g_caller_side[0] || s == g_caller_side[1] || s == g_caller_side[2]))
+    return true;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return false;
   const Side& sd = g_side[dev];
@@ -938,17 +967,24 @@ int32_t* g_static_scratch_ptr[kMaxStaticDevices] = {};
 
 // Device address of the array on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
-int static_scratch_ptr(int32_t** out) {
+// with the device current.  Outside stream capture it is looked up on every
+// call (so a context torn down and re-created on the same ordinal, e.g.
+// after cudaDeviceReset, gets the new address) and remembered; inside a
+// capture the remembered address is used, so the first call on a device
+// must come before any capture on it (MOE_ERR_ARG otherwise).
+int static_scratch_ptr(cudaStream_t s, int32_t** out) {
   int dev = 0;
   MOE_CK(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxStaticDevices) return MOE_ERR_ARG;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  MOE_CK(cudaStreamIsCapturing(s, &cap));
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_scratch_ptr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     MOE_CK(cudaGetSymbolAddress(&p, moe_static_scratch));
     g_static_scratch_ptr[dev] = static_cast<int32_t*>(p);
   }
+  if (g_static_scratch_ptr[dev] == nullptr) return MOE_ERR_ARG;
   *out = g_static_scratch_ptr[dev];
   return MOE_OK;
 }
@@ -971,7 +1007,7 @@ int moe_dispatch_static(const moe_config_t* c, const int32_t* topk_idx,
   const size_t need = ((size_t)L.n_disp_blocks * c->E + (size_t)L.n_disp_blocks) * sizeof(int32_t);
   if (need > MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_ARG;
   int32_t* base = nullptr;
-  MOE_TRY(static_scratch_ptr(&base));
+  MOE_TRY(static_scratch_ptr(s, &base));
   return dispatch_impl(c, L, topk_idx, sentinel_mask, x, counts, kept, offsets, slot_row,
                        row_slot, tile_expert, stats, x_perm, base,
                        base + (size_t)L.n_disp_blocks * c->E, s);
@@ -990,6 +1026,32 @@ int moe_aux_loss(const moe_config_t* c, const float* probs, const float* lse,
   prof_begin(s);
   MOE_CK((launch_k(aux_final_kernel, 1, 512, 0, s, part, counts, L.n_aux_chunks, c->T, c->E, c->aux_alpha,
                                      c->z_lambda, losses)));
+  MOE_LAUNCHED(s, "aux_final");
+  return MOE_OK;
+}
+
+int moe_aux_stats(const moe_config_t* c, const float* probs, const float* lse, float* sums,
+                  void* ws, cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!probs || !lse || !sums || !ws || c->seq_len > 0 || c->expert_choice) return MOE_ERR_ARG;
+  const Layout L = layout_of(c);
+  float* part = wsp<float>(ws, L.off_aux);
+  prof_begin(s);
+  MOE_CK((launch_k(aux_partial_kernel, L.n_aux_chunks, 256, 0, s, probs, lse, c->T, c->E, part)));
+  MOE_LAUNCHED(s, "aux_partial");
+  prof_begin(s);
+  MOE_CK((launch_k(aux_sums_kernel, 1, 512, 0, s, part, L.n_aux_chunks, c->E, sums)));
+  MOE_LAUNCHED(s, "aux_sums");
+  return MOE_OK;
+}
+
+int moe_aux_loss_global(const moe_config_t* c, const int32_t* counts, const float* sums,
+                        float* losses, cudaStream_t s) {
+  MOE_TRY(validate(c));
+  if (!counts || !sums || !losses || c->seq_len > 0 || c->expert_choice) return MOE_ERR_ARG;
+  prof_begin(s);
+  MOE_CK((launch_k(aux_final_kernel, 1, 512, 0, s, sums, counts, 1, (int)loss_tokens_of(c), c->E,
+                   c->aux_alpha, c->z_lambda, losses)));
   MOE_LAUNCHED(s, "aux_final");
   return MOE_OK;
 }
@@ -1262,6 +1324,9 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   Side* sd = nullptr;
   MOE_TRY(side_streams(&sd));
   cudaStream_t r = sd->st[0], w1 = sd->st[1], w2 = sd->st[2];
+  if (g_caller_side != nullptr) {
+    r = g_caller_side[0]; w1 = g_caller_side[1]; w2 = g_caller_side[2];
+  }
   if (!g_side_enabled) r = w1 = w2 = s;
   MOE_TRY(fork_join(sd->ev[0], s, r));
   if (use_tc(c)) MOE_TRY(fork_join(sd->ev[1], s, w1));
@@ -1269,7 +1334,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   {
     RouterBwdArgs a{T, E, K, c->score_fn, c->renorm, c->route_scale, c->aux_alpha, c->z_lambda,
                     logits, probs, lse, topk_idx, topk_w, slot_row, dg, counts, ds, dlogits_out,
-                    dg_out, 0, nullptr, nullptr, nullptr, 0};
+                    dg_out, 0, nullptr, nullptr, nullptr, 0, (float)loss_tokens_of(c)};
     if (c->seq_len > 0 && c->aux_alpha != 0.f) {
       // per-sequence f for the sequence-wise aux gradient
       a.seq_len = c->seq_len;
@@ -1611,6 +1676,16 @@ const char* moe_status_string(int st) {
 }
 
 int moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+int moe_set_backward_streams(const cudaStream_t* streams) {
+  if (streams == nullptr) {
+    g_caller_side = nullptr;
+    return MOE_OK;
+  }
+  for (int i = 0; i < 3; ++i) g_caller_side_st[i] = streams[i];
+  g_caller_side = g_caller_side_st;
+  return MOE_OK;
+}
 
 int moe_set_side_streams(int enable) {
   const int prev = g_side_enabled ? 1 : 0;

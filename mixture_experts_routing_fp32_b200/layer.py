@@ -9,7 +9,13 @@ and issues the entry points in order on the current stream:
             before returning); gather=True: moe_dispatch computes the
             layout only and the gate/up GEMM reads the token rows of x
             itself (no permuted copy of x; bf16 layers)
-  backward: moe_backward
+  backward: moe_backward (its three side streams owned by the layer)
+
+aux_group (a torch.distributed process group): the batch aux and z losses
+are scoped over all ranks of the group (equal per-rank token counts): the
+forward sums the ranks' expert counts and statistics (moe_aux_stats, then
+an all-reduce, then moe_aux_loss_global) and the backward uses the summed
+counts and the global token count.
 
 No host synchronisation happens inside forward or backward.
 """
@@ -18,11 +24,16 @@ from __future__ import annotations
 import torch
 
 from . import api
-from ._lib import MOE_BF16
+from ._lib import MOE_BF16, MoeConfig
 
 
 class MoELayer:
-    def __init__(self, cfg, device="cuda", gather=False):
+    def __init__(self, cfg, device="cuda", gather=False, aux_group=None):
+        cfg = MoeConfig.from_buffer_copy(cfg)
+        self.aux_group = aux_group
+        if aux_group is not None:
+            import torch.distributed as dist
+            cfg.loss_tokens = cfg.T * dist.get_world_size(aux_group)
         self.cfg = cfg
         self.gather = bool(gather)
         self.device = torch.device(device)
@@ -50,9 +61,13 @@ class MoELayer:
         self.ws = e((max(int(z.ws_bytes), 256),), torch.uint8)
         # expert choice: 1 where expert e did not pick token t (slot t*E + e)
         self.ec_mask = e((T * K,), torch.uint8) if c.expert_choice else None
+        if aux_group is not None:
+            self.counts_g = e((E,), i32)          # counts summed over the group
+            self.aux_sums = e((E + 1,), f32)      # sum_t p_{t,e}, sum_t lse_t^2
         self._grads_ready = False
         self._inputs = None
         self._aux_stream = None
+        self._bwd_streams = None
         # aux/z losses on a side stream during the expert GEMMs (False: in
         # order on the caller's stream)
         self.side_streams = True
@@ -91,6 +106,9 @@ class MoELayer:
                          self.stats, self.x_perm, self.ws)
         main = torch.cuda.current_stream(self.device)
         aux = c.aux_alpha != 0.0 or c.z_lambda != 0.0
+        if aux and self.aux_group is not None:
+            self._global_aux()
+            aux = False
         if aux and not self.side_streams:
             self._aux(None)
             aux = False
@@ -121,24 +139,47 @@ class MoELayer:
             api.moe_aux_loss(c, self.probs, self.lse, self.counts, self.losses, self.ws,
                              stream=stream)
 
+    def _global_aux(self):
+        """Losses over the whole group: local statistics, all-reduce, losses."""
+        from .dist import allreduce_aux_stats
+        c = self.cfg
+        api.moe_aux_stats(c, self.probs, self.lse, self.aux_sums, self.ws)
+        self.counts_g.copy_(self.counts)
+        allreduce_aux_stats(self.counts_g, self.aux_sums, self.aux_group)
+        api.moe_aux_loss_global(c, self.counts_g, self.aux_sums, self.losses)
+
+    def _loss_counts(self):
+        return self.counts_g if self.aux_group is not None else self.counts
+
     def update_bias(self, sel_bias, gamma):
-        """Selection-bias load-control step on this batch's counts (in place,
-        on the current stream; after forward)."""
-        api.moe_bias_update(self.cfg, self.counts, sel_bias, gamma)
+        """Selection-bias load-control step on this batch's counts (the
+        group's summed counts with aux_group; in place, on the current
+        stream; after forward)."""
+        api.moe_bias_update(self.cfg, self._loss_counts(), sel_bias, gamma)
         return sel_bias
 
     # -- backward ----------------------------------------------------------
-    def backward(self, dy, want_dg=True, want_dlogits=True):
+    def backward(self, dy, want_dg=True, want_dlogits=True, loss_counts=None):
+        """All gradients (moe_backward).  loss_counts: the expert counts the
+        aux-loss gradient uses (default: this batch's, or the group's sums
+        with aux_group)."""
         self._alloc_grads()
         x, w_r, w13, w_down, w13_s, w_down_s = self._inputs
-        api.moe_backward(
-            self.cfg, x, w_r, self.logits, self.probs, self.lse, self.topk_idx,
-            self.topk_w, self.counts, self.kept, self.offsets, self.slot_row,
-            self.row_slot, self.tile_expert, self.stats, self.x_perm, self.a13,
-            self.h, self.o, w13, w_down, w13_s, w_down_s, dy, self.dx, self.dw_r,
-            self.dw13, self.dw_down, self.dw13_s, self.dw_down_s,
-            self.dg if want_dg else None, self.dlogits if want_dlogits else None,
-            self.ws)
+        if self._bwd_streams is None:
+            self._bwd_streams = [torch.cuda.Stream(self.device) for _ in range(3)]
+        api.moe_set_backward_streams(self._bwd_streams)
+        try:
+            api.moe_backward(
+                self.cfg, x, w_r, self.logits, self.probs, self.lse, self.topk_idx,
+                self.topk_w, self._loss_counts() if loss_counts is None else loss_counts,
+                self.kept, self.offsets, self.slot_row,
+                self.row_slot, self.tile_expert, self.stats, self.x_perm, self.a13,
+                self.h, self.o, w13, w_down, w13_s, w_down_s, dy, self.dx, self.dw_r,
+                self.dw13, self.dw_down, self.dw13_s, self.dw_down_s,
+                self.dg if want_dg else None, self.dlogits if want_dlogits else None,
+                self.ws)
+        finally:
+            api.moe_set_backward_streams(None)
         return self.dx
 
     def step(self, x, dy, **weights):

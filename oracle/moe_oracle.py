@@ -93,7 +93,7 @@ class Routing:
 
 def route(logits, K, *, score_fn=SOFTMAX, renorm=1, n_groups=1,
           topk_groups=1, group_score=GROUP_MAX, route_scale=1.0,
-          sel_bias=None) -> Routing:
+          sel_bias=None, idx_given=None) -> Routing:
     """Scores, group-limited top-K selection and gate weights.
 
     Score function ([STA324] §8.2, §8.6):
@@ -115,6 +115,9 @@ def route(logits, K, *, score_fn=SOFTMAX, renorm=1, n_groups=1,
       B (renorm=1), softmax: g_k = exp(s_k) / sum_{j in T} exp(s_j)
       B (renorm=1), sigmoid: g_k = p_k / (sum_{j in T} p_j + 1e-20)
     then g *= route_scale ([TRAIN]: implementations may add a scaling).
+    idx_given (tests only): a [T,K] selection to use instead of this
+    function's own top-K (another implementation's choices on near-tie
+    tokens); scores, margins and the gate-weight formulas are unchanged.
     """
     s32 = np.asarray(logits)
     s = f64(s32)
@@ -148,6 +151,8 @@ def route(logits, K, *, score_fn=SOFTMAX, renorm=1, n_groups=1,
 
     order = np.argsort(-u, axis=1, kind="stable")
     idx = order[:, :K].copy()
+    if idx_given is not None:
+        idx = np.asarray(idx_given).astype(np.int64).reshape(T, K)
     usorted = np.take_along_axis(u, order, axis=1)
     # smallest gap between consecutive selection scores among the top K+1:
     # both which experts are chosen and their slot order hang on these
@@ -321,6 +326,20 @@ def aux_loss(counts, p, alpha, E):
     return float(alpha * E * np.dot(f, P)), f, P
 
 
+def aux_loss_from_stats(counts, p_sum, n_tokens, alpha, E):
+    """aux_loss() from pooled statistics of a batch split into parts (for
+    example data-parallel ranks): counts summed over the parts, p_sum[e] =
+    sum over all the batch's tokens of p_{t,e}, n_tokens = its token count,
+    so P_e = p_sum_e / n_tokens.  [STA324] §8.5: the balance statistic may
+    be taken over the whole batch or over all devices.
+    """
+    counts = f64(counts)
+    tot = counts.sum()
+    f = counts / tot if tot > 0 else np.zeros_like(counts)
+    P = f64(p_sum) / float(n_tokens)
+    return float(alpha * E * np.dot(f, P))
+
+
 def z_loss(lse, lam):
     """Router z-loss lambda * mean_t (logsumexp_e s_{t,e})^2.
 
@@ -375,23 +394,24 @@ def opts_of(cfg) -> Opts:
                 seq_len=getattr(cfg, "seq_len", 0))
 
 
-def route_layer(L: Layer, o: Opts) -> Routing:
+def route_layer(L: Layer, o: Opts, idx_given=None) -> Routing:
     s = router_logits(L.x, L.w_r, L.logit_offset, o.logits_fp32)
     return route(s, o.K, score_fn=o.score_fn, renorm=o.renorm,
                  n_groups=o.n_groups, topk_groups=o.topk_groups,
                  group_score=o.group_score, route_scale=o.route_scale,
-                 sel_bias=L.sel_bias)
+                 sel_bias=L.sel_bias, idx_given=idx_given)
 
 
-def forward(L: Layer, o: Opts):
+def forward(L: Layer, o: Opts, idx_given=None):
     """y_t = sum_{k kept} g_{t,k} E_{idx_k}(x_t) (+ shared(x_t)), plus losses.
 
     [8MOE] Router / Gating Network: y = sum_i G(x)_i E_i(x); [STA324] §8.8:
     a token appears K times, so outputs accumulate; §8.7: the shared expert
     runs on every token, unweighted, and takes no top-K slot.
     Returns a dict with routing, dispatch, per-slot SwiGLU values and y.
+    idx_given (tests only): see route().
     """
-    return forward_routed(L, o, route_layer(L, o))
+    return forward_routed(L, o, route_layer(L, o, idx_given))
 
 
 def forward_routed(L: Layer, o: Opts, R: Routing):
@@ -609,6 +629,54 @@ def token_forward_backward(L: Layer, o: Opts, R: Routing, Dp: Dispatch, t,
     return dict(y=y[0], dg=dg, ds=ds, dx=dx[0])
 
 
+def tokens_forward_backward(L: Layer, o: Opts, R: Routing, Dp: Dispatch, toks,
+                            dy_toks):
+    """y, dg, ds and dx of the tokens `toks` (exact), as token_forward_backward
+    on each of them, but expert by expert: every expert's weights are fetched
+    once for all the sampled slots it serves (full-size layers regenerate
+    them on demand).  Returns arrays with one row per entry of `toks`.
+    """
+    toks = np.asarray(toks, dtype=np.int64)
+    n = toks.size
+    K = o.K
+    T = L.x.shape[0]
+    xt = f64(L.x[toks])
+    dyt = f64(dy_toks).reshape(n, -1)
+    D = xt.shape[1]
+    y = np.zeros((n, D))
+    dg = np.zeros((n, K))
+    dx = np.zeros((n, D))
+    by_e = {}
+    for i, t in enumerate(toks):
+        for k, e in token_slots(Dp, int(t), K):
+            by_e.setdefault(e, []).append((i, k))
+    # per token, its slots' terms are added in k order
+    contrib = {}
+    for e in sorted(by_e):
+        ik = np.array(by_e[e])
+        ii, kk = ik[:, 0], ik[:, 1]
+        w13, wd = L.w13(e), L.wd(e)
+        a, b, h, oo = swiglu_forward(xt[ii], w13, wd)
+        g = R.g[toks[ii], kk]
+        dg[ii, kk] = (oo * dyt[ii]).sum(axis=1)
+        dxr, _, _ = swiglu_backward(xt[ii], a, b, h, g[:, None] * dyt[ii], w13, wd)
+        for r in range(ii.size):
+            contrib[(int(ii[r]), int(kk[r]))] = (g[r] * oo[r], dxr[r])
+    for (i, k) in sorted(contrib):
+        y[i] += contrib[(i, k)][0]
+        dx[i] += contrib[(i, k)][1]
+    if L.w13_s is not None:
+        a, b, h, oo = swiglu_forward(xt, L.w13_s, L.wd_s)
+        y += oo
+        dxr, _, _ = swiglu_backward(xt, a, b, h, dyt, L.w13_s, L.wd_s)
+        dx += dxr
+    Rt = Routing(logits=R.logits[toks], p=R.p[toks], lse=R.lse[toks],
+                 idx=R.idx[toks], g=R.g[toks], margin=R.margin[toks])
+    ds = router_backward(Rt, dg, o, Dp.counts, T_total=T)
+    dx += ds @ f64(L.w_r)
+    return dict(y=y, dg=dg, ds=ds, dx=dx)
+
+
 def expert_column_grads(L: Layer, o: Opts, R: Routing, Dp: Dispatch, e, j,
                         dy_rows):
     """dW13[e][j,:], dW13[e][F+j,:] and dW_down[e][:,j] from the expert's rows.
@@ -616,31 +684,38 @@ def expert_column_grads(L: Layer, o: Opts, R: Routing, Dp: Dispatch, e, j,
     dy_rows(tokens) -> [n, D] upstream gradient rows.  Needs only rows j and
     F+j of W13[e] and column j of W_down[e] (passed by the callables
     w13_rows(e, rows) / wd_col(e, j) when present on L, else sliced).
+    j may be a list of columns: each result then has one row per column.
     """
+    js = np.atleast_1d(np.asarray(j, dtype=np.int64))
     K = o.K
     slots = np.nonzero((Dp.expert == e) & (Dp.rank >= 0))[0]
     slots = slots[np.argsort(Dp.rank[slots])]
     toks = slots // K
-    F = None
     if hasattr(L, "w13_rows"):
         F = L.F
-        wg = f64(L.w13_rows(e, [j, F + j]))
-        wdj = f64(L.wd_col(e, j))
+        wg = f64(L.w13_rows(e, np.concatenate([js, F + js])))
+        wdj = np.stack([f64(L.wd_col(e, int(c))) for c in js], axis=1)   # [D, n_j]
     else:
         w13 = f64(L.w13(e))
         F = w13.shape[0] // 2
-        wg = w13[[j, F + j]]
-        wdj = f64(L.wd(e))[:, j]
+        wg = w13[np.concatenate([js, F + js])]
+        wdj = f64(L.wd(e))[:, js]
     D = wg.shape[1]
+    nj = js.size
     if slots.size == 0:
-        return np.zeros(D), np.zeros(D), np.zeros(D)
-    xr = f64(L.x[toks])
-    a = xr @ wg[0]
-    b = xr @ wg[1]
-    do = R.g.reshape(-1)[slots, None] * f64(dy_rows(toks))
-    dh = do @ wdj
-    sa = 1.0 / (1.0 + np.exp(-a))
-    da = dh * b * sa * (1.0 + a * (1.0 - sa))
-    db = dh * silu(a)
-    h = silu(a) * b
-    return da @ xr, db @ xr, do.T @ h
+        z = np.zeros((nj, D))
+        out = (z, z.copy(), z.copy())
+    else:
+        xr = f64(L.x[toks])
+        a = xr @ wg[:nj].T                     # [rows, n_j]
+        b = xr @ wg[nj:].T
+        do = R.g.reshape(-1)[slots, None] * f64(dy_rows(toks))
+        dh = do @ wdj
+        sa = 1.0 / (1.0 + np.exp(-a))
+        da = dh * b * sa * (1.0 + a * (1.0 - sa))
+        db = dh * silu(a)
+        h = silu(a) * b
+        out = (da.T @ xr, db.T @ xr, (do.T @ h).T)
+    if np.ndim(j) == 0:
+        return tuple(v[0] for v in out)
+    return out

@@ -38,8 +38,8 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_config_struct_layout_matches_header():
-    # 12 int32 fields, then float, int32, 3 floats, 3 int32 = 20 x 4 bytes
-    assert ctypes.sizeof(C.MoeConfig) == 20 * 4
+    # 12 int32 fields, then float, int32, 3 floats, 4 int32 = 21 x 4 bytes
+    assert ctypes.sizeof(C.MoeConfig) == 21 * 4
     assert ctypes.sizeof(C.MoeSizes) == 40
 
 
@@ -85,6 +85,9 @@ def test_sizes(lib, T, D, E, K, F, c, ns):
     dict(expert_choice=1, K=4, capacity_factor=1.0, renorm=1),   # ... and variant A
     dict(expert_choice=1, K=4, capacity_factor=1.0, renorm=0, aux_alpha=0.01),
     dict(dtype="fp16"),               # maps to fp32 -> still valid; replaced below
+    dict(loss_tokens=32),             # global loss token count below T
+    dict(loss_tokens=-1),
+    dict(loss_tokens=128, seq_len=32),    # global scope is for the batch losses only
 ])
 def test_invalid_configs_rejected(lib, bad):
     kw = dict(T=64, D=32, E=4, K=2, F=64)
@@ -140,3 +143,18 @@ def test_package_has_no_cpu_fallback():
         if name.endswith(".py"):
             src = open(os.path.join(pkg, name)).read()
             assert "oracle" not in src.replace("never imports the oracle", ""), name
+
+
+def test_global_loss_entry_points_validate_on_host(lib):
+    """moe_aux_stats / moe_aux_loss_global refuse NULL buffers and the
+    sequence-wise configuration before any launch; a loss token count of at
+    least T is accepted."""
+    ok = api.make_config(64, 32, 4, 2, 64, dtype="fp32", aux_alpha=0.01, loss_tokens=256)
+    out = C.MoeSizes()
+    assert lib.moe_get_sizes(ctypes.byref(ok), ctypes.byref(out)) == C.MOE_OK
+    assert lib.moe_aux_stats(ctypes.byref(ok), None, None, None, None, None) == C.MOE_ERR_ARG
+    assert lib.moe_aux_loss_global(ctypes.byref(ok), None, None, None, None) == C.MOE_ERR_ARG
+    seq = api.make_config(64, 32, 4, 2, 64, dtype="fp32", aux_alpha=0.01, seq_len=32)
+    dummy = ctypes.c_void_p(256)
+    assert lib.moe_aux_stats(ctypes.byref(seq), dummy, dummy, dummy, dummy, None) == C.MOE_ERR_ARG
+    assert lib.moe_set_backward_streams(None) == C.MOE_OK

@@ -58,11 +58,28 @@ def host(t):
     return t.detach().float().cpu().numpy() if t.dtype != torch.int32 else t.cpu().numpy()
 
 
-def check_dispatch(cfg, layer, R, Dp):
-    """Bit-exact routing / permutation (or validity when a near-tie flipped)."""
+def gpu_routed_oracle(cfg, layer, R):
+    """The GPU's selection checked against the oracle's (bit-exact except on
+    near-tie tokens, fp32 margin < 1e-5), then the oracle's dispatch of the
+    GPU's own selection: the permutation every later output depends on.
+    Returns (flipped tokens, oracle Dispatch of the GPU's idx)."""
     idx = layer.topk_idx.cpu().numpy()
     diff = np.nonzero((idx != R.idx).any(axis=1))[0]
     assert np.all(R.margin[diff] < O.NEAR_TIE), ("non-near-tie routing mismatch", diff[:10])
+    mask = W.make_input(cfg, "sentinel_mask").numpy() if cfg.sentinel_frac else None
+    Dp = O.dispatch(idx, cfg.E, cfg.capacity_factor, cfg.min_capacity, mask)
+    return diff, Dp
+
+
+def check_dispatch(cfg, layer, R, Dp=None):
+    """Bit-exact routing and permutation.  The selection matches the oracle's
+    except on near-tie tokens; the dispatch (counts, kept, drops, sentinels,
+    every slot's expert and rank) matches the oracle's counting sort of the
+    GPU's own selection exactly.  Returns (number of flipped tokens, that
+    oracle Dispatch)."""
+    diff, Dg = gpu_routed_oracle(cfg, layer, R)
+    if diff.size == 0 and Dp is not None:
+        assert np.array_equal(Dg.rank, Dp.rank) and np.array_equal(Dg.expert, Dp.expert)
     E, K, T = cfg.E, cfg.K, cfg.T
     counts, kept = host(layer.counts), host(layer.kept)
     offsets, stats = host(layer.offsets), host(layer.stats)
@@ -90,55 +107,43 @@ def check_dispatch(cfg, layer, R, Dp):
     if cfg.n_shared:
         pad_rows[offsets[E]:offsets[E] + T] = False
     assert np.all(row_slot[:n_rows][pad_rows] == -1)
-    assert np.all(host(layer.x_perm)[:n_rows][pad_rows] == 0)
-    if diff.size == 0:
-        assert np.array_equal(counts, Dp.counts)
-        assert np.array_equal(kept, Dp.kept)
-        assert int(stats[0]) == Dp.n_drop
-        assert int(stats[1]) == Dp.n_sentinel
-        assert np.array_equal(ex, np.where(Dp.rank >= 0, Dp.expert, -1))
-        assert np.array_equal(rk, Dp.rank)
-    else:
-        # A near-tie flipped a choice or a slot order, so the permutation is
-        # checked for validity against the GPU's own indices: each expert's
-        # kept slots are its first min(n_e, C) valid slots in flat-slot
-        # order, ranked 0, 1, ... (the definition of the stable counting
-        # sort with capacity), and everything else is dropped or sentinel.
-        e_slot = idx.reshape(-1).astype(np.int64)
-        if cfg.sentinel_frac:
-            e_slot = np.where(W.make_input(cfg, "sentinel_mask").numpy().astype(bool), -1, e_slot)
-        C = None if cfg.capacity_factor <= 0 else max(
-            int(np.ceil(cfg.capacity_factor * T * K / E)), cfg.min_capacity)
-        for e in range(E):
-            js = np.nonzero(e_slot == e)[0]                # increasing flat order
-            assert counts[e] == js.size
-            keep = js if C is None else js[:C]
-            assert kept[e] == keep.size
-            assert np.array_equal(rk[keep], np.arange(keep.size))
-            assert np.all(ex[keep] == e)
-            assert np.all(rk[js[keep.size:]] == -1)
-        assert np.all(rk[e_slot < 0] == -1)
-    return diff.size
+    if layer.x_perm is not None:
+        assert np.all(host(layer.x_perm)[:n_rows][pad_rows] == 0)
+    assert np.array_equal(counts, Dg.counts)
+    assert np.array_equal(kept, Dg.kept)
+    assert int(stats[0]) == Dg.n_drop
+    assert int(stats[1]) == Dg.n_sentinel
+    assert np.array_equal(ex, np.where(Dg.rank >= 0, Dg.expert, -1))
+    assert np.array_equal(rk, Dg.rank)
+    assert np.all(slot_row[Dg.sentinel] == -2) and np.all(slot_row[Dg.dropped] == -1)
+    return diff.size, Dg
+
+
+def oracle_on_gpu_routing(cfg, layer, L=None):
+    """Oracle forward + backward on the GPU's own top-K selection (identical
+    to the oracle's own except on near-tie tokens, which route_layer checks
+    and counts).  Returns (fw, bw, flips)."""
+    L = L or oracle_layer(cfg)
+    o = O.opts_of(cfg)
+    R_own = O.route_layer(L, o)
+    flips, _ = check_dispatch(cfg, layer, R_own)
+    fw = O.forward(L, o, idx_given=layer.topk_idx.cpu().numpy())
+    bw = O.backward(L, o, fw, W.make_input(cfg, "dy").double().numpy())
+    return fw, bw, flips
 
 
 @pytest.mark.parametrize("name", [n for n, c in W.REDUCED.items() if not c.expert_choice])
 def test_parity_reduced(name):
     cfg = W.REDUCED[name]
     layer, inp = run_gpu(cfg)
-    L = oracle_layer(cfg)
-    o = O.opts_of(cfg)
-    fw = O.forward(L, o)
-    dy = W.make_input(cfg, "dy").double().numpy()
-    bw = O.backward(L, o, fw, dy)
-    R, Dp = fw["R"], fw["Dp"]
+    fw, bw, flips = oracle_on_gpu_routing(cfg, layer)
+    R = fw["R"]
     tl = tol(cfg)
     # router (fp32 on both sides)
     assert rel_l2(host(layer.logits), R.logits) < 1e-5
     assert rel_l2(host(layer.probs), R.p) < 1e-5
     assert rel_l2(host(layer.lse), R.lse) < 1e-5
-    flips = check_dispatch(cfg, layer, R, Dp)
-    same = (layer.topk_idx.cpu().numpy() == R.idx).all(axis=1)
-    assert rel_l2(host(layer.topk_w)[same], R.g[same]) < 1e-5
+    assert rel_l2(host(layer.topk_w), R.g) < 1e-5
     # forward output and losses
     assert rel_l2(host(layer.y), fw["y"]) < tl
     if cfg.aux_alpha:
@@ -189,10 +194,10 @@ def test_tensor_core_path_matches_simt_path(name):
     for attr in ("dw13", "dw_down", "dw_r"):
         a, b = getattr(tc, attr).float(), getattr(simt, attr).float()
         assert (a - b).norm() / b.norm() < (1e-2 if not flip.any() else 5e-2), attr
-    if flip.any():
-        return
     # the two paths may align expert segments differently (CTA-pair tiles
     # use 256-row segments): compare every slot's expert and rank instead
+    # (each path's permutation is also checked against the oracle's
+    # counting sort of its own selection in test_parity_reduced)
     def expert_rank(L):
         sr = L.slot_row.long()
         kept = sr >= 0
@@ -201,8 +206,10 @@ def test_tensor_core_path_matches_simt_path(name):
         e[kept] = L.tile_expert.long()[sr[kept] // 128]
         r[kept] = sr[kept] - L.offsets.long()[e[kept]]
         return e, r
-    for a, b in zip(expert_rank(tc), expert_rank(simt)):
-        assert torch.equal(a, b)
+    if not flip.any():
+        for a, b in zip(expert_rank(tc), expert_rank(simt)):
+            assert torch.equal(a, b)
+    print("%s: tensor-core vs SIMT selection flips %d" % (name, int(flip.sum())))
 
 
 def test_k1_variant_b_router_grad_is_exactly_aux_only():
@@ -272,30 +279,43 @@ def test_sentinel_slots_are_marked_minus_two():
     assert np.all(sr[~mask] >= -1)
 
 
+def ec_oracle_on_gpu_choice(cfg, layer):
+    """Expert-choice oracle on the GPU's own picks: each expert's C picks
+    bit-exact against the oracle's except experts whose C-th and (C+1)-th
+    fp32 scores nearly tie (counted); then the oracle's forward and backward
+    with the GPU's picks.  Returns (Lc, o, fw, bw, R, n_flipped_experts)."""
+    from oracle import expert_choice as X
+    L = oracle_layer(cfg)
+    R, chosen_own, C = X.route(L, cfg.capacity_factor, cfg.min_capacity)
+    T, E = cfg.T, cfg.E
+    chosen = layer.ec_mask.cpu().numpy().reshape(T, E) == 0
+    assert np.all(chosen.sum(axis=0) == C)
+    flip = (chosen != chosen_own).any(axis=0)
+    assert np.all(X.ec_margin(R.p, C)[flip] < O.NEAR_TIE), np.nonzero(flip)[0]
+    Lc = X.layer_for(L, chosen)
+    o = X.opts_for(E, cfg.z_lambda)
+    fw = O.forward_routed(Lc, o, R)
+    fw["chosen"], fw["C"] = chosen, C
+    bw = O.backward(Lc, o, fw, W.make_input(cfg, "dy").double().numpy())
+    return Lc, o, fw, bw, R, int(flip.sum())
+
+
 @pytest.mark.parametrize("name", ["ec8", "olmoe_ec"])
 def test_expert_choice_parity(name):
     """Expert choice against its oracle: every expert's picks bit-exact
-    (except experts whose C-th and (C+1)-th fp32 scores nearly tie), exactly
-    C rows per expert, outputs and all gradients within the bf16 tolerance."""
-    from oracle import expert_choice as X
+    (except experts whose C-th and (C+1)-th fp32 scores nearly tie, where the
+    oracle then runs on the GPU's picks), exactly C rows per expert, outputs
+    and all gradients within the bf16 tolerance."""
     cfg = W.REDUCED[name]
     layer, inp = run_gpu(cfg)
-    L = oracle_layer(cfg)
-    Lc, o, fw = X.forward(L, cfg.capacity_factor, cfg.min_capacity, z_lambda=cfg.z_lambda)
-    R = fw["R"]
-    T, E, C = cfg.T, cfg.E, fw["C"]
+    Lc, o, fw, bw, R, flips = ec_oracle_on_gpu_choice(cfg, layer)
+    E, C = cfg.E, fw["C"]
     assert rel_l2(host(layer.logits), R.logits) < 1e-5
     assert rel_l2(host(layer.probs), R.p) < 1e-5
-    chosen = (layer.ec_mask.cpu().numpy().reshape(T, E) == 0)
-    assert np.all(chosen.sum(axis=0) == C)
-    flip = (chosen != fw["chosen"]).any(axis=0)
-    if flip.any():
-        assert np.all(X.ec_margin(R.p, C)[flip] < O.NEAR_TIE), np.nonzero(flip)[0]
-        return
     assert np.array_equal(host(layer.counts), np.full(E, C))
+    Dp = fw["Dp"]
+    assert np.array_equal(host(layer.slot_row) >= 0, Dp.rank >= 0)
     assert rel_l2(host(layer.y), fw["y"]) < tol(cfg)
-    dy = W.make_input(cfg, "dy").double().numpy()
-    bw = O.backward(Lc, o, fw, dy)
     for attr, ref in (("dx", bw["dx"]), ("dw_r", bw["dw_r"]), ("dg", bw["dg"]),
                       ("dlogits", bw["ds"])):
         assert rel_l2(host(getattr(layer, attr)), ref) < tol(cfg), attr
@@ -303,6 +323,8 @@ def test_expert_choice_parity(name):
     assert rel_l2(host(layer.dw_down), np.stack([bw["dwd"][e] for e in range(E)])) < tol(cfg)
     if cfg.z_lambda:
         assert abs(float(layer.losses[1]) - fw["z"]) <= 1e-5 * abs(fw["z"])
+    print("%s: expert-choice near-tie flips %d (experts), GPU near-ties %d" % (
+        name, flips, int(layer.near_ties[0])))
 
 
 def padding_rows(layer, cfg):
@@ -338,7 +360,7 @@ def assert_gather_identical(cfg, ref, fused):
                                   "olmoe_ec"])
 def test_fused_gather_matches_permuted_copy(name):
     """gate/up A rows (forward) and gate/up weight-gradient B rows (backward)
-    read from the token rows of x by tile::gather4 copies inside the GEMMs
+    copied from the token rows of x by the GEMMs' producer warp (cp.async)
     (single CTAs and CTA pairs, shared expert, expert choice, capacity
     drops, sentinels) against the same GEMMs on the dispatch's permuted copy
     of x, and against the oracle."""
@@ -347,16 +369,15 @@ def test_fused_gather_matches_permuted_copy(name):
     fused, _ = run_gpu(cfg, inp=inp, gather=True)
     assert_gather_identical(cfg, ref, fused)
     if cfg.expert_choice:
-        return   # expert-choice oracle parity: test_expert_choice_parity on the same GEMMs
-    L = oracle_layer(cfg)
-    o = O.opts_of(cfg)
-    fw = O.forward(L, o)
-    if (fused.topk_idx.cpu().numpy() != fw["R"].idx).any():
-        return   # a near-tie flip: the permuted-copy path's parity test covers it
-    bw = O.backward(L, o, fw, W.make_input(cfg, "dy").double().numpy())
+        _, _, fw, bw, _, flips = ec_oracle_on_gpu_choice(cfg, fused)
+    else:
+        fw, bw, flips = oracle_on_gpu_routing(cfg, fused)
     assert rel_l2(host(fused.y), fw["y"]) < tol(cfg)
     assert rel_l2(host(fused.dx), bw["dx"]) < tol(cfg)
     assert rel_l2(host(fused.dw13), np.stack([bw["dw13"][e] for e in range(cfg.E)])) < tol(cfg)
+    assert rel_l2(host(fused.dw_down), np.stack([bw["dwd"][e] for e in range(cfg.E)])) < tol(cfg)
+    assert rel_l2(host(fused.dw_r), bw["dw_r"]) < tol(cfg)
+    print("%s fused gather: near-tie flips %d" % (name, flips))
 
 
 @pytest.mark.parametrize("name", ["mm_b", "mm_mask", "mm_pair"])

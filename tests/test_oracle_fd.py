@@ -155,3 +155,62 @@ def test_sampled_helpers_match_full_oracle(name):
         np.testing.assert_allclose(a, bw["dw13"][e][j], rtol=1e-9, atol=1e-12)
         np.testing.assert_allclose(b, bw["dw13"][e][cfg.F + j], rtol=1e-9, atol=1e-12)
         np.testing.assert_allclose(c, bw["dwd"][e][:, j], rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("name", ["olmoe", "mix", "ds3"])
+def test_batched_sampled_helpers_match_full_oracle(name):
+    """The expert-major sampled-token pass and the multi-column weight
+    gradients used by the full-size checks give the rows of the
+    finite-difference-pinned full forward/backward."""
+    from tests.helpers import LazyLayer
+    cfg = W.REDUCED[name].replace(T=160, D=64, F=48)
+    L = oracle_layer(cfg)
+    o = O.opts_of(cfg)
+    dy = W.make_input(cfg, "dy").double().numpy()
+    fw = O.forward(L, o)
+    bw = O.backward(L, o, fw, dy)
+    R, Dp = fw["R"], fw["Dp"]
+    toks = np.array([0, 7, 33, 34, 90, cfg.T - 1])
+    r = O.tokens_forward_backward(L, o, R, Dp, toks, dy[toks])
+    np.testing.assert_allclose(r["y"], fw["y"][toks], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(r["dg"], bw["dg"][toks], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(r["ds"], bw["ds"][toks], rtol=1e-9, atol=1e-13)
+    np.testing.assert_allclose(r["dx"], bw["dx"][toks], rtol=1e-9, atol=1e-12)
+    LL = LazyLayer(cfg, L.x)
+    js = [0, 5, cfg.F - 1]
+    for e in (0, cfg.E - 1):
+        a, b, c = O.expert_column_grads(LL, o, R, Dp, e, js, lambda rows: dy[rows])
+        np.testing.assert_allclose(a, bw["dw13"][e][js], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(b, bw["dw13"][e][[cfg.F + j for j in js]], rtol=1e-9,
+                                   atol=1e-12)
+        np.testing.assert_allclose(c, bw["dwd"][e][:, js].T, rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("name", ["mix", "ds3", "olmoe"])
+def test_given_selection_keeps_the_gate_formulas(name):
+    """route(idx_given=...) with the oracle's own choices changes nothing;
+    with another valid choice on one token it recomputes that token's gate
+    weights by the same formula (A: the scores; B: renormalised over the
+    given set) and leaves every other token as it was."""
+    cfg = W.REDUCED[name].replace(T=40, D=32, F=16)
+    L = oracle_layer(cfg)
+    o = O.opts_of(cfg)
+    R = O.route_layer(L, o)
+    R2 = O.route_layer(L, o, idx_given=R.idx)
+    for f in ("idx", "g", "margin"):
+        np.testing.assert_array_equal(getattr(R2, f), getattr(R, f))
+    idx = R.idx.copy()
+    t = 3
+    other = [e for e in range(cfg.E) if e not in idx[t]][0]
+    idx[t, -1] = other
+    R3 = O.route_layer(L, o, idx_given=idx)
+    keep = np.arange(cfg.T) != t
+    np.testing.assert_array_equal(R3.g[keep], R.g[keep])
+    sel = R.p[t, idx[t]]
+    if cfg.score_fn == O.SOFTMAX and cfg.renorm:
+        exp = sel / sel.sum()
+    elif cfg.renorm:
+        exp = sel / (sel.sum() + O.SIGMOID_EPS)
+    else:
+        exp = sel
+    np.testing.assert_allclose(R3.g[t], exp * cfg.route_scale, rtol=1e-12)

@@ -411,3 +411,21 @@ def test_swiglu_backward_matches_autograd():
     np.testing.assert_allclose(dx, x.grad.numpy(), rtol=1e-11, atol=1e-13)
     np.testing.assert_allclose(dw13, w13.grad.numpy(), rtol=1e-11, atol=1e-13)
     np.testing.assert_allclose(dwd, wd.grad.numpy(), rtol=1e-11, atol=1e-13)
+
+
+def test_aux_loss_from_pooled_stats():
+    """The pooled-statistics form gives the page's worked example (E=2,
+    f=[.75,.25], P=[.6,.4], alpha=.01 -> .011, [STA324] §8.5) and equals the
+    batch loss on the concatenated batch when split into two parts."""
+    assert abs(O.aux_loss_from_stats([3, 1], [1.2, 0.8], 2, 0.01, 2) - 0.011) < 1e-15
+    rng = np.random.default_rng(3)
+    T, E, K = 50, 6, 2
+    s = rng.normal(size=(T, E))
+    R = O.route(s, K, renorm=0)
+    Dp = O.dispatch(R.idx, E)
+    full, _, _ = O.aux_loss(Dp.counts, R.p, 0.01, E)
+    a, b = slice(0, 21), slice(21, T)
+    ca = O.dispatch(R.idx[a], E).counts
+    cb = O.dispatch(R.idx[b], E).counts
+    pooled = O.aux_loss_from_stats(ca + cb, R.p[a].sum(0) + R.p[b].sum(0), T, 0.01, E)
+    assert abs(pooled - full) < 1e-15
