@@ -111,6 +111,24 @@ enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SIMT = 1 };   /* cfg.gemm_impl */
  *              whole batch or all devices): the aux gradient then uses the
  *              counts passed to moe_backward (the all-reduced ones) and both
  *              gradients divide by N.  Requires seq_len = 0, expert_choice = 0.
+ *   expert_base, n_local_experts
+ *              expert parallelism ([HF48687]: under expert parallelism every
+ *              rank sees the global routing and the slots of experts it
+ *              does not hold are sentinels, whose expert output is zero;
+ *              [8MOE] DeepSpeed / [TRAIN] all-to-all flow).  With
+ *              n_local_experts = El > 0 this call holds routed experts
+ *              [expert_base, expert_base + El): moe_router, the aux / z
+ *              losses and the router gradient stay over all E experts
+ *              (logits, probs [T,E], counts [E]); moe_dispatch gives the
+ *              slots of other experts slot_row = -2 (counted in stats[1])
+ *              and lays out only the local experts (kept [El], offsets
+ *              [El+2], tile_expert values < El, capacity still
+ *              ceil(c*T*K/E)); the expert weights and their gradients are
+ *              [El, ...].  y, dx, dW_r, dlogits and dg of the shards sum to
+ *              those of the whole layer (add the aux / z losses on one shard
+ *              only).  Requires the tensor-core path (bf16, D and F
+ *              multiples of 128), n_shared = 0, seq_len = 0 and token
+ *              choice.
  * Limits: 1 <= K <= min(E, 16) (expert choice: K = E); E <= 512; n_groups <= 32, E % n_groups == 0,
  * topk_groups * (E / n_groups) >= K; D % 8 == 0; F % 8 == 0.
  */
@@ -132,6 +150,8 @@ typedef struct {
                             scope the losses over the global batch set the
                             global token count (>= T) and pass the all-reduced
                             counts (moe_aux_stats, moe_aux_loss_global) */
+  int32_t expert_base;     /* expert parallelism: first routed expert this call's */
+  int32_t n_local_experts; /* expert FFN holds (0 = all E experts, no sharding) */
 } moe_config_t;
 
 typedef struct {

@@ -41,7 +41,8 @@ class MoeConfig(ctypes.Structure):
                 ("capacity_factor", c_float), ("min_capacity", c_int32),
                 ("route_scale", c_float), ("aux_alpha", c_float),
                 ("z_lambda", c_float), ("gemm_impl", c_int32), ("seq_len", c_int32),
-                ("expert_choice", c_int32), ("loss_tokens", c_int32)]
+                ("expert_choice", c_int32), ("loss_tokens", c_int32),
+                ("expert_base", c_int32), ("n_local_experts", c_int32)]
 
 
 class MoeSizes(ctypes.Structure):

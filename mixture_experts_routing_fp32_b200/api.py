@@ -27,7 +27,8 @@ def make_config(T, D, E, K, F, *, n_shared=0, dtype="bf16", score_fn=0,
                 renorm=1, n_groups=1, topk_groups=1, group_score=0,
                 capacity_factor=0.0, min_capacity=0, route_scale=1.0,
                 aux_alpha=0.0, z_lambda=0.0, gemm_impl=0, seq_len=0,
-                expert_choice=0, loss_tokens=0) -> MoeConfig:
+                expert_choice=0, loss_tokens=0, expert_base=0,
+                n_local_experts=0) -> MoeConfig:
     return MoeConfig(
         T=T, D=D, E=E, K=K, F=F, n_shared=n_shared,
         dtype=C.MOE_BF16 if dtype in ("bf16", torch.bfloat16) else C.MOE_FP32,
@@ -36,7 +37,7 @@ def make_config(T, D, E, K, F, *, n_shared=0, dtype="bf16", score_fn=0,
         capacity_factor=capacity_factor, min_capacity=min_capacity,
         route_scale=route_scale, aux_alpha=aux_alpha, z_lambda=z_lambda,
         gemm_impl=gemm_impl, seq_len=seq_len, expert_choice=expert_choice,
-        loss_tokens=loss_tokens)
+        loss_tokens=loss_tokens, expert_base=expert_base, n_local_experts=n_local_experts)
 
 
 def config_from(obj, **over) -> MoeConfig:
@@ -44,7 +45,7 @@ def config_from(obj, **over) -> MoeConfig:
     names = ("n_shared", "dtype", "score_fn", "renorm", "n_groups",
              "topk_groups", "group_score", "capacity_factor", "min_capacity",
              "route_scale", "aux_alpha", "z_lambda", "seq_len", "expert_choice",
-             "loss_tokens")
+             "loss_tokens", "expert_base", "n_local_experts")
     kw = {n: getattr(obj, n) for n in names if hasattr(obj, n)}
     kw.update(over)
     return make_config(obj.T, obj.D, obj.E, obj.K, obj.F, **kw)

@@ -73,8 +73,8 @@ __device__ __forceinline__ int warp_count(const int (&ev)[kDispIters], int32_t* 
 // first slot of expert e, and is advanced), capacity drop, slot <-> row maps.
 __device__ __forceinline__ void warp_rank(const int (&ev)[kDispIters], int64_t j0,
                                           int64_t n_slots, int64_t C, int64_t rows_max,
-                                          int32_t* row, const int32_t* seg_off,
-                                          int32_t* __restrict__ slot_row,
+                                          int32_t* row, const int32_t* seg_off, int ebase,
+                                          int El, int32_t* __restrict__ slot_row,
                                           int32_t* __restrict__ row_slot) {
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
@@ -90,9 +90,11 @@ __device__ __forceinline__ void warp_rank(const int (&ev)[kDispIters], int64_t j
     if (e >= 0 && (peers & lt) == 0) row[e] += __popc(peers);
     __syncwarp();
     if (e != -2) {
-      int32_t r = e == -1 ? -2 : -1;     // -2: sentinel, -1: dropped
-      if (e >= 0 && (C < 0 || rank < C)) {
-        r = seg_off[e] + rank;
+      // -2: sentinel or another shard's expert, -1: dropped
+      const bool local = e >= ebase && e < ebase + El;
+      int32_t r = (e == -1 || (e >= 0 && !local)) ? -2 : -1;
+      if (local && (C < 0 || rank < C)) {
+        r = seg_off[e - ebase] + rank;
         if (r < rows_max) row_slot[r] = (int32_t)j;
         else { set_dev_error(MOE_DEVERR_ROWS); r = -1; }
       }
@@ -101,33 +103,42 @@ __device__ __forceinline__ void warp_rank(const int (&ev)[kDispIters], int64_t j
   }
 }
 
-// Block-wide: from per-expert totals (tot[e], shared) derive counts, kept
-// (capacity), segment offsets aligned to `align` rows (seg[e], shared, and
-// offsets[] in global memory), the tile -> expert map and the stats words.
+// Block-wide: from per-expert totals (tot[e], shared, over all E experts)
+// derive counts (all E), and for the local experts [ebase, ebase + El):
+// kept (capacity), segment offsets aligned to `align` rows (seg[l], shared,
+// and offsets[] in global memory), the tile -> local expert map and the
+// stats words.  Valid slots of other experts count as sentinels here.
 // Called by every thread of the block; ends with a __syncthreads.
-__device__ void finish_layout(const int32_t* tot, int32_t* seg, int E, int T, int n_shared,
-                              int64_t C, int64_t rows_max, int align, int32_t sentinels,
-                              int32_t* __restrict__ counts, int32_t* __restrict__ kept,
-                              int32_t* __restrict__ offsets, int32_t* __restrict__ tile_expert,
-                              int32_t* __restrict__ stats, int32_t* __restrict__ row_slot) {
+__device__ void finish_layout(const int32_t* tot, int32_t* seg, int E, int ebase, int El, int T,
+                              int n_shared, int64_t C, int64_t rows_max, int align,
+                              int32_t sentinels, int32_t* __restrict__ counts,
+                              int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
+                              int32_t* __restrict__ tile_expert, int32_t* __restrict__ stats,
+                              int32_t* __restrict__ row_slot) {
   __shared__ unsigned long long drop_s;
+  __shared__ unsigned long long remote_s;
   __shared__ int32_t total_s;
-  if (threadIdx.x == 0) drop_s = 0;
+  if (threadIdx.x == 0) { drop_s = 0; remote_s = 0; }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int32_t run = tot[e];
     counts[e] = run;
+    if (e < ebase || e >= ebase + El) {
+      if (run) atomicAdd(&remote_s, (unsigned long long)run);
+      continue;
+    }
+    const int l = e - ebase;
     const int32_t k = (C >= 0 && run > C) ? (int32_t)C : run;
-    kept[e] = k;
+    kept[l] = k;
     if (run > k) atomicAdd(&drop_s, (unsigned long long)(run - k));
-    seg[e] = (k + align - 1) / align * align;
+    seg[l] = (k + align - 1) / align * align;
   }
   __syncthreads();
-  // exclusive scan of the padded sizes by warp 0 (E <= 512: 16 per lane)
+  // exclusive scan of the padded sizes by warp 0 (El <= 512: 16 per lane)
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    const int per = (E + 31) / 32;
-    const int e0 = lane * per, e1 = min(E, e0 + per);
+    const int per = (El + 31) / 32;
+    const int e0 = lane * per, e1 = min(El, e0 + per);
     int64_t local = 0;
     for (int e = e0; e < e1; ++e) local += seg[e];
     int64_t incl = local;
@@ -143,33 +154,34 @@ __device__ void finish_layout(const int32_t* tot, int32_t* seg, int E, int T, in
       const int64_t shared_rows = n_shared ? ((int64_t)T + align - 1) / align * align : 0;
       int64_t total = routed + shared_rows;
       if (total > rows_max) { set_dev_error(MOE_DEVERR_ROWS); total = rows_max; }
-      offsets[E] = (int32_t)routed;
-      offsets[E + 1] = (int32_t)total;
+      offsets[El] = (int32_t)routed;
+      offsets[El + 1] = (int32_t)total;
       stats[0] = (int32_t)drop_s;
-      stats[1] = sentinels;
+      stats[1] = sentinels + (int32_t)remote_s;
       stats[2] = (int32_t)total;
       stats[3] = (int32_t)(total / kRowTile);
-      seg[E] = (int32_t)routed;
+      seg[El] = (int32_t)routed;
       total_s = (int32_t)total;
     }
   }
   __syncthreads();
   const int64_t total = total_s;
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+  for (int e = threadIdx.x; e <= El; e += blockDim.x) {
     const int64_t beg = seg[e];
-    const int64_t end = (e < E) ? seg[e + 1] : total;
-    if (e < E) offsets[e] = (int32_t)beg;
+    const int64_t end = (e < El) ? seg[e + 1] : total;
+    if (e < El) offsets[e] = (int32_t)beg;
     for (int64_t r = beg; r < end && r < total; r += kRowTile) tile_expert[r / kRowTile] = e;
   }
   // rows that hold no routed slot (each expert's padding, the shared
   // expert's rows) get row_slot = -1; the rank pass fills the others
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  for (int e = warp; e < E; e += nw) {
-    const int32_t k = (C >= 0 && tot[e] > C) ? (int32_t)C : tot[e];
+  for (int e = warp; e < El; e += nw) {
+    const int32_t run = tot[ebase + e];
+    const int32_t k = (C >= 0 && run > C) ? (int32_t)C : run;
     const int64_t end = seg[e + 1] < total ? (int64_t)seg[e + 1] : total;
     for (int64_t r = seg[e] + k + lane; r < end; r += 32) row_slot[r] = -1;
   }
-  for (int64_t r = (int64_t)seg[E] + threadIdx.x; r < total; r += blockDim.x) row_slot[r] = -1;
+  for (int64_t r = (int64_t)seg[El] + threadIdx.x; r < total; r += blockDim.x) row_slot[r] = -1;
   __syncthreads();
 }
 
@@ -200,13 +212,13 @@ disp_hist_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ ma
 // bases), then the layout (counts, kept, offsets, tile map, stats).
 __global__ void __launch_bounds__(1024)
 disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ block_sent,
-                 int n_blocks, int E, int T, int n_shared, int64_t C,
+                 int n_blocks, int E, int ebase, int El, int T, int n_shared, int64_t C,
                  int64_t rows_max, int align, int32_t* __restrict__ counts,
                  int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
                  int32_t* __restrict__ tile_expert, int32_t* __restrict__ stats,
                  int32_t* __restrict__ row_slot) {
   pdl_begin();
-  extern __shared__ int32_t sh[];     // tot[E], seg[E + 1]
+  extern __shared__ int32_t sh[];     // tot[E], seg[El + 1]
   int32_t* tot = sh;
   int32_t* seg = sh + E;
   __shared__ int32_t sent_total;
@@ -226,8 +238,8 @@ disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ b
   for (int b = threadIdx.x; b < n_blocks; b += blockDim.x) ls += block_sent[b];
   if (ls) atomicAdd(&sent_total, ls);
   __syncthreads();
-  finish_layout(tot, seg, E, T, n_shared, C, rows_max, align, sent_total, counts, kept, offsets,
-                tile_expert, stats, row_slot);
+  finish_layout(tot, seg, E, ebase, El, T, n_shared, C, rows_max, align, sent_total, counts, kept,
+                offsets, tile_expert, stats, row_slot);
 }
 
 // Pass 3: stable rank of every slot inside its expert, capacity drop,
@@ -235,16 +247,16 @@ disp_scan_kernel(int32_t* __restrict__ block_hist, const int32_t* __restrict__ b
 // with the same expert inside a 32-slot group are ranked by lane.
 __global__ void __launch_bounds__(256)
 disp_rank_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ mask,
-                 int64_t n_slots, int E, int64_t C, int64_t rows_max,
+                 int64_t n_slots, int E, int ebase, int El, int64_t C, int64_t rows_max,
                  const int32_t* __restrict__ block_base,
                  const int32_t* __restrict__ offsets,
                  int32_t* __restrict__ slot_row, int32_t* __restrict__ row_slot) {
   pdl_begin();
-  extern __shared__ int32_t wh[];   // [kDispWarps][E] per-warp counters, then seg_off[E]
+  extern __shared__ int32_t wh[];   // [kDispWarps][E] per-warp counters, then seg_off[El]
   int32_t* seg_off = wh + kDispWarps * E;
   const int warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kDispWarps * E; i += blockDim.x) wh[i] = 0;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) seg_off[e] = offsets[e];
+  for (int e = threadIdx.x; e < El; e += blockDim.x) seg_off[e] = offsets[e];
   const int64_t j0 = (int64_t)blockIdx.x * kDispChunk + (int64_t)warp * kDispIters * 32;
   int ev[kDispIters];
   warp_load_slots(idx, mask, n_slots, E, j0, kDispIters, ev);
@@ -261,7 +273,7 @@ disp_rank_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ ma
     }
   }
   __syncthreads();
-  warp_rank(ev, j0, n_slots, C, rows_max, wh + warp * E, seg_off, slot_row, row_slot);
+  warp_rank(ev, j0, n_slots, C, rows_max, wh + warp * E, seg_off, ebase, El, slot_row, row_slot);
 }
 
 // Passes 1-3 in one block for up to kSmallSlots slots: 32 warps each own
@@ -269,13 +281,14 @@ disp_rank_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ ma
 // order gives the same stable ranks as the multi-block passes.
 __global__ void __launch_bounds__(1024)
 disp_small_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ mask,
-                  int64_t n_slots, int E, int T, int n_shared, int64_t C, int64_t rows_max,
+                  int64_t n_slots, int E, int ebase, int El, int T, int n_shared, int64_t C,
+                  int64_t rows_max,
                   int align, int32_t* __restrict__ counts, int32_t* __restrict__ kept,
                   int32_t* __restrict__ offsets, int32_t* __restrict__ tile_expert,
                   int32_t* __restrict__ stats, int32_t* __restrict__ slot_row,
                   int32_t* __restrict__ row_slot) {
   pdl_begin();
-  extern __shared__ int32_t wh[];   // [kSmallWarps][E] counters, tot[E], seg[E + 1]
+  extern __shared__ int32_t wh[];   // [kSmallWarps][E] counters, tot[E], seg[El + 1]
   int32_t* tot = wh + kSmallWarps * E;
   int32_t* seg = tot + E;
   __shared__ int32_t sent_total;
@@ -300,9 +313,9 @@ disp_small_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ m
     tot[e] = run;
   }
   __syncthreads();
-  finish_layout(tot, seg, E, T, n_shared, C, rows_max, align, sent_total, counts, kept, offsets,
-                tile_expert, stats, row_slot);
-  warp_rank(ev, j0, n_slots, C, rows_max, wh + warp * E, seg, slot_row, row_slot);
+  finish_layout(tot, seg, E, ebase, El, T, n_shared, C, rows_max, align, sent_total, counts, kept,
+                offsets, tile_expert, stats, row_slot);
+  warp_rank(ev, j0, n_slots, C, rows_max, wh + warp * E, seg, ebase, El, slot_row, row_slot);
 }
 
 // Pass 4: gather x rows into expert order; zero padding rows; shared rows.

@@ -19,6 +19,7 @@
 #include "expert_choice.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "router_tc.cuh"
 
 using namespace moe;
 
@@ -132,8 +133,23 @@ int validate(const moe_config_t* c) {
   // loss (its sequences live on one rank) or expert choice
   if (c->loss_tokens < 0 || (c->loss_tokens > 0 && c->loss_tokens < c->T)) return MOE_ERR_ARG;
   if (c->loss_tokens > 0 && (c->seq_len != 0 || c->expert_choice)) return MOE_ERR_ARG;
+  // expert shards: a range of the routed experts, on the tensor-core path,
+  // token choice, no shared expert
+  if (c->expert_base < 0 || c->n_local_experts < 0 ||
+      (int64_t)c->expert_base + c->n_local_experts > c->E)
+    return MOE_ERR_ARG;
+  if (c->expert_base > 0 && c->n_local_experts == 0) return MOE_ERR_ARG;
+  if (c->n_local_experts > 0 &&
+      (c->expert_choice || c->n_shared || c->seq_len || c->dtype != MOE_BF16 ||
+       c->gemm_impl != MOE_GEMM_AUTO ||
+       (c->D % 128) || (c->F % 128)))
+    return MOE_ERR_ARG;
   return MOE_OK;
 }
+
+// Routed experts this call's expert FFN holds (expert parallelism), and the first.
+int local_E(const moe_config_t* c) { return c->n_local_experts > 0 ? c->n_local_experts : c->E; }
+int expert_base(const moe_config_t* c) { return c->n_local_experts > 0 ? c->expert_base : 0; }
 
 // Token count the batch aux and z losses average over.
 int64_t loss_tokens_of(const moe_config_t* c) { return c->loss_tokens > 0 ? c->loss_tokens : c->T; }
@@ -166,6 +182,18 @@ int64_t capacity_of(const moe_config_t* c);
 // when the expert GEMMs do and E >= 8; below that the SIMT kernels are as
 // fast.  Ep = E rounded up to 64 (split width).
 bool router_tc(const moe_config_t* c) { return use_tc(c) && c->E >= 8; }
+// Token-choice routing inside the tensor-core logits kernel: up to 64
+// experts, no group limit, K in {1, 2, 4, 8} (MOE_ROUTER_FUSED=0: the
+// partial-logit GEMM and a separate routing kernel instead, for
+// cross-checks).
+bool router_fused_tc(const moe_config_t* c) {
+  static const bool on = [] {
+    const char* v = std::getenv("MOE_ROUTER_FUSED");
+    return !(v != nullptr && v[0] == '0');
+  }();
+  return on && router_tc(c) && !c->expert_choice && c->E <= 64 && c->n_groups == 1 &&
+         (c->K == 1 || c->K == 2 || c->K == 4 || c->K == 8);
+}
 int64_t router_ep(const moe_config_t* c) { return (c->E + 63) / 64 * 64; }
 
 // Row GEMMs run on CTA pairs (two SMs share each 256-row MMA) when experts
@@ -214,11 +242,12 @@ Layout layout_of(const moe_config_t* c) {
   Layout L{};
   L.C = capacity_of(c);
   L.n_slots = (int64_t)c->T * c->K;
+  const int64_t El = local_E(c);
   const int64_t kept_total = c->expert_choice ? (int64_t)c->E * ec_capacity(c)
                              : L.C < 0        ? L.n_slots
-                                              : std::min<int64_t>(L.n_slots, (int64_t)c->E * L.C);
+                                              : std::min<int64_t>(L.n_slots, El * L.C);
   const int64_t align = row_align(c);
-  const int64_t pad = (align - 1) * std::min<int64_t>(c->E, kept_total);
+  const int64_t pad = (align - 1) * std::min<int64_t>(El, kept_total);
   L.rows_max = round_up(kept_total + pad, align) + (c->n_shared ? round_up(c->T, align) : 0);
   if (L.rows_max == 0) L.rows_max = align;
   L.align = (int)align;
@@ -305,6 +334,22 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t n3, int64_t rows, int64_t 
                   dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { g_last_cuda_error = (int)cudaErrorInvalidValue; return MOE_ERR_CUDA; }
+  return MOE_OK;
+}
+
+// Three-way bf16 splits of W_r as a 3-D tensor [3][EP][D] (hi, mid, lo),
+// one box {64 columns, EP rows, 3 planes} per k block.
+int make_map_splits(CUtensorMap* m, const void* ptr, int64_t EP, int64_t D) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) { g_last_cuda_error = (int)cudaErrorNotSupported; return MOE_ERR_CUDA; }
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)EP, 3};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)(EP * D * 2)};
+  cuuint32_t box[3] = {64, (cuuint32_t)EP, 3};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) { g_last_cuda_error = (int)cudaErrorInvalidValue; return MOE_ERR_CUDA; }
   return MOE_OK;
 }
@@ -417,8 +462,8 @@ int run_tc(int bn, const char* name, const CUtensorMap& a, const CUtensorMap& b,
 int64_t row_tiles_estimate(const moe_config_t* c, const Layout& L) {
   const int64_t kept_total = c->expert_choice ? (int64_t)c->E * ec_capacity(c)
                              : L.C < 0        ? L.n_slots
-                                              : std::min<int64_t>(L.n_slots, (int64_t)c->E * L.C);
-  const int64_t rows = kept_total + 64 * std::min<int64_t>(c->E, kept_total);
+                                              : std::min<int64_t>(L.n_slots, (int64_t)local_E(c) * L.C);
+  const int64_t rows = kept_total + 64 * std::min<int64_t>(local_E(c), kept_total);
   return ceil_div(rows, kRowTile) + (c->n_shared ? ceil_div(c->T, kRowTile) : 0);
 }
 
@@ -489,6 +534,40 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
   RouteArgs a{c->T, c->E, c->K, c->score_fn, c->renorm, c->n_groups, c->topk_groups,
               c->group_score, c->route_scale, bias, logits, probs, lse, idx, w, ties};
   MOE_CK(cudaMemsetAsync(ties, 0, sizeof(int32_t), s));
+  if (router_fused_tc(c)) {
+    // logits on tensor cores (the three splits accumulated in one tensor-
+    // memory accumulator) and the routing in the same kernel's epilogue
+    const Layout L = layout_of(c);
+    const int EP = c->E <= 32 ? 32 : 64;
+    auto* wf = wsp<__nv_bfloat16>(ws, L.off_wf);
+    prof_begin(s);
+    MOE_CK((launch_k(split_w_kernel, grid_for((int64_t)EP * c->D / 32), 256, 0, s, w_r, c->E,
+                     EP, c->D, wf, (__nv_bfloat16*)nullptr)));
+    MOE_LAUNCHED(s, "router_split_w");
+    CUtensorMap mX, mW;
+    MOE_TRY(make_map(&mX, x, 1, c->T, c->D, 128, false));
+    MOE_TRY(make_map_splits(&mW, wf, EP, c->D));
+    const int grid = (int)std::min<int64_t>(num_sms(), ceil_div(c->T, 128));
+    auto go = [&](auto kern, size_t smem) -> int {
+      MOE_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      prof_begin(s);
+      MOE_CK((launch_k(kern, grid, rtc::kThreads, smem, s, mX, mW, a, off, c->D)));
+      MOE_LAUNCHED(s, "router_tc");
+      return MOE_OK;
+    };
+    auto by_k = [&](auto ep) -> int {
+      constexpr int P = decltype(ep)::value;
+      constexpr size_t sm = rtc::Smem<P>::kBytes;
+      switch (c->K) {
+        case 1: return go(rtc::router_tc_kernel<P, 1>, sm);
+        case 2: return go(rtc::router_tc_kernel<P, 2>, sm);
+        case 4: return go(rtc::router_tc_kernel<P, 4>, sm);
+        default: return go(rtc::router_tc_kernel<P, 8>, sm);
+      }
+    };
+    if (EP == 32) return by_k(std::integral_constant<int, 32>{});
+    return by_k(std::integral_constant<int, 64>{});
+  }
   if (router_tc(c)) {
     // logits parts = x . (W_hi | W_mid | W_lo)^T on tensor cores (dense GEMM,
     // fp32 out), then routing sums the parts
@@ -729,7 +808,7 @@ int group_rows(int64_t Kd, bool pair) {
 tc::Params rows_params(const moe_config_t* c, int Kd, int nN, const int32_t* tile_expert,
                        const int32_t* stats, bool pair = false) {
   tc::Params p{};
-  p.E = c->E; p.F = c->F; p.Kd = Kd; p.nN = nN; p.group_m = group_rows(Kd, pair);
+  p.E = local_E(c); p.F = c->F; p.Kd = Kd; p.nN = nN; p.group_m = group_rows(Kd, pair);
   p.tile_expert = tile_expert; p.stats = stats; p.T = c->T;
   return p;
 }
@@ -743,15 +822,15 @@ int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_id
                   const uint8_t* sentinel_mask, const void* x, int32_t* counts, int32_t* kept,
                   int32_t* offsets, int32_t* slot_row, int32_t* row_slot, int32_t* tile_expert,
                   int32_t* stats, void* x_perm, int32_t* bhist, int32_t* bsent, cudaStream_t s) {
-  const int E = c->E;
+  const int E = c->E, eb = expert_base(c), El = local_E(c);
   if (L.n_slots <= kSmallSlots) {
     const size_t smem = ((size_t)kSmallWarps * E + 2 * E + 1) * sizeof(int32_t);
     MOE_CK(cudaFuncSetAttribute(disp_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem));
     prof_begin(s);
     MOE_CK((launch_k(disp_small_kernel, 1, kSmallWarps * 32, smem, s, topk_idx, sentinel_mask,
-                     L.n_slots, E, c->T, c->n_shared, L.C, L.rows_max, L.align, counts, kept,
-                     offsets, tile_expert, stats, slot_row, row_slot)));
+                     L.n_slots, E, eb, El, c->T, c->n_shared, L.C, L.rows_max, L.align, counts,
+                     kept, offsets, tile_expert, stats, slot_row, row_slot)));
     MOE_LAUNCHED(s, "dispatch_small");
   } else {
     prof_begin(s);
@@ -760,13 +839,13 @@ int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_id
     MOE_LAUNCHED(s, "dispatch_hist");
     prof_begin(s);
     MOE_CK((launch_k(disp_scan_kernel, 1, 1024, (2 * E + 1) * sizeof(int32_t), s, bhist, bsent,
-                     L.n_disp_blocks, E, c->T, c->n_shared, L.C, L.rows_max, L.align, counts,
-                     kept, offsets, tile_expert, stats, row_slot)));
+                     L.n_disp_blocks, E, eb, El, c->T, c->n_shared, L.C, L.rows_max, L.align,
+                     counts, kept, offsets, tile_expert, stats, row_slot)));
     MOE_LAUNCHED(s, "dispatch_scan");
     prof_begin(s);
     MOE_CK((launch_k(disp_rank_kernel, L.n_disp_blocks, 256,
                      (size_t)(kDispWarps + 1) * E * sizeof(int32_t), s, topk_idx, sentinel_mask,
-                     L.n_slots, E, L.C, L.rows_max, bhist, offsets, slot_row, row_slot)));
+                     L.n_slots, E, eb, El, L.C, L.rows_max, bhist, offsets, slot_row, row_slot)));
     MOE_LAUNCHED(s, "dispatch_rank");
   }
   if (x_perm == nullptr) return MOE_OK;   // layout only: the GEMMs gather x rows
@@ -774,11 +853,11 @@ int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_id
   prof_begin(s);
   if (c->dtype == MOE_BF16)
     MOE_CK((launch_k(disp_gather_kernel<__nv_bfloat16>, grid, 256, 0, s,
-                     static_cast<const __nv_bfloat16*>(x), c->D, c->K, E, c->T, offsets, stats,
+                     static_cast<const __nv_bfloat16*>(x), c->D, c->K, El, c->T, offsets, stats,
                      row_slot, static_cast<__nv_bfloat16*>(x_perm))));
   else
     MOE_CK((launch_k(disp_gather_kernel<float>, grid, 256, 0, s, static_cast<const float*>(x),
-                     c->D, c->K, E, c->T, offsets, stats, row_slot,
+                     c->D, c->K, El, c->T, offsets, stats, row_slot,
                      static_cast<float*>(x_perm))));
   MOE_LAUNCHED(s, "dispatch_gather");
   return MOE_OK;
@@ -1092,7 +1171,7 @@ int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, co
                   const void* w_down_s, void* a13, void* h, void* o, cudaStream_t s,
                   const int32_t* slot_row = nullptr, const float* topk_w = nullptr,
                   void* y = nullptr) {
-  const int D = c->D, F = c->F, E = c->E;
+  const int D = c->D, F = c->F, E = local_E(c);
   const bool gather = x_perm == nullptr;
   CUtensorMap mA, mB, mBs;
   const int64_t mt = row_tiles_estimate(c, L);
@@ -1251,7 +1330,7 @@ int moe_combine(const moe_config_t* c, const void* o, const int32_t* slot_row,
       prof_begin(s);
       MOE_CK((launch_k(combine_bf16_kernel<decltype(kt)::value>, grid, 256, 0, s,
                        static_cast<const __nv_bfloat16*>(o), slot_row, topk_w, offsets,
-                       c->n_shared, c->T, c->D, c->E, static_cast<__nv_bfloat16*>(y))));
+                       c->n_shared, c->T, c->D, local_E(c), static_cast<__nv_bfloat16*>(y))));
       MOE_LAUNCHED(s, "combine");
       return MOE_OK;
     };
@@ -1264,10 +1343,10 @@ int moe_combine(const moe_config_t* c, const void* o, const int32_t* slot_row,
   if (c->dtype == MOE_BF16)
     MOE_CK((launch_k(combine_kernel<__nv_bfloat16>, grid, 256, 0, s,
         static_cast<const __nv_bfloat16*>(o), slot_row, topk_w, offsets, c->n_shared, c->T,
-        c->D, c->K, c->E, static_cast<__nv_bfloat16*>(y))));
+        c->D, c->K, local_E(c), static_cast<__nv_bfloat16*>(y))));
   else
     MOE_CK((launch_k(combine_kernel<float>, grid, 256, 0, s, static_cast<const float*>(o), slot_row, topk_w,
-                                               offsets, c->n_shared, c->T, c->D, c->K, c->E,
+                                               offsets, c->n_shared, c->T, c->D, c->K, local_E(c),
                                                static_cast<float*>(y))));
   MOE_LAUNCHED(s, "combine");
   return MOE_OK;
@@ -1291,6 +1370,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   if (c->n_shared && (!w13_s || !w_down_s || !dw13_s || !dw_down_s)) return MOE_ERR_ARG;
   const Layout L = layout_of(c);
   const int D = c->D, F = c->F, E = c->E, T = c->T, K = c->K;
+  const int El = local_E(c);   // routed experts of the expert GEMMs (E unless sharded)
   float* dg = wsp<float>(ws, L.off_dg);
   float* ds = wsp<float>(ws, L.off_ds);
   float* dwr_part = wsp<float>(ws, L.off_dwr);
@@ -1309,11 +1389,11 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     if (bf)
       MOE_CK((launch_k(bwd_rows_kernel<__nv_bfloat16>, grid, 256, 0, s,
           static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dy), topk_w,
-          row_slot, offsets, stats, K, E, T, D, dg, static_cast<__nv_bfloat16*>(dO))));
+          row_slot, offsets, stats, K, El, T, D, dg, static_cast<__nv_bfloat16*>(dO))));
     else
       MOE_CK((launch_k(bwd_rows_kernel<float>, grid, 256, 0, s,
           static_cast<const float*>(o), static_cast<const float*>(dy), topk_w, row_slot, offsets,
-          stats, K, E, T, D, dg, static_cast<float*>(dO))));
+          stats, K, El, T, D, dg, static_cast<float*>(dO))));
     MOE_LAUNCHED(s, "bwd_gate_grad_rows");
   }
   // The router gradient chain (2, 7) runs on side stream r, concurrently
@@ -1389,13 +1469,13 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   if (use_tc(c)) {
     CUtensorMap mA, mB, mBs;
     const int64_t mt = row_tiles_estimate(c, L);
-    const int groups = E + c->n_shared;
+    const int groups = El + c->n_shared;
     const bool pr = pair_rows(c);                 // CTA-pair row tiles
     const int64_t units = pr ? L.tiles_max / 2 : L.tiles_max;
     // 3. dgrad down + SwiGLU backward: dA13 = swiglu'(dO . w_down[e])
     const int bn3 = pick_bn(F, mt, false, F, pr);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 128, false));
-    MOE_TRY(make_map(&mB, w_down, E, D, F, 64, true));                 // dims {F, D, E}
+    MOE_TRY(make_map(&mB, w_down, El, D, F, 64, true));                // dims {F, D, El}
     MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, 64, true));
     {
       tc::Params p = rows_params(c, D, F / bn3, tile_expert, stats, pr);
@@ -1417,7 +1497,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     MOE_TRY(make_map(&mB, h, 1, L.rows_max, F, 64, false));
     {
       tc::Params p{};
-      p.E = E; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
+      p.E = El; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
       p.n_groups = groups; p.nMo = D / (pw4 ? 256 : 128); p.nNo = F / bn4; p.No = F;
       p.strideCE = (int64_t)D * F;
       p.out = static_cast<__nv_bfloat16*>(dw_down);
@@ -1435,7 +1515,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     // itself: dx[t] = dX_perm[row(t)] + ds_t . W_r, once ds is ready
     const int bn5 = pick_bn(D, mt, false, F, pr);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 128, false));
-    MOE_TRY(make_map(&mB, w13, E, 2 * F, D, 64, true));                  // dims {D, 2F, E}
+    MOE_TRY(make_map(&mB, w13, El, 2 * F, D, 64, true));                 // dims {D, 2F, El}
     MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, 64, true));
     {
       tc::Params p = rows_params(c, 2 * F, D / bn5, tile_expert, stats, pr);
@@ -1466,7 +1546,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     MOE_TRY(make_map(&mB, g6 ? x : x_perm, 1, g6 ? T : L.rows_max, D, 64, false));
     {
       tc::Params p{};
-      p.E = E; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
+      p.E = El; p.F = F; p.offsets = offsets; p.kept = kept; p.T = T;
       p.n_groups = groups; p.nMo = 2 * F / (pw6 ? 256 : 128); p.nNo = D / bn6; p.No = D;
       p.strideCE = (int64_t)2 * F * D;
       p.out = static_cast<__nv_bfloat16*>(dw13);
@@ -1612,7 +1692,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       prof_begin(s);
       MOE_CK((launch_k(dx_sum_kernel<decltype(kt)::value>, grid_for(T), 256, 0, s, R,
                        static_cast<const __nv_bfloat16*>(dXp), slot_row, offsets, c->n_shared,
-                       T, D, E, K, static_cast<__nv_bfloat16*>(dx))));
+                       T, D, El, K, static_cast<__nv_bfloat16*>(dx))));
       MOE_LAUNCHED(s, "dx_unpermute_sum");
       return MOE_OK;
     };

@@ -1,0 +1,327 @@
+// Router on tensor cores with the routing in the epilogue: fp32 logits
+// x . W_r^T, softmax / sigmoid scores, top-K with lower-index ties, gate
+// weights of variant A or B, LSE and the near-tie count, in one kernel.
+//
+// Follows "08 MoE" (STA324 notes) §8.2 (s = x W_r, TopK on the logits,
+// variant A = truncate, variant B = softmax over the selected logits) and
+// §8.6 (sigmoid affinities with a selection-only bias, weights from the raw
+// affinity); the "8-MoE" lecture notes (Switch Transformers: the router in
+// full precision).
+//
+// The fp32 product x . W_r^T (x bf16) runs as bf16 MMAs on three-way bf16
+// splits of W_r (hi, mid, lo: |w - hi - mid - lo| <= 2^-24 |w|), all three
+// accumulated into ONE fp32 accumulator in tensor memory: for every 16-wide
+// k step the MMA thread issues x.hi, x.mid, x.lo into the same columns, so
+// the accumulator holds the fp32-accurate logits and no partial-logit
+// tensor ever reaches global memory.  Each stage carries one 128 x 64 tile
+// of x and the three 64-column k blocks of the splits (one 3-D TMA box).
+//
+// Roles (192 threads, one CTA per SM, persistent over 128-token tiles):
+//   warp 0   TMA producer (x tile + split box per stage, STAGES-deep ring)
+//   warp 1   MMA issuer (M=128, N=EP, 12 MMAs per stage), double-buffered
+//            accumulator (2 x EP tensor-memory columns)
+//   warps 2-5 epilogue: one thread per token (its tensor-memory lane) reads
+//            the token's EP logits, routes it, and the warp writes its 32
+//            tokens' logits and probs rows as contiguous blocks through a
+//            shared staging tile; the accumulator is released as soon as
+//            it is read, so routing overlaps the next tile's main loop.
+// Every barrier wait is bounded (see tc::mbar_wait); on timeout the kernel
+// records MOE_DEVERR_TIMEOUT, drains its copies and MMAs and returns.
+#pragma once
+#include "gemm_tc.cuh"
+#include "router.cuh"
+
+namespace moe {
+namespace rtc {
+
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+
+template <int EP>
+struct Smem {
+  static constexpr int kA = 128 * 64 * 2;         // x tile of one k block
+  static constexpr int kB = 3 * EP * 128;         // hi | mid | lo k blocks of W_r
+  static constexpr int kStage = kA + kB;
+  static constexpr int STAGES = EP == 32 ? 6 : 4;
+  static constexpr int kBars = (2 * STAGES + 5) * 8;
+  static constexpr int kStgLd = EP + 1;           // staging row stride (floats)
+  static constexpr int kParOff = STAGES * kStage + kBars + 16;   // offset, bias [64] each
+  static constexpr int kStgOff = kParOff + 2 * 64 * 4;
+  static constexpr int kBytes = 1024 + kStgOff + kEpiWarps * 32 * kStgLd * 4;
+  static_assert(kBytes <= 232448, "shared memory per CTA");
+};
+
+// Writes rows [row0, row0 + nrows) of a [T, E] fp32 tensor from the warp's
+// staging tile (row r at stg + r * ld): the rows are contiguous in global
+// memory, so the warp stores them as one block (16-byte stores when E is a
+// multiple of 4).
+__device__ __forceinline__ void block_store_rows(float* __restrict__ g, int64_t row0, int nrows,
+                                                 int E, const float* stg, int ld, int lane) {
+  float* dst = g + row0 * E;
+  const int n = nrows * E;
+  if ((E & 3) == 0) {
+    for (int i = 4 * lane; i < n; i += 128) {
+      const int r = i / E, c = i - r * E;
+      const float* sp = stg + r * ld + c;
+      *reinterpret_cast<float4*>(dst + i) = make_float4(sp[0], sp[1], sp[2], sp[3]);
+    }
+  } else {
+    for (int i = lane; i < n; i += 32) {
+      const int r = i / E;
+      dst[i] = stg[r * ld + (i - r * E)];
+    }
+  }
+}
+
+// (v, e, s) into the descending list of N = K + 1 entries: strictly larger
+// values move ahead, so among equal values the one seen first (the lower
+// expert index) stays ahead.
+template <int N>
+__device__ __forceinline__ void topk_insert(float (&lu)[N], int (&le)[N], float (&ls)[N], float v,
+                                            int e, float s) {
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const bool gt = v > lu[j];
+    const float tv = lu[j], ts = ls[j];
+    const int te = le[j];
+    lu[j] = gt ? v : tv; le[j] = gt ? e : te; ls[j] = gt ? s : ts;
+    v = gt ? tv : v; e = gt ? te : e; s = gt ? ts : s;
+  }
+}
+
+template <int EP, int K>
+__global__ void __launch_bounds__(kThreads, 1)
+router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,
+                 const RouteArgs a, const float* __restrict__ offset, int D) {
+  using S = Smem<EP>;
+  constexpr int STAGES = S::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int abort_flag_s;
+  volatile int* abort_flag = &abort_flag_s;
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t bars = base + STAGES * S::kStage;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
+  auto accf_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
+  auto acce_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
+  const uint32_t done_bar = bars + 8u * (2 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * S::kStage + S::kBars);
+  float* off_s = reinterpret_cast<float*>(gbase + S::kParOff);
+  float* bias_s = off_s + 64;
+  constexpr uint32_t kCols = 2 * EP <= 64 ? 64u : 128u;   // two accumulators
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (a.T + 127) / 128;
+  const int nk = D / 64;
+  if (threadIdx.x == 0) {
+    abort_flag_s = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(full_bar(s), 1);
+      tc::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(accf_bar(b), 1);
+      tc::mbar_init(acce_bar(b), kEpiWarps);
+    }
+    tc::mbar_init(done_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {
+    __syncwarp();
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     tc::smem_u32(tmem_slot)),
+                 "r"(kCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_begin();   // the set-up above touched only this CTA's shared and tensor memory
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued_parity[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!tc::mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t sa = base + stage * S::kStage;
+          const uint32_t fb = full_bar(stage);
+          tc::mbar_expect_tx(fb, S::kStage);
+          issued_parity[stage] = (int)phase;
+          tc::tma_2d(sa, &mapX, fb, kb * 64, t * 128);
+          tc::tma_3d(sa + S::kA, &mapW, fb, kb * 64, 0, 0);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_parity[s] >= 0) tc::mbar_wait(full_bar(s), (uint32_t)issued_parity[s], abort_flag);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = tc::make_idesc(128, EP, false, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        if (!tc::mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag)) break;
+        tc::tc_fence_after();
+        const uint32_t dt = tmem + acc * EP;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!tc::mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t sa = base + stage * S::kStage;
+          const uint32_t sb = sa + S::kA;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = tc::sw128_desc(sa + ks * 32, 16, 1024);
+#pragma unroll
+            for (int sp = 0; sp < 3; ++sp) {
+              const uint64_t bd = tc::sw128_desc(sb + sp * EP * 128 + ks * 32, 16, 1024);
+              tc::umma(dt, ad, bd, idesc, (kb | ks | sp) != 0 ? 1u : 0u);
+            }
+          }
+          tc::umma_commit(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc::umma_commit(accf_bar(acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      tc::umma_commit(done_bar);
+      tc::mbar_wait(done_bar, 0, abort_flag);
+    }
+  } else {
+    // ---------------- epilogue: route one token per thread ----------------
+    const int E = a.E;
+    const int ew = warp - 2;
+    for (int e = ew * 32 + lane; e < 64; e += kEpiWarps * 32) {
+      off_s[e] = (offset != nullptr && e < E) ? offset[e] : 0.f;
+      bias_s[e] = (a.sel_bias != nullptr && e < E) ? a.sel_bias[e] : 0.f;
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory");   // epilogue warps only
+    const int q = warp & 3;                                  // tensor-memory lane quarter
+    float* stg = reinterpret_cast<float*>(gbase + S::kStgOff) + ew * 32 * S::kStgLd;
+    const float NEG = -INFINITY;
+    const bool sigm = a.score_fn != MOE_SOFTMAX;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+      bool ok = (lane == 0) ? tc::mbar_wait(accf_bar(acc), acc_phase, abort_flag) : true;
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      tc::tc_fence_after();
+      float s[EP];
+      {
+        uint32_t r[32];
+        const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + acc * EP;
+#pragma unroll
+        for (int c = 0; c < EP; c += 32) {
+          tc::tmem_ld32(tb + c, r);
+          tc::tmem_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(r[i]);
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(acce_bar(acc));   // accumulator free for tile t + 2
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+
+      const int64_t row0 = (int64_t)t * 128 + q * 32;
+      if (row0 >= a.T) continue;
+      const int nrows = (int)((a.T - row0) < 32 ? (a.T - row0) : 32);
+      const int64_t tok = row0 + lane;
+      const bool valid = lane < nrows;
+      // logits (+ offset), staged and stored as one block
+      float m = NEG;
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        if (e < E) {
+          s[e] += off_s[e];
+          stg[lane * S::kStgLd + e] = s[e];
+          m = fmaxf(m, s[e]);
+        }
+      }
+      __syncwarp();
+      block_store_rows(a.logits, row0, nrows, E, stg, S::kStgLd, lane);
+      __syncwarp();
+      // logsumexp, scores
+      float z = 0.f;
+#pragma unroll
+      for (int e = 0; e < EP; ++e)
+        if (e < E) z += expf(s[e] - m);
+      const float lse = m + logf(z);
+#pragma unroll
+      for (int e = 0; e < EP; ++e)
+        if (e < E)
+          stg[lane * S::kStgLd + e] = sigm ? 1.0f / (1.0f + expf(-s[e])) : expf(s[e] - m) / z;
+      __syncwarp();
+      block_store_rows(a.probs, row0, nrows, E, stg, S::kStgLd, lane);
+      // top-K (+1): selection score u = s (softmax) or sigmoid(s) + b
+      float lu[K + 1], ls[K + 1];
+      int le[K + 1];
+#pragma unroll
+      for (int j = 0; j <= K; ++j) { lu[j] = NEG; le[j] = 0x7fffffff; ls[j] = 0.f; }
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        if (e < E) {
+          const float u = sigm ? stg[lane * S::kStgLd + e] + bias_s[e] : s[e];
+          topk_insert<K + 1>(lu, le, ls, u, e, s[e]);
+        }
+      }
+      __syncwarp();   // the staging tile is reused by the next tile
+      float margin = INFINITY;
+#pragma unroll
+      for (int k = 1; k <= K; ++k)
+        if (lu[k] != NEG) margin = fminf(margin, lu[k - 1] - lu[k]);
+      const unsigned tie = __ballot_sync(0xffffffffu, valid && margin < kNearTie);
+      if (lane == 0 && tie != 0u) atomicAdd(a.near_ties, __popc(tie));
+      // gate weights
+      float g[K];
+      float denom = 0.f;
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        if (!sigm) g[k] = a.renorm ? expf(ls[k] - ls[0]) : expf(ls[k] - m) / z;
+        else g[k] = 1.0f / (1.0f + expf(-ls[k]));
+        denom += g[k];
+      }
+      if (a.renorm && sigm) denom += 1e-20f;
+      if (valid) {
+        a.lse[tok] = lse;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          const float w = (a.renorm ? g[k] / denom : g[k]) * a.route_scale;
+          a.topk_idx[tok * K + k] = le[k];
+          a.topk_w[tok * K + k] = w;
+        }
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 0) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols)
+                 : "memory");
+  }
+}
+
+}  // namespace rtc
+}  // namespace moe

@@ -11,6 +11,11 @@ and issues the entry points in order on the current stream:
             itself (no permuted copy of x; bf16 layers)
   backward: moe_backward (its three side streams owned by the layer)
 
+Expert shards (cfg.n_local_experts > 0, expert parallelism): the router and
+the losses cover all E experts, the expert FFN only experts [expert_base,
+expert_base + n_local_experts) (w13, w_down and their gradients hold those);
+y, dx, dw_r, dlogits and dg of the shards sum to the whole layer's.
+
 aux_group (a torch.distributed process group): the batch aux and z losses
 are scoped over all ranks of the group (equal per-rank token counts): the
 forward sums the ranks' expert counts and statistics (moe_aux_stats, then
@@ -43,14 +48,16 @@ class MoELayer:
         act = torch.bfloat16 if c.dtype == MOE_BF16 else torch.float32
         self.act_dtype = act
         T, D, E, K, F = c.T, c.D, c.E, c.K, c.F
+        El = c.n_local_experts or E          # experts of this call's expert FFN
+        self.n_local = El
         R = int(z.rows_max)
         f32, i32 = torch.float32, torch.int32
         e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
         self.logits, self.probs, self.lse = e((T, E), f32), e((T, E), f32), e((T,), f32)
         self.topk_idx, self.topk_w = e((T, K), i32), e((T, K), f32)
         self.near_ties = e((1,), i32)
-        self.counts, self.kept = e((E,), i32), e((E,), i32)
-        self.offsets = e((E + 2,), i32)
+        self.counts, self.kept = e((E,), i32), e((El,), i32)
+        self.offsets = e((El + 2,), i32)
         self.slot_row, self.row_slot = e((T * K,), i32), e((R,), i32)
         self.tile_expert, self.stats = e((int(z.tiles_max),), i32), e((4,), i32)
         self.x_perm = None if self.gather else e((R, D), act)
@@ -79,10 +86,11 @@ class MoELayer:
             return
         c, dev, act, f32 = self.cfg, self.device, self.act_dtype, torch.float32
         T, D, E, K, F = c.T, c.D, c.E, c.K, c.F
+        El = self.n_local
         e = lambda shape, dt: torch.empty(shape, dtype=dt, device=dev)
         self.dx = e((T, D), act)
         self.dw_r = e((E, D), f32)
-        self.dw13, self.dw_down = e((E, 2 * F, D), act), e((E, D, F), act)
+        self.dw13, self.dw_down = e((El, 2 * F, D), act), e((El, D, F), act)
         self.dw13_s = e((2 * F, D), act) if c.n_shared else None
         self.dw_down_s = e((D, F), act) if c.n_shared else None
         self.dg = e((T, K), f32)

@@ -38,8 +38,8 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_config_struct_layout_matches_header():
-    # 12 int32 fields, then float, int32, 3 floats, 4 int32 = 21 x 4 bytes
-    assert ctypes.sizeof(C.MoeConfig) == 21 * 4
+    # 12 int32 fields, then float, int32, 3 floats, 6 int32 = 23 x 4 bytes
+    assert ctypes.sizeof(C.MoeConfig) == 23 * 4
     assert ctypes.sizeof(C.MoeSizes) == 40
 
 
@@ -158,3 +158,19 @@ def test_global_loss_entry_points_validate_on_host(lib):
     dummy = ctypes.c_void_p(256)
     assert lib.moe_aux_stats(ctypes.byref(seq), dummy, dummy, dummy, dummy, None) == C.MOE_ERR_ARG
     assert lib.moe_set_backward_streams(None) == C.MOE_OK
+
+
+def test_shard_configs_refused_on_the_host(lib):
+    """Shards need the tensor-core path, token choice, no shared expert and
+    a range inside [0, E); refused before any launch."""
+    L = lib
+    out = C.MoeSizes()
+    ok = api.make_config(256, 128, 8, 2, 128, expert_base=4, n_local_experts=4)
+    assert L.moe_get_sizes(ctypes.byref(ok), ctypes.byref(out)) == C.MOE_OK
+    for bad in (dict(expert_base=6, n_local_experts=4), dict(expert_base=2),
+                dict(n_local_experts=4, n_shared=1), dict(n_local_experts=4, dtype="fp32"),
+                dict(n_local_experts=4, D=96)):
+        kw = dict(T=256, D=128, E=8, K=2, F=128)
+        kw.update(bad)
+        c = api.make_config(**kw)
+        assert L.moe_get_sizes(ctypes.byref(c), ctypes.byref(out)) == C.MOE_ERR_ARG, bad

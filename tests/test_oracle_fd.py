@@ -214,3 +214,61 @@ def test_given_selection_keeps_the_gate_formulas(name):
     else:
         exp = sel
     np.testing.assert_allclose(R3.g[t], exp * cfg.route_scale, rtol=1e-12)
+
+
+def shard_oracle(L, o, R, lo, hi):
+    """The oracle of one expert shard [lo, hi) under expert parallelism
+    ([HF48687]): the global routing R, slots of experts outside the shard
+    marked as sentinels (no row, no output, zero gate gradient), no aux or
+    z term (those are added once, from the global counts)."""
+    from dataclasses import replace
+    off = (R.idx < lo) | (R.idx >= hi)
+    m = off.reshape(-1) if L.sentinel_mask is None else (off.reshape(-1) | L.sentinel_mask.astype(bool))
+    Ls = replace(L, sentinel_mask=m)
+    os_ = replace(o, aux_alpha=0.0, z_lambda=0.0)
+    return Ls, os_, O.forward_routed(Ls, os_, R)
+
+
+@pytest.mark.parametrize("name", ["olmoe", "mix"])
+def test_expert_shards_sum_to_the_layer(name):
+    """Expert parallelism in the replicated-token form: every shard routes
+    all tokens over all experts and keeps only its own experts' slots (the
+    others are sentinels whose expert output is zero); y, dx, dW_r, dlogits
+    and dg summed over the shards, plus the aux and z terms taken once from
+    the global counts, equal the unsharded layer, and each expert's weight
+    gradient comes from its own shard.  Negative control ([HF48687]): with
+    the sentinel slots' outputs not zeroed (expert 0's output leaking in)
+    every shard's router gradient is wrong, and for variant A so is their
+    sum (under variant B the leak adds the same constant to all K slots of
+    a token, which the renormalisation cancels in the sum)."""
+    cfg = W.REDUCED[name].replace(T=160, D=64, F=48)
+    L = oracle_layer(cfg)
+    o = O.opts_of(cfg)
+    dy = W.make_input(cfg, "dy").double().numpy()
+    fw = O.forward(L, o)
+    bw = O.backward(L, o, fw, dy)
+    R, E, K = fw["R"], cfg.E, cfg.K
+    x, wr = O.f64(L.x), O.f64(L.w_r)
+    # the aux / z part of the router gradient, once, from the global counts
+    ds_aux = O.router_backward(R, np.zeros((cfg.T, K)), o, fw["Dp"].counts)
+    tot = {"y": 0.0, "dg": 0.0, "ds": ds_aux, "dx": ds_aux @ wr, "dw_r": ds_aux.T @ x}
+    leak = ds_aux
+    _, _, _, o0 = O.swiglu_forward(np.repeat(x, K, axis=0), L.w13(0), L.wd(0))
+    cuts = [0, E // 2, E]
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        Ls, os_, fs = shard_oracle(L, o, R, lo, hi)
+        bs = O.backward(Ls, os_, fs, dy)
+        tot["y"] = tot["y"] + fs["y"]
+        for k in ("dx", "dw_r", "ds", "dg"):
+            tot[k] = tot[k] + bs[k]
+        for e in range(lo, hi):
+            np.testing.assert_allclose(bs["dw13"][e], bw["dw13"][e], rtol=1e-10, atol=1e-14)
+            np.testing.assert_allclose(bs["dwd"][e], bw["dwd"][e], rtol=1e-10, atol=1e-14)
+        bl = O.backward(Ls, os_, fs, dy, sentinel_unmasked=o0)
+        assert np.linalg.norm(bl["ds"] - bs["ds"]) > 1e-3 * np.linalg.norm(bs["ds"])
+        leak = leak + bl["ds"]
+    for k, ref in (("y", fw["y"]), ("dx", bw["dx"]), ("dw_r", bw["dw_r"]), ("ds", bw["ds"]),
+                   ("dg", bw["dg"])):
+        np.testing.assert_allclose(tot[k], ref, rtol=1e-9, atol=1e-12, err_msg=k)
+    if not cfg.renorm:
+        assert np.linalg.norm(leak - bw["ds"]) > 1e-3 * np.linalg.norm(bw["ds"])
