@@ -349,9 +349,9 @@ int moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
 
 /*
  * moe_expert_ffn_gather — moe_expert_ffn without the permuted copy of x:
- * the gate/up GEMM loads its A rows straight from the token rows of x with
- * TMA tile::gather4 copies (four rows of 64 columns per copy), so x_perm is
- * never written or read.  Same method, one HBM round trip less: the pages
+ * the gate/up GEMM's producer warp copies its A rows straight from the
+ * token rows of x (16-byte cp.async copies into the swizzled layout a TMA
+ * box would produce), so x_perm is never written or read.  Same method, one HBM round trip less: the pages
  * group tokens into contiguous per-expert blocks before the grouped GEMM
  * ([8MOE] MoE 高效推理; [STA324 §8.8]); here the grouping happens inside the
  * GEMM's operand load.
@@ -428,9 +428,9 @@ int moe_combine(const moe_config_t* cfg, const void* o,
  * (dX_perm row + ds_t . W_r, rounded once; tokens without a row get the
  * router part alone) instead of a separate unpermute-sum.
  * x_perm may be NULL on the tensor-core path (bf16 layers): the gate/up
- * weight-gradient GEMM then gathers its x rows by row_slot with tile::gather4
- * copies, as moe_expert_ffn_gather does (MOE_ERR_ARG for NULL x_perm on the
- * SIMT path).
+ * weight-gradient GEMM then copies its x rows by row_slot in its producer
+ * warp (cp.async), as moe_expert_ffn_gather does (MOE_ERR_ARG for NULL
+ * x_perm on the SIMT path).
  * Inside the call, independent chains (the router gradient, the two
  * weight-gradient GEMMs) are forked onto three side streams and joined back
  * into `stream` before the call returns, so the results are ordered on

@@ -11,8 +11,9 @@
 //     every tile's expert comes from the dispatch's tile -> expert map, so
 //     experts without rows cost nothing;
 //   * warp 0: TMA producer (128B-swizzled boxes into a STAGES-deep ring);
-//     warp 1: one thread issues tcgen05.mma (M=128, N=BN, K=16) into a
-//     double-buffered fp32 accumulator in tensor memory; warps 2-9: epilogue
+//     warp 1: one thread issues tcgen05.mma (M=128, N=BN, K=16) into a ring
+//     of fp32 accumulators in tensor memory (two, or four when BN = 128);
+//     warps 2-9: epilogue
 //     (two warps per tensor-memory lane quarter; tcgen05.ld, fused SwiGLU /
 //     SwiGLU-backward, bf16 stores), overlapped with the next tile's main
 //     loop;
@@ -539,10 +540,14 @@ __device__ __forceinline__ Tile decode(int t, const Params& p, int rank, int n_m
 template <int BN, int STAGES, bool PAIR>
 struct Smem {
   static constexpr int BNC = PAIR ? BN / 2 : BN;
+  // accumulators in tensor memory (512 columns): four of BN = 128 columns,
+  // else two, so short tiles (few k blocks) run ahead of the epilogue
+  static constexpr int NACC = BN <= 128 ? 4 : 2;
   static constexpr int kA = BM * BK * 2;        // 16 KB
   static constexpr int kB = BNC * BK * 2;
   static constexpr int kStage = kA + kB;
-  static constexpr int kBars = (3 * STAGES + 5) * 8;   // full, empty, copies-done, acc, done
+  // full, empty, copies-done per stage; full, empty per accumulator; done
+  static constexpr int kBars = (3 * STAGES + 2 * NACC + 1) * 8;
   // token table of the gathering producer (128 rows)
   static constexpr int kTokOff = STAGES * kStage + kBars + 16;
   // epilogue staging tiles (one per epilogue warp), 128-byte aligned
@@ -552,10 +557,9 @@ struct Smem {
 };
 
 // GATHER: the row operand comes from the token rows of x (Params.row_slot)
-// by tile::gather4 copies issued by the whole producer warp: the A rows of a
-// ROWS tile (gate/up + SwiGLU), or the B rows of a WGRAD k block (gate/up
-// weight gradient).  mapA (ROWS) or mapB (WGRAD) is then x [T, D] with a
-// {64, 1} box.
+// by 16-byte cp.async copies issued by the whole producer warp: the A rows
+// of a ROWS tile (gate/up + SwiGLU), or the B rows of a WGRAD k block
+// (gate/up weight gradient); the other operand still arrives by TMA box.
 template <int BN, int STAGES, int MODE, bool A_MN, bool B_MN, int EPI, bool PAIR,
           bool GATHER = false>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -563,6 +567,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
             const __grid_constant__ CUtensorMap mapBs, const Params p, int total_hint) {
   using S = Smem<BN, STAGES, PAIR>;
   constexpr int BNC = S::BNC;
+  constexpr int NACC = S::NACC;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int abort_flag_s;
   volatile int* abort_flag = &abort_flag_s;
@@ -573,11 +578,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   auto full_bar = [&](int s) { return bars + 8u * s; };
   auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
   auto accf_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
-  auto acce_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
-  const uint32_t done_bar = bars + 8u * (2 * STAGES + 4);
+  auto acce_bar = [&](int b) { return bars + 8u * (2 * STAGES + NACC + b); };
+  const uint32_t done_bar = bars + 8u * (2 * STAGES + 2 * NACC);
   // gathered rows in a pair's second CTA: its lanes' cp.async copies arrive
   // here; warp 1 forwards each completed stage to the leader's full barrier
-  auto cpd_bar = [&](int s) { return bars + 8u * (2 * STAGES + 5 + s); };
+  auto cpd_bar = [&](int s) { return bars + 8u * (2 * STAGES + 2 * NACC + 1 + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * S::kStage + S::kBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -585,10 +590,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   const bool leader = rank == 0;
   const int unit = PAIR ? blockIdx.x >> 1 : blockIdx.x;   // this CTA's tile stream
   const int n_units = PAIR ? gridDim.x >> 1 : gridDim.x;
-  // tensor memory: two BN-column fp32 accumulators; tcgen05.alloc takes a
+  // tensor memory: NACC BN-column fp32 accumulators; tcgen05.alloc takes a
   // power of two between 32 and 512 columns
-  constexpr uint32_t kCols = (2 * BN <= 128) ? 128u : (2 * BN <= 256) ? 256u : 512u;
-  static_assert(2 * BN <= 512 && (kCols & (kCols - 1)) == 0, "tensor-memory columns");
+  constexpr uint32_t kCols = (NACC * BN <= 128) ? 128u : (NACC * BN <= 256) ? 256u : 512u;
+  static_assert(NACC * BN <= 512 && (kCols & (kCols - 1)) == 0, "tensor-memory columns");
   static_assert(!PAIR || (BNC % 64 == 0), "pair tiles hold whole 64-column B boxes");
 
   if (threadIdx.x == 0) {
@@ -602,7 +607,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       mbar_init(empty_bar(s), 1);
       mbar_init(cpd_bar(s), 32);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NACC; ++b) {
       mbar_init(accf_bar(b), 1);
       mbar_init(acce_bar(b), kEpiWarps * (PAIR ? 2 : 1));   // both CTAs' epilogues
     }
@@ -917,8 +922,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
         if (!ok) break;
         if constexpr (PAIR) umma_commit_pair_both(accf_bar(acc));
         else umma_commit(accf_bar(acc));
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
       }
       // all MMAs issued by this thread complete before teardown
       if constexpr (PAIR) umma_commit_pair_local(done_bar);
@@ -1131,8 +1135,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
         if (!PAIR || leader) mbar_arrive(acce_bar(acc));
         else mbar_arrive_remote(mapa(acce_bar(acc), 0));   // the leader's barrier
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
     }
   }
   tc_fence_before();

@@ -9,17 +9,19 @@
 // full precision).
 //
 // The fp32 product x . W_r^T (x bf16) runs as bf16 MMAs on three-way bf16
-// splits of W_r (hi, mid, lo: |w - hi - mid - lo| <= 2^-24 |w|), all three
-// accumulated into ONE fp32 accumulator in tensor memory: for every 16-wide
-// k step the MMA thread issues x.hi, x.mid, x.lo into the same columns, so
-// the accumulator holds the fp32-accurate logits and no partial-logit
-// tensor ever reaches global memory.  Each stage carries one 128 x 64 tile
-// of x and the three 64-column k blocks of the splits (one 3-D TMA box).
+// splits of W_r (hi, mid, lo: |w - hi - mid - lo| <= 2^-24 |w|).  The
+// splits are stacked along N: one MMA per 16-wide k step, N = 3 EP, gives
+// three fp32 accumulators in tensor memory (x.hi | x.mid | x.lo, each
+// accumulating products of its own magnitude), which the epilogue sums per
+// expert as (hi + mid) + lo: fp32-accurate logits without a partial-logit
+// tensor in global memory.  Each stage carries one 128 x 64 tile of x and
+// the three 64-column k blocks of the splits (one 3-D TMA box, which lands
+// as the 3 EP rows of one K-major B operand).
 //
 // Roles (192 threads, one CTA per SM, persistent over 128-token tiles):
 //   warp 0   TMA producer (x tile + split box per stage, STAGES-deep ring)
-//   warp 1   MMA issuer (M=128, N=EP, 12 MMAs per stage), double-buffered
-//            accumulator (2 x EP tensor-memory columns)
+//   warp 1   MMA issuer (M=128, N=3 EP, 4 MMAs per stage), double-buffered
+//            accumulators (2 x 3 EP tensor-memory columns)
 //   warps 2-5 epilogue: one thread per token (its tensor-memory lane) reads
 //            the token's EP logits, routes it, and the warp writes its 32
 //            tokens' logits and probs rows as contiguous blocks through a
@@ -110,7 +112,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * S::kStage + S::kBars);
   float* off_s = reinterpret_cast<float*>(gbase + S::kParOff);
   float* bias_s = off_s + 64;
-  constexpr uint32_t kCols = 2 * EP <= 64 ? 64u : 128u;   // two accumulators
+  constexpr int NA = 3 * EP;                                // one accumulator's columns
+  constexpr uint32_t kCols = 2 * NA <= 256 ? 256u : 512u;  // two accumulators
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = (a.T + 127) / 128;
@@ -170,7 +173,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = tc::make_idesc(128, EP, false, false);
+      constexpr uint32_t idesc = tc::make_idesc(128, NA, false, false);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -179,7 +182,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         if (!tc::mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag)) break;
         tc::tc_fence_after();
-        const uint32_t dt = tmem + acc * EP;
+        const uint32_t dt = tmem + acc * NA;
         for (int kb = 0; kb < nk; ++kb) {
           if (!tc::mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
           tc::tc_fence_after();
@@ -188,11 +191,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             const uint64_t ad = tc::sw128_desc(sa + ks * 32, 16, 1024);
-#pragma unroll
-            for (int sp = 0; sp < 3; ++sp) {
-              const uint64_t bd = tc::sw128_desc(sb + sp * EP * 128 + ks * 32, 16, 1024);
-              tc::umma(dt, ad, bd, idesc, (kb | ks | sp) != 0 ? 1u : 0u);
-            }
+            const uint64_t bd = tc::sw128_desc(sb + ks * 32, 16, 1024);
+            tc::umma(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
           }
           tc::umma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -227,14 +227,18 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
       tc::tc_fence_after();
       float s[EP];
       {
-        uint32_t r[32];
-        const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + acc * EP;
+        // logit = (x.hi + x.mid) + x.lo, per expert column
+        uint32_t r0[32], r1[32], r2[32];
+        const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + acc * NA;
 #pragma unroll
         for (int c = 0; c < EP; c += 32) {
-          tc::tmem_ld32(tb + c, r);
+          tc::tmem_ld32(tb + c, r0);
+          tc::tmem_ld32(tb + EP + c, r1);
+          tc::tmem_ld32(tb + 2 * EP + c, r2);
           tc::tmem_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(r[i]);
+          for (int i = 0; i < 32; ++i)
+            s[c + i] = (__uint_as_float(r0[i]) + __uint_as_float(r1[i])) + __uint_as_float(r2[i]);
         }
       }
       tc::tc_fence_before();
