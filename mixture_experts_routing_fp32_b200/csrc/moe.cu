@@ -20,6 +20,7 @@
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "router_tc.cuh"
+#include "bulk_rows.cuh"
 
 using namespace moe;
 
@@ -336,6 +337,16 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t n3, int64_t rows, int64_t 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) { g_last_cuda_error = (int)cudaErrorInvalidValue; return MOE_ERR_CUDA; }
   return MOE_OK;
+}
+
+// The dispatch's row gather on the bulk-copy engine (MOE_GATHER_BULK=0:
+// the warp-per-row copy kernel instead, for comparison).
+bool gather_bulk() {
+  static const bool on = [] {
+    const char* v = std::getenv("MOE_GATHER_BULK");
+    return !(v != nullptr && v[0] == '0');
+  }();
+  return on;
 }
 
 // Three-way bf16 splits of W_r as a 3-D tensor [3][EP][D] (hi, mid, lo),
@@ -849,6 +860,28 @@ int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_id
     MOE_LAUNCHED(s, "dispatch_rank");
   }
   if (x_perm == nullptr) return MOE_OK;   // layout only: the GEMMs gather x rows
+  if (c->dtype == MOE_BF16 && gather_bulk()) {
+    // whole rows on the bulk-copy engine: NB rows per buffer set
+    const uint32_t rbp = bulk::padded_row_bytes(c->D);
+    const int fit = (int)std::max<uint32_t>(1u, (uint32_t)bulk::kBufBytes / rbp);
+    auto go = [&](auto nb) -> int {
+      constexpr int NB = decltype(nb)::value;
+      const size_t smem = bulk::gather_smem(NB, c->D);
+      MOE_CK(cudaFuncSetAttribute(bulk::gather_kernel<NB>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      const int grid = (int)std::min<int64_t>((int64_t)bulk::kCtasPerSm * num_sms(), L.rows_max);
+      prof_begin(s);
+      MOE_CK((launch_k(bulk::gather_kernel<NB>, grid, 32, smem, s,
+                       static_cast<const __nv_bfloat16*>(x), c->D, c->K, El, c->T, offsets, stats,
+                       row_slot, static_cast<__nv_bfloat16*>(x_perm))));
+      MOE_LAUNCHED(s, "dispatch_gather");
+      return MOE_OK;
+    };
+    if (fit >= 8) return go(std::integral_constant<int, 8>{});
+    if (fit >= 4) return go(std::integral_constant<int, 4>{});
+    if (fit >= 2) return go(std::integral_constant<int, 2>{});
+    return go(std::integral_constant<int, 1>{});
+  }
   const int grid = grid_for(L.rows_max);
   prof_begin(s);
   if (c->dtype == MOE_BF16)

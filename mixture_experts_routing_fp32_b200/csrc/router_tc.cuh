@@ -22,11 +22,17 @@
 //   warp 0   TMA producer (x tile + split box per stage, STAGES-deep ring)
 //   warp 1   MMA issuer (M=128, N=3 EP, 4 MMAs per stage), double-buffered
 //            accumulators (2 x 3 EP tensor-memory columns)
-//   warps 2-5 epilogue: one thread per token (its tensor-memory lane) reads
-//            the token's EP logits, routes it, and the warp writes its 32
-//            tokens' logits and probs rows as contiguous blocks through a
-//            shared staging tile; the accumulator is released as soon as
-//            it is read, so routing overlaps the next tile's main loop.
+//   warps 2-9 epilogue, in two phases per tile:
+//            1. warps 2-5 (one per tensor-memory lane quarter) read their 32
+//               tokens' accumulators, sum the splits per expert, add the
+//               logit offset and write the logits into a shared tile
+//               [128 tokens x E]; the accumulator is released at once, so
+//               the next tile's main loop overlaps the routing;
+//            2. all eight warps route: warp w takes tokens 16w..16w+15,
+//               lane l the token 16w + (l & 15) and half (l >> 4) of the
+//               experts; partner lanes combine their max, sum and top-K
+//               lists by shuffles; each warp stores its 16 tokens' logits
+//               and probs rows as one contiguous block.
 // Every barrier wait is bounded (see tc::mbar_wait); on timeout the kernel
 // records MOE_DEVERR_TIMEOUT, drains its copies and MMAs and returns.
 #pragma once
@@ -36,7 +42,8 @@
 namespace moe {
 namespace rtc {
 
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;     // routing warps (the first four also read tensor memory)
+constexpr int kTmemWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 template <int EP>
@@ -49,7 +56,7 @@ struct Smem {
   static constexpr int kStgLd = EP + 1;           // staging row stride (floats)
   static constexpr int kParOff = STAGES * kStage + kBars + 16;   // offset, bias [64] each
   static constexpr int kStgOff = kParOff + 2 * 64 * 4;
-  static constexpr int kBytes = 1024 + kStgOff + kEpiWarps * 32 * kStgLd * 4;
+  static constexpr int kBytes = 1024 + kStgOff + 128 * kStgLd * 4;   // one [128 x EP] tile
   static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
@@ -75,15 +82,14 @@ __device__ __forceinline__ void block_store_rows(float* __restrict__ g, int64_t 
   }
 }
 
-// (v, e, s) into the descending list of N = K + 1 entries: strictly larger
-// values move ahead, so among equal values the one seen first (the lower
-// expert index) stays ahead.
+// (v, e, s) into the list of N = K + 1 entries kept in selection order:
+// larger score first, equal scores by lower expert index.
 template <int N>
 __device__ __forceinline__ void topk_insert(float (&lu)[N], int (&le)[N], float (&ls)[N], float v,
                                             int e, float s) {
 #pragma unroll
   for (int j = 0; j < N; ++j) {
-    const bool gt = v > lu[j];
+    const bool gt = v > lu[j] || (v == lu[j] && e < le[j]);
     const float tv = lu[j], ts = ls[j];
     const int te = le[j];
     lu[j] = gt ? v : tv; le[j] = gt ? e : te; ls[j] = gt ? s : ts;
@@ -99,6 +105,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
   constexpr int STAGES = S::STAGES;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int abort_flag_s;
+  __shared__ int epi_stop_s;   // written before, read after an epilogue barrier
   volatile int* abort_flag = &abort_flag_s;
   const uint32_t raw = tc::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -120,13 +127,14 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
   const int nk = D / 64;
   if (threadIdx.x == 0) {
     abort_flag_s = 0;
+    epi_stop_s = 0;
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(full_bar(s), 1);
       tc::mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(accf_bar(b), 1);
-      tc::mbar_init(acce_bar(b), kEpiWarps);
+      tc::mbar_init(acce_bar(b), kTmemWarps);
     }
     tc::mbar_init(done_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -206,115 +214,147 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
       tc::mbar_wait(done_bar, 0, abort_flag);
     }
   } else {
-    // ---------------- epilogue: route one token per thread ----------------
+    // ---------------- epilogue ----------------
+    constexpr int HE = EP / 2;                               // experts per lane
     const int E = a.E;
     const int ew = warp - 2;
     for (int e = ew * 32 + lane; e < 64; e += kEpiWarps * 32) {
       off_s[e] = (offset != nullptr && e < E) ? offset[e] : 0.f;
       bias_s[e] = (a.sel_bias != nullptr && e < E) ? a.sel_bias[e] : 0.f;
     }
-    asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory");   // epilogue warps only
-    const int q = warp & 3;                                  // tensor-memory lane quarter
-    float* stg = reinterpret_cast<float*>(gbase + S::kStgOff) + ew * 32 * S::kStgLd;
+    auto epi_sync = [] {   // the eight epilogue warps only
+      asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory");
+    };
+    epi_sync();
+    float* stg = reinterpret_cast<float*>(gbase + S::kStgOff);   // [128][kStgLd]
     const float NEG = -INFINITY;
     const bool sigm = a.score_fn != MOE_SOFTMAX;
+    const int half = lane >> 4;
+    const int rloc = ew * 16 + (lane & 15);                  // this lane's token in the tile
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-      bool ok = (lane == 0) ? tc::mbar_wait(accf_bar(acc), acc_phase, abort_flag) : true;
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      tc::tc_fence_after();
-      float s[EP];
-      {
-        // logit = (x.hi + x.mid) + x.lo, per expert column
-        uint32_t r0[32], r1[32], r2[32];
-        const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + acc * NA;
+      // phase 1: splits -> logits (+ offset) in the shared tile
+      bool ok = true;
+      if (ew < kTmemWarps) {
+        const int q = warp & 3;                              // tensor-memory lane quarter
+        ok = (lane == 0) ? tc::mbar_wait(accf_bar(acc), acc_phase, abort_flag) : true;
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (ok) {
+          tc::tc_fence_after();
+          uint32_t r0[32], r1[32], r2[32];
+          const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + acc * NA;
+          float* srow = stg + (q * 32 + lane) * S::kStgLd;
 #pragma unroll
-        for (int c = 0; c < EP; c += 32) {
-          tc::tmem_ld32(tb + c, r0);
-          tc::tmem_ld32(tb + EP + c, r1);
-          tc::tmem_ld32(tb + 2 * EP + c, r2);
-          tc::tmem_wait();
+          for (int c = 0; c < EP; c += 32) {
+            tc::tmem_ld32(tb + c, r0);
+            tc::tmem_ld32(tb + EP + c, r1);
+            tc::tmem_ld32(tb + 2 * EP + c, r2);
+            tc::tmem_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            s[c + i] = (__uint_as_float(r0[i]) + __uint_as_float(r1[i])) + __uint_as_float(r2[i]);
+            for (int i = 0; i < 32; ++i)
+              srow[c + i] = ((__uint_as_float(r0[i]) + __uint_as_float(r1[i])) +
+                             __uint_as_float(r2[i])) + off_s[c + i];
+          }
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(acce_bar(acc));   // accumulator free for tile t + 2
+        } else if (lane == 0) {
+          epi_stop_s = 1;   // a wait gave up: every epilogue warp leaves after the barrier
         }
       }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(acce_bar(acc));   // accumulator free for tile t + 2
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
-
-      const int64_t row0 = (int64_t)t * 128 + q * 32;
-      if (row0 >= a.T) continue;
-      const int nrows = (int)((a.T - row0) < 32 ? (a.T - row0) : 32);
-      const int64_t tok = row0 + lane;
-      const bool valid = lane < nrows;
-      // logits (+ offset), staged and stored as one block
-      float m = NEG;
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      epi_sync();
+      if (*reinterpret_cast<volatile int*>(&epi_stop_s)) break;   // same decision in all eight warps
+      // phase 2: route 16 tokens per warp, two lanes per token
+      const int64_t row0 = (int64_t)t * 128 + ew * 16;
+      if (row0 < a.T) {
+        const int nrows = (int)((a.T - row0) < 16 ? (a.T - row0) : 16);
+        const int64_t tok = (int64_t)t * 128 + rloc;
+        const bool valid = tok < a.T;
+        float* srow = stg + rloc * S::kStgLd;
+        block_store_rows(a.logits, row0, nrows, E, stg + ew * 16 * S::kStgLd, S::kStgLd, lane);
+        // this lane's experts: e = half * HE + j
+        float sv[HE], ex[HE];
+        float m = NEG;
 #pragma unroll
-      for (int e = 0; e < EP; ++e) {
-        if (e < E) {
-          s[e] += off_s[e];
-          stg[lane * S::kStgLd + e] = s[e];
-          m = fmaxf(m, s[e]);
+        for (int j = 0; j < HE; ++j) {
+          const int e = half * HE + j;
+          sv[j] = e < E ? srow[e] : NEG;
+          m = fmaxf(m, sv[j]);
         }
-      }
-      __syncwarp();
-      block_store_rows(a.logits, row0, nrows, E, stg, S::kStgLd, lane);
-      __syncwarp();
-      // logsumexp, scores
-      float z = 0.f;
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        float z = 0.f;
 #pragma unroll
-      for (int e = 0; e < EP; ++e)
-        if (e < E) z += expf(s[e] - m);
-      const float lse = m + logf(z);
-#pragma unroll
-      for (int e = 0; e < EP; ++e)
-        if (e < E)
-          stg[lane * S::kStgLd + e] = sigm ? 1.0f / (1.0f + expf(-s[e])) : expf(s[e] - m) / z;
-      __syncwarp();
-      block_store_rows(a.probs, row0, nrows, E, stg, S::kStgLd, lane);
-      // top-K (+1): selection score u = s (softmax) or sigmoid(s) + b
-      float lu[K + 1], ls[K + 1];
-      int le[K + 1];
-#pragma unroll
-      for (int j = 0; j <= K; ++j) { lu[j] = NEG; le[j] = 0x7fffffff; ls[j] = 0.f; }
-#pragma unroll
-      for (int e = 0; e < EP; ++e) {
-        if (e < E) {
-          const float u = sigm ? stg[lane * S::kStgLd + e] + bias_s[e] : s[e];
-          topk_insert<K + 1>(lu, le, ls, u, e, s[e]);
+        for (int j = 0; j < HE; ++j) {
+          ex[j] = half * HE + j < E ? __expf(sv[j] - m) : 0.f;
+          z += ex[j];
         }
-      }
-      __syncwarp();   // the staging tile is reused by the next tile
-      float margin = INFINITY;
+        z += __shfl_xor_sync(0xffffffffu, z, 16);
+        const float inv_z = 1.0f / z;
+        const float lse = m + logf(z);
+        __syncwarp();                                         // logits rows stored
+        // scores (softmax probs or sigmoid affinities) into the same rows
 #pragma unroll
-      for (int k = 1; k <= K; ++k)
-        if (lu[k] != NEG) margin = fminf(margin, lu[k - 1] - lu[k]);
-      const unsigned tie = __ballot_sync(0xffffffffu, valid && margin < kNearTie);
-      if (lane == 0 && tie != 0u) atomicAdd(a.near_ties, __popc(tie));
-      // gate weights
-      float g[K];
-      float denom = 0.f;
+        for (int j = 0; j < HE; ++j) {
+          const int e = half * HE + j;
+          if (e < E) {
+            ex[j] = sigm ? 1.0f / (1.0f + __expf(-sv[j])) : ex[j] * inv_z;
+            srow[e] = ex[j];
+          }
+        }
+        __syncwarp();
+        block_store_rows(a.probs, row0, nrows, E, stg + ew * 16 * S::kStgLd, S::kStgLd, lane);
+        // top-(K+1) of this lane's experts (selection score u = s, or
+        // sigmoid + bias), then merged with the partner lane's list
+        float lu[K + 1], ls[K + 1];
+        int le[K + 1];
 #pragma unroll
-      for (int k = 0; k < K; ++k) {
-        if (!sigm) g[k] = a.renorm ? expf(ls[k] - ls[0]) : expf(ls[k] - m) / z;
-        else g[k] = 1.0f / (1.0f + expf(-ls[k]));
-        denom += g[k];
-      }
-      if (a.renorm && sigm) denom += 1e-20f;
-      if (valid) {
-        a.lse[tok] = lse;
+        for (int k = 0; k <= K; ++k) { lu[k] = NEG; le[k] = 0x7fffffff; ls[k] = 0.f; }
+#pragma unroll
+        for (int j = 0; j < HE; ++j) {
+          const int e = half * HE + j;
+          if (e < E) topk_insert<K + 1>(lu, le, ls, sigm ? ex[j] + bias_s[e] : sv[j], e, sv[j]);
+        }
+        float pu[K + 1], ps[K + 1];
+        int pe[K + 1];
+#pragma unroll
+        for (int k = 0; k <= K; ++k) {
+          pu[k] = __shfl_xor_sync(0xffffffffu, lu[k], 16);
+          pe[k] = __shfl_xor_sync(0xffffffffu, le[k], 16);
+          ps[k] = __shfl_xor_sync(0xffffffffu, ls[k], 16);
+        }
+#pragma unroll
+        for (int k = 0; k <= K; ++k)
+          if (pu[k] != NEG) topk_insert<K + 1>(lu, le, ls, pu[k], pe[k], ps[k]);
+        float margin = INFINITY;
+#pragma unroll
+        for (int k = 1; k <= K; ++k)
+          if (lu[k] != NEG) margin = fminf(margin, lu[k - 1] - lu[k]);
+        const bool writer = valid && half == 0;
+        const unsigned tie = __ballot_sync(0xffffffffu, writer && margin < kNearTie);
+        if (lane == 0 && tie != 0u) atomicAdd(a.near_ties, __popc(tie));
+        // gate weights
+        float g[K];
+        float denom = 0.f;
 #pragma unroll
         for (int k = 0; k < K; ++k) {
-          const float w = (a.renorm ? g[k] / denom : g[k]) * a.route_scale;
-          a.topk_idx[tok * K + k] = le[k];
-          a.topk_w[tok * K + k] = w;
+          if (!sigm) g[k] = a.renorm ? __expf(ls[k] - ls[0]) : __expf(ls[k] - m) * inv_z;
+          else g[k] = 1.0f / (1.0f + __expf(-ls[k]));
+          denom += g[k];
+        }
+        if (a.renorm && sigm) denom += 1e-20f;
+        const float inv_d = 1.0f / denom;
+        if (writer) {
+          a.lse[tok] = lse;
+#pragma unroll
+          for (int k = 0; k < K; ++k) {
+            a.topk_idx[tok * K + k] = le[k];
+            a.topk_w[tok * K + k] = (a.renorm ? g[k] * inv_d : g[k]) * a.route_scale;
+          }
         }
       }
+      epi_sync();   // the shared tile is rewritten by the next tile's phase 1
     }
   }
   tc::tc_fence_before();

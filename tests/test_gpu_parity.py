@@ -109,6 +109,15 @@ def check_dispatch(cfg, layer, R, Dp=None):
     assert np.all(row_slot[:n_rows][pad_rows] == -1)
     if layer.x_perm is not None:
         assert np.all(host(layer.x_perm)[:n_rows][pad_rows] == 0)
+        # every gathered row is its token's row of x, bit for bit
+        dev = layer.x_perm.device
+        xg = W.make_input(cfg, "x", dev)
+        rt = torch.from_numpy(rows.astype(np.int64)).to(dev)
+        tt = torch.from_numpy((kept_slots // K).astype(np.int64)).to(dev)
+        assert torch.equal(layer.x_perm[rt], xg[tt])
+        if cfg.n_shared:
+            s0 = int(offsets[E])
+            assert torch.equal(layer.x_perm[s0:s0 + T], xg)
     assert np.array_equal(counts, Dg.counts)
     assert np.array_equal(kept, Dg.kept)
     assert int(stats[0]) == Dg.n_drop
