@@ -720,62 +720,72 @@ bias_update_kernel(const int32_t* __restrict__ counts, int E, float gamma,
   }
 }
 
-// bf16 dx for few experts (E <= 8) and a compile-time K: one warp per
-// token, dx_t = sum_e ds[t,e] w_r[e,:] + sum_k dX_perm[row(t,k)] (k
-// ascending) + the shared row; each lane 8 columns of a 256-column chunk,
-// every row load of a chunk in flight together.
+// dx for few experts (E <= 8, bf16): dx_t = sum_e ds[t,e] W_r[e,:] (e
+// ascending, fp32) + sum_{k kept} dX_perm[row(t,k),:] (k ascending) + the
+// shared row.  Block (c, g) owns the 256-column slice c (8 columns per
+// lane) and token group g: it stages that slice of W_r in shared memory
+// once, then each warp takes one token at a time (two in flight), so the
+// router term costs no global traffic beyond ds and every warp keeps few
+// registers (full occupancy: many row loads in flight per SM).
 template <int KT>
 __global__ void __launch_bounds__(256)
 dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
                 const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__ slot_row,
-                const int32_t* __restrict__ offsets, int n_shared, int Tn, int D, int E,
+                const int32_t* __restrict__ offsets, int n_shared, int Tn, int D, int E, int El,
                 __nv_bfloat16* __restrict__ dx) {
   pdl_begin();
   constexpr int kE = 8;
+  __shared__ __align__(16) float ws[kE][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t shared0 = n_shared ? (int64_t)offsets[E] : -1;
-  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < Tn; t += (int64_t)gridDim.x * 8) {
-    int32_t my_row = -1;
-    float my_ds = 0.f;
-    if (lane < KT) my_row = slot_row[t * KT + lane];
-    if (lane < E) my_ds = ds[t * E + lane];
-    int32_t rows[KT];
-    float dse[kE];
-#pragma unroll
-    for (int k = 0; k < KT; ++k) rows[k] = __shfl_sync(0xffffffffu, my_row, k);
-#pragma unroll
-    for (int e = 0; e < kE; ++e) dse[e] = __shfl_sync(0xffffffffu, my_ds, e);
-    const int64_t srow = n_shared ? shared0 + t : -1;
-    for (int d = lane * 8; d < D; d += 256) {
-      uint4 r[KT + 1];
-#pragma unroll
-      for (int k = 0; k <= KT; ++k) {
-        const int64_t row = k < KT ? (int64_t)rows[k] : srow;
-        r[k] = row >= 0 ? *reinterpret_cast<const uint4*>(dXp + row * D + d)
-                        : make_uint4(0, 0, 0, 0);
-      }
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int e = 0; e < kE; ++e) {
-        if (e < E) {
-          float w[8];
-          load8(w_r + (int64_t)e * D + d, w);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = fmaf(dse[e], w[i], acc[i]);
-        }
-      }
-#pragma unroll
-      for (int k = 0; k <= KT; ++k) {
-        if ((k < KT && rows[k] >= 0) || (k == KT && srow >= 0)) {
-          float v[8];
-          bf16x8_to_f32(r[k], v);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] += v[i];
-        }
-      }
-      store8(dx + t * D + d, acc);
-    }
+  const int c0 = blockIdx.x * 256;
+  for (int i = threadIdx.x; i < kE * 256; i += 256) {
+    const int e = i / 256, col = c0 + (i & 255);
+    ws[e][i & 255] = (e < E && col < D) ? w_r[(int64_t)e * D + col] : 0.f;
   }
+  __syncthreads();
+  const int d = c0 + lane * 8;
+  if (d >= D) return;                      // no barrier below
+  const int64_t shared0 = n_shared ? (int64_t)offsets[El] : -1;
+  const int64_t stride = (int64_t)gridDim.y * 8;
+  auto one = [&](int64_t t) {
+    const int32_t my_row = lane < KT ? slot_row[t * KT + lane] : -1;
+    const float my_ds = lane < E ? ds[t * E + lane] : 0.f;
+    uint4 r[KT + 1];
+#pragma unroll
+    for (int k = 0; k <= KT; ++k) {
+      const int64_t row = k < KT ? (int64_t)__shfl_sync(0xffffffffu, my_row, k)
+                                 : (n_shared ? shared0 + t : -1);
+      r[k] = row >= 0 ? *reinterpret_cast<const uint4*>(dXp + row * D + d)
+                      : make_uint4(0, 0, 0, 0);
+    }
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+      const float de = __shfl_sync(0xffffffffu, my_ds, e);
+      if (e < E) {
+        const float4 w0 = *reinterpret_cast<const float4*>(&ws[e][lane * 8]);
+        const float4 w1 = *reinterpret_cast<const float4*>(&ws[e][lane * 8 + 4]);
+        acc[0] = fmaf(de, w0.x, acc[0]); acc[1] = fmaf(de, w0.y, acc[1]);
+        acc[2] = fmaf(de, w0.z, acc[2]); acc[3] = fmaf(de, w0.w, acc[3]);
+        acc[4] = fmaf(de, w1.x, acc[4]); acc[5] = fmaf(de, w1.y, acc[5]);
+        acc[6] = fmaf(de, w1.z, acc[6]); acc[7] = fmaf(de, w1.w, acc[7]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k <= KT; ++k) {
+      float v[8];
+      bf16x8_to_f32(r[k], v);   // absent rows were loaded as zeros
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += v[i];
+    }
+    store8(dx + t * D + d, acc);
+  };
+  int64_t t = (int64_t)blockIdx.y * 8 + warp;
+  for (; t + stride < Tn; t += 2 * stride) {
+    one(t);
+    one(t + stride);
+  }
+  if (t < Tn) one(t);
 }
 
 // bf16 dx when the router part R = ds . W_r [T, D] fp32 comes from the

@@ -541,8 +541,10 @@ template <int BN, int STAGES, bool PAIR>
 struct Smem {
   static constexpr int BNC = PAIR ? BN / 2 : BN;
   // accumulators in tensor memory (512 columns): four of BN = 128 columns,
-  // else two, so short tiles (few k blocks) run ahead of the epilogue
-  static constexpr int NACC = BN <= 128 ? 4 : 2;
+  // two of 192 or 256, so short tiles (few k blocks) run ahead of the
+  // epilogue; one of BN = 512 (CTA pairs), which halves the operand bytes
+  // per MMA and leaves the epilogue unoverlapped
+  static constexpr int NACC = BN <= 128 ? 4 : BN <= 256 ? 2 : 1;
   static constexpr int kA = BM * BK * 2;        // 16 KB
   static constexpr int kB = BNC * BK * 2;
   static constexpr int kStage = kA + kB;
@@ -568,6 +570,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   using S = Smem<BN, STAGES, PAIR>;
   constexpr int BNC = S::BNC;
   constexpr int NACC = S::NACC;
+  // N of one MMA (at most 256) and MMAs per k step; the B rows of MMA block
+  // m sit at sb + m * BLK * 128 in each CTA (BLK rows per CTA and block)
+  constexpr int NBM = BN > 256 ? BN / 256 : 1;
+  constexpr int NMM = BN / NBM;
+  constexpr int BLK = PAIR ? NMM / 2 : NMM;
+  static_assert(BN <= 256 || (PAIR && !GATHER), "BN = 512 only on CTA pairs, box-loaded operands");
   extern __shared__ uint8_t smem_raw[];
   __shared__ int abort_flag_s;
   volatile int* abort_flag = &abort_flag_s;
@@ -816,23 +824,32 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
             const uint32_t lfb = mapa(fb, 0);           // the leader's full barrier
             if (MODE == MODE_ROWS) {
               tma_2d_pair(sa, &mapA, lfb, kb * BK, d.m0, pol_a);
-              if (EPI == EPI_SWIGLU) {
-                // this CTA holds the gate (rank 0) or the up (rank 1) half
-                tma_3d_pair(sb, mb, lfb, kb * BK, (rank ? p.F : 0) + d.n0, eb);
-              } else if (!B_MN) {
-                tma_3d_pair(sb, mb, lfb, kb * BK, d.n0 + rank * BNC, eb);
-              } else {
 #pragma unroll
-                for (int c = 0; c < BNC / 64; ++c)
-                  tma_3d_pair(sb + c * 8192, mb, lfb, d.n0 + rank * BNC + c * 64, kb * BK, eb);
+              for (int m = 0; m < NBM; ++m) {
+                const uint32_t sbm = sb + m * BLK * 128;
+                if (EPI == EPI_SWIGLU) {
+                  // this CTA holds the gate (rank 0) or the up (rank 1) rows
+                  // of MMA block m: j = n0 + m BLK ...
+                  tma_3d_pair(sbm, mb, lfb, kb * BK, (rank ? p.F : 0) + d.n0 + m * BLK, eb);
+                } else if (!B_MN) {
+                  tma_3d_pair(sbm, mb, lfb, kb * BK, d.n0 + m * NMM + rank * BLK, eb);
+                } else {
+#pragma unroll
+                  for (int c = 0; c < BLK / 64; ++c)
+                    tma_3d_pair(sbm + c * 8192, mb, lfb, d.n0 + m * NMM + rank * BLK + c * 64,
+                                kb * BK, eb);
+                }
               }
             } else {
               const int r = d.row0 + kb * BK;
               tma_2d_pair_nohint(sa, &mapA, lfb, d.m0, r);
               tma_2d_pair_nohint(sa + 8192, &mapA, lfb, d.m0 + 64, r);
 #pragma unroll
-              for (int c = 0; c < BNC / 64; ++c)
-                tma_2d_pair_nohint(sb + c * 8192, &mapB, lfb, d.n0 + rank * BNC + c * 64, r);
+              for (int m = 0; m < NBM; ++m)
+#pragma unroll
+                for (int c = 0; c < BLK / 64; ++c)
+                  tma_2d_pair_nohint(sb + m * BLK * 128 + c * 8192, &mapB, lfb,
+                                     d.n0 + m * NMM + rank * BLK + c * 64, r);
             }
           } else {
             if (MODE == MODE_ROWS) {
@@ -886,7 +903,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     }
     // ---------------- MMA issuer (the pair leader only) ----------------
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = make_idesc(PAIR ? 2 * BM : BM, BN, A_MN, B_MN);
+      constexpr uint32_t idesc = make_idesc(PAIR ? 2 * BM : BM, NMM, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -910,10 +927,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           for (int ks = 0; ks < BK / 16; ++ks) {
             const uint64_t ad = A_MN ? sw128_desc(sa + ks * 2048, 8192, 1024)
                                      : sw128_desc(sa + ks * 32, 16, 1024);
-            const uint64_t bd = B_MN ? sw128_desc(sb + ks * 2048, 8192, 1024)
-                                     : sw128_desc(sb + ks * 32, 16, 1024);
-            if constexpr (PAIR) umma_pair(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
-            else umma(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int m = 0; m < NBM; ++m) {
+              const uint32_t sbm = sb + m * BLK * 128;
+              const uint64_t bd = B_MN ? sw128_desc(sbm + ks * 2048, 8192, 1024)
+                                       : sw128_desc(sbm + ks * 32, 16, 1024);
+              if constexpr (PAIR) umma_pair(dt + m * NMM, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+              else umma(dt + m * NMM, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+            }
           }
           if constexpr (PAIR) umma_commit_pair_both(empty_bar(stage));
           else umma_commit(empty_bar(stage));
@@ -1072,14 +1093,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           staged_store32_tok(stg, v, p.tout + col0 + c, p.ld_out, my_tok, pol_out);
         }
       } else if constexpr (EPI == EPI_SWIGLU) {
+        // accumulator columns of MMA block m: gate j in [m JB, (m+1) JB) at
+        // [2 m JB, 2 m JB + JB), up for the same j at the next JB columns
+        constexpr int JB = BN / 2 < 128 ? BN / 2 : 128;
         __nv_bfloat16* a13 = p.out + row0 * p.ld_out + d.n0 + hh * HJ;
         __nv_bfloat16* hr = p.out2 + row0 * p.ld_out2 + d.n0 + hh * HJ;
 #pragma unroll
         for (int c = 0; c < HJ; c += 32) {
           uint32_t rg[32], ru[32];
           float ga[32], ub[32];
-          tmem_ld32(tbase + hh * HJ + c, rg);
-          tmem_ld32(tbase + BN / 2 + hh * HJ + c, ru);
+          const int jl = hh * HJ + c;
+          const int gc = (jl / JB) * 2 * JB + jl % JB;
+          tmem_ld32(tbase + gc, rg);
+          tmem_ld32(tbase + gc + JB, ru);
           tmem_wait();
           u2f32(rg, ga);
           u2f32(ru, ub);

@@ -9,6 +9,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <numeric>
 #include <type_traits>
 #include <utility>
 
@@ -20,7 +21,6 @@
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "router_tc.cuh"
-#include "bulk_rows.cuh"
 
 using namespace moe;
 
@@ -339,16 +339,6 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t n3, int64_t rows, int64_t 
   return MOE_OK;
 }
 
-// The dispatch's row gather on the bulk-copy engine (MOE_GATHER_BULK=0:
-// the warp-per-row copy kernel instead, for comparison).
-bool gather_bulk() {
-  static const bool on = [] {
-    const char* v = std::getenv("MOE_GATHER_BULK");
-    return !(v != nullptr && v[0] == '0');
-  }();
-  return on;
-}
-
 // Three-way bf16 splits of W_r as a 3-D tensor [3][EP][D] (hi, mid, lo),
 // one box {64 columns, EP rows, 3 planes} per k block.
 int make_map_splits(CUtensorMap* m, const void* ptr, int64_t EP, int64_t D) {
@@ -445,6 +435,11 @@ int run_tc(int bn, const char* name, const CUtensorMap& a, const CUtensorMap& b,
            cudaStream_t s) {
   if constexpr (PAIR) {
     // per CTA: A 16 KB + half of B per stage
+    if constexpr (!GATHER) {
+      if (bn == 512)
+        return launch_tc<512, 4, MODE, AMN, BMN, EPI, true, false>(name, a, b, bs, p, total_max,
+                                                                  total_hint, s);
+    }
     if (bn == 256)
       return launch_tc<256, 6, MODE, AMN, BMN, EPI, true, GATHER>(name, a, b, bs, p, total_max,
                                                                  total_hint, s);
@@ -478,20 +473,27 @@ int64_t row_tiles_estimate(const moe_config_t* c, const Layout& L) {
   return ceil_div(rows, kRowTile) + (c->n_shared ? ceil_div(c->T, kRowTile) : 0);
 }
 
-// Output tile width BN in {256, 192, 128} minimising the busiest SM's time,
-// waves x BN / efficiency(BN): a narrower tile loads the same 128-row A
-// tile for fewer columns, so it moves more bytes per FLOP and keeps the
-// tensor pipe less busy (measured: BN=128 about 0.8 of BN=256 per column).
-// Ties keep the wider tile.  SwiGLU tiles hold BN/2 gate and BN/2 up
-// columns of F.
-int pick_bn(int64_t N, int64_t mtiles, bool swiglu, int64_t F, bool pair = false) {
+// Output tile width BN in {512, 256, 192, 128} minimising the busiest SM's
+// time, waves x BN / efficiency(BN): a narrower tile loads the same A rows
+// for fewer columns, so it moves more bytes per FLOP and keeps the tensor
+// pipe less busy (measured: BN=128 about 0.8 of BN=256 per column; a
+// 256-row CTA pair with BN=256 is limited by operand delivery into the SM,
+// which BN=512 halves per MMA).  BN=512 runs on CTA pairs with one
+// accumulator, so its epilogue is not overlapped: it is offered only for
+// tiles of at least kMinKb512 k blocks (nk; 0 = unknown).  Ties keep the
+// wider tile.  SwiGLU tiles hold BN/2 gate and BN/2 up columns of F.
+constexpr int64_t kMinKb512 = 48;
+bool bn512_enabled();
+int pick_bn(int64_t N, int64_t mtiles, bool swiglu, int64_t F, bool pair = false,
+            int64_t nk = 0) {
   const int64_t sms = pair ? num_sms() / 2 : num_sms();
   if (pair) mtiles = ceil_div(mtiles, 2);
   int best = 0;
   int64_t best_cost = INT64_MAX;
-  for (int bn : {256, 192, 128}) {
+  for (int bn : {512, 256, 192, 128}) {
     if (pair && bn == 192) continue;
-    const int64_t eff_pct = bn == 256 ? 100 : bn == 192 ? 95 : 80;
+    if (bn == 512 && !(pair && nk >= kMinKb512 && bn512_enabled())) continue;
+    const int64_t eff_pct = bn == 512 ? 125 : bn == 256 ? 100 : bn == 192 ? 95 : 80;
     int64_t nt;
     if (swiglu) {
       if (bn == 192 || F % (bn / 2)) continue;
@@ -808,6 +810,15 @@ int fork_join(cudaEvent_t ev, cudaStream_t from, cudaStream_t to) {
   return MOE_OK;
 }
 
+// 512-wide CTA-pair tiles (MOE_BN512=0 keeps BN <= 256, for comparison).
+bool bn512_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("MOE_BN512");
+    return !(v != nullptr && v[0] == '0');
+  }();
+  return on;
+}
+
 // Row tiles per rasterisation group: as many 128-row A tiles of depth Kd as
 // fit in about 48 MiB of L2, so they stay resident while the group sweeps
 // the weight column slices.
@@ -860,28 +871,6 @@ int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_id
     MOE_LAUNCHED(s, "dispatch_rank");
   }
   if (x_perm == nullptr) return MOE_OK;   // layout only: the GEMMs gather x rows
-  if (c->dtype == MOE_BF16 && gather_bulk()) {
-    // whole rows on the bulk-copy engine: NB rows per buffer set
-    const uint32_t rbp = bulk::padded_row_bytes(c->D);
-    const int fit = (int)std::max<uint32_t>(1u, (uint32_t)bulk::kBufBytes / rbp);
-    auto go = [&](auto nb) -> int {
-      constexpr int NB = decltype(nb)::value;
-      const size_t smem = bulk::gather_smem(NB, c->D);
-      MOE_CK(cudaFuncSetAttribute(bulk::gather_kernel<NB>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-      const int grid = (int)std::min<int64_t>((int64_t)bulk::kCtasPerSm * num_sms(), L.rows_max);
-      prof_begin(s);
-      MOE_CK((launch_k(bulk::gather_kernel<NB>, grid, 32, smem, s,
-                       static_cast<const __nv_bfloat16*>(x), c->D, c->K, El, c->T, offsets, stats,
-                       row_slot, static_cast<__nv_bfloat16*>(x_perm))));
-      MOE_LAUNCHED(s, "dispatch_gather");
-      return MOE_OK;
-    };
-    if (fit >= 8) return go(std::integral_constant<int, 8>{});
-    if (fit >= 4) return go(std::integral_constant<int, 4>{});
-    if (fit >= 2) return go(std::integral_constant<int, 2>{});
-    return go(std::integral_constant<int, 1>{});
-  }
   const int grid = grid_for(L.rows_max);
   prof_begin(s);
   if (c->dtype == MOE_BF16)
@@ -1212,10 +1201,12 @@ int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, co
   const int64_t units = pr ? L.tiles_max / 2 : L.tiles_max;
   // gate/up + SwiGLU: A = x_perm [rows, D] (or rows of x [T, D] copied by
   // the GEMM's producer warp: mapA unused); B = w13 [E, 2F, D] K-major
-  const int bn1 = pick_bn(2 * F, mt, true, F, pr);
+  const int bn1 = pick_bn(2 * F, mt, true, F, pr, D / 64);
   MOE_TRY(make_map(&mA, gather ? x : x_perm, 1, gather ? c->T : L.rows_max, D, 128, false));
-  MOE_TRY(make_map(&mB, w13, E, 2 * F, D, bn1 / 2, true));
-  MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, bn1 / 2, true));
+  // B boxes: the gate / up rows of one MMA block (at most 128 per CTA)
+  const uint32_t box1 = (uint32_t)std::min(bn1 / 2, 128);
+  MOE_TRY(make_map(&mB, w13, E, 2 * F, D, box1, true));
+  MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, box1, true));
   tc::Params p = rows_params(c, D, F / (bn1 / 2), tile_expert, stats, pr);
   p.out = static_cast<__nv_bfloat16*>(a13); p.ld_out = 2 * F;
   p.out2 = static_cast<__nv_bfloat16*>(h); p.ld_out2 = F;
@@ -1234,8 +1225,8 @@ int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, co
     MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
   // down: A = h [rows, F]; B = w_down [E, D, F] K-major (a pair CTA loads
   // half of the BN rows)
-  const int bn2 = pick_bn(D, mt, false, F, pr);
-  const uint32_t box2 = pr ? bn2 / 2 : bn2;
+  const int bn2 = pick_bn(D, mt, false, F, pr, F / 64);
+  const uint32_t box2 = pr ? (uint32_t)std::min(bn2 / 2, 128) : (uint32_t)bn2;
   MOE_TRY(make_map(&mA, h, 1, L.rows_max, F, 128, false));
   MOE_TRY(make_map(&mB, w_down, E, D, F, box2, true));
   MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, box2, true));
@@ -1412,7 +1403,10 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   void* dXp = wsp<void>(ws, L.off_dX);
   void* dH = wsp<void>(ws, L.off_dH);
   const bool bf = c->dtype == MOE_BF16;
-  const bool rtc = router_tc(c);
+  // the router's backward products (dW_r, the router part of dx) on tensor
+  // cores from E > 8 (and for expert choice); with up to 8 experts CUDA
+  // cores form them next to the data they are added to
+  const bool rtc = router_tc(c) && (E > 8 || c->expert_choice);
   const bool dx1 = token_epilogues(c) && !rtc;   // dx from the dgrad gate/up epilogue
 
   // 1. per row: gate gradient dg = <o, dy>, and dO = g * dy
@@ -1506,7 +1500,9 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     const bool pr = pair_rows(c);                 // CTA-pair row tiles
     const int64_t units = pr ? L.tiles_max / 2 : L.tiles_max;
     // 3. dgrad down + SwiGLU backward: dA13 = swiglu'(dO . w_down[e])
-    const int bn3 = pick_bn(F, mt, false, F, pr);
+    const int bn3 = pick_bn(F, mt, false, F, pr, D / 64);
+    // k blocks of an average weight-gradient tile (the group's rows)
+    const int64_t wg_kb = ceil_div(row_tiles_estimate(c, L) * kRowTile, (int64_t)groups * 64);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 128, false));
     MOE_TRY(make_map(&mB, w_down, El, D, F, 64, true));                // dims {F, D, El}
     MOE_TRY(make_map(&mBs, c->n_shared ? w_down_s : w_down, 1, D, F, 64, true));
@@ -1525,7 +1521,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     // 4. wgrad down: dW_down[e] = dO^T h over the expert's rows (CTA pairs
     // split the 256-row output tiles)
     const bool pw4 = (D % 256) == 0;
-    const int bn4 = pick_bn(F, (int64_t)groups * (D / 128), false, F, pw4);
+    const int bn4 = pick_bn(F, (int64_t)groups * (D / 128), false, F, pw4, wg_kb);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 64, false));
     MOE_TRY(make_map(&mB, h, 1, L.rows_max, F, 64, false));
     {
@@ -1546,7 +1542,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     // 5. dgrad gate/up: dX_perm = dA13 . w13[e]; with one slot per token
     // (no shared expert, CUDA-core router term) the epilogue writes dx
     // itself: dx[t] = dX_perm[row(t)] + ds_t . W_r, once ds is ready
-    const int bn5 = pick_bn(D, mt, false, F, pr);
+    const int bn5 = pick_bn(D, mt, false, F, pr, 2 * F / 64);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 128, false));
     MOE_TRY(make_map(&mB, w13, El, 2 * F, D, 64, true));                 // dims {D, 2F, El}
     MOE_TRY(make_map(&mBs, c->n_shared ? w13_s : w13, 1, 2 * F, D, 64, true));
@@ -1574,7 +1570,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     // producer warp copies the B rows from x by row_slot; mapB unused)
     const bool pw6 = ((2 * F) % 256) == 0;
     const bool g6 = x_perm == nullptr;
-    const int bn6 = pick_bn(D, (int64_t)groups * (2 * F / 128), false, F, pw6);
+    const int bn6 = pick_bn(D, (int64_t)groups * (2 * F / 128), false, F, pw6, wg_kb);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 64, false));
     MOE_TRY(make_map(&mB, g6 ? x : x_perm, 1, g6 ? T : L.rows_max, D, 64, false));
     {
@@ -1735,11 +1731,17 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     else if (K == 8) MOE_TRY(go(std::integral_constant<int, 8>{}));
     else MOE_TRY(go(std::integral_constant<int, 0>{}));
   } else if (bf && E <= 8 && (K == 1 || K == 2 || K == 4 || K == 8)) {
+    // blocks (slice c, token group g): the W_r slice in shared memory, one
+    // token per warp at a time
+    const int nch = (int)ceil_div(D, 256);
+    const int groups = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(T, 8),
+                                                                   ceil_div((int64_t)num_sms() * 8, nch)));
     auto go = [&](auto kt) -> int {
+      constexpr int KT = decltype(kt)::value;
       prof_begin(s);
-      MOE_CK((launch_k(dx_small_kernel<decltype(kt)::value>, grid_for(T), 256, 0, s, ds, w_r,
-                       static_cast<const __nv_bfloat16*>(dXp), slot_row, offsets, c->n_shared,
-                       T, D, E, static_cast<__nv_bfloat16*>(dx))));
+      MOE_CK((launch_k(dx_small_kernel<KT>, dim3((unsigned)nch, (unsigned)groups), 256, 0, s, ds,
+                       w_r, static_cast<const __nv_bfloat16*>(dXp), slot_row, offsets,
+                       c->n_shared, T, D, E, El, static_cast<__nv_bfloat16*>(dx))));
       MOE_LAUNCHED(s, "dx_unpermute_router");
       return MOE_OK;
     };

@@ -125,6 +125,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = (a.T + 127) / 128;
   const int nk = D / 64;
+  // Tiles start their k loop at different k blocks, so the CTAs running at
+  // the same time do not all load the same W_r block from L2 at once; the
+  // accumulation order is fixed by the tile index (deterministic).
+  auto rot_of = [&](int t) { return (int)(((int64_t)t * 5) % nk); };
   if (threadIdx.x == 0) {
     abort_flag_s = 0;
     epi_stop_s = 0;
@@ -164,7 +168,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
       for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        for (int kb = 0; kb < nk; ++kb) {
+        const int rot = rot_of(t);
+        for (int i = 0; i < nk; ++i) {
+          const int kb = i + rot < nk ? i + rot : i + rot - nk;
           if (!tc::mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t sa = base + stage * S::kStage;
           const uint32_t fb = full_bar(stage);
@@ -191,7 +197,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
         if (!tc::mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag)) break;
         tc::tc_fence_after();
         const uint32_t dt = tmem + acc * NA;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < nk; ++kb) {   // k blocks in the producer's (rotated) order
           if (!tc::mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
           tc::tc_fence_after();
           const uint32_t sa = base + stage * S::kStage;
@@ -274,48 +280,41 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
         const bool valid = tok < a.T;
         float* srow = stg + rloc * S::kStgLd;
         block_store_rows(a.logits, row0, nrows, E, stg + ew * 16 * S::kStgLd, S::kStgLd, lane);
-        // this lane's experts: e = half * HE + j
-        float sv[HE], ex[HE];
+        // this lane's experts e = half * HE + j, read from the shared tile in
+        // rolled loops (the code stays small: it runs once per tile)
+        const int e0 = half * HE;
+        const int e1 = min(E, e0 + HE);
         float m = NEG;
-#pragma unroll
-        for (int j = 0; j < HE; ++j) {
-          const int e = half * HE + j;
-          sv[j] = e < E ? srow[e] : NEG;
-          m = fmaxf(m, sv[j]);
-        }
+#pragma unroll 4
+        for (int e = e0; e < e1; ++e) m = fmaxf(m, srow[e]);
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-        float z = 0.f;
+        // top-(K+1) of this lane's experts (selection score u = s, or
+        // sigmoid + bias), before the row is overwritten with the scores
+        float lu[K + 1], ls[K + 1];
+        int le[K + 1];
 #pragma unroll
-        for (int j = 0; j < HE; ++j) {
-          ex[j] = half * HE + j < E ? __expf(sv[j] - m) : 0.f;
-          z += ex[j];
+        for (int k = 0; k <= K; ++k) { lu[k] = NEG; le[k] = 0x7fffffff; ls[k] = 0.f; }
+        float z = 0.f;
+#pragma unroll 2
+        for (int e = e0; e < e1; ++e) {
+          const float sv = srow[e];
+          z += __expf(sv - m);
+          const float u = sigm ? 1.0f / (1.0f + __expf(-sv)) + bias_s[e] : sv;
+          if (u > lu[K]) topk_insert<K + 1>(lu, le, ls, u, e, sv);
         }
         z += __shfl_xor_sync(0xffffffffu, z, 16);
         const float inv_z = 1.0f / z;
         const float lse = m + logf(z);
         __syncwarp();                                         // logits rows stored
         // scores (softmax probs or sigmoid affinities) into the same rows
-#pragma unroll
-        for (int j = 0; j < HE; ++j) {
-          const int e = half * HE + j;
-          if (e < E) {
-            ex[j] = sigm ? 1.0f / (1.0f + __expf(-sv[j])) : ex[j] * inv_z;
-            srow[e] = ex[j];
-          }
+#pragma unroll 4
+        for (int e = e0; e < e1; ++e) {
+          const float sv = srow[e];
+          srow[e] = sigm ? 1.0f / (1.0f + __expf(-sv)) : __expf(sv - m) * inv_z;
         }
         __syncwarp();
         block_store_rows(a.probs, row0, nrows, E, stg + ew * 16 * S::kStgLd, S::kStgLd, lane);
-        // top-(K+1) of this lane's experts (selection score u = s, or
-        // sigmoid + bias), then merged with the partner lane's list
-        float lu[K + 1], ls[K + 1];
-        int le[K + 1];
-#pragma unroll
-        for (int k = 0; k <= K; ++k) { lu[k] = NEG; le[k] = 0x7fffffff; ls[k] = 0.f; }
-#pragma unroll
-        for (int j = 0; j < HE; ++j) {
-          const int e = half * HE + j;
-          if (e < E) topk_insert<K + 1>(lu, le, ls, sigm ? ex[j] + bias_s[e] : sv[j], e, sv[j]);
-        }
+        // merge with the partner lane's list
         float pu[K + 1], ps[K + 1];
         int pe[K + 1];
 #pragma unroll
