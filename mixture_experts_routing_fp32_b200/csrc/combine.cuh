@@ -154,6 +154,69 @@ combine_bf16_kernel(const __nv_bfloat16* __restrict__ o, const int32_t* __restri
   }
 }
 
+// bf16 combine for K <= 2: as combine_bf16_kernel, with four 256-column
+// chunks per step (more row loads in flight per warp for few rows per
+// token).  Same fixed k order and fp32 accumulation.
+template <int KT>
+__global__ void __launch_bounds__(256, 2)
+combine_bf16_wide_kernel(const __nv_bfloat16* __restrict__ o, const int32_t* __restrict__ slot_row,
+                    const float* __restrict__ topk_w, const int32_t* __restrict__ offsets,
+                    int n_shared, int Tn, int D, int E, __nv_bfloat16* __restrict__ y) {
+  pdl_begin();
+  constexpr int NC = 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t shared0 = n_shared ? (int64_t)offsets[E] : -1;
+  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < Tn; t += (int64_t)gridDim.x * 8) {
+    int32_t my_row = -1;
+    float my_g = 0.f;
+    if (lane < KT) {
+      my_row = slot_row[t * KT + lane];
+      my_g = topk_w[t * KT + lane];
+    }
+    int64_t rows[KT + 1];
+    float g[KT];
+#pragma unroll
+    for (int k = 0; k < KT; ++k) {
+      rows[k] = __shfl_sync(0xffffffffu, my_row, k);
+      g[k] = __shfl_sync(0xffffffffu, my_g, k);
+    }
+    rows[KT] = n_shared ? shared0 + t : -1;
+    for (int d0 = lane * 8; d0 < D; d0 += 256 * NC) {
+      uint4 r[NC][KT + 1];
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int d = d0 + 256 * c;
+#pragma unroll
+        for (int k = 0; k <= KT; ++k)
+          r[c][k] = (rows[k] >= 0 && d < D) ? *reinterpret_cast<const uint4*>(o + rows[k] * D + d)
+                                            : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int d = d0 + 256 * c;
+        if (d >= D) continue;
+        float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+          if (rows[k] >= 0) {
+            float v[8];
+            bf16x8_to_f32(r[c][k], v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a[i] = fmaf(g[k], v[i], a[i]);
+          }
+        }
+        if (rows[KT] >= 0) {
+          float v[8];
+          bf16x8_to_f32(r[c][KT], v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[i] += v[i];
+        }
+        store8(y + t * D + d, a);
+      }
+    }
+  }
+}
+
 // Per permuted row: routed rows -> dg[slot] = <o[r], dy[t]> and
 // dO[r] = g * dy[t]; shared rows -> dO[r] = dy[t]; padding -> 0.  A row's
 // kind is decided by row_slot alone (the dispatch sets -1 on padding and
@@ -218,6 +281,80 @@ bwd_rows_kernel(const T* __restrict__ o, const T* __restrict__ dy,
       if (lane == 0) dg_slot[slot] = dot;
     }
   }
+}
+
+// The gate-gradient pass in token order (bf16, K in {1, 2, 4, 8}): each
+// token's dy row is read once; for each kept slot k, dg[slot] = <o[row_k],
+// dy_t> (the same per-row accumulation order as bwd_rows_kernel) and
+// dO[row_k] = g_k dy_t; the shared expert's row gets dO = dy_t; then the
+// padding rows of dO are zeroed.
+template <int KT>
+__global__ void __launch_bounds__(256)
+bwd_tok_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dy,
+               const float* __restrict__ topk_w, const int32_t* __restrict__ slot_row,
+               const int32_t* __restrict__ row_slot, const int32_t* __restrict__ offsets,
+               const int32_t* __restrict__ stats, int n_shared, int El, int Tn, int D,
+               float* __restrict__ dg_slot, __nv_bfloat16* __restrict__ dO) {
+  pdl_begin();
+  constexpr int NB = KT == 1 ? 4 : KT == 2 ? 2 : 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t shared0 = n_shared ? (int64_t)offsets[El] : -1;
+  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < Tn; t += (int64_t)gridDim.x * 8) {
+    int32_t my_row = -1;
+    float my_g = 0.f;
+    if (lane < KT) {
+      my_row = slot_row[t * KT + lane];
+      my_g = topk_w[t * KT + lane];
+    }
+    int64_t rows[KT];
+    float g[KT], dot[KT];
+#pragma unroll
+    for (int k = 0; k < KT; ++k) {
+      rows[k] = __shfl_sync(0xffffffffu, my_row, k);
+      g[k] = __shfl_sync(0xffffffffu, my_g, k);
+      dot[k] = 0.f;
+    }
+    const int64_t srow = n_shared ? shared0 + t : -1;
+    for (int d0 = lane * 8; d0 < D; d0 += 256 * NB) {
+      Raw8<__nv_bfloat16> rd[NB], ro[NB][KT];
+#pragma unroll
+      for (int j = 0; j < NB; ++j) {
+        const int d = d0 + 256 * j;
+        const int dc = d < D ? d : lane * 8;
+        rd[j].load(dy + t * D + dc);
+#pragma unroll
+        for (int k = 0; k < KT; ++k)
+          if (rows[k] >= 0) ro[j][k].load(o + rows[k] * D + dc);
+      }
+#pragma unroll
+      for (int j = 0; j < NB; ++j) {
+        const int d = d0 + 256 * j;
+        if (d >= D) continue;
+        float dv[8];
+        rd[j].widen(dv);
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+          if (rows[k] >= 0) {
+            float ov[8], w[8];
+            ro[j][k].widen(ov);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              dot[k] = fmaf(ov[i], dv[i], dot[k]);
+              w[i] = dv[i] * g[k];
+            }
+            store8(dO + rows[k] * D + d, w);
+          }
+        }
+        if (srow >= 0) store8(dO + srow * D + d, dv);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < KT; ++k) {
+      const float v = warp_sum(dot[k]);
+      if (lane == 0 && rows[k] >= 0) dg_slot[t * KT + k] = v;
+    }
+  }
+  zero_padding_rows(dO, stats[2], D, row_slot, shared0, n_shared ? Tn : 0);
 }
 
 struct RouterBwdArgs {

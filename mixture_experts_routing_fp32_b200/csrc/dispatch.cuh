@@ -359,4 +359,67 @@ disp_gather_kernel(const TX* __restrict__ x, int D, int K, int E, int T,
   }
 }
 
+// Padding rows (row_slot < 0 outside the shared expert's rows) of a
+// permuted buffer set to zero: each warp checks 32 rows per step.
+template <typename TX>
+__device__ __forceinline__ void zero_padding_rows(TX* __restrict__ buf, int64_t n_rows, int D,
+                                                  const int32_t* __restrict__ row_slot,
+                                                  int64_t shared0, int64_t shared_n) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t base = ((int64_t)blockIdx.x * 8 + warp) * 32; base < n_rows;
+       base += (int64_t)gridDim.x * 8 * 32) {
+    const int64_t r = base + lane;
+    const bool pad = r < n_rows && row_slot[r] < 0 && !(r >= shared0 && r < shared0 + shared_n);
+    unsigned m = __ballot_sync(0xffffffffu, pad);
+    while (m != 0u) {
+      const int64_t rr = base + __ffs(m) - 1;
+      m &= m - 1u;
+      for (int d = lane * 8; d < D; d += 256) zero8(buf + rr * D + d);
+    }
+  }
+}
+
+// Pass 4 in token order (K in {1, 2, 4, 8}): each token's row of x is read
+// once and written to the rows of its kept slots (and its shared-expert
+// row); then the padding rows are zeroed.  One warp per token, NB
+// 256-column steps of loads in flight before their stores.
+template <typename TX, int KT>
+__global__ void __launch_bounds__(256)
+disp_gather_tok_kernel(const TX* __restrict__ x, int D, int El, int T, int n_shared,
+                       const int32_t* __restrict__ offsets, const int32_t* __restrict__ stats,
+                       const int32_t* __restrict__ slot_row, const int32_t* __restrict__ row_slot,
+                       TX* __restrict__ x_perm) {
+  pdl_begin();
+  constexpr int NB = KT <= 2 ? 4 : 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t shared0 = n_shared ? (int64_t)offsets[El] : -1;
+  for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < T; t += (int64_t)gridDim.x * 8) {
+    const int32_t my_row = lane < KT ? slot_row[t * KT + lane] : -1;
+    int64_t rows[KT + 1];
+#pragma unroll
+    for (int k = 0; k < KT; ++k) rows[k] = __shfl_sync(0xffffffffu, my_row, k);
+    rows[KT] = n_shared ? shared0 + t : -1;
+    const TX* src = x + t * D;
+    for (int d0 = lane * 8; d0 < D; d0 += 256 * NB) {
+      Raw8<TX> v[NB];
+#pragma unroll
+      for (int j = 0; j < NB; ++j) {
+        const int d = d0 + 256 * j;
+        v[j].load(src + (d < D ? d : lane * 8));
+      }
+#pragma unroll
+      for (int k = 0; k <= KT; ++k) {
+        if (rows[k] >= 0) {
+#pragma unroll
+          for (int j = 0; j < NB; ++j) {
+            const int d = d0 + 256 * j;
+            if (d < D) v[j].store(x_perm + rows[k] * D + d);
+          }
+        }
+      }
+    }
+  }
+  zero_padding_rows(x_perm, stats[2], D, row_slot, shared0, n_shared ? T : 0);
+}
+
 }  // namespace moe

@@ -819,6 +819,17 @@ bool bn512_enabled() {
   return on;
 }
 
+// Tile width of the weight-gradient GEMMs: pick_bn's choice, or
+// MOE_WGRAD_BN (128 or 256, if it divides the output width) for tuning.
+int wgrad_bn(int bn, int64_t n_out) {
+  static const int forced = [] {
+    const char* v = std::getenv("MOE_WGRAD_BN");
+    return v != nullptr ? std::atoi(v) : 0;
+  }();
+  if ((forced == 128 || forced == 256) && n_out % forced == 0) return forced;
+  return bn;
+}
+
 // Row tiles per rasterisation group: as many 128-row A tiles of depth Kd as
 // fit in about 48 MiB of L2, so they stay resident while the group sweeps
 // the weight column slices.
@@ -871,6 +882,29 @@ int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_id
     MOE_LAUNCHED(s, "dispatch_rank");
   }
   if (x_perm == nullptr) return MOE_OK;   // layout only: the GEMMs gather x rows
+  if (!c->expert_choice && (c->K == 1 || c->K == 2 || c->K == 4 || c->K == 8)) {
+    // token order: each token's row of x read once for all its slots
+    auto go = [&](auto tx, auto kt) -> int {
+      using TX = decltype(tx);
+      constexpr int KT = decltype(kt)::value;
+      prof_begin(s);
+      MOE_CK((launch_k(disp_gather_tok_kernel<TX, KT>, grid_for(c->T), 256, 0, s,
+                       static_cast<const TX*>(x), c->D, El, c->T, c->n_shared, offsets, stats,
+                       slot_row, row_slot, static_cast<TX*>(x_perm))));
+      MOE_LAUNCHED(s, "dispatch_gather");
+      return MOE_OK;
+    };
+    auto by_k = [&](auto tx) -> int {
+      switch (c->K) {
+        case 1: return go(tx, std::integral_constant<int, 1>{});
+        case 2: return go(tx, std::integral_constant<int, 2>{});
+        case 4: return go(tx, std::integral_constant<int, 4>{});
+        default: return go(tx, std::integral_constant<int, 8>{});
+      }
+    };
+    if (c->dtype == MOE_BF16) return by_k(__nv_bfloat16{});
+    return by_k(float{});
+  }
   const int grid = grid_for(L.rows_max);
   prof_begin(s);
   if (c->dtype == MOE_BF16)
@@ -1352,7 +1386,12 @@ int moe_combine(const moe_config_t* c, const void* o, const int32_t* slot_row,
   if (c->dtype == MOE_BF16 && (c->K == 1 || c->K == 2 || c->K == 4 || c->K == 8)) {
     auto go = [&](auto kt) -> int {
       prof_begin(s);
-      MOE_CK((launch_k(combine_bf16_kernel<decltype(kt)::value>, grid, 256, 0, s,
+      constexpr int KT = decltype(kt)::value;
+      auto kern = [] {
+        if constexpr (KT <= 2) return combine_bf16_wide_kernel<KT>;
+        else return combine_bf16_kernel<KT>;
+      }();
+      MOE_CK((launch_k(kern, grid, 256, 0, s,
                        static_cast<const __nv_bfloat16*>(o), slot_row, topk_w, offsets,
                        c->n_shared, c->T, c->D, local_E(c), static_cast<__nv_bfloat16*>(y))));
       MOE_LAUNCHED(s, "combine");
@@ -1404,13 +1443,28 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   void* dH = wsp<void>(ws, L.off_dH);
   const bool bf = c->dtype == MOE_BF16;
   // the router's backward products (dW_r, the router part of dx) on tensor
-  // cores from E > 8 (and for expert choice); with up to 8 experts CUDA
-  // cores form them next to the data they are added to
-  const bool rtc = router_tc(c) && (E > 8 || c->expert_choice);
+  // cores from E >= 8 (measured faster than the CUDA-core forms at E = 8)
+  const bool rtc = router_tc(c);
   const bool dx1 = token_epilogues(c) && !rtc;   // dx from the dgrad gate/up epilogue
 
-  // 1. per row: gate gradient dg = <o, dy>, and dO = g * dy
-  {
+  // 1. per row: gate gradient dg = <o, dy>, and dO = g * dy (token order:
+  // each token's dy row read once for all its slots)
+  if (bf && !c->expert_choice && (K == 1 || K == 2 || K == 4 || K == 8)) {
+    auto go = [&](auto kt) -> int {
+      constexpr int KT = decltype(kt)::value;
+      prof_begin(s);
+      MOE_CK((launch_k(bwd_tok_kernel<KT>, grid_for(T), 256, 0, s,
+                       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dy),
+                       topk_w, slot_row, row_slot, offsets, stats, c->n_shared, El, T, D, dg,
+                       static_cast<__nv_bfloat16*>(dO))));
+      MOE_LAUNCHED(s, "bwd_gate_grad_rows");
+      return MOE_OK;
+    };
+    if (K == 1) MOE_TRY(go(std::integral_constant<int, 1>{}));
+    else if (K == 2) MOE_TRY(go(std::integral_constant<int, 2>{}));
+    else if (K == 4) MOE_TRY(go(std::integral_constant<int, 4>{}));
+    else MOE_TRY(go(std::integral_constant<int, 8>{}));
+  } else {
     const int grid = grid_for(L.rows_max);
     prof_begin(s);
     if (bf)
@@ -1500,7 +1554,9 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     const bool pr = pair_rows(c);                 // CTA-pair row tiles
     const int64_t units = pr ? L.tiles_max / 2 : L.tiles_max;
     // 3. dgrad down + SwiGLU backward: dA13 = swiglu'(dO . w_down[e])
-    const int bn3 = pick_bn(F, mt, false, F, pr, D / 64);
+    // (BN = 512 leaves this epilogue -- a13 read, dA13 written -- unoverlapped:
+    // measured slower than BN = 256 on the Mixtral-shaped layer)
+    const int bn3 = pick_bn(F, mt, false, F, pr, 0);
     // k blocks of an average weight-gradient tile (the group's rows)
     const int64_t wg_kb = ceil_div(row_tiles_estimate(c, L) * kRowTile, (int64_t)groups * 64);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 128, false));
@@ -1521,7 +1577,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     // 4. wgrad down: dW_down[e] = dO^T h over the expert's rows (CTA pairs
     // split the 256-row output tiles)
     const bool pw4 = (D % 256) == 0;
-    const int bn4 = pick_bn(F, (int64_t)groups * (D / 128), false, F, pw4, wg_kb);
+    const int bn4 = wgrad_bn(pick_bn(F, (int64_t)groups * (D / 128), false, F, pw4, wg_kb), F);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 64, false));
     MOE_TRY(make_map(&mB, h, 1, L.rows_max, F, 64, false));
     {
@@ -1570,7 +1626,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     // producer warp copies the B rows from x by row_slot; mapB unused)
     const bool pw6 = ((2 * F) % 256) == 0;
     const bool g6 = x_perm == nullptr;
-    const int bn6 = pick_bn(D, (int64_t)groups * (2 * F / 128), false, F, pw6, wg_kb);
+    const int bn6 = wgrad_bn(pick_bn(D, (int64_t)groups * (2 * F / 128), false, F, pw6, wg_kb), D);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 64, false));
     MOE_TRY(make_map(&mB, g6 ? x : x_perm, 1, g6 ? T : L.rows_max, D, 64, false));
     {
