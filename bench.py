@@ -166,7 +166,7 @@ def hbm_bytes(cfg, kept_total, rows_used):
     M = expert_rows(cfg, kept_total)
     router = T * D * a + E * D * 4 + 2 * T * E * 4 + T * 4 + T * K * 8
     return {
-        "router_fused": router, "router_logits": T * D * a + E * D * 4 + T * E * 4,
+        "router_fused": router, "router_tc": router, "router_logits": T * D * a + E * D * 4 + T * E * 4,
         "router_route": 3 * T * E * 4 + T * 4 + T * K * 8,
         "dispatch_gather": T * D * a + rows_used * D * a,
         "combine": M * D * a + T * D * a + T * K * 8,

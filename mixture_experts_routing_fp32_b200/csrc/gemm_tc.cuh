@@ -433,6 +433,26 @@ __device__ __forceinline__ void staged_store32(uint32_t stg, const float (&v)[32
   __syncwarp();
 }
 
+// staged_store32 of values already packed to bf16 (pk[4 j + i] holds the
+// pairs of columns 8 j + 2 i, 8 j + 2 i + 1).
+__device__ __forceinline__ void staged_store32_pk(uint32_t stg, const uint4 (&pk)[4],
+                                                  __nv_bfloat16* w0, int64_t ld, uint64_t pol) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) sts128(stg + lane * kStgRow + j * 16, pk[j]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i * 8 + (lane >> 2), pc = lane & 3;
+    const uint4 u = lds128(stg + r * kStgRow + pc * 16);
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(
+                     w0 + r * ld + pc * 8),
+                 "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w), "l"(pol)
+                 : "memory");
+  }
+  __syncwarp();
+}
+
 // staged_store32 to scattered rows: block row i goes to w0 + tok_i * ld,
 // where tok_i is lane i's `tok` (rows with tok < 0 are skipped).
 __device__ __forceinline__ void staged_store32_tok(uint32_t stg, const float (&v)[32],
@@ -1040,7 +1060,42 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       if (!ok) break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * BN;
-      if constexpr (EPI == EPI_STORE || EPI == EPI_WGRAD) {
+      if constexpr ((EPI == EPI_STORE || EPI == EPI_WGRAD) && HC <= 128) {
+        // the whole accumulator slice is read (packed to bf16 in registers)
+        // and released before the stores, so the next tile's MMAs need not
+        // wait for this tile's global stores
+        __nv_bfloat16* w0;
+        int64_t ld;
+        if (EPI == EPI_STORE) {
+          w0 = p.out + row0 * p.ld_out + d.n0 + hh * HC;
+          ld = p.ld_out;
+        } else {
+          __nv_bfloat16* og = d.e < p.E ? p.out + (int64_t)d.e * p.strideCE : p.out_shared;
+          w0 = og + row0 * p.No + d.n0 + hh * HC;
+          ld = p.No;
+        }
+        uint4 pk[HC / 32][4];
+#pragma unroll
+        for (int c = 0; c < HC; c += 32) {
+          uint32_t r[32];
+          float v[32];
+          tmem_ld32(tbase + hh * HC + c, r);
+          tmem_wait();
+          u2f32(r, v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) pk[c / 32][j] = pack8_bf16(v + 8 * j);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (!PAIR || leader) mbar_arrive(acce_bar(acc));
+          else mbar_arrive_remote(mapa(acce_bar(acc), 0));   // the leader's barrier
+        }
+#pragma unroll
+        for (int c = 0; c < HC; c += 32) staged_store32_pk(stg, pk[c / 32], w0 + c, ld, pol_out);
+        if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
+        continue;
+      } else if constexpr (EPI == EPI_STORE || EPI == EPI_WGRAD) {
         __nv_bfloat16* w0;
         int64_t ld;
         if (EPI == EPI_STORE) {

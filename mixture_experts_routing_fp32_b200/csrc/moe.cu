@@ -184,15 +184,15 @@ int64_t capacity_of(const moe_config_t* c);
 // fast.  Ep = E rounded up to 64 (split width).
 bool router_tc(const moe_config_t* c) { return use_tc(c) && c->E >= 8; }
 // Token-choice routing inside the tensor-core logits kernel: up to 64
-// experts, no group limit, K in {1, 2, 4, 8} (MOE_ROUTER_FUSED=0: the
-// partial-logit GEMM and a separate routing kernel instead, for
-// cross-checks).
+// experts, no group limit, K in {1, 2, 4, 8} (MOE_ROUTER_FUSED=0: for
+// E >= 8 the partial-logit GEMM and a separate routing kernel instead, for
+// fewer experts the CUDA-core router; for cross-checks).
 bool router_fused_tc(const moe_config_t* c) {
   static const bool on = [] {
     const char* v = std::getenv("MOE_ROUTER_FUSED");
     return !(v != nullptr && v[0] == '0');
   }();
-  return on && router_tc(c) && !c->expert_choice && c->E <= 64 && c->n_groups == 1 &&
+  return on && use_tc(c) && !c->expert_choice && c->E <= 64 && c->n_groups == 1 &&
          (c->K == 1 || c->K == 2 || c->K == 4 || c->K == 8);
 }
 int64_t router_ep(const moe_config_t* c) { return (c->E + 63) / 64 * 64; }
@@ -270,9 +270,11 @@ Layout layout_of(const moe_config_t* c) {
   L.off_dA13 = take((size_t)L.rows_max * 2 * c->F * a);
   L.off_dX = take((size_t)L.rows_max * c->D * a);
   L.off_dH = use_tc(c) ? off : take((size_t)L.rows_max * c->F * a);
-  if (router_tc(c)) {
+  if (router_tc(c) || router_fused_tc(c)) {
     L.Ep = router_ep(c);
     L.off_wf = take((size_t)3 * L.Ep * c->D * 2);
+  }
+  if (router_tc(c)) {
     L.off_wb = take((size_t)3 * L.Ep * c->D * 2);
     L.off_rparts = take((size_t)c->T * 3 * L.Ep * 4);
     L.off_dsf = take((size_t)c->T * 3 * L.Ep * 2);
@@ -335,22 +337,6 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t n3, int64_t rows, int64_t 
                   dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) { g_last_cuda_error = (int)cudaErrorInvalidValue; return MOE_ERR_CUDA; }
-  return MOE_OK;
-}
-
-// Three-way bf16 splits of W_r as a 3-D tensor [3][EP][D] (hi, mid, lo),
-// one box {64 columns, EP rows, 3 planes} per k block.
-int make_map_splits(CUtensorMap* m, const void* ptr, int64_t EP, int64_t D) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) { g_last_cuda_error = (int)cudaErrorNotSupported; return MOE_ERR_CUDA; }
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)EP, 3};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)(EP * D * 2)};
-  cuuint32_t box[3] = {64, (cuuint32_t)EP, 3};
-  cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
-                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) { g_last_cuda_error = (int)cudaErrorInvalidValue; return MOE_ERR_CUDA; }
   return MOE_OK;
 }
@@ -548,38 +534,98 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
               c->group_score, c->route_scale, bias, logits, probs, lse, idx, w, ties};
   MOE_CK(cudaMemsetAsync(ties, 0, sizeof(int32_t), s));
   if (router_fused_tc(c)) {
-    // logits on tensor cores (the three splits accumulated in one tensor-
-    // memory accumulator) and the routing in the same kernel's epilogue
+    // logits on tensor cores (the three splits stacked along N of one MMA)
+    // and the routing in the same kernel's epilogue
     const Layout L = layout_of(c);
-    const int EP = c->E <= 32 ? 32 : 64;
+    // split width: E rounded up to 8, 16, 32 or 64 (fewer W_r bytes per
+    // tile for few experts)
+    const int EP = c->E <= 8 ? 8 : c->E <= 16 ? 16 : c->E <= 32 ? 32 : 64;
     auto* wf = wsp<__nv_bfloat16>(ws, L.off_wf);
     prof_begin(s);
     MOE_CK((launch_k(split_w_kernel, grid_for((int64_t)EP * c->D / 32), 256, 0, s, w_r, c->E,
                      EP, c->D, wf, (__nv_bfloat16*)nullptr)));
     MOE_LAUNCHED(s, "router_split_w");
+    // E > 16: CTA pairs (each CTA streams half of the split rows)
+    const bool pair = EP >= 32;
+    // Tile height: as many 128-token rounds as the token count needs over
+    // all CTAs, then the tokens spread evenly over them (a multiple of 8,
+    // at least 64 so that few tokens do not spread over many CTAs that each
+    // stream all of W_r).
+    if (c->T == 0) return MOE_OK;
+    static int max_pairs = 0;   // resident CTA pairs (the same for every split width)
+    if (pair && max_pairs == 0) {
+      auto k = rtc::router_tc_kernel<64, 8, true>;
+      constexpr int sm = rtc::Smem<64, true>::kBytes;
+      MOE_CK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, sm));
+      cudaLaunchConfig_t lc = {};
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      lc.gridDim = dim3(2 * (num_sms() / 2));
+      lc.blockDim = dim3(rtc::kThreads);
+      lc.dynamicSmemBytes = sm;
+      lc.attrs = at;
+      lc.numAttrs = 1;
+      int n = 0;
+      MOE_CK(cudaOccupancyMaxActiveClusters(&n, k, &lc));
+      max_pairs = n > 0 ? n : num_sms() / 2;
+    }
+    const int ctas = pair ? 2 * max_pairs : num_sms();
+    const int64_t rounds = ceil_div(c->T, (int64_t)128 * ctas);
+    int bm = (int)round_up(ceil_div(c->T, rounds * ctas), 8);
+    bm = std::max(64, std::min(128, bm));
+    const int64_t units = ceil_div(c->T, (int64_t)(pair ? 2 * bm : bm));
+    const int NA = (3 * EP + 15) / 16 * 16;
     CUtensorMap mX, mW;
-    MOE_TRY(make_map(&mX, x, 1, c->T, c->D, 128, false));
-    MOE_TRY(make_map_splits(&mW, wf, EP, c->D));
-    const int grid = (int)std::min<int64_t>(num_sms(), ceil_div(c->T, 128));
-    auto go = [&](auto kern, size_t smem) -> int {
+    MOE_TRY(make_map(&mX, x, 1, c->T, c->D, (uint32_t)bm, false));
+    MOE_TRY(make_map(&mW, wf, 1, 3 * EP, c->D, (uint32_t)(pair ? NA / 2 : 3 * EP), false));
+    auto go = [&](auto kern, size_t smem, auto pr) -> int {
+      constexpr bool PR = decltype(pr)::value;
       MOE_CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-      prof_begin(s);
-      MOE_CK((launch_k(kern, grid, rtc::kThreads, smem, s, mX, mW, a, off, c->D)));
+      if constexpr (PR) {
+        cudaLaunchConfig_t lc = {};
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        lc.blockDim = dim3(rtc::kThreads);
+        lc.dynamicSmemBytes = smem;
+        lc.stream = s;
+        lc.attrs = attr;
+        lc.gridDim = dim3((unsigned)(2 * std::min<int64_t>(max_pairs, units)));
+        lc.numAttrs = pdl_enabled() ? 2 : 1;
+        prof_begin(s);
+        MOE_CK(cudaLaunchKernelEx(&lc, kern, mX, mW, a, off, c->D, bm));
+      } else {
+        prof_begin(s);
+        MOE_CK((launch_k(kern, (int)std::min<int64_t>(num_sms(), units), rtc::kThreads, smem, s,
+                         mX, mW, a, off, c->D, bm)));
+      }
       MOE_LAUNCHED(s, "router_tc");
       return MOE_OK;
     };
-    auto by_k = [&](auto ep) -> int {
+    auto by_k = [&](auto ep, auto pr) -> int {
       constexpr int P = decltype(ep)::value;
-      constexpr size_t sm = rtc::Smem<P>::kBytes;
+      constexpr bool PR = decltype(pr)::value;
+      constexpr size_t sm = rtc::Smem<P, PR>::kBytes;
       switch (c->K) {
-        case 1: return go(rtc::router_tc_kernel<P, 1>, sm);
-        case 2: return go(rtc::router_tc_kernel<P, 2>, sm);
-        case 4: return go(rtc::router_tc_kernel<P, 4>, sm);
-        default: return go(rtc::router_tc_kernel<P, 8>, sm);
+        case 1: return go(rtc::router_tc_kernel<P, 1, PR>, sm, pr);
+        case 2: return go(rtc::router_tc_kernel<P, 2, PR>, sm, pr);
+        case 4: return go(rtc::router_tc_kernel<P, 4, PR>, sm, pr);
+        default: return go(rtc::router_tc_kernel<P, 8, PR>, sm, pr);
       }
     };
-    if (EP == 32) return by_k(std::integral_constant<int, 32>{});
-    return by_k(std::integral_constant<int, 64>{});
+    using NoPair = std::false_type;
+    using Pair = std::true_type;
+    if (EP == 8) return by_k(std::integral_constant<int, 8>{}, NoPair{});
+    if (EP == 16) return by_k(std::integral_constant<int, 16>{}, NoPair{});
+    if (EP == 32) return by_k(std::integral_constant<int, 32>{}, Pair{});
+    return by_k(std::integral_constant<int, 64>{}, Pair{});
   }
   if (router_tc(c)) {
     // logits parts = x . (W_hi | W_mid | W_lo)^T on tensor cores (dense GEMM,
@@ -943,7 +989,7 @@ int moe_router(const moe_config_t* c, const void* x, const float* w_r, const flo
   if (!x || !w_r || !logits || !probs || !lse || !topk_idx || !topk_w || !near_ties)
     return MOE_ERR_ARG;
   if (c->expert_choice) return MOE_ERR_ARG;   // moe_route_expert_choice
-  if (router_tc(c) && ws == nullptr) return MOE_ERR_ARG;
+  if ((router_tc(c) || router_fused_tc(c)) && ws == nullptr) return MOE_ERR_ARG;
   if (c->dtype == MOE_BF16)
     return router_impl(c, static_cast<const __nv_bfloat16*>(x), w_r, logit_offset, sel_bias,
                        logits, probs, lse, topk_idx, topk_w, near_ties, ws, s);

@@ -10,18 +10,28 @@
 //
 // The fp32 product x . W_r^T (x bf16) runs as bf16 MMAs on three-way bf16
 // splits of W_r (hi, mid, lo: |w - hi - mid - lo| <= 2^-24 |w|).  The
-// splits are stacked along N: one MMA per 16-wide k step, N = 3 EP, gives
-// three fp32 accumulators in tensor memory (x.hi | x.mid | x.lo, each
-// accumulating products of its own magnitude), which the epilogue sums per
-// expert as (hi + mid) + lo: fp32-accurate logits without a partial-logit
-// tensor in global memory.  Each stage carries one 128 x 64 tile of x and
-// the three 64-column k blocks of the splits (one 3-D TMA box, which lands
-// as the 3 EP rows of one K-major B operand).
+// splits are stacked along N ([hi; mid; lo], 3 EP rows, EP = E rounded up
+// to 8, 16, 32 or 64): one MMA per 16-wide k step gives three fp32
+// accumulators in tensor memory (x.hi | x.mid | x.lo, each accumulating
+// products of its own magnitude), which the epilogue sums per expert as
+// (hi + mid) + lo: fp32-accurate logits without a partial-logit tensor in
+// global memory.
 //
-// Roles (192 threads, one CTA per SM, persistent over 128-token tiles):
-//   warp 0   TMA producer (x tile + split box per stage, STAGES-deep ring)
-//   warp 1   MMA issuer (M=128, N=3 EP, 4 MMAs per stage), double-buffered
-//            accumulators (2 x 3 EP tensor-memory columns)
+// Tiles: each CTA takes bm tokens per tile (bm <= 128, a multiple of 8,
+// chosen by the host so that the tiles spread evenly over the SMs); the MMA
+// is always M = 128 (M = 256 for a pair) and the accumulator rows past bm
+// are not read.  For E > 16 two CTAs of a cluster share each MMA
+// (cta_group::2, M = 256): each loads its own bm token rows and half of the
+// stacked split rows, so a CTA streams half of W_r per tile.  Each stage
+// carries two k blocks: two bm x 64 tiles of x and two 64-column blocks of
+// the split rows (half as many barrier round trips per byte as one k block
+// per stage: measured faster, most at the power-capped clocks of a full
+// step).
+//
+// Roles (320 threads, one CTA per SM, persistent over tiles):
+//   warp 0   TMA producer (x tile + split rows per stage, STAGES-deep ring)
+//   warp 1   MMA issuer (the pair leader only for a pair; N = 3 EP rounded
+//            up to 16, 4 MMAs per stage), double-buffered accumulators
 //   warps 2-9 epilogue, in two phases per tile:
 //            1. warps 2-5 (one per tensor-memory lane quarter) read their 32
 //               tokens' accumulators, sum the splits per expert, add the
@@ -36,6 +46,8 @@
 // Every barrier wait is bounded (see tc::mbar_wait); on timeout the kernel
 // records MOE_DEVERR_TIMEOUT, drains its copies and MMAs and returns.
 #pragma once
+#include <type_traits>
+
 #include "gemm_tc.cuh"
 #include "router.cuh"
 
@@ -45,30 +57,53 @@ namespace rtc {
 constexpr int kEpiWarps = 8;     // routing warps (the first four also read tensor memory)
 constexpr int kTmemWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kSmemMax = 232448;   // dynamic shared memory per CTA
 
-template <int EP>
+// EP: split width; PAIR: two CTAs per MMA (each holds NB = NA / 2 rows of
+// the stacked splits).
+template <int EP, bool PAIR>
 struct Smem {
-  static constexpr int kA = 128 * 64 * 2;         // x tile of one k block
-  static constexpr int kB = 3 * EP * 128;         // hi | mid | lo k blocks of W_r
-  static constexpr int kStage = kA + kB;
-  static constexpr int STAGES = EP == 32 ? 6 : 4;
+  static constexpr int NA = (3 * EP + 15) / 16 * 16;   // MMA N (24 runs as 32)
+  static constexpr int NAS = (NA + 31) / 32 * 32;      // accumulator stride (columns)
+  static constexpr int NB = PAIR ? NA / 2 : NA;        // B rows in this CTA
+  static constexpr int kA = 128 * 64 * 2;              // x tile of one k block (bm <= 128 rows)
+  // stage: [x kb | x kb+1 | splits kb | splits kb+1]
+  // split rows one stage receives: a pair's box is NB rows (rows past 3 EP
+  // are zero-filled); a single CTA's box is the 3 EP rows (the N = 32 MMA
+  // of EP = 8 also reads 8 unwritten rows, whose columns are never read)
+  static constexpr int kBoxB = PAIR ? NB * 128 : 3 * EP * 128;
+  static constexpr int kB = (NB * 128 + 1023) / 1024 * 1024;
+  static constexpr int kStage = 2 * (kA + kB);   // two k blocks per stage
+  static constexpr int kStgLd = EP + 1;                // staging row stride (floats)
+  static constexpr int kStg = 128 * kStgLd * 4;        // one [128 x EP] staging tile
+  static constexpr int kFixed = 1024 + 2048 + kStg;    // alignment, barriers, params, staging
+  static constexpr int kFit = (kSmemMax - kFixed) / kStage;
+  static constexpr int STAGES = kFit < 8 ? kFit : 8;
   static constexpr int kBars = (2 * STAGES + 5) * 8;
-  static constexpr int kStgLd = EP + 1;           // staging row stride (floats)
   static constexpr int kParOff = STAGES * kStage + kBars + 16;   // offset, bias [64] each
   static constexpr int kStgOff = kParOff + 2 * 64 * 4;
-  static constexpr int kBytes = 1024 + kStgOff + 128 * kStgLd * 4;   // one [128 x EP] tile
-  static_assert(kBytes <= 232448, "shared memory per CTA");
+  static constexpr int kBytes = 1024 + kStgOff + kStg;
+  static_assert(STAGES >= 3, "pipeline depth");
+  static_assert(kBytes + 64 <= kSmemMax, "shared memory per CTA (with the static words)");
+  static_assert(!PAIR || NB % 8 == 0, "whole 8-row swizzle atoms per CTA");
 };
 
 // Writes rows [row0, row0 + nrows) of a [T, E] fp32 tensor from the warp's
 // staging tile (row r at stg + r * ld): the rows are contiguous in global
 // memory, so the warp stores them as one block (16-byte stores when E is a
-// multiple of 4).
+// multiple of 4; E = EP divides by a constant).
+template <int EP>
 __device__ __forceinline__ void block_store_rows(float* __restrict__ g, int64_t row0, int nrows,
                                                  int E, const float* stg, int ld, int lane) {
   float* dst = g + row0 * E;
   const int n = nrows * E;
-  if ((E & 3) == 0) {
+  if (E == EP) {
+    for (int i = 4 * lane; i < n; i += 128) {
+      const int r = i / EP, c = i % EP;
+      const float* sp = stg + r * ld + c;
+      *reinterpret_cast<float4*>(dst + i) = make_float4(sp[0], sp[1], sp[2], sp[3]);
+    }
+  } else if ((E & 3) == 0) {
     for (int i = 4 * lane; i < n; i += 128) {
       const int r = i / E, c = i - r * E;
       const float* sp = stg + r * ld + c;
@@ -82,26 +117,32 @@ __device__ __forceinline__ void block_store_rows(float* __restrict__ g, int64_t 
   }
 }
 
-// (v, e, s) into the list of N = K + 1 entries kept in selection order:
-// larger score first, equal scores by lower expert index.
+// (v, e) into a list of N entries kept in selection order (larger score
+// first), where v ranks below every entry whose score it does not exceed
+// (the entries came from lower expert indices); v is not NaN.
+// Branch-free: position j takes max(lu[j], min(lu[j-1], v)) (its entry, v,
+// or the entry pushed down from j - 1), and its index follows the two
+// comparisons of v with lu[j] and lu[j-1]; going down from the last
+// position, only two comparisons are live at a time.
 template <int N>
-__device__ __forceinline__ void topk_insert(float (&lu)[N], int (&le)[N], float (&ls)[N], float v,
-                                            int e, float s) {
+__device__ __forceinline__ void topk_push(float (&lu)[N], int (&le)[N], float v, int e) {
+  bool beats_j = v > lu[N - 1];
 #pragma unroll
-  for (int j = 0; j < N; ++j) {
-    const bool gt = v > lu[j] || (v == lu[j] && e < le[j]);
-    const float tv = lu[j], ts = ls[j];
-    const int te = le[j];
-    lu[j] = gt ? v : tv; le[j] = gt ? e : te; ls[j] = gt ? s : ts;
-    v = gt ? tv : v; e = gt ? te : e; s = gt ? ts : s;
+  for (int j = N - 1; j > 0; --j) {
+    const bool beats_prev = v > lu[j - 1];
+    le[j] = beats_j ? (beats_prev ? le[j - 1] : e) : le[j];
+    lu[j] = fmaxf(lu[j], fminf(lu[j - 1], v));
+    beats_j = beats_prev;
   }
+  le[0] = beats_j ? e : le[0];
+  lu[0] = fmaxf(lu[0], v);
 }
 
-template <int EP, int K>
+template <int EP, int K, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,
-                 const RouteArgs a, const float* __restrict__ offset, int D) {
-  using S = Smem<EP>;
+                 const RouteArgs a, const float* __restrict__ offset, int D, int bm) {
+  using S = Smem<EP, PAIR>;
   constexpr int STAGES = S::STAGES;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int abort_flag_s;
@@ -119,16 +160,24 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * S::kStage + S::kBars);
   float* off_s = reinterpret_cast<float*>(gbase + S::kParOff);
   float* bias_s = off_s + 64;
-  constexpr int NA = 3 * EP;                                // one accumulator's columns
-  constexpr uint32_t kCols = 2 * NA <= 256 ? 256u : 512u;  // two accumulators
+  constexpr int NA = S::NA;                                 // MMA width
+  constexpr int NAS = S::NAS;                               // accumulator stride
+  constexpr uint32_t kCols = 2 * NAS <= 64 ? 64u : 2 * NAS <= 128 ? 128u
+                           : 2 * NAS <= 256 ? 256u : 512u;  // two accumulators
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = (a.T + 127) / 128;
+  const int rank = PAIR ? (int)tc::cluster_rank() : 0;     // 0 = pair leader
+  const bool leader = rank == 0;
+  const int unit = PAIR ? blockIdx.x >> 1 : blockIdx.x;    // this CTA's tile stream
+  const int n_units = PAIR ? gridDim.x >> 1 : gridDim.x;
+  const int U = PAIR ? 2 * bm : bm;                         // tokens per tile (both CTAs)
+  const int n_tiles = (a.T + U - 1) / U;
   const int nk = D / 64;
   // Tiles start their k loop at different k blocks, so the CTAs running at
   // the same time do not all load the same W_r block from L2 at once; the
   // accumulation order is fixed by the tile index (deterministic).
-  auto rot_of = [&](int t) { return (int)(((int64_t)t * 5) % nk); };
+  const int nk2 = nk / 2;                                  // stages per tile
+  auto rot_of = [&](int t) { return (int)(((int64_t)t * 5) % nk2); };
   if (threadIdx.x == 0) {
     abort_flag_s = 0;
     epi_stop_s = 0;
@@ -138,7 +187,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(accf_bar(b), 1);
-      tc::mbar_init(acce_bar(b), kTmemWarps);
+      tc::mbar_init(acce_bar(b), kTmemWarps * (PAIR ? 2 : 1));   // both CTAs' readers
     }
     tc::mbar_init(done_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -146,82 +195,117 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
   }
   if (warp == 0) {
     __syncwarp();
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     tc::smem_u32(tmem_slot)),
-                 "r"(kCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       tc::smem_u32(tmem_slot)),
+                   "r"(kCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       tc::smem_u32(tmem_slot)),
+                   "r"(kCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc::tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) tc::cluster_sync();   // both CTAs' barriers exist before any remote use
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_begin();   // the set-up above touched only this CTA's shared and tensor memory
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer ----------------
+      // ---------------- TMA producer (both CTAs of a pair) ----------------
       int stage = 0;
       uint32_t phase = 0;
       int issued_parity[STAGES];
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+      const uint32_t tx = 2u * (uint32_t)(bm * 128 + S::kBoxB) * (PAIR ? 2u : 1u);
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      for (int t = unit; t < n_tiles && ok; t += n_units) {
         const int rot = rot_of(t);
-        for (int i = 0; i < nk; ++i) {
-          const int kb = i + rot < nk ? i + rot : i + rot - nk;
+        const int row = t * U + rank * bm;                   // this CTA's first token
+        for (int i = 0; i < nk2; ++i) {
+          const int kb = 2 * (i + rot < nk2 ? i + rot : i + rot - nk2);
           if (!tc::mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t sa = base + stage * S::kStage;
           const uint32_t fb = full_bar(stage);
-          tc::mbar_expect_tx(fb, S::kStage);
+          if (!PAIR || leader) tc::mbar_expect_tx(fb, tx);
           issued_parity[stage] = (int)phase;
-          tc::tma_2d(sa, &mapX, fb, kb * 64, t * 128);
-          tc::tma_3d(sa + S::kA, &mapW, fb, kb * 64, 0, 0);
+          if constexpr (PAIR) {
+            const uint32_t lfb = tc::mapa(fb, 0);           // the leader's full barrier
+            tc::tma_2d_pair_nohint(sa, &mapX, lfb, kb * 64, row);
+            tc::tma_2d_pair_nohint(sa + S::kA, &mapX, lfb, kb * 64 + 64, row);
+            tc::tma_2d_pair_nohint(sa + 2 * S::kA, &mapW, lfb, kb * 64, rank * S::NB);
+            tc::tma_2d_pair_nohint(sa + 2 * S::kA + S::kB, &mapW, lfb, kb * 64 + 64, rank * S::NB);
+          } else {
+            tc::tma_2d(sa, &mapX, fb, kb * 64, row);
+            tc::tma_2d(sa + S::kA, &mapX, fb, kb * 64 + 64, row);
+            tc::tma_2d(sa + 2 * S::kA, &mapW, fb, kb * 64, 0);
+            tc::tma_2d(sa + 2 * S::kA + S::kB, &mapW, fb, kb * 64 + 64, 0);
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      for (int s = 0; s < STAGES; ++s)
-        if (issued_parity[s] >= 0) tc::mbar_wait(full_bar(s), (uint32_t)issued_parity[s], abort_flag);
+      // drain: the copies have landed before teardown (a pair's copies all
+      // complete on the leader's barriers)
+      if (!PAIR || leader)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_parity[s] >= 0)
+            tc::mbar_wait(full_bar(s), (uint32_t)issued_parity[s], abort_flag);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = tc::make_idesc(128, NA, false, false);
+      constexpr uint32_t idesc = tc::make_idesc(PAIR ? 256 : 128, NA, false, false);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      for (int t = unit; t < n_tiles && ok; t += n_units) {
         if (!tc::mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag)) break;
         tc::tc_fence_after();
-        const uint32_t dt = tmem + acc * NA;
-        for (int kb = 0; kb < nk; ++kb) {   // k blocks in the producer's (rotated) order
+        const uint32_t dt = tmem + acc * NAS;
+        for (int kb = 0; kb < nk2; ++kb) {   // k block pairs in the producer's (rotated) order
           if (!tc::mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
           tc::tc_fence_after();
           const uint32_t sa = base + stage * S::kStage;
-          const uint32_t sb = sa + S::kA;
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = tc::sw128_desc(sa + ks * 32, 16, 1024);
-            const uint64_t bd = tc::sw128_desc(sb + ks * 32, 16, 1024);
-            tc::umma(dt, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+          for (int sub = 0; sub < 2; ++sub) {
+            const uint32_t sas = sa + sub * S::kA;
+            const uint32_t sbs = sa + 2 * S::kA + sub * S::kB;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = tc::sw128_desc(sas + ks * 32, 16, 1024);
+              const uint64_t bd = tc::sw128_desc(sbs + ks * 32, 16, 1024);
+              const uint32_t accum = (kb | sub | ks) != 0 ? 1u : 0u;
+              if constexpr (PAIR) tc::umma_pair(dt, ad, bd, idesc, accum);
+              else tc::umma(dt, ad, bd, idesc, accum);
+            }
           }
-          tc::umma_commit(empty_bar(stage));
+          if constexpr (PAIR) tc::umma_commit_pair_both(empty_bar(stage));
+          else tc::umma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc::umma_commit(accf_bar(acc));
+        if constexpr (PAIR) tc::umma_commit_pair_both(accf_bar(acc));
+        else tc::umma_commit(accf_bar(acc));
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
-      tc::umma_commit(done_bar);
+      if constexpr (PAIR) tc::umma_commit_pair_local(done_bar);
+      else tc::umma_commit(done_bar);
       tc::mbar_wait(done_bar, 0, abort_flag);
     }
   } else {
     // ---------------- epilogue ----------------
     constexpr int HE = EP / 2;                               // experts per lane
+    constexpr int CH = HE < 8 ? HE : 8;                      // unrolled chunk
     const int E = a.E;
     const int ew = warp - 2;
     for (int e = ew * 32 + lane; e < 64; e += kEpiWarps * 32) {
@@ -239,7 +323,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
     const int rloc = ew * 16 + (lane & 15);                  // this lane's token in the tile
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    for (int t = unit; t < n_tiles; t += n_units) {
       // phase 1: splits -> logits (+ offset) in the shared tile
       bool ok = true;
       if (ew < kTmemWarps) {
@@ -248,23 +332,40 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (ok) {
           tc::tc_fence_after();
-          uint32_t r0[32], r1[32], r2[32];
-          const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + acc * NA;
+          const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + acc * NAS;
           float* srow = stg + (q * 32 + lane) * S::kStgLd;
+          if constexpr (EP >= 32) {
+            uint32_t r0[32], r1[32], r2[32];
 #pragma unroll
-          for (int c = 0; c < EP; c += 32) {
-            tc::tmem_ld32(tb + c, r0);
-            tc::tmem_ld32(tb + EP + c, r1);
-            tc::tmem_ld32(tb + 2 * EP + c, r2);
+            for (int c = 0; c < EP; c += 32) {
+              tc::tmem_ld32(tb + c, r0);
+              tc::tmem_ld32(tb + EP + c, r1);
+              tc::tmem_ld32(tb + 2 * EP + c, r2);
+              tc::tmem_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                srow[c + i] = ((__uint_as_float(r0[i]) + __uint_as_float(r1[i])) +
+                               __uint_as_float(r2[i])) + off_s[c + i];
+            }
+          } else {
+            // all three splits of the (8 or 16) experts in one or two loads
+            constexpr int NC = NAS / 32;
+            uint32_t r[NC][32];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) tc::tmem_ld32(tb + 32 * c, r[c]);
             tc::tmem_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              srow[c + i] = ((__uint_as_float(r0[i]) + __uint_as_float(r1[i])) +
-                             __uint_as_float(r2[i])) + off_s[c + i];
+            for (int i = 0; i < EP; ++i)
+              srow[i] = ((__uint_as_float(r[i / 32][i % 32]) +
+                          __uint_as_float(r[(EP + i) / 32][(EP + i) % 32])) +
+                         __uint_as_float(r[(2 * EP + i) / 32][(2 * EP + i) % 32])) + off_s[i];
           }
           tc::tc_fence_before();
           __syncwarp();
-          if (lane == 0) tc::mbar_arrive(acce_bar(acc));   // accumulator free for tile t + 2
+          if (lane == 0) {   // accumulator free for tile t + 2 (the pair leader's barrier)
+            if (!PAIR || leader) tc::mbar_arrive(acce_bar(acc));
+            else tc::mbar_arrive_remote(tc::mapa(acce_bar(acc), 0));
+          }
         } else if (lane == 0) {
           epi_stop_s = 1;   // a wait gave up: every epilogue warp leaves after the barrier
         }
@@ -273,59 +374,94 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
       epi_sync();
       if (*reinterpret_cast<volatile int*>(&epi_stop_s)) break;   // same decision in all eight warps
       // phase 2: route 16 tokens per warp, two lanes per token
-      const int64_t row0 = (int64_t)t * 128 + ew * 16;
-      if (row0 < a.T) {
-        const int nrows = (int)((a.T - row0) < 16 ? (a.T - row0) : 16);
-        const int64_t tok = (int64_t)t * 128 + rloc;
-        const bool valid = tok < a.T;
+      const int64_t tok0 = (int64_t)t * U + rank * bm;       // this CTA's first token
+      const int r0 = ew * 16;                                // this warp's first row
+      if (r0 < bm && tok0 + r0 < a.T) {
+        const int nrows = (int)min((int64_t)min(16, bm - r0), a.T - (tok0 + r0));
+        const int64_t tok = tok0 + rloc;
+        const bool valid = rloc < bm && tok < a.T;
         float* srow = stg + rloc * S::kStgLd;
-        block_store_rows(a.logits, row0, nrows, E, stg + ew * 16 * S::kStgLd, S::kStgLd, lane);
-        // this lane's experts e = half * HE + j, read from the shared tile in
-        // rolled loops (the code stays small: it runs once per tile)
+        block_store_rows<EP>(a.logits, tok0 + r0, nrows, E, stg + r0 * S::kStgLd, S::kStgLd, lane);
+        // this lane's experts e = e0 + j (j < HE, e < E), read from the
+        // shared row in unrolled chunks of CH (straight-line code, no
+        // data-dependent branches)
         const int e0 = half * HE;
-        const int e1 = min(E, e0 + HE);
         float m = NEG;
-#pragma unroll 4
-        for (int e = e0; e < e1; ++e) m = fmaxf(m, srow[e]);
+#pragma unroll 1
+        for (int jc = 0; jc < HE; jc += CH) {
+#pragma unroll
+          for (int jj = 0; jj < CH; ++jj) {
+            const int e = e0 + jc + jj;
+            if (e < E) m = fmaxf(m, srow[e]);
+          }
+        }
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-        // top-(K+1) of this lane's experts (selection score u = s, or
-        // sigmoid + bias), before the row is overwritten with the scores
-        float lu[K + 1], ls[K + 1];
+        // softmax denominator, and the top-(K+1) of this lane's experts by
+        // selection score (u = s, or sigmoid + bias), kept in selection
+        // order (larger first, equal scores by lower expert index)
+        float lu[K + 1];
         int le[K + 1];
 #pragma unroll
-        for (int k = 0; k <= K; ++k) { lu[k] = NEG; le[k] = 0x7fffffff; ls[k] = 0.f; }
+        for (int k = 0; k <= K; ++k) { lu[k] = NEG; le[k] = 0x7fffffff; }
         float z = 0.f;
-#pragma unroll 2
-        for (int e = e0; e < e1; ++e) {
-          const float sv = srow[e];
-          z += __expf(sv - m);
-          const float u = sigm ? 1.0f / (1.0f + __expf(-sv)) + bias_s[e] : sv;
-          if (u > lu[K]) topk_insert<K + 1>(lu, le, ls, u, e, sv);
-        }
+        // (the score function is uniform: one loop per form)
+        auto select = [&](auto sig) {
+          constexpr bool SIG = decltype(sig)::value;
+#pragma unroll 1
+          for (int jc = 0; jc < HE; jc += CH) {
+#pragma unroll
+            for (int jj = 0; jj < CH; ++jj) {
+              const int e = e0 + jc + jj;
+              const bool in = e < E;
+              const float sv = in ? srow[e] : NEG;
+              z += in ? __expf(sv - m) : 0.f;
+              float u = SIG ? 1.0f / (1.0f + __expf(-sv)) + bias_s[e] : sv;
+              u = (in && u == u) ? u : NEG;     // padding experts and NaN never selected
+              topk_push<K + 1>(lu, le, u, e);   // e ascending: an equal score stays behind
+            }
+          }
+        };
+        if (sigm) select(std::true_type{});
+        else select(std::false_type{});
         z += __shfl_xor_sync(0xffffffffu, z, 16);
         const float inv_z = 1.0f / z;
         const float lse = m + logf(z);
-        __syncwarp();                                         // logits rows stored
-        // scores (softmax probs or sigmoid affinities) into the same rows
-#pragma unroll 4
-        for (int e = e0; e < e1; ++e) {
-          const float sv = srow[e];
-          srow[e] = sigm ? 1.0f / (1.0f + __expf(-sv)) : __expf(sv - m) * inv_z;
-        }
-        __syncwarp();
-        block_store_rows(a.probs, row0, nrows, E, stg + ew * 16 * S::kStgLd, S::kStgLd, lane);
-        // merge with the partner lane's list
-        float pu[K + 1], ps[K + 1];
+        // merge the partner lane's list: its experts all lie above this
+        // lane's for half 0 (the lane that writes), so an equal score from
+        // the partner stays behind
+        float pu[K + 1];
         int pe[K + 1];
 #pragma unroll
-        for (int k = 0; k <= K; ++k) {
+        for (int k = 0; k <= K; ++k) {   // both lists exchanged before either changes
           pu[k] = __shfl_xor_sync(0xffffffffu, lu[k], 16);
           pe[k] = __shfl_xor_sync(0xffffffffu, le[k], 16);
-          ps[k] = __shfl_xor_sync(0xffffffffu, ls[k], 16);
         }
 #pragma unroll
-        for (int k = 0; k <= K; ++k)
-          if (pu[k] != NEG) topk_insert<K + 1>(lu, le, ls, pu[k], pe[k], ps[k]);
+        for (int k = 0; k <= K; ++k) topk_push<K + 1>(lu, le, pu[k], pe[k]);
+        // logits of the selected experts (the row still holds logits)
+        float ls[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k) ls[k] = srow[min(le[k], E - 1)];
+        __syncwarp();                                   // logits rows stored and read
+        // scores (softmax probs or sigmoid affinities) into the same rows
+        auto scores = [&](auto sig) {
+          constexpr bool SIG = decltype(sig)::value;
+#pragma unroll 1
+          for (int jc = 0; jc < HE; jc += CH) {
+#pragma unroll
+            for (int jj = 0; jj < CH; ++jj) {
+              const int e = e0 + jc + jj;
+              if (e < E) {
+                const float sv = srow[e];
+                srow[e] = SIG ? 1.0f / (1.0f + __expf(-sv)) : __expf(sv - m) * inv_z;
+              }
+            }
+          }
+        };
+        if (sigm) scores(std::true_type{});
+        else scores(std::false_type{});
+        __syncwarp();
+        block_store_rows<EP>(a.probs, tok0 + r0, nrows, E, stg + r0 * S::kStgLd, S::kStgLd, lane);
         float margin = INFINITY;
 #pragma unroll
         for (int k = 1; k <= K; ++k)
@@ -358,11 +494,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant
   }
   tc::tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) tc::cluster_sync();   // the leader's MMAs into both CTAs are done
   tc::tc_fence_after();
   if (warp == 0) {
     __syncwarp();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols)
-                 : "memory");
+    if constexpr (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols)
+                   : "memory");
   }
 }
 

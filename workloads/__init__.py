@@ -123,6 +123,15 @@ REDUCED = {
                                           seq_len=100),
     "ds3_seq": CONFIGS["ds3"].replace(name="ds3_seq_small", T=300, D=256, F=128,
                                       aux_alpha=1e-3, seq_len=100),
+    # router split widths 16 and 32 (the E = 32 router runs on CTA pairs):
+    # sigmoid + selection bias, variant B; softmax, variant A with aux + z
+    "e16_sig": LayerConfig("e16_sig_small", T=900, D=256, E=16, K=4, F=256, score_fn=SIGMOID,
+                           renorm=1, sel_bias_range=0.1),
+    "e32": LayerConfig("e32_small", T=1500, D=384, E=32, K=2, F=256, renorm=0,
+                       aux_alpha=0.01, z_lambda=1e-3),
+    # more tokens than one 128-row round of router tiles over all CTAs: several
+    # tiles per CTA pair, ragged last tile
+    "olmoe_tiles": CONFIGS["olmoe"].replace(name="olmoe_tiles_small", T=20000, D=128, F=128),
     # expert choice: 8 experts (with z-loss, C = 128 of 512 tokens) and the
     # OLMoE-shaped 64 experts at reduced size
     "ec8": LayerConfig("ec8_small", T=512, D=256, E=8, K=8, F=256, renorm=0,
