@@ -70,6 +70,9 @@ def parse():
                     help="override the config's token count (small cases for profiling)")
     ap.add_argument("--experts", type=int, default=0,
                     help="override the config's expert count (small cases for profiling)")
+    ap.add_argument("--only", default="", choices=["", "router"],
+                    help="router: time moe_router alone on the config's shape (one JSON line, "
+                         "GB/s of the router kernel; for profiling captures)")
     return ap.parse_args()
 
 
@@ -768,10 +771,63 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_router_only(args):
+    """moe_router alone on the config's shape: L2 flushed before each call,
+    CUDA-event time of each library launch (LaunchProfile)."""
+    from mixture_experts_routing_fp32_b200 import api, config_from, moe_check_status
+    from mixture_experts_routing_fp32_b200.build import build
+    build()
+    dev = torch.device("cuda", 0)
+    base = W.CONFIGS[args.config]
+    if args.tokens:
+        base = base.replace(T=args.tokens)
+    if args.experts:
+        base = base.replace(E=args.experts)
+    cfg = config_from(base)
+    T, E, K = base.T, base.E, base.K
+    x = W.make_input(base, "x", dev)
+    w_r = W.make_input(base, "w_r", dev)
+    off = W.make_input(base, "logit_offset", dev) if base.hot_expert_offset else None
+    bias = W.make_input(base, "sel_bias", dev) if base.sel_bias_range else None
+    f32 = dict(dtype=torch.float32, device=dev)
+    logits, probs = torch.empty(T, E, **f32), torch.empty(T, E, **f32)
+    lse, w = torch.empty(T, **f32), torch.empty(T, K, **f32)
+    idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+    ties = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.empty(api.moe_get_sizes(cfg).ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    prof = api.LaunchProfile(16)
+    per = {}
+    for i in range(max(args.warmup, 3) + args.steps):
+        flush.fill_(i & 255)
+        prof.reset()
+        api.moe_router(cfg, x, w_r, off, bias, logits, probs, lse, idx, w, ties, ws)
+        torch.cuda.synchronize(dev)
+        if i >= max(args.warmup, 3):
+            for n, ms, _ in prof.read():
+                per.setdefault(n, []).append(ms)
+    moe_check_status()
+    med = {n: sorted(v)[len(v) // 2] for n, v in per.items()}
+    a = 2 if base.dtype == "bf16" else 4
+    nbytes = T * base.D * a + E * base.D * 4 + 2 * T * E * 4 + T * 4 + T * K * 8
+    kern = "router_tc" if "router_tc" in med else max(med, key=med.get)
+    hbm, _, _, src = measured_peaks()
+    gbs = nbytes / (med[kern] * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "router kernel GB/s (algorithmic bytes / CUDA-event time, L2 flushed)",
+        "value": round(gbs, 1), "unit": "GB/s", "kernel": kern,
+        "frac_of_hbm": round(gbs / hbm, 4), "peak_source": src, "bytes": nbytes,
+        "kernels_ms": {n: round(v, 5) for n, v in med.items()}, "steps": args.steps,
+        "config": {"workload": "%s: T=%d D=%d E=%d K=%d" % (base.name, T, base.D, E, K)},
+        "near_ties": int(ties.item())}))
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.only == "router":
+        run_router_only(args)
     else:
         run_ours(args)
 
