@@ -373,7 +373,7 @@ template <int BN, int ST, int MODE, bool AMN, bool BMN, int EPI, bool PAIR, bool
 int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
               const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
               cudaStream_t s) {
-  using S = tc::Smem<BN, ST, PAIR>;
+  using S = tc::KernelSmem<BN, ST, MODE, PAIR, GATHER>;
   auto k = tc::gemm_kernel<BN, ST, MODE, AMN, BMN, EPI, PAIR, GATHER>;
   MOE_CK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes));
   if constexpr (PAIR) {
@@ -426,9 +426,19 @@ int run_tc(int bn, const char* name, const CUtensorMap& a, const CUtensorMap& b,
         return launch_tc<512, 4, MODE, AMN, BMN, EPI, true, false>(name, a, b, bs, p, total_max,
                                                                   total_hint, s);
     }
+    if constexpr (!GATHER) {
+      if (bn == 256)   // two k blocks per stage (tc::stage_kb)
+        return launch_tc<256, 3, MODE, AMN, BMN, EPI, true, false>(name, a, b, bs, p, total_max,
+                                                                  total_hint, s);
+    }
     if (bn == 256)
       return launch_tc<256, 6, MODE, AMN, BMN, EPI, true, GATHER>(name, a, b, bs, p, total_max,
                                                                  total_hint, s);
+    if constexpr (!GATHER) {
+      if (bn == 128)
+        return launch_tc<128, 4, MODE, AMN, BMN, EPI, true, false>(name, a, b, bs, p, total_max,
+                                                                  total_hint, s);
+    }
     if (bn == 128)
       return launch_tc<128, 8, MODE, AMN, BMN, EPI, true, GATHER>(name, a, b, bs, p, total_max,
                                                                  total_hint, s);
@@ -441,6 +451,11 @@ int run_tc(int bn, const char* name, const CUtensorMap& a, const CUtensorMap& b,
       if (bn == 192)
         return launch_tc<192, 5, MODE, AMN, BMN, EPI, false, GATHER>(name, a, b, bs, p,
                                                                     total_max, total_hint, s);
+    }
+    if constexpr (!GATHER) {
+      if (bn == 128)
+        return launch_tc<128, 3, MODE, AMN, BMN, EPI, false, false>(name, a, b, bs, p, total_max,
+                                                                   total_hint, s);
     }
     if (bn == 128)
       return launch_tc<128, 6, MODE, AMN, BMN, EPI, false, GATHER>(name, a, b, bs, p, total_max,
