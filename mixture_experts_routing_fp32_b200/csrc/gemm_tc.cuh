@@ -578,18 +578,19 @@ struct Smem {
   static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
-// k blocks per pipeline stage: two for 256-wide pair tiles and 128-wide
-// tiles (stages of 48-64 KB per CTA instead of 24-32 KB, about the same
-// bytes in flight with half the barrier round trips; measured 4-15% faster
-// on the OLMoE-, Mixtral- and DeepSeek-shaped GEMMs and 23% on the
-// router weight gradient, results bit-identical), else one (the 512-wide
-// tiles' 48 KB stages, the 192/256-wide single-CTA tiles and the gathering
-// producer).  The kernel and its launch both take the shared-memory layout
-// from here.
+// k blocks per pipeline stage: two for pair tiles and 128-wide tiles
+// (stages of 48-96 KB per CTA instead of 24-48 KB, about the same bytes in
+// flight with half the barrier round trips; measured 3-15% faster on the
+// OLMoE-, Mixtral- and DeepSeek-shaped GEMMs and 23% on the router weight
+// gradient, results bit-identical), else one (the 192/256-wide single-CTA
+// tiles, where two 80-96 KB stages measured slower than 4-5 of one k
+// block, and the gathering producer).  The kernel and its launch both take
+// the shared-memory layout from here.
 template <int BN, int STAGES, int MODE, bool PAIR, bool GATHER>
 constexpr int stage_kb() {
-  return (!GATHER && ((PAIR && BN == 256 && STAGES == 3) || (PAIR && BN == 128 && STAGES == 4) ||
-                      (!PAIR && BN == 128 && STAGES == 3))) ? 2 : 1;
+  return (!GATHER && ((PAIR && BN == 512 && STAGES == 2) || (PAIR && BN == 256 && STAGES == 3) ||
+                      (PAIR && BN == 128 && STAGES == 4) || (!PAIR && BN == 128 && STAGES == 3)))
+             ? 2 : 1;
 }
 template <int BN, int STAGES, int MODE, bool PAIR, bool GATHER>
 using KernelSmem = Smem<BN, STAGES, PAIR, stage_kb<BN, STAGES, MODE, PAIR, GATHER>()>;

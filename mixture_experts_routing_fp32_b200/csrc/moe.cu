@@ -422,8 +422,8 @@ int run_tc(int bn, const char* name, const CUtensorMap& a, const CUtensorMap& b,
   if constexpr (PAIR) {
     // per CTA: A 16 KB + half of B per stage
     if constexpr (!GATHER) {
-      if (bn == 512)
-        return launch_tc<512, 4, MODE, AMN, BMN, EPI, true, false>(name, a, b, bs, p, total_max,
+      if (bn == 512)   // two stages of two k blocks (tc::stage_kb)
+        return launch_tc<512, 2, MODE, AMN, BMN, EPI, true, false>(name, a, b, bs, p, total_max,
                                                                   total_hint, s);
     }
     if constexpr (!GATHER) {
