@@ -434,7 +434,11 @@ int moe_combine(const moe_config_t* cfg, const void* o,
  * Inside the call, independent chains (the router gradient, the two
  * weight-gradient GEMMs) are forked onto three side streams and joined back
  * into `stream` before the call returns, so the results are ordered on
- * `stream` like any other call.  The side streams are the caller's when set
+ * `stream` like any other call.  When each weight-gradient GEMM is 2 TFLOP
+ * or more (4·rows·F·D with the expected rows), everything runs in order on
+ * `stream` instead: two persistent GEMMs at once only share the SMs.  The
+ * fork/join still happens (events recorded on `stream` itself).  The side
+ * streams are the caller's when set
  * with moe_set_backward_streams (recommended: one set per layer, so that
  * independent layers' backward passes do not queue behind one another);
  * otherwise the library creates three streams and eight events per host
