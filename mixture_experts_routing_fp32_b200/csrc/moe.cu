@@ -522,6 +522,33 @@ int group_rows(int64_t Kd, bool pair = false);
 // logits), one warp per token.
 int route_launch(const moe_config_t* c, const RouteArgs& a, const float* logits,
                  const float* parts, int64_t Ep, const float* off, cudaStream_t s) {
+  // from the partial logits with E a multiple of 32 and groups (if any) of
+  // 32 experts: E / 32 lanes per token, one per 32-expert chunk
+  const int L = c->E / 32;
+  if (parts != nullptr && c->E % 32 == 0 && L <= 32 && (L & (L - 1)) == 0 &&
+      (c->n_groups == 1 || c->E / c->n_groups == 32) && c->K <= 8) {
+    auto go = [&](auto l, auto km) -> int {
+      constexpr int LL = decltype(l)::value, KM = decltype(km)::value;
+      const int grid = (int)ceil_div((int64_t)c->T * LL, 256);
+      prof_begin(s);
+      MOE_CK((launch_k(router_route_lanes_kernel<LL, KM>, grid, 256, 0, s, parts, (int)Ep, off, a)));
+      MOE_LAUNCHED(s, "router_route");
+      return MOE_OK;
+    };
+    auto by_k = [&](auto l) -> int {
+      if (c->K <= 2) return go(l, std::integral_constant<int, 2>{});
+      if (c->K <= 4) return go(l, std::integral_constant<int, 4>{});
+      return go(l, std::integral_constant<int, 8>{});
+    };
+    switch (L) {
+      case 1: return by_k(std::integral_constant<int, 1>{});
+      case 2: return by_k(std::integral_constant<int, 2>{});
+      case 4: return by_k(std::integral_constant<int, 4>{});
+      case 8: return by_k(std::integral_constant<int, 8>{});
+      case 16: return by_k(std::integral_constant<int, 16>{});
+      default: return by_k(std::integral_constant<int, 32>{});
+    }
+  }
   const size_t sm = 8 * (size_t)c->E * 4;
   const int grid = grid_for(c->T);
   auto go = [&](auto nv) -> int {

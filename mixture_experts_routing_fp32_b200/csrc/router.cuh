@@ -380,4 +380,190 @@ router_route_parts_kernel(const float* __restrict__ parts, int Ep,
   }
 }
 
+// (v, e) into a list of N entries kept in selection order (larger score
+// first, equal scores by lower expert index).  `first`: v comes from a
+// lower expert index than every entry (an equal score goes in front), else
+// from a higher one (an equal score stays behind).  Branch-free: position
+// j takes max(lu[j], min(lu[j-1], v)) (its entry, v, or the entry pushed
+// down from j - 1) and its index follows the comparisons of v with lu[j]
+// and lu[j-1]; going down from the last position, only two comparisons are
+// live at a time.  v is not NaN; v = -inf is never inserted.
+template <int N>
+__device__ __forceinline__ void topk_push(float (&lu)[N], int (&le)[N], float v, int e,
+                                          bool first = false) {
+  const bool real = v != -INFINITY;
+  auto beats = [&](float x) { return v > x || (first && real && v == x); };
+  bool beats_j = beats(lu[N - 1]);
+#pragma unroll
+  for (int j = N - 1; j > 0; --j) {
+    const bool beats_prev = beats(lu[j - 1]);
+    le[j] = beats_j ? (beats_prev ? le[j - 1] : e) : le[j];
+    lu[j] = fmaxf(lu[j], fminf(lu[j - 1], v));
+    beats_j = beats_prev;
+  }
+  le[0] = beats_j ? e : le[0];
+  lu[0] = fmaxf(lu[0], v);
+}
+
+// Routing from the three partial-logit blocks with L = E / 32 lanes per
+// token (E a multiple of 32, at most 1024): lane j of a token holds experts
+// 32 j .. 32 j + 31 — group j when the group limit has 32 experts per
+// group (the DeepSeek-shaped 8 groups of 32).  Each lane sums its logits'
+// parts in the partial-logit path's order, writes its logits and scores,
+// scores its group, and keeps the top-(K+1) of its experts by a
+// branch-free push; the L lanes exchange group scores (rank of each group,
+// lower group index first on ties) and merge their lists by shuffles in
+// log2 L rounds.  The selection, the near-tie margins (among the top K+1,
+// and between the last kept and the first dropped group) and the gate
+// weights follow route_token; its warp-wide argmax rounds took 0.1 ms on
+// the DeepSeek shape.
+template <int L, int KM>
+__global__ void __launch_bounds__(256)
+router_route_lanes_kernel(const float* __restrict__ parts, int Ep,
+                          const float* __restrict__ offset, RouteArgs a) {
+  pdl_begin();
+  constexpr int N = KM + 1;
+  const float NEG = -INFINITY;
+  const int lane = threadIdx.x & 31;
+  const int j = lane % L;                    // this lane's 32-expert chunk
+  const int base = lane - j;                 // the token's first lane
+  const int64_t tok = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / L;
+  const bool valid = tok < a.T;
+  const int64_t t = valid ? tok : (int64_t)a.T - 1;   // whole warps take part in the shuffles
+  const int E = a.E;
+  const int e0 = 32 * j;
+  const bool sigm = a.score_fn != MOE_SOFTMAX;
+  // logits: (hi + mid) + lo + offset, as the partial-logit path sums them
+  float sv[32];
+  const float* pr = parts + t * 3 * (int64_t)Ep + e0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 h = *reinterpret_cast<const float4*>(pr + 4 * q);
+    const float4 m = *reinterpret_cast<const float4*>(pr + Ep + 4 * q);
+    const float4 l = *reinterpret_cast<const float4*>(pr + 2 * Ep + 4 * q);
+    sv[4 * q] = (h.x + m.x) + l.x;
+    sv[4 * q + 1] = (h.y + m.y) + l.y;
+    sv[4 * q + 2] = (h.z + m.z) + l.z;
+    sv[4 * q + 3] = (h.w + m.w) + l.w;
+  }
+  if (offset != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) sv[i] += offset[e0 + i];
+  }
+  // logsumexp over the token's L lanes
+  float mx = NEG;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) mx = fmaxf(mx, sv[i]);
+#pragma unroll
+  for (int d = 1; d < L; d <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+  float z = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) z += expf(sv[i] - mx);
+#pragma unroll
+  for (int d = 1; d < L; d <<= 1) z += __shfl_xor_sync(0xffffffffu, z, d);
+  const float lse = mx + logf(z);
+  // scores and selection scores; logits and scores rows written
+  float u[32];
+  float* lrow = a.logits + t * E + e0;
+  float* prow = a.probs + t * E + e0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    float pv[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int i = 4 * q + r;
+      pv[r] = sigm ? 1.0f / (1.0f + expf(-sv[i])) : expf(sv[i] - mx) / z;
+      u[i] = sigm ? pv[r] + (a.sel_bias != nullptr ? a.sel_bias[e0 + i] : 0.f) : sv[i];
+      if (!(u[i] == u[i])) u[i] = NEG;      // NaN never selected
+    }
+    if (valid) {
+      *reinterpret_cast<float4*>(lrow + 4 * q) = make_float4(sv[4 * q], sv[4 * q + 1],
+                                                             sv[4 * q + 2], sv[4 * q + 3]);
+      *reinterpret_cast<float4*>(prow + 4 * q) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+    }
+  }
+  // group limit: this lane's chunk is one group
+  float gmargin = INFINITY;
+  if (a.n_groups > 1) {
+    float b1 = NEG, b2 = NEG;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float v = u[i];
+      if (v > b1) { b2 = b1; b1 = v; } else if (v > b2) { b2 = v; }
+    }
+    const float gs = (a.group_score == MOE_GMAX) ? b1 : b1 + b2;
+    float gall[L];
+#pragma unroll
+    for (int q = 0; q < L; ++q) gall[q] = __shfl_sync(0xffffffffu, gs, base + q);
+    const int tg = a.topk_groups;
+    int rank = 0;
+    float last = NEG, next = NEG;
+#pragma unroll
+    for (int q = 0; q < L; ++q) {
+      int rq = 0;
+#pragma unroll
+      for (int q2 = 0; q2 < L; ++q2)
+        rq += (gall[q2] > gall[q] || (gall[q2] == gall[q] && q2 < q)) ? 1 : 0;
+      if (q == j) rank = rq;
+      if (rq == tg - 1) last = gall[q];
+      if (rq == tg) next = gall[q];
+    }
+    if (tg < L) gmargin = last - next;
+    if (rank >= tg) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) u[i] = NEG;
+    }
+  }
+  // top-(K+1): this lane's experts in ascending order, then the other lanes'
+  float lu[N];
+  int le[N];
+#pragma unroll
+  for (int k = 0; k < N; ++k) { lu[k] = NEG; le[k] = 0x7fffffff; }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) topk_push<N>(lu, le, u[i], e0 + i);
+#pragma unroll
+  for (int d = 1; d < L; d <<= 1) {
+    float pu[N];
+    int pe[N];
+#pragma unroll
+    for (int k = 0; k < N; ++k) {   // both lists exchanged before either changes
+      pu[k] = __shfl_xor_sync(0xffffffffu, lu[k], d);
+      pe[k] = __shfl_xor_sync(0xffffffffu, le[k], d);
+    }
+    const bool lower = (j & d) != 0;   // the partner's experts lie below this lane's
+#pragma unroll
+    for (int k = 0; k < N; ++k) topk_push<N>(lu, le, pu[k], pe[k], lower);
+  }
+  const int K = a.K;
+  float margin = INFINITY;
+#pragma unroll
+  for (int k = 1; k < N; ++k)
+    if (k <= K && lu[k] != NEG) margin = fminf(margin, lu[k - 1] - lu[k]);
+  const bool writer = valid && j == 0;
+  const unsigned tie = __ballot_sync(0xffffffffu, writer && (margin < kNearTie || gmargin < kNearTie));
+  if (lane == 0 && tie != 0u) atomicAdd(a.near_ties, __popc(tie));
+  __syncwarp();   // the logits and scores rows above are visible to the warp
+  if (writer) {
+    a.lse[t] = lse;
+    float g[KM], sel_s0 = 0.f, denom = 0.f;
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      if (k >= K) break;
+      const int e = min(le[k], E - 1);   // (fewer than K finite scores: NaN logits)
+      const float sk = a.logits[t * E + e], pk = a.probs[t * E + e];
+      if (k == 0) sel_s0 = sk;
+      g[k] = (!sigm && a.renorm) ? expf(sk - sel_s0) : pk;
+      denom += g[k];
+    }
+    if (a.renorm) denom = sigm ? denom + 1e-20f : denom;
+#pragma unroll
+    for (int k = 0; k < KM; ++k) {
+      if (k >= K) break;
+      float w = a.renorm ? g[k] / denom : g[k];
+      a.topk_idx[t * K + k] = le[k];
+      a.topk_w[t * K + k] = w * a.route_scale;
+    }
+  }
+}
+
 }  // namespace moe

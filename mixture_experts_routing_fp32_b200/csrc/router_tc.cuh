@@ -117,27 +117,6 @@ __device__ __forceinline__ void block_store_rows(float* __restrict__ g, int64_t 
   }
 }
 
-// (v, e) into a list of N entries kept in selection order (larger score
-// first), where v ranks below every entry whose score it does not exceed
-// (the entries came from lower expert indices); v is not NaN.
-// Branch-free: position j takes max(lu[j], min(lu[j-1], v)) (its entry, v,
-// or the entry pushed down from j - 1), and its index follows the two
-// comparisons of v with lu[j] and lu[j-1]; going down from the last
-// position, only two comparisons are live at a time.
-template <int N>
-__device__ __forceinline__ void topk_push(float (&lu)[N], int (&le)[N], float v, int e) {
-  bool beats_j = v > lu[N - 1];
-#pragma unroll
-  for (int j = N - 1; j > 0; --j) {
-    const bool beats_prev = v > lu[j - 1];
-    le[j] = beats_j ? (beats_prev ? le[j - 1] : e) : le[j];
-    lu[j] = fmaxf(lu[j], fminf(lu[j - 1], v));
-    beats_j = beats_prev;
-  }
-  le[0] = beats_j ? e : le[0];
-  lu[0] = fmaxf(lu[0], v);
-}
-
 template <int EP, int K, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap mapX, const __grid_constant__ CUtensorMap mapW,

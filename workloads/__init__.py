@@ -129,6 +129,10 @@ REDUCED = {
                            renorm=1, sel_bias_range=0.1),
     "e32": LayerConfig("e32_small", T=1500, D=384, E=32, K=2, F=256, renorm=0,
                        aux_alpha=0.01, z_lambda=1e-3),
+    # 128 experts without a group limit: routing from the partial logits
+    # with four lanes per token (the logits GEMM, then the routing kernel)
+    "e128": LayerConfig("e128_small", T=600, D=256, E=128, K=4, F=128, renorm=1,
+                        aux_alpha=0.01, z_lambda=1e-3, hot_expert_offset=1.0),
     # more tokens than one 128-row round of router tiles over all CTAs: several
     # tiles per CTA pair, ragged last tile
     "olmoe_tiles": CONFIGS["olmoe"].replace(name="olmoe_tiles_small", T=20000, D=128, F=128),
