@@ -199,10 +199,10 @@ def measured_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def recorded_traffic(kernel, workload):
-    """DRAM bytes per launch from a committed ncu summary, if the files that
-    define that kernel still hash to what they were when it was captured
-    (else None)."""
+def recorded_traffic(kernel, workload, tokens, experts):
+    """DRAM bytes per launch from a committed ncu summary, if it was captured
+    on this workload's shape and the files that define that kernel still
+    hash to what they were then (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -210,6 +210,8 @@ def recorded_traffic(kernel, workload):
         j = json.load(f)
     e = j.get(workload, {}).get(kernel)
     if not e or e.get("source_hash") != source_hash(e.get("files")):
+        return None
+    if e.get("T", tokens) != tokens or e.get("E", experts) != experts:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -554,7 +556,7 @@ def run_ours(args):
                 "peak_source": "%s copy bandwidth" % peak_src}
     roof.update({"kernel": dom, "launch_ms": round(dom_ms, 5), "timing": timing_src,
                  "launches_per_step": n_dom,
-                 "traffic": recorded_traffic(dom, base.name)})
+                 "traffic": recorded_traffic(dom, base.name, base.T, base.E)})
     gemm_names = sorted(k for k in flops if k in tot)
     gemm_total_ms = sum(tot[k] for k in gemm_names)
     gemm_tflops = (sum(flops[k] for k in gemm_names) / (gemm_total_ms * 1e-3) / 1e12
