@@ -143,7 +143,19 @@ def oracle_on_gpu_routing(cfg, layer, L=None):
 
 @pytest.mark.parametrize("name", [n for n, c in W.REDUCED.items() if not c.expert_choice])
 def test_parity_reduced(name):
-    cfg = W.REDUCED[name]
+    check_layer_parity(name, W.REDUCED[name])
+
+
+@pytest.mark.parametrize("name", list(W.EDGE))
+def test_parity_edge_shapes(name):
+    """One token, a few tokens, select-all, padding experts in the router's
+    split, the general routing kernel, K = 1 in the fused router, sigmoid
+    without a bias, 512 experts with groups: the same bar as the reduced
+    configs."""
+    check_layer_parity(name, W.EDGE[name])
+
+
+def check_layer_parity(name, cfg):
     layer, inp = run_gpu(cfg)
     fw, bw, flips = oracle_on_gpu_routing(cfg, layer)
     R = fw["R"]

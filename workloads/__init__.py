@@ -145,10 +145,39 @@ REDUCED = {
 }
 
 
+# Edge shapes of the routing path (same input recipe): a token count below
+# one router or expert tile, select-all (K = E), expert counts that are not a
+# split width (padding experts in the router's split), a count the four-lane
+# routing kernel does not take, K = 1 in the fused router, sigmoid without a
+# selection bias, and 512 experts with a group limit.
+EDGE = {
+    "t1_e64": CONFIGS["olmoe"].replace(name="edge_t1_e64", T=1, D=128, F=128),
+    "t1_e4": CONFIGS["mm_b"].replace(name="edge_t1_e4", T=1, D=128, F=128),
+    "t5_e8_cap": CONFIGS["mix"].replace(name="edge_t5_e8_cap", T=5, D=256, F=128),
+    "t3_e256_groups": CONFIGS["ds3"].replace(name="edge_t3_e256_groups", T=3, D=256, F=128),
+    "t130_e32": LayerConfig("edge_t130_e32", T=130, D=128, E=32, K=4, F=128, renorm=1,
+                            aux_alpha=0.01),
+    "k8_e8": LayerConfig("edge_k8_e8", T=300, D=128, E=8, K=8, F=128, renorm=1,
+                         aux_alpha=0.01, z_lambda=1e-3),
+    "k4_e4": LayerConfig("edge_k4_e4", T=200, D=128, E=4, K=4, F=128, renorm=0),
+    "e48": LayerConfig("edge_e48", T=400, D=128, E=48, K=4, F=128, renorm=1,
+                       z_lambda=1e-3, hot_expert_offset=1.0),
+    "e12_sig": LayerConfig("edge_e12_sig", T=257, D=128, E=12, K=2, F=128,
+                           score_fn=SIGMOID, renorm=1, route_scale=2.5),
+    "e96_k6": LayerConfig("edge_e96_k6", T=333, D=128, E=96, K=6, F=128, renorm=0,
+                          aux_alpha=0.01),
+    "e64_k1": LayerConfig("edge_e64_k1", T=500, D=128, E=64, K=1, F=128, renorm=1,
+                          aux_alpha=0.01),
+    "e512_groups": LayerConfig("edge_e512_groups", T=64, D=128, E=512, K=8, F=128,
+                               score_fn=SIGMOID, renorm=1, n_groups=16, topk_groups=4,
+                               route_scale=2.5, sel_bias_range=0.1),
+}
+
+
 def get(name: str) -> LayerConfig:
     if name in CONFIGS:
         return CONFIGS[name]
-    for c in REDUCED.values():
+    for c in list(REDUCED.values()) + list(EDGE.values()):
         if c.name == name:
             return c
     raise KeyError(name)
