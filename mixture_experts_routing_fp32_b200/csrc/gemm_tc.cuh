@@ -366,6 +366,28 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---- TMA stores (shared -> global, bulk async-groups of the issuing thread)
+// Box `src` (shared, laid out as the map's swizzle wants) to the tensor of
+// `map` at element coordinates (x, y); x * 2 bytes is a multiple of 16 and
+// both coordinates are non-negative (rows past the tensor are clipped).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until at most one committed group still reads its shared source.
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// Waits until every committed group has completed its global writes.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // 32 floats -> 32 bf16 at p (64 bytes, 16-byte aligned), with an L2 policy.
 __device__ __forceinline__ void store32_bf16(__nv_bfloat16* p, const float (&v)[32],
                                              uint64_t pol) {
@@ -451,6 +473,18 @@ __device__ __forceinline__ void staged_store32_pk(uint32_t stg, const uint4 (&pk
                  : "memory");
   }
   __syncwarp();
+}
+
+// Staging of one TMA-store box: 32 rows x 32 bf16 columns (64-byte rows)
+// in the 64-byte swizzle (16-byte chunk j of row r sits at chunk
+// j ^ ((r >> 1) & 3)), so the 16-byte stores of any 8 consecutive lanes
+// fall in distinct banks.  Lane r writes row r; `buf` is 512-byte aligned.
+constexpr int kTmaBox = 32 * 64;
+__device__ __forceinline__ void stage_box_sw64(uint32_t buf, const float (&v)[32]) {
+  const int r = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    sts128(buf + r * 64 + ((j ^ ((r >> 1) & 3)) << 4), pack8_bf16(v + 8 * j));
 }
 
 // staged_store32 to scattered rows: block row i goes to w0 + tok_i * ld,
@@ -572,9 +606,12 @@ struct Smem {
   static constexpr int kBars = (3 * STAGES + 2 * NACC + 1) * 8;
   // token table of the gathering producer (128 rows)
   static constexpr int kTokOff = STAGES * kStage + kBars + 16;
-  // epilogue staging tiles (one per epilogue warp), 128-byte aligned
-  static constexpr int kEpiOff = (kTokOff + 512 + 127) / 128 * 128;
-  static constexpr int kBytes = 1024 + kEpiOff + kEpiWarps * kStgBytes;
+  // epilogue staging per epilogue warp: a 2.5 KB tile, or for the
+  // 512-wide tiles (whose epilogues store through TMA) two 2 KB boxes;
+  // 512-byte aligned (the boxes' swizzle)
+  static constexpr int kStgW = BN == 512 ? 2 * kTmaBox : kStgBytes;
+  static constexpr int kEpiOff = (kTokOff + 512 + 511) / 512 * 512;
+  static constexpr int kBytes = 1024 + kEpiOff + kEpiWarps * kStgW;
   static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
@@ -599,11 +636,16 @@ using KernelSmem = Smem<BN, STAGES, PAIR, stage_kb<BN, STAGES, MODE, PAIR, GATHE
 // by 16-byte cp.async copies issued by the whole producer warp: the A rows
 // of a ROWS tile (gate/up + SwiGLU), or the B rows of a WGRAD k block
 // (gate/up weight gradient); the other operand still arrives by TMA box.
+// mapO / mapO2: the outputs of the 512-wide SwiGLU (a13, h) and plain-store
+// (out) epilogues as 2-D bf16 tensors with 32 x 32 boxes in the 64-byte
+// swizzle (kTmaOut); unused by the other instantiations.
 template <int BN, int STAGES, int MODE, bool A_MN, bool B_MN, int EPI, bool PAIR,
           bool GATHER = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-            const __grid_constant__ CUtensorMap mapBs, const Params p, int total_hint) {
+            const __grid_constant__ CUtensorMap mapBs, const __grid_constant__ CUtensorMap mapO,
+            const __grid_constant__ CUtensorMap mapO2, const Params p, int total_hint) {
+  constexpr bool kTmaOut = BN == 512 && (EPI == EPI_SWIGLU || EPI == EPI_STORE);
   constexpr int KB = stage_kb<BN, STAGES, MODE, PAIR, GATHER>();
   using S = KernelSmem<BN, STAGES, MODE, PAIR, GATHER>;
   constexpr int BNC = S::BNC;
@@ -1014,7 +1056,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     constexpr int HC = BN / 2;           // columns per warp (plain epilogues)
     constexpr int HJ = BN / 4;           // gate (= up) columns per warp (SwiGLU)
     const uint64_t pol_out = policy_evict_first();
-    const uint32_t stg = base + S::kEpiOff + (warp - 2) * kStgBytes;   // staging tile
+    const uint32_t stg = base + S::kEpiOff + (warp - 2) * S::kStgW;   // staging tile
+    // 512-wide tiles leave the epilogue unoverlapped with the next tile's
+    // main loop: their output blocks go out as TMA stores from two staging
+    // boxes (lane 0 issues and tracks them), which moves the bytes faster
+    // than the warp's own global stores
+    int box = 0;
+    auto tma_out = [&](const float (&v)[32], const CUtensorMap* map, int x, int64_t y) {
+      const uint32_t buf = stg + box * kTmaBox;
+      box ^= 1;
+      if (lane == 0) bulk_wait_read_1();   // the store that last read `buf` is done with it
+      __syncwarp();
+      stage_box_sw64(buf, v);
+      fence_proxy_async();                 // visible to the async proxy
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(map, buf, x, (int)y);
+        bulk_commit();
+      }
+    };
     if constexpr (EPI == EPI_COMBINE1 || EPI == EPI_DX1) {
       // tokens whose slot holds no row (sentinel, dropped): y_t = 0, or
       // dx_t = ds_t . W_r (the router part alone), while the first tile's
@@ -1147,7 +1207,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_ld32(tbase + hh * HC + c, r);
           tmem_wait();
           u2f32(r, v);
-          staged_store32(stg, v, w0 + c, ld, pol_out);
+          if constexpr (kTmaOut) tma_out(v, &mapO, d.n0 + hh * HC + c, row0);
+          else staged_store32(stg, v, w0 + c, ld, pol_out);
         }
       } else if constexpr (EPI == EPI_COMBINE1 || EPI == EPI_DX1) {
         const int col0 = d.n0 + hh * HC;
@@ -1198,11 +1259,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_wait();
           u2f32(rg, ga);
           u2f32(ru, ub);
-          staged_store32(stg, ga, a13 + c, p.ld_out, pol_out);
-          staged_store32(stg, ub, a13 + p.F + c, p.ld_out, pol_out);
+          const int xc = d.n0 + hh * HJ + c;   // column of gate j (up: + F) and of h
+          if constexpr (kTmaOut) {
+            tma_out(ga, &mapO, xc, row0);
+            tma_out(ub, &mapO, p.F + xc, row0);
+          } else {
+            staged_store32(stg, ga, a13 + c, p.ld_out, pol_out);
+            staged_store32(stg, ub, a13 + p.F + c, p.ld_out, pol_out);
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) ga[i] = ga[i] * fast_sigmoid(ga[i]) * ub[i];
-          staged_store32(stg, ga, hr + c, p.ld_out2, pol_out);
+          if constexpr (kTmaOut) tma_out(ga, &mapO2, xc, row0);
+          else staged_store32(stg, ga, hr + c, p.ld_out2, pol_out);
         }
       } else if constexpr (EPI == EPI_F32 || EPI == EPI_WGRAD_F32) {
         const int64_t row = row0 + lane;
@@ -1252,6 +1320,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       }
       if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
     }
+  }
+  if constexpr (kTmaOut) {
+    if (warp >= 2 && lane == 0) bulk_wait_all();   // this warp's output stores are written
   }
   tc_fence_before();
   __syncthreads();

@@ -369,12 +369,38 @@ cudaError_t launch_k(void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&lc, kern, std::forward<A>(args)...);
 }
 
+// Output tensors of the epilogues that store through TMA (512-wide
+// SwiGLU: a13, h; 512-wide plain store: out), see make_store_map.
+struct OutMaps {
+  CUtensorMap o1, o2;
+};
+
+// bf16 tensor [rows][cols] as TMA-store target: box {32, 32}, 64-byte swizzle.
+int make_store_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) { g_last_cuda_error = (int)cudaErrorNotSupported; return MOE_ERR_CUDA; }
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { g_last_cuda_error = (int)cudaErrorInvalidValue; return MOE_ERR_CUDA; }
+  return MOE_OK;
+}
+
 template <int BN, int ST, int MODE, bool AMN, bool BMN, int EPI, bool PAIR, bool GATHER>
 int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
               const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
-              cudaStream_t s) {
+              cudaStream_t s, const OutMaps* om) {
   using S = tc::KernelSmem<BN, ST, MODE, PAIR, GATHER>;
   auto k = tc::gemm_kernel<BN, ST, MODE, AMN, BMN, EPI, PAIR, GATHER>;
+  // the 512-wide SwiGLU and plain-store epilogues write through TMA
+  constexpr bool tma_out = BN == 512 && (EPI == tc::EPI_SWIGLU || EPI == tc::EPI_STORE);
+  if (tma_out && om == nullptr) return MOE_ERR_ARG;
+  const CUtensorMap& o1 = om != nullptr ? om->o1 : a;
+  const CUtensorMap& o2 = om != nullptr ? om->o2 : a;
   MOE_CK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes));
   if constexpr (PAIR) {
     // as many CTA pairs as can be resident at once (one per two SMs of a GPC)
@@ -403,13 +429,13 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
     lc.gridDim = dim3(2 * pairs);
     lc.numAttrs = pdl_enabled() ? 2 : 1;
     prof_begin(s);
-    MOE_CK(cudaLaunchKernelEx(&lc, k, a, b, bs, p, total_hint));
+    MOE_CK(cudaLaunchKernelEx(&lc, k, a, b, bs, o1, o2, p, total_hint));
     MOE_LAUNCHED(s, name);
   } else {
     const int grid = (int)std::min<int64_t>(num_sms(), total_max);
     if (grid <= 0) return MOE_OK;
     prof_begin(s);
-    MOE_CK((launch_k(k, grid, tc::kThreads, S::kBytes, s, a, b, bs, p, total_hint)));
+    MOE_CK((launch_k(k, grid, tc::kThreads, S::kBytes, s, a, b, bs, o1, o2, p, total_hint)));
     MOE_LAUNCHED(s, name);
   }
   return MOE_OK;
@@ -418,48 +444,48 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
 template <int MODE, bool AMN, bool BMN, int EPI, bool PAIR = false, bool GATHER = false>
 int run_tc(int bn, const char* name, const CUtensorMap& a, const CUtensorMap& b,
            const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
-           cudaStream_t s) {
+           cudaStream_t s, const OutMaps* om = nullptr) {
   if constexpr (PAIR) {
     // per CTA: A 16 KB + half of B per stage
     if constexpr (!GATHER) {
       if (bn == 512)   // two stages of two k blocks (tc::stage_kb)
         return launch_tc<512, 2, MODE, AMN, BMN, EPI, true, false>(name, a, b, bs, p, total_max,
-                                                                  total_hint, s);
+                                                                  total_hint, s, om);
     }
     if constexpr (!GATHER) {
       if (bn == 256)   // two k blocks per stage (tc::stage_kb)
         return launch_tc<256, 3, MODE, AMN, BMN, EPI, true, false>(name, a, b, bs, p, total_max,
-                                                                  total_hint, s);
+                                                                  total_hint, s, om);
     }
     if (bn == 256)
       return launch_tc<256, 6, MODE, AMN, BMN, EPI, true, GATHER>(name, a, b, bs, p, total_max,
-                                                                 total_hint, s);
+                                                                 total_hint, s, om);
     if constexpr (!GATHER) {
       if (bn == 128)
         return launch_tc<128, 4, MODE, AMN, BMN, EPI, true, false>(name, a, b, bs, p, total_max,
-                                                                  total_hint, s);
+                                                                  total_hint, s, om);
     }
     if (bn == 128)
       return launch_tc<128, 8, MODE, AMN, BMN, EPI, true, GATHER>(name, a, b, bs, p, total_max,
-                                                                 total_hint, s);
+                                                                 total_hint, s, om);
     return MOE_ERR_ARG;
   } else {
     if (bn == 256)
       return launch_tc<256, 4, MODE, AMN, BMN, EPI, false, GATHER>(name, a, b, bs, p, total_max,
-                                                                  total_hint, s);
+                                                                  total_hint, s, om);
     if constexpr (EPI != tc::EPI_SWIGLU) {
       if (bn == 192)
         return launch_tc<192, 5, MODE, AMN, BMN, EPI, false, GATHER>(name, a, b, bs, p,
-                                                                    total_max, total_hint, s);
+                                                                    total_max, total_hint, s, om);
     }
     if constexpr (!GATHER) {
       if (bn == 128)
         return launch_tc<128, 3, MODE, AMN, BMN, EPI, false, false>(name, a, b, bs, p, total_max,
-                                                                   total_hint, s);
+                                                                   total_hint, s, om);
     }
     if (bn == 128)
       return launch_tc<128, 6, MODE, AMN, BMN, EPI, false, GATHER>(name, a, b, bs, p, total_max,
-                                                                  total_hint, s);
+                                                                  total_hint, s, om);
     return MOE_ERR_ARG;
   }
 }
@@ -1324,7 +1350,8 @@ int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, co
   const int64_t units = pr ? L.tiles_max / 2 : L.tiles_max;
   // gate/up + SwiGLU: A = x_perm [rows, D] (or rows of x [T, D] copied by
   // the GEMM's producer warp: mapA unused); B = w13 [E, 2F, D] K-major
-  const int bn1 = pick_bn(2 * F, mt, true, F, pr, D / 64);
+  // (512-wide tiles load their rows by TMA box only: not with the gather)
+  const int bn1 = pick_bn(2 * F, mt, true, F, pr, gather ? 0 : D / 64);
   MOE_TRY(make_map(&mA, gather ? x : x_perm, 1, gather ? c->T : L.rows_max, D, 128, false));
   // B boxes: the gate / up rows of one MMA block (at most 128 per CTA)
   const uint32_t box1 = (uint32_t)std::min(bn1 / 2, 128);
@@ -1338,10 +1365,13 @@ int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, co
   p.gx = static_cast<const __nv_bfloat16*>(x);
   const char* n1 = "tc_gate_up_swiglu";
   const int64_t tot1 = units * p.nN;
+  OutMaps om1;   // a13 and h as TMA-store targets (512-wide tiles)
+  MOE_TRY(make_store_map(&om1.o1, a13, L.rows_max, 2 * F));
+  MOE_TRY(make_store_map(&om1.o2, h, L.rows_max, F));
   if (pr && gather)
     MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, true, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
   else if (pr)
-    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s, &om1)));
   else if (gather)
     MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, false, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
   else
@@ -1365,9 +1395,12 @@ int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, co
     return run_tc<tc::MODE_ROWS, false, false, tc::EPI_COMBINE1>(
         bn2, n2, mA, mB, mBs, q, units * q.nN, 0, s);
   }
+  OutMaps om2;   // o as TMA-store target (512-wide tiles)
+  MOE_TRY(make_store_map(&om2.o1, o, L.rows_max, D));
+  om2.o2 = om2.o1;
   if (pr)
     return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE, true>(
-        bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
+        bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s, &om2);
   return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE>(
       bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
 }
@@ -1711,9 +1744,13 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
         else
           MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_DX1>(
               bn5, "tc_dgrad_gate_up_dx", mA, mB, mBs, p, units * p.nN, 0, s)));
-      } else if (pr)
+      } else if (pr) {
+        OutMaps om5;   // dX_perm as TMA-store target (512-wide tiles)
+        MOE_TRY(make_store_map(&om5.o1, dXp, L.rows_max, D));
+        om5.o2 = om5.o1;
         MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE, true>(
-            bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s)));
+            bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s, &om5)));
+      }
       else
         MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE>(
             bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s)));
@@ -1722,7 +1759,8 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     // producer warp copies the B rows from x by row_slot; mapB unused)
     const bool pw6 = ((2 * F) % 256) == 0;
     const bool g6 = x_perm == nullptr;
-    const int bn6 = wgrad_bn(pick_bn(D, (int64_t)groups * (2 * F / 128), false, F, pw6, wg_kb), D);
+    const int bn6 =
+        wgrad_bn(pick_bn(D, (int64_t)groups * (2 * F / 128), false, F, pw6, g6 ? 0 : wg_kb), D);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 64, false));
     MOE_TRY(make_map(&mB, g6 ? x : x_perm, 1, g6 ? T : L.rows_max, D, 64, false));
     {
