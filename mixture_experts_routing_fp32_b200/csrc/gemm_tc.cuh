@@ -636,16 +636,18 @@ using KernelSmem = Smem<BN, STAGES, PAIR, stage_kb<BN, STAGES, MODE, PAIR, GATHE
 // by 16-byte cp.async copies issued by the whole producer warp: the A rows
 // of a ROWS tile (gate/up + SwiGLU), or the B rows of a WGRAD k block
 // (gate/up weight gradient); the other operand still arrives by TMA box.
-// mapO / mapO2: the outputs of the 512-wide SwiGLU (a13, h) and plain-store
-// (out) epilogues as 2-D bf16 tensors with 32 x 32 boxes in the 64-byte
-// swizzle (kTmaOut); unused by the other instantiations.
+// mapO / mapO2: the outputs of the 512-wide SwiGLU (a13, h), plain-store
+// (out) and weight-gradient (the routed experts' out as [E * rows, No], the
+// shared expert's out_shared) epilogues as 2-D bf16 tensors with 32 x 32
+// boxes in the 64-byte swizzle (kTmaOut); unused by the other
+// instantiations.
 template <int BN, int STAGES, int MODE, bool A_MN, bool B_MN, int EPI, bool PAIR,
           bool GATHER = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
             const __grid_constant__ CUtensorMap mapBs, const __grid_constant__ CUtensorMap mapO,
             const __grid_constant__ CUtensorMap mapO2, const Params p, int total_hint) {
-  constexpr bool kTmaOut = BN == 512 && (EPI == EPI_SWIGLU || EPI == EPI_STORE);
+  constexpr bool kTmaOut = BN == 512 && (EPI == EPI_SWIGLU || EPI == EPI_STORE || EPI == EPI_WGRAD);
   constexpr int KB = stage_kb<BN, STAGES, MODE, PAIR, GATHER>();
   using S = KernelSmem<BN, STAGES, MODE, PAIR, GATHER>;
   constexpr int BNC = S::BNC;
@@ -1207,8 +1209,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_ld32(tbase + hh * HC + c, r);
           tmem_wait();
           u2f32(r, v);
-          if constexpr (kTmaOut) tma_out(v, &mapO, d.n0 + hh * HC + c, row0);
-          else staged_store32(stg, v, w0 + c, ld, pol_out);
+          if constexpr (kTmaOut && EPI == EPI_STORE) {
+            tma_out(v, &mapO, d.n0 + hh * HC + c, row0);
+          } else if constexpr (kTmaOut) {   // weight gradient: expert d.e's rows
+            if (d.e < p.E) tma_out(v, &mapO, d.n0 + hh * HC + c, d.e * (p.strideCE / p.No) + row0);
+            else tma_out(v, &mapO2, d.n0 + hh * HC + c, row0);
+          } else {
+            staged_store32(stg, v, w0 + c, ld, pol_out);
+          }
         }
       } else if constexpr (EPI == EPI_COMBINE1 || EPI == EPI_DX1) {
         const int col0 = d.n0 + hh * HC;

@@ -370,7 +370,8 @@ cudaError_t launch_k(void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cu
 }
 
 // Output tensors of the epilogues that store through TMA (512-wide
-// SwiGLU: a13, h; 512-wide plain store: out), see make_store_map.
+// SwiGLU: a13, h; plain store: out; weight gradient: the routed experts'
+// [E * rows, cols] and the shared expert's), see make_store_map.
 struct OutMaps {
   CUtensorMap o1, o2;
 };
@@ -396,8 +397,10 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
               cudaStream_t s, const OutMaps* om) {
   using S = tc::KernelSmem<BN, ST, MODE, PAIR, GATHER>;
   auto k = tc::gemm_kernel<BN, ST, MODE, AMN, BMN, EPI, PAIR, GATHER>;
-  // the 512-wide SwiGLU and plain-store epilogues write through TMA
-  constexpr bool tma_out = BN == 512 && (EPI == tc::EPI_SWIGLU || EPI == tc::EPI_STORE);
+  // the 512-wide SwiGLU, plain-store and weight-gradient epilogues write
+  // through TMA
+  constexpr bool tma_out =
+      BN == 512 && (EPI == tc::EPI_SWIGLU || EPI == tc::EPI_STORE || EPI == tc::EPI_WGRAD);
   if (tma_out && om == nullptr) return MOE_ERR_ARG;
   const CUtensorMap& o1 = om != nullptr ? om->o1 : a;
   const CUtensorMap& o2 = om != nullptr ? om->o2 : a;
@@ -1717,9 +1720,13 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       p.out = static_cast<__nv_bfloat16*>(dw_down);
       p.out_shared = static_cast<__nv_bfloat16*>(dw_down_s);
       const int total = p.n_groups * p.nMo * p.nNo;
+      OutMaps om4;   // dW_down as [El * D, F] and the shared expert's [D, F]
+      MOE_TRY(make_store_map(&om4.o1, dw_down, (int64_t)El * D, F));
+      if (c->n_shared) MOE_TRY(make_store_map(&om4.o2, dw_down_s, D, F));
+      else om4.o2 = om4.o1;
       if (pw4)
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, true>(
-            bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1)));
+            bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1, &om4)));
       else
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
             bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1)));
@@ -1774,12 +1781,16 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       p.gx = static_cast<const __nv_bfloat16*>(x);
       const int total = p.n_groups * p.nMo * p.nNo;
       const char* n6 = "tc_wgrad_gate_up";
+      OutMaps om6;   // dW13 as [El * 2F, D] and the shared expert's [2F, D]
+      MOE_TRY(make_store_map(&om6.o1, dw13, (int64_t)El * 2 * F, D));
+      if (c->n_shared) MOE_TRY(make_store_map(&om6.o2, dw13_s, 2 * F, D));
+      else om6.o2 = om6.o1;
       if (pw6 && g6)
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, true, true>(
             bn6, n6, mA, mB, mB, p, total, total, w2)));
       else if (pw6)
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, true>(
-            bn6, n6, mA, mB, mB, p, total, total, w2)));
+            bn6, n6, mA, mB, mB, p, total, total, w2, &om6)));
       else if (g6)
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, false, true>(
             bn6, n6, mA, mB, mB, p, total, total, w2)));
