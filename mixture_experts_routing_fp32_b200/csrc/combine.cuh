@@ -376,7 +376,8 @@ struct RouterBwdArgs {
   int seq_len;
   const float* seq_f;
   // bf16 splits of ds for the tensor-core router products (or null):
-  // dsf [T, 3 Ep] = (hi | mid | lo), dsb [T, 3 Ep] = (hi | hi | mid)
+  // dsf [T, 3 Ep] = (hi | mid | lo), dsb [T, 3 Ep] = (hi | hi | mid) (or
+  // null: the router part of dx is formed on CUDA cores)
   __nv_bfloat16* dsf;
   __nv_bfloat16* dsb;
   int Ep;
@@ -529,12 +530,16 @@ router_bwd_kernel(RouterBwdArgs a) {
           __nv_bfloat16 hi, mid, lo;
           split3_bf16(ds[i], hi, mid, lo);
           a.dsf[b + e] = hi; a.dsf[b + a.Ep + e] = mid; a.dsf[b + 2 * a.Ep + e] = lo;
-          a.dsb[b + e] = hi; a.dsb[b + a.Ep + e] = hi; a.dsb[b + 2 * a.Ep + e] = mid;
+          if (a.dsb != nullptr) {
+            a.dsb[b + e] = hi; a.dsb[b + a.Ep + e] = hi; a.dsb[b + 2 * a.Ep + e] = mid;
+          }
         }
       }
       for (int e = E + lane; e < a.Ep; e += 32) {
         a.dsf[b + e] = z; a.dsf[b + a.Ep + e] = z; a.dsf[b + 2 * a.Ep + e] = z;
-        a.dsb[b + e] = z; a.dsb[b + a.Ep + e] = z; a.dsb[b + 2 * a.Ep + e] = z;
+        if (a.dsb != nullptr) {
+          a.dsb[b + e] = z; a.dsb[b + a.Ep + e] = z; a.dsb[b + 2 * a.Ep + e] = z;
+        }
       }
     }
     if (a.dg_out != nullptr && lane < K) {
@@ -881,7 +886,7 @@ dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
   }
   __syncthreads();
   const int d = c0 + lane * 8;
-  if (d >= D) return;                      // no barrier below
+  const bool live = d < D;                 // (every lane takes part in the shuffles)
   const int64_t shared0 = n_shared ? (int64_t)offsets[El] : -1;
   const int64_t stride = (int64_t)gridDim.y * 8;
   auto one = [&](int64_t t) {
@@ -892,15 +897,15 @@ dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
     for (int k = 0; k <= KT; ++k) {
       const int64_t row = k < KT ? (int64_t)__shfl_sync(0xffffffffu, my_row, k)
                                  : (n_shared ? shared0 + t : -1);
-      r[k] = row >= 0 ? *reinterpret_cast<const uint4*>(dXp + row * D + d)
-                      : make_uint4(0, 0, 0, 0);
+      r[k] = (live && row >= 0) ? *reinterpret_cast<const uint4*>(dXp + row * D + d)
+                                : make_uint4(0, 0, 0, 0);
     }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int e = 0; e < kE; ++e) {
       const float de = __shfl_sync(0xffffffffu, my_ds, e);
       if (e < E) {
-        const float4 w0 = *reinterpret_cast<const float4*>(&ws[e][lane * 8]);
+        const float4 w0 = *reinterpret_cast<const float4*>(&ws[e][lane * 8]);   // 0 if !live
         const float4 w1 = *reinterpret_cast<const float4*>(&ws[e][lane * 8 + 4]);
         acc[0] = fmaf(de, w0.x, acc[0]); acc[1] = fmaf(de, w0.y, acc[1]);
         acc[2] = fmaf(de, w0.z, acc[2]); acc[3] = fmaf(de, w0.w, acc[3]);
@@ -915,7 +920,7 @@ dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += v[i];
     }
-    store8(dx + t * D + d, acc);
+    if (live) store8(dx + t * D + d, acc);
   };
   int64_t t = (int64_t)blockIdx.y * 8 + warp;
   for (; t + stride < Tn; t += 2 * stride) {

@@ -183,6 +183,20 @@ int64_t capacity_of(const moe_config_t* c);
 // when the expert GEMMs do and E >= 8; below that the SIMT kernels are as
 // fast.  Ep = E rounded up to 64 (split width).
 bool router_tc(const moe_config_t* c) { return use_tc(c) && c->E >= 8; }
+// The backward's router part of dx on CUDA cores inside the unpermute-sum
+// (bf16 token choice, E <= 8, K in {1, 2, 4, 8}); MOE_ROUTER_DX_TC=1 keeps
+// the tensor-core product for E = 8 (for cross-checks).
+bool small_router_dx(const moe_config_t* c) {
+  static const bool force_tc = [] {
+    const char* v = std::getenv("MOE_ROUTER_DX_TC");
+    return v != nullptr && v[0] == '1';
+  }();
+  return !force_tc && c->dtype == MOE_BF16 && !c->expert_choice && c->E <= 8 &&
+         (c->K == 1 || c->K == 2 || c->K == 4 || c->K == 8);
+}
+bool router_dx_tc(const moe_config_t* c) {
+  return router_tc(c) && (c->expert_choice || !small_router_dx(c));
+}
 // Token-choice routing inside the tensor-core logits kernel: up to 64
 // experts, no group limit, K in {1, 2, 4, 8} (MOE_ROUTER_FUSED=0: for
 // E >= 8 the partial-logit GEMM and a separate routing kernel instead, for
@@ -275,11 +289,13 @@ Layout layout_of(const moe_config_t* c) {
     L.off_wf = take((size_t)3 * L.Ep * c->D * 2);
   }
   if (router_tc(c)) {
-    L.off_wb = take((size_t)3 * L.Ep * c->D * 2);
     L.off_rparts = take((size_t)c->T * 3 * L.Ep * 4);
     L.off_dsf = take((size_t)c->T * 3 * L.Ep * 2);
-    L.off_dsb = take((size_t)c->T * 3 * L.Ep * 2);
     L.off_dwr3 = take((size_t)3 * L.Ep * c->D * 4);
+  }
+  if (router_dx_tc(c)) {   // the router part of dx on tensor cores
+    L.off_wb = take((size_t)3 * L.Ep * c->D * 2);
+    L.off_dsb = take((size_t)c->T * 3 * L.Ep * 2);
     L.off_rdx = take((size_t)c->T * c->D * 4);
   }
   if (c->seq_len > 0) {
@@ -1571,6 +1587,11 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   // cores from E >= 8 (measured faster than the CUDA-core forms at E = 8)
   const bool rtc = router_tc(c);
   const bool dx1 = token_epilogues(c) && !rtc;   // dx from the dgrad gate/up epilogue
+  // the router part of dx from the tensor-core product (fp32 R [T, D], then
+  // a gather-sum) unless E <= 8 with bf16 token choice: there the
+  // unpermute-sum kernel forms ds . W_r itself in fp32 (8 FMAs per element)
+  // and the [T, D] fp32 round trip disappears
+  const bool dx_tc = router_dx_tc(c);
 
   // 1. per row: gate gradient dg = <o, dy>, and dO = g * dy (token order:
   // each token's dy row read once for all its slots)
@@ -1638,7 +1659,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     }
     if (rtc) {
       a.dsf = wsp<__nv_bfloat16>(ws, L.off_dsf);
-      a.dsb = wsp<__nv_bfloat16>(ws, L.off_dsb);
+      a.dsb = dx_tc ? wsp<__nv_bfloat16>(ws, L.off_dsb) : nullptr;
       a.Ep = (int)L.Ep;
     }
     const int grid = grid_for(T);
@@ -1668,7 +1689,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     else MOE_CK((launch_k(router_bwd_kernel<16>, grid, 256, 0, s, a)));
     MOE_LAUNCHED(s, "router_bwd");
     }
-    if (rtc) {
+    if (dx_tc) {
       // (hi; mid; hi) split of W_r for the router part of dx
       prof_begin(s);
       MOE_CK((launch_k(split_w_kernel, grid_for(L.Ep * D / 32), 256, 0, s, w_r, E, (int)L.Ep, D,
@@ -1904,7 +1925,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
                        static_cast<const float*>(dXp), slot_row, offsets, c->n_shared, T, D, E,
                        static_cast<float*>(dx))));
     MOE_LAUNCHED(s, "dx_unpermute_sum");
-  } else if (rtc) {
+  } else if (dx_tc) {
     const int64_t n3 = 3 * L.Ep;
     float* R = wsp<float>(ws, L.off_rdx);
     CUtensorMap mA, mB;
