@@ -986,15 +986,23 @@ dx_sum_kernel(const float* __restrict__ R, const __nv_bfloat16* __restrict__ dXp
 }
 
 // dW_r from the three partial products of the tensor-core path
-// (part [3 Ep, D]: ds_hi^T x | ds_mid^T x | ds_lo^T x), summed in that order.
+// (part [3 Ep, D]: ds_hi^T x | ds_mid^T x | ds_lo^T x), summed in that order,
+// for each of the n_split token ranges (partials n_split apart, 3 Ep D
+// elements each), the ranges added in order.
 __global__ void __launch_bounds__(256)
-dwr_reduce3_kernel(const float* __restrict__ part, int E, int Ep, int D,
+dwr_reduce3_kernel(const float* __restrict__ part, int E, int Ep, int D, int n_split,
                    float* __restrict__ dw_r) {
   pdl_begin();
-  const int64_t n = (int64_t)E * D, stride = (int64_t)Ep * D;
+  const int64_t n = (int64_t)E * D, stride = (int64_t)Ep * D, sstride = 3 * stride;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    dw_r[i] = (part[i] + part[stride + i]) + part[2 * stride + i];
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float acc = (part[i] + part[stride + i]) + part[2 * stride + i];
+    for (int s = 1; s < n_split; ++s) {
+      const float* q = part + s * sstride;
+      acc += (q[i] + q[stride + i]) + q[2 * stride + i];
+    }
+    dw_r[i] = acc;
+  }
 }
 
 }  // namespace moe

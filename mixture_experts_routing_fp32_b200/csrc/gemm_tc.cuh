@@ -75,7 +75,10 @@ struct Params {
   __nv_bfloat16* out_shared;               // WGRAD: shared group output
   // dense variants
   int dense_m;                 // ROWS: > 0 = one group of dense_m rows, no tile map
-  int dense_rows;              // WGRAD: > 0 = one group of dense_rows rows
+  int dense_rows;              // WGRAD: > 0 = dense_rows rows, no groups of experts:
+  int dense_split;             //   group g takes rows [g, g + 1) * dense_split (a K
+                               //   split, multiple of 64; 0 = one group of all rows)
+                               //   and writes its partial at out_f32 + g * strideCE
   int m_limit;                 // WGRAD_F32: output rows
   float* out_f32; int64_t ld_f32;          // F32 epilogues
   // gathered rows (the GATHER kernels copy token rows of x instead of
@@ -582,8 +585,11 @@ __device__ __forceinline__ Tile decode(int t, const Params& p, int rank, int n_m
     d.e = g;
     d.m0 = (rem / p.nNo) * MU + rank * BM;
     d.n0 = (rem % p.nNo) * BN;
-    d.row0 = p.dense_rows > 0 ? 0 : p.offsets[g];
-    const int rows = p.dense_rows > 0 ? p.dense_rows : g < p.E ? p.kept[g] : p.T;
+    const int split = p.dense_split > 0 ? p.dense_split : p.dense_rows;
+    d.row0 = p.dense_rows > 0 ? g * split : p.offsets[g];
+    const int rows = p.dense_rows > 0 ? min(split, p.dense_rows - d.row0)
+                     : g < p.E           ? p.kept[g]
+                                         : p.T;
     d.nk = (rows + BK - 1) / BK;
   }
   return d;
@@ -1283,7 +1289,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       } else if constexpr (EPI == EPI_F32 || EPI == EPI_WGRAD_F32) {
         const int64_t row = row0 + lane;
         const bool rv = row < (EPI == EPI_F32 ? (int64_t)p.dense_m : (int64_t)p.m_limit);
-        float* dst = p.out_f32 + row * p.ld_f32 + d.n0 + hh * HC;
+        float* dst = p.out_f32 + row * p.ld_f32 + d.n0 + hh * HC +
+                     (EPI == EPI_WGRAD_F32 ? (int64_t)d.e * p.strideCE : 0);   // K-split partial
 #pragma unroll
         for (int c = 0; c < HC; c += 32) {
           uint32_t r[32];

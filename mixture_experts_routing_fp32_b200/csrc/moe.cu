@@ -210,6 +210,18 @@ bool router_fused_tc(const moe_config_t* c) {
          (c->K == 1 || c->K == 2 || c->K == 4 || c->K == 8);
 }
 int64_t router_ep(const moe_config_t* c) { return (c->E + 63) / 64 * 64; }
+// Token ranges of the tensor-core dW_r product (a K split): with few output
+// tiles (3 Ep / 128 x D / 128, E <= 64 and a narrow D) up to four ranges,
+// so about one tile per SM of the 148 runs; the partials are summed in
+// range order.  Returns the rows per range (a multiple of 64).
+int dwr_split_rows(const moe_config_t* c) {
+  const int64_t tiles = ceil_div(3 * router_ep(c), 128) * ceil_div(c->D, 128);
+  const int64_t want = std::max<int64_t>(1, std::min<int64_t>(4, 148 / tiles));
+  return (int)round_up(ceil_div(c->T, want), 64);
+}
+int dwr_splits(const moe_config_t* c) {
+  return (int)ceil_div(c->T, dwr_split_rows(c));
+}
 
 // Row GEMMs run on CTA pairs (two SMs share each 256-row MMA) when experts
 // hold enough rows that aligning their segments to 256 rows wastes little
@@ -291,7 +303,7 @@ Layout layout_of(const moe_config_t* c) {
   if (router_tc(c)) {
     L.off_rparts = take((size_t)c->T * 3 * L.Ep * 4);
     L.off_dsf = take((size_t)c->T * 3 * L.Ep * 2);
-    L.off_dwr3 = take((size_t)3 * L.Ep * c->D * 4);
+    L.off_dwr3 = take((size_t)dwr_splits(c) * 3 * L.Ep * c->D * 4);
   }
   if (router_dx_tc(c)) {   // the router part of dx on tensor cores
     L.off_wb = take((size_t)3 * L.Ep * c->D * 2);
@@ -1853,16 +1865,18 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     const int64_t nmo = ceil_div(n3, kRowTile);
     const int bn = pick_bn(D, nmo, false, 0, false);
     tc::Params p{};
-    p.E = 1; p.n_groups = 1; p.dense_rows = T; p.T = T;
+    p.E = 1; p.dense_rows = T; p.T = T;
+    p.n_groups = dwr_splits(c); p.dense_split = dwr_split_rows(c);   // token ranges
+    p.strideCE = n3 * D;                                            // partial stride
     p.nMo = (int)nmo; p.nNo = D / bn; p.No = D;
     p.m_limit = (int)n3;
     p.out_f32 = wsp<float>(ws, L.off_dwr3); p.ld_f32 = D;
-    const int total = p.nMo * p.nNo;
+    const int total = p.n_groups * p.nMo * p.nNo;
     MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD_F32>(
         bn, "router_dw_tc", mA, mB, mB, p, total, total, s)));
     prof_begin(s);
     MOE_CK((launch_k(dwr_reduce3_kernel, grid_for((int64_t)E * D / 32), 256, 0, s,
-                     wsp<const float>(ws, L.off_dwr3), E, (int)L.Ep, D, dw_r)));
+                     wsp<const float>(ws, L.off_dwr3), E, (int)L.Ep, D, dwr_splits(c), dw_r)));
     MOE_LAUNCHED(s, "router_dw_reduce3");
   } else {
     cudaStream_t s = r;
