@@ -483,11 +483,10 @@ __device__ __forceinline__ void staged_store32_pk(uint32_t stg, const uint4 (&pk
 // j ^ ((r >> 1) & 3)), so the 16-byte stores of any 8 consecutive lanes
 // fall in distinct banks.  Lane r writes row r; `buf` is 512-byte aligned.
 constexpr int kTmaBox = 32 * 64;
-__device__ __forceinline__ void stage_box_sw64(uint32_t buf, const float (&v)[32]) {
+__device__ __forceinline__ void stage_box_sw64(uint32_t buf, const uint4 (&u)[4]) {
   const int r = threadIdx.x & 31;
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    sts128(buf + r * 64 + ((j ^ ((r >> 1) & 3)) << 4), pack8_bf16(v + 8 * j));
+  for (int j = 0; j < 4; ++j) sts128(buf + r * 64 + ((j ^ ((r >> 1) & 3)) << 4), u[j]);
 }
 
 // staged_store32 to scattered rows: block row i goes to w0 + tok_i * ld,
@@ -612,10 +611,11 @@ struct Smem {
   static constexpr int kBars = (3 * STAGES + 2 * NACC + 1) * 8;
   // token table of the gathering producer (128 rows)
   static constexpr int kTokOff = STAGES * kStage + kBars + 16;
-  // epilogue staging per epilogue warp: a 2.5 KB tile, or for the
-  // 512-wide tiles (whose epilogues store through TMA) two 2 KB boxes;
-  // 512-byte aligned (the boxes' swizzle)
-  static constexpr int kStgW = BN == 512 ? 2 * kTmaBox : kStgBytes;
+  // epilogue staging per epilogue warp: two 2 KB boxes for the epilogues
+  // that store through TMA, a 2.5 KB tile for the others (the 192-wide
+  // tiles, whose five stages leave no room for the boxes); 512-byte aligned
+  // (the boxes' swizzle)
+  static constexpr int kStgW = BN == 192 ? kStgBytes : 2 * kTmaBox;
   static constexpr int kEpiOff = (kTokOff + 512 + 511) / 512 * 512;
   static constexpr int kBytes = 1024 + kEpiOff + kEpiWarps * kStgW;
   static_assert(kBytes <= 232448, "shared memory per CTA");
@@ -642,18 +642,18 @@ using KernelSmem = Smem<BN, STAGES, PAIR, stage_kb<BN, STAGES, MODE, PAIR, GATHE
 // by 16-byte cp.async copies issued by the whole producer warp: the A rows
 // of a ROWS tile (gate/up + SwiGLU), or the B rows of a WGRAD k block
 // (gate/up weight gradient); the other operand still arrives by TMA box.
-// mapO / mapO2: the outputs of the 512-wide SwiGLU (a13, h), plain-store
-// (out) and weight-gradient (the routed experts' out as [E * rows, No], the
-// shared expert's out_shared) epilogues as 2-D bf16 tensors with 32 x 32
-// boxes in the 64-byte swizzle (kTmaOut); unused by the other
-// instantiations.
+// mapO / mapO2: the outputs of the SwiGLU (a13, h), plain-store (out) and
+// weight-gradient (the routed experts' out as [E * rows, No], the shared
+// expert's out_shared) epilogues as 2-D bf16 tensors with 32 x 32 boxes in
+// the 64-byte swizzle (kTmaOut: every tile width but 192); unused by the
+// other instantiations.
 template <int BN, int STAGES, int MODE, bool A_MN, bool B_MN, int EPI, bool PAIR,
           bool GATHER = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
             const __grid_constant__ CUtensorMap mapBs, const __grid_constant__ CUtensorMap mapO,
             const __grid_constant__ CUtensorMap mapO2, const Params p, int total_hint) {
-  constexpr bool kTmaOut = BN == 512 && (EPI == EPI_SWIGLU || EPI == EPI_STORE || EPI == EPI_WGRAD);
+  constexpr bool kTmaOut = BN != 192 && (EPI == EPI_SWIGLU || EPI == EPI_STORE || EPI == EPI_WGRAD);
   constexpr int KB = stage_kb<BN, STAGES, MODE, PAIR, GATHER>();
   using S = KernelSmem<BN, STAGES, MODE, PAIR, GATHER>;
   constexpr int BNC = S::BNC;
@@ -1065,22 +1065,40 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     constexpr int HJ = BN / 4;           // gate (= up) columns per warp (SwiGLU)
     const uint64_t pol_out = policy_evict_first();
     const uint32_t stg = base + S::kEpiOff + (warp - 2) * S::kStgW;   // staging tile
-    // 512-wide tiles leave the epilogue unoverlapped with the next tile's
-    // main loop: their output blocks go out as TMA stores from two staging
-    // boxes (lane 0 issues and tracks them), which moves the bytes faster
-    // than the warp's own global stores
+    // Output blocks (32 rows x 32 columns, bf16) go out as TMA stores from
+    // two staging boxes (lane 0 issues and tracks them): they move the bytes
+    // faster than the warp's own global stores, which shortens the 512-wide
+    // tiles' unoverlapped epilogue and frees the others' epilogue warps
+    // sooner.  u: this lane's row of the block, packed.
     int box = 0;
-    auto tma_out = [&](const float (&v)[32], const CUtensorMap* map, int x, int64_t y) {
+    auto tma_out_pk = [&](const uint4 (&u)[4], const CUtensorMap* map, int x, int64_t y) {
       const uint32_t buf = stg + box * kTmaBox;
       box ^= 1;
       if (lane == 0) bulk_wait_read_1();   // the store that last read `buf` is done with it
       __syncwarp();
-      stage_box_sw64(buf, v);
+      stage_box_sw64(buf, u);
       fence_proxy_async();                 // visible to the async proxy
       __syncwarp();
       if (lane == 0) {
         tma_store_2d(map, buf, x, (int)y);
         bulk_commit();
+      }
+    };
+    auto tma_out = [&](const float (&v)[32], const CUtensorMap* map, int x, int64_t y) {
+      uint4 u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) u[j] = pack8_bf16(v + 8 * j);
+      tma_out_pk(u, map, x, y);
+    };
+    // a plain-store / weight-gradient block at column x of this warp's rows
+    // (weight gradient: expert d.e's rows of the stacked routed experts, or
+    // the shared expert's tensor)
+    auto tma_out_tile = [&](const Tile& d, const uint4 (&u)[4], int x, int64_t row0) {
+      if constexpr (EPI == EPI_WGRAD) {
+        if (d.e < p.E) tma_out_pk(u, &mapO, x, d.e * (p.strideCE / p.No) + row0);
+        else tma_out_pk(u, &mapO2, x, row0);
+      } else {
+        tma_out_pk(u, &mapO, x, row0);
       }
     };
     if constexpr (EPI == EPI_COMBINE1 || EPI == EPI_DX1) {
@@ -1194,7 +1212,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           else mbar_arrive_remote(mapa(acce_bar(acc), 0));   // the leader's barrier
         }
 #pragma unroll
-        for (int c = 0; c < HC; c += 32) staged_store32_pk(stg, pk[c / 32], w0 + c, ld, pol_out);
+        for (int c = 0; c < HC; c += 32) {
+          if constexpr (kTmaOut) tma_out_tile(d, pk[c / 32], d.n0 + hh * HC + c, row0);
+          else staged_store32_pk(stg, pk[c / 32], w0 + c, ld, pol_out);
+        }
         if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
         continue;
       } else if constexpr (EPI == EPI_STORE || EPI == EPI_WGRAD) {
@@ -1215,11 +1236,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_ld32(tbase + hh * HC + c, r);
           tmem_wait();
           u2f32(r, v);
-          if constexpr (kTmaOut && EPI == EPI_STORE) {
-            tma_out(v, &mapO, d.n0 + hh * HC + c, row0);
-          } else if constexpr (kTmaOut) {   // weight gradient: expert d.e's rows
-            if (d.e < p.E) tma_out(v, &mapO, d.n0 + hh * HC + c, d.e * (p.strideCE / p.No) + row0);
-            else tma_out(v, &mapO2, d.n0 + hh * HC + c, row0);
+          if constexpr (kTmaOut) {
+            uint4 u[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) u[j] = pack8_bf16(v + 8 * j);
+            tma_out_tile(d, u, d.n0 + hh * HC + c, row0);
           } else {
             staged_store32(stg, v, w0 + c, ld, pol_out);
           }

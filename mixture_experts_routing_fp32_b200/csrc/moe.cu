@@ -397,9 +397,9 @@ cudaError_t launch_k(void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&lc, kern, std::forward<A>(args)...);
 }
 
-// Output tensors of the epilogues that store through TMA (512-wide
-// SwiGLU: a13, h; plain store: out; weight gradient: the routed experts'
-// [E * rows, cols] and the shared expert's), see make_store_map.
+// Output tensors of the epilogues that store through TMA (SwiGLU: a13, h;
+// plain store: out; weight gradient: the routed experts' [E * rows, cols]
+// and the shared expert's), see make_store_map.
 struct OutMaps {
   CUtensorMap o1, o2;
 };
@@ -425,10 +425,10 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
               cudaStream_t s, const OutMaps* om) {
   using S = tc::KernelSmem<BN, ST, MODE, PAIR, GATHER>;
   auto k = tc::gemm_kernel<BN, ST, MODE, AMN, BMN, EPI, PAIR, GATHER>;
-  // the 512-wide SwiGLU, plain-store and weight-gradient epilogues write
-  // through TMA
+  // the SwiGLU, plain-store and weight-gradient epilogues write through TMA
+  // (all tile widths but 192)
   constexpr bool tma_out =
-      BN == 512 && (EPI == tc::EPI_SWIGLU || EPI == tc::EPI_STORE || EPI == tc::EPI_WGRAD);
+      BN != 192 && (EPI == tc::EPI_SWIGLU || EPI == tc::EPI_STORE || EPI == tc::EPI_WGRAD);
   if (tma_out && om == nullptr) return MOE_ERR_ARG;
   const CUtensorMap& o1 = om != nullptr ? om->o1 : a;
   const CUtensorMap& o2 = om != nullptr ? om->o2 : a;
@@ -1396,17 +1396,17 @@ int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, co
   p.gx = static_cast<const __nv_bfloat16*>(x);
   const char* n1 = "tc_gate_up_swiglu";
   const int64_t tot1 = units * p.nN;
-  OutMaps om1;   // a13 and h as TMA-store targets (512-wide tiles)
+  OutMaps om1;   // a13 and h as TMA-store targets
   MOE_TRY(make_store_map(&om1.o1, a13, L.rows_max, 2 * F));
   MOE_TRY(make_store_map(&om1.o2, h, L.rows_max, F));
   if (pr && gather)
-    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, true, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, true, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s, &om1)));
   else if (pr)
     MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s, &om1)));
   else if (gather)
-    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, false, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU, false, true>(bn1, n1, mA, mB, mBs, p, tot1, 0, s, &om1)));
   else
-    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU>(bn1, n1, mA, mB, mBs, p, tot1, 0, s)));
+    MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_SWIGLU>(bn1, n1, mA, mB, mBs, p, tot1, 0, s, &om1)));
   // down: A = h [rows, F]; B = w_down [E, D, F] K-major (a pair CTA loads
   // half of the BN rows)
   const int bn2 = pick_bn(D, mt, false, F, pr, F / 64);
@@ -1426,14 +1426,14 @@ int expert_ffn_tc(const moe_config_t* c, const Layout& L, const void* x_perm, co
     return run_tc<tc::MODE_ROWS, false, false, tc::EPI_COMBINE1>(
         bn2, n2, mA, mB, mBs, q, units * q.nN, 0, s);
   }
-  OutMaps om2;   // o as TMA-store target (512-wide tiles)
+  OutMaps om2;   // o as TMA-store target
   MOE_TRY(make_store_map(&om2.o1, o, L.rows_max, D));
   om2.o2 = om2.o1;
   if (pr)
     return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE, true>(
         bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s, &om2);
   return run_tc<tc::MODE_ROWS, false, false, tc::EPI_STORE>(
-      bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s);
+      bn2, "tc_down", mA, mB, mBs, q, units * q.nN, 0, s, &om2);
 }
 
 // One slot per token and no shared expert: the combine and the
@@ -1762,7 +1762,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
             bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1, &om4)));
       else
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-            bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1)));
+            bn4, "tc_wgrad_down", mA, mB, mB, p, total, total, w1, &om4)));
     }
     // 5. dgrad gate/up: dX_perm = dA13 . w13[e]; with one slot per token
     // (no shared expert, CUDA-core router term) the epilogue writes dx
@@ -1784,16 +1784,17 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
         else
           MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_DX1>(
               bn5, "tc_dgrad_gate_up_dx", mA, mB, mBs, p, units * p.nN, 0, s)));
-      } else if (pr) {
-        OutMaps om5;   // dX_perm as TMA-store target (512-wide tiles)
+      } else {
+        OutMaps om5;   // dX_perm as TMA-store target
         MOE_TRY(make_store_map(&om5.o1, dXp, L.rows_max, D));
         om5.o2 = om5.o1;
-        MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE, true>(
-            bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s, &om5)));
+        if (pr)
+          MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE, true>(
+              bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s, &om5)));
+        else
+          MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE>(
+              bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s, &om5)));
       }
-      else
-        MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_STORE>(
-            bn5, "tc_dgrad_gate_up", mA, mB, mBs, p, units * p.nN, 0, s)));
     }
     // 6. wgrad gate/up: dW13[e] = dA13^T x_perm (x_perm == nullptr: the
     // producer warp copies the B rows from x by row_slot; mapB unused)
@@ -1820,16 +1821,16 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       else om6.o2 = om6.o1;
       if (pw6 && g6)
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, true, true>(
-            bn6, n6, mA, mB, mB, p, total, total, w2)));
+            bn6, n6, mA, mB, mB, p, total, total, w2, &om6)));
       else if (pw6)
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, true>(
             bn6, n6, mA, mB, mB, p, total, total, w2, &om6)));
       else if (g6)
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD, false, true>(
-            bn6, n6, mA, mB, mB, p, total, total, w2)));
+            bn6, n6, mA, mB, mB, p, total, total, w2, &om6)));
       else
         MOE_TRY((run_tc<tc::MODE_WGRAD, true, true, tc::EPI_WGRAD>(
-            bn6, n6, mA, mB, mB, p, total, total, w2)));
+            bn6, n6, mA, mB, mB, p, total, total, w2, &om6)));
     }
   } else {
     auto go = [&](auto tag) -> int {
