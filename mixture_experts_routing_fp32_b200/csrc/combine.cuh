@@ -864,70 +864,138 @@ bias_update_kernel(const int32_t* __restrict__ counts, int E, float gamma,
 
 // dx for few experts (E <= 8, bf16): dx_t = sum_e ds[t,e] W_r[e,:] (e
 // ascending, fp32) + sum_{k kept} dX_perm[row(t,k),:] (k ascending) + the
-// shared row.  Block (c, g) owns the 256-column slice c (8 columns per
-// lane) and token group g: it stages that slice of W_r in shared memory
-// once, then each warp takes one token at a time (two in flight), so the
-// router term costs no global traffic beyond ds and every warp keeps few
-// registers (full occupancy: many row loads in flight per SM).
+// shared row.  A block has 16 warps, one per 256-column slice of the row (8
+// columns per lane), and walks its token group; each lane keeps its 8
+// columns of every expert's W_r row in registers for the whole launch.  The
+// 16 warps take the same tokens in the same order, so the slices of one
+// routed row are read close together in time (whole rows, as DRAM pages
+// like).  A warp streams its tokens in stages of NB tokens through a ring
+// of stages in shared memory filled by cp.async (16 bytes per lane per
+// routed row, 4 bytes per ds value, zero-filled for dropped and sentinel
+// slots); the slot rows of the stage issued next are loaded one iteration
+// ahead.
 template <int KT>
-__global__ void __launch_bounds__(256)
+struct DxRing {
+  static constexpr int NB = KT >= 4 ? 1 : 4 / KT;      // tokens per stage
+  static constexpr int S = KT == 8 ? 2 : 4;             // stages per warp
+  static constexpr int kRows = NB * KT * 512;           // routed rows, 16 B per lane
+  static constexpr int kStage = kRows + NB * 8 * 4;     // + ds [NB][E <= 8] fp32
+  static constexpr int kWarps = 16;
+  static constexpr int kBytes = kWarps * S * kStage;
+};
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void cp_async_zfill(uint32_t dst, const void* src, int bytes, bool valid) {
+  if (bytes == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(valid ? 16 : 0) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+                 "r"(valid ? 4 : 0) : "memory");
+}
+template <int KT>
+__global__ void __launch_bounds__(512, 1)
 dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
                 const __nv_bfloat16* __restrict__ dXp, const int32_t* __restrict__ slot_row,
                 const int32_t* __restrict__ offsets, int n_shared, int Tn, int D, int E, int El,
                 __nv_bfloat16* __restrict__ dx) {
   pdl_begin();
-  constexpr int kE = 8;
-  __shared__ __align__(16) float ws[kE][256];
+  using R = DxRing<KT>;
+  constexpr int kE = 8, NB = R::NB, S = R::S;
+  extern __shared__ __align__(16) uint8_t dx_ring[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c0 = blockIdx.x * 256;
-  for (int i = threadIdx.x; i < kE * 256; i += 256) {
-    const int e = i / 256, col = c0 + (i & 255);
-    ws[e][i & 255] = (e < E && col < D) ? w_r[(int64_t)e * D + col] : 0.f;
+  const int slice = blockIdx.x * R::kWarps + warp;
+  if (slice * 256 >= D) return;            // a whole warp past the row (no block barrier)
+  const int d = slice * 256 + lane * 8;
+  const bool live = d < D;                 // (every lane of the warp takes part in its shuffles)
+  float w[kE][8];
+#pragma unroll
+  for (int e = 0; e < kE; ++e) {
+    if (live && e < E) {
+      load8(w_r + (int64_t)e * D + d, w[e]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[e][i] = 0.f;
+    }
   }
-  __syncthreads();
-  const int d = c0 + lane * 8;
-  const bool live = d < D;                 // (every lane takes part in the shuffles)
   const int64_t shared0 = n_shared ? (int64_t)offsets[El] : -1;
-  const int64_t stride = (int64_t)gridDim.y * 8;
-  auto one = [&](int64_t t) {
-    const int32_t my_row = lane < KT ? slot_row[t * KT + lane] : -1;
-    const float my_ds = lane < E ? ds[t * E + lane] : 0.f;
-    uint4 r[KT + 1];
-#pragma unroll
-    for (int k = 0; k <= KT; ++k) {
-      const int64_t row = k < KT ? (int64_t)__shfl_sync(0xffffffffu, my_row, k)
-                                 : (n_shared ? shared0 + t : -1);
-      r[k] = (live && row >= 0) ? *reinterpret_cast<const uint4*>(dXp + row * D + d)
-                                : make_uint4(0, 0, 0, 0);
-    }
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int e = 0; e < kE; ++e) {
-      const float de = __shfl_sync(0xffffffffu, my_ds, e);
-      if (e < E) {
-        const float4 w0 = *reinterpret_cast<const float4*>(&ws[e][lane * 8]);   // 0 if !live
-        const float4 w1 = *reinterpret_cast<const float4*>(&ws[e][lane * 8 + 4]);
-        acc[0] = fmaf(de, w0.x, acc[0]); acc[1] = fmaf(de, w0.y, acc[1]);
-        acc[2] = fmaf(de, w0.z, acc[2]); acc[3] = fmaf(de, w0.w, acc[3]);
-        acc[4] = fmaf(de, w1.x, acc[4]); acc[5] = fmaf(de, w1.y, acc[5]);
-        acc[6] = fmaf(de, w1.z, acc[6]); acc[7] = fmaf(de, w1.w, acc[7]);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k <= KT; ++k) {
-      float v[8];
-      bf16x8_to_f32(r[k], v);   // absent rows were loaded as zeros
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += v[i];
-    }
-    if (live) store8(dx + t * D + d, acc);
+  const int64_t stride = gridDim.y;
+  const int64_t first = blockIdx.y;                            // this block's tokens:
+  const int64_t nt = first < Tn ? (Tn - 1 - first) / stride + 1 : 0;   // first + n stride
+  const int64_t nst = (nt + NB - 1) / NB;                      // stages
+  const uint32_t ring = smem_addr(dx_ring) + warp * S * R::kStage;
+  // lane l < NB K: the row of slot l % K of the stage's token l / K
+  auto stage_row = [&](int64_t st) -> int32_t {
+    const int64_t n = st * NB + lane / KT;
+    return (st < nst && lane < NB * KT && n < nt)
+               ? slot_row[(first + n * stride) * KT + lane % KT] : -1;
   };
-  int64_t t = (int64_t)blockIdx.y * 8 + warp;
-  for (; t + stride < Tn; t += 2 * stride) {
-    one(t);
-    one(t + stride);
+  auto issue = [&](int64_t st, int32_t my_row) {
+    const uint32_t buf = ring + (uint32_t)(st % S) * R::kStage;
+#pragma unroll
+    for (int q = 0; q < NB * KT; ++q) {
+      const int32_t row = __shfl_sync(0xffffffffu, my_row, q);
+      const bool ok = live && row >= 0;
+      cp_async_zfill(buf + q * 512 + lane * 16, dXp + (ok ? (int64_t)row * D + d : 0), 16, ok);
+    }
+    if (lane < NB * kE) {                  // ds of the stage's tokens
+      const int j = lane / kE, e = lane % kE;
+      const int64_t n = st * NB + j;
+      const bool ok = st < nst && n < nt && e < E;
+      cp_async_zfill(buf + R::kRows + lane * 4, ds + (ok ? (first + n * stride) * E + e : 0), 4, ok);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  // prologue: stages 0 .. S-2 in flight, the rows of stage S-1 loaded
+#pragma unroll
+  for (int st = 0; st < S - 1; ++st) issue(st, stage_row(st));
+  int32_t next_row = stage_row(S - 1);
+  for (int64_t st = 0; st < nst; ++st) {
+    const int32_t my_row = next_row;
+    next_row = stage_row(st + S);          // consumed next iteration
+    issue(st + S - 1, my_row);             // (empty groups past the last stage)
+    asm volatile("cp.async.wait_group %0;" ::"n"(S - 1) : "memory");
+    __syncwarp();                          // every lane's copies of stage st landed
+    const uint32_t buf = ring + (uint32_t)(st % S) * R::kStage;
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      const int64_t n = st * NB + j;
+      if (n >= nt) break;                  // warp-uniform
+      const int64_t t = first + n * stride;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < kE; ++e) {
+        if (e < E) {
+          float de;
+          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(de) : "r"(buf + R::kRows + (j * kE + e) * 4));
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(de, w[e][i], acc[i]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < KT; ++k) {
+        uint4 u;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
+                     : "r"(buf + (j * KT + k) * 512 + lane * 16));
+        float v[8];
+        bf16x8_to_f32(u, v);               // dropped / sentinel slots: zeros
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += v[i];
+      }
+      if (!live) continue;
+      if (shared0 >= 0) {                  // the shared expert's row, last
+        float v[8];
+        load8(dXp + (shared0 + t) * D + d, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += v[i];
+      }
+      store8(dx + t * D + d, acc);
+    }
+    __syncwarp();                          // stage st read before it is refilled
   }
-  if (t < Tn) one(t);
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // bf16 dx when the router part R = ds . W_r [T, D] fp32 comes from the

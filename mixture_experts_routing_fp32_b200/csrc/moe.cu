@@ -1968,15 +1968,17 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     else if (K == 8) MOE_TRY(go(std::integral_constant<int, 8>{}));
     else MOE_TRY(go(std::integral_constant<int, 0>{}));
   } else if (bf && E <= 8 && (K == 1 || K == 2 || K == 4 || K == 8)) {
-    // blocks (slice c, token group g): the W_r slice in shared memory, one
-    // token per warp at a time
-    const int nch = (int)ceil_div(D, 256);
-    const int groups = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(T, 8),
-                                                                   ceil_div((int64_t)num_sms() * 8, nch)));
+    // blocks (16 slices of 256 columns, token group g), one per SM (each
+    // holds a ring of cp.async stages per warp in shared memory)
+    const int nch = (int)ceil_div(ceil_div(D, 256), 16);
+    const int groups = (int)std::max<int64_t>(1, std::min<int64_t>(T, num_sms() / nch));
     auto go = [&](auto kt) -> int {
       constexpr int KT = decltype(kt)::value;
+      constexpr int sm = DxRing<KT>::kBytes;
+      MOE_CK(cudaFuncSetAttribute(dx_small_kernel<KT>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, sm));
       prof_begin(s);
-      MOE_CK((launch_k(dx_small_kernel<KT>, dim3((unsigned)nch, (unsigned)groups), 256, 0, s, ds,
+      MOE_CK((launch_k(dx_small_kernel<KT>, dim3((unsigned)nch, (unsigned)groups), 512, sm, s, ds,
                        w_r, static_cast<const __nv_bfloat16*>(dXp), slot_row, offsets,
                        c->n_shared, T, D, E, El, static_cast<__nv_bfloat16*>(dx))));
       MOE_LAUNCHED(s, "dx_unpermute_router");
