@@ -149,7 +149,8 @@ REDUCED = {
 # one router or expert tile, select-all (K = E), expert counts that are not a
 # split width (padding experts in the router's split), a count the four-lane
 # routing kernel does not take, K = 1 in the fused router, sigmoid without a
-# selection bias, and 512 experts with a group limit.
+# selection bias, 512 experts with a group limit, and few experts with a
+# shared expert.
 EDGE = {
     "t1_e64": CONFIGS["olmoe"].replace(name="edge_t1_e64", T=1, D=128, F=128),
     "t1_e4": CONFIGS["mm_b"].replace(name="edge_t1_e4", T=1, D=128, F=128),
@@ -171,6 +172,13 @@ EDGE = {
     "e512_groups": LayerConfig("edge_e512_groups", T=64, D=128, E=512, K=8, F=128,
                                score_fn=SIGMOID, renorm=1, n_groups=16, topk_groups=4,
                                route_scale=2.5, sel_bias_range=0.1),
+    # the router part of dx on CUDA cores (E <= 8) with a shared expert and
+    # a row width that ends inside a 256-column slice; K = 1 with a shared
+    # expert (no token-order epilogues)
+    "e8_shared_d384": LayerConfig("edge_e8_shared_d384", T=300, D=384, E=8, K=2, F=128,
+                                  n_shared=1, renorm=1, aux_alpha=0.01, capacity_factor=1.25),
+    "e4_k1_shared": LayerConfig("edge_e4_k1_shared", T=333, D=256, E=4, K=1, F=128,
+                                n_shared=1, renorm=0, aux_alpha=5e-4, sentinel_frac=0.05),
 }
 
 
