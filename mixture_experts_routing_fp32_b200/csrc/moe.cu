@@ -965,13 +965,15 @@ bool bn512_enabled() {
 }
 
 // Tile width of the weight-gradient GEMMs: pick_bn's choice, or
-// MOE_WGRAD_BN (128 or 256, if it divides the output width) for tuning.
-int wgrad_bn(int bn, int64_t n_out) {
+// MOE_WGRAD_BN (128, 256, or 512 on CTA pairs without the row gather, if it
+// divides the output width) for tuning.
+int wgrad_bn(int bn, int64_t n_out, bool pair512) {
   static const int forced = [] {
     const char* v = std::getenv("MOE_WGRAD_BN");
     return v != nullptr ? std::atoi(v) : 0;
   }();
-  if ((forced == 128 || forced == 256) && n_out % forced == 0) return forced;
+  if ((forced == 128 || forced == 256 || (forced == 512 && pair512)) && n_out % forced == 0)
+    return forced;
   return bn;
 }
 
@@ -1742,7 +1744,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     // 4. wgrad down: dW_down[e] = dO^T h over the expert's rows (CTA pairs
     // split the 256-row output tiles)
     const bool pw4 = (D % 256) == 0;
-    const int bn4 = wgrad_bn(pick_bn(F, (int64_t)groups * (D / 128), false, F, pw4, wg_kb), F);
+    const int bn4 = wgrad_bn(pick_bn(F, (int64_t)groups * (D / 128), false, F, pw4, wg_kb), F, pw4);
     MOE_TRY(make_map(&mA, dO, 1, L.rows_max, D, 64, false));
     MOE_TRY(make_map(&mB, h, 1, L.rows_max, F, 64, false));
     {
@@ -1801,7 +1803,8 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     const bool pw6 = ((2 * F) % 256) == 0;
     const bool g6 = x_perm == nullptr;
     const int bn6 =
-        wgrad_bn(pick_bn(D, (int64_t)groups * (2 * F / 128), false, F, pw6, g6 ? 0 : wg_kb), D);
+        wgrad_bn(pick_bn(D, (int64_t)groups * (2 * F / 128), false, F, pw6, g6 ? 0 : wg_kb), D,
+                 pw6 && !g6);
     MOE_TRY(make_map(&mA, dA13, 1, L.rows_max, 2 * F, 64, false));
     MOE_TRY(make_map(&mB, g6 ? x : x_perm, 1, g6 ? T : L.rows_max, D, 64, false));
     {
