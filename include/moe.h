@@ -18,7 +18,12 @@
  *     `cfg` is a HOST pointer.  All buffers are owned and allocated by the
  *     caller; the library never allocates or frees memory.
  *   - All layouts are row-major and contiguous.  T tokens, D model dim,
- *     E routed experts, K experts per token, F expert FFN dim.
+ *     E routed experts, K experts per token, F expert FFN dim.  On the
+ *     tensor-core path the kernels read and write activation, expert-weight
+ *     and gradient buffers through TMA, so each must start on a 16-byte
+ *     boundary (any cudaMalloc'd or torch buffer does); a misaligned one
+ *     makes the call return MOE_ERR_CUDA when its tensor map is built
+ *     (kernels of that call that come earlier may already have run).
  *     "act" = activation / expert-weight element type, cfg->dtype:
  *     MOE_BF16 (__nv_bfloat16) or MOE_FP32 (float).  The router is fp32.
  *   - Calls are asynchronous on `stream` and never synchronise, except
@@ -426,7 +431,10 @@ int moe_combine(const moe_config_t* cfg, const void* o,
  * With one slot per token (K = 1), no shared expert and E < 8 on the
  * tensor-core path, dx is written by the dgrad gate/up GEMM's epilogue
  * (dX_perm row + ds_t . W_r, rounded once; tokens without a row get the
- * router part alone) instead of a separate unpermute-sum.
+ * router part alone) instead of a separate unpermute-sum.  The router part
+ * ds_t . W_r is formed in fp32 on CUDA cores for bf16 token choice with
+ * E <= 8, else (E > 8, expert choice) on tensor cores from exact bf16
+ * splits of ds and W_r (the three leading terms, fp32 accumulation).
  * x_perm may be NULL on the tensor-core path (bf16 layers): the gate/up
  * weight-gradient GEMM then copies its x rows by row_slot in its producer
  * warp (cp.async), as moe_expert_ffn_gather does (MOE_ERR_ARG for NULL
