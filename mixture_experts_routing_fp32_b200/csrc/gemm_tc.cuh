@@ -386,6 +386,10 @@ __device__ __forceinline__ void bulk_commit() {
 __device__ __forceinline__ void bulk_wait_read_1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
+// Waits until no committed group still reads its shared source.
+__device__ __forceinline__ void bulk_wait_read_0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 // Waits until every committed group has completed its global writes.
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -608,7 +612,8 @@ struct Smem {
   static constexpr int kB = BNC * BK * 2;
   static constexpr int kStage = KB * (kA + kB);   // KB k blocks: [A0 A1 .. | B0 B1 ..]
   // full, empty, copies-done per stage; full, empty per accumulator; done
-  static constexpr int kBars = (3 * STAGES + 2 * NACC + 1) * 8;
+  // (+kEpiWarps: the SwiGLU-backward epilogue warps' own load barriers)
+  static constexpr int kBars = (3 * STAGES + 2 * NACC + 1 + kEpiWarps) * 8;
   // token table of the gathering producer (128 rows)
   static constexpr int kTokOff = STAGES * kStage + kBars + 16;
   // epilogue staging per epilogue warp: two 2 KB boxes for the epilogues
@@ -654,6 +659,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
             const __grid_constant__ CUtensorMap mapBs, const __grid_constant__ CUtensorMap mapO,
             const __grid_constant__ CUtensorMap mapO2, const Params p, int total_hint) {
   constexpr bool kTmaOut = BN != 192 && (EPI == EPI_SWIGLU || EPI == EPI_STORE || EPI == EPI_WGRAD);
+  // SwiGLU backward: the saved a13 blocks come in by TMA (mapO) into the
+  // warp's two staging boxes, dA13 is computed in place and stored by TMA
+  // (mapO2)
+  constexpr bool kTmaBwd = BN != 192 && EPI == EPI_SWIGLU_BWD;
   constexpr int KB = stage_kb<BN, STAGES, MODE, PAIR, GATHER>();
   using S = KernelSmem<BN, STAGES, MODE, PAIR, GATHER>;
   constexpr int BNC = S::BNC;
@@ -679,6 +688,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   // gathered rows in a pair's second CTA: its lanes' cp.async copies arrive
   // here; warp 1 forwards each completed stage to the leader's full barrier
   auto cpd_bar = [&](int s) { return bars + 8u * (2 * STAGES + 2 * NACC + 1 + s); };
+  // epilogue warp w's barrier for its TMA loads of saved a13 blocks
+  auto epi_bar = [&](int w) { return bars + 8u * (3 * STAGES + 2 * NACC + 1 + w); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + STAGES * S::kStage + S::kBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -708,6 +719,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       mbar_init(acce_bar(b), kEpiWarps * (PAIR ? 2 : 1));   // both CTAs' epilogues
     }
     mbar_init(done_bar, 1);
+    for (int w = 0; w < kEpiWarps; ++w) mbar_init(epi_bar(w), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -1137,6 +1149,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     }
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t bwd_phase = 0;   // parity of this warp's a13 load barrier
     Tile nxt = decode_at(unit);
     for (int t = unit; t < total; t += n_units) {
       const Tile d = nxt;
@@ -1155,7 +1168,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       constexpr int kPf = kNch < 2 ? kNch : 2;
       uint4 pa[EPI == EPI_SWIGLU_BWD ? kPf : 1][4], pb[EPI == EPI_SWIGLU_BWD ? kPf : 1][4];
       const __nv_bfloat16* a13s = p.aux + row0 * p.ld_aux + d.n0 + hh * HC;
-      if constexpr (EPI == EPI_SWIGLU_BWD) {
+      // SwiGLU backward through TMA: the first chunk's gate / up blocks of
+      // a13 into the boxes (once the last stores have read them)
+      const uint32_t eb = epi_bar(warp - 2);
+      auto bwd_load = [&](int c) {
+        if (lane == 0) {
+          bulk_wait_read_0();
+          mbar_expect_tx(eb, 2 * kTmaBox);
+          tma_2d(stg, &mapO, eb, d.n0 + hh * HC + c, (int)row0);
+          tma_2d(stg + kTmaBox, &mapO, eb, p.F + d.n0 + hh * HC + c, (int)row0);
+        }
+      };
+      if constexpr (kTmaBwd) {
+        bwd_load(0);
+      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
 #pragma unroll
         for (int c = 0; c < kPf; ++c) {
           block_load32(a13s + 32 * c, p.ld_aux, pa[c]);
@@ -1321,6 +1347,47 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           u2f32(r, v);
           if (rv) store32_f32(dst + c, v);
         }
+      } else if constexpr (kTmaBwd) {
+#pragma unroll 1
+        for (int c = 0; c < HC; c += 32) {
+          uint32_t r[32];
+          float dh[32], av[32], bv[32];
+          tmem_ld32(tbase + hh * HC + c, r);
+          mbar_wait(eb, bwd_phase, abort_flag);   // this chunk's a13 blocks landed
+          bwd_phase ^= 1u;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t o = lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
+            bf16x8_to_f(lds128(stg + o), av + 8 * j);
+            bf16x8_to_f(lds128(stg + kTmaBox + o), bv + 8 * j);
+          }
+          tmem_wait();
+          u2f32(r, dh);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float sg = fast_sigmoid(av[i]);
+            const float da = dh[i] * bv[i] * sg * (1.f + av[i] * (1.f - sg));
+            bv[i] = dh[i] * av[i] * sg;
+            av[i] = da;
+          }
+          uint4 ua[4], ub[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            ua[j] = pack8_bf16(av + 8 * j);
+            ub[j] = pack8_bf16(bv + 8 * j);
+          }
+          stage_box_sw64(stg, ua);              // dA13 in place of the a13 blocks
+          stage_box_sw64(stg + kTmaBox, ub);
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            const int xg = d.n0 + hh * HC + c;
+            tma_store_2d(&mapO2, stg, xg, (int)row0);
+            tma_store_2d(&mapO2, stg + kTmaBox, p.F + xg, (int)row0);
+            bulk_commit();
+          }
+          if (c + 32 < HC) bwd_load(c + 32);
+        }
       } else {  // EPI_SWIGLU_BWD
         __nv_bfloat16* da13 = p.out + row0 * p.ld_out + d.n0 + hh * HC;
 #pragma unroll
@@ -1357,7 +1424,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
     }
   }
-  if constexpr (kTmaOut) {
+  if constexpr (kTmaOut || kTmaBwd) {
     if (warp >= 2 && lane == 0) bulk_wait_all();   // this warp's output stores are written
   }
   tc_fence_before();

@@ -397,14 +397,16 @@ cudaError_t launch_k(void (*kern)(KP...), dim3 grid, dim3 block, size_t smem, cu
   return cudaLaunchKernelEx(&lc, kern, std::forward<A>(args)...);
 }
 
-// Output tensors of the epilogues that store through TMA (SwiGLU: a13, h;
-// plain store: out; weight gradient: the routed experts' [E * rows, cols]
-// and the shared expert's), see make_store_map.
+// Tensors the epilogues move through TMA (SwiGLU: a13, h; plain store: out;
+// weight gradient: the routed experts' [E * rows, cols] and the shared
+// expert's; SwiGLU backward: the saved a13 it loads, dA13), see
+// make_store_map.
 struct OutMaps {
   CUtensorMap o1, o2;
 };
 
-// bf16 tensor [rows][cols] as TMA-store target: box {32, 32}, 64-byte swizzle.
+// bf16 tensor [rows][cols] for the epilogues' TMA loads and stores: box
+// {32, 32}, 64-byte swizzle.
 int make_store_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) { g_last_cuda_error = (int)cudaErrorNotSupported; return MOE_ERR_CUDA; }
@@ -425,10 +427,10 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
               cudaStream_t s, const OutMaps* om) {
   using S = tc::KernelSmem<BN, ST, MODE, PAIR, GATHER>;
   auto k = tc::gemm_kernel<BN, ST, MODE, AMN, BMN, EPI, PAIR, GATHER>;
-  // the SwiGLU, plain-store and weight-gradient epilogues write through TMA
-  // (all tile widths but 192)
-  constexpr bool tma_out =
-      BN != 192 && (EPI == tc::EPI_SWIGLU || EPI == tc::EPI_STORE || EPI == tc::EPI_WGRAD);
+  // the SwiGLU, plain-store, weight-gradient and SwiGLU-backward epilogues
+  // move their blocks through TMA (all tile widths but 192)
+  constexpr bool tma_out = BN != 192 && (EPI == tc::EPI_SWIGLU || EPI == tc::EPI_STORE ||
+                                         EPI == tc::EPI_WGRAD || EPI == tc::EPI_SWIGLU_BWD);
   if (tma_out && om == nullptr) return MOE_ERR_ARG;
   const CUtensorMap& o1 = om != nullptr ? om->o1 : a;
   const CUtensorMap& o2 = om != nullptr ? om->o2 : a;
@@ -1733,12 +1735,15 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       tc::Params p = rows_params(c, D, F / bn3, tile_expert, stats, pr);
       p.out = static_cast<__nv_bfloat16*>(dA13); p.ld_out = 2 * F;
       p.aux = static_cast<const __nv_bfloat16*>(a13); p.ld_aux = 2 * F;
+      OutMaps om3;   // the saved a13 (TMA loads) and dA13 (TMA stores)
+      MOE_TRY(make_store_map(&om3.o1, a13, L.rows_max, 2 * F));
+      MOE_TRY(make_store_map(&om3.o2, dA13, L.rows_max, 2 * F));
       if (pr)
         MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD, true>(
-            bn3, "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, units * p.nN, 0, s)));
+            bn3, "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, units * p.nN, 0, s, &om3)));
       else
         MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_SWIGLU_BWD>(
-            bn3, "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, units * p.nN, 0, s)));
+            bn3, "tc_dgrad_down_swiglu_bwd", mA, mB, mBs, p, units * p.nN, 0, s, &om3)));
     }
     MOE_TRY(fork_join(sd->ev[2], s, w2));
     // 4. wgrad down: dW_down[e] = dO^T h over the expert's rows (CTA pairs
