@@ -1161,15 +1161,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
         continue;
       }
       const int64_t row0 = d.m0 + q * 32;   // this warp's first row
-      // SwiGLU backward: this warp's first a and b blocks are fetched
-      // (coalesced) before the accumulator wait so their latency overlaps
-      // the main loop; each later block is fetched kPf blocks ahead.
+      // SwiGLU backward: this warp's first a and b blocks of the saved a13
+      // are requested before the accumulator wait so their latency overlaps
+      // the main loop (192-wide tiles: coalesced loads, each later block
+      // fetched kPf blocks ahead; others: TMA into the staging boxes, each
+      // later chunk's blocks once the previous chunk's dA13 stores have read
+      // the boxes).
       constexpr int kNch = HC / 32;
       constexpr int kPf = kNch < 2 ? kNch : 2;
       uint4 pa[EPI == EPI_SWIGLU_BWD ? kPf : 1][4], pb[EPI == EPI_SWIGLU_BWD ? kPf : 1][4];
       const __nv_bfloat16* a13s = p.aux + row0 * p.ld_aux + d.n0 + hh * HC;
-      // SwiGLU backward through TMA: the first chunk's gate / up blocks of
-      // a13 into the boxes (once the last stores have read them)
       const uint32_t eb = epi_bar(warp - 2);
       auto bwd_load = [&](int c) {
         if (lane == 0) {
