@@ -197,6 +197,19 @@ bool small_router_dx(const moe_config_t* c) {
 bool router_dx_tc(const moe_config_t* c) {
   return router_tc(c) && (c->expert_choice || !small_router_dx(c));
 }
+// dW_r = ds^T x on tensor cores (three-way bf16 splits of ds, token-range
+// split) on the tensor-core path; for E < 8 with token choice only (the
+// expert-choice backward forms both router splits together), where it
+// measured level with the two-stage SIMT form on the MiniMind shape
+// (25.5 us either way, the step 1 us shorter); MOE_ROUTER_DW_TC=0 keeps
+// the SIMT form there.
+bool router_dw_tc(const moe_config_t* c) {
+  static const bool small = [] {
+    const char* v = std::getenv("MOE_ROUTER_DW_TC");
+    return !(v != nullptr && v[0] == '0');
+  }();
+  return router_tc(c) || (small && use_tc(c) && !c->expert_choice);
+}
 // Token-choice routing inside the tensor-core logits kernel: up to 64
 // experts, no group limit, K in {1, 2, 4, 8} (MOE_ROUTER_FUSED=0: for
 // E >= 8 the partial-logit GEMM and a separate routing kernel instead, for
@@ -296,12 +309,10 @@ Layout layout_of(const moe_config_t* c) {
   L.off_dA13 = take((size_t)L.rows_max * 2 * c->F * a);
   L.off_dX = take((size_t)L.rows_max * c->D * a);
   L.off_dH = use_tc(c) ? off : take((size_t)L.rows_max * c->F * a);
-  if (router_tc(c) || router_fused_tc(c)) {
-    L.Ep = router_ep(c);
-    L.off_wf = take((size_t)3 * L.Ep * c->D * 2);
-  }
-  if (router_tc(c)) {
-    L.off_rparts = take((size_t)c->T * 3 * L.Ep * 4);
+  if (router_tc(c) || router_fused_tc(c) || router_dw_tc(c)) L.Ep = router_ep(c);
+  if (router_tc(c) || router_fused_tc(c)) L.off_wf = take((size_t)3 * L.Ep * c->D * 2);
+  if (router_tc(c)) L.off_rparts = take((size_t)c->T * 3 * L.Ep * 4);
+  if (router_dw_tc(c)) {
     L.off_dsf = take((size_t)c->T * 3 * L.Ep * 2);
     L.off_dwr3 = take((size_t)dwr_splits(c) * 3 * L.Ep * c->D * 4);
   }
@@ -1608,6 +1619,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   // unpermute-sum kernel forms ds . W_r itself in fp32 (8 FMAs per element)
   // and the [T, D] fp32 round trip disappears
   const bool dx_tc = router_dx_tc(c);
+  const bool dw_tc = router_dw_tc(c);
 
   // 1. per row: gate gradient dg = <o, dy>, and dO = g * dy (token order:
   // each token's dy row read once for all its slots)
@@ -1673,7 +1685,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
                              c->score_fn == MOE_SOFTMAX ? 0 : 1, nullptr,
                              wsp<float>(ws, L.off_seqf), ws, r));
     }
-    if (rtc) {
+    if (dw_tc) {
       a.dsf = wsp<__nv_bfloat16>(ws, L.off_dsf);
       a.dsb = dx_tc ? wsp<__nv_bfloat16>(ws, L.off_dsb) : nullptr;
       a.Ep = (int)L.Ep;
@@ -1865,7 +1877,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
   // 7. dW_r = ds^T x on the router stream: on tensor cores as
   // (ds_hi | ds_mid | ds_lo)^T x then the sum of the three parts; else two
   // deterministic SIMT stages
-  if (rtc) {
+  if (dw_tc) {
     cudaStream_t s = r;
     const int64_t n3 = 3 * L.Ep;
     CUtensorMap mA, mB;
