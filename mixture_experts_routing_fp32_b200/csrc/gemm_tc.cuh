@@ -1207,10 +1207,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       if (!ok) break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * BN;
-      if constexpr ((EPI == EPI_STORE || EPI == EPI_WGRAD) && HC <= 128) {
-        // the whole accumulator slice is read (packed to bf16 in registers)
-        // and released before the stores, so the next tile's MMAs need not
-        // wait for this tile's global stores
+      if constexpr ((EPI == EPI_STORE || EPI == EPI_WGRAD) && HC <= (kTmaOut ? 256 : 128)) {
+        // the whole accumulator slice is read (packed to bf16 in registers:
+        // up to 128 of them for the 512-wide tiles) and released before the
+        // stores, so the next tile's MMAs need not wait for this tile's
+        // global stores
         __nv_bfloat16* w0;
         int64_t ld;
         if (EPI == EPI_STORE) {
