@@ -493,6 +493,23 @@ __device__ __forceinline__ void stage_box_sw64(uint32_t buf, const uint4 (&u)[4]
   for (int j = 0; j < 4; ++j) sts128(buf + r * 64 + ((j ^ ((r >> 1) & 3)) << 4), u[j]);
 }
 
+// Staging of one fp32 TMA-store box: 32 rows x 32 floats (128-byte rows) in
+// the 128-byte swizzle (16-byte chunk j of row r at chunk j ^ (r % 8)), so
+// the 16-byte stores of any 8 consecutive lanes fall in distinct banks.
+// Lane r writes row r; `buf` is 1024-byte aligned.
+__device__ __forceinline__ void stage_box_f32_sw128(uint32_t buf, const float (&v)[32]) {
+  const int r = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint4 u;
+    u.x = __float_as_uint(v[4 * j]);
+    u.y = __float_as_uint(v[4 * j + 1]);
+    u.z = __float_as_uint(v[4 * j + 2]);
+    u.w = __float_as_uint(v[4 * j + 3]);
+    sts128(buf + r * 128 + ((j ^ (r & 7)) << 4), u);
+  }
+}
+
 // staged_store32 to scattered rows: block row i goes to w0 + tok_i * ld,
 // where tok_i is lane i's `tok` (rows with tok < 0 are skipped).
 __device__ __forceinline__ void staged_store32_tok(uint32_t stg, const float (&v)[32],
@@ -617,11 +634,11 @@ struct Smem {
   // token table of the gathering producer (128 rows)
   static constexpr int kTokOff = STAGES * kStage + kBars + 16;
   // epilogue staging per epilogue warp: two 2 KB boxes for the epilogues
-  // that store through TMA, a 2.5 KB tile for the others (the 192-wide
-  // tiles, whose five stages leave no room for the boxes); 512-byte aligned
-  // (the boxes' swizzle)
+  // that store through TMA (or one 4 KB fp32 box), a 2.5 KB tile for the
+  // others (the 192-wide tiles, whose five stages leave no room for the
+  // boxes); 1024-byte aligned (the fp32 box's 128-byte swizzle)
   static constexpr int kStgW = BN == 192 ? kStgBytes : 2 * kTmaBox;
-  static constexpr int kEpiOff = (kTokOff + 512 + 511) / 512 * 512;
+  static constexpr int kEpiOff = (kTokOff + 512 + 1023) / 1024 * 1024;
   static constexpr int kBytes = 1024 + kEpiOff + kEpiWarps * kStgW;
   static_assert(kBytes <= 232448, "shared memory per CTA");
 };
@@ -663,6 +680,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
   // warp's two staging boxes, dA13 is computed in place and stored by TMA
   // (mapO2)
   constexpr bool kTmaBwd = BN != 192 && EPI == EPI_SWIGLU_BWD;
+  // fp32 outputs (the router products): one 32 x 32 fp32 box per warp in
+  // the 128-byte swizzle, stored by TMA (mapO)
+  constexpr bool kTmaF32 = BN != 192 && EPI == EPI_F32;
   constexpr int KB = stage_kb<BN, STAGES, MODE, PAIR, GATHER>();
   using S = KernelSmem<BN, STAGES, MODE, PAIR, GATHER>;
   constexpr int BNC = S::BNC;
@@ -1347,7 +1367,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           tmem_ld32(tbase + hh * HC + c, r);
           tmem_wait();
           u2f32(r, v);
-          if (rv) store32_f32(dst + c, v);
+          if constexpr (kTmaF32) {   // rows past dense_m: clipped by the tensor map
+            if (lane == 0) bulk_wait_read_0();   // the last store has read the box
+            __syncwarp();
+            stage_box_f32_sw128(stg, v);
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&mapO, stg, d.n0 + hh * HC + c, (int)row0);
+              bulk_commit();
+            }
+          } else {
+            if (rv) store32_f32(dst + c, v);
+          }
         }
       } else if constexpr (kTmaBwd) {
 #pragma unroll 1
@@ -1426,7 +1458,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
       if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
     }
   }
-  if constexpr (kTmaOut || kTmaBwd) {
+  if constexpr (kTmaOut || kTmaBwd || kTmaF32) {
     if (warp >= 2 && lane == 0) bulk_wait_all();   // this warp's output stores are written
   }
   tc_fence_before();

@@ -432,6 +432,21 @@ int make_store_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols) 
   return MOE_OK;
 }
 
+// fp32 tensor [rows][cols] as TMA-store target: box {32, 32}, 128-byte swizzle.
+int make_store_map_f32(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) { g_last_cuda_error = (int)cudaErrorNotSupported; return MOE_ERR_CUDA; }
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { g_last_cuda_error = (int)cudaErrorInvalidValue; return MOE_ERR_CUDA; }
+  return MOE_OK;
+}
+
 template <int BN, int ST, int MODE, bool AMN, bool BMN, int EPI, bool PAIR, bool GATHER>
 int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
               const CUtensorMap& bs, const tc::Params& p, int64_t total_max, int total_hint,
@@ -441,7 +456,8 @@ int launch_tc(const char* name, const CUtensorMap& a, const CUtensorMap& b,
   // the SwiGLU, plain-store, weight-gradient and SwiGLU-backward epilogues
   // move their blocks through TMA (all tile widths but 192)
   constexpr bool tma_out = BN != 192 && (EPI == tc::EPI_SWIGLU || EPI == tc::EPI_STORE ||
-                                         EPI == tc::EPI_WGRAD || EPI == tc::EPI_SWIGLU_BWD);
+                                         EPI == tc::EPI_WGRAD || EPI == tc::EPI_SWIGLU_BWD ||
+                                         EPI == tc::EPI_F32);
   if (tma_out && om == nullptr) return MOE_ERR_ARG;
   const CUtensorMap& o1 = om != nullptr ? om->o1 : a;
   const CUtensorMap& o2 = om != nullptr ? om->o2 : a;
@@ -759,8 +775,11 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
     p.E = 1; p.Kd = c->D; p.nN = (int)(n3 / bn); p.group_m = group_rows(c->D);
     p.dense_m = c->T;
     p.out_f32 = parts; p.ld_f32 = n3;
+    OutMaps om;   // the partial logits as TMA-store target
+    MOE_TRY(make_store_map_f32(&om.o1, parts, c->T, n3));
+    om.o2 = om.o1;
     MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_F32>(
-        bn, "router_logits_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+        bn, "router_logits_tc", mA, mB, mB, p, mtiles * p.nN, 0, s, &om)));
     return route_launch(c, a, nullptr, parts, Ep, off, s);
   }
   const size_t fused_smem = 8 * (size_t)c->E * 4;
@@ -1177,8 +1196,11 @@ int route_ec_impl(const moe_config_t* c, const TX* x, const float* w_r, const fl
     p.E = 1; p.Kd = c->D; p.nN = (int)(n3 / bn); p.group_m = group_rows(c->D);
     p.dense_m = c->T;
     p.out_f32 = pt; p.ld_f32 = n3;
+    OutMaps om;   // the partial logits as TMA-store target
+    MOE_TRY(make_store_map_f32(&om.o1, pt, c->T, n3));
+    om.o2 = om.o1;
     MOE_TRY((run_tc<tc::MODE_ROWS, false, false, tc::EPI_F32>(
-        bn, "router_logits_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+        bn, "router_logits_tc", mA, mB, mB, p, mtiles * p.nN, 0, s, &om)));
     parts = pt;
   } else {
     dim3 g1((unsigned)ceil_div(c->T, 64), (unsigned)ceil_div(E, 64));
@@ -1944,8 +1966,11 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     p.E = 1; p.Kd = (int)n3; p.nN = D / bn; p.group_m = group_rows(n3);
     p.dense_m = T;
     p.out_f32 = Rdx; p.ld_f32 = D;
+    OutMaps om;   // R as TMA-store target
+    MOE_TRY(make_store_map_f32(&om.o1, Rdx, T, D));
+    om.o2 = om.o1;
     MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_F32>(
-        bn, "router_dx_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+        bn, "router_dx_tc", mA, mB, mB, p, mtiles * p.nN, 0, s, &om)));
   }
   if (dx1) {
     // done
@@ -1972,8 +1997,11 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     p.E = 1; p.Kd = (int)n3; p.nN = D / bn; p.group_m = group_rows(n3);
     p.dense_m = T;
     p.out_f32 = R; p.ld_f32 = D;
+    OutMaps om;   // R as TMA-store target
+    MOE_TRY(make_store_map_f32(&om.o1, R, T, D));
+    om.o2 = om.o1;
     MOE_TRY((run_tc<tc::MODE_ROWS, false, true, tc::EPI_F32>(
-        bn, "router_dx_tc", mA, mB, mB, p, mtiles * p.nN, 0, s)));
+        bn, "router_dx_tc", mA, mB, mB, p, mtiles * p.nN, 0, s, &om)));
     auto go = [&](auto kt) -> int {
       prof_begin(s);
       MOE_CK((launch_k(dx_sum_kernel<decltype(kt)::value>, grid_for(T), 256, 0, s, R,
