@@ -1344,16 +1344,47 @@ gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
           u2f32(ru, ub);
           const int xc = d.n0 + hh * HJ + c;   // column of gate j (up: + F) and of h
           if constexpr (kTmaOut) {
-            tma_out(ga, &mapO, xc, row0);
-            tma_out(ub, &mapO, p.F + xc, row0);
+            // gate and up blocks: both boxes, one fence, one bulk group
+            uint4 ug[4], uu[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              ug[j] = pack8_bf16(ga + 8 * j);
+              uu[j] = pack8_bf16(ub + 8 * j);
+            }
+            if (lane == 0) bulk_wait_read_0();   // the last h store has read box 0
+            __syncwarp();
+            stage_box_sw64(stg, ug);
+            stage_box_sw64(stg + kTmaBox, uu);
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&mapO, stg, xc, (int)row0);
+              tma_store_2d(&mapO, stg + kTmaBox, p.F + xc, (int)row0);
+              bulk_commit();
+            }
           } else {
             staged_store32(stg, ga, a13 + c, p.ld_out, pol_out);
             staged_store32(stg, ub, a13 + p.F + c, p.ld_out, pol_out);
           }
 #pragma unroll
           for (int i = 0; i < 32; ++i) ga[i] = ga[i] * fast_sigmoid(ga[i]) * ub[i];
-          if constexpr (kTmaOut) tma_out(ga, &mapO2, xc, row0);
-          else staged_store32(stg, ga, hr + c, p.ld_out2, pol_out);
+          if constexpr (kTmaOut) {
+            // h block: box 0 once the gate / up stores have read it
+            uint4 uh[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) uh[j] = pack8_bf16(ga + 8 * j);
+            if (lane == 0) bulk_wait_read_0();
+            __syncwarp();
+            stage_box_sw64(stg, uh);
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&mapO2, stg, xc, (int)row0);
+              bulk_commit();
+            }
+          } else {
+            staged_store32(stg, ga, hr + c, p.ld_out2, pol_out);
+          }
         }
       } else if constexpr (EPI == EPI_F32 || EPI == EPI_WGRAD_F32) {
         const int64_t row = row0 + lane;
