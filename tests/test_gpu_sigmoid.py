@@ -73,7 +73,7 @@ def test_fast_sigmoid_error_bound(sig_lib):
     ref = 1.0 / (1.0 + np.exp(-x.astype(np.float64)))
     rel = np.abs(y - ref) / ref
     # fp32 precision: the exponential's approximation and the rounding of
-    # 1 + e and of the Newton steps (a few ulp), plus the rounding of the
+    # 1 + e and of the approximate divide (a few ulp), plus the rounding of the
     # exponent's argument -x log2(e), which scales with |x| (2^-24 |x| log2(e)
     # ln 2 relative, where the logistic follows e^x)
     bound = 5e-7 + 8e-8 * np.abs(x.astype(np.float64))
