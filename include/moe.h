@@ -23,7 +23,10 @@
  *     and gradient buffers through TMA, so each must start on a 16-byte
  *     boundary (any cudaMalloc'd or torch buffer does); a misaligned one
  *     makes the call return MOE_ERR_CUDA when its tensor map is built
- *     (kernels of that call that come earlier may already have run).
+ *     (kernels of that call that come earlier may already have run).  x
+ *     and W_r, which every path reads with 16-byte loads, are checked
+ *     first: moe_router, moe_route_expert_choice and moe_backward return
+ *     MOE_ERR_ARG, having launched nothing, when either is misaligned.
  *     "act" = activation / expert-weight element type, cfg->dtype:
  *     MOE_BF16 (__nv_bfloat16) or MOE_FP32 (float).  The router is fp32.
  *   - Calls are asynchronous on `stream` and never synchronise, except

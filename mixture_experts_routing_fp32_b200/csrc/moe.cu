@@ -670,7 +670,7 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
     const int EP = c->E <= 8 ? 8 : c->E <= 16 ? 16 : c->E <= 32 ? 32 : 64;
     auto* wf = wsp<__nv_bfloat16>(ws, L.off_wf);
     prof_begin(s);
-    MOE_CK((launch_k(split_w_kernel, grid_for((int64_t)EP * c->D / 32), 256, 0, s, w_r, c->E,
+    MOE_CK((launch_k(split_w_kernel, grid_for((int64_t)EP * c->D / 256), 256, 0, s, w_r, c->E,
                      EP, c->D, wf, (__nv_bfloat16*)nullptr)));
     MOE_LAUNCHED(s, "router_split_w");
     // E > 16: CTA pairs (each CTA streams half of the split rows)
@@ -763,7 +763,7 @@ int router_impl(const moe_config_t* c, const TX* x, const float* w_r, const floa
     auto* wf = wsp<__nv_bfloat16>(ws, L.off_wf);
     float* parts = wsp<float>(ws, L.off_rparts);
     prof_begin(s);
-    MOE_CK((launch_k(split_w_kernel, grid_for(Ep * c->D / 32), 256, 0, s, w_r, c->E, (int)Ep,
+    MOE_CK((launch_k(split_w_kernel, grid_for(Ep * c->D / 256), 256, 0, s, w_r, c->E, (int)Ep,
                      c->D, wf, (__nv_bfloat16*)nullptr)));
     MOE_LAUNCHED(s, "router_split_w");
     const int64_t mtiles = ceil_div(c->T, kRowTile);
@@ -1104,6 +1104,9 @@ int dispatch_impl(const moe_config_t* c, const Layout& L, const int32_t* topk_id
 // ===========================================================================
 extern "C" {
 
+// x and W_r are read with 16-byte vector loads (and x through TMA).
+static bool misaligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) != 0; }
+
 int moe_get_sizes(const moe_config_t* cfg, moe_sizes_t* out) {
   MOE_TRY(validate(cfg));
   if (out == nullptr) return MOE_ERR_ARG;
@@ -1122,6 +1125,7 @@ int moe_router(const moe_config_t* c, const void* x, const float* w_r, const flo
   MOE_TRY(validate(c));
   if (!x || !w_r || !logits || !probs || !lse || !topk_idx || !topk_w || !near_ties)
     return MOE_ERR_ARG;
+  if (misaligned16(x) || misaligned16(w_r)) return MOE_ERR_ARG;
   if (c->expert_choice) return MOE_ERR_ARG;   // moe_route_expert_choice
   if ((router_tc(c) || router_fused_tc(c)) && ws == nullptr) return MOE_ERR_ARG;
   if (c->dtype == MOE_BF16)
@@ -1184,7 +1188,7 @@ int route_ec_impl(const moe_config_t* c, const TX* x, const float* w_r, const fl
     auto* wf = wsp<__nv_bfloat16>(ws, L.off_wf);
     float* pt = wsp<float>(ws, L.off_rparts);
     prof_begin(s);
-    MOE_CK((launch_k(split_w_kernel, grid_for(Ep * c->D / 32), 256, 0, s, w_r, E, (int)Ep,
+    MOE_CK((launch_k(split_w_kernel, grid_for(Ep * c->D / 256), 256, 0, s, w_r, E, (int)Ep,
                      c->D, wf, (__nv_bfloat16*)nullptr)));
     MOE_LAUNCHED(s, "router_split_w");
     const int64_t mtiles = ceil_div(c->T, kRowTile);
@@ -1240,6 +1244,7 @@ int moe_route_expert_choice(const moe_config_t* c, const void* x, const float* w
   if (!c->expert_choice || !x || !w_r || !logits || !probs || !lse || !topk_idx || !topk_w ||
       !sentinel_mask || !near_ties)
     return MOE_ERR_ARG;
+  if (misaligned16(x) || misaligned16(w_r)) return MOE_ERR_ARG;
   if (router_tc(c) && ws == nullptr) return MOE_ERR_ARG;
   if (c->dtype == MOE_BF16)
     return route_ec_impl(c, static_cast<const __nv_bfloat16*>(x), w_r, logit_offset, logits,
@@ -1619,6 +1624,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
       !offsets || !slot_row || !row_slot || !tile_expert || !stats || !a13 || !h ||
       !o || !w13 || !w_down || !dy || !dx || !dw_r || !dw13 || !dw_down || !ws)
     return MOE_ERR_ARG;
+  if (misaligned16(x) || misaligned16(w_r)) return MOE_ERR_ARG;
   if (!x_perm && !use_tc(c)) return MOE_ERR_ARG;   // only the tensor-core wgrad gathers
   if (c->n_shared && (!w13_s || !w_down_s || !dw13_s || !dw_down_s)) return MOE_ERR_ARG;
   const Layout L = layout_of(c);
@@ -1742,7 +1748,7 @@ int moe_backward(const moe_config_t* c, const void* x, const float* w_r, const f
     if (dx_tc) {
       // (hi; mid; hi) split of W_r for the router part of dx
       prof_begin(s);
-      MOE_CK((launch_k(split_w_kernel, grid_for(L.Ep * D / 32), 256, 0, s, w_r, E, (int)L.Ep, D,
+      MOE_CK((launch_k(split_w_kernel, grid_for(L.Ep * D / 256), 256, 0, s, w_r, E, (int)L.Ep, D,
                        (__nv_bfloat16*)nullptr, wsp<__nv_bfloat16>(ws, L.off_wb))));
       MOE_LAUNCHED(s, "router_split_w");
     }

@@ -336,19 +336,56 @@ __device__ __forceinline__ void split3_bf16(float v, __nv_bfloat16& hi, __nv_bfl
 
 // w [E,D] f32 -> wf [3 Ep, D] = (hi; mid; lo) and, if wb, wb = (hi; mid; hi)
 // (the latter pairs with (hi | hi | mid) splits of a second fp32 operand).
+// One thread per 8 consecutive elements of a row (D % 8 == 0): two 16-byte
+// loads (w is 16-byte aligned: the entry points check it) and one 16-byte
+// store per split row (wf and wb are 256-byte aligned workspace blocks, Ep D
+// elements per split a multiple of 8).
+__device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 a, __nv_bfloat16 b) {
+  return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+}
+
 __global__ void __launch_bounds__(256)
 split_w_kernel(const float* __restrict__ w, int E, int Ep, int D,
                __nv_bfloat16* __restrict__ wf, __nv_bfloat16* __restrict__ wb) {
   pdl_begin();
   const int64_t n = (int64_t)Ep * D;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t e = i / D;
-    const float v = e < E ? w[i] : 0.f;
-    __nv_bfloat16 hi, mid, lo;
-    split3_bf16(v, hi, mid, lo);
-    if (wf != nullptr) { wf[i] = hi; wf[n + i] = mid; wf[2 * n + i] = lo; }
-    if (wb != nullptr) { wb[i] = hi; wb[n + i] = mid; wb[2 * n + i] = hi; }
+  const int64_t nv = n / 8;
+  const int dv = D / 8;
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nv;
+       v += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = v * 8;
+    float f[8];
+    if (v / dv < E) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(w + i));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(w + i) + 1);
+      f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+      f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] = 0.f;
+    }
+    uint32_t hi[4], mid[4], lo[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat16 h0, m0, l0, h1, m1, l1;
+      split3_bf16(f[2 * j], h0, m0, l0);
+      split3_bf16(f[2 * j + 1], h1, m1, l1);
+      hi[j] = pack_bf16x2(h0, h1);
+      mid[j] = pack_bf16x2(m0, m1);
+      lo[j] = pack_bf16x2(l0, l1);
+    }
+    const uint4 vh = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    const uint4 vm = make_uint4(mid[0], mid[1], mid[2], mid[3]);
+    if (wf != nullptr) {
+      *reinterpret_cast<uint4*>(wf + i) = vh;
+      *reinterpret_cast<uint4*>(wf + n + i) = vm;
+      *reinterpret_cast<uint4*>(wf + 2 * n + i) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    if (wb != nullptr) {
+      *reinterpret_cast<uint4*>(wb + i) = vh;
+      *reinterpret_cast<uint4*>(wb + n + i) = vm;
+      *reinterpret_cast<uint4*>(wb + 2 * n + i) = vh;
+    }
   }
 }
 

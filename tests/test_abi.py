@@ -136,6 +136,23 @@ def test_fused_paths_rejected_where_unsupported(lib):
     assert lib.moe_expert_ffn_combine(ctypes.byref(cfg), *a) == C.MOE_ERR_ARG
 
 
+def test_misaligned_x_or_router_weight_rejected_before_any_launch(lib):
+    """x and W_r are read with 16-byte vector loads: a pointer off that
+    boundary is refused on the host (the dummy addresses are never
+    dereferenced)."""
+    cfg = api.make_config(64, 32, 4, 2, 64, dtype="fp32")
+    ok, off = ctypes.c_void_p(256), ctypes.c_void_p(260)
+    for i in (0, 1):                     # x, w_r
+        args = [ok] * 12
+        args[i] = off
+        args[-1] = None                  # stream
+        assert lib.moe_router(ctypes.byref(cfg), *args) == C.MOE_ERR_ARG
+        args = [ok] * 33
+        args[i] = off
+        args[-1] = None
+        assert lib.moe_backward(ctypes.byref(cfg), *args) == C.MOE_ERR_ARG
+
+
 def test_package_has_no_cpu_fallback():
     # the product path never imports the oracle
     pkg = os.path.join(ROOT, "mixture_experts_routing_fp32_b200")
