@@ -894,6 +894,29 @@ __device__ __forceinline__ void cp_async_zfill(uint32_t dst, const void* src, in
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
                  "r"(valid ? 4 : 0) : "memory");
 }
+// Packed pairs of fp32 lanes (sm_100: one instruction rounds each half as
+// its scalar counterpart does, round to nearest, no flush to zero).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 template <int KT>
 __global__ void __launch_bounds__(512, 1)
 dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
@@ -909,15 +932,18 @@ dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
   if (slice * 256 >= D) return;            // a whole warp past the row (no block barrier)
   const int d = slice * 256 + lane * 8;
   const bool live = d < D;                 // (every lane of the warp takes part in its shuffles)
-  float w[kE][8];
+  uint64_t w[kE][4];                       // column pairs (2i, 2i + 1)
 #pragma unroll
   for (int e = 0; e < kE; ++e) {
+    float f[8];
     if (live && e < E) {
-      load8(w_r + (int64_t)e * D + d, w[e]);
+      load8(w_r + (int64_t)e * D + d, f);
     } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) w[e][i] = 0.f;
+      for (int i = 0; i < 8; ++i) f[i] = 0.f;
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[e][i] = f2_pack(f[2 * i], f[2 * i + 1]);
   }
   const int64_t shared0 = n_shared ? (int64_t)offsets[El] : -1;
   const int64_t stride = gridDim.y;
@@ -963,14 +989,18 @@ dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
       const int64_t n = st * NB + j;
       if (n >= nt) break;                  // warp-uniform
       const int64_t t = first + n * stride;
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // fp32 pairs: per column the same operations in the same order as
+      // the scalar form acc = fma(ds_e, w_e, acc) (e ascending), acc += row
+      // (k ascending)
+      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};   // (+0, +0)
 #pragma unroll
       for (int e = 0; e < kE; ++e) {
         if (e < E) {
           float de;
           asm volatile("ld.shared.f32 %0, [%1];" : "=f"(de) : "r"(buf + R::kRows + (j * kE + e) * 4));
+          const uint64_t de2 = f2_pack(de, de);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = fmaf(de, w[e][i], acc[i]);
+          for (int i = 0; i < 4; ++i) acc2[i] = f2_fma(de2, w[e][i], acc2[i]);
         }
       }
 #pragma unroll
@@ -982,7 +1012,14 @@ dx_small_kernel(const float* __restrict__ ds, const float* __restrict__ w_r,
         float v[8];
         bf16x8_to_f32(u, v);               // dropped / sentinel slots: zeros
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += v[i];
+        for (int i = 0; i < 4; ++i) acc2[i] = f2_add(acc2[i], f2_pack(v[2 * i], v[2 * i + 1]));
+      }
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 a = f2_unpack(acc2[i]);
+        acc[2 * i] = a.x;
+        acc[2 * i + 1] = a.y;
       }
       if (!live) continue;
       if (shared0 >= 0) {                  // the shared expert's row, last
