@@ -390,7 +390,7 @@ disp_gather_tok_kernel(const TX* __restrict__ x, int D, int El, int T, int n_sha
                        const int32_t* __restrict__ slot_row, const int32_t* __restrict__ row_slot,
                        TX* __restrict__ x_perm) {
   pdl_begin();
-  constexpr int NB = KT <= 2 ? 4 : 2;
+  constexpr int NB = 4;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t shared0 = n_shared ? (int64_t)offsets[El] : -1;
   for (int64_t t = (int64_t)blockIdx.x * 8 + warp; t < T; t += (int64_t)gridDim.x * 8) {
